@@ -1,0 +1,200 @@
+/*
+ * s4kv -- int4 KIVI-quantized paged KV cache and GQA decode attention
+ * for NVIDIA B200 (sm_100a).  Plain C ABI: no CUDA, PyTorch or C++ types
+ * cross this boundary.  Device memory is passed as untyped pointers and
+ * streams as `void *` holding a cudaStream_t (NULL = the legacy default
+ * stream).
+ *
+ * What is computed (sources: web pages on the subject, cited by title and
+ * section):
+ *  - "S4 KV -- int4 KV-Cache-Kompression fuer vLLM" (intro, "Funktionsweise"
+ *    step 1, "Lieferumfang"): the paged KV cache is held in int4, KIVI
+ *    style -- keys asymmetric int4 per channel, values int4 per token;
+ *    models with head_dim 128 only, refused at start-up otherwise.
+ *  - "PagedAttention reduziert den KV-Cache-Speicherbedarf beim
+ *    LLM-Serving erheblich" ("Wichtigste Kernpunkte & Evidenz") and
+ *    "KV-Cache und PagedAttention: Warum Ihr LLM-Server langsamer wird"
+ *    ("Wie PagedAttention das loest"): fixed 16-token pages addressed
+ *    through per-sequence page tables, physical pages shareable between
+ *    sequences (shared prefixes).
+ *  - "KV-Cache-Optimierung -- PagedAttention, quantisierter KV, Speculative
+ *    Cache" ("Begriffe auf dieser Seite", GQA): a group of query heads
+ *    shares one K/V head.
+ * The pages print no quantizer formula; this library defines it as: over
+ * a group of fp16 values x, in IEEE fp32,
+ *     mn = min x, mx = max x (IEEE total order: -0 below +0),
+ *     s  = (mx - mn) / 15,
+ *     code = (s == 0) ? 0 : clamp(rint((x - mn) / s), 0, 15),
+ * with rint rounding half to even; stored scale = fp16_rne(s), stored zero
+ * = fp16(mn) (exact); dequantized value = code * scale + zero in fp32.
+ * Key groups: one channel over the 16 tokens of a page.  Value groups:
+ * 32 consecutive channels of one token.  A page's keys and values are
+ * quantized together when its 16th token is appended; until then the
+ * page's tokens stay in an fp16 residual buffer of the sequence.
+ *
+ * Memory layout (all device memory is owned and allocated by the caller;
+ * the library allocates nothing and keeps no per-cache state):
+ *  pool     uint8 [num_pages][num_kv_heads][S4KV_BLOCK_BYTES], 128-byte
+ *           aligned.  One block per (physical page, kv head):
+ *             [   0,1024) key codes   : 256 little-endian 32-bit words
+ *             [1024,2048) value codes : 256 little-endian 32-bit words
+ *             [2048,2304) key scale   : fp16 [128 channels]
+ *             [2304,2560) key zero    : fp16 [128 channels]
+ *             [2560,2688) value scale : fp16 [4 groups][16 tokens]
+ *             [2688,2816) value zero  : fp16 [4 groups][16 tokens]
+ *           Code word w = 128*h + 4*lane + q, lane = 4*n + i (n < 8,
+ *           i < 4, q < 4); nibble j (bits 4j..4j+3) of the word holds
+ *             keys  : token 8*(j&1) + n,
+ *                     channel 32*i + 4*(4*h+q) + 2*((j>>1)&1) + (j>>2)
+ *             values: token 2*i + (j>>2) + 8*((j>>1)&1),
+ *                     channel 32*((4*h+q)>>1) + 4*n + 2*((4*h+q)&1) + (j&1)
+ *           (each 32-bit word is one lane's tensor-core operand fragment;
+ *           s4kv_dequant_page returns the natural [token][channel] order).
+ *  res_k,   fp16 [max_seqs][num_kv_heads][16][128] each.  Row r of batch
+ *  res_v    row b holds token 16*floor(L/16) + r of that sequence for
+ *           r < L mod 16 (L = its current length); other rows are
+ *           unspecified.
+ *  err_flag one uint32 word (may be NULL).  Kernels OR S4KV_EFLAG_* bits
+ *           into it instead of faulting; read it with s4kv_get_error.
+ *
+ * Calls are asynchronous on the given stream, do no host<->device copies
+ * (except s4kv_get_error) and validate every host-visible argument before
+ * launching anything: an invalid call returns a status and launches
+ * nothing.  Device-side inconsistencies (page ids out of range, a
+ * slot_mapping that disagrees with block_tables) set err_flag bits and the
+ * offending element is skipped or clamped; no kernel traps or faults on
+ * purpose.  Distinct caches may be used from different host threads.
+ */
+#ifndef S4KV_H
+#define S4KV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define S4KV_VERSION 1
+#define S4KV_HEAD_DIM 128
+#define S4KV_PAGE_TOKENS 16
+#define S4KV_VALUE_GROUP 32
+#define S4KV_BLOCK_BYTES 2816
+#define S4KV_MAX_GQA_GROUP 8
+
+/* status codes returned by every call */
+#define S4KV_OK 0
+#define S4KV_ERR_INVALID_ARG 1  /* NULL pointer, bad size, misalignment */
+#define S4KV_ERR_UNSUPPORTED 2  /* head_dim != 128, page != 16, group > 8 */
+#define S4KV_ERR_CUDA 3         /* a CUDA runtime call failed */
+#define S4KV_ERR_DEVICE_CHECK 4 /* s4kv_get_error found err_flag bits */
+#define S4KV_ERR_WORKSPACE 5    /* workspace NULL or smaller than required */
+
+/* err_flag bits (device side) */
+#define S4KV_EFLAG_PAGE_RANGE 1u /* a block_tables entry outside [0, num_pages) */
+#define S4KV_EFLAG_SLOT 2u       /* slot_mapping != block_tables[b][pos/16]*16 + pos%16 */
+#define S4KV_EFLAG_SEQ_LEN 4u    /* seq_lens / cu_new inconsistent with the call */
+#define S4KV_EFLAG_TIMEOUT 8u    /* a bounded pipeline wait gave up */
+
+/* Caller-owned description of one layer's cache.  Plain data; the library
+ * never frees or retains it. */
+typedef struct s4kv_cache {
+    void *pool;         /* device, see layout above */
+    void *res_k;        /* device, fp16 */
+    void *res_v;        /* device, fp16 */
+    uint32_t *err_flag; /* device, optional */
+    int32_t num_pages;
+    int32_t num_kv_heads;
+    int32_t max_seqs;
+    int32_t head_dim;    /* must be S4KV_HEAD_DIM */
+    int32_t page_tokens; /* must be S4KV_PAGE_TOKENS */
+} s4kv_cache_t;
+
+/* Library version (S4KV_VERSION). */
+int s4kv_version(void);
+
+/* Human-readable text of a status code (static storage). */
+const char *s4kv_status_string(int status);
+
+/* Fail-fast model check ("S4 KV", "Lieferumfang": unsupported models are
+ * refused at start-up): OK for head_dim 128, 16-token pages and
+ * num_q_heads = G * num_kv_heads with 1 <= G <= 8; S4KV_ERR_UNSUPPORTED
+ * otherwise; S4KV_ERR_INVALID_ARG for non-positive sizes. Host only. */
+int s4kv_check_model(int head_dim, int page_tokens, int num_q_heads,
+                     int num_kv_heads);
+
+/* Bytes the caller must allocate for a cache of num_pages physical pages
+ * ("KV-Cache-Quantisierung: Kapazitaet und Qualitaetspruefung", "Gewichte,
+ * laufenden Zustand und reservierten Speicher trennen": the payload
+ * formula 2 x kv_heads x head_dim x tokens x bytes, here with int4 codes
+ * plus scale/zero metadata).  Host only; either output may be NULL. */
+int s4kv_cache_layout(int num_pages, int num_kv_heads, int max_seqs,
+                      size_t *pool_bytes, size_t *residual_bytes);
+
+/* Append new tokens' K/V and quantize every page they complete.
+ *  k, v          device fp16 [n_tokens][num_kv_heads][128], 16-B aligned,
+ *                sequence b's new tokens at rows cu_new[b]..cu_new[b+1]-1
+ *                in position order.
+ *  slot_mapping  device int64 [n_tokens]: block_tables[b][pos/16]*16 +
+ *                pos%16 for each new token (checked; mismatch -> flag).
+ *  cu_new        device int32 [batch+1], cu_new[0] = 0, nondecreasing,
+ *                cu_new[batch] = n_tokens.
+ *  seq_lens      device int32 [batch]: lengths AFTER the append.
+ *  block_tables  device int32 [batch][max_pages_per_seq].
+ *  max_new_per_seq  host bound on any sequence's new-token count (sizes
+ *                the launch; a larger count sets S4KV_EFLAG_SEQ_LEN).
+ * The residual rows a page needs are read before any are overwritten, so a
+ * single call may both complete a page and start the next one.  Full pages
+ * are written once; pages not completed by this call are not touched (a
+ * shared-prefix page is never rewritten).  Re-running an identical call is
+ * idempotent. */
+int s4kv_append(const s4kv_cache_t *cache, const void *k, const void *v,
+                int n_tokens, const int64_t *slot_mapping,
+                const int32_t *cu_new, const int32_t *seq_lens,
+                const int32_t *block_tables, int batch,
+                int max_pages_per_seq, int max_new_per_seq, void *stream);
+
+/* Bytes of device workspace s4kv_decode_attention needs on the CURRENT
+ * device for this batch and kv head count.  The workspace must be
+ * zero-filled once after allocation; every completed decode call leaves
+ * its counters at zero again.  Needs a CUDA device (S4KV_ERR_CUDA if none). */
+int s4kv_decode_workspace_size(int batch, int num_kv_heads, size_t *bytes);
+
+/* GQA paged decode attention over the quantized pages plus the residual.
+ *  q       device fp16 [batch][num_q_heads][128], 16-B aligned; query head
+ *          j reads kv head j / (num_q_heads / num_kv_heads).
+ *  seq_lens, block_tables as for s4kv_append (lengths including the tokens
+ *          already appended for this step).
+ *  sm_scale  logit scale (1/sqrt(128) for standard attention).
+ *  out     device fp16 [batch][num_q_heads][128], 8-B aligned:
+ *          softmax(sm_scale * q.K^T) V over the sequence's tokens, with
+ *          dequantized full pages and fp16 residual rows; a sequence of
+ *          length 0 gets zeros.
+ *  workspace  device, >= s4kv_decode_workspace_size bytes, 16-B aligned.
+ * Work is split along the KV sequence over all SMs; the last split of a
+ * (sequence, kv head) to finish merges the partial results (log-sum-exp).
+ * Calls sharing one workspace must not overlap on the device. */
+int s4kv_decode_attention(const s4kv_cache_t *cache, const void *q,
+                          int num_q_heads, const int32_t *seq_lens,
+                          const int32_t *block_tables, int batch,
+                          int max_pages_per_seq, float sm_scale, void *out,
+                          void *workspace, size_t workspace_bytes,
+                          void *stream);
+
+/* Dequantize one physical page for all kv heads into natural order:
+ * out_k, out_v device [num_kv_heads][16][128], fp32 if out_fp32 != 0
+ * (x = code*scale + zero, exact product, one rounding) else fp16 (the fp32
+ * value rounded to nearest even).  16-B aligned. */
+int s4kv_dequant_page(const s4kv_cache_t *cache, int physical_page,
+                      void *out_k, void *out_v, int out_fp32, void *stream);
+
+/* Synchronize `stream`, read the cache's err_flag into *flags and clear it
+ * when `clear` != 0.  Returns S4KV_ERR_DEVICE_CHECK when bits were set. */
+int s4kv_get_error(const s4kv_cache_t *cache, uint32_t *flags, int clear,
+                   void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* S4KV_H */

@@ -1,0 +1,512 @@
+/*
+ * s4kv CPU oracle -- TEST INFRASTRUCTURE ONLY.
+ *
+ * A plain, slow, single-threaded restatement of what the int4 KIVI paged
+ * KV cache computes.  Only the tests, the smoke check and the benchmark's
+ * CPU-baseline leg may load this file; the CUDA library never does, and the
+ * two share no code, header, table or constant.
+ *
+ * Sources (web pages on the subject; cited by title and section):
+ *   [S4KV]  "S4 KV -- int4 KV-Cache-Kompression fuer vLLM", intro,
+ *           "Funktionsweise" step 1, "Lieferumfang": keys are quantized to
+ *           asymmetric int4 per channel, values to int4 per token (KIVI
+ *           style); head_dim 128 only, with fail-fast otherwise.
+ *   [KVOPT] "KV-Cache-Optimierung -- PagedAttention, quantisierter KV,
+ *           Speculative Cache", "Kernpunkte" and "Begriffe auf dieser
+ *           Seite" (GQA: a group of query heads shares one K/V head;
+ *           PagedAttention: fixed-size blocks addressed like OS pages).
+ *   [PAGED] "PagedAttention reduziert den KV-Cache-Speicherbedarf beim
+ *           LLM-Serving erheblich", "Wichtigste Kernpunkte & Evidenz":
+ *           16-token pages addressed through page tables.
+ *   [CAP]   adechristanto.de, "KV-Cache-Quantisierung: Kapazitaet und
+ *           Qualitaetspruefung", section "Gewichte, laufenden Zustand und
+ *           reservierten Speicher trennen": KV payload bytes =
+ *           2 x layers x kv_heads x head_dim x tokens x bytes per element.
+ *
+ * The pages fix the KIVI axis split but print no formula.  This library
+ * states the quantizer as: over a group of fp16 values x, in fp32,
+ *   mn = min x, mx = max x, s = (mx - mn) / 15,
+ *   code = (s == 0) ? 0 : clamp(rint((x - mn) / s), 0, 15),
+ * stored scale = fp16_rne(s), stored zero = fp16(mn) (exact); the
+ * dequantized value is code * scale + zero, evaluated in fp32.  A key group
+ * is one channel over the 16 tokens of a page; a value group is 32
+ * consecutive channels of one token.  Minimum and maximum are taken in IEEE
+ * total order, so -0 counts below +0.
+ *
+ * Page block layout (2816 bytes per (physical page, kv head)):
+ *   [   0,1024) key codes   : 256 little-endian 32-bit words
+ *   [1024,2048) value codes : 256 little-endian 32-bit words
+ *   [2048,2304) key scale   : fp16 [128 channels]
+ *   [2304,2560) key zero    : fp16 [128 channels]
+ *   [2560,2688) value scale : fp16 [4 groups][16 tokens]
+ *   [2688,2816) value zero  : fp16 [4 groups][16 tokens]
+ * Code word w (0..255) splits as w = 128*h + 4*lane + q with lane = 4*n + i
+ * (n 0..7, i 0..3, q 0..3).  Nibble j (bits 4j..4j+3) of the word holds
+ *   keys  : token 8*(j&1) + n,
+ *           channel 32*i + 4*(4*h + q) + 2*((j>>1)&1) + (j>>2);
+ *   values: token 2*i + (j>>2) + 8*((j>>1)&1),
+ *           channel 32*((4*h+q)>>1) + 4*n + 2*((4*h+q)&1) + (j&1).
+ * Residual buffers hold fp16 [max_seqs][kv_heads][16][128] each for keys
+ * and values: row r of sequence b is its token 16*floor(L/16) + r while
+ * r < L mod 16; other rows are unspecified.
+ *
+ * Parity status of every function here is pinned by tests in
+ * tests/test_oracle.py (see the header of that file for which pin covers
+ * which function).  Build: gcc -O2 -ffp-contract=off -fno-fast-math.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define HEAD_DIM 128
+#define PAGE 16
+#define VGROUP 32
+#define BLOCK_BYTES 2816
+#define KCODE_OFF 0
+#define VCODE_OFF 1024
+#define KSCALE_OFF 2048
+#define KZERO_OFF 2304
+#define VSCALE_OFF 2560
+#define VZERO_OFF 2688
+
+/* ---------------------------------------------------------------- fp16 -- */
+
+/* IEEE binary16 -> binary32, exact.  Textbook decoding of the bit fields. */
+float s4kv_ref_half_to_float(uint16_t h) {
+    int sign = (h >> 15) & 1;
+    int e = (h >> 10) & 0x1f;
+    int m = h & 0x3ff;
+    float v;
+    if (e == 0) {
+        v = ldexpf((float)m, -24); /* subnormal: m * 2^-24 */
+    } else if (e == 31) {
+        v = m ? NAN : INFINITY;
+    } else {
+        v = ldexpf((float)(1024 + m), e - 25); /* (1 + m/1024) * 2^(e-15) */
+    }
+    return sign ? -v : v;
+}
+
+/* binary32 -> binary16 with round-to-nearest-even.  The magnitude is scaled
+ * to an integer count of units in the last place of the target format
+ * (exact: a power-of-two scaling), rounded with nearbyint (ties to even
+ * under the default rounding mode), and the bit fields are assembled. */
+uint16_t s4kv_ref_float_to_half(float f) {
+    uint16_t sign = signbit(f) ? 0x8000 : 0;
+    if (isnan(f)) return sign | 0x7e00;
+    double a = fabs((double)f);
+    if (isinf(f)) return sign | 0x7c00;
+    if (a < ldexp(1.0, -14)) {
+        /* subnormal range: unit is 2^-24; a count of 1024 is the smallest
+         * normal, whose bit pattern 0x0400 is the count itself */
+        double q = nearbyint(ldexp(a, 24));
+        return sign | (uint16_t)q;
+    }
+    int e2;
+    frexp(a, &e2);        /* a = mant * 2^e2, mant in [0.5, 1) */
+    int E = e2 - 1;       /* a = (2*mant) * 2^E, 2*mant in [1, 2) */
+    double q = nearbyint(ldexp(a, 10 - E)); /* in [1024, 2048] */
+    if (q == 2048.0) {
+        q = 1024.0;
+        E += 1;
+    }
+    if (E + 15 >= 31) return sign | 0x7c00; /* overflow to infinity */
+    return sign | (uint16_t)(((E + 15) << 10) | ((int)q - 1024));
+}
+
+/* ----------------------------------------------------------- quantizer -- */
+
+/* a < b in IEEE total order restricted to non-NaN values (-0 < +0). */
+static int total_less(float a, float b) {
+    if (a < b) return 1;
+    if (a == b && signbit(a) && !signbit(b)) return 1;
+    return 0;
+}
+
+/* Asymmetric int4 quantization of one group of n fp16 values (the KIVI
+ * step of [S4KV] "Funktionsweise" 1).  x[k*stride] are the fp16 inputs;
+ * codes[k*code_stride] receive the 4-bit codes.  Returns the fp32 scale so
+ * that tests can check the rounding bound against it. */
+float s4kv_ref_quantize_group(const uint16_t *x, int n, int stride,
+                              uint8_t *codes, int code_stride,
+                              uint16_t *scale_h, uint16_t *zero_h) {
+    float mn = s4kv_ref_half_to_float(x[0]);
+    float mx = mn;
+    for (int k = 1; k < n; ++k) {
+        float xv = s4kv_ref_half_to_float(x[k * stride]);
+        if (total_less(xv, mn)) mn = xv;
+        if (total_less(mx, xv)) mx = xv;
+    }
+    volatile float range = mx - mn; /* one fp32 rounding */
+    volatile float s = range / 15.0f; /* one fp32 rounding */
+    for (int k = 0; k < n; ++k) {
+        float xv = s4kv_ref_half_to_float(x[k * stride]);
+        int code = 0;
+        if (s != 0.0f) {
+            volatile float d = xv - mn;
+            volatile float t = d / s;
+            float r = nearbyintf(t); /* ties to even */
+            if (r < 0.0f) r = 0.0f;
+            if (r > 15.0f) r = 15.0f;
+            code = (int)r;
+        }
+        codes[k * code_stride] = (uint8_t)code;
+    }
+    *scale_h = s4kv_ref_float_to_half(s);
+    *zero_h = s4kv_ref_float_to_half(mn);
+    return s;
+}
+
+/* ------------------------------------------------------------- packing -- */
+
+/* (token, channel) -> (word, nibble) of the key code region. */
+void s4kv_ref_key_code_slot(int t, int c, int *word, int *nibble) {
+    int i = c / 32, kt = (c % 32) / 4, e = c % 4;
+    int n = t % 8;
+    *nibble = (t / 8) + 2 * (e / 2) + 4 * (e % 2);
+    *word = 128 * (kt / 4) + 4 * (4 * n + i) + (kt % 4);
+}
+
+/* (token, channel) -> (word, nibble) of the value code region. */
+void s4kv_ref_value_code_slot(int t, int c, int *word, int *nibble) {
+    int grp = c / 32, n = (c % 32) / 4, e = c % 4;
+    int m = 2 * grp + e / 2;
+    int i = (t % 8) / 2;
+    *nibble = (e % 2) + 2 * (t / 8) + 4 * (t % 2);
+    *word = 128 * (m / 4) + 4 * (4 * n + i) + (m % 4);
+}
+
+static void put_nibble(uint8_t *region, int word, int nibble, int code) {
+    uint8_t *byte = region + 4 * word + nibble / 2; /* little-endian word */
+    int sh = 4 * (nibble % 2);
+    *byte = (uint8_t)((*byte & ~(0xf << sh)) | ((code & 0xf) << sh));
+}
+
+static int get_nibble(const uint8_t *region, int word, int nibble) {
+    const uint8_t *byte = region + 4 * word + nibble / 2;
+    return (*byte >> (4 * (nibble % 2))) & 0xf;
+}
+
+static void put_half(uint8_t *p, uint16_t h) { memcpy(p, &h, 2); }
+static uint16_t get_half(const uint8_t *p) {
+    uint16_t h;
+    memcpy(&h, p, 2);
+    return h;
+}
+
+/* Quantize one full page of one kv head.  kp, vp: fp16 [16][128] rows.
+ * Writes the 2816-byte block. */
+void s4kv_ref_quantize_page(const uint16_t *kp, const uint16_t *vp,
+                            uint8_t *block) {
+    uint8_t kc[PAGE][HEAD_DIM], vc[PAGE][HEAD_DIM];
+    memset(block, 0, BLOCK_BYTES);
+    /* keys: one group per channel, over the page's 16 tokens */
+    for (int c = 0; c < HEAD_DIM; ++c) {
+        uint16_t sh, zh;
+        s4kv_ref_quantize_group(kp + c, PAGE, HEAD_DIM, &kc[0][c], HEAD_DIM,
+                                &sh, &zh);
+        put_half(block + KSCALE_OFF + 2 * c, sh);
+        put_half(block + KZERO_OFF + 2 * c, zh);
+    }
+    /* values: one group per token and 32-channel slice */
+    for (int t = 0; t < PAGE; ++t) {
+        for (int g = 0; g < HEAD_DIM / VGROUP; ++g) {
+            uint16_t sh, zh;
+            s4kv_ref_quantize_group(vp + t * HEAD_DIM + g * VGROUP, VGROUP, 1,
+                                    &vc[t][g * VGROUP], 1, &sh, &zh);
+            put_half(block + VSCALE_OFF + 2 * (g * PAGE + t), sh);
+            put_half(block + VZERO_OFF + 2 * (g * PAGE + t), zh);
+        }
+    }
+    for (int t = 0; t < PAGE; ++t) {
+        for (int c = 0; c < HEAD_DIM; ++c) {
+            int w, nb;
+            s4kv_ref_key_code_slot(t, c, &w, &nb);
+            put_nibble(block + KCODE_OFF, w, nb, kc[t][c]);
+            s4kv_ref_value_code_slot(t, c, &w, &nb);
+            put_nibble(block + VCODE_OFF, w, nb, vc[t][c]);
+        }
+    }
+}
+
+/* Read back the codes of one block in natural [token][channel] order. */
+void s4kv_ref_unpack_codes(const uint8_t *block, uint8_t *kcodes,
+                           uint8_t *vcodes) {
+    for (int t = 0; t < PAGE; ++t) {
+        for (int c = 0; c < HEAD_DIM; ++c) {
+            int w, nb;
+            s4kv_ref_key_code_slot(t, c, &w, &nb);
+            kcodes[t * HEAD_DIM + c] = (uint8_t)get_nibble(block + KCODE_OFF, w, nb);
+            s4kv_ref_value_code_slot(t, c, &w, &nb);
+            vcodes[t * HEAD_DIM + c] = (uint8_t)get_nibble(block + VCODE_OFF, w, nb);
+        }
+    }
+}
+
+/* Dequantize one block: x = code * scale + zero, in fp32 (the product of a
+ * 4-bit code and an fp16 scale is exact in fp32, so this is one rounding).
+ * kout, vout: fp32 [16][128]. */
+void s4kv_ref_dequant_block(const uint8_t *block, float *kout, float *vout) {
+    uint8_t kc[PAGE * HEAD_DIM], vc[PAGE * HEAD_DIM];
+    s4kv_ref_unpack_codes(block, kc, vc);
+    for (int t = 0; t < PAGE; ++t) {
+        for (int c = 0; c < HEAD_DIM; ++c) {
+            float ks = s4kv_ref_half_to_float(get_half(block + KSCALE_OFF + 2 * c));
+            float kz = s4kv_ref_half_to_float(get_half(block + KZERO_OFF + 2 * c));
+            int g = c / VGROUP;
+            float vs = s4kv_ref_half_to_float(get_half(block + VSCALE_OFF + 2 * (g * PAGE + t)));
+            float vz = s4kv_ref_half_to_float(get_half(block + VZERO_OFF + 2 * (g * PAGE + t)));
+            volatile float kprod = (float)kc[t * HEAD_DIM + c] * ks;
+            volatile float vprod = (float)vc[t * HEAD_DIM + c] * vs;
+            kout[t * HEAD_DIM + c] = kprod + kz;
+            vout[t * HEAD_DIM + c] = vprod + vz;
+        }
+    }
+}
+
+/* --------------------------------------------------------------- cache -- */
+
+/* Return codes shared with the tests (values of the library's header are
+ * not included here on purpose; the tests compare meanings, not numbers). */
+#define REF_OK 0
+#define REF_BAD_ARG 1
+#define REF_BAD_SLOT 2
+
+/* Bytes of one (page, kv head) block of this layout, derived from its
+ * parts: 4-bit codes for K and V plus fp16 scale/zero metadata. */
+long s4kv_ref_block_bytes(void) {
+    long codes = 2L * PAGE * HEAD_DIM / 2;                   /* K + V, 4 bits */
+    long kmeta = 2L * HEAD_DIM * 2;                          /* scale + zero */
+    long vmeta = 2L * PAGE * (HEAD_DIM / VGROUP) * 2;        /* scale + zero */
+    return codes + kmeta + vmeta;
+}
+
+/* The KV payload formula of [CAP]: 2 x layers x kv_heads x head_dim x
+ * tokens x bytes per element (no metadata, no block rounding). */
+double s4kv_ref_kv_payload_bytes(long layers, long kv_heads, long head_dim,
+                                 long tokens, double bytes_per_elem) {
+    return 2.0 * (double)layers * (double)kv_heads * (double)head_dim *
+           (double)tokens * bytes_per_elem;
+}
+
+/* Append new fp16 K/V tokens (token-major [n_tokens][kv_heads][128]) to the
+ * cache, one token at a time in sequence order: each token is written to its
+ * sequence's residual row pos mod 16; when that row is 15 the page is
+ * complete and is quantized from the residual into the physical page
+ * block_tables[b][pos/16] ([PAGED] page tables; [S4KV] per-channel keys and
+ * per-token values, keys quantized once the page is full).
+ * cu_new[b]..cu_new[b+1] are sequence b's new tokens; seq_lens[b] is its
+ * length after the append.  slot_mapping[tok] must equal
+ * block_tables[b][pos/16] * 16 + pos % 16. */
+int s4kv_ref_append(uint8_t *pool, uint16_t *res_k, uint16_t *res_v,
+                    int num_pages, int num_kv_heads, int max_seqs,
+                    const uint16_t *k, const uint16_t *v, int n_tokens,
+                    const int64_t *slot_mapping, const int32_t *cu_new,
+                    const int32_t *seq_lens, const int32_t *block_tables,
+                    int batch, int max_pages_per_seq) {
+    if (batch < 0 || batch > max_seqs || n_tokens < 0) return REF_BAD_ARG;
+    if (cu_new[0] != 0 || cu_new[batch] != n_tokens) return REF_BAD_ARG;
+    const long row = HEAD_DIM;
+    for (int b = 0; b < batch; ++b) {
+        int n_b = cu_new[b + 1] - cu_new[b];
+        int L = seq_lens[b];
+        int L0 = L - n_b;
+        if (n_b < 0 || L0 < 0 || (L + PAGE - 1) / PAGE > max_pages_per_seq)
+            return REF_BAD_ARG;
+        for (int j = 0; j < n_b; ++j) {
+            int pos = L0 + j;
+            int tok = cu_new[b] + j;
+            int page = block_tables[(long)b * max_pages_per_seq + pos / PAGE];
+            if (page < 0 || page >= num_pages) return REF_BAD_SLOT;
+            if (slot_mapping[tok] != (int64_t)page * PAGE + pos % PAGE)
+                return REF_BAD_SLOT;
+            int r = pos % PAGE;
+            for (int h = 0; h < num_kv_heads; ++h) {
+                uint16_t *rk = res_k + (((long)b * num_kv_heads + h) * PAGE) * row;
+                uint16_t *rv = res_v + (((long)b * num_kv_heads + h) * PAGE) * row;
+                memcpy(rk + r * row, k + ((long)tok * num_kv_heads + h) * row, 2 * row);
+                memcpy(rv + r * row, v + ((long)tok * num_kv_heads + h) * row, 2 * row);
+                if (r == PAGE - 1) {
+                    uint8_t *blk = pool + ((long)page * num_kv_heads + h) * BLOCK_BYTES;
+                    s4kv_ref_quantize_page(rk, rv, blk);
+                }
+            }
+        }
+    }
+    return REF_OK;
+}
+
+/* Dequantize one physical page for all kv heads.  out_k, out_v: fp32
+ * [kv_heads][16][128]. */
+int s4kv_ref_dequant_page(const uint8_t *pool, int num_pages, int num_kv_heads,
+                          int physical_page, float *out_k, float *out_v) {
+    if (physical_page < 0 || physical_page >= num_pages) return REF_BAD_ARG;
+    for (int h = 0; h < num_kv_heads; ++h) {
+        const uint8_t *blk = pool + ((long)physical_page * num_kv_heads + h) * BLOCK_BYTES;
+        s4kv_ref_dequant_block(blk, out_k + (long)h * PAGE * HEAD_DIM,
+                               out_v + (long)h * PAGE * HEAD_DIM);
+    }
+    return REF_OK;
+}
+
+/* Gather the K and V rows (fp32 [L][128]) of sequence b, kv head h: full
+ * pages are dequantized page by page, the tail comes from the fp16
+ * residual. */
+static void sequence_kv(const uint8_t *pool, const uint16_t *res_k,
+                        const uint16_t *res_v, int num_kv_heads,
+                        const int32_t *bt_row, int L, int b, int h,
+                        float *K, float *V) {
+    int full = L / PAGE;
+    for (int p = 0; p < full; ++p) {
+        const uint8_t *blk = pool + ((long)bt_row[p] * num_kv_heads + h) * BLOCK_BYTES;
+        s4kv_ref_dequant_block(blk, K + (long)p * PAGE * HEAD_DIM,
+                               V + (long)p * PAGE * HEAD_DIM);
+    }
+    for (int t = full * PAGE; t < L; ++t) {
+        int r = t % PAGE;
+        const uint16_t *rk = res_k + (((long)b * num_kv_heads + h) * PAGE + r) * HEAD_DIM;
+        const uint16_t *rv = res_v + (((long)b * num_kv_heads + h) * PAGE + r) * HEAD_DIM;
+        for (int c = 0; c < HEAD_DIM; ++c) {
+            K[(long)t * HEAD_DIM + c] = s4kv_ref_half_to_float(rk[c]);
+            V[(long)t * HEAD_DIM + c] = s4kv_ref_half_to_float(rv[c]);
+        }
+    }
+}
+
+/* GQA decode attention over the cache ([KVOPT] GQA: query head j reads kv
+ * head j / (num_q_heads / num_kv_heads)).  For each sequence b and query
+ * head: logits_t = sm_scale * sum_c q_c * k_tc over the L_b tokens, a
+ * two-pass softmax (max, then exp and sum) and out = sum_t p_t v_t / sum p.
+ * q: fp16 [batch][num_q_heads][128]; out: fp64 [batch][num_q_heads][128].
+ * use_double selects fp64 (1) or fp32 (0) for every step after the fp32
+ * dequantization.  Sequences of length 0 give an all-zero output. */
+int s4kv_ref_decode_attention(const uint8_t *pool, const uint16_t *res_k,
+                              const uint16_t *res_v, int num_pages,
+                              int num_kv_heads, const uint16_t *q,
+                              int num_q_heads, const int32_t *seq_lens,
+                              const int32_t *block_tables, int batch,
+                              int max_pages_per_seq, double sm_scale,
+                              int use_double, double *out) {
+    if (num_kv_heads <= 0 || num_q_heads % num_kv_heads != 0) return REF_BAD_ARG;
+    int G = num_q_heads / num_kv_heads;
+    for (int b = 0; b < batch; ++b) {
+        int L = seq_lens[b];
+        const int32_t *bt_row = block_tables + (long)b * max_pages_per_seq;
+        if (L < 0 || (L + PAGE - 1) / PAGE > max_pages_per_seq) return REF_BAD_ARG;
+        for (int p = 0; p < L / PAGE; ++p)
+            if (bt_row[p] < 0 || bt_row[p] >= num_pages) return REF_BAD_SLOT;
+        for (int h = 0; h < num_kv_heads; ++h) {
+            /* rounded up to whole pages: sequence_kv fills full pages */
+            size_t rows = (size_t)((L + PAGE - 1) / PAGE + 1) * PAGE;
+            float *K = (float *)malloc(sizeof(float) * rows * HEAD_DIM);
+            float *V = (float *)malloc(sizeof(float) * rows * HEAD_DIM);
+            double *logit = (double *)malloc(sizeof(double) * (size_t)(L > 0 ? L : 1));
+            if (!K || !V || !logit) { free(K); free(V); free(logit); return REF_BAD_ARG; }
+            sequence_kv(pool, res_k, res_v, num_kv_heads, bt_row, L, b, h, K, V);
+            for (int g = 0; g < G; ++g) {
+                int qh = h * G + g;
+                const uint16_t *qv = q + ((long)b * num_q_heads + qh) * HEAD_DIM;
+                double *o = out + ((long)b * num_q_heads + qh) * HEAD_DIM;
+                if (L == 0) {
+                    for (int c = 0; c < HEAD_DIM; ++c) o[c] = 0.0;
+                    continue;
+                }
+                if (use_double) {
+                    double mx = -INFINITY;
+                    for (int t = 0; t < L; ++t) {
+                        double acc = 0.0;
+                        for (int c = 0; c < HEAD_DIM; ++c)
+                            acc += (double)s4kv_ref_half_to_float(qv[c]) * (double)K[(long)t * HEAD_DIM + c];
+                        logit[t] = sm_scale * acc;
+                        if (logit[t] > mx) mx = logit[t];
+                    }
+                    double sum = 0.0;
+                    for (int t = 0; t < L; ++t) {
+                        logit[t] = exp(logit[t] - mx);
+                        sum += logit[t];
+                    }
+                    for (int c = 0; c < HEAD_DIM; ++c) {
+                        double acc = 0.0;
+                        for (int t = 0; t < L; ++t) acc += logit[t] * (double)V[(long)t * HEAD_DIM + c];
+                        o[c] = acc / sum;
+                    }
+                } else {
+                    float mx = -INFINITY;
+                    float sc = (float)sm_scale;
+                    for (int t = 0; t < L; ++t) {
+                        float acc = 0.0f;
+                        for (int c = 0; c < HEAD_DIM; ++c)
+                            acc += s4kv_ref_half_to_float(qv[c]) * K[(long)t * HEAD_DIM + c];
+                        logit[t] = (double)(sc * acc);
+                        if ((float)logit[t] > mx) mx = (float)logit[t];
+                    }
+                    float sum = 0.0f;
+                    for (int t = 0; t < L; ++t) {
+                        float e = expf((float)logit[t] - mx);
+                        logit[t] = (double)e;
+                        sum += e;
+                    }
+                    for (int c = 0; c < HEAD_DIM; ++c) {
+                        float acc = 0.0f;
+                        for (int t = 0; t < L; ++t) acc += (float)logit[t] * V[(long)t * HEAD_DIM + c];
+                        o[c] = (double)(acc / sum);
+                    }
+                }
+            }
+            free(K);
+            free(V);
+            free(logit);
+        }
+    }
+    return REF_OK;
+}
+
+/* Attention on unquantized fp16 K/V rows given directly ([n][128] per
+ * (sequence, kv head)); used only to report the quantization error.
+ * k, v: fp16 [total_tokens][num_kv_heads][128] with sequence b occupying
+ * rows cu[b]..cu[b+1]. */
+int s4kv_ref_attention_fp16(const uint16_t *k, const uint16_t *v,
+                            const int32_t *cu, int num_kv_heads,
+                            const uint16_t *q, int num_q_heads, int batch,
+                            double sm_scale, double *out) {
+    int G = num_q_heads / num_kv_heads;
+    for (int b = 0; b < batch; ++b) {
+        int L = cu[b + 1] - cu[b];
+        double *logit = (double *)malloc(sizeof(double) * (size_t)(L > 0 ? L : 1));
+        if (!logit) return REF_BAD_ARG;
+        for (int qh = 0; qh < num_q_heads; ++qh) {
+            int h = qh / G;
+            const uint16_t *qv = q + ((long)b * num_q_heads + qh) * HEAD_DIM;
+            double *o = out + ((long)b * num_q_heads + qh) * HEAD_DIM;
+            if (L == 0) {
+                for (int c = 0; c < HEAD_DIM; ++c) o[c] = 0.0;
+                continue;
+            }
+            double mx = -INFINITY;
+            for (int t = 0; t < L; ++t) {
+                const uint16_t *kr = k + ((long)(cu[b] + t) * num_kv_heads + h) * HEAD_DIM;
+                double acc = 0.0;
+                for (int c = 0; c < HEAD_DIM; ++c)
+                    acc += (double)s4kv_ref_half_to_float(qv[c]) * (double)s4kv_ref_half_to_float(kr[c]);
+                logit[t] = sm_scale * acc;
+                if (logit[t] > mx) mx = logit[t];
+            }
+            double sum = 0.0;
+            for (int t = 0; t < L; ++t) {
+                logit[t] = exp(logit[t] - mx);
+                sum += logit[t];
+            }
+            for (int c = 0; c < HEAD_DIM; ++c) {
+                double acc = 0.0;
+                for (int t = 0; t < L; ++t) {
+                    const uint16_t *vr = v + ((long)(cu[b] + t) * num_kv_heads + h) * HEAD_DIM;
+                    acc += logit[t] * (double)s4kv_ref_half_to_float(vr[c]);
+                }
+                o[c] = acc / sum;
+            }
+        }
+        free(logit);
+    }
+    return REF_OK;
+}

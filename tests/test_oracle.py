@@ -1,0 +1,459 @@
+"""Pins for the CPU oracle: each test ties an oracle function to something other
+than the oracle itself -- a figure the pages print, a closed form, a textbook
+or library routine, an invariant, or brute force on tiny inputs.
+
+Which pin covers which oracle function:
+  half_to_float / float_to_half : numpy's IEEE binary16 conversion (exhaustive
+                                   and on rounding ties)
+  quantize_group                : closed forms (exact grids, all-equal groups,
+                                   signed zeros) and the exact-rational rounding
+                                   bound |x - (code*s + min)| <= s*(1/2 + 2e-6)
+  key/value code slots, packing : bijection over all (token, channel); the
+                                   per-channel / per-token closed forms read back
+  block_bytes, kv_payload_bytes : the pages' worked sizes (tests/golden/kv_bytes.txt)
+                                   and the ~3x density claim
+  append                        : chunking invariance; closed-form page contents;
+                                   slot_mapping check
+  dequant                       : closed-form grids dequantize exactly
+  decode_attention              : textbook softmax attention (numpy) on inputs the
+                                   quantizer represents exactly; single key; uniform
+                                   weights; page permutation and shared-prefix
+                                   invariance; GQA identical queries; fp32 vs fp64
+"""
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+
+HD, PAGE = 128, 16
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def f16bits(x):
+    return np.asarray(x, np.float16).view(np.uint16)
+
+
+# ------------------------------------------------------------------ fp16 --
+
+def test_half_to_float_exhaustive(oracle_mod):
+    bits = np.arange(65536, dtype=np.uint32)
+    ref = bits.astype(np.uint16).view(np.float16).astype(np.float32)
+    got = np.array([oracle_mod.half_to_float(int(b)) for b in bits], np.float32)
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(got), nan)
+    assert np.array_equal(got[~nan].view(np.uint32), ref[~nan].view(np.uint32))
+
+
+def test_float_to_half_matches_numpy_including_ties(oracle_mod):
+    rng = np.random.default_rng(7)
+    vals = [rng.standard_normal(4000).astype(np.float32) * s for s in (1e-7, 1e-5, 1e-3, 1, 100, 3e4)]
+    vals.append(np.array([0.0, -0.0, 65504, 65519.99, 65520, 65536, 1e10, -1e10,
+                          2 ** -24, 2 ** -25, 3 * 2 ** -26, 2 ** -14, np.inf, -np.inf], np.float32))
+    # exact ties halfway between neighbouring halves (exact in fp32)
+    h = rng.integers(0, 0x7BFF, 4000).astype(np.uint16)
+    lo = h.view(np.float16).astype(np.float32)
+    hi = (h + 1).view(np.float16).astype(np.float32)
+    vals.append(((lo.astype(np.float64) + hi) / 2).astype(np.float32))
+    x = np.concatenate(vals).astype(np.float32)
+    ref = x.astype(np.float16).view(np.uint16)
+    got = np.array([oracle_mod.float_to_half(float(v)) for v in x], np.uint16)
+    assert np.array_equal(got, ref)
+
+
+# ------------------------------------------------------------- quantizer --
+
+def test_quantize_group_integer_grid(oracle_mod):
+    x = np.arange(16, dtype=np.float16)
+    codes, sh, zh, s = oracle_mod.quantize_group(x)
+    assert list(codes) == list(range(16))
+    assert s == 1.0 and sh == 0x3C00 and zh == 0
+
+
+def test_quantize_group_shifted_progression(oracle_mod):
+    d, a = 2.0 ** -3, -1.5
+    k = np.array([3, 0, 15, 7, 9, 1, 14, 2, 5, 6, 8, 10, 4, 11, 12, 13])
+    x = (a + k * d).astype(np.float16)
+    codes, sh, zh, s = oracle_mod.quantize_group(x)
+    assert list(codes) == list(k)
+    assert s == d and sh == f16bits(d) and zh == f16bits(a)
+
+
+def test_quantize_group_all_equal_and_signed_zero(oracle_mod):
+    codes, sh, zh, s = oracle_mod.quantize_group(np.full(32, 0.7, np.float16))
+    assert s == 0.0 and sh == 0 and (codes == 0).all() and zh == f16bits(0.7)
+    z = np.array([0.0, -0.0] * 8, np.float16)
+    codes, sh, zh, s = oracle_mod.quantize_group(z)
+    assert s == 0.0 and (codes == 0).all() and zh == 0x8000  # min in total order is -0
+
+
+def _bound_ok(x16, codes, s32, zero_bits):
+    mn = Fraction(float(np.uint16(zero_bits).view(np.float16)))
+    S = Fraction(s32)
+    for xv, c in zip(x16.astype(np.float64), codes):
+        err = abs(Fraction(float(xv)) - (c * S + mn))
+        if err > S * Fraction(1, 2) + S * Fraction(2, 10 ** 6):
+            return False
+    return True
+
+
+@pytest.mark.parametrize("kind", ["normal", "subnormal", "large", "outlier", "two-level"])
+def test_quantize_group_rounding_bound(oracle_mod, kind):
+    rng = np.random.default_rng(11)
+    for trial in range(60):
+        n = 16 if trial % 2 else 32
+        if kind == "normal":
+            x = rng.standard_normal(n)
+        elif kind == "subnormal":
+            x = rng.integers(-40, 40, n) * 2.0 ** -24
+        elif kind == "large":
+            x = rng.uniform(-60000, 60000, n)
+        elif kind == "outlier":
+            x = rng.standard_normal(n)
+            x[rng.integers(n)] *= 300
+        else:
+            x = rng.choice([-2.5, 3.25], n)
+        x16 = np.asarray(x).astype(np.float16)
+        codes, sh, zh, s = oracle_mod.quantize_group(x16)
+        assert codes.min() >= 0 and codes.max() <= 15
+        assert zh == x16[np.argmin(x16)].view(np.uint16) or float(x16.min()) == 0.0
+        if s > 0:
+            assert codes[np.argmin(x16)] == 0 and codes[np.argmax(x16)] == 15
+            assert _bound_ok(x16, codes, s, zh)
+        assert sh == np.float32(s).astype(np.float16).view(np.uint16)
+
+
+# ---------------------------------------------------------------- layout --
+
+def test_code_slots_are_a_bijection(oracle_mod):
+    for slot in (oracle_mod.key_code_slot, oracle_mod.value_code_slot):
+        seen = set()
+        for t in range(PAGE):
+            for c in range(HD):
+                w, nb = slot(t, c)
+                assert 0 <= w < 256 and 0 <= nb < 8
+                seen.add((w, nb))
+        assert len(seen) == PAGE * HD
+
+
+def _fragment_position(word, nibble):
+    """Where a nibble lands in the warp-level MMA operand, per the PTX ISA's
+    fragment table for mma.m16n8k16 (row-major A, f16): lane = 4*g + t holds
+    a0 = (row g, cols 2t, 2t+1), a1 = (row g+8, same cols), a2 = (row g,
+    cols 2t+8, 2t+9), a3 = (row g+8, cols 2t+8, 2t+9), the lower column in the
+    low half.  The library unpacks nibble j of a lane's word into register
+    j & 3, half j >> 2.  Returns (tile, lane, row, col)."""
+    tile = 4 * (word // 128) + word % 4
+    lane = (word % 128) // 4
+    g, t = lane // 4, lane % 4
+    r, e = nibble & 3, nibble >> 2
+    return tile, lane, g + 8 * (r & 1), 2 * t + e + 8 * (r >> 1)
+
+
+def test_code_layout_is_the_mma_operand_order(oracle_mod):
+    """Each 32-bit code word is one lane's tensor-core A fragment: for keys,
+    rows are tokens and the k axis of tile kt is lane t's channels
+    32t + 4kt + {0,1} (cols 2t, 2t+1) and + {2,3} (cols 2t+8, 2t+9), matching
+    a B fragment that holds channels 32t..32t+31; for values, rows of M-tile m
+    are channels 32*(m//2) + 4*(row%8) + 2*(m%2) + row//8 and the k axis is the
+    token index."""
+    for t in range(PAGE):
+        for c in range(HD):
+            tile, lane, row, col = _fragment_position(*oracle_mod.key_code_slot(t, c))
+            tq = lane % 4
+            k_slot_channel = 32 * tq + 4 * tile + ((col - 2 * tq) if col < 8 else 2 + (col - 2 * tq - 8))
+            assert (row, k_slot_channel) == (t, c)
+            tile, lane, row, col = _fragment_position(*oracle_mod.value_code_slot(t, c))
+            ch = 32 * (tile // 2) + 4 * (row % 8) + 2 * (tile % 2) + row // 8
+            assert (col, ch) == (t, c)
+
+
+def _grid_page(rng, per="key"):
+    """fp16 [16][128] whose groups are exact 16-level grids: returns the page,
+    expected codes, and per-group (scale, zero)."""
+    if per == "key":   # group = channel over the 16 tokens
+        d = 2.0 ** rng.integers(-6, 0, HD)
+        a = rng.integers(-64, 64, HD) * d
+        codes = np.stack([rng.permutation(16) for _ in range(HD)], axis=1)  # [t][c]
+        x = (a[None, :] + codes * d[None, :]).astype(np.float16)
+        return x, codes, d, a
+    # value: group = 32 channels of one token; two copies of a 16-level grid
+    d = 2.0 ** rng.integers(-6, 0, (PAGE, 4))
+    a = rng.integers(-64, 64, (PAGE, 4)) * d
+    codes = np.zeros((PAGE, HD), np.int64)
+    for t in range(PAGE):
+        for g in range(4):
+            codes[t, 32 * g:32 * g + 32] = np.concatenate([rng.permutation(16), rng.permutation(16)])
+    x = (a.repeat(32, axis=1) + codes * d.repeat(32, axis=1)).astype(np.float16)
+    return x, codes, d, a
+
+
+def test_page_axis_split_closed_form(oracle_mod):
+    """Keys are quantized per channel and values per token in 32-channel
+    groups ("S4 KV", "Funktionsweise" 1): on exact grids the stored scale is
+    the grid step of exactly that group and the codes are the grid indices."""
+    rng = np.random.default_rng(3)
+    k, kc_ref, kd, ka = _grid_page(rng, "key")
+    v, vc_ref, vd, va = _grid_page(rng, "value")
+    blk = oracle_mod.quantize_page(k, v)
+    assert blk.size == 2816
+    kc, vc = oracle_mod.unpack_codes(blk)
+    assert np.array_equal(kc, kc_ref) and np.array_equal(vc, vc_ref)
+    ks = blk[2048:2304].view(np.float16).astype(np.float64)
+    kz = blk[2304:2560].view(np.float16).astype(np.float64)
+    vs = blk[2560:2688].view(np.float16).astype(np.float64).reshape(4, 16)
+    vz = blk[2688:2816].view(np.float16).astype(np.float64).reshape(4, 16)
+    assert np.array_equal(ks, kd) and np.array_equal(kz, ka)
+    assert np.array_equal(vs, vd.T) and np.array_equal(vz, va.T)
+    kdq, vdq = oracle_mod.dequant_block(blk)
+    assert np.array_equal(kdq, k.astype(np.float32)) and np.array_equal(vdq, v.astype(np.float32))
+
+
+# ------------------------------------------------------------ byte model --
+
+def test_kv_byte_formula_reproduces_page_figures(oracle_mod):
+    rows = [l.split() for l in open(os.path.join(GOLDEN, "kv_bytes.txt"))
+            if l.strip() and not l.startswith("#")]
+    assert len(rows) == 4
+    for r in rows:
+        L, H, D, T, by, lo, hi = int(r[0]), int(r[1]), int(r[2]), int(r[3]), float(r[4]), float(r[5]), float(r[6])
+        got = oracle_mod.kv_payload_bytes(L, H, D, T, by)
+        assert lo <= got <= hi, (r, got)
+    assert oracle_mod.kv_payload_bytes(80, 8, 128, 4096, 2) == 1342177280
+
+
+def test_density_about_three_times(oracle_mod):
+    """"S4 KV" intro and "Highlights": about 3x more KV density than fp16;
+    "KV-Cache-Optimierung", "Warum es zaehlt": INT4 quarters the payload."""
+    fp16 = oracle_mod.kv_payload_bytes(1, 1, 128, 16, 2.0)
+    assert fp16 == 8192
+    blk = oracle_mod.block_bytes()
+    assert blk == 2816
+    assert 2.75 <= fp16 / blk <= 3.25
+    assert fp16 / oracle_mod.kv_payload_bytes(1, 1, 128, 16, 0.5) == 4.0
+
+
+# ---------------------------------------------------------------- append --
+
+def _append_all(oracle_mod, cache, k, v, lens_before, lens_after, bt, chunk=None):
+    """Append tokens lens_before..lens_after for every sequence (k, v are the
+    per-sequence full streams) in chunks of `chunk` tokens per call."""
+    B = len(lens_after)
+    cur = np.array(lens_before, np.int64)
+    tgt = np.array(lens_after, np.int64)
+    while (cur < tgt).any():
+        take = tgt - cur if chunk is None else np.minimum(tgt - cur, chunk)
+        ks, vs, pos_list = [], [], []
+        for b in range(B):
+            pos = np.arange(cur[b], cur[b] + take[b])
+            pos_list.append(pos)
+            ks.append(k[b][pos])
+            vs.append(v[b][pos])
+        from int4_kivi_quantized_s4kv_b200 import workloads
+        sm = workloads.slot_mapping(bt, pos_list)
+        cu = np.concatenate([[0], np.cumsum(take)]).astype(np.int32)
+        rc = cache.append(np.concatenate(ks), np.concatenate(vs), sm, cu,
+                          (cur + take).astype(np.int32), bt)
+        assert rc == 0
+        cur = cur + take
+
+
+def _rand_kv(rng, B, H, lens):
+    k = [rng.standard_normal((L, H, HD)).astype(np.float16) for L in lens]
+    v = [rng.standard_normal((L, H, HD)).astype(np.float16) for L in lens]
+    return k, v
+
+
+def _tables(rng, lens, extra=3):
+    need = [(L + PAGE - 1) // PAGE for L in lens]
+    NP = sum(need) + extra
+    perm = rng.permutation(NP).astype(np.int32)
+    bt = np.full((len(lens), max(need)), -1, np.int32)
+    c = 0
+    for b, n in enumerate(need):
+        bt[b, :n] = perm[c:c + n]
+        c += n
+    return bt, NP
+
+
+def test_append_chunking_invariance(oracle_mod):
+    rng = np.random.default_rng(5)
+    lens = [37, 50, 16, 5]
+    H = 2
+    k, v = _rand_kv(rng, 4, H, lens)
+    bt, NP = _tables(rng, lens)
+    caches = []
+    for chunk in (None, 1, 7, 16, 23):
+        c = oracle_mod.OracleCache(NP, H, 4)
+        _append_all(oracle_mod, c, k, v, [0] * 4, lens, bt, chunk)
+        caches.append(c)
+    for c in caches[1:]:
+        assert np.array_equal(c.pool, caches[0].pool)
+        for b, L in enumerate(lens):
+            r = L % PAGE
+            assert np.array_equal(c.res_k[b, :, :r], caches[0].res_k[b, :, :r])
+            assert np.array_equal(c.res_v[b, :, :r], caches[0].res_v[b, :, :r])
+    # residual rows are the sequence's tail tokens, bit for bit
+    for b, L in enumerate(lens):
+        r = L % PAGE
+        tail = k[b][L - r:L].transpose(1, 0, 2)
+        assert np.array_equal(caches[0].res_k[b, :, :r], tail.view(np.uint16))
+
+
+def test_append_page_contents_closed_form(oracle_mod):
+    rng = np.random.default_rng(9)
+    kp, kcodes, kd, ka = _grid_page(rng, "key")
+    vp, vcodes, vd, va = _grid_page(rng, "value")
+    k = [kp[:, None, :]]
+    v = [vp[:, None, :]]
+    bt = np.array([[2]], np.int32)
+    c = oracle_mod.OracleCache(4, 1, 1)
+    _append_all(oracle_mod, c, k, v, [0], [16], bt, chunk=5)
+    kc, vc = oracle_mod.unpack_codes(c.pool[2, 0])
+    assert np.array_equal(kc, kcodes) and np.array_equal(vc, vcodes)
+    assert (c.pool[[0, 1, 3]] == 0).all()
+
+
+def test_append_rejects_inconsistent_slot(oracle_mod):
+    c = oracle_mod.OracleCache(4, 1, 1)
+    k = np.zeros((3, 1, HD), np.float16)
+    bt = np.array([[1]], np.int32)
+    sm = np.array([16, 17, 19], np.int64)  # third token should be slot 18
+    rc = c.append(k, k, sm, np.array([0, 3], np.int32), np.array([3], np.int32), bt)
+    assert rc != 0
+
+
+# ------------------------------------------------------- decode attention --
+
+def _textbook_attention(q, K, V, scale):
+    """softmax(scale * q K^T) V in float64 with numpy, per (b, q head)."""
+    s = scale * (K.astype(np.float64) @ q.astype(np.float64))
+    s -= s.max()
+    p = np.exp(s)
+    return (p[:, None] * V.astype(np.float64)).sum(0) / p.sum()
+
+
+def _build_cache(oracle_mod, k, v, lens, bt, NP, H, chunk=None):
+    c = oracle_mod.OracleCache(NP, H, len(lens))
+    _append_all(oracle_mod, c, k, v, [0] * len(lens), lens, bt, chunk)
+    return c
+
+
+def test_decode_matches_textbook_attention_on_exact_grids(oracle_mod):
+    """On K/V the quantizer represents exactly, decode attention must equal
+    plain softmax attention (numpy, float64) on the original fp16 values: this
+    pins page addressing, GQA head mapping, the residual and the softmax."""
+    rng = np.random.default_rng(21)
+    H, G = 2, 4
+    lens = [37, 64, 3, 50]
+    k, v = [], []
+    for L in lens:
+        npg = (L + PAGE - 1) // PAGE
+        kk = np.zeros((npg * PAGE, H, HD), np.float16)
+        vv = np.zeros((npg * PAGE, H, HD), np.float16)
+        for p in range(npg):
+            for h in range(H):
+                kk[p * PAGE:(p + 1) * PAGE, h] = _grid_page(rng, "key")[0]
+                vv[p * PAGE:(p + 1) * PAGE, h] = _grid_page(rng, "value")[0]
+        k.append(kk[:L])
+        v.append(vv[:L])
+    bt, NP = _tables(rng, lens)
+    c = _build_cache(oracle_mod, k, v, lens, bt, NP, H, chunk=9)
+    q = rng.standard_normal((len(lens), H * G, HD)).astype(np.float16)
+    out = c.decode_attention(q, np.array(lens, np.int32), bt)
+    scale = 1 / np.sqrt(HD)
+    for b, L in enumerate(lens):
+        for qh in range(H * G):
+            ref = _textbook_attention(q[b, qh], k[b][:, qh // G], v[b][:, qh // G], scale)
+            assert np.allclose(out[b, qh], ref, rtol=1e-12, atol=1e-12)
+
+
+def test_single_key_returns_its_value(oracle_mod):
+    rng = np.random.default_rng(1)
+    k, v = _rand_kv(rng, 3, 1, [1, 1, 1])
+    bt, NP = _tables(rng, [1, 1, 1])
+    c = _build_cache(oracle_mod, k, v, [1, 1, 1], bt, NP, 1)
+    q = rng.standard_normal((3, 4, HD)).astype(np.float16)
+    out = c.decode_attention(q, np.array([1, 1, 1], np.int32), bt)
+    for b in range(3):
+        for qh in range(4):
+            assert np.array_equal(out[b, qh], v[b][0, 0].astype(np.float64))
+
+
+def test_zero_query_gives_mean_of_values(oracle_mod):
+    """q = 0 makes every weight equal; with values constant inside each
+    quantization group the dequantized values are exact, so the output is the
+    plain mean of the fp16 inputs."""
+    rng = np.random.default_rng(2)
+    lens = [37, 16]
+    H = 1
+    k, _ = _rand_kv(rng, 2, H, lens)
+    v = []
+    for L in lens:
+        base = rng.standard_normal((L, H, 4)).astype(np.float16)
+        v.append(np.repeat(base, 32, axis=2))
+    bt, NP = _tables(rng, lens)
+    c = _build_cache(oracle_mod, k, v, lens, bt, NP, H)
+    q = np.zeros((2, 2, HD), np.float16)
+    out = c.decode_attention(q, np.array(lens, np.int32), bt)
+    for b in range(2):
+        ref = v[b][:, 0].astype(np.float64).mean(0)
+        assert np.allclose(out[b, 0], ref, rtol=0, atol=1e-12)
+
+
+def test_page_permutation_and_shared_prefix_invariance(oracle_mod):
+    rng = np.random.default_rng(4)
+    H, lens = 2, [64, 70]
+    prefix = 32
+    k0, v0 = _rand_kv(rng, 1, H, [70])
+    k1, v1 = _rand_kv(rng, 1, H, [70])
+    k1[0][:prefix], v1[0][:prefix] = k0[0][:prefix], v0[0][:prefix]
+    k, v = [k0[0][:64], k1[0]], [v0[0][:64], v1[0]]
+    q = rng.standard_normal((2, 2 * H, HD)).astype(np.float16)
+    sl = np.array(lens, np.int32)
+    outs = []
+    for seed in (0, 1):
+        bt, NP = _tables(np.random.default_rng(seed), lens)
+        c = _build_cache(oracle_mod, k, v, lens, bt, NP, H)
+        outs.append(c.decode_attention(q, sl, bt))
+    assert np.array_equal(outs[0], outs[1])
+    # shared: sequence 1 points its first two pages at sequence 0's pages
+    bt, NP = _tables(np.random.default_rng(2), lens)
+    c = _build_cache(oracle_mod, k, v, lens, bt, NP, H)
+    bt_shared = bt.copy()
+    bt_shared[1, :2] = bt[0, :2]
+    out_shared = c.decode_attention(q, sl, bt_shared)
+    assert np.array_equal(out_shared, outs[0])
+
+
+def test_gqa_identical_queries_identical_outputs(oracle_mod):
+    rng = np.random.default_rng(6)
+    lens = [45]
+    k, v = _rand_kv(rng, 1, 2, lens)
+    bt, NP = _tables(rng, lens)
+    c = _build_cache(oracle_mod, k, v, lens, bt, NP, 2)
+    q = rng.standard_normal((1, 8, HD)).astype(np.float16)
+    q[0, 4:8] = q[0, 4]
+    out = c.decode_attention(q, np.array(lens, np.int32), bt)
+    for j in range(5, 8):
+        assert np.array_equal(out[0, j], out[0, 4])
+    assert not np.array_equal(out[0, 0], out[0, 4])
+
+
+def test_fp32_oracle_close_to_fp64(oracle_mod):
+    from int4_kivi_quantized_s4kv_b200 import workloads as W
+    spec = W.SPECS["tiny"]
+    lens = W.final_lens(spec)
+    plan = W.page_plan(spec)
+    k = [W.kv_sequence_np(spec, 0, b, int(L))[0] for b, L in enumerate(lens)]
+    v = [W.kv_sequence_np(spec, 0, b, int(L))[1] for b, L in enumerate(lens)]
+    c = _build_cache(oracle_mod, k, v, list(lens), plan.block_tables, plan.num_pages, 1)
+    q = W.queries_np(spec, 0)
+    o64 = c.decode_attention(q, lens, plan.block_tables, use_double=True)
+    o32 = c.decode_attention(q, lens, plan.block_tables, use_double=False)
+    assert np.abs(o64 - o32).max() < 1e-4
+    # quantization error against unquantized fp16 attention: information only
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    ref = oracle_mod.attention_fp16(np.concatenate(k), np.concatenate(v), cu, 1, q)
+    err = np.abs(o64 - ref).max()
+    assert np.isfinite(err) and err < 1.0
