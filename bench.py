@@ -1,0 +1,466 @@
+#!/usr/bin/env python3
+"""Benchmark of the int4 KIVI paged decode step on B200.
+
+One step = for every layer of the workload: s4kv_append of the step's new
+token(s) (quantizing every page it completes) followed by
+s4kv_decode_attention over the whole cache.  Inputs are seeded synthetic
+tensors shaped like the named model layer (see
+int4_kivi_quantized_s4kv_b200/workloads.py), resident in HBM before timing.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+    python bench.py --impl reference ...   # the CPU oracle on a bounded sample
+
+Prints ONE JSON line (rank 0).  `value` is algorithmic bytes per step (pages
+read once per unique physical page and kv head, residual rows, q, plus the
+append's K/V in and residual out) divided by the device time of a step, over
+all ranks.  Multi-GPU runs are independent replicas (weak scaling, no
+collective on the data path); the step time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from int4_kivi_quantized_s4kv_b200 import workloads as W  # noqa: E402
+
+METRIC = "int4 paged decode attn: achieved HBM GB/s (% of B200 peak), tokens/s"
+DEFAULT_WORKLOAD = "llama3.1-8b"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def measured_hbm_peak():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+# ----------------------------------------------------------------- clocks --
+
+class ClockSampler:
+    """Reads SM clocks and throttle reasons through NVML while running (read
+    only; no GPU setting is changed)."""
+
+    REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+               "sw_power_cap": 0x4, "hw_power_brake_slowdown": 0x80}
+
+    def __init__(self, device_index: int, period_s: float = 0.01):
+        self.samples = []
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._t = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self._nv = None
+        self.period = period_s
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                clk = nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM)
+                rs = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self._h)
+                util = nv.nvmlDeviceGetUtilizationRates(self._h).gpu
+                self.samples.append((clk, rs, util))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self._nv is not None:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+
+    def stop(self):
+        if self._t is not None:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        loaded = [s for s in self.samples if s[2] > 0] or self.samples
+        reasons = set()
+        for _, rs, _ in loaded:
+            for name, bit in self.REASONS.items():
+                if rs & bit:
+                    reasons.add(name)
+        return {"sm_mhz": float(statistics.median(s[0] for s in loaded)), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(reasons), "samples": len(loaded)}
+
+
+# -------------------------------------------------------------- workload --
+
+def step_bytes(spec, plan, lens):
+    d = W.decode_bytes(spec, lens, plan)
+    new = W.step_new_tokens(spec)
+    kv_new = int(new.sum()) * spec.num_kv_heads * 128 * 2 * 2   # k and v read
+    append = 2 * kv_new                                         # residual write (upper bound)
+    return d, append
+
+
+class DeviceWorkload:
+    """All layers' caches of one workload on one GPU, filled through the C
+    ABI, plus the step's inputs."""
+
+    def __init__(self, spec: W.Spec, device, seed_offset: int = 0, prefill_tokens_per_call=1 << 18):
+        import torch
+        import int4_kivi_quantized_s4kv_b200 as S
+        self.S, self.torch = S, torch
+        if seed_offset:
+            import dataclasses
+            spec = dataclasses.replace(spec, seed=spec.seed + 1000 * seed_offset)
+        self.spec, self.device = spec, device
+        self.ctx = W.context_lens(spec)
+        self.lens = W.final_lens(spec)
+        self.new = W.step_new_tokens(spec)
+        self.plan = W.page_plan(spec)
+        B, H = spec.batch, spec.num_kv_heads
+        dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(device)  # noqa: E731
+        self.bt = dev(self.plan.block_tables)
+        self.seq_lens = dev(self.lens)
+        pos = [np.arange(self.ctx[b], self.lens[b]) for b in range(B)]
+        self.step_slots = dev(W.slot_mapping(self.plan.block_tables, pos))
+        self.step_cu = dev(np.concatenate([[0], np.cumsum(self.new)]).astype(np.int32))
+        self.max_new = int(self.new.max())
+        self.caches, self.q, self.k_new, self.v_new = [], [], [], []
+        for layer in range(spec.layers):
+            cache = S.S4KVCache(self.plan.num_pages, H, B, device=device)
+            ks = torch.from_numpy(W.key_channel_scale(spec, layer)).to(device)
+            kn, vn = [], []
+            b = 0
+            while b < B:
+                # a batch of sequences per prefill call, bounded in tokens
+                b1, tok = b, 0
+                while b1 < B and (tok == 0 or tok + int(self.ctx[b1]) <= prefill_tokens_per_call):
+                    tok += int(self.ctx[b1])
+                    b1 += 1
+                kk, vv, slots, counts = [], [], [], []
+                for bb in range(b, b1):
+                    k_seq, v_seq = W.kv_sequence_torch(spec, layer, bb, int(self.lens[bb]), device, ks)
+                    c = int(self.ctx[bb])
+                    kk.append(k_seq[:c])
+                    vv.append(v_seq[:c])
+                    kn.append(k_seq[c:])
+                    vn.append(v_seq[c:])
+                    slots.append(W.slot_mapping(self.plan.block_tables[bb:bb + 1], [np.arange(c)]))
+                    counts.append(c)
+                cnt = np.zeros(B, np.int64)
+                cnt[b:b1] = counts
+                if cnt.sum() > 0:
+                    # sequences outside [b, b1) append nothing: their lengths are not read
+                    S.s4kv_append(cache, torch.cat(kk).contiguous(), torch.cat(vv).contiguous(),
+                                  dev(np.concatenate(slots)), dev(np.concatenate([[0], np.cumsum(cnt)]).astype(np.int32)),
+                                  dev(self.ctx), self.bt, int(max(counts)))
+                b = b1
+            torch.cuda.synchronize(device)
+            self.caches.append(cache)
+            self.k_new.append(torch.cat(kn).contiguous())
+            self.v_new.append(torch.cat(vn).contiguous())
+            self.q.append(W.queries_torch(spec, layer, device))
+        self.out = [torch.empty_like(q) for q in self.q]
+        self.ws = S.decode_workspace(B, H, device)
+        for c in self.caches:
+            flags = S.s4kv_get_error(c)
+            if flags:
+                raise RuntimeError(f"device flags {flags} after prefill")
+
+    def step(self, dec_events=None):
+        S = self.S
+        for layer in range(self.spec.layers):
+            S.s4kv_append(self.caches[layer], self.k_new[layer], self.v_new[layer], self.step_slots,
+                          self.step_cu, self.seq_lens, self.bt, self.max_new)
+            if dec_events is not None:
+                dec_events[0].append(self.torch.cuda.Event(enable_timing=True))
+                dec_events[1].append(self.torch.cuda.Event(enable_timing=True))
+                dec_events[0][-1].record()
+            S.s4kv_decode_attention(self.caches[layer], self.q[layer], self.seq_lens, self.bt,
+                                    self.out[layer], self.ws)
+            if dec_events is not None:
+                dec_events[1][-1].record()
+
+    def launches_per_step(self):
+        return 2 * self.spec.layers
+
+
+# ------------------------------------------------------------ CPU oracle --
+
+class OracleSample:
+    """The oracle on a bounded sample of the workload: `n_units` (sequence, kv
+    head) pairs of layer 0, prefilled untimed; one call of `run()` is the
+    step (append of the new token(s) + decode) for the sampled sequences."""
+
+    def __init__(self, spec: W.Spec, n_seqs: int):
+        import oracle
+        oracle.build()
+        n_seqs = max(1, min(n_seqs, spec.batch))
+        self.spec = spec
+        ctx, lens = W.context_lens(spec), W.final_lens(spec)
+        plan = W.page_plan(spec)
+        self.seqs = list(range(n_seqs))
+        # compact page tables for the sample (shared pages become private)
+        need = [(int(lens[b]) + 15) // 16 for b in self.seqs]
+        bt = np.full((n_seqs, max(need)), -1, np.int32)
+        c = 0
+        for j, n in enumerate(need):
+            bt[j, :n] = np.arange(c, c + n)
+            c += n
+        self.bt = bt
+        self.cache = oracle.OracleCache(c + 1, spec.num_kv_heads, n_seqs)
+        self.ctx = ctx[self.seqs]
+        self.lens = lens[self.seqs]
+        k, v = zip(*[W.kv_sequence_np(spec, 0, b, int(lens[b])) for b in self.seqs])
+        cu = np.concatenate([[0], np.cumsum(self.ctx)]).astype(np.int32)
+        sm = W.slot_mapping(bt, [np.arange(int(x)) for x in self.ctx])
+        rc = self.cache.append(np.concatenate([k[j][:self.ctx[j]] for j in range(n_seqs)]),
+                               np.concatenate([v[j][:self.ctx[j]] for j in range(n_seqs)]),
+                               sm, cu, self.ctx, bt)
+        assert rc == 0
+        self.k_new = np.concatenate([k[j][self.ctx[j]:] for j in range(n_seqs)])
+        self.v_new = np.concatenate([v[j][self.ctx[j]:] for j in range(n_seqs)])
+        self.sm_new = W.slot_mapping(bt, [np.arange(self.ctx[j], self.lens[j]) for j in range(n_seqs)])
+        self.cu_new = np.concatenate([[0], np.cumsum(self.lens - self.ctx)]).astype(np.int32)
+        self.q = W.queries_np(spec, 0)[self.seqs]
+        sub = W.Spec(**{**spec.__dict__, "batch": n_seqs, "shared_prefix_tokens": 0,
+                        "ctx_kind": "fixed", "ctx_fixed": tuple(int(x) for x in self.ctx)})
+        self.bytes = W.decode_bytes(sub, self.lens, W.PagePlan(bt, c + 1, 0, c))["algorithmic"]
+        self.tokens = n_seqs
+
+    def run(self):
+        rc = self.cache.append(self.k_new, self.v_new, self.sm_new, self.cu_new, self.lens, self.bt)
+        assert rc == 0
+        return self.cache.decode_attention(self.q, self.lens, self.bt)
+
+
+def cpu_baseline(spec, budget_s=12.0):
+    probe = OracleSample(spec, 1)
+    t0 = time.perf_counter()
+    probe.run()
+    t1 = time.perf_counter() - t0
+    n = int(max(1, min(spec.batch, budget_s / max(t1, 1e-3))))
+    samp = OracleSample(spec, n) if n > 1 else probe
+    t0 = time.perf_counter()
+    samp.run()
+    dt = time.perf_counter() - t0
+    return {"value": samp.bytes / dt / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"{n} of {spec.batch} sequences of layer 0 (all kv heads), one step "
+                      f"(append + decode), {dt:.1f} s single-threaded",
+            "tokens_per_s": samp.tokens / dt, "seconds": dt}
+
+
+# ------------------------------------------------------------------ main --
+
+def _dist():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def config_dict(spec, extra=None):
+    d = {"workload": spec.name, "model_shape": spec.description, "layers": spec.layers,
+         "batch": spec.batch, "num_q_heads": spec.num_q_heads, "num_kv_heads": spec.num_kv_heads,
+         "head_dim": 128, "page_tokens": 16}
+    if extra:
+        d.update(extra)
+    return d
+
+
+def run_reference(args, spec):
+    world, rank, _ = _dist()
+    if rank != 0:
+        return 0
+    total = args.steps + args.warmup
+    probe = OracleSample(spec, 1)
+    t0 = time.perf_counter()
+    probe.run()
+    t1 = time.perf_counter() - t0
+    per_step_budget = max(0.05, 150.0 / max(total, 1))
+    n = int(max(1, min(spec.batch, per_step_budget / max(t1, 1e-3))))
+    samp = OracleSample(spec, n) if n > 1 else probe
+    for _ in range(args.warmup):
+        samp.run()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        samp.run()
+    dt = (time.perf_counter() - t0) / max(args.steps, 1)
+    val = samp.bytes / dt / 1e9
+    sample = f"{n} of {spec.batch} sequences of layer 0 per step (append + decode), single-threaded"
+    line = {"impl": "reference", "metric": METRIC, "value": val, "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": config_dict(spec, {"sample": sample}),
+            "cpu_baseline": {"value": val, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
+            "e2e": {"value": val, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+            "tokens_per_s": samp.tokens / dt}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="s4kv", choices=["s4kv", "reference"])
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=W.CONFIG_ORDER)
+    ap.add_argument("--batch", type=int, default=None,
+                    help="override the workload's batch (smaller profiling cases)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    spec = W.SPECS[args.workload]
+    if args.batch is not None:
+        import dataclasses
+        spec = dataclasses.replace(spec, batch=args.batch, name=f"{spec.name}-b{args.batch}")
+    if args.impl == "reference":
+        return run_reference(args, spec)
+    if args.warmup < 3:
+        args.warmup = 3
+
+    import torch
+    world, rank, local = _dist()
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    from int4_kivi_quantized_s4kv_b200 import build
+    if rank == 0:
+        build.build()
+    if world > 1:
+        torch.distributed.barrier()
+
+    wl = DeviceWorkload(spec, device, seed_offset=rank)
+    dbytes, abytes = step_bytes(wl.spec, wl.plan, wl.lens)
+    bytes_per_step = (dbytes["algorithmic"] + abytes) * spec.layers
+    decode_bytes_per_launch = dbytes["algorithmic"]
+
+    for _ in range(args.warmup):
+        wl.step()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    clocks = ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ
+                          else int(os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local]))
+    clocks.start()
+    ev = ([], [])
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    t_start.record()
+    for _ in range(args.steps):
+        wl.step(ev)
+    t_end.record()
+    torch.cuda.synchronize()
+    clocks.stop()
+    step_ms = t_start.elapsed_time(t_end) / args.steps
+    dec_ms = [a.elapsed_time(b) for a, b in zip(*ev)]
+    dec_avg_ms = sum(dec_ms) / len(dec_ms)
+    if world > 1:
+        t = torch.tensor([step_ms], device=device)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        step_ms = float(t.item())
+
+    # end to end through the public API: pinned host inputs in, output out
+    h_q = [q.cpu().pin_memory() for q in wl.q]
+    h_k = [k.cpu().pin_memory() for k in wl.k_new]
+    h_v = [v.cpu().pin_memory() for v in wl.v_new]
+    h_out = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in wl.out]
+    h2d = sum(t.numel() * t.element_size() for t in h_q + h_k + h_v)
+    d2h = sum(t.numel() * t.element_size() for t in h_out)
+
+    def e2e_step():
+        for layer in range(spec.layers):
+            wl.q[layer].copy_(h_q[layer], non_blocking=True)
+            wl.k_new[layer].copy_(h_k[layer], non_blocking=True)
+            wl.v_new[layer].copy_(h_v[layer], non_blocking=True)
+        wl.step()
+        for layer in range(spec.layers):
+            h_out[layer].copy_(wl.out[layer], non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    e_start = torch.cuda.Event(enable_timing=True)
+    e_end = torch.cuda.Event(enable_timing=True)
+    e_steps = max(3, min(args.steps, 50))
+    e_start.record()
+    for _ in range(e_steps):
+        e2e_step()
+    e_end.record()
+    torch.cuda.synchronize()
+    e2e_ms = e_start.elapsed_time(e_end) / e_steps
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=device)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+
+    flags = [wl.S.s4kv_get_error(c) for c in wl.caches]
+    if any(flags):
+        raise RuntimeError(f"device error flags {flags}")
+
+    peak, peak_kind = measured_hbm_peak()
+    value = world * bytes_per_step / (step_ms * 1e-3) / 1e9
+    achieved = decode_bytes_per_launch / (dec_avg_ms * 1e-3) / 1e9
+    tokens = int(wl.new.sum())
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(spec)
+    if world > 1:
+        torch.distributed.barrier()
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "int4 codes, f16 MMA operands, f32 accumulate",
+            "data": "synthetic (seeded Gaussian K/V/q with outlier key channels; no dataset)",
+            "config": config_dict(spec, {
+                "parallelism": f"replicas x{world}" if world > 1 else "1 GPU",
+                "context": {"min": int(wl.ctx.min()), "max": int(wl.ctx.max()), "mean": float(wl.ctx.mean())},
+                "new_tokens_per_seq": int(wl.new.max()),
+                "shared_prefix_tokens": spec.shared_prefix_tokens,
+                "decode_bytes_per_layer": dbytes, "append_bytes_per_layer": abytes,
+                "l2": f"inputs larger than L2: {bytes_per_step / 1e9:.2f} GB read per step vs 126 MB L2"
+                      if bytes_per_step > 2e8 else "inputs smaller than L2",
+            }),
+            "pct_of_peak": {"measured_hbm": value / world / peak, "spec_8tbs": value / world / 8000.0},
+            "tokens_per_s": world * tokens / (step_ms * 1e-3),
+            "sequences_per_s": world * spec.batch / (step_ms * 1e-3),
+            "kv_tokens_per_s": world * spec.layers * int(wl.lens.sum()) / (step_ms * 1e-3),
+            "roofline": {"bound": "hbm", "kernel": "decode_kernel", "achieved": achieved, "peak": peak,
+                         "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak, "traffic": None,
+                         "bytes_per_launch": decode_bytes_per_launch, "avg_launch_ms": dec_avg_ms},
+            "e2e": {"value": world * bytes_per_step / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+                    "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": args.steps * wl.launches_per_step(),
+            "clocks": clocks.summary(),
+        }
+        if cpu is not None:
+            line["cpu_baseline"] = cpu
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -71,6 +71,12 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#if defined(__GNUC__)
+#define S4KV_API __attribute__((visibility("default")))
+#else
+#define S4KV_API
+#endif
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -111,16 +117,16 @@ typedef struct s4kv_cache {
 } s4kv_cache_t;
 
 /* Library version (S4KV_VERSION). */
-int s4kv_version(void);
+S4KV_API int s4kv_version(void);
 
 /* Human-readable text of a status code (static storage). */
-const char *s4kv_status_string(int status);
+S4KV_API const char *s4kv_status_string(int status);
 
 /* Fail-fast model check ("S4 KV", "Lieferumfang": unsupported models are
  * refused at start-up): OK for head_dim 128, 16-token pages and
  * num_q_heads = G * num_kv_heads with 1 <= G <= 8; S4KV_ERR_UNSUPPORTED
  * otherwise; S4KV_ERR_INVALID_ARG for non-positive sizes. Host only. */
-int s4kv_check_model(int head_dim, int page_tokens, int num_q_heads,
+S4KV_API int s4kv_check_model(int head_dim, int page_tokens, int num_q_heads,
                      int num_kv_heads);
 
 /* Bytes the caller must allocate for a cache of num_pages physical pages
@@ -128,7 +134,7 @@ int s4kv_check_model(int head_dim, int page_tokens, int num_q_heads,
  * laufenden Zustand und reservierten Speicher trennen": the payload
  * formula 2 x kv_heads x head_dim x tokens x bytes, here with int4 codes
  * plus scale/zero metadata).  Host only; either output may be NULL. */
-int s4kv_cache_layout(int num_pages, int num_kv_heads, int max_seqs,
+S4KV_API int s4kv_cache_layout(int num_pages, int num_kv_heads, int max_seqs,
                       size_t *pool_bytes, size_t *residual_bytes);
 
 /* Append new tokens' K/V and quantize every page they complete.
@@ -148,7 +154,7 @@ int s4kv_cache_layout(int num_pages, int num_kv_heads, int max_seqs,
  * are written once; pages not completed by this call are not touched (a
  * shared-prefix page is never rewritten).  Re-running an identical call is
  * idempotent. */
-int s4kv_append(const s4kv_cache_t *cache, const void *k, const void *v,
+S4KV_API int s4kv_append(const s4kv_cache_t *cache, const void *k, const void *v,
                 int n_tokens, const int64_t *slot_mapping,
                 const int32_t *cu_new, const int32_t *seq_lens,
                 const int32_t *block_tables, int batch,
@@ -158,7 +164,7 @@ int s4kv_append(const s4kv_cache_t *cache, const void *k, const void *v,
  * device for this batch and kv head count.  The workspace must be
  * zero-filled once after allocation; every completed decode call leaves
  * its counters at zero again.  Needs a CUDA device (S4KV_ERR_CUDA if none). */
-int s4kv_decode_workspace_size(int batch, int num_kv_heads, size_t *bytes);
+S4KV_API int s4kv_decode_workspace_size(int batch, int num_kv_heads, size_t *bytes);
 
 /* GQA paged decode attention over the quantized pages plus the residual.
  *  q       device fp16 [batch][num_q_heads][128], 16-B aligned; query head
@@ -174,7 +180,7 @@ int s4kv_decode_workspace_size(int batch, int num_kv_heads, size_t *bytes);
  * Work is split along the KV sequence over all SMs; the last split of a
  * (sequence, kv head) to finish merges the partial results (log-sum-exp).
  * Calls sharing one workspace must not overlap on the device. */
-int s4kv_decode_attention(const s4kv_cache_t *cache, const void *q,
+S4KV_API int s4kv_decode_attention(const s4kv_cache_t *cache, const void *q,
                           int num_q_heads, const int32_t *seq_lens,
                           const int32_t *block_tables, int batch,
                           int max_pages_per_seq, float sm_scale, void *out,
@@ -185,12 +191,12 @@ int s4kv_decode_attention(const s4kv_cache_t *cache, const void *q,
  * out_k, out_v device [num_kv_heads][16][128], fp32 if out_fp32 != 0
  * (x = code*scale + zero, exact product, one rounding) else fp16 (the fp32
  * value rounded to nearest even).  16-B aligned. */
-int s4kv_dequant_page(const s4kv_cache_t *cache, int physical_page,
+S4KV_API int s4kv_dequant_page(const s4kv_cache_t *cache, int physical_page,
                       void *out_k, void *out_v, int out_fp32, void *stream);
 
 /* Synchronize `stream`, read the cache's err_flag into *flags and clear it
  * when `clear` != 0.  Returns S4KV_ERR_DEVICE_CHECK when bits were set. */
-int s4kv_get_error(const s4kv_cache_t *cache, uint32_t *flags, int clear,
+S4KV_API int s4kv_get_error(const s4kv_cache_t *cache, uint32_t *flags, int clear,
                    void *stream);
 
 #ifdef __cplusplus

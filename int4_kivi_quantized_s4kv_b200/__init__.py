@@ -1,0 +1,197 @@
+"""Python binding of the s4kv C ABI (``include/s4kv.h``).
+
+Argument marshalling only: every step of the path runs in the CUDA kernels
+of ``libs4kv.so``.  PyTorch provides device memory and streams.  There is no
+CPU fallback: the first call raises if the library is missing.
+
+    cache = S4KVCache(num_pages, num_kv_heads, max_seqs, device="cuda")
+    s4kv_append(cache, k, v, slot_mapping, cu_new, seq_lens, block_tables, max_new)
+    ws = decode_workspace(batch, num_kv_heads, device)
+    s4kv_decode_attention(cache, q, seq_lens, block_tables, out, ws)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+HEAD_DIM = 128
+PAGE_TOKENS = 16
+VALUE_GROUP = 32
+BLOCK_BYTES = 2816
+MAX_GQA_GROUP = 8
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_DEVICE_CHECK, ERR_WORKSPACE = range(6)
+EFLAG_PAGE_RANGE, EFLAG_SLOT, EFLAG_SEQ_LEN, EFLAG_TIMEOUT = 1, 2, 4, 8
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libs4kv.so")
+
+class s4kv_cache_t(ctypes.Structure):
+    _fields_ = [("pool", ctypes.c_void_p), ("res_k", ctypes.c_void_p), ("res_v", ctypes.c_void_p),
+                ("err_flag", ctypes.c_void_p), ("num_pages", ctypes.c_int32),
+                ("num_kv_heads", ctypes.c_int32), ("max_seqs", ctypes.c_int32),
+                ("head_dim", ctypes.c_int32), ("page_tokens", ctypes.c_int32)]
+
+
+_P, _I, _SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+_CP = ctypes.POINTER(s4kv_cache_t)
+_SIGS = {
+    "s4kv_version": ([], _I),
+    "s4kv_status_string": ([_I], ctypes.c_char_p),
+    "s4kv_check_model": ([_I, _I, _I, _I], _I),
+    "s4kv_cache_layout": ([_I, _I, _I, ctypes.POINTER(_SZ), ctypes.POINTER(_SZ)], _I),
+    "s4kv_append": ([_CP, _P, _P, _I, _P, _P, _P, _P, _I, _I, _I, _P], _I),
+    "s4kv_decode_workspace_size": ([_I, _I, ctypes.POINTER(_SZ)], _I),
+    "s4kv_decode_attention": ([_CP, _P, _I, _P, _P, _I, _I, ctypes.c_float, _P, _P, _SZ, _P], _I),
+    "s4kv_dequant_page": ([_CP, _I, _P, _P, _I, _P], _I),
+    "s4kv_get_error": ([_CP, ctypes.POINTER(ctypes.c_uint32), _I, _P], _I),
+}
+EXPORTED = tuple(_SIGS)
+_lib = None
+
+
+def lib():
+    """The loaded libs4kv.so; raises if it was not built (no CPU fallback)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(
+                f"{LIB_PATH} is missing: build it with `python -m int4_kivi_quantized_s4kv_b200.build` "
+                "(there is no CPU fallback)")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (args, res) in _SIGS.items():
+            f = getattr(L, name)
+            f.argtypes = args
+            f.restype = res
+        _lib = L
+    return _lib
+
+
+class S4KVError(RuntimeError):
+    def __init__(self, status: int, what: str = ""):
+        self.status = status
+        super().__init__(f"{what}: {s4kv_status_string(status)} (status {status})")
+
+
+def _check(status: int, what: str):
+    if status != OK:
+        raise S4KVError(status, what)
+
+
+def _stream(stream):
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _ptr(t, dtype=None, name="tensor"):
+    if t is None:
+        return None
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+# ------------------------------------------------------------ host calls --
+
+def s4kv_version() -> int:
+    return lib().s4kv_version()
+
+
+def s4kv_status_string(status: int) -> str:
+    return lib().s4kv_status_string(status).decode()
+
+
+def s4kv_check_model(head_dim: int, page_tokens: int, num_q_heads: int, num_kv_heads: int) -> int:
+    return lib().s4kv_check_model(head_dim, page_tokens, num_q_heads, num_kv_heads)
+
+
+def s4kv_cache_layout(num_pages: int, num_kv_heads: int, max_seqs: int) -> tuple[int, int]:
+    pb, rb = _SZ(0), _SZ(0)
+    _check(lib().s4kv_cache_layout(num_pages, num_kv_heads, max_seqs, ctypes.byref(pb), ctypes.byref(rb)),
+           "s4kv_cache_layout")
+    return pb.value, rb.value
+
+
+def s4kv_decode_workspace_size(batch: int, num_kv_heads: int) -> int:
+    n = _SZ(0)
+    _check(lib().s4kv_decode_workspace_size(batch, num_kv_heads, ctypes.byref(n)), "s4kv_decode_workspace_size")
+    return n.value
+
+
+# ----------------------------------------------------------------- cache --
+
+class S4KVCache:
+    """Caller-owned device memory of one layer's cache (torch tensors) and the
+    plain C descriptor the library reads."""
+
+    def __init__(self, num_pages: int, num_kv_heads: int, max_seqs: int, device="cuda"):
+        import torch
+        pool_bytes, res_bytes = s4kv_cache_layout(num_pages, num_kv_heads, max_seqs)
+        self.num_pages, self.num_kv_heads, self.max_seqs = num_pages, num_kv_heads, max_seqs
+        self.pool = torch.zeros((num_pages, num_kv_heads, BLOCK_BYTES), dtype=torch.uint8, device=device)
+        self.res_k = torch.zeros((max_seqs, num_kv_heads, PAGE_TOKENS, HEAD_DIM), dtype=torch.float16, device=device)
+        self.res_v = torch.zeros_like(self.res_k)
+        self.err_flag = torch.zeros(1, dtype=torch.int32, device=device)
+        assert self.pool.numel() == pool_bytes and self.res_k.numel() * 2 == res_bytes
+        self.c = s4kv_cache_t(self.pool.data_ptr(), self.res_k.data_ptr(), self.res_v.data_ptr(),
+                              self.err_flag.data_ptr(), num_pages, num_kv_heads, max_seqs,
+                              HEAD_DIM, PAGE_TOKENS)
+
+    @property
+    def ref(self):
+        return ctypes.byref(self.c)
+
+
+def decode_workspace(batch: int, num_kv_heads: int, device="cuda"):
+    """Zero-filled workspace of the size s4kv_decode_attention needs."""
+    import torch
+    n = s4kv_decode_workspace_size(batch, num_kv_heads)
+    return torch.zeros(max(n, 16), dtype=torch.uint8, device=device)
+
+
+# ----------------------------------------------------------- device calls --
+
+def s4kv_append(cache: S4KVCache, k, v, slot_mapping, cu_new, seq_lens, block_tables,
+                max_new_per_seq: int, stream=None):
+    import torch
+    batch, max_pages = block_tables.shape
+    n_tokens = k.shape[0]
+    st = lib().s4kv_append(cache.ref, _ptr(k, torch.float16, "k"), _ptr(v, torch.float16, "v"), n_tokens,
+                          _ptr(slot_mapping, torch.int64, "slot_mapping"), _ptr(cu_new, torch.int32, "cu_new"),
+                          _ptr(seq_lens, torch.int32, "seq_lens"), _ptr(block_tables, torch.int32, "block_tables"),
+                          batch, max_pages, int(max_new_per_seq), _stream(stream))
+    _check(st, "s4kv_append")
+
+
+def s4kv_decode_attention(cache: S4KVCache, q, seq_lens, block_tables, out, workspace,
+                          sm_scale: float | None = None, stream=None):
+    import torch
+    batch, num_q_heads, _ = q.shape
+    if sm_scale is None:
+        sm_scale = HEAD_DIM ** -0.5
+    st = lib().s4kv_decode_attention(cache.ref, _ptr(q, torch.float16, "q"), num_q_heads,
+                                    _ptr(seq_lens, torch.int32, "seq_lens"),
+                                    _ptr(block_tables, torch.int32, "block_tables"), batch,
+                                    block_tables.shape[1], float(sm_scale), _ptr(out, torch.float16, "out"),
+                                    _ptr(workspace, torch.uint8, "workspace"), workspace.numel(),
+                                    _stream(stream))
+    _check(st, "s4kv_decode_attention")
+
+
+def s4kv_dequant_page(cache: S4KVCache, physical_page: int, out_k, out_v, out_fp32: bool = True,
+                      stream=None):
+    st = lib().s4kv_dequant_page(cache.ref, int(physical_page), _ptr(out_k), _ptr(out_v),
+                                1 if out_fp32 else 0, _stream(stream))
+    _check(st, "s4kv_dequant_page")
+
+
+def s4kv_get_error(cache: S4KVCache, clear: bool = True, stream=None) -> int:
+    flags = ctypes.c_uint32(0)
+    st = lib().s4kv_get_error(cache.ref, ctypes.byref(flags), 1 if clear else 0, _stream(stream))
+    if st not in (OK, ERR_DEVICE_CHECK):
+        raise S4KVError(st, "s4kv_get_error")
+    return flags.value

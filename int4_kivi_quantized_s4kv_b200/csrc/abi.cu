@@ -1,0 +1,258 @@
+// Host side of the s4kv C ABI: argument validation, workspace sizing and
+// kernel launches.  Every host-visible argument is checked before anything
+// is launched; the library allocates no memory and keeps no per-cache state
+// (only a per-device record of the decode kernel's launch shape).
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "kernels.cuh"
+
+
+
+using namespace s4kv;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceShape {
+  bool ready = false;
+  int num_sms = 0;
+  int ctas_per_sm = 0;
+  int num_ctas = 0;
+  int num_workers = 0;
+};
+
+std::mutex g_mu;
+DeviceShape g_shape[kMaxDevices];
+
+// Decode launch shape of the current device: one persistent CTA per
+// resident slot on every SM.
+int device_shape(DeviceShape *out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return S4KV_ERR_CUDA;
+  }
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceShape &d = g_shape[dev];
+  if (!d.ready) {
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+      cudaGetLastError();
+      return S4KV_ERR_CUDA;
+    }
+    if (prepare_decode_kernel() != cudaSuccess) {
+      cudaGetLastError();
+      return S4KV_ERR_CUDA;
+    }
+    const int per = decode_ctas_per_sm();
+    if (per <= 0 || sms <= 0) return S4KV_ERR_CUDA;
+    d.num_sms = sms;
+    d.ctas_per_sm = per;
+    d.num_ctas = sms * per;
+    d.num_workers = d.num_ctas * decode_warps_per_cta();
+    d.ready = true;
+  }
+  *out = d;
+  return S4KV_OK;
+}
+
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int check_cache(const s4kv_cache_t *c) {
+  if (c == nullptr) return S4KV_ERR_INVALID_ARG;
+  if (c->head_dim != S4KV_HEAD_DIM || c->page_tokens != S4KV_PAGE_TOKENS) return S4KV_ERR_UNSUPPORTED;
+  if (c->pool == nullptr || c->res_k == nullptr || c->res_v == nullptr) return S4KV_ERR_INVALID_ARG;
+  if (c->num_pages <= 0 || c->num_kv_heads <= 0 || c->max_seqs <= 0) return S4KV_ERR_INVALID_ARG;
+  if (!aligned(c->pool, 128) || !aligned(c->res_k, 16) || !aligned(c->res_v, 16)) return S4KV_ERR_INVALID_ARG;
+  if (c->err_flag != nullptr && !aligned(c->err_flag, 4)) return S4KV_ERR_INVALID_ARG;
+  return S4KV_OK;
+}
+
+// Workspace carve-up: [tickets: batch*kv_heads u32, padded to 256 B]
+// [m,l: 2*workers*8 float2] [partial O: 2*workers*8*128 float].
+struct WsLayout {
+  size_t tickets, ml, part, total;
+};
+
+WsLayout ws_layout(int batch, int num_kv_heads, int num_workers) {
+  auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
+  WsLayout w;
+  w.tickets = 0;
+  w.ml = up(static_cast<size_t>(batch) * num_kv_heads * sizeof(uint32_t));
+  w.part = w.ml + up(static_cast<size_t>(2) * num_workers * 8 * 2 * sizeof(float));
+  w.total = w.part + static_cast<size_t>(2) * num_workers * 8 * S4KV_HEAD_DIM * sizeof(float);
+  return w;
+}
+
+}  // namespace
+
+extern "C" {
+
+int s4kv_version(void) { return S4KV_VERSION; }
+
+const char *s4kv_status_string(int status) {
+  switch (status) {
+    case S4KV_OK: return "ok";
+    case S4KV_ERR_INVALID_ARG: return "invalid argument";
+    case S4KV_ERR_UNSUPPORTED: return "unsupported model shape (head_dim 128, 16-token pages, GQA group <= 8 only)";
+    case S4KV_ERR_CUDA: return "CUDA runtime error";
+    case S4KV_ERR_DEVICE_CHECK: return "device-side check failed (err_flag set)";
+    case S4KV_ERR_WORKSPACE: return "workspace missing or too small";
+    default: return "unknown status";
+  }
+}
+
+int s4kv_check_model(int head_dim, int page_tokens, int num_q_heads, int num_kv_heads) {
+  if (head_dim <= 0 || page_tokens <= 0 || num_q_heads <= 0 || num_kv_heads <= 0) return S4KV_ERR_INVALID_ARG;
+  if (head_dim != S4KV_HEAD_DIM || page_tokens != S4KV_PAGE_TOKENS) return S4KV_ERR_UNSUPPORTED;
+  if (num_q_heads % num_kv_heads != 0) return S4KV_ERR_UNSUPPORTED;
+  const int g = num_q_heads / num_kv_heads;
+  if (g < 1 || g > S4KV_MAX_GQA_GROUP) return S4KV_ERR_UNSUPPORTED;
+  return S4KV_OK;
+}
+
+int s4kv_cache_layout(int num_pages, int num_kv_heads, int max_seqs, size_t *pool_bytes,
+                      size_t *residual_bytes) {
+  if (num_pages <= 0 || num_kv_heads <= 0 || max_seqs <= 0) return S4KV_ERR_INVALID_ARG;
+  if (pool_bytes) *pool_bytes = static_cast<size_t>(num_pages) * num_kv_heads * S4KV_BLOCK_BYTES;
+  if (residual_bytes)
+    *residual_bytes = static_cast<size_t>(max_seqs) * num_kv_heads * S4KV_PAGE_TOKENS * S4KV_HEAD_DIM * 2;
+  return S4KV_OK;
+}
+
+int s4kv_append(const s4kv_cache_t *cache, const void *k, const void *v, int n_tokens,
+                const int64_t *slot_mapping, const int32_t *cu_new, const int32_t *seq_lens,
+                const int32_t *block_tables, int batch, int max_pages_per_seq, int max_new_per_seq,
+                void *stream) {
+  int rc = check_cache(cache);
+  if (rc != S4KV_OK) return rc;
+  if (n_tokens < 0 || batch < 0 || batch > cache->max_seqs || max_pages_per_seq <= 0) return S4KV_ERR_INVALID_ARG;
+  if (n_tokens == 0 || batch == 0) return S4KV_OK;
+  if (max_new_per_seq <= 0 || max_new_per_seq > n_tokens) return S4KV_ERR_INVALID_ARG;
+  if (!k || !v || !slot_mapping || !cu_new || !seq_lens || !block_tables) return S4KV_ERR_INVALID_ARG;
+  if (!aligned(k, 16) || !aligned(v, 16) || !aligned(slot_mapping, 8) || !aligned(cu_new, 4) ||
+      !aligned(seq_lens, 4) || !aligned(block_tables, 4))
+    return S4KV_ERR_INVALID_ARG;
+  const long long slots = (S4KV_PAGE_TOKENS - 1 + static_cast<long long>(max_new_per_seq) + S4KV_PAGE_TOKENS - 1) / S4KV_PAGE_TOKENS;
+  if (slots > 0x7FFFFFFF || batch > 65535 || cache->num_kv_heads > 65535) return S4KV_ERR_INVALID_ARG;
+  AppendParams p;
+  p.pool = static_cast<uint8_t *>(cache->pool);
+  p.res_k = static_cast<__half *>(cache->res_k);
+  p.res_v = static_cast<__half *>(cache->res_v);
+  p.err = cache->err_flag;
+  p.k = static_cast<const __half *>(k);
+  p.v = static_cast<const __half *>(v);
+  p.slot_mapping = slot_mapping;
+  p.cu_new = cu_new;
+  p.seq_lens = seq_lens;
+  p.block_tables = block_tables;
+  p.num_pages = cache->num_pages;
+  p.num_kv_heads = cache->num_kv_heads;
+  p.max_pages = max_pages_per_seq;
+  p.max_new = max_new_per_seq;
+  p.n_tokens = n_tokens;
+  launch_append(p, batch, max_new_per_seq, static_cast<cudaStream_t>(stream));
+  if (cudaGetLastError() != cudaSuccess) return S4KV_ERR_CUDA;
+  return S4KV_OK;
+}
+
+int s4kv_decode_workspace_size(int batch, int num_kv_heads, size_t *bytes) {
+  if (batch < 0 || num_kv_heads <= 0 || bytes == nullptr) return S4KV_ERR_INVALID_ARG;
+  DeviceShape d;
+  const int rc = device_shape(&d);
+  if (rc != S4KV_OK) return rc;
+  *bytes = ws_layout(batch, num_kv_heads, d.num_workers).total;
+  return S4KV_OK;
+}
+
+int s4kv_decode_attention(const s4kv_cache_t *cache, const void *q, int num_q_heads,
+                          const int32_t *seq_lens, const int32_t *block_tables, int batch,
+                          int max_pages_per_seq, float sm_scale, void *out, void *workspace,
+                          size_t workspace_bytes, void *stream) {
+  int rc = check_cache(cache);
+  if (rc != S4KV_OK) return rc;
+  rc = s4kv_check_model(cache->head_dim, cache->page_tokens, num_q_heads, cache->num_kv_heads);
+  if (rc != S4KV_OK) return rc;
+  if (batch < 0 || batch > cache->max_seqs || max_pages_per_seq <= 0) return S4KV_ERR_INVALID_ARG;
+  if (!(std::isfinite(sm_scale)) || sm_scale <= 0.0f) return S4KV_ERR_INVALID_ARG;
+  if (batch == 0) return S4KV_OK;
+  if (!q || !seq_lens || !block_tables || !out) return S4KV_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(out, 8) || !aligned(seq_lens, 4) || !aligned(block_tables, 4))
+    return S4KV_ERR_INVALID_ARG;
+  DeviceShape d;
+  rc = device_shape(&d);
+  if (rc != S4KV_OK) return rc;
+  const WsLayout w = ws_layout(batch, cache->num_kv_heads, d.num_workers);
+  if (workspace == nullptr || workspace_bytes < w.total || !aligned(workspace, 16)) return S4KV_ERR_WORKSPACE;
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  DecodeParams p;
+  p.pool = static_cast<const uint8_t *>(cache->pool);
+  p.res_k = static_cast<const __half *>(cache->res_k);
+  p.res_v = static_cast<const __half *>(cache->res_v);
+  p.q = static_cast<const __half *>(q);
+  p.out = static_cast<__half *>(out);
+  p.seq_lens = seq_lens;
+  p.block_tables = block_tables;
+  p.tickets = reinterpret_cast<uint32_t *>(ws + w.tickets);
+  p.part_ml = reinterpret_cast<float2 *>(ws + w.ml);
+  p.part = reinterpret_cast<float *>(ws + w.part);
+  p.err = cache->err_flag;
+  p.batch = batch;
+  p.num_q_heads = num_q_heads;
+  p.num_kv_heads = cache->num_kv_heads;
+  p.group = num_q_heads / cache->num_kv_heads;
+  p.max_pages = max_pages_per_seq;
+  p.num_pages = cache->num_pages;
+  p.scale_log2 = static_cast<float>(static_cast<double>(sm_scale) * 1.4426950408889634);
+  p.num_workers = d.num_workers;
+  launch_decode(p, d.num_ctas, static_cast<cudaStream_t>(stream));
+  if (cudaGetLastError() != cudaSuccess) return S4KV_ERR_CUDA;
+  return S4KV_OK;
+}
+
+int s4kv_dequant_page(const s4kv_cache_t *cache, int physical_page, void *out_k, void *out_v,
+                      int out_fp32, void *stream) {
+  int rc = check_cache(cache);
+  if (rc != S4KV_OK) return rc;
+  if (physical_page < 0 || physical_page >= cache->num_pages) return S4KV_ERR_INVALID_ARG;
+  if (!out_k || !out_v || !aligned(out_k, 16) || !aligned(out_v, 16)) return S4KV_ERR_INVALID_ARG;
+  DequantParams p;
+  p.pool = static_cast<const uint8_t *>(cache->pool);
+  p.out_k = out_k;
+  p.out_v = out_v;
+  p.physical_page = physical_page;
+  p.num_kv_heads = cache->num_kv_heads;
+  p.out_fp32 = out_fp32 ? 1 : 0;
+  launch_dequant(p, static_cast<cudaStream_t>(stream));
+  if (cudaGetLastError() != cudaSuccess) return S4KV_ERR_CUDA;
+  return S4KV_OK;
+}
+
+int s4kv_get_error(const s4kv_cache_t *cache, uint32_t *flags, int clear, void *stream) {
+  if (cache == nullptr || flags == nullptr) return S4KV_ERR_INVALID_ARG;
+  *flags = 0;
+  if (cache->err_flag == nullptr) return S4KV_OK;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint32_t host = 0;
+  if (cudaMemcpyAsync(&host, cache->err_flag, sizeof(uint32_t), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess) {
+    cudaGetLastError();
+    return S4KV_ERR_CUDA;
+  }
+  if (clear && host != 0) {
+    if (cudaMemsetAsync(cache->err_flag, 0, sizeof(uint32_t), s) != cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess) {
+      cudaGetLastError();
+      return S4KV_ERR_CUDA;
+    }
+  }
+  *flags = host;
+  return host ? S4KV_ERR_DEVICE_CHECK : S4KV_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,162 @@
+// Internal device helpers of the s4kv CUDA library (sm_100a only).
+#pragma once
+
+#include <cuda_fp16.h>
+#include <cstdint>
+
+#include "s4kv.h"
+
+namespace s4kv {
+
+constexpr int kHeadDim = S4KV_HEAD_DIM;
+constexpr int kPage = S4KV_PAGE_TOKENS;
+constexpr int kVGroup = S4KV_VALUE_GROUP;
+constexpr int kBlockBytes = S4KV_BLOCK_BYTES;
+constexpr int kKCodeOff = 0;
+constexpr int kVCodeOff = 1024;
+constexpr int kKScaleOff = 2048;
+constexpr int kKZeroOff = 2304;
+constexpr int kVScaleOff = 2560;
+constexpr int kVZeroOff = 2688;
+
+__device__ __forceinline__ void flag_error(uint32_t *err, uint32_t bits) {
+  if (err != nullptr) atomicOr(err, bits);
+}
+
+// ---------------------------------------------------------------- bit ops --
+
+// (a & b) | c in one LOP3.
+__device__ __forceinline__ uint32_t and_or(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+
+__device__ __forceinline__ uint32_t h2_as_u32(__half2 h) {
+  return *reinterpret_cast<uint32_t *>(&h);
+}
+__device__ __forceinline__ __half2 u32_as_h2(uint32_t u) {
+  return *reinterpret_cast<__half2 *>(&u);
+}
+
+// Four 4-bit codes of a packed word -> the four f16x2 registers of one lane's
+// m16n8k16 operand fragment.  Nibble j goes to register j & 3, half j >> 2.
+// A nibble at bits 0-3 of a half becomes fp16 1024 + c (exponent fixed by the
+// 0x6400 pattern); at bits 4-7 it becomes 1024 + 16c.  The offset and the
+// factor 16 are removed exactly in fp16.
+__device__ __forceinline__ void unpack_codes(uint32_t w, uint32_t &a0, uint32_t &a1,
+                                             uint32_t &a2, uint32_t &a3) {
+  const uint32_t w8 = w >> 8;
+  const __half2 k1024 = u32_as_h2(0x64006400u);   // 1024
+  const __half2 k16th = u32_as_h2(0x2C002C00u);   // 1/16
+  const __half2 kneg64 = u32_as_h2(0xD400D400u);  // -64
+  a0 = h2_as_u32(__hsub2(u32_as_h2(and_or(w, 0x000F000Fu, 0x64006400u)), k1024));
+  a1 = h2_as_u32(__hfma2(u32_as_h2(and_or(w, 0x00F000F0u, 0x64006400u)), k16th, kneg64));
+  a2 = h2_as_u32(__hsub2(u32_as_h2(and_or(w8, 0x000F000Fu, 0x64006400u)), k1024));
+  a3 = h2_as_u32(__hfma2(u32_as_h2(and_or(w8, 0x00F000F0u, 0x64006400u)), k16th, kneg64));
+}
+
+// ------------------------------------------------------------- warp MMA --
+
+// D += A * B, m16n8k16, A row-major f16, B col-major f16, fp32 accumulate.
+__device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1,
+                                         uint32_t a2, uint32_t a3, uint32_t b0,
+                                         uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+      "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Transpose of an 8x8 b16 matrix held as one b16x2 register per lane.
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
+  uint32_t y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
+}
+
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// --------------------------------------------------------- shared memory --
+
+__device__ __forceinline__ uint32_t smem_addr(const void *p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr));
+  return v;
+}
+
+__device__ __forceinline__ uint32_t lds32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
+}
+
+// ------------------------------------------------ mbarrier + bulk copies --
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+// Make barrier initialisation visible to the async (bulk-copy) proxy.
+__device__ __forceinline__ void fence_barrier_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Order this thread's earlier generic-proxy shared-memory accesses before
+// later async-proxy accesses (a bulk copy reusing a stage).
+__device__ __forceinline__ void fence_proxy_async() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+
+// One 1-D bulk copy global -> this CTA's shared memory, completing on `bar`.
+// No multicast.  dst, src 16-byte aligned; bytes a multiple of 16.
+__device__ __forceinline__ void bulk_copy_g2s(uint32_t dst, const void *src, uint32_t bytes,
+                                              uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+      "l"(src), "r"(bytes), "r"(bar)
+      : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(done)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return done != 0;
+}
+
+// Bounded wait for the phase with the given parity: gives up after roughly
+// `limit_cycles` SM clock cycles and returns false.
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
+                                                  long long limit_cycles) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (clock64() - t0 > limit_cycles) return false;
+  }
+}
+
+}  // namespace s4kv

@@ -1,0 +1,52 @@
+// s4kv_dequant_page device side: one physical page, all kv heads, back to
+// natural [token][channel] order.  x = code * scale + zero in fp32 (the
+// product of a 4-bit code and an fp16 scale is exact, so this is a single
+// rounding); the fp16 output is that fp32 value rounded to nearest even.
+#include "kernels.cuh"
+
+namespace s4kv {
+
+__device__ __forceinline__ uint32_t code_at(const uint8_t *region, int word, int nibble) {
+  const uint32_t w = reinterpret_cast<const uint32_t *>(region)[word];
+  return (w >> (4 * nibble)) & 0xFu;
+}
+
+__global__ void __launch_bounds__(128) dequant_kernel(const DequantParams p) {
+  const int h = blockIdx.x;
+  const int c = threadIdx.x;  // channel
+  const uint8_t *blk = p.pool + (static_cast<long>(p.physical_page) * p.num_kv_heads + h) * kBlockBytes;
+  const float ks = __half2float(reinterpret_cast<const __half *>(blk + kKScaleOff)[c]);
+  const float kz = __half2float(reinterpret_cast<const __half *>(blk + kKZeroOff)[c]);
+  const int g = c / kVGroup;
+  // key fragment coordinates of channel c: lane quarter i, tile kt, pair e
+  const int ki = c >> 5, kt = (c & 31) >> 2, ke = c & 3;
+  // value fragment coordinates of channel c: M-tile m, row group n
+  const int vn = (c & 31) >> 2, ve = c & 3, vm = 2 * g + (ve >> 1);
+  for (int t = 0; t < kPage; ++t) {
+    const int kword = 128 * (kt >> 2) + 4 * (4 * (t & 7) + ki) + (kt & 3);
+    const int knib = (t >> 3) + 2 * (ke >> 1) + 4 * (ke & 1);
+    const int vi = (t & 7) >> 1;
+    const int vword = 128 * (vm >> 2) + 4 * (4 * vn + vi) + (vm & 3);
+    const int vnib = (ve & 1) + 2 * (t >> 3) + 4 * (t & 1);
+    const float kcode = static_cast<float>(code_at(blk + kKCodeOff, kword, knib));
+    const float vcode = static_cast<float>(code_at(blk + kVCodeOff, vword, vnib));
+    const float vs = __half2float(reinterpret_cast<const __half *>(blk + kVScaleOff)[g * kPage + t]);
+    const float vz = __half2float(reinterpret_cast<const __half *>(blk + kVZeroOff)[g * kPage + t]);
+    const float kx = __fadd_rn(__fmul_rn(kcode, ks), kz);
+    const float vx = __fadd_rn(__fmul_rn(vcode, vs), vz);
+    const long o = (static_cast<long>(h) * kPage + t) * kHeadDim + c;
+    if (p.out_fp32) {
+      static_cast<float *>(p.out_k)[o] = kx;
+      static_cast<float *>(p.out_v)[o] = vx;
+    } else {
+      static_cast<__half *>(p.out_k)[o] = __float2half_rn(kx);
+      static_cast<__half *>(p.out_v)[o] = __float2half_rn(vx);
+    }
+  }
+}
+
+void launch_dequant(const DequantParams &p, cudaStream_t stream) {
+  dequant_kernel<<<p.num_kv_heads, 128, 0, stream>>>(p);
+}
+
+}  // namespace s4kv

@@ -1,0 +1,67 @@
+// Launch parameters and launchers of the s4kv kernels (internal).
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+
+namespace s4kv {
+
+struct AppendParams {
+  uint8_t *pool;
+  __half *res_k;
+  __half *res_v;
+  uint32_t *err;
+  const __half *k;
+  const __half *v;
+  const int64_t *slot_mapping;
+  const int32_t *cu_new;
+  const int32_t *seq_lens;
+  const int32_t *block_tables;
+  int num_pages;
+  int num_kv_heads;
+  int max_pages;
+  int max_new;
+  int n_tokens;
+};
+
+struct DequantParams {
+  const uint8_t *pool;
+  void *out_k;
+  void *out_v;
+  int physical_page;
+  int num_kv_heads;
+  int out_fp32;
+};
+
+struct DecodeParams {
+  const uint8_t *pool;
+  const __half *res_k;
+  const __half *res_v;
+  const __half *q;
+  __half *out;
+  const int32_t *seq_lens;
+  const int32_t *block_tables;
+  float *part;        // [2 * num_workers][8][128] partial O (unnormalised)
+  float2 *part_ml;    // [2 * num_workers][8] (running max m, sum l)
+  uint32_t *tickets;  // [batch * num_kv_heads], zero between calls
+  uint32_t *err;
+  int batch;
+  int num_q_heads;
+  int num_kv_heads;
+  int group;
+  int max_pages;
+  int num_pages;
+  float scale_log2;   // sm_scale * log2(e)
+  int num_workers;
+};
+
+void launch_append(const AppendParams &p, int batch, int max_new, cudaStream_t stream);
+void launch_dequant(const DequantParams &p, cudaStream_t stream);
+void launch_decode(const DecodeParams &p, int num_ctas, cudaStream_t stream);
+int decode_ctas_per_sm();
+int decode_warps_per_cta();
+cudaError_t prepare_decode_kernel();
+size_t decode_smem_bytes();
+
+}  // namespace s4kv
