@@ -119,13 +119,10 @@ class DeviceWorkload:
     """All layers' caches of one workload on one GPU, filled through the C
     ABI, plus the step's inputs."""
 
-    def __init__(self, spec: W.Spec, device, seed_offset: int = 0, prefill_tokens_per_call=1 << 18):
+    def __init__(self, spec: W.Spec, device, prefill_tokens_per_call=1 << 18):
         import torch
         import int4_kivi_quantized_s4kv_b200 as S
         self.S, self.torch = S, torch
-        if seed_offset:
-            import dataclasses
-            spec = dataclasses.replace(spec, seed=spec.seed + 1000 * seed_offset)
         self.spec, self.device = spec, device
         self.ctx = W.context_lens(spec)
         self.lens = W.final_lens(spec)
@@ -145,22 +142,25 @@ class DeviceWorkload:
             ks = torch.from_numpy(W.key_channel_scale(spec, layer)).to(device)
             kn, vn = [], []
             b = 0
+            # the shared prefix's pages are written once, by sequence 0; the
+            # other sequences append from the prefix boundary (a page boundary)
+            start = [0] + [spec.shared_prefix_tokens] * (B - 1)
             while b < B:
                 # a batch of sequences per prefill call, bounded in tokens
                 b1, tok = b, 0
-                while b1 < B and (tok == 0 or tok + int(self.ctx[b1]) <= prefill_tokens_per_call):
-                    tok += int(self.ctx[b1])
+                while b1 < B and (tok == 0 or tok + int(self.ctx[b1]) - start[b1] <= prefill_tokens_per_call):
+                    tok += int(self.ctx[b1]) - start[b1]
                     b1 += 1
                 kk, vv, slots, counts = [], [], [], []
                 for bb in range(b, b1):
                     k_seq, v_seq = W.kv_sequence_torch(spec, layer, bb, int(self.lens[bb]), device, ks)
-                    c = int(self.ctx[bb])
-                    kk.append(k_seq[:c])
-                    vv.append(v_seq[:c])
+                    c, c0 = int(self.ctx[bb]), start[bb]
+                    kk.append(k_seq[c0:c])
+                    vv.append(v_seq[c0:c])
                     kn.append(k_seq[c:])
                     vn.append(v_seq[c:])
-                    slots.append(W.slot_mapping(self.plan.block_tables[bb:bb + 1], [np.arange(c)]))
-                    counts.append(c)
+                    slots.append(W.slot_mapping(self.plan.block_tables[bb:bb + 1], [np.arange(c0, c)]))
+                    counts.append(c - c0)
                 cnt = np.zeros(B, np.int64)
                 cnt[b:b1] = counts
                 if cnt.sum() > 0:
@@ -273,6 +273,31 @@ def _dist():
     return world, rank, local
 
 
+def replica_spec(spec, rank: int):
+    """Rank r's replica of the workload: same shapes, its own seeds (each
+    rank decodes its own batch; no data crosses GPUs)."""
+    if rank == 0:
+        return spec
+    import dataclasses
+    return dataclasses.replace(spec, seed=spec.seed + 1000 * rank)
+
+
+def reduce_max(x: float, world: int, device) -> float:
+    """Max over ranks of a per-rank time (the only collective in the bench)."""
+    if world <= 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_gbs(world: int, bytes_per_step_per_rank: float, step_ms: float) -> float:
+    """Whole-job throughput: bytes all ranks processed per step / slowest step."""
+    return world * bytes_per_step_per_rank / (step_ms * 1e-3) / 1e9
+
+
 def config_dict(spec, extra=None):
     d = {"workload": spec.name, "model_shape": spec.description, "layers": spec.layers,
          "batch": spec.batch, "num_q_heads": spec.num_q_heads, "num_kv_heads": spec.num_kv_heads,
@@ -349,7 +374,7 @@ def main(argv=None):
     if world > 1:
         torch.distributed.barrier()
 
-    wl = DeviceWorkload(spec, device, seed_offset=rank)
+    wl = DeviceWorkload(replica_spec(spec, rank), device)
     dbytes, abytes = step_bytes(wl.spec, wl.plan, wl.lens)
     bytes_per_step = (dbytes["algorithmic"] + abytes) * spec.layers
     decode_bytes_per_launch = dbytes["algorithmic"]
@@ -375,10 +400,7 @@ def main(argv=None):
     step_ms = t_start.elapsed_time(t_end) / args.steps
     dec_ms = [a.elapsed_time(b) for a, b in zip(*ev)]
     dec_avg_ms = sum(dec_ms) / len(dec_ms)
-    if world > 1:
-        t = torch.tensor([step_ms], device=device)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        step_ms = float(t.item())
+    step_ms = reduce_max(step_ms, world, device)
 
     # end to end through the public API: pinned host inputs in, output out
     h_q = [q.cpu().pin_memory() for q in wl.q]
@@ -409,17 +431,14 @@ def main(argv=None):
     e_end.record()
     torch.cuda.synchronize()
     e2e_ms = e_start.elapsed_time(e_end) / e_steps
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=device)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = reduce_max(e2e_ms, world, device)
 
     flags = [wl.S.s4kv_get_error(c) for c in wl.caches]
     if any(flags):
         raise RuntimeError(f"device error flags {flags}")
 
     peak, peak_kind = measured_hbm_peak()
-    value = world * bytes_per_step / (step_ms * 1e-3) / 1e9
+    value = aggregate_gbs(world, bytes_per_step, step_ms)
     achieved = decode_bytes_per_launch / (dec_avg_ms * 1e-3) / 1e9
     tokens = int(wl.new.sum())
     cpu = None
@@ -449,7 +468,7 @@ def main(argv=None):
             "roofline": {"bound": "hbm", "kernel": "decode_kernel", "achieved": achieved, "peak": peak,
                          "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak, "traffic": None,
                          "bytes_per_launch": decode_bytes_per_launch, "avg_launch_ms": dec_avg_ms},
-            "e2e": {"value": world * bytes_per_step / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+            "e2e": {"value": aggregate_gbs(world, bytes_per_step, e2e_ms), "unit": "GB/s",
                     "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": args.steps * wl.launches_per_step(),
             "clocks": clocks.summary(),

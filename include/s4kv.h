@@ -39,7 +39,9 @@
  *             [   0,1024) key codes   : 256 little-endian 32-bit words
  *             [1024,2048) value codes : 256 little-endian 32-bit words
  *             [2048,2304) key scale   : fp16 [128 channels]
- *             [2304,2560) key zero    : fp16 [128 channels]
+ *             [2304,2560) key zero    : fp16 [8 k-tiles][16 k-slots]:
+ *                                       channel c at k-tile (c%32)/4, slot
+ *                                       2*(c/32) + (c%2) + 8*((c%4)/2)
  *             [2560,2688) value scale : fp16 [4 groups][16 tokens]
  *             [2688,2816) value zero  : fp16 [4 groups][16 tokens]
  *           Code word w = 128*h + 4*lane + q, lane = 4*n + i (n < 8,
@@ -48,8 +50,10 @@
  *                     channel 32*i + 4*(4*h+q) + 2*((j>>1)&1) + (j>>2)
  *             values: token 2*i + (j>>2) + 8*((j>>1)&1),
  *                     channel 32*((4*h+q)>>1) + 4*n + 2*((4*h+q)&1) + (j&1)
- *           (each 32-bit word is one lane's tensor-core operand fragment;
- *           s4kv_dequant_page returns the natural [token][channel] order).
+ *           (each 32-bit word is one lane's tensor-core operand fragment,
+ *           and the key zero points follow the same k order, so one
+ *           ldmatrix row is a lane quad's k columns; s4kv_dequant_page
+ *           returns the natural [token][channel] order).
  *  res_k,   fp16 [max_seqs][num_kv_heads][16][128] each.  Row r of batch
  *  res_v    row b holds token 16*floor(L/16) + r of that sequence for
  *           r < L mod 16 (L = its current length); other rows are

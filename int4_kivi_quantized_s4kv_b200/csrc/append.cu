@@ -115,7 +115,9 @@ __global__ void __launch_bounds__(128) append_kernel(const AppendParams p) {
 #pragma unroll
         for (int t = 0; t < kPage; ++t) kc[t][c] = static_cast<uint8_t>(group_code(__half2float(ks[t][c]), mn, s));
         reinterpret_cast<__half *>(blk + kKScaleOff)[c] = __float2half_rn(s);
-        reinterpret_cast<__half *>(blk + kKZeroOff)[c] = __float2half_rn(mn);
+        // zero points in the MMA k order: tile (c%32)/4, slot 2(c/32) + (c%2) + 8((c%4)/2)
+        const int zslot = 16 * ((c & 31) >> 2) + 2 * (c >> 5) + (c & 1) + 8 * ((c & 3) >> 1);
+        reinterpret_cast<__half *>(blk + kKZeroOff)[zslot] = __float2half_rn(mn);
       }
       // values: threads 0..63 each quantize one (token, 32-channel group)
       if (tid < kPage * (kHeadDim / kVGroup)) {

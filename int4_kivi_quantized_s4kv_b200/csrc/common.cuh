@@ -58,11 +58,23 @@ __device__ __forceinline__ void unpack_codes(uint32_t w, uint32_t &a0, uint32_t 
 
 // ------------------------------------------------------------- warp MMA --
 
+// Register-only instructions are emitted as plain (non-volatile) asm so the
+// compiler may schedule them freely around each other; S4KV_ASM_VOLATILE=1
+// pins them in program order instead.
+#ifndef S4KV_ASM_VOLATILE
+#define S4KV_ASM_VOLATILE 0
+#endif
+#if S4KV_ASM_VOLATILE
+#define S4KV_ASM asm volatile
+#else
+#define S4KV_ASM asm
+#endif
+
 // D += A * B, m16n8k16, A row-major f16, B col-major f16, fp32 accumulate.
 __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1,
                                          uint32_t a2, uint32_t a3, uint32_t b0,
                                          uint32_t b1) {
-  asm volatile(
+  S4KV_ASM(
       "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
       "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
@@ -72,13 +84,13 @@ __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1
 // Transpose of an 8x8 b16 matrix held as one b16x2 register per lane.
 __device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
   uint32_t y;
-  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+  S4KV_ASM("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
   return y;
 }
 
 __device__ __forceinline__ float fast_exp2(float x) {
   float y;
-  asm("ex2.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
 
@@ -88,18 +100,30 @@ __device__ __forceinline__ uint32_t smem_addr(const void *p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
-__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+// Shared loads at [base + OFF] with OFF folded into the instruction.
+template <int OFF>
+__device__ __forceinline__ uint4 lds128(uint32_t base) {
   uint4 v;
-  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4+%5];"
                : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "r"(addr));
+               : "r"(base), "n"(OFF));
   return v;
 }
 
-__device__ __forceinline__ uint32_t lds32(uint32_t addr) {
+template <int OFF>
+__device__ __forceinline__ uint32_t lds32(uint32_t base) {
   uint32_t v;
-  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+  asm volatile("ld.shared.u32 %0, [%1+%2];" : "=r"(v) : "r"(base), "n"(OFF));
   return v;
+}
+
+// Four 8x8 b16 matrices from shared memory, one row address per lane (lanes
+// 8m..8m+7 give matrix m's rows), straight into an MMA operand fragment.
+__device__ __forceinline__ void ldmatrix_x4(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2,
+                                            uint32_t &r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
 }
 
 // ------------------------------------------------ mbarrier + bulk copies --
@@ -135,8 +159,23 @@ __device__ __forceinline__ void bulk_copy_g2s(uint32_t dst, const void *src, uin
       : "memory");
 }
 
+// Test (and, for up to S4KV_WAIT_HINT_NS nanoseconds, wait) for completion
+// of the barrier phase with the given parity.  A suspended warp leaves its
+// issue slots to the other warps instead of spinning.
+#ifndef S4KV_WAIT_HINT_NS
+#define S4KV_WAIT_HINT_NS 0
+#endif
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t done;
+#if S4KV_WAIT_HINT_NS > 0
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(done)
+      : "r"(bar), "r"(parity), "n"(S4KV_WAIT_HINT_NS)
+      : "memory");
+#else
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
@@ -144,6 +183,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
       : "=r"(done)
       : "r"(bar), "r"(parity)
       : "memory");
+#endif
   return done != 0;
 }
 

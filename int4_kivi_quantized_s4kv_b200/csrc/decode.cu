@@ -33,43 +33,64 @@
 //    halves), giving fp32-level accuracy.  The packed page layout makes each
 //    lane's 32-bit code word its own operand fragment (one 16-byte shared
 //    load per 4 tiles, 1 shift + 4 LOP3 + 4 fp16 ops to unpack 8 codes).
-//    The softmax is the usual online update in the exp2 domain; P is moved
+//    The softmax is an online update in the exp2 domain whose reference
+//    only moves when a page's maximum passes it (with a headroom of 4, so
+//    every weight stays <= 1 and no fp16 operand can overflow); P is moved
 //    from the QK accumulator layout to the PV operand layout with movmatrix.
+//  * Pipelining.  Within a warp, the QK MMAs of page j+2, the softmax of page
+//    j+1 and the PV MMAs of page j are issued in one straight-line block, so
+//    the softmax's shuffle/exp latency overlaps tensor-core work.
 #include <cfloat>
 
 #include "kernels.cuh"
 
 namespace s4kv {
 
-constexpr int kStages = 4;
-constexpr int kWarpsPerCta = 4;
+// Build-time tuning constants (stages per warp ring, worker warps per CTA,
+// CTAs per SM the register budget is sized for).
+#ifndef S4KV_DECODE_STAGES
+#define S4KV_DECODE_STAGES 6
+#endif
+#ifndef S4KV_DECODE_WARPS
+#define S4KV_DECODE_WARPS 4
+#endif
+#ifndef S4KV_DECODE_MIN_CTAS
+#define S4KV_DECODE_MIN_CTAS 3
+#endif
+constexpr int kStages = S4KV_DECODE_STAGES;
+constexpr int kWarpsPerCta = S4KV_DECODE_WARPS;
 constexpr int kThreads = 32 * kWarpsPerCta;
 constexpr long long kWaitLimitCycles = 2000000000LL;  // about one second
 constexpr unsigned kFull = 0xFFFFFFFFu;
+constexpr float kHeadroom = 4.0f;  // log2 headroom of the softmax reference
 
 size_t decode_smem_bytes() {
   return static_cast<size_t>(kWarpsPerCta) * kStages * (kBlockBytes + 8);
 }
 
-struct Segment {
-  long long start;  // flattened index of the segment's first page
-  int b, h;
-  int len;          // tokens of sequence b
-  int np;           // pages of b (full pages + a partial residual page)
-  int nfull;        // full (quantized) pages of b
-};
-
 __device__ __forceinline__ int clamp_len(int L, int max_pages) {
   return min(max(L, 0), max_pages * kPage);
 }
 
-__device__ __forceinline__ void set_seq(Segment &c, int len) {
+// Position in the flattened (sequence, kv head, page) order.
+struct Cursor {
+  long long start;    // flattened index of the segment's first page
+  const int32_t *bt;  // block_tables row of sequence b
+  int b, h;
+  int len;            // tokens of sequence b
+  int np;             // pages of b (full pages + a partial residual page)
+  int nfull;          // full (quantized) pages of b
+};
+
+__device__ __forceinline__ void set_seq(Cursor &c, const DecodeParams &p, int b, int len) {
+  c.b = b;
   c.len = len;
   c.np = (len + kPage - 1) / kPage;
   c.nfull = len / kPage;
+  c.bt = p.block_tables + static_cast<long>(b) * p.max_pages;
 }
 
-__device__ __forceinline__ void next_segment(Segment &c, const DecodeParams &p) {
+__device__ __forceinline__ void next_segment(Cursor &c, const DecodeParams &p) {
   c.start += c.np;
   if (++c.h == p.num_kv_heads) {
     c.h = 0;
@@ -79,8 +100,7 @@ __device__ __forceinline__ void next_segment(Segment &c, const DecodeParams &p) 
       if (L > 0) break;
       ++b;
     }
-    c.b = b;
-    set_seq(c, b < p.batch ? L : 0);
+    set_seq(c, p, b, b < p.batch ? L : 0);
   }
 }
 
@@ -89,40 +109,114 @@ __device__ __forceinline__ long long worker_of(long long x, long long T, long lo
   return ((x + 1) * W + T - 1) / T - 1;
 }
 
-// Online-softmax update for one 16-token page.  S: this lane's logits
-// (tokens n, n+8; heads 2i, 2i+1).  Produces P^T fragments (hi, lo) in the
-// PV operand layout: head n, tokens 2i, 2i+1 (t0) and 2i+8, 2i+9 (t1).
-__device__ __forceinline__ void softmax_page(const float (&S)[4], float scale_log2, float &m0,
-                                             float &m1, float &l0, float &l1, float (&O)[8][4],
-                                             float (&Z)[4], uint32_t &t0h, uint32_t &t1h,
-                                             uint32_t &t0l, uint32_t &t1l) {
+// Running softmax state of one lane: heads 2i, 2i+1 of the group.
+struct Online {
+  float ref0, ref1;  // log2-domain reference: weights are exp2(s - ref) <= 1
+  float l0, l1;      // partial sums of weights over this lane's tokens
+  float O[8][4];     // PV accumulators (M-tile, C fragment)
+  float Z[4];        // value zero-point term: sum_t zV[g][t] P[t][h]
+};
+
+// Per-lane shared addresses of one stage: the stage base plus this lane's
+// offset into the code words (16*lane), the key scale/zero rows (64*i), the
+// value scale pairs (4*i) and the value zero rows (32*(n%4) + 4*i).
+// The two zero-point operands are broadcast rows, fetched with ldmatrix:
+// kzero = this lane's row address in the key zero points (lanes 16..31 read
+// k columns 8..15), vzero = this lane's row address in the value zero points
+// (row r of the operand holds group r % 4).
+struct StageAddr {
+  uint32_t code, kmeta, vscale, kzero, vzero;
+};
+
+__device__ __forceinline__ StageAddr stage_addr_of(uint32_t stage_base, int lane) {
+  const int i = lane & 3;
+  const uint32_t half_k = (lane >> 4) ? 16u : 0u;
+  return StageAddr{stage_base + 16u * lane, stage_base + 64u * i, stage_base + 4u * i,
+                   stage_base + kKZeroOff + half_k,
+                   stage_base + kVZeroOff + 32u * ((lane & 7) & 3) + half_k};
+}
+
+// Logits of one quantized page: this lane's S^T[tokens n, n+8][heads 2i,
+// 2i+1] before scaling.
+__device__ __forceinline__ void qk_page(const StageAddr &a, const uint32_t (&qf)[16], float (&S)[4]) {
+  // three independent accumulators (hi part, lo part, zero-point term) keep
+  // the dependent MMA chains 8 deep instead of 24
+  float Sh[4] = {0.f, 0.f, 0.f, 0.f}, Sl[4] = {0.f, 0.f, 0.f, 0.f}, Sz[4] = {0.f, 0.f, 0.f, 0.f};
+  const uint4 kw0 = lds128<kKCodeOff>(a.code);
+  const uint4 kw1 = lds128<kKCodeOff + 512>(a.code);
+  const uint32_t kws[8] = {kw0.x, kw0.y, kw0.z, kw0.w, kw1.x, kw1.y, kw1.z, kw1.w};
+  uint32_t sk[16];
+  {
+    const uint4 s0 = lds128<kKScaleOff>(a.kmeta), s1 = lds128<kKScaleOff + 16>(a.kmeta);
+    const uint4 s2 = lds128<kKScaleOff + 32>(a.kmeta), s3 = lds128<kKScaleOff + 48>(a.kmeta);
+    const uint4 sv[4] = {s0, s1, s2, s3};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      sk[4 * k] = sv[k].x; sk[4 * k + 1] = sv[k].y; sk[4 * k + 2] = sv[k].z; sk[4 * k + 3] = sv[k].w;
+    }
+  }
+#pragma unroll
+  for (int kt = 0; kt < 8; ++kt) {
+    uint32_t a0, a1, a2, a3;
+    unpack_codes(kws[kt], a0, a1, a2, a3);
+    const __half2 qb0 = u32_as_h2(qf[2 * kt]), qb1 = u32_as_h2(qf[2 * kt + 1]);
+    const __half2 s0 = u32_as_h2(sk[2 * kt]), s1 = u32_as_h2(sk[2 * kt + 1]);
+    // q * sK split into fp16 hi + lo; the lo part is the exact remainder
+    const __half2 h0 = __hmul2(qb0, s0), h1 = __hmul2(qb1, s1);
+    const __half2 r0 = __hfma2(qb0, s0, __hneg2(h0));
+    const __half2 r1 = __hfma2(qb1, s1, __hneg2(h1));
+    mma16816(Sh, a0, a1, a2, a3, h2_as_u32(h0), h2_as_u32(h1));
+    mma16816(Sl, a0, a1, a2, a3, h2_as_u32(r0), h2_as_u32(r1));
+    // key zero point: every A row is zK (one ldmatrix), so each row gets sum_c zK q
+    uint32_t z0, z1, z2, z3;
+    ldmatrix_x4(a.kzero + 32 * kt, z0, z1, z2, z3);
+    mma16816(Sz, z0, z1, z2, z3, qf[2 * kt], qf[2 * kt + 1]);
+  }
+#pragma unroll
+  for (int k = 0; k < 4; ++k) S[k] = (Sh[k] + Sl[k]) + Sz[k];
+}
+
+// Online softmax for one 16-token page.  S: this lane's logits (tokens n,
+// n+8; heads 2i, 2i+1).  Writes P^T fragments in the PV operand layout
+// (head n; tokens 2i, 2i+1 and 2i+8, 2i+9) as fp16 hi (P[0], P[1]) and lo
+// (P[2], P[3]) parts.  The reference moves (and the state is rescaled) only
+// when a page maximum passes it, for any lane of the warp.
+__device__ __forceinline__ void softmax_page(const float (&S)[4], float scale_log2, Online &st,
+                                             uint32_t (&P)[4]) {
   const float s0 = S[0] * scale_log2, s1 = S[1] * scale_log2;
   const float s2 = S[2] * scale_log2, s3 = S[3] * scale_log2;
-  float pm0 = fmaxf(s0, s2), pm1 = fmaxf(s1, s3);
+  // common case: no logit passes the reference, one vote and no shuffles
+  if (__any_sync(kFull, fmaxf(s0, s2) > st.ref0 || fmaxf(s1, s3) > st.ref1)) {
+    float pm0 = fmaxf(s0, s2), pm1 = fmaxf(s1, s3);
 #pragma unroll
-  for (int off = 4; off < 32; off <<= 1) {
-    pm0 = fmaxf(pm0, __shfl_xor_sync(kFull, pm0, off));
-    pm1 = fmaxf(pm1, __shfl_xor_sync(kFull, pm1, off));
-  }
-  const float mn0 = fmaxf(m0, pm0), mn1 = fmaxf(m1, pm1);
-  const float a0 = fast_exp2(m0 - mn0), a1 = fast_exp2(m1 - mn1);
-  m0 = mn0;
-  m1 = mn1;
-  const float p0 = fast_exp2(s0 - mn0), p2 = fast_exp2(s2 - mn0);
-  const float p1 = fast_exp2(s1 - mn1), p3 = fast_exp2(s3 - mn1);
-  l0 = l0 * a0 + (p0 + p2);
-  l1 = l1 * a1 + (p1 + p3);
+    for (int off = 4; off < 32; off <<= 1) {
+      pm0 = fmaxf(pm0, __shfl_xor_sync(kFull, pm0, off));
+      pm1 = fmaxf(pm1, __shfl_xor_sync(kFull, pm1, off));
+    }
+    const bool up0 = pm0 > st.ref0, up1 = pm1 > st.ref1;
+    const float n0 = up0 ? pm0 + kHeadroom : st.ref0;
+    const float n1 = up1 ? pm1 + kHeadroom : st.ref1;
+    const float a0 = fast_exp2(st.ref0 - n0), a1 = fast_exp2(st.ref1 - n1);
+    st.ref0 = n0;
+    st.ref1 = n1;
+    st.l0 *= a0;
+    st.l1 *= a1;
 #pragma unroll
-  for (int mt = 0; mt < 8; ++mt) {
-    O[mt][0] *= a0;
-    O[mt][1] *= a1;
-    O[mt][2] *= a0;
-    O[mt][3] *= a1;
+    for (int mt = 0; mt < 8; ++mt) {
+      st.O[mt][0] *= a0;
+      st.O[mt][1] *= a1;
+      st.O[mt][2] *= a0;
+      st.O[mt][3] *= a1;
+    }
+    st.Z[0] *= a0;
+    st.Z[1] *= a1;
+    st.Z[2] *= a0;
+    st.Z[3] *= a1;
   }
-  Z[0] *= a0;
-  Z[1] *= a1;
-  Z[2] *= a0;
-  Z[3] *= a1;
+  const float p0 = fast_exp2(s0 - st.ref0), p2 = fast_exp2(s2 - st.ref0);
+  const float p1 = fast_exp2(s1 - st.ref1), p3 = fast_exp2(s3 - st.ref1);
+  st.l0 += p0 + p2;
+  st.l1 += p1 + p3;
   // P in fp16 hi + lo, rows = tokens, cols = heads; then transpose
   const __half2 h01 = __floats2half2_rn(p0, p1);
   const __half2 h23 = __floats2half2_rn(p2, p3);
@@ -130,80 +224,52 @@ __device__ __forceinline__ void softmax_page(const float (&S)[4], float scale_lo
   const float2 b23 = __half22float2(h23);
   const __half2 l01 = __floats2half2_rn(p0 - b01.x, p1 - b01.y);
   const __half2 l23 = __floats2half2_rn(p2 - b23.x, p3 - b23.y);
-  t0h = movmatrix_trans(h2_as_u32(h01));
-  t1h = movmatrix_trans(h2_as_u32(h23));
-  t0l = movmatrix_trans(h2_as_u32(l01));
-  t1l = movmatrix_trans(h2_as_u32(l23));
+  P[0] = movmatrix_trans(h2_as_u32(h01));
+  P[1] = movmatrix_trans(h2_as_u32(h23));
+  P[2] = movmatrix_trans(h2_as_u32(l01));
+  P[3] = movmatrix_trans(h2_as_u32(l23));
 }
 
-// One quantized page from shared memory (stage at shared address `blk`).
-__device__ __forceinline__ void page_step(uint32_t blk, const uint32_t (&qf)[16], int lane,
-                                          float scale_log2, float &m0, float &m1, float &l0,
-                                          float &l1, float (&O)[8][4], float (&Z)[4]) {
-  const int n = lane >> 2, i = lane & 3;
-  float S[4] = {0.f, 0.f, 0.f, 0.f};
-  const uint4 kw0 = lds128(blk + kKCodeOff + 16 * lane);
-  const uint4 kw1 = lds128(blk + kKCodeOff + 512 + 16 * lane);
-  const uint32_t kws[8] = {kw0.x, kw0.y, kw0.z, kw0.w, kw1.x, kw1.y, kw1.z, kw1.w};
+// O += V^T P for one quantized page.
+template <int G4>
+__device__ __forceinline__ void pv_group(const StageAddr &a, const uint32_t (&P)[4], const uint32_t (&vws)[8],
+                                         Online &st) {
+  const __half2 sv0 = u32_as_h2(lds32<kVScaleOff + 32 * G4>(a.vscale));
+  const __half2 sv1 = u32_as_h2(lds32<kVScaleOff + 32 * G4 + 16>(a.vscale));
+  // (P * sV) in fp16 hi + lo: P-hi * sV exactly as two halves, plus P-lo * sV
+  const __half2 bh0 = __hmul2(u32_as_h2(P[0]), sv0);
+  const __half2 bh1 = __hmul2(u32_as_h2(P[1]), sv1);
+  const __half2 bl0 = __hfma2(u32_as_h2(P[2]), sv0, __hfma2(u32_as_h2(P[0]), sv0, __hneg2(bh0)));
+  const __half2 bl1 = __hfma2(u32_as_h2(P[3]), sv1, __hfma2(u32_as_h2(P[1]), sv1, __hneg2(bh1)));
 #pragma unroll
-  for (int hf = 0; hf < 2; ++hf) {
-    const uint4 sa = lds128(blk + kKScaleOff + 64 * i + 32 * hf);
-    const uint4 sb = lds128(blk + kKScaleOff + 64 * i + 32 * hf + 16);
-    const uint4 za = lds128(blk + kKZeroOff + 64 * i + 32 * hf);
-    const uint4 zb = lds128(blk + kKZeroOff + 64 * i + 32 * hf + 16);
-    const uint32_t sk[8] = {sa.x, sa.y, sa.z, sa.w, sb.x, sb.y, sb.z, sb.w};
-    const uint32_t zk[8] = {za.x, za.y, za.z, za.w, zb.x, zb.y, zb.z, zb.w};
-#pragma unroll
-    for (int q4 = 0; q4 < 4; ++q4) {
-      const int kt = 4 * hf + q4;
-      uint32_t a0, a1, a2, a3;
-      unpack_codes(kws[kt], a0, a1, a2, a3);
-      const __half2 qb0 = u32_as_h2(qf[2 * kt]), qb1 = u32_as_h2(qf[2 * kt + 1]);
-      const __half2 s0 = u32_as_h2(sk[2 * q4]), s1 = u32_as_h2(sk[2 * q4 + 1]);
-      const __half2 h0 = __hmul2(qb0, s0), h1 = __hmul2(qb1, s1);
-      const __half2 r0 = __hfma2(qb0, s0, __hneg2(h0));
-      const __half2 r1 = __hfma2(qb1, s1, __hneg2(h1));
-      mma16816(S, a0, a1, a2, a3, h2_as_u32(h0), h2_as_u32(h1));
-      mma16816(S, a0, a1, a2, a3, h2_as_u32(r0), h2_as_u32(r1));
-      // key zero point: every A row is zK, so each row gets sum_c zK q
-      mma16816(S, zk[2 * q4], zk[2 * q4], zk[2 * q4 + 1], zk[2 * q4 + 1], qf[2 * kt], qf[2 * kt + 1]);
-    }
+  for (int j = 0; j < 2; ++j) {
+    const int mt = 2 * G4 + j;
+    uint32_t a0, a1, a2, a3;
+    unpack_codes(vws[mt], a0, a1, a2, a3);
+    mma16816(st.O[mt], a0, a1, a2, a3, h2_as_u32(bh0), h2_as_u32(bh1));
+    mma16816(st.O[mt], a0, a1, a2, a3, h2_as_u32(bl0), h2_as_u32(bl1));
   }
-  uint32_t t0h, t1h, t0l, t1l;
-  softmax_page(S, scale_log2, m0, m1, l0, l1, O, Z, t0h, t1h, t0l, t1l);
+}
 
-  const uint4 vw0 = lds128(blk + kVCodeOff + 16 * lane);
-  const uint4 vw1 = lds128(blk + kVCodeOff + 512 + 16 * lane);
+__device__ __forceinline__ void pv_page(const StageAddr &a, const uint32_t (&P)[4], Online &st) {
+  const uint4 vw0 = lds128<kVCodeOff>(a.code);
+  const uint4 vw1 = lds128<kVCodeOff + 512>(a.code);
   const uint32_t vws[8] = {vw0.x, vw0.y, vw0.z, vw0.w, vw1.x, vw1.y, vw1.z, vw1.w};
-#pragma unroll
-  for (int g = 0; g < 4; ++g) {
-    const __half2 sv0 = u32_as_h2(lds32(blk + kVScaleOff + 32 * g + 4 * i));
-    const __half2 sv1 = u32_as_h2(lds32(blk + kVScaleOff + 32 * g + 4 * i + 16));
-    const __half2 bh0 = __hmul2(u32_as_h2(t0h), sv0);
-    const __half2 bh1 = __hmul2(u32_as_h2(t1h), sv1);
-    const __half2 bl0 = __hfma2(u32_as_h2(t0l), sv0, __hfma2(u32_as_h2(t0h), sv0, __hneg2(bh0)));
-    const __half2 bl1 = __hfma2(u32_as_h2(t1l), sv1, __hfma2(u32_as_h2(t1h), sv1, __hneg2(bh1)));
-#pragma unroll
-    for (int j = 0; j < 2; ++j) {
-      const int mt = 2 * g + j;
-      uint32_t a0, a1, a2, a3;
-      unpack_codes(vws[mt], a0, a1, a2, a3);
-      mma16816(O[mt], a0, a1, a2, a3, h2_as_u32(bh0), h2_as_u32(bh1));
-      mma16816(O[mt], a0, a1, a2, a3, h2_as_u32(bl0), h2_as_u32(bl1));
-    }
-  }
-  // value zero points: A row r carries group r % 4's zV, B = P
-  const uint32_t zv0 = lds32(blk + kVZeroOff + 32 * (n & 3) + 4 * i);
-  const uint32_t zv1 = lds32(blk + kVZeroOff + 32 * (n & 3) + 4 * i + 16);
-  mma16816(Z, zv0, zv0, zv1, zv1, t0h, t1h);
-  mma16816(Z, zv0, zv0, zv1, zv1, t0l, t1l);
+  pv_group<0>(a, P, vws, st);
+  pv_group<1>(a, P, vws, st);
+  pv_group<2>(a, P, vws, st);
+  pv_group<3>(a, P, vws, st);
+  // value zero points: A row r carries group r % 4's zV (one ldmatrix), B = P
+  uint32_t z0, z1, z2, z3;
+  ldmatrix_x4(a.vzero, z0, z1, z2, z3);
+  mma16816(st.Z, z0, z1, z2, z3, P[0], P[1]);
+  mma16816(st.Z, z0, z1, z2, z3, P[2], P[3]);
 }
 
 // The partial last page, read straight from the fp16 residual (r rows valid).
-__device__ __forceinline__ void residual_step(const __half *rk, const __half *rv, int r,
+__device__ __forceinline__ void residual_page(const __half *rk, const __half *rv, int r,
                                               const uint32_t (&qf)[16], int lane, float scale_log2,
-                                              float &m0, float &m1, float &l0, float &l1,
-                                              float (&O)[8][4], float (&Z)[4]) {
+                                              Online &st) {
   const int n = lane >> 2, i = lane & 3;
   uint32_t kn[16], kn8[16];
 #pragma unroll
@@ -220,8 +286,8 @@ __device__ __forceinline__ void residual_step(const __half *rk, const __half *rv
     mma16816(S, kn[2 * kt], kn8[2 * kt], kn[2 * kt + 1], kn8[2 * kt + 1], qf[2 * kt], qf[2 * kt + 1]);
   if (n >= r) S[0] = S[1] = -INFINITY;
   if (n + 8 >= r) S[2] = S[3] = -INFINITY;
-  uint32_t t0h, t1h, t0l, t1l;
-  softmax_page(S, scale_log2, m0, m1, l0, l1, O, Z, t0h, t1h, t0l, t1l);
+  uint32_t P[4];
+  softmax_page(S, scale_log2, st, P);
   // V^T fragments: rows = channels 32g + 4n + {0..3}, k = tokens
   const int tok[4] = {2 * i, 2 * i + 1, 2 * i + 8, 2 * i + 9};
 #pragma unroll
@@ -238,13 +304,78 @@ __device__ __forceinline__ void residual_step(const __half *rk, const __half *rv
       const uint32_t x2 = j ? vv[2].y : vv[2].x, x3 = j ? vv[3].y : vv[3].x;
       const uint32_t a0 = __byte_perm(x0, x1, 0x5410), a1 = __byte_perm(x0, x1, 0x7632);
       const uint32_t a2 = __byte_perm(x2, x3, 0x5410), a3 = __byte_perm(x2, x3, 0x7632);
-      mma16816(O[2 * g + j], a0, a1, a2, a3, t0h, t1h);
-      mma16816(O[2 * g + j], a0, a1, a2, a3, t0l, t1l);
+      mma16816(st.O[2 * g + j], a0, a1, a2, a3, P[0], P[1]);
+      mma16816(st.O[2 * g + j], a0, a1, a2, a3, P[2], P[3]);
     }
   }
 }
 
-__global__ void __launch_bounds__(kThreads, 4) decode_kernel(const DecodeParams p) {
+// Slot of worker w's partial for the segment starting at flattened page
+// seg_start: a worker whose range starts inside the segment stored it as its
+// first piece (slot 2w), the segment's first worker as its last (2w + 1)
+// unless its range starts exactly at the segment.
+__device__ __forceinline__ long long piece_slot(long long w, long long wf, long long seg_start, long long T,
+                                                long long W) {
+  return 2 * w + ((w == wf && w * T / W < seg_start) ? 1 : 0);
+}
+
+__device__ __forceinline__ void merge_pieces(const DecodeParams &p, long obase, int G, long long wf, long long wl,
+                                          long long seg_start, long long T, long long W, int lane) {
+  const int npieces = static_cast<int>(wl - wf + 1);
+  float acc[8][4];
+  float M[8], Ls[8];
+#pragma unroll
+  for (int h = 0; h < 8; ++h) {
+    M[h] = -INFINITY;
+    Ls[h] = 0.f;
+    acc[h][0] = acc[h][1] = acc[h][2] = acc[h][3] = 0.f;
+  }
+  // pass 1: maxima per head, pieces spread over lanes
+  for (int k0 = 0; k0 < npieces; k0 += 32) {
+    const int k = k0 + lane;
+    if (k < npieces) {
+      const long long sl = piece_slot(wf + k, wf, seg_start, T, W);
+#pragma unroll
+      for (int h = 0; h < 8; ++h)
+        if (h < G) M[h] = fmaxf(M[h], __ldcg(p.part_ml + sl * 8 + h).x);
+    }
+  }
+#pragma unroll
+  for (int h = 0; h < 8; ++h)
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) M[h] = fmaxf(M[h], __shfl_xor_sync(kFull, M[h], off));
+  // pass 2: weighted sums; each lane owns channels 4*lane..4*lane+3
+#pragma unroll 2
+  for (int k = 0; k < npieces; ++k) {
+    const long long sl = piece_slot(wf + k, wf, seg_start, T, W);
+    const float2 *ml = p.part_ml + sl * 8;
+    const float4 *o = reinterpret_cast<const float4 *>(p.part + sl * 8 * kHeadDim) + lane;
+#pragma unroll
+    for (int h = 0; h < 8; ++h) {
+      if (h < G) {
+        const float2 m_l = __ldcg(ml + h);
+        const float4 ov = __ldcg(o + h * (kHeadDim / 4));
+        const float wt = fast_exp2(m_l.x - M[h]);
+        Ls[h] += wt * m_l.y;
+        acc[h][0] += wt * ov.x;
+        acc[h][1] += wt * ov.y;
+        acc[h][2] += wt * ov.z;
+        acc[h][3] += wt * ov.w;
+      }
+    }
+  }
+#pragma unroll
+  for (int h = 0; h < 8; ++h) {
+    if (h < G) {
+      const float inv = 1.0f / Ls[h];
+      const __half2 u = __floats2half2_rn(acc[h][0] * inv, acc[h][1] * inv);
+      const __half2 v = __floats2half2_rn(acc[h][2] * inv, acc[h][3] * inv);
+      *reinterpret_cast<uint2 *>(p.out + obase + h * kHeadDim + 4 * lane) = make_uint2(h2_as_u32(u), h2_as_u32(v));
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, S4KV_DECODE_MIN_CTAS) decode_kernel(const DecodeParams p) {
   extern __shared__ __align__(128) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n = lane >> 2, i = lane & 3;
@@ -318,52 +449,104 @@ __global__ void __launch_bounds__(kThreads, 4) decode_kernel(const DecodeParams 
   }
   bs = __shfl_sync(kFull, bs, src);
   pre = __shfl_sync(kFull, pre, src);
-  Segment cc;
-  cc.b = bs;
-  set_seq(cc, clamp_len(__ldg(p.seq_lens + bs), p.max_pages));
+  Cursor cc;
+  set_seq(cc, p, bs, clamp_len(__ldg(p.seq_lens + bs), p.max_pages));
   cc.h = static_cast<int>((s - H * pre) / cc.np);
   cc.start = H * pre + static_cast<long long>(cc.h) * cc.np;
+  const int range = static_cast<int>(e - s);
+  const int p_first = static_cast<int>(s - cc.start);
 
-  // ---- producer: issue the next quantized page of [s, e) into the ring
-  Segment pc = cc;
-  long long px = s;
+  // ---- producer: issue the next quantized page of [s, e) into the ring.
+  // It walks the same pieces as the consumer: per piece a pointer into the
+  // block table and a count of quantized pages still to issue.
+  const long long page_stride = static_cast<long long>(H) * kBlockBytes;
+  Cursor pc = cc;
+  int p_page = p_first;       // page index of the producer's current piece start
+  int p_left = range;         // pages of [s, e) from the current piece on
+  int p_q = 0;                // quantized pages left in the current piece
+  const int32_t *p_bt = nullptr;
+  const uint8_t *p_head = nullptr;
+  uint32_t p_stage = 0;       // stage index * kBlockBytes
+  uint32_t p_bar = bar0;
   int issued = 0;
-  auto produce = [&]() {
-    while (px < e) {
-      if (px >= pc.start + pc.np) next_segment(pc, p);
-      const int pp = static_cast<int>(px - pc.start);
-      ++px;
-      if (pp < pc.nfull) {
-        int phys = __ldg(p.block_tables + static_cast<long>(pc.b) * p.max_pages + pp);
-        if (phys < 0 || phys >= p.num_pages) {
-          if (lane == 0) flag_error(p.err, S4KV_EFLAG_PAGE_RANGE);
-          phys = 0;
-        }
-        const int st = issued % kStages;
-        if (lane == 0) {
-          mbar_arrive_expect_tx(bar0 + 8 * st, kBlockBytes);
-          bulk_copy_g2s(ring0 + st * kBlockBytes,
-                        p.pool + (static_cast<long>(phys) * H + pc.h) * kBlockBytes, kBlockBytes,
-                        bar0 + 8 * st);
-        }
-        ++issued;
-        return;
-      }
-    }
+  auto p_piece = [&]() {      // set up the piece starting at p_page
+    const int take = min(p_left, pc.np - p_page);
+    p_q = max(0, min(p_page + take, pc.nfull) - p_page);
+    p_bt = pc.bt + p_page;
+    p_head = p.pool + static_cast<long long>(pc.h) * kBlockBytes;
+    p_left -= take;
   };
+  p_piece();
+  auto produce = [&]() {
+    while (p_q == 0) {
+      if (p_left == 0) return;
+      next_segment(pc, p);
+      p_page = 0;
+      p_piece();
+    }
+    int phys = __ldg(p_bt++);
+    --p_q;
+    if (static_cast<unsigned>(phys) >= static_cast<unsigned>(p.num_pages)) {
+      if (lane == 0) flag_error(p.err, S4KV_EFLAG_PAGE_RANGE);
+      phys = 0;
+    }
+    if (lane == 0) {
+      mbar_arrive_expect_tx(p_bar, kBlockBytes);
+      bulk_copy_g2s(ring0 + p_stage, p_head + phys * page_stride, kBlockBytes, p_bar);
+    }
+    p_stage += kBlockBytes;
+    p_bar += 8;
+    if (p_stage == kStages * kBlockBytes) {
+      p_stage = 0;
+      p_bar = bar0;
+    }
+    ++issued;
+  };
+  static_assert(kStages >= 4, "the pipeline holds three stages at once");
 #pragma unroll 1
   for (int k = 0; k < kStages; ++k) produce();
 
-  // ---- consumer
-  long long x = s;
+  // ---- consumer.  A ring position: stage offset, barrier address, parity.
+  struct Pos {
+    uint32_t off, bar, phase;
+  };
+  auto next_pos = [&](Pos q) {
+    q.off += kBlockBytes;
+    q.bar += 8;
+    if (q.off == kStages * kBlockBytes) {
+      q.off = 0;
+      q.bar = bar0;
+      q.phase ^= 1u;
+    }
+    return q;
+  };
   int consumed = 0;
   bool failed = false;
-  while (x < e) {
-    if (x >= cc.start + cc.np) next_segment(cc, p);
-    const long long seg_end = cc.start + cc.np;
-    const long long piece_end = min(e, seg_end);
-    const bool complete = cc.start >= s && seg_end <= e;
-    const bool first_piece = (x == s);
+  Pos c0{0u, bar0, 0u};
+  auto wait_copy = [&](const Pos &q) {
+    const bool ok = mbar_wait_bounded(q.bar, q.phase, kWaitLimitCycles);
+    return !__any_sync(kFull, !ok);
+  };
+  auto addr = [&](const Pos &q) { return stage_addr_of(ring0 + q.off, lane); };
+  auto release = [&]() {      // the page at c0 has been read completely
+    fence_proxy_async();
+    __syncwarp();
+    ++consumed;
+    c0 = next_pos(c0);
+    produce();
+  };
+
+  int page = p_first, rem = range;
+  bool first = true;
+  while (rem > 0 && !failed) {
+    if (page == cc.np) {
+      next_segment(cc, p);
+      page = 0;
+    }
+    const int take = min(rem, cc.np - page);
+    const int p1 = page + take;
+    const bool complete = (page == 0) && (p1 == cc.np);
+    const int nq = max(0, min(p1, cc.nfull) - page);
 
     uint32_t qf[16];
     if (n < G) {
@@ -378,36 +561,90 @@ __global__ void __launch_bounds__(kThreads, 4) decode_kernel(const DecodeParams 
 #pragma unroll
       for (int k = 0; k < 16; ++k) qf[k] = 0u;
     }
-    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
-    float O[8][4], Z[4] = {0.f, 0.f, 0.f, 0.f};
+    Online st;
+    st.ref0 = st.ref1 = -INFINITY;
+    st.l0 = st.l1 = 0.f;
 #pragma unroll
-    for (int mt = 0; mt < 8; ++mt) O[mt][0] = O[mt][1] = O[mt][2] = O[mt][3] = 0.f;
+    for (int mt = 0; mt < 8; ++mt) st.O[mt][0] = st.O[mt][1] = st.O[mt][2] = st.O[mt][3] = 0.f;
+    st.Z[0] = st.Z[1] = st.Z[2] = st.Z[3] = 0.f;
 
+    if (nq > 0) {
+      // software pipeline over the piece's quantized pages: each step issues
+      // QK(j+2), PV(j) and the softmax of page j+1 in one block; two steps
+      // per loop trip swap the roles of the P / S registers
+      uint32_t Pa[4], Pb[4];
+      float Sa[4], Sb[4];
+      Pos c2 = next_pos(next_pos(c0));
+      if (!wait_copy(c0)) {
+        failed = true;
+        break;
+      }
+      {
+        float S0[4];
+        qk_page(addr(c0), qf, S0);
+        if (nq > 1) {
+          const Pos c1 = next_pos(c0);
+          if (!wait_copy(c1)) {
+            failed = true;
+            break;
+          }
+          qk_page(addr(c1), qf, Sa);
+        }
+        softmax_page(S0, p.scale_log2, st, Pa);
+      }
+      // one pipeline step: in (Pcur = P(j), Snext = S(j+1)), out (Pnext, Snext2)
+      auto step = [&](const uint32_t (&Pcur)[4], const float (&Snext)[4], uint32_t (&Pnext)[4],
+                      float (&Snext2)[4]) {
+        qk_page(addr(c2), qf, Snext2);
+        pv_page(addr(c0), Pcur, st);
+        softmax_page(Snext, p.scale_log2, st, Pnext);  // after PV(j): a rescale covers it
+        release();
+        c2 = next_pos(c2);
+      };
+      int j = 0;
+      bool odd = false;     // false: (Pa, Sa) hold (P(j), S(j+1)); true: (Pb, Sb)
 #pragma unroll 1
-    for (; x < piece_end; ++x) {
-      const int pp = static_cast<int>(x - cc.start);
-      if (pp < cc.nfull) {
-        const int st = consumed % kStages;
-        const uint32_t par = (consumed / kStages) & 1;
-        const bool ok = mbar_wait_bounded(bar0 + 8 * st, par, kWaitLimitCycles);
-        if (__any_sync(kFull, !ok)) {
+      while (j + 2 < nq) {
+        if (!wait_copy(c2)) {
           failed = true;
           break;
         }
-        page_step(ring0 + st * kBlockBytes, qf, lane, p.scale_log2, m0, m1, l0, l1, O, Z);
-        fence_proxy_async();
-        __syncwarp();
-        ++consumed;
-        produce();
+        step(Pa, Sa, Pb, Sb);
+        ++j;
+        if (j + 2 >= nq) {
+          odd = true;
+          break;
+        }
+        if (!wait_copy(c2)) {
+          failed = true;
+          break;
+        }
+        step(Pb, Sb, Pa, Sa);
+        ++j;
+      }
+      if (failed) break;
+      // the last one or two pages
+      uint32_t Pt[4];
+      if (odd) {
+        pv_page(addr(c0), Pb, st);
+        if (nq > 1) softmax_page(Sb, p.scale_log2, st, Pt);
       } else {
-        const long rbase = (static_cast<long>(cc.b) * H + cc.h) * kPage * kHeadDim;
-        residual_step(p.res_k + rbase, p.res_v + rbase, cc.len % kPage, qf, lane, p.scale_log2, m0,
-                      m1, l0, l1, O, Z);
+        pv_page(addr(c0), Pa, st);
+        if (nq > 1) softmax_page(Sa, p.scale_log2, st, Pt);
+      }
+      release();
+      if (nq > 1) {
+        pv_page(addr(c0), Pt, st);
+        release();
       }
     }
-    if (failed) break;
+    if (p1 == cc.np && cc.np > cc.nfull) {
+      const long rbase = (static_cast<long>(cc.b) * H + cc.h) * kPage * kHeadDim;
+      residual_page(p.res_k + rbase, p.res_v + rbase, cc.len % kPage, qf, lane, p.scale_log2, st);
+    }
 
     // ---- finish the piece
+    float l0 = st.l0, l1 = st.l1;
 #pragma unroll
     for (int off = 4; off < 32; off <<= 1) {
       l0 += __shfl_xor_sync(kFull, l0, off);
@@ -416,15 +653,15 @@ __global__ void __launch_bounds__(kThreads, 4) decode_kernel(const DecodeParams 
     float za[4], zb[4];
 #pragma unroll
     for (int g = 0; g < 4; ++g) {
-      za[g] = __shfl_sync(kFull, Z[0], 4 * g + i);
-      zb[g] = __shfl_sync(kFull, Z[1], 4 * g + i);
+      za[g] = __shfl_sync(kFull, st.Z[0], 4 * g + i);
+      zb[g] = __shfl_sync(kFull, st.Z[1], 4 * g + i);
     }
 #pragma unroll
     for (int mt = 0; mt < 8; ++mt) {
-      O[mt][0] += za[mt >> 1];
-      O[mt][2] += za[mt >> 1];
-      O[mt][1] += zb[mt >> 1];
-      O[mt][3] += zb[mt >> 1];
+      st.O[mt][0] += za[mt >> 1];
+      st.O[mt][2] += za[mt >> 1];
+      st.O[mt][1] += zb[mt >> 1];
+      st.O[mt][3] += zb[mt >> 1];
     }
     const long obase = (static_cast<long>(cc.b) * p.num_q_heads + cc.h * G) * kHeadDim;
     if (complete) {
@@ -433,33 +670,34 @@ __global__ void __launch_bounds__(kThreads, 4) decode_kernel(const DecodeParams 
       for (int g = 0; g < 4; ++g) {
         const int ch = 32 * g + 4 * n;
         if (2 * i < G) {
-          const __half2 u = __floats2half2_rn(O[2 * g][0] * inv0, O[2 * g][2] * inv0);
-          const __half2 v = __floats2half2_rn(O[2 * g + 1][0] * inv0, O[2 * g + 1][2] * inv0);
+          const __half2 u = __floats2half2_rn(st.O[2 * g][0] * inv0, st.O[2 * g][2] * inv0);
+          const __half2 v = __floats2half2_rn(st.O[2 * g + 1][0] * inv0, st.O[2 * g + 1][2] * inv0);
           *reinterpret_cast<uint2 *>(p.out + obase + (2 * i) * kHeadDim + ch) = make_uint2(h2_as_u32(u), h2_as_u32(v));
         }
         if (2 * i + 1 < G) {
-          const __half2 u = __floats2half2_rn(O[2 * g][1] * inv1, O[2 * g][3] * inv1);
-          const __half2 v = __floats2half2_rn(O[2 * g + 1][1] * inv1, O[2 * g + 1][3] * inv1);
+          const __half2 u = __floats2half2_rn(st.O[2 * g][1] * inv1, st.O[2 * g][3] * inv1);
+          const __half2 v = __floats2half2_rn(st.O[2 * g + 1][1] * inv1, st.O[2 * g + 1][3] * inv1);
           *reinterpret_cast<uint2 *>(p.out + obase + (2 * i + 1) * kHeadDim + ch) = make_uint2(h2_as_u32(u), h2_as_u32(v));
         }
       }
     } else {
-      const long long slot = 2 * worker + (first_piece ? 0 : 1);
+      const long long slot = 2 * worker + (first ? 0 : 1);
       float *dst = p.part + slot * 8 * kHeadDim;
 #pragma unroll
       for (int g = 0; g < 4; ++g) {
         const int ch = 32 * g + 4 * n;
         *reinterpret_cast<float4 *>(dst + (2 * i) * kHeadDim + ch) =
-            make_float4(O[2 * g][0], O[2 * g][2], O[2 * g + 1][0], O[2 * g + 1][2]);
+            make_float4(st.O[2 * g][0], st.O[2 * g][2], st.O[2 * g + 1][0], st.O[2 * g + 1][2]);
         *reinterpret_cast<float4 *>(dst + (2 * i + 1) * kHeadDim + ch) =
-            make_float4(O[2 * g][1], O[2 * g][3], O[2 * g + 1][1], O[2 * g + 1][3]);
+            make_float4(st.O[2 * g][1], st.O[2 * g][3], st.O[2 * g + 1][1], st.O[2 * g + 1][3]);
       }
       if (n == 0) {
-        p.part_ml[slot * 8 + 2 * i] = make_float2(m0, l0);
-        p.part_ml[slot * 8 + 2 * i + 1] = make_float2(m1, l1);
+        p.part_ml[slot * 8 + 2 * i] = make_float2(st.ref0, l0);
+        p.part_ml[slot * 8 + 2 * i + 1] = make_float2(st.ref1, l1);
       }
       __threadfence();
       __syncwarp();
+      const long long seg_end = cc.start + cc.np;
       const long long wf = worker_of(cc.start, T, W), wl = worker_of(seg_end - 1, T, W);
       uint32_t last = 0;
       if (lane == 0) {
@@ -468,41 +706,26 @@ __global__ void __launch_bounds__(kThreads, 4) decode_kernel(const DecodeParams 
       }
       last = __shfl_sync(kFull, last, 0);
       if (last) {
+        // merge every piece of this (sequence, kv head): log-sum-exp.  Lanes
+        // take pieces for (m, l) (warp reductions); for O each lane owns 4
+        // channels of every head and loads the pieces independently.
         __threadfence();
-        for (int hh = 0; hh < G; ++hh) {
-          float M = -INFINITY;
-          for (long long w = wf; w <= wl; ++w) {
-            const long long sl = 2 * w + ((w == wf && w * T / W < cc.start) ? 1 : 0);
-            M = fmaxf(M, __ldcg(p.part_ml + sl * 8 + hh).x);
-          }
-          float Ls = 0.f;
-          float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-          for (long long w = wf; w <= wl; ++w) {
-            const long long sl = 2 * w + ((w == wf && w * T / W < cc.start) ? 1 : 0);
-            const float2 ml = __ldcg(p.part_ml + sl * 8 + hh);
-            const float wt = fast_exp2(ml.x - M);
-            Ls += wt * ml.y;
-            const float4 o = __ldcg(reinterpret_cast<const float4 *>(p.part + sl * 8 * kHeadDim + hh * kHeadDim) + lane);
-            acc.x += wt * o.x;
-            acc.y += wt * o.y;
-            acc.z += wt * o.z;
-            acc.w += wt * o.w;
-          }
-          const float inv = 1.0f / Ls;
-          const __half2 u = __floats2half2_rn(acc.x * inv, acc.y * inv);
-          const __half2 v = __floats2half2_rn(acc.z * inv, acc.w * inv);
-          *reinterpret_cast<uint2 *>(p.out + obase + hh * kHeadDim + 4 * lane) = make_uint2(h2_as_u32(u), h2_as_u32(v));
-        }
+        merge_pieces(p, obase, G, wf, wl, cc.start, T, W, lane);
         if (lane == 0) p.tickets[static_cast<long>(cc.b) * H + cc.h] = 0u;
       }
     }
+    rem -= take;
+    page = p1;
+    first = false;
   }
 
   if (failed) {
     if (lane == 0) flag_error(p.err, S4KV_EFLAG_TIMEOUT);
     // wait (bounded) for the copies still in flight before the CTA exits
-    for (int j = consumed; j < issued; ++j)
-      mbar_wait_bounded(bar0 + 8 * (j % kStages), (j / kStages) & 1, kWaitLimitCycles);
+    for (int j = consumed; j < issued; ++j) {
+      mbar_wait_bounded(c0.bar, c0.phase, kWaitLimitCycles);
+      c0 = next_pos(c0);
+    }
   }
 }
 

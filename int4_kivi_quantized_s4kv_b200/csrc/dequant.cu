@@ -16,7 +16,8 @@ __global__ void __launch_bounds__(128) dequant_kernel(const DequantParams p) {
   const int c = threadIdx.x;  // channel
   const uint8_t *blk = p.pool + (static_cast<long>(p.physical_page) * p.num_kv_heads + h) * kBlockBytes;
   const float ks = __half2float(reinterpret_cast<const __half *>(blk + kKScaleOff)[c]);
-  const float kz = __half2float(reinterpret_cast<const __half *>(blk + kKZeroOff)[c]);
+  const int zslot = 16 * ((c & 31) >> 2) + 2 * (c >> 5) + (c & 1) + 8 * ((c & 3) >> 1);
+  const float kz = __half2float(reinterpret_cast<const __half *>(blk + kKZeroOff)[zslot]);
   const int g = c / kVGroup;
   // key fragment coordinates of channel c: lane quarter i, tile kt, pair e
   const int ki = c >> 5, kt = (c & 31) >> 2, ke = c & 3;

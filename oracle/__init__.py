@@ -55,6 +55,8 @@ def lib():
         L.s4kv_ref_quantize_group.restype = f32
         L.s4kv_ref_key_code_slot.argtypes = [i32, i32, P, P]
         L.s4kv_ref_value_code_slot.argtypes = [i32, i32, P, P]
+        L.s4kv_ref_key_zero_slot.argtypes = [i32]
+        L.s4kv_ref_key_zero_slot.restype = i32
         L.s4kv_ref_quantize_page.argtypes = [P, P, P]
         L.s4kv_ref_unpack_codes.argtypes = [P, P, P]
         L.s4kv_ref_dequant_block.argtypes = [P, P, P]
@@ -123,6 +125,11 @@ def value_code_slot(t: int, c: int) -> tuple[int, int]:
     nb = np.zeros(1, np.int32)
     lib().s4kv_ref_value_code_slot(t, c, _p(w), _p(nb))
     return int(w[0]), int(nb[0])
+
+
+def key_zero_slot(c: int) -> int:
+    """Position (in halves, within the key-zero region) of channel c."""
+    return int(lib().s4kv_ref_key_zero_slot(int(c)))
 
 
 def quantize_page(kp, vp) -> np.ndarray:

@@ -37,7 +37,8 @@
  *   [   0,1024) key codes   : 256 little-endian 32-bit words
  *   [1024,2048) value codes : 256 little-endian 32-bit words
  *   [2048,2304) key scale   : fp16 [128 channels]
- *   [2304,2560) key zero    : fp16 [128 channels]
+ *   [2304,2560) key zero    : fp16 [8 k-tiles][16 k-slots], channel c at
+ *                             k-tile (c%32)/4, slot 2*(c/32) + (c%2) + 8*((c%4)/2)
  *   [2560,2688) value scale : fp16 [4 groups][16 tokens]
  *   [2688,2816) value zero  : fp16 [4 groups][16 tokens]
  * Code word w (0..255) splits as w = 128*h + 4*lane + q with lane = 4*n + i
@@ -160,6 +161,13 @@ float s4kv_ref_quantize_group(const uint16_t *x, int n, int stride,
 
 /* ------------------------------------------------------------- packing -- */
 
+/* Position (in halves) of channel c's key zero point: the zero points are
+ * stored in the order in which the MMA k axis visits the channels. */
+int s4kv_ref_key_zero_slot(int c) {
+    int i = c / 32, kt = (c % 32) / 4, e = c % 4;
+    return 16 * kt + 2 * i + (e % 2) + 8 * (e / 2);
+}
+
 /* (token, channel) -> (word, nibble) of the key code region. */
 void s4kv_ref_key_code_slot(int t, int c, int *word, int *nibble) {
     int i = c / 32, kt = (c % 32) / 4, e = c % 4;
@@ -207,7 +215,7 @@ void s4kv_ref_quantize_page(const uint16_t *kp, const uint16_t *vp,
         s4kv_ref_quantize_group(kp + c, PAGE, HEAD_DIM, &kc[0][c], HEAD_DIM,
                                 &sh, &zh);
         put_half(block + KSCALE_OFF + 2 * c, sh);
-        put_half(block + KZERO_OFF + 2 * c, zh);
+        put_half(block + KZERO_OFF + 2 * s4kv_ref_key_zero_slot(c), zh);
     }
     /* values: one group per token and 32-channel slice */
     for (int t = 0; t < PAGE; ++t) {
@@ -253,7 +261,7 @@ void s4kv_ref_dequant_block(const uint8_t *block, float *kout, float *vout) {
     for (int t = 0; t < PAGE; ++t) {
         for (int c = 0; c < HEAD_DIM; ++c) {
             float ks = s4kv_ref_half_to_float(get_half(block + KSCALE_OFF + 2 * c));
-            float kz = s4kv_ref_half_to_float(get_half(block + KZERO_OFF + 2 * c));
+            float kz = s4kv_ref_half_to_float(get_half(block + KZERO_OFF + 2 * s4kv_ref_key_zero_slot(c)));
             int g = c / VGROUP;
             float vs = s4kv_ref_half_to_float(get_half(block + VSCALE_OFF + 2 * (g * PAGE + t)));
             float vz = s4kv_ref_half_to_float(get_half(block + VZERO_OFF + 2 * (g * PAGE + t)));

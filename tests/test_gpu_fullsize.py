@@ -1,0 +1,85 @@
+"""Full-size parity in the launch configuration bench.py times: each workload
+is built at its full shape by bench.DeviceWorkload (device-side seeded K/V,
+appends through the C ABI), one step runs, and sampled (layer, sequence)
+pairs are recomputed one by one by the oracle from the same K/V (copied back
+from the device generator): their pool pages and residual rows bit-exact,
+their decode outputs within 2e-3 + 1e-3 |ref|."""
+import gc
+
+import numpy as np
+import pytest
+
+from int4_kivi_quantized_s4kv_b200 import workloads as W
+from tests.helpers import assert_attention_close
+
+pytestmark = pytest.mark.gpu
+
+PAGE = 16
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    import torch
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import oracle
+    oracle.build()
+    from int4_kivi_quantized_s4kv_b200 import build
+    build.build()
+
+
+def _check_sequence(wl, layer, b):
+    import torch
+    import oracle
+    spec = wl.spec
+    L = int(wl.lens[b])
+    H = spec.num_kv_heads
+    k, v = W.kv_sequence_torch(spec, layer, b, L, wl.device)
+    k, v = k.cpu().numpy(), v.cpu().numpy()
+    need = (L + PAGE - 1) // PAGE
+    bt = np.arange(need, dtype=np.int32)[None, :]
+    oc = oracle.OracleCache(need + 1, H, 1)
+    sm = W.slot_mapping(bt, [np.arange(L)])
+    assert oc.append(k, v, sm, np.array([0, L], np.int32), np.array([L], np.int32), bt) == 0
+    # cache bytes of this sequence's pages and residual rows
+    full = L // PAGE
+    gpu_pages = wl.plan.block_tables[b, :full]
+    pool = wl.caches[layer].pool[torch.from_numpy(gpu_pages.astype(np.int64)).to(wl.device)].cpu().numpy()
+    assert np.array_equal(pool, oc.pool[:full]), f"pool pages of layer {layer} seq {b}"
+    r = L % PAGE
+    rk = wl.caches[layer].res_k[b, :, :r].cpu().numpy().view(np.uint16)
+    assert np.array_equal(rk, oc.res_k[0, :, :r]), f"residual of layer {layer} seq {b}"
+    q = wl.q[layer][b:b + 1].cpu().numpy()
+    ref = oc.decode_attention(q, np.array([L], np.int32), bt)[0]
+    got = wl.out[layer][b].float().cpu().numpy()
+    return assert_attention_close(got, ref, f"{spec.name} layer {layer} seq {b} (L={L})")
+
+
+SAMPLES = {
+    "qwen2.5-7b": [(0, 0), (0, 31), (0, 63)],
+    "llama3.1-8b": [(0, 0), (0, 128), (0, 255)],
+    "llama3-70b": [(0, 0), (0, 15)],
+    "llama3.2-3b-step": [(0, "longest"), (13, 5), (27, "shortest")],
+}
+
+
+@pytest.mark.parametrize("name", list(SAMPLES))
+def test_full_size_sampled_parity(name):
+    import torch
+    import bench
+    spec = W.SPECS[name]
+    wl = bench.DeviceWorkload(spec, torch.device("cuda", 0))
+    for _ in range(2):       # the step is idempotent: run it twice like warm-up
+        wl.step()
+    torch.cuda.synchronize()
+    for c in wl.caches:
+        assert wl.S.s4kv_get_error(c) == 0
+    for layer, b in SAMPLES[name]:
+        if b == "longest":
+            b = int(np.argmax(wl.lens))
+        elif b == "shortest":
+            b = int(np.argmin(wl.lens))
+        _check_sequence(wl, layer, b)
+    del wl
+    gc.collect()
+    torch.cuda.empty_cache()

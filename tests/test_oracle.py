@@ -9,7 +9,9 @@ Which pin covers which oracle function:
                                    signed zeros) and the exact-rational rounding
                                    bound |x - (code*s + min)| <= s*(1/2 + 2e-6)
   key/value code slots, packing : bijection over all (token, channel); the
-                                   per-channel / per-token closed forms read back
+                                   per-channel / per-token closed forms read back;
+                                   the PTX mma.m16n8k16 fragment table (codes and
+                                   the k order of the key zero points)
   block_bytes, kv_payload_bytes : the pages' worked sizes (tests/golden/kv_bytes.txt)
                                    and the ~3x density claim
   append                        : chunking invariance; closed-form page contents;
@@ -168,6 +170,22 @@ def test_code_layout_is_the_mma_operand_order(oracle_mod):
             assert (col, ch) == (t, c)
 
 
+def test_key_zero_order_is_the_mma_k_order(oracle_mod):
+    """Key zero points are stored in the order the m16n8k16 k axis visits
+    channels: k-tile kt, slot s holds the channel whose code sits in k column
+    s of tile kt (same map as the code layout), so one ldmatrix row of 8
+    halves is a lane quad's k columns."""
+    seen = set()
+    for c in range(HD):
+        pos = oracle_mod.key_zero_slot(c)
+        kt, slot = divmod(pos, 16)
+        seen.add(pos)
+        # the key code of channel c, token 0, sits in tile kt at column `slot`
+        tile, lane, row, col = _fragment_position(*oracle_mod.key_code_slot(0, c))
+        assert (tile, col) == (kt, slot)
+    assert seen == set(range(HD))
+
+
 def _grid_page(rng, per="key"):
     """fp16 [16][128] whose groups are exact 16-level grids: returns the page,
     expected codes, and per-group (scale, zero)."""
@@ -200,7 +218,8 @@ def test_page_axis_split_closed_form(oracle_mod):
     kc, vc = oracle_mod.unpack_codes(blk)
     assert np.array_equal(kc, kc_ref) and np.array_equal(vc, vc_ref)
     ks = blk[2048:2304].view(np.float16).astype(np.float64)
-    kz = blk[2304:2560].view(np.float16).astype(np.float64)
+    kz_slots = blk[2304:2560].view(np.float16).astype(np.float64)
+    kz = np.array([kz_slots[oracle_mod.key_zero_slot(c)] for c in range(HD)])
     vs = blk[2560:2688].view(np.float16).astype(np.float64).reshape(4, 16)
     vz = blk[2688:2816].view(np.float16).astype(np.float64).reshape(4, 16)
     assert np.array_equal(ks, kd) and np.array_equal(kz, ka)
