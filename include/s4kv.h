@@ -191,6 +191,33 @@ S4KV_API int s4kv_decode_attention(const s4kv_cache_t *cache, const void *q,
                           void *workspace, size_t workspace_bytes,
                           void *stream);
 
+/* Size of the fixed scratch array behind s4kv_decode_attention_noalloc. */
+#define S4KV_NOALLOC_SCRATCH_BYTES (24u * 1024u * 1024u)
+
+/* Decode attention that allocates nothing and takes no workspace.  The source
+ * pages have no counterpart to this call: it exists for callers that cannot
+ * call cudaMalloc, such as a plugin inside a host engine that owns the
+ * device's whole memory pool, or a latency-critical path that cannot afford
+ * cudaMalloc's implicit device-wide synchronisation.
+ *  Arguments and result: as s4kv_decode_attention, without the workspace.
+ *  Scratch: one device array of S4KV_NOALLOC_SCRATCH_BYTES (24 MiB) inside
+ *          the library; every GPU that loads the library holds it until the
+ *          process exits.  A batch whose decode workspace
+ *          (s4kv_decode_workspace_size) would exceed it is rejected with
+ *          S4KV_ERR_WORKSPACE and nothing is launched.
+ *  Set-up: the first call on a device looks up the array's device address
+ *          (make that first call before any stream capture).
+ *  Sharing: each call clears, on `stream`, the part of the array that must
+ *          start at zero; all calls on a device share the array and it keeps
+ *          the last call's contents, so calls whose kernels overlap on the
+ *          GPU race.
+ * No cudaMalloc, cudaFree or other allocating routine is called. */
+S4KV_API int s4kv_decode_attention_noalloc(const s4kv_cache_t *cache, const void *q,
+                                           int num_q_heads, const int32_t *seq_lens,
+                                           const int32_t *block_tables, int batch,
+                                           int max_pages_per_seq, float sm_scale,
+                                           void *out, void *stream);
+
 /* Dequantize one physical page for all kv heads into natural order:
  * out_k, out_v device [num_kv_heads][16][128], fp32 if out_fp32 != 0
  * (x = code*scale + zero, exact product, one rounding) else fp16 (the fp32

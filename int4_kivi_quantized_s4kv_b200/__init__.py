@@ -19,6 +19,7 @@ PAGE_TOKENS = 16
 VALUE_GROUP = 32
 BLOCK_BYTES = 2816
 MAX_GQA_GROUP = 8
+NOALLOC_SCRATCH_BYTES = 24 * 1024 * 1024
 
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_DEVICE_CHECK, ERR_WORKSPACE = range(6)
 EFLAG_PAGE_RANGE, EFLAG_SLOT, EFLAG_SEQ_LEN, EFLAG_TIMEOUT = 1, 2, 4, 8
@@ -43,6 +44,7 @@ _SIGS = {
     "s4kv_append": ([_CP, _P, _P, _I, _P, _P, _P, _P, _I, _I, _I, _P], _I),
     "s4kv_decode_workspace_size": ([_I, _I, ctypes.POINTER(_SZ)], _I),
     "s4kv_decode_attention": ([_CP, _P, _I, _P, _P, _I, _I, ctypes.c_float, _P, _P, _SZ, _P], _I),
+    "s4kv_decode_attention_noalloc": ([_CP, _P, _I, _P, _P, _I, _I, ctypes.c_float, _P, _P], _I),
     "s4kv_dequant_page": ([_CP, _I, _P, _P, _I, _P], _I),
     "s4kv_get_error": ([_CP, ctypes.POINTER(ctypes.c_uint32), _I, _P], _I),
 }
@@ -180,6 +182,23 @@ def s4kv_decode_attention(cache: S4KVCache, q, seq_lens, block_tables, out, work
                                     _ptr(workspace, torch.uint8, "workspace"), workspace.numel(),
                                     _stream(stream))
     _check(st, "s4kv_decode_attention")
+
+
+def s4kv_decode_attention_noalloc(cache: S4KVCache, q, seq_lens, block_tables, out,
+                                  sm_scale: float | None = None, stream=None):
+    """Decode attention for callers that cannot allocate device memory: the
+    scratch is a fixed 24 MiB array inside the library (shared by all calls
+    on a device; overlapping calls race)."""
+    import torch
+    batch, num_q_heads, _ = q.shape
+    if sm_scale is None:
+        sm_scale = HEAD_DIM ** -0.5
+    st = lib().s4kv_decode_attention_noalloc(cache.ref, _ptr(q, torch.float16, "q"), num_q_heads,
+                                            _ptr(seq_lens, torch.int32, "seq_lens"),
+                                            _ptr(block_tables, torch.int32, "block_tables"), batch,
+                                            block_tables.shape[1], float(sm_scale),
+                                            _ptr(out, torch.float16, "out"), _stream(stream))
+    _check(st, "s4kv_decode_attention_noalloc")
 
 
 def s4kv_dequant_page(cache: S4KVCache, physical_page: int, out_k, out_v, out_fp32: bool = True,
