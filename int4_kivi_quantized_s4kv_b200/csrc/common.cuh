@@ -117,13 +117,15 @@ __device__ __forceinline__ uint32_t lds32(uint32_t base) {
   return v;
 }
 
-// Four 8x8 b16 matrices from shared memory, one row address per lane (lanes
-// 8m..8m+7 give matrix m's rows), straight into an MMA operand fragment.
+// Four 8x8 b16 matrices from shared memory at [addr + OFF], one row address
+// per lane (lanes 8m..8m+7 give matrix m's rows), straight into an MMA
+// operand fragment.
+template <int OFF>
 __device__ __forceinline__ void ldmatrix_x4(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2,
                                             uint32_t &r3) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4+%5];"
                : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-               : "r"(addr));
+               : "r"(addr), "n"(OFF));
 }
 
 // ------------------------------------------------ mbarrier + bulk copies --

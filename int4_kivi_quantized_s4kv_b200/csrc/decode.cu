@@ -64,8 +64,15 @@ constexpr long long kWaitLimitCycles = 2000000000LL;  // about one second
 constexpr unsigned kFull = 0xFFFFFFFFu;
 constexpr float kHeadroom = 4.0f;  // log2 headroom of the softmax reference
 
+// Query fragments of the current piece can live in a per-warp shared slice
+// ([4 k-tile pairs][32 lanes][16 B]) instead of 16 registers per lane.
+#ifndef S4KV_Q_IN_SMEM
+#define S4KV_Q_IN_SMEM 0
+#endif
+constexpr int kQBytesPerWarp = S4KV_Q_IN_SMEM ? 2048 : 0;
+
 size_t decode_smem_bytes() {
-  return static_cast<size_t>(kWarpsPerCta) * kStages * (kBlockBytes + 8);
+  return static_cast<size_t>(kWarpsPerCta) * (kStages * (kBlockBytes + 8) + kQBytesPerWarp);
 }
 
 __device__ __forceinline__ int clamp_len(int L, int max_pages) {
@@ -138,39 +145,66 @@ __device__ __forceinline__ StageAddr stage_addr_of(uint32_t stage_base, int lane
 
 // Logits of one quantized page: this lane's S^T[tokens n, n+8][heads 2i,
 // 2i+1] before scaling.
-__device__ __forceinline__ void qk_page(const StageAddr &a, const uint32_t (&qf)[16], float (&S)[4]) {
+// Query fragments of this lane: in registers, or in the warp's shared slice.
+struct QFrag {
+#if S4KV_Q_IN_SMEM
+  uint32_t addr;  // this lane's 16 B in k-tile pair 0; pair m at + 512 m
+  __device__ __forceinline__ uint4 pair(int m) const { return m == 0 ? lds128<0>(addr) : m == 1 ? lds128<512>(addr) : m == 2 ? lds128<1024>(addr) : lds128<1536>(addr); }
+#else
+  uint32_t w[16];
+  __device__ __forceinline__ uint4 pair(int m) const { return make_uint4(w[4 * m], w[4 * m + 1], w[4 * m + 2], w[4 * m + 3]); }
+#endif
+};
+
+// Key zero-point operand of k-tile kt (kt is a constant after unrolling, so
+// the switch folds to one ldmatrix with an immediate offset).
+__device__ __forceinline__ void ldmatrix_kzero(uint32_t base, int kt, uint32_t &z0, uint32_t &z1, uint32_t &z2,
+                                               uint32_t &z3) {
+  switch (kt) {
+    case 0: ldmatrix_x4<0>(base, z0, z1, z2, z3); break;
+    case 1: ldmatrix_x4<32>(base, z0, z1, z2, z3); break;
+    case 2: ldmatrix_x4<64>(base, z0, z1, z2, z3); break;
+    case 3: ldmatrix_x4<96>(base, z0, z1, z2, z3); break;
+    case 4: ldmatrix_x4<128>(base, z0, z1, z2, z3); break;
+    case 5: ldmatrix_x4<160>(base, z0, z1, z2, z3); break;
+    case 6: ldmatrix_x4<192>(base, z0, z1, z2, z3); break;
+    default: ldmatrix_x4<224>(base, z0, z1, z2, z3); break;
+  }
+}
+
+__device__ __forceinline__ void qk_page(const StageAddr &a, const QFrag &q, float (&S)[4]) {
   // three independent accumulators (hi part, lo part, zero-point term) keep
   // the dependent MMA chains 8 deep instead of 24
   float Sh[4] = {0.f, 0.f, 0.f, 0.f}, Sl[4] = {0.f, 0.f, 0.f, 0.f}, Sz[4] = {0.f, 0.f, 0.f, 0.f};
   const uint4 kw0 = lds128<kKCodeOff>(a.code);
   const uint4 kw1 = lds128<kKCodeOff + 512>(a.code);
   const uint32_t kws[8] = {kw0.x, kw0.y, kw0.z, kw0.w, kw1.x, kw1.y, kw1.z, kw1.w};
-  uint32_t sk[16];
-  {
-    const uint4 s0 = lds128<kKScaleOff>(a.kmeta), s1 = lds128<kKScaleOff + 16>(a.kmeta);
-    const uint4 s2 = lds128<kKScaleOff + 32>(a.kmeta), s3 = lds128<kKScaleOff + 48>(a.kmeta);
-    const uint4 sv[4] = {s0, s1, s2, s3};
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      sk[4 * k] = sv[k].x; sk[4 * k + 1] = sv[k].y; sk[4 * k + 2] = sv[k].z; sk[4 * k + 3] = sv[k].w;
+  for (int m = 0; m < 4; ++m) {
+    // key scales and query words for k-tiles 2m, 2m+1 (four channel pairs)
+    const uint4 sv = m == 0 ? lds128<kKScaleOff>(a.kmeta) : m == 1 ? lds128<kKScaleOff + 16>(a.kmeta)
+                   : m == 2 ? lds128<kKScaleOff + 32>(a.kmeta) : lds128<kKScaleOff + 48>(a.kmeta);
+    const uint4 qv = q.pair(m);
+    const uint32_t sk[4] = {sv.x, sv.y, sv.z, sv.w};
+    const uint32_t qw[4] = {qv.x, qv.y, qv.z, qv.w};
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int kt = 2 * m + h;
+      uint32_t a0, a1, a2, a3;
+      unpack_codes(kws[kt], a0, a1, a2, a3);
+      const __half2 qb0 = u32_as_h2(qw[2 * h]), qb1 = u32_as_h2(qw[2 * h + 1]);
+      const __half2 s0 = u32_as_h2(sk[2 * h]), s1 = u32_as_h2(sk[2 * h + 1]);
+      // q * sK split into fp16 hi + lo; the lo part is the exact remainder
+      const __half2 h0 = __hmul2(qb0, s0), h1 = __hmul2(qb1, s1);
+      const __half2 r0 = __hfma2(qb0, s0, __hneg2(h0));
+      const __half2 r1 = __hfma2(qb1, s1, __hneg2(h1));
+      mma16816(Sh, a0, a1, a2, a3, h2_as_u32(h0), h2_as_u32(h1));
+      mma16816(Sl, a0, a1, a2, a3, h2_as_u32(r0), h2_as_u32(r1));
+      // key zero point: every A row is zK (one ldmatrix), so each row gets sum_c zK q
+      uint32_t z0, z1, z2, z3;
+      ldmatrix_kzero(a.kzero, 2 * m + h, z0, z1, z2, z3);
+      mma16816(Sz, z0, z1, z2, z3, qw[2 * h], qw[2 * h + 1]);
     }
-  }
-#pragma unroll
-  for (int kt = 0; kt < 8; ++kt) {
-    uint32_t a0, a1, a2, a3;
-    unpack_codes(kws[kt], a0, a1, a2, a3);
-    const __half2 qb0 = u32_as_h2(qf[2 * kt]), qb1 = u32_as_h2(qf[2 * kt + 1]);
-    const __half2 s0 = u32_as_h2(sk[2 * kt]), s1 = u32_as_h2(sk[2 * kt + 1]);
-    // q * sK split into fp16 hi + lo; the lo part is the exact remainder
-    const __half2 h0 = __hmul2(qb0, s0), h1 = __hmul2(qb1, s1);
-    const __half2 r0 = __hfma2(qb0, s0, __hneg2(h0));
-    const __half2 r1 = __hfma2(qb1, s1, __hneg2(h1));
-    mma16816(Sh, a0, a1, a2, a3, h2_as_u32(h0), h2_as_u32(h1));
-    mma16816(Sl, a0, a1, a2, a3, h2_as_u32(r0), h2_as_u32(r1));
-    // key zero point: every A row is zK (one ldmatrix), so each row gets sum_c zK q
-    uint32_t z0, z1, z2, z3;
-    ldmatrix_x4(a.kzero + 32 * kt, z0, z1, z2, z3);
-    mma16816(Sz, z0, z1, z2, z3, qf[2 * kt], qf[2 * kt + 1]);
   }
 #pragma unroll
   for (int k = 0; k < 4; ++k) S[k] = (Sh[k] + Sl[k]) + Sz[k];
@@ -261,14 +295,14 @@ __device__ __forceinline__ void pv_page(const StageAddr &a, const uint32_t (&P)[
   pv_group<3>(a, P, vws, st);
   // value zero points: A row r carries group r % 4's zV (one ldmatrix), B = P
   uint32_t z0, z1, z2, z3;
-  ldmatrix_x4(a.vzero, z0, z1, z2, z3);
+  ldmatrix_x4<0>(a.vzero, z0, z1, z2, z3);
   mma16816(st.Z, z0, z1, z2, z3, P[0], P[1]);
   mma16816(st.Z, z0, z1, z2, z3, P[2], P[3]);
 }
 
 // The partial last page, read straight from the fp16 residual (r rows valid).
 __device__ __forceinline__ void residual_page(const __half *rk, const __half *rv, int r,
-                                              const uint32_t (&qf)[16], int lane, float scale_log2,
+                                              const QFrag &q, int lane, float scale_log2,
                                               Online &st) {
   const int n = lane >> 2, i = lane & 3;
   uint32_t kn[16], kn8[16];
@@ -282,8 +316,11 @@ __device__ __forceinline__ void residual_page(const __half *rk, const __half *rv
   }
   float S[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-  for (int kt = 0; kt < 8; ++kt)
-    mma16816(S, kn[2 * kt], kn8[2 * kt], kn[2 * kt + 1], kn8[2 * kt + 1], qf[2 * kt], qf[2 * kt + 1]);
+  for (int m = 0; m < 4; ++m) {
+    const uint4 qv = q.pair(m);
+    mma16816(S, kn[4 * m], kn8[4 * m], kn[4 * m + 1], kn8[4 * m + 1], qv.x, qv.y);
+    mma16816(S, kn[4 * m + 2], kn8[4 * m + 2], kn[4 * m + 3], kn8[4 * m + 3], qv.z, qv.w);
+  }
   if (n >= r) S[0] = S[1] = -INFINITY;
   if (n + 8 >= r) S[2] = S[3] = -INFINITY;
   uint32_t P[4];
@@ -381,6 +418,8 @@ __global__ void __launch_bounds__(kThreads, S4KV_DECODE_MIN_CTAS) decode_kernel(
   const int n = lane >> 2, i = lane & 3;
   const uint32_t ring0 = smem_addr(smem) + warp * kStages * kBlockBytes;
   const uint32_t bar0 = smem_addr(smem) + kWarpsPerCta * kStages * kBlockBytes + warp * kStages * 8;
+  const uint32_t qslice = smem_addr(smem) + kWarpsPerCta * kStages * (kBlockBytes + 8) + warp * kQBytesPerWarp;
+  (void)qslice;
   const long long worker = static_cast<long long>(blockIdx.x) * kWarpsPerCta + warp;
   const int B = p.batch, H = p.num_kv_heads, G = p.group;
 
@@ -494,12 +533,9 @@ __global__ void __launch_bounds__(kThreads, S4KV_DECODE_MIN_CTAS) decode_kernel(
       mbar_arrive_expect_tx(p_bar, kBlockBytes);
       bulk_copy_g2s(ring0 + p_stage, p_head + phys * page_stride, kBlockBytes, p_bar);
     }
-    p_stage += kBlockBytes;
-    p_bar += 8;
-    if (p_stage == kStages * kBlockBytes) {
-      p_stage = 0;
-      p_bar = bar0;
-    }
+    const bool wrap = (p_stage == (kStages - 1) * kBlockBytes);
+    p_stage = wrap ? 0u : p_stage + kBlockBytes;
+    p_bar = wrap ? bar0 : p_bar + 8;
     ++issued;
   };
   static_assert(kStages >= 4, "the pipeline holds three stages at once");
@@ -511,19 +547,17 @@ __global__ void __launch_bounds__(kThreads, S4KV_DECODE_MIN_CTAS) decode_kernel(
     uint32_t off, bar, phase;
   };
   auto next_pos = [&](Pos q) {
-    q.off += kBlockBytes;
-    q.bar += 8;
-    if (q.off == kStages * kBlockBytes) {
-      q.off = 0;
-      q.bar = bar0;
-      q.phase ^= 1u;
-    }
+    const bool wrap = (q.off == (kStages - 1) * kBlockBytes);
+    q.off = wrap ? 0u : q.off + kBlockBytes;
+    q.bar = wrap ? bar0 : q.bar + 8;
+    q.phase ^= wrap ? 1u : 0u;
     return q;
   };
   int consumed = 0;
   bool failed = false;
   Pos c0{0u, bar0, 0u};
   auto wait_copy = [&](const Pos &q) {
+    if (__all_sync(kFull, mbar_try_wait(q.bar, q.phase))) return true;
     const bool ok = mbar_wait_bounded(q.bar, q.phase, kWaitLimitCycles);
     return !__any_sync(kFull, !ok);
   };
@@ -548,18 +582,31 @@ __global__ void __launch_bounds__(kThreads, S4KV_DECODE_MIN_CTAS) decode_kernel(
     const bool complete = (page == 0) && (p1 == cc.np);
     const int nq = max(0, min(p1, cc.nfull) - page);
 
-    uint32_t qf[16];
-    if (n < G) {
-      const uint4 *qp = reinterpret_cast<const uint4 *>(
-          p.q + (static_cast<long>(cc.b) * p.num_q_heads + cc.h * G + n) * kHeadDim + 32 * i);
+    QFrag qf;
+    {
+      uint4 qv[4] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0),
+                     make_uint4(0, 0, 0, 0)};
+      if (n < G) {
+        const uint4 *qp = reinterpret_cast<const uint4 *>(
+            p.q + (static_cast<long>(cc.b) * p.num_q_heads + cc.h * G + n) * kHeadDim + 32 * i);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) qv[k] = __ldg(qp + k);
+      }
+#if S4KV_Q_IN_SMEM
+      qf.addr = qslice + 16u * lane;
+      __syncwarp();  // the previous piece's reads of the slice are done
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(qf.addr + 512u * k), "r"(qv[k].x), "r"(qv[k].y),
+                     "r"(qv[k].z), "r"(qv[k].w)
+                     : "memory");
+      __syncwarp();
+#else
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
-        const uint4 v = __ldg(qp + k);
-        qf[4 * k] = v.x; qf[4 * k + 1] = v.y; qf[4 * k + 2] = v.z; qf[4 * k + 3] = v.w;
+        qf.w[4 * k] = qv[k].x; qf.w[4 * k + 1] = qv[k].y; qf.w[4 * k + 2] = qv[k].z; qf.w[4 * k + 3] = qv[k].w;
       }
-    } else {
-#pragma unroll
-      for (int k = 0; k < 16; ++k) qf[k] = 0u;
+#endif
     }
     Online st;
     st.ref0 = st.ref1 = -INFINITY;
