@@ -46,6 +46,35 @@ def measured_hbm_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+# ---------------------------------------------------------------- traffic --
+
+KERNEL_SOURCES = ["int4_kivi_quantized_s4kv_b200/csrc/decode.cu", "int4_kivi_quantized_s4kv_b200/csrc/common.cuh",
+                  "int4_kivi_quantized_s4kv_b200/csrc/kernels.cuh", "include/s4kv.h"]
+
+
+def kernel_sources_sha() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def recorded_traffic(algorithmic_bytes: float):
+    """DRAM bytes (read + write) per decode launch from the committed ncu
+    capture, scaled from the captured case by algorithmic bytes; None when
+    the decode kernel's sources changed since the capture."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "decode_traffic.json")) as f:
+            rec = json.load(f)
+    except Exception:
+        return None
+    if rec.get("kernel_sources_sha256") != kernel_sources_sha():
+        return None
+    return algorithmic_bytes * rec["dram_bytes"] / rec["algorithmic_bytes"]
+
+
 # ----------------------------------------------------------------- clocks --
 
 class ClockSampler:
@@ -466,7 +495,8 @@ def main(argv=None):
             "sequences_per_s": world * spec.batch / (step_ms * 1e-3),
             "kv_tokens_per_s": world * spec.layers * int(wl.lens.sum()) / (step_ms * 1e-3),
             "roofline": {"bound": "hbm", "kernel": "decode_kernel", "achieved": achieved, "peak": peak,
-                         "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak, "traffic": None,
+                         "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
+                         "traffic": recorded_traffic(decode_bytes_per_launch),
                          "bytes_per_launch": decode_bytes_per_launch, "avg_launch_ms": dec_avg_ms},
             "e2e": {"value": aggregate_gbs(world, bytes_per_step, e2e_ms), "unit": "GB/s",
                     "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
