@@ -119,6 +119,7 @@ __device__ __forceinline__ long long worker_of(long long x, long long T, long lo
 // Running softmax state of one lane: heads 2i, 2i+1 of the group.
 struct Online {
   float ref0, ref1;  // log2-domain reference: weights are exp2(s - ref) <= 1
+  float thr0, thr1;  // raw-logit threshold ref / scale (rounded down)
   float l0, l1;      // partial sums of weights over this lane's tokens
   float O[8][4];     // PV accumulators (M-tile, C fragment)
   float Z[4];        // value zero-point term: sum_t zV[g][t] P[t][h]
@@ -176,6 +177,9 @@ __device__ __forceinline__ void qk_page(const StageAddr &a, const QFrag &q, floa
   // three independent accumulators (hi part, lo part, zero-point term) keep
   // the dependent MMA chains 8 deep instead of 24
   float Sh[4] = {0.f, 0.f, 0.f, 0.f}, Sl[4] = {0.f, 0.f, 0.f, 0.f}, Sz[4] = {0.f, 0.f, 0.f, 0.f};
+  // Sl and Sz both collect small terms (lo parts, zero points); even k-tiles
+  // put their lo part in Sl and zero point in Sz, odd k-tiles the reverse,
+  // so the two chains stay balanced and S = Sh + (Sl + Sz).
   const uint4 kw0 = lds128<kKCodeOff>(a.code);
   const uint4 kw1 = lds128<kKCodeOff + 512>(a.code);
   const uint32_t kws[8] = {kw0.x, kw0.y, kw0.z, kw0.w, kw1.x, kw1.y, kw1.z, kw1.w};
@@ -199,11 +203,11 @@ __device__ __forceinline__ void qk_page(const StageAddr &a, const QFrag &q, floa
       const __half2 r0 = __hfma2(qb0, s0, __hneg2(h0));
       const __half2 r1 = __hfma2(qb1, s1, __hneg2(h1));
       mma16816(Sh, a0, a1, a2, a3, h2_as_u32(h0), h2_as_u32(h1));
-      mma16816(Sl, a0, a1, a2, a3, h2_as_u32(r0), h2_as_u32(r1));
+      mma16816(h ? Sz : Sl, a0, a1, a2, a3, h2_as_u32(r0), h2_as_u32(r1));
       // key zero point: every A row is zK (one ldmatrix), so each row gets sum_c zK q
       uint32_t z0, z1, z2, z3;
       ldmatrix_kzero(a.kzero, 2 * m + h, z0, z1, z2, z3);
-      mma16816(Sz, z0, z1, z2, z3, qw[2 * h], qw[2 * h + 1]);
+      mma16816(h ? Sl : Sz, z0, z1, z2, z3, qw[2 * h], qw[2 * h + 1]);
     }
   }
 #pragma unroll
@@ -217,11 +221,10 @@ __device__ __forceinline__ void qk_page(const StageAddr &a, const QFrag &q, floa
 // when a page maximum passes it, for any lane of the warp.
 __device__ __forceinline__ void softmax_page(const float (&S)[4], float scale_log2, Online &st,
                                              uint32_t (&P)[4]) {
-  const float s0 = S[0] * scale_log2, s1 = S[1] * scale_log2;
-  const float s2 = S[2] * scale_log2, s3 = S[3] * scale_log2;
-  // common case: no logit passes the reference, one vote and no shuffles
-  if (__any_sync(kFull, fmaxf(s0, s2) > st.ref0 || fmaxf(s1, s3) > st.ref1)) {
-    float pm0 = fmaxf(s0, s2), pm1 = fmaxf(s1, s3);
+  // common case: no logit passes the reference (compared on the raw logits
+  // against ref / scale, kept in thr), one vote and no shuffles
+  if (__any_sync(kFull, fmaxf(S[0], S[2]) > st.thr0 || fmaxf(S[1], S[3]) > st.thr1)) {
+    float pm0 = fmaxf(S[0], S[2]) * scale_log2, pm1 = fmaxf(S[1], S[3]) * scale_log2;
 #pragma unroll
     for (int off = 4; off < 32; off <<= 1) {
       pm0 = fmaxf(pm0, __shfl_xor_sync(kFull, pm0, off));
@@ -233,6 +236,9 @@ __device__ __forceinline__ void softmax_page(const float (&S)[4], float scale_lo
     const float a0 = fast_exp2(st.ref0 - n0), a1 = fast_exp2(st.ref1 - n1);
     st.ref0 = n0;
     st.ref1 = n1;
+    // largest raw logit whose weight stays <= 1 (rounded down: never above)
+    st.thr0 = __fdiv_rd(n0, scale_log2);
+    st.thr1 = __fdiv_rd(n1, scale_log2);
     st.l0 *= a0;
     st.l1 *= a1;
 #pragma unroll
@@ -247,8 +253,8 @@ __device__ __forceinline__ void softmax_page(const float (&S)[4], float scale_lo
     st.Z[2] *= a0;
     st.Z[3] *= a1;
   }
-  const float p0 = fast_exp2(s0 - st.ref0), p2 = fast_exp2(s2 - st.ref0);
-  const float p1 = fast_exp2(s1 - st.ref1), p3 = fast_exp2(s3 - st.ref1);
+  const float p0 = fast_exp2(fmaf(S[0], scale_log2, -st.ref0)), p2 = fast_exp2(fmaf(S[2], scale_log2, -st.ref0));
+  const float p1 = fast_exp2(fmaf(S[1], scale_log2, -st.ref1)), p3 = fast_exp2(fmaf(S[3], scale_log2, -st.ref1));
   st.l0 += p0 + p2;
   st.l1 += p1 + p3;
   // P in fp16 hi + lo, rows = tokens, cols = heads; then transpose
@@ -496,8 +502,10 @@ __global__ void __launch_bounds__(kThreads, S4KV_DECODE_MIN_CTAS) decode_kernel(
   const int p_first = static_cast<int>(s - cc.start);
 
   // ---- producer: issue the next quantized page of [s, e) into the ring.
-  // It walks the same pieces as the consumer: per piece a pointer into the
-  // block table and a count of quantized pages still to issue.
+  // It walks the same pieces as the consumer.  The page ids of a piece are
+  // read 32 at a time into a window (lane l holds the l-th) with one
+  // coalesced load, and taken with a shuffle, so no per-page global load
+  // sits on the warp's critical path.
   const long long page_stride = static_cast<long long>(H) * kBlockBytes;
   Cursor pc = cc;
   int p_page = p_first;       // page index of the producer's current piece start
@@ -505,15 +513,21 @@ __global__ void __launch_bounds__(kThreads, S4KV_DECODE_MIN_CTAS) decode_kernel(
   int p_q = 0;                // quantized pages left in the current piece
   const int32_t *p_bt = nullptr;
   const uint8_t *p_head = nullptr;
+  int p_win = 0, p_widx = 0;  // window of page ids, next index into it
   uint32_t p_stage = 0;       // stage index * kBlockBytes
   uint32_t p_bar = bar0;
   int issued = 0;
+  auto p_window = [&]() {     // the next (up to) 32 page ids of the piece
+    p_win = lane < p_q ? __ldg(p_bt + lane) : 0;
+    p_widx = 0;
+  };
   auto p_piece = [&]() {      // set up the piece starting at p_page
     const int take = min(p_left, pc.np - p_page);
     p_q = max(0, min(p_page + take, pc.nfull) - p_page);
     p_bt = pc.bt + p_page;
     p_head = p.pool + static_cast<long long>(pc.h) * kBlockBytes;
     p_left -= take;
+    p_window();
   };
   p_piece();
   auto produce = [&]() {
@@ -523,7 +537,12 @@ __global__ void __launch_bounds__(kThreads, S4KV_DECODE_MIN_CTAS) decode_kernel(
       p_page = 0;
       p_piece();
     }
-    int phys = __ldg(p_bt++);
+    if (p_widx == 32) {
+      p_bt += 32;
+      p_window();
+    }
+    int phys = __shfl_sync(kFull, p_win, p_widx);
+    ++p_widx;
     --p_q;
     if (static_cast<unsigned>(phys) >= static_cast<unsigned>(p.num_pages)) {
       if (lane == 0) flag_error(p.err, S4KV_EFLAG_PAGE_RANGE);
@@ -610,6 +629,7 @@ __global__ void __launch_bounds__(kThreads, S4KV_DECODE_MIN_CTAS) decode_kernel(
     }
     Online st;
     st.ref0 = st.ref1 = -INFINITY;
+    st.thr0 = st.thr1 = -INFINITY;
     st.l0 = st.l1 = 0.f;
 #pragma unroll
     for (int mt = 0; mt < 8; ++mt) st.O[mt][0] = st.O[mt][1] = st.O[mt][2] = st.O[mt][3] = 0.f;
