@@ -118,9 +118,9 @@ __device__ __forceinline__ long long worker_of(long long x, long long T, long lo
 
 // Running softmax state of one lane: heads 2i, 2i+1 of the group.
 struct Online {
-  float ref0, ref1;  // log2-domain reference: weights are exp2(s - ref) <= 1
+  float2 nref;       // minus the log2-domain reference: weights are exp2(s - ref) <= 1
   float thr0, thr1;  // raw-logit threshold ref / scale (rounded down)
-  float l0, l1;      // partial sums of weights over this lane's tokens
+  float2 l;          // partial sums of weights over this lane's tokens
   float O[8][4];     // PV accumulators (M-tile, C fragment)
   float Z[4];        // value zero-point term: sum_t zV[g][t] P[t][h]
 };
@@ -158,7 +158,10 @@ struct QFrag {
 };
 
 // Key zero-point operand of k-tile kt (kt is a constant after unrolling, so
-// the switch folds to one ldmatrix with an immediate offset).
+// the switch folds to one ldmatrix with an immediate offset).  Its rows are
+// all the same, so two of the four registers repeat the other two; they are
+// loaded as such, because an MMA's A operand must sit in four consecutive
+// registers and one register passed twice would cost copies.
 __device__ __forceinline__ void ldmatrix_kzero(uint32_t base, int kt, uint32_t &z0, uint32_t &z1, uint32_t &z2,
                                                uint32_t &z3) {
   switch (kt) {
@@ -204,14 +207,18 @@ __device__ __forceinline__ void qk_page(const StageAddr &a, const QFrag &q, floa
       const __half2 r1 = __hfma2(qb1, s1, __hneg2(h1));
       mma16816(Sh, a0, a1, a2, a3, h2_as_u32(h0), h2_as_u32(h1));
       mma16816(h ? Sz : Sl, a0, a1, a2, a3, h2_as_u32(r0), h2_as_u32(r1));
-      // key zero point: every A row is zK (one ldmatrix), so each row gets sum_c zK q
+      // key zero point: every A row is zK, so each row gets sum_c zK q
       uint32_t z0, z1, z2, z3;
       ldmatrix_kzero(a.kzero, 2 * m + h, z0, z1, z2, z3);
       mma16816(h ? Sl : Sz, z0, z1, z2, z3, qw[2 * h], qw[2 * h + 1]);
     }
   }
-#pragma unroll
-  for (int k = 0; k < 4; ++k) S[k] = (Sh[k] + Sl[k]) + Sz[k];
+  const float2 s01 = add2(add2(make_float2(Sh[0], Sh[1]), make_float2(Sl[0], Sl[1])), make_float2(Sz[0], Sz[1]));
+  const float2 s23 = add2(add2(make_float2(Sh[2], Sh[3]), make_float2(Sl[2], Sl[3])), make_float2(Sz[2], Sz[3]));
+  S[0] = s01.x;
+  S[1] = s01.y;
+  S[2] = s23.x;
+  S[3] = s23.y;
 }
 
 // Online softmax for one 16-token page.  S: this lane's logits (tokens n,
@@ -230,40 +237,45 @@ __device__ __forceinline__ void softmax_page(const float (&S)[4], float scale_lo
       pm0 = fmaxf(pm0, __shfl_xor_sync(kFull, pm0, off));
       pm1 = fmaxf(pm1, __shfl_xor_sync(kFull, pm1, off));
     }
-    const bool up0 = pm0 > st.ref0, up1 = pm1 > st.ref1;
-    const float n0 = up0 ? pm0 + kHeadroom : st.ref0;
-    const float n1 = up1 ? pm1 + kHeadroom : st.ref1;
-    const float a0 = fast_exp2(st.ref0 - n0), a1 = fast_exp2(st.ref1 - n1);
-    st.ref0 = n0;
-    st.ref1 = n1;
+    const float r0 = -st.nref.x, r1 = -st.nref.y;
+    const float n0 = pm0 > r0 ? pm0 + kHeadroom : r0;
+    const float n1 = pm1 > r1 ? pm1 + kHeadroom : r1;
+    const float2 a = make_float2(fast_exp2(r0 - n0), fast_exp2(r1 - n1));
+    st.nref = make_float2(-n0, -n1);
     // largest raw logit whose weight stays <= 1 (rounded down: never above)
     st.thr0 = __fdiv_rd(n0, scale_log2);
     st.thr1 = __fdiv_rd(n1, scale_log2);
-    st.l0 *= a0;
-    st.l1 *= a1;
+    st.l = mul2(st.l, a);
 #pragma unroll
     for (int mt = 0; mt < 8; ++mt) {
-      st.O[mt][0] *= a0;
-      st.O[mt][1] *= a1;
-      st.O[mt][2] *= a0;
-      st.O[mt][3] *= a1;
+      const float2 o01 = mul2(make_float2(st.O[mt][0], st.O[mt][1]), a);
+      const float2 o23 = mul2(make_float2(st.O[mt][2], st.O[mt][3]), a);
+      st.O[mt][0] = o01.x;
+      st.O[mt][1] = o01.y;
+      st.O[mt][2] = o23.x;
+      st.O[mt][3] = o23.y;
     }
-    st.Z[0] *= a0;
-    st.Z[1] *= a1;
-    st.Z[2] *= a0;
-    st.Z[3] *= a1;
+    const float2 z01 = mul2(make_float2(st.Z[0], st.Z[1]), a);
+    const float2 z23 = mul2(make_float2(st.Z[2], st.Z[3]), a);
+    st.Z[0] = z01.x;
+    st.Z[1] = z01.y;
+    st.Z[2] = z23.x;
+    st.Z[3] = z23.y;
   }
-  const float p0 = fast_exp2(fmaf(S[0], scale_log2, -st.ref0)), p2 = fast_exp2(fmaf(S[2], scale_log2, -st.ref0));
-  const float p1 = fast_exp2(fmaf(S[1], scale_log2, -st.ref1)), p3 = fast_exp2(fmaf(S[3], scale_log2, -st.ref1));
-  st.l0 += p0 + p2;
-  st.l1 += p1 + p3;
+  // exponents (S * scale - ref) for (heads 2i, 2i+1) of tokens n and n+8
+  const float2 sc = make_float2(scale_log2, scale_log2);
+  const float2 x01 = fma2(make_float2(S[0], S[1]), sc, st.nref);
+  const float2 x23 = fma2(make_float2(S[2], S[3]), sc, st.nref);
+  const float2 p01 = make_float2(fast_exp2(x01.x), fast_exp2(x01.y));
+  const float2 p23 = make_float2(fast_exp2(x23.x), fast_exp2(x23.y));
+  st.l = add2(st.l, add2(p01, p23));
   // P in fp16 hi + lo, rows = tokens, cols = heads; then transpose
-  const __half2 h01 = __floats2half2_rn(p0, p1);
-  const __half2 h23 = __floats2half2_rn(p2, p3);
-  const float2 b01 = __half22float2(h01);
-  const float2 b23 = __half22float2(h23);
-  const __half2 l01 = __floats2half2_rn(p0 - b01.x, p1 - b01.y);
-  const __half2 l23 = __floats2half2_rn(p2 - b23.x, p3 - b23.y);
+  const __half2 h01 = __floats2half2_rn(p01.x, p01.y);
+  const __half2 h23 = __floats2half2_rn(p23.x, p23.y);
+  const float2 d01 = sub2(p01, __half22float2(h01));
+  const float2 d23 = sub2(p23, __half22float2(h23));
+  const __half2 l01 = __floats2half2_rn(d01.x, d01.y);
+  const __half2 l23 = __floats2half2_rn(d23.x, d23.y);
   P[0] = movmatrix_trans(h2_as_u32(h01));
   P[1] = movmatrix_trans(h2_as_u32(h23));
   P[2] = movmatrix_trans(h2_as_u32(l01));
@@ -514,8 +526,6 @@ __global__ void __launch_bounds__(kThreads, S4KV_DECODE_MIN_CTAS) decode_kernel(
   const int32_t *p_bt = nullptr;
   const uint8_t *p_head = nullptr;
   int p_win = 0, p_widx = 0;  // window of page ids, next index into it
-  uint32_t p_stage = 0;       // stage index * kBlockBytes
-  uint32_t p_bar = bar0;
   int issued = 0;
   auto p_window = [&]() {     // the next (up to) 32 page ids of the piece
     p_win = lane < p_q ? __ldg(p_bt + lane) : 0;
@@ -530,7 +540,9 @@ __global__ void __launch_bounds__(kThreads, S4KV_DECODE_MIN_CTAS) decode_kernel(
     p_window();
   };
   p_piece();
-  auto produce = [&]() {
+  // fills the stage at byte offset `stage` (barrier `bar`): the ring is kept
+  // full, so that is always the stage the consumer released last
+  auto produce = [&](uint32_t stage, uint32_t bar) {
     while (p_q == 0) {
       if (p_left == 0) return;
       next_segment(pc, p);
@@ -549,17 +561,14 @@ __global__ void __launch_bounds__(kThreads, S4KV_DECODE_MIN_CTAS) decode_kernel(
       phys = 0;
     }
     if (lane == 0) {
-      mbar_arrive_expect_tx(p_bar, kBlockBytes);
-      bulk_copy_g2s(ring0 + p_stage, p_head + phys * page_stride, kBlockBytes, p_bar);
+      mbar_arrive_expect_tx(bar, kBlockBytes);
+      bulk_copy_g2s(ring0 + stage, p_head + phys * page_stride, kBlockBytes, bar);
     }
-    const bool wrap = (p_stage == (kStages - 1) * kBlockBytes);
-    p_stage = wrap ? 0u : p_stage + kBlockBytes;
-    p_bar = wrap ? bar0 : p_bar + 8;
     ++issued;
   };
   static_assert(kStages >= 4, "the pipeline holds three stages at once");
 #pragma unroll 1
-  for (int k = 0; k < kStages; ++k) produce();
+  for (int k = 0; k < kStages; ++k) produce(static_cast<uint32_t>(k) * kBlockBytes, bar0 + 8u * k);
 
   // ---- consumer.  A ring position: stage offset, barrier address, parity.
   struct Pos {
@@ -585,8 +594,9 @@ __global__ void __launch_bounds__(kThreads, S4KV_DECODE_MIN_CTAS) decode_kernel(
     fence_proxy_async();
     __syncwarp();
     ++consumed;
+    const Pos done = c0;
     c0 = next_pos(c0);
-    produce();
+    produce(done.off, done.bar);
   };
 
   int page = p_first, rem = range;
@@ -628,9 +638,9 @@ __global__ void __launch_bounds__(kThreads, S4KV_DECODE_MIN_CTAS) decode_kernel(
 #endif
     }
     Online st;
-    st.ref0 = st.ref1 = -INFINITY;
+    st.nref = make_float2(INFINITY, INFINITY);
     st.thr0 = st.thr1 = -INFINITY;
-    st.l0 = st.l1 = 0.f;
+    st.l = make_float2(0.f, 0.f);
 #pragma unroll
     for (int mt = 0; mt < 8; ++mt) st.O[mt][0] = st.O[mt][1] = st.O[mt][2] = st.O[mt][3] = 0.f;
     st.Z[0] = st.Z[1] = st.Z[2] = st.Z[3] = 0.f;
@@ -711,7 +721,7 @@ __global__ void __launch_bounds__(kThreads, S4KV_DECODE_MIN_CTAS) decode_kernel(
     }
 
     // ---- finish the piece
-    float l0 = st.l0, l1 = st.l1;
+    float l0 = st.l.x, l1 = st.l.y;
 #pragma unroll
     for (int off = 4; off < 32; off <<= 1) {
       l0 += __shfl_xor_sync(kFull, l0, off);
@@ -759,8 +769,8 @@ __global__ void __launch_bounds__(kThreads, S4KV_DECODE_MIN_CTAS) decode_kernel(
             make_float4(st.O[2 * g][1], st.O[2 * g][3], st.O[2 * g + 1][1], st.O[2 * g + 1][3]);
       }
       if (n == 0) {
-        p.part_ml[slot * 8 + 2 * i] = make_float2(st.ref0, l0);
-        p.part_ml[slot * 8 + 2 * i + 1] = make_float2(st.ref1, l1);
+        p.part_ml[slot * 8 + 2 * i] = make_float2(-st.nref.x, l0);
+        p.part_ml[slot * 8 + 2 * i + 1] = make_float2(-st.nref.y, l1);
       }
       __threadfence();
       __syncwarp();
