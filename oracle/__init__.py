@@ -70,6 +70,8 @@ def lib():
         L.s4kv_ref_decode_attention.argtypes = [P, P, P, i32, i32, P, i32, P, P, i32, i32, f64, i32, P]
         L.s4kv_ref_decode_attention.restype = i32
         L.s4kv_ref_attention_fp16.argtypes = [P, P, P, i32, P, i32, i32, f64, P]
+        L.s4kv_ref_prefill_attention.argtypes = [P, P, P, i32, i32, P, i32, P, P, P, i32, i32, f64, P]
+        L.s4kv_ref_prefill_attention.restype = i32
         L.s4kv_ref_attention_fp16.restype = i32
         _lib = L
         del i64
@@ -218,6 +220,27 @@ class OracleCache:
             bt.shape[1], float(sm_scale), 1 if use_double else 0, _p(out))
         if rc != 0:
             raise ValueError(f"decode_attention rc={rc}")
+        return out
+
+    def prefill_attention(self, q, cu_new, seq_lens, block_tables, sm_scale=None) -> np.ndarray:
+        """Causal attention of the appended chunk's query rows (q: fp16
+        [n_tokens][num_q_heads][128], sequence b owning rows cu_new[b]..)
+        over the cache after the append; fp64 [n_tokens][num_q_heads][128]."""
+        qb = np.ascontiguousarray(_u16(q))
+        n_tokens, num_q_heads, d = qb.shape
+        assert d == HEAD_DIM
+        cu = np.ascontiguousarray(cu_new, dtype=np.int32)
+        sl = np.ascontiguousarray(seq_lens, dtype=np.int32)
+        bt = np.ascontiguousarray(block_tables, dtype=np.int32)
+        if sm_scale is None:
+            sm_scale = 1.0 / np.sqrt(HEAD_DIM)
+        out = np.zeros((n_tokens, num_q_heads, HEAD_DIM), np.float64)
+        rc = lib().s4kv_ref_prefill_attention(
+            _p(self.pool), _p(self.res_k), _p(self.res_v), self.num_pages,
+            self.num_kv_heads, _p(qb), num_q_heads, _p(cu), _p(sl), _p(bt),
+            len(sl), bt.shape[1], float(sm_scale), _p(out))
+        if rc != 0:
+            raise ValueError(f"prefill_attention rc={rc}")
         return out
 
 

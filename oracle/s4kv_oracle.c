@@ -470,6 +470,77 @@ int s4kv_ref_decode_attention(const uint8_t *pool, const uint16_t *res_k,
     return REF_OK;
 }
 
+/* Causal attention of a chunk of new query tokens over the cache after the
+ * chunk was appended (the prefill / chunked-append side of the same cache).
+ * Sequence b owns query rows cu_new[b] .. cu_new[b+1]-1 of q (fp16
+ * [n_tokens][num_q_heads][128]); with n = cu_new[b+1] - cu_new[b] and
+ * L = seq_lens[b] (after the append), query row j of b sits at position
+ * L - n + j and attends to the cache's tokens 0 .. L - n + j: full pages
+ * dequantized, the partial last page from the fp16 residual, exactly the
+ * keys and values decode attention reads.  Per query head, fp64 logits
+ * sm_scale * q.k, a two-pass softmax and the weighted sum of values.
+ * out: fp64 [n_tokens][num_q_heads][128]; rows of no sequence are left
+ * untouched. */
+int s4kv_ref_prefill_attention(const uint8_t *pool, const uint16_t *res_k,
+                               const uint16_t *res_v, int num_pages,
+                               int num_kv_heads, const uint16_t *q,
+                               int num_q_heads, const int32_t *cu_new,
+                               const int32_t *seq_lens,
+                               const int32_t *block_tables, int batch,
+                               int max_pages_per_seq, double sm_scale,
+                               double *out) {
+    if (num_kv_heads <= 0 || num_q_heads % num_kv_heads != 0) return REF_BAD_ARG;
+    int G = num_q_heads / num_kv_heads;
+    for (int b = 0; b < batch; ++b) {
+        int L = seq_lens[b];
+        int n = cu_new[b + 1] - cu_new[b];
+        const int32_t *bt_row = block_tables + (long)b * max_pages_per_seq;
+        if (L < 0 || n < 0 || n > L || (L + PAGE - 1) / PAGE > max_pages_per_seq) return REF_BAD_ARG;
+        if (n == 0) continue;
+        for (int p = 0; p < L / PAGE; ++p)
+            if (bt_row[p] < 0 || bt_row[p] >= num_pages) return REF_BAD_SLOT;
+        size_t rows = (size_t)((L + PAGE - 1) / PAGE + 1) * PAGE;
+        float *K = (float *)malloc(sizeof(float) * rows * HEAD_DIM);
+        float *V = (float *)malloc(sizeof(float) * rows * HEAD_DIM);
+        double *w = (double *)malloc(sizeof(double) * (size_t)L);
+        if (!K || !V || !w) { free(K); free(V); free(w); return REF_BAD_ARG; }
+        for (int h = 0; h < num_kv_heads; ++h) {
+            sequence_kv(pool, res_k, res_v, num_kv_heads, bt_row, L, b, h, K, V);
+            for (int j = 0; j < n; ++j) {
+                int pos = L - n + j;
+                long row = cu_new[b] + j;
+                for (int g = 0; g < G; ++g) {
+                    int qh = h * G + g;
+                    const uint16_t *qv = q + (row * num_q_heads + qh) * HEAD_DIM;
+                    double *o = out + (row * num_q_heads + qh) * HEAD_DIM;
+                    double mx = -INFINITY;
+                    for (int t = 0; t <= pos; ++t) {
+                        double acc = 0.0;
+                        for (int c = 0; c < HEAD_DIM; ++c)
+                            acc += (double)s4kv_ref_half_to_float(qv[c]) * (double)K[(long)t * HEAD_DIM + c];
+                        w[t] = sm_scale * acc;
+                        if (w[t] > mx) mx = w[t];
+                    }
+                    double sum = 0.0;
+                    for (int t = 0; t <= pos; ++t) {
+                        w[t] = exp(w[t] - mx);
+                        sum += w[t];
+                    }
+                    for (int c = 0; c < HEAD_DIM; ++c) {
+                        double acc = 0.0;
+                        for (int t = 0; t <= pos; ++t) acc += w[t] * (double)V[(long)t * HEAD_DIM + c];
+                        o[c] = acc / sum;
+                    }
+                }
+            }
+        }
+        free(K);
+        free(V);
+        free(w);
+    }
+    return REF_OK;
+}
+
 /* Attention on unquantized fp16 K/V rows given directly ([n][128] per
  * (sequence, kv head)); used only to report the quantization error.
  * k, v: fp16 [total_tokens][num_kv_heads][128] with sequence b occupying

@@ -21,6 +21,10 @@ Which pin covers which oracle function:
                                    quantizer represents exactly; single key; uniform
                                    weights; page permutation and shared-prefix
                                    invariance; GQA identical queries; fp32 vs fp64
+  prefill_attention             : textbook causal softmax attention (numpy) on
+                                   inputs the quantizer represents exactly, per
+                                   query position; the chunk's last row equals
+                                   decode attention
 """
 import os
 from fractions import Fraction
@@ -476,3 +480,69 @@ def test_fp32_oracle_close_to_fp64(oracle_mod):
     ref = oracle_mod.attention_fp16(np.concatenate(k), np.concatenate(v), cu, 1, q)
     err = np.abs(o64 - ref).max()
     assert np.isfinite(err) and err < 1.0
+
+
+# ------------------------------------------------------------ prefill --
+
+def _grid_streams(rng, lens, H):
+    k, v = [], []
+    for L in lens:
+        npg = (L + PAGE - 1) // PAGE
+        kk = np.zeros((npg * PAGE, H, HD), np.float16)
+        vv = np.zeros((npg * PAGE, H, HD), np.float16)
+        for p in range(npg):
+            for h in range(H):
+                kk[p * PAGE:(p + 1) * PAGE, h] = _grid_page(rng, "key")[0]
+                vv[p * PAGE:(p + 1) * PAGE, h] = _grid_page(rng, "value")[0]
+        k.append(kk[:L])
+        v.append(vv[:L])
+    return k, v
+
+
+def test_prefill_matches_textbook_causal_attention_on_exact_grids(oracle_mod):
+    """A chunk of n new tokens appended to a context of L - n tokens: every
+    query row at position pos must equal plain softmax attention (numpy,
+    float64) over the original fp16 keys and values 0..pos.  On exact grids
+    the dequantized cache is the input itself, so this pins the causal
+    limit, the position of each chunk row, the GQA map and the page walk."""
+    rng = np.random.default_rng(31)
+    H, G = 2, 3
+    before = [21, 0, 32, 5]
+    after = [40, 17, 50, 37]
+    k, v = _grid_streams(rng, after, H)
+    bt, NP = _tables(rng, after)
+    c = oracle_mod.OracleCache(NP, H, len(after))
+    _append_all(oracle_mod, c, k, v, [0] * 4, before, bt)
+    _append_all(oracle_mod, c, k, v, before, after, bt)
+    n = np.array(after) - np.array(before)
+    cu = np.concatenate([[0], np.cumsum(n)]).astype(np.int32)
+    q = rng.standard_normal((int(cu[-1]), H * G, HD)).astype(np.float16)
+    out = c.prefill_attention(q, cu, np.array(after, np.int32), bt)
+    scale = 1 / np.sqrt(HD)
+    for b in range(4):
+        for j in range(n[b]):
+            pos = before[b] + j
+            row = cu[b] + j
+            for qh in range(H * G):
+                ref = _textbook_attention(q[row, qh], k[b][:pos + 1, qh // G], v[b][:pos + 1, qh // G], scale)
+                assert np.allclose(out[row, qh], ref, rtol=1e-12, atol=1e-12), (b, j, qh)
+
+
+def test_prefill_last_row_is_decode(oracle_mod):
+    """The last row of a chunk sits at position L - 1 and sees the whole
+    sequence: it must be exactly what decode attention gives for that query."""
+    rng = np.random.default_rng(32)
+    H, G = 2, 4
+    before = [30, 16, 1]
+    after = [47, 33, 20]
+    k, v = _rand_kv(rng, 3, H, after)
+    bt, NP = _tables(rng, after)
+    c = oracle_mod.OracleCache(NP, H, 3)
+    _append_all(oracle_mod, c, k, v, [0] * 3, after, bt)
+    n = np.array(after) - np.array(before)
+    cu = np.concatenate([[0], np.cumsum(n)]).astype(np.int32)
+    q = rng.standard_normal((int(cu[-1]), H * G, HD)).astype(np.float16)
+    out = c.prefill_attention(q, cu, np.array(after, np.int32), bt, sm_scale=0.07)
+    last = q[cu[1:] - 1]
+    dec = c.decode_attention(last, np.array(after, np.int32), bt, sm_scale=0.07)
+    assert np.array_equal(out[cu[1:] - 1], dec)
