@@ -218,6 +218,35 @@ S4KV_API int s4kv_decode_attention_noalloc(const s4kv_cache_t *cache, const void
                                            int max_pages_per_seq, float sm_scale,
                                            void *out, void *stream);
 
+/* Causal attention of a chunk of new query tokens over the cache (the
+ * prefill / chunked-append side of the same paged int4 cache; GQA map of
+ * "KV-Cache-Optimierung -- PagedAttention, quantisierter KV, Speculative
+ * Cache", "Begriffe auf dieser Seite"; dequantization of "S4 KV -- int4
+ * KV-Cache-Kompression fuer vLLM", "Funktionsweise" step 1).  Call it after
+ * s4kv_append has written the chunk (same cu_new, seq_lens, block_tables).
+ *  q       device fp16 [n_tokens][num_q_heads][128], 16-B aligned, token
+ *          major like the appended k and v: sequence b owns rows
+ *          cu_new[b] .. cu_new[b+1]-1.
+ *  cu_new, seq_lens (lengths AFTER the append), block_tables: as for
+ *          s4kv_append; n = cu_new[b+1] - cu_new[b] must not exceed
+ *          seq_lens[b] (else S4KV_EFLAG_SEQ_LEN and the sequence is skipped).
+ *  max_new_per_seq  host bound on any n (sizes the launch; rows beyond it
+ *          are not computed).
+ *  out     device fp16 [n_tokens][num_q_heads][128], 16-B aligned: row j of
+ *          sequence b (position L - n + j) gets softmax(sm_scale * q.K^T) V
+ *          over the cache's tokens 0 .. L - n + j; rows of no sequence are
+ *          left untouched.
+ * Runs on the tcgen05 tensor cores with the dequantized keys and values and
+ * the softmax weights as fp16 MMA operands (fp32 accumulation), so results
+ * agree with exact attention to about fp16 precision of those operands.
+ * Allocates nothing; needs about 205 KB of shared memory per CTA. */
+S4KV_API int s4kv_prefill_attention(const s4kv_cache_t *cache, const void *q,
+                                    int num_q_heads, int n_tokens,
+                                    const int32_t *cu_new, const int32_t *seq_lens,
+                                    const int32_t *block_tables, int batch,
+                                    int max_pages_per_seq, int max_new_per_seq,
+                                    float sm_scale, void *out, void *stream);
+
 /* Dequantize one physical page for all kv heads into natural order:
  * out_k, out_v device [num_kv_heads][16][128], fp32 if out_fp32 != 0
  * (x = code*scale + zero, exact product, one rounding) else fp16 (the fp32

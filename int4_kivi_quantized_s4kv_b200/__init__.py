@@ -45,6 +45,7 @@ _SIGS = {
     "s4kv_decode_workspace_size": ([_I, _I, ctypes.POINTER(_SZ)], _I),
     "s4kv_decode_attention": ([_CP, _P, _I, _P, _P, _I, _I, ctypes.c_float, _P, _P, _SZ, _P], _I),
     "s4kv_decode_attention_noalloc": ([_CP, _P, _I, _P, _P, _I, _I, ctypes.c_float, _P, _P], _I),
+    "s4kv_prefill_attention": ([_CP, _P, _I, _I, _P, _P, _P, _I, _I, _I, ctypes.c_float, _P, _P], _I),
     "s4kv_dequant_page": ([_CP, _I, _P, _P, _I, _P], _I),
     "s4kv_get_error": ([_CP, ctypes.POINTER(ctypes.c_uint32), _I, _P], _I),
 }
@@ -199,6 +200,24 @@ def s4kv_decode_attention_noalloc(cache: S4KVCache, q, seq_lens, block_tables, o
                                             block_tables.shape[1], float(sm_scale),
                                             _ptr(out, torch.float16, "out"), _stream(stream))
     _check(st, "s4kv_decode_attention_noalloc")
+
+
+def s4kv_prefill_attention(cache: S4KVCache, q, cu_new, seq_lens, block_tables, out,
+                           max_new_per_seq: int, sm_scale: float | None = None, stream=None):
+    """Causal attention of the appended chunk's query rows (q: fp16
+    [n_tokens][num_q_heads][128], sequence b owning rows cu_new[b]..) over the
+    cache after s4kv_append wrote the chunk; fills out [n_tokens][num_q_heads][128]."""
+    import torch
+    n_tokens, num_q_heads, _ = q.shape
+    if sm_scale is None:
+        sm_scale = HEAD_DIM ** -0.5
+    st = lib().s4kv_prefill_attention(cache.ref, _ptr(q, torch.float16, "q"), num_q_heads, n_tokens,
+                                     _ptr(cu_new, torch.int32, "cu_new"),
+                                     _ptr(seq_lens, torch.int32, "seq_lens"),
+                                     _ptr(block_tables, torch.int32, "block_tables"), seq_lens.shape[0],
+                                     block_tables.shape[1], int(max_new_per_seq), float(sm_scale),
+                                     _ptr(out, torch.float16, "out"), _stream(stream))
+    _check(st, "s4kv_prefill_attention")
 
 
 def s4kv_dequant_page(cache: S4KVCache, physical_page: int, out_k, out_v, out_fp32: bool = True,

@@ -215,6 +215,59 @@ int s4kv_decode_attention(const s4kv_cache_t *cache, const void *q, int num_q_he
   return S4KV_OK;
 }
 
+int s4kv_prefill_attention(const s4kv_cache_t *cache, const void *q, int num_q_heads, int n_tokens,
+                           const int32_t *cu_new, const int32_t *seq_lens, const int32_t *block_tables,
+                           int batch, int max_pages_per_seq, int max_new_per_seq, float sm_scale, void *out,
+                           void *stream) {
+  int rc = check_cache(cache);
+  if (rc != S4KV_OK) return rc;
+  rc = s4kv_check_model(cache->head_dim, cache->page_tokens, num_q_heads, cache->num_kv_heads);
+  if (rc != S4KV_OK) return rc;
+  if (n_tokens < 0 || batch < 0 || batch > cache->max_seqs || max_pages_per_seq <= 0) return S4KV_ERR_INVALID_ARG;
+  if (!(std::isfinite(sm_scale)) || sm_scale <= 0.0f) return S4KV_ERR_INVALID_ARG;
+  if (n_tokens == 0 || batch == 0) return S4KV_OK;
+  if (max_new_per_seq <= 0 || max_new_per_seq > n_tokens) return S4KV_ERR_INVALID_ARG;
+  if (!q || !cu_new || !seq_lens || !block_tables || !out) return S4KV_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(out, 16) || !aligned(cu_new, 4) || !aligned(seq_lens, 4) ||
+      !aligned(block_tables, 4))
+    return S4KV_ERR_INVALID_ARG;
+  const int group = num_q_heads / cache->num_kv_heads;
+  const long long tiles = (static_cast<long long>(max_new_per_seq) + (128 / group) - 1) / (128 / group);
+  if (tiles > 0x7FFFFFFF || batch > 65535 || cache->num_kv_heads > 65535) return S4KV_ERR_INVALID_ARG;
+  static std::once_flag prepared[kMaxDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return S4KV_ERR_CUDA;
+  }
+  cudaError_t perr = cudaSuccess;
+  std::call_once(prepared[dev], [&]() { perr = prepare_prefill_kernel(); });
+  if (perr != cudaSuccess) {
+    cudaGetLastError();
+    return S4KV_ERR_CUDA;
+  }
+  PrefillParams p;
+  p.pool = static_cast<const uint8_t *>(cache->pool);
+  p.res_k = static_cast<const __half *>(cache->res_k);
+  p.res_v = static_cast<const __half *>(cache->res_v);
+  p.q = static_cast<const __half *>(q);
+  p.out = static_cast<__half *>(out);
+  p.cu_new = cu_new;
+  p.seq_lens = seq_lens;
+  p.block_tables = block_tables;
+  p.err = cache->err_flag;
+  p.n_tokens = n_tokens;
+  p.num_q_heads = num_q_heads;
+  p.num_kv_heads = cache->num_kv_heads;
+  p.group = group;
+  p.max_pages = max_pages_per_seq;
+  p.num_pages = cache->num_pages;
+  p.scale_log2 = static_cast<float>(static_cast<double>(sm_scale) * 1.4426950408889634);
+  launch_prefill(p, batch, max_new_per_seq, static_cast<cudaStream_t>(stream));
+  if (cudaGetLastError() != cudaSuccess) return S4KV_ERR_CUDA;
+  return S4KV_OK;
+}
+
 int s4kv_dequant_page(const s4kv_cache_t *cache, int physical_page, void *out_k, void *out_v,
                       int out_fp32, void *stream) {
   int rc = check_cache(cache);

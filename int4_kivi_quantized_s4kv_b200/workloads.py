@@ -96,8 +96,23 @@ SPECS = {
         outlier_frac=0.02, outlier_scale=8.0,
         description="Llama-3.2-3B-shaped full decode step, 28 layers, batch 128, "
                     "contexts lognormal clipped to [128,16384]"),
+    # chunked prefill: the step appends a chunk of new tokens per sequence and
+    # runs causal attention of the chunk over the cache
+    "llama3.1-8b-prefill": Spec(
+        "llama3.1-8b-prefill", layers=1, batch=4, num_q_heads=32, num_kv_heads=8, seed=6,
+        ctx_kind="fixed", ctx_a=6144, step_new=(2048,),
+        key_lognormal_sigma=0.75,
+        description="Llama-3.1-8B-shaped layer, 4 sequences, a 2048-token chunk "
+                    "appended to a 6144-token context, causal attention of the chunk"),
+    "llama3-70b-prefill": Spec(
+        "llama3-70b-prefill", layers=1, batch=2, num_q_heads=64, num_kv_heads=8, seed=7,
+        ctx_kind="fixed", ctx_a=14336, step_new=(2048,),
+        outlier_frac=0.01, outlier_scale=10.0,
+        description="Llama-3-70B-shaped layer, 2 sequences, a 2048-token chunk "
+                    "appended to a 14336-token context, causal attention of the chunk"),
 }
 CONFIG_ORDER = ["tiny", "qwen2.5-7b", "llama3.1-8b", "llama3-70b", "llama3.2-3b-step"]
+PREFILL_ORDER = ["llama3.1-8b-prefill", "llama3-70b-prefill"]
 
 
 def scaled(spec: Spec, batch: int | None = None, ctx_scale: float | None = None,
@@ -327,3 +342,16 @@ def decode_bytes(spec: Spec, lens: np.ndarray | None = None, plan: PagePlan | No
             "algorithmic": pages_unique + residual + q,
             "logical": pages_logical + residual + q,
             "kv_tokens": int(lens.sum())}
+
+
+def chunk_queries_np(spec: Spec, layer: int, n_rows: int, step: int = 0) -> np.ndarray:
+    """fp16 q [n_rows][num_q_heads][128] for every appended token of a step."""
+    r = _rng(spec.seed, 606, layer, step)
+    return r.standard_normal((n_rows, spec.num_q_heads, HEAD_DIM), dtype=np.float32).astype(np.float16)
+
+
+def chunk_queries_torch(spec: Spec, layer: int, n_rows: int, device, step: int = 0):
+    import torch
+    g = _torch_gen(device, (spec.seed, 606, layer, step))
+    return torch.randn((n_rows, spec.num_q_heads, HEAD_DIM), generator=g,
+                       device=device, dtype=torch.float32).half()

@@ -97,6 +97,21 @@ def test_invalid_calls_rejected_before_launch(S):
     assert dec(ctypes.byref(c), P(fake), 8, P(fake), P(fake), 1, 1, -1.0, P(fake), P(fake), 1 << 30, st) == S.ERR_INVALID_ARG
     assert dec(ctypes.byref(c), None, 8, P(fake), P(fake), 1, 1, 0.088, P(fake), P(fake), 1 << 30, st) == S.ERR_INVALID_ARG
     assert dec(ctypes.byref(c), P(fake), 8, P(fake), P(fake), 0, 1, 0.088, P(fake), P(fake), 1 << 30, st) == S.OK
+    # prefill
+    pre = L.s4kv_prefill_attention
+    args = lambda **kw: dict(dict(cache=ctypes.byref(c), q=P(fake), hq=8, n=4, cu=P(fake), sl=P(fake), bt=P(fake),
+                                  batch=1, maxp=1, maxnew=4, scale=0.088, out=P(fake)), **kw)
+    call = lambda a: pre(a["cache"], a["q"], a["hq"], a["n"], a["cu"], a["sl"], a["bt"], a["batch"], a["maxp"],
+                         a["maxnew"], a["scale"], a["out"], st)
+    assert call(args(hq=18)) == S.ERR_UNSUPPORTED
+    assert call(args(cache=ctypes.byref(bad_dim))) == S.ERR_UNSUPPORTED
+    assert call(args(scale=float("nan"))) == S.ERR_INVALID_ARG
+    assert call(args(q=None)) == S.ERR_INVALID_ARG
+    assert call(args(out=P(fake + 8))) == S.ERR_INVALID_ARG
+    assert call(args(maxnew=0)) == S.ERR_INVALID_ARG
+    assert call(args(maxnew=5)) == S.ERR_INVALID_ARG  # more than n_tokens
+    assert call(args(batch=5)) == S.ERR_INVALID_ARG   # batch > max_seqs
+    assert call(args(n=0)) == S.OK and call(args(batch=0)) == S.OK  # nothing to do
     # dequant
     assert L.s4kv_dequant_page(ctypes.byref(c), 10, P(fake), P(fake), 1, st) == S.ERR_INVALID_ARG
     assert L.s4kv_dequant_page(ctypes.byref(c), -1, P(fake), P(fake), 1, st) == S.ERR_INVALID_ARG

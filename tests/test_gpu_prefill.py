@@ -1,0 +1,116 @@
+"""GPU parity of s4kv_prefill_attention (causal attention of an appended
+chunk over the int4 paged cache) against the fp64 oracle, through the C ABI.
+
+The cache is built on both sides from the same seeded fp16 inputs (context
+appended first, then the chunk) and must be bit-exact; the attention output
+must be within |gpu - oracle| <= 2e-3 + 1e-3 |oracle| element-wise.  The
+CUDA path feeds the tensor cores fp16 operands (dequantized keys and values,
+softmax weights), which that bound covers with margin.
+"""
+import numpy as np
+import pytest
+
+from helpers import assert_attention_close
+
+HD, PAGE = 128, 16
+
+pytestmark = pytest.mark.gpu
+
+
+class PrefillCase:
+    def __init__(self, seed, H, G, before, after, outliers=8, context_chunk=64):
+        import torch
+        import oracle
+        import int4_kivi_quantized_s4kv_b200 as S
+        rng = np.random.default_rng(seed)
+        self.S, self.H, self.G = S, H, G
+        self.before = np.array(before, np.int64)
+        self.after = np.array(after, np.int64)
+        B = len(after)
+        # keys with a few outlier channels per kv head, values plain N(0, 1)
+        scale = np.ones((H, HD))
+        for h in range(H):
+            scale[h, rng.choice(HD, outliers, replace=False)] = 10.0
+        self.k = [(rng.standard_normal((L, H, HD)) * scale).astype(np.float16) for L in after]
+        self.v = [rng.standard_normal((L, H, HD)).astype(np.float16) for L in after]
+        need = [(L + PAGE - 1) // PAGE for L in after]
+        NP = sum(need) + 5
+        perm = rng.permutation(NP).astype(np.int32)
+        self.bt = np.full((B, max(max(need), 1)), -1, np.int32)
+        c = 0
+        for b, m in enumerate(need):
+            self.bt[b, :m] = perm[c:c + m]
+            c += m
+        self.oc = oracle.OracleCache(NP, H, B)
+        self.gpu = S.S4KVCache(NP, H, B, device="cuda")
+        self.dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
+        self.bt_dev = self.dev(self.bt)
+        self._append(np.zeros(B, np.int64), self.before, context_chunk)
+        self.n = self.after - self.before
+        self.cu = np.concatenate([[0], np.cumsum(self.n)]).astype(np.int32)
+        self._append(self.before, self.after, None)
+        self.q = rng.standard_normal((int(self.cu[-1]), H * G, HD)).astype(np.float16)
+
+    def _append(self, before, after, chunk):
+        from helpers import append_batches
+        for k, v, sm, cu, sl, mx in append_batches(before, after, self.k, self.v, self.bt, chunk):
+            if mx == 0:
+                continue
+            assert self.oc.append(k, v, sm, cu, sl, self.bt) == 0
+            self.S.s4kv_append(self.gpu, self.dev(k), self.dev(v), self.dev(sm), self.dev(cu), self.dev(sl),
+                               self.bt_dev, mx)
+
+    def run(self, sm_scale=None):
+        import torch
+        qd = self.dev(self.q)
+        out = torch.full_like(qd, float("nan"))
+        self.S.s4kv_prefill_attention(self.gpu, qd, self.dev(self.cu), self.dev(self.after.astype(np.int32)),
+                                      self.bt_dev, out, int(max(self.n.max(), 1)), sm_scale)
+        torch.cuda.synchronize()
+        assert self.S.s4kv_get_error(self.gpu) == 0
+        got = out.float().cpu().numpy()
+        ref = self.oc.prefill_attention(self.q, self.cu, self.after.astype(np.int32), self.bt, sm_scale)
+        return got, ref
+
+
+@pytest.mark.parametrize("G", [4, 1, 3, 8])
+def test_prefill_matches_oracle(G):
+    # chunks from position 0, across page and key-tile boundaries, a long
+    # chunk spanning several query tiles, and a single new token
+    case = PrefillCase(40 + G, 2, G, before=[0, 100, 5, 250], after=[37, 164, 300, 251])
+    got, ref = case.run()
+    err = assert_attention_close(got, ref, f"prefill G={G}")
+    print(f"G={G} max abs err {err:.3g}")
+
+
+def test_prefill_odd_groups_and_empty_chunk():
+    # G = 7 (18-token query tiles, 126 rows) and G = 5; one sequence gets no
+    # new tokens, one chunk ends exactly on a page boundary
+    for G in (7, 5):
+        case = PrefillCase(50 + G, 1, G, before=[16, 40, 0], after=[16, 64, 129])
+        got, ref = case.run(sm_scale=0.05)
+        assert_attention_close(got, ref, f"prefill G={G}")
+
+
+def test_prefill_long_chunk_over_long_context():
+    # 512-token chunks over 1.5K-token contexts: many key tiles, lazy
+    # rescaling of the running output, sequence-level tiling of the grid
+    case = PrefillCase(60, 2, 8, before=[1536, 1000], after=[2048, 1512], context_chunk=512)
+    got, ref = case.run()
+    assert_attention_close(got, ref, "prefill long")
+
+
+def test_prefill_last_row_matches_decode():
+    # the chunk's last row sees the whole sequence, as decode does
+    import torch
+    case = PrefillCase(70, 2, 4, before=[10, 60], after=[75, 200])
+    got, ref = case.run()
+    last = case.cu[1:] - 1
+    S = case.S
+    qd = case.dev(case.q[last])
+    out = torch.empty_like(qd)
+    ws = S.decode_workspace(2, 2)
+    S.s4kv_decode_attention(case.gpu, qd, case.dev(case.after.astype(np.int32)), case.bt_dev, out, ws)
+    torch.cuda.synchronize()
+    assert_attention_close(out.float().cpu().numpy(), ref[last], "decode of the last rows")
+    assert_attention_close(got[last], ref[last], "prefill of the last rows")
