@@ -44,7 +44,7 @@ namespace s4kv {
 
 namespace {
 
-constexpr int kThreadsP = 128;
+constexpr int kThreadsP = 512;
 constexpr int kKeyTile = 128;                    // keys per tile (MMA N of S)
 constexpr int kPagesPerTile = kKeyTile / kPage;  // 8
 constexpr uint32_t kOpBytes = 128 * 128 * 2;     // one fp16 [128][128] operand
@@ -62,7 +62,8 @@ constexpr uint32_t kOffV = 3 * kOpBytes;
 constexpr uint32_t kOffP = 4 * kOpBytes;
 constexpr uint32_t kOffStage = 5 * kOpBytes;
 constexpr uint32_t kOffBar = kOffStage + 2 * kStageBytes;  // 4 mbarriers + tmem slot
-constexpr uint32_t kSmemBytes = kOffBar + 64 + 1024;      // + alignment slack
+constexpr uint32_t kOffRed = kOffBar + 64;                 // [4][128] fp32 row partials
+constexpr uint32_t kSmemBytes = kOffRed + 4 * 128 * 4 + 1024;  // + alignment slack
 
 __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity) {
   if (mbar_try_wait(bar, parity)) return true;
@@ -185,14 +186,15 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(const PrefillPara
   __syncthreads();
   if (tid == 0) fetch(0);
 
-  // ---- Q tile: row r = (token r / G, head r % G); rows >= rows are zero
+  // ---- Q tile: row r = (token r / G, head r % G); rows >= rows are zero.
+  // Four threads per row, four 16-byte chunks each.
   {
-    const int r = tid;
+    const int r = tid >> 2, cq = tid & 3;
     const int tl = r / G, g = r - tl * G;
     const uint4 *src = reinterpret_cast<const uint4 *>(
         p.q + (static_cast<long>(c_lo + t0 + tl) * p.num_q_heads + h * G + g) * kHeadDim);
-#pragma unroll 4
-    for (int c = 0; c < 16; ++c) {
+#pragma unroll
+    for (int c = 4 * cq; c < 4 * cq + 4; ++c) {
       uint4 v = make_uint4(0, 0, 0, 0);
       if (r < rows) v = __ldg(src + c);
       sts128(sQ + tc05::sw128_offset(r, 8 * c, 128), v);
@@ -202,19 +204,40 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(const PrefillPara
   tc05::fence_after_sync();
   const uint32_t tmem = lds32_at(tslot);
   const uint32_t tS = tmem, tO = tmem + 128;
-  const uint32_t lane_base = static_cast<uint32_t>(32 * warp) << 16;
 
-  // per-thread constants of the dequant mapping: word w = tid + 128 e of a
-  // code region; its lane index is tid / 4, its tile 4 e + tid % 4
-  const int wl = tid >> 2, wq = tid & 3;
-  const int dn = wl >> 2, di = wl & 3;
+  // ---- dequant mapping: 64 threads per page of the key tile; thread word
+  // w = widx + 64 e (e = 0..3) of a code region, i.e. MMA lane (w % 128) / 4
+  // and tile 4 (w / 128) + w % 4
+  const int dpage = tid >> 6, widx = tid & 63;
+  const int dq = widx & 3, dlane0 = widx >> 2;
+  // swizzled store offsets of this thread's words (they do not change from
+  // tile to tile): keys row 16 dpage + dn (and + 8 rows = + 1024 bytes),
+  // channels 32 di + 4 t; values rows cb, cb + 1, keys 16 dpage + 2 di (+ 8)
+  uint32_t kofs[4], vofs[4][4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const int lane = dlane0 + 16 * (e & 1), t = 4 * (e >> 1) + dq;
+    const int dn = lane >> 2, di = lane & 3;
+    kofs[e] = tc05::sw128_offset(dpage * 16 + dn, 32 * di + 4 * t, 128);
+    const int cb = 32 * (t >> 1) + 4 * dn + 2 * (t & 1);
+    const int key = dpage * 16 + 2 * di;
+    vofs[e][0] = tc05::sw128_offset(cb, key, 128);
+    vofs[e][1] = tc05::sw128_offset(cb + 1, key, 128);
+    vofs[e][2] = tc05::sw128_offset(cb, key + 8, 128);
+    vofs[e][3] = tc05::sw128_offset(cb + 1, key + 8, 128);
+  }
 
-  // softmax state of row tid
-  const int row = tid;
+  // ---- softmax mapping: warp w reads tensor-memory lanes 32 (w % 4) ..
+  // (row r = 32 (w % 4) + lane) and key columns 32 (w / 4) .. + 31
+  const int qd = warp & 3, cq = warp >> 2;
+  const int row = 32 * qd + (tid & 31);
+  const uint32_t lane_base = static_cast<uint32_t>(32 * qd) << 16;
   const bool row_ok = row < rows;
   const int pos_row = pos_first + (row_ok ? row / G : 0);
-  float ref = -INFINITY, lsum = 0.f;
+  float ref = -INFINITY;
+  float2 lsum = make_float2(0.f, 0.f);  // this thread's columns only
   const float sl2 = p.scale_log2;
+  float *red = reinterpret_cast<float *>(smem_raw + (base + kOffRed - raw));  // [4][128]
 
   bool failed = false;
   int kt = 0;
@@ -226,85 +249,59 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(const PrefillPara
       failed = true;
       break;
     }
-
-    // ---- dequantize key tile kt into sK and sV (V transposed)
     const uint32_t stg = stage0 + s * kStageBytes;
-#pragma unroll 1
-    for (int pl = 0; pl < kPagesPerTile; ++pl) {
-      const int pg = kt * kPagesPerTile + pl;
-      if (pg < nfull) {
-        const uint32_t blk = stg + pl * kBlockBytes;
+    const int pg = kt * kPagesPerTile + dpage;
+    const uint32_t blk = stg + dpage * kBlockBytes;
+    const int rres = (pg == nfull && pg < np) ? L - nfull * kPage : 0;  // residual rows of a partial page
+    const long res_base = (static_cast<long>(b) * H + h) * kPage * kHeadDim;
+
+    // ---- keys of tile kt -> sK (hi) and sKlo; S(kt-1) finished before the
+    // softmax of kt-1, so both are free
+    if (pg < nfull) {
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int t = 4 * e + wq;                 // MMA tile index of word w
-          const int w = tid + 128 * e;
-          // keys: tokens dn, dn + 8; channels c0 .. c0 + 3
-          {
-            uint32_t a0, a1, a2, a3;
-            unpack_codes(lds32_at(blk + kKCodeOff + 4 * w), a0, a1, a2, a3);
-            const int c0 = 32 * di + 4 * t;
-            const uint2 sc = lds64_at(blk + kKScaleOff + 2 * c0);
-            const uint32_t zslot = 16 * t + 2 * di;
-            const uint32_t z01 = lds32_at(blk + kKZeroOff + 2 * zslot);
-            const uint32_t z23 = lds32_at(blk + kKZeroOff + 2 * (zslot + 8));
-            const float2 s01 = __half22float2(u32_as_h2(sc.x)), s23 = __half22float2(u32_as_h2(sc.y));
-            const float2 zf01 = __half22float2(u32_as_h2(z01)), zf23 = __half22float2(u32_as_h2(z23));
-            uint32_t hi0, lo0, hi1, lo1, hi2, lo2, hi3, lo3;
-            split_key(a0, s01, zf01, hi0, lo0);
-            split_key(a1, s01, zf01, hi1, lo1);
-            split_key(a2, s23, zf23, hi2, lo2);
-            split_key(a3, s23, zf23, hi3, lo3);
-            const uint32_t r0 = static_cast<uint32_t>(pl * 16 + dn);
-            const uint32_t o0 = tc05::sw128_offset(r0, c0, 128);
-            const uint32_t o1 = tc05::sw128_offset(r0 + 8, c0, 128);
-            sts64(sK + o0, hi0, hi2);
-            sts64(sK + o1, hi1, hi3);
-            sts64(sKlo + o0, lo0, lo2);
-            sts64(sKlo + o1, lo1, lo3);
-          }
-          // values: channels cb, cb + 1; tokens 2 di, 2 di + 1 (+ 8)
-          {
-            uint32_t a0, a1, a2, a3;
-            unpack_codes(lds32_at(blk + kVCodeOff + 4 * w), a0, a1, a2, a3);
-            const int g = t >> 1;
-            const int cb = 32 * g + 4 * dn + 2 * (t & 1);
-            const uint32_t sv_lo = lds32_at(blk + kVScaleOff + 2 * (16 * g + 2 * di));
-            const uint32_t sv_hi = lds32_at(blk + kVScaleOff + 2 * (16 * g + 2 * di + 8));
-            const uint32_t zv_lo = lds32_at(blk + kVZeroOff + 2 * (16 * g + 2 * di));
-            const uint32_t zv_hi = lds32_at(blk + kVZeroOff + 2 * (16 * g + 2 * di + 8));
-            const int key = pl * 16 + 2 * di;
-            sts32(sV + tc05::sw128_offset(cb, key, 128), hfma2_u32(a0, sv_lo, zv_lo));
-            sts32(sV + tc05::sw128_offset(cb + 1, key, 128), hfma2_u32(a1, sv_lo, zv_lo));
-            sts32(sV + tc05::sw128_offset(cb, key + 8, 128), hfma2_u32(a2, sv_hi, zv_hi));
-            sts32(sV + tc05::sw128_offset(cb + 1, key + 8, 128), hfma2_u32(a3, sv_hi, zv_hi));
-          }
-        }
-      } else {
-        // the partial last page (fp16 residual rows < L % 16) or no page:
-        // copy the valid rows, zero the rest, so masked keys hold finite values
-        const int r = (pg == nfull && pg < np) ? L - nfull * kPage : 0;
-        const __half *rk = p.res_k + (static_cast<long>(b) * H + h) * kPage * kHeadDim;
-        const __half *rv = p.res_v + (static_cast<long>(b) * H + h) * kPage * kHeadDim;
-#pragma unroll 1
-        for (int e = tid; e < kPage * kHeadDim; e += kThreadsP) {
-          const int tk = e >> 7, c = e & 127;
-          uint16_t kb = 0, vb = 0;
-          if (tk < r) {
-            kb = __half_as_ushort(rk[tk * kHeadDim + c]);
-            vb = __half_as_ushort(rv[tk * kHeadDim + c]);
-          }
-          const uint32_t ko = tc05::sw128_offset(pl * 16 + tk, c, 128);
-          sts16(sK + ko, kb);
-          sts16(sKlo + ko, 0);
-          sts16(sV + tc05::sw128_offset(c, pl * 16 + tk, 128), vb);
-        }
+      for (int e = 0; e < 4; ++e) {
+        const int w = widx + 64 * e;
+        const int lane = dlane0 + 16 * (e & 1), t = 4 * (e >> 1) + dq;
+        const int dn = lane >> 2, di = lane & 3;
+        uint32_t a0, a1, a2, a3;
+        unpack_codes(lds32_at(blk + kKCodeOff + 4 * w), a0, a1, a2, a3);
+        const int c0 = 32 * di + 4 * t;
+        const uint2 sc = lds64_at(blk + kKScaleOff + 2 * c0);
+        const uint32_t zslot = 16 * t + 2 * di;
+        const uint32_t z01 = lds32_at(blk + kKZeroOff + 2 * zslot);
+        const uint32_t z23 = lds32_at(blk + kKZeroOff + 2 * (zslot + 8));
+        const float2 s01 = __half22float2(u32_as_h2(sc.x)), s23 = __half22float2(u32_as_h2(sc.y));
+        const float2 zf01 = __half22float2(u32_as_h2(z01)), zf23 = __half22float2(u32_as_h2(z23));
+        uint32_t hi0, lo0, hi1, lo1, hi2, lo2, hi3, lo3;
+        split_key(a0, s01, zf01, hi0, lo0);
+        split_key(a1, s01, zf01, hi1, lo1);
+        split_key(a2, s23, zf23, hi2, lo2);
+        split_key(a3, s23, zf23, hi3, lo3);
+        const uint32_t o0 = kofs[e], o1 = kofs[e] + 1024;
+        sts64(sK + o0, hi0, hi2);
+        sts64(sK + o1, hi1, hi3);
+        sts64(sKlo + o0, lo0, lo2);
+        sts64(sKlo + o1, lo1, lo3);
+      }
+    } else {
+      // the partial last page (fp16 residual rows < L % 16) or no page: copy
+      // the valid rows, zero the rest, so masked keys hold finite values
+      const __half *rk = p.res_k + res_base;
+#pragma unroll 4
+      for (int e = widx; e < kPage * kHeadDim / 2; e += 64) {
+        const int tk = e >> 6, c = 2 * (e & 63);
+        uint32_t kb = 0;
+        if (tk < rres) kb = *reinterpret_cast<const uint32_t *>(rk + tk * kHeadDim + c);
+        const uint32_t ko = tc05::sw128_offset(dpage * 16 + tk, c, 128);
+        sts32(sK + ko, kb);
+        sts32(sKlo + ko, 0u);
       }
     }
     fence_proxy_async();
     tc05::fence_before_sync();
     __syncthreads();
 
-    // ---- S = Q K_hi^T + Q K_lo^T
+    // ---- S = Q K_hi^T + Q K_lo^T (overlaps the value dequantization below)
     if (tid == 0) {
       tc05::fence_after_sync();
 #pragma unroll
@@ -320,6 +317,38 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(const PrefillPara
       }
       tc05::mma_commit(bar_s);
     }
+
+    // ---- values of tile kt -> sV (transposed), once O += P V of kt-1 is done
+    if (kt > 0 && !wait_bounded(bar_o, (kt - 1) & 1)) failed = true;
+    if (pg < nfull) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int w = widx + 64 * e;
+        const int lane = dlane0 + 16 * (e & 1), t = 4 * (e >> 1) + dq;
+        const int di = lane & 3;
+        uint32_t a0, a1, a2, a3;
+        unpack_codes(lds32_at(blk + kVCodeOff + 4 * w), a0, a1, a2, a3);
+        const int g = t >> 1;
+        const uint32_t sv_lo = lds32_at(blk + kVScaleOff + 2 * (16 * g + 2 * di));
+        const uint32_t sv_hi = lds32_at(blk + kVScaleOff + 2 * (16 * g + 2 * di + 8));
+        const uint32_t zv_lo = lds32_at(blk + kVZeroOff + 2 * (16 * g + 2 * di));
+        const uint32_t zv_hi = lds32_at(blk + kVZeroOff + 2 * (16 * g + 2 * di + 8));
+        sts32(sV + vofs[e][0], hfma2_u32(a0, sv_lo, zv_lo));
+        sts32(sV + vofs[e][1], hfma2_u32(a1, sv_lo, zv_lo));
+        sts32(sV + vofs[e][2], hfma2_u32(a2, sv_hi, zv_hi));
+        sts32(sV + vofs[e][3], hfma2_u32(a3, sv_hi, zv_hi));
+      }
+    } else {
+      const __half *rv = p.res_v + res_base;
+#pragma unroll 4
+      for (int e = widx; e < kPage * kHeadDim; e += 64) {
+        const int tk = e >> 7, c = e & 127;
+        uint16_t vb = 0;
+        if (tk < rres) vb = __half_as_ushort(rv[tk * kHeadDim + c]);
+        sts16(sV + tc05::sw128_offset(c, dpage * 16 + tk, 128), vb);
+      }
+    }
+    fence_proxy_async();
     if (!wait_bounded(bar_s, kt & 1)) failed = true;
     if (__syncthreads_or(failed)) {
       failed = true;
@@ -327,70 +356,81 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(const PrefillPara
     }
     tc05::fence_after_sync();
 
-    // ---- online softmax of row tid over this key tile
+    // ---- online softmax: row `row`, key columns 32 cq .. 32 cq + 31.  A key
+    // tile wholly before the tile's first query position needs no mask
+    // (rows past the tile's last row hold q = 0, so finite logits, and are
+    // never written out).
     {
-      const int key0 = kt * kKeyTile;
+      const int key0 = kt * kKeyTile + 32 * cq;
+      const bool full = kt * kKeyTile + kKeyTile - 1 <= pos_first;
+      uint32_t v[32];
+      tc05::tmem_ld32(tS + lane_base + 32 * cq, v);
+      tc05::tmem_wait_ld();
       float mx = -INFINITY;
-#pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        uint32_t v[32];
-        tc05::tmem_ld32(tS + lane_base + 32 * c, v);
-        tc05::tmem_wait_ld();
+      if (full) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) mx = fmaxf(mx, __uint_as_float(v[j]));
+        mx *= sl2;
+      } else {
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
-          const bool ok = row_ok && key0 + 32 * c + j <= pos_row;
-          if (ok) mx = fmaxf(mx, __uint_as_float(v[j]) * sl2);
+          const bool ok = row_ok && key0 + j <= pos_row;
+          const float x = ok ? __uint_as_float(v[j]) : -INFINITY;
+          v[j] = __float_as_uint(x);
+          mx = fmaxf(mx, x);
         }
+        mx *= sl2;
       }
-      // the reference moves only when this row's maximum passes it by > 8
+      red[cq * 128 + row] = mx;
+      __syncthreads();
+      mx = fmaxf(fmaxf(red[row], red[128 + row]), fmaxf(red[256 + row], red[384 + row]));
+      // the reference moves only when the row maximum passes it by > 8
       const bool move = mx > ref + kSlack;
       const float new_ref = move ? mx : ref;
       const float alpha = move ? fast_exp2(ref - new_ref) : 1.0f;  // 0 when ref was -inf
       if (__any_sync(0xFFFFFFFFu, move) && kt > 0) {
-        // rescale this warp's rows of O (tensor-memory load / store are warp-wide)
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          uint32_t v[32];
-          tc05::tmem_ld32(tO + lane_base + 32 * c, v);
-          tc05::tmem_wait_ld();
-#pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * alpha);
-          tc05::tmem_st32(tO + lane_base + 32 * c, v);
-        }
-        tc05::tmem_wait_st();
-      }
-      lsum *= alpha;
-      ref = new_ref;
-#pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        uint32_t v[32];
-        tc05::tmem_ld32(tS + lane_base + 32 * c, v);
+        // this warp's rows, columns 32 cq .. of O (warp-wide tensor-memory access)
+        uint32_t o[32];
+        tc05::tmem_ld32(tO + lane_base + 32 * cq, o);
         tc05::tmem_wait_ld();
-        uint32_t hp[16];
+        const float2 a2 = make_float2(alpha, alpha);
 #pragma unroll
         for (int j = 0; j < 32; j += 2) {
-          const bool ok0 = row_ok && key0 + 32 * c + j <= pos_row;
-          const bool ok1 = row_ok && key0 + 32 * c + j + 1 <= pos_row;
-          const float p0 = ok0 ? fast_exp2(fmaf(__uint_as_float(v[j]), sl2, -ref)) : 0.f;
-          const float p1 = ok1 ? fast_exp2(fmaf(__uint_as_float(v[j + 1]), sl2, -ref)) : 0.f;
-          const __half2 ph = __floats2half2_rn(p0, p1);
-          // the row sum takes the fp16 weights the MMA multiplies with, so a
-          // dominant key's value comes through exactly
-          const float2 pf = __half22float2(ph);
-          lsum += pf.x + pf.y;
-          hp[j >> 1] = h2_as_u32(ph);
+          const float2 r = mul2(make_float2(__uint_as_float(o[j]), __uint_as_float(o[j + 1])), a2);
+          o[j] = __float_as_uint(r.x);
+          o[j + 1] = __float_as_uint(r.y);
         }
-#pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4)
-          sts128(sP + tc05::sw128_offset(row, 32 * c + 8 * q4, 128),
-                 make_uint4(hp[4 * q4], hp[4 * q4 + 1], hp[4 * q4 + 2], hp[4 * q4 + 3]));
+        tc05::tmem_st32(tO + lane_base + 32 * cq, o);
+        tc05::tmem_wait_st();
       }
+      lsum = mul2(lsum, make_float2(alpha, alpha));
+      ref = new_ref;
+      // weights exp2(s * scale - ref); masked logits are -inf and give 0
+      // (ref is finite for every row with a valid key; a row without one has
+      // only masked logits, and its -inf reference is replaced by 0 so that
+      // no inf - inf appears)
+      const float nref = ref == -INFINITY ? 0.f : -ref;
+      const float2 sc = make_float2(sl2, sl2), nr = make_float2(nref, nref);
+      uint32_t hp[16];
+#pragma unroll
+      for (int j = 0; j < 32; j += 2) {
+        const float2 x = fma2(make_float2(__uint_as_float(v[j]), __uint_as_float(v[j + 1])), sc, nr);
+        const __half2 ph = __floats2half2_rn(fast_exp2(x.x), fast_exp2(x.y));
+        // the row sum takes the fp16 weights the MMA multiplies with, so a
+        // dominant key's value comes through exactly
+        lsum = add2(lsum, __half22float2(ph));
+        hp[j >> 1] = h2_as_u32(ph);
+      }
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4)
+        sts128(sP + tc05::sw128_offset(row, 32 * cq + 8 * q4, 128),
+               make_uint4(hp[4 * q4], hp[4 * q4 + 1], hp[4 * q4 + 2], hp[4 * q4 + 3]));
     }
     fence_proxy_async();
     tc05::fence_before_sync();
     __syncthreads();
 
-    // ---- O += P V
+    // ---- O += P V (overlaps the next tile's key dequantization)
     if (tid == 0) {
       tc05::fence_after_sync();
 #pragma unroll
@@ -401,33 +441,30 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(const PrefillPara
       }
       tc05::mma_commit(bar_o);
     }
-    if (!wait_bounded(bar_o, kt & 1)) failed = true;
-    if (__syncthreads_or(failed)) {
-      failed = true;
-      break;
-    }
-    tc05::fence_after_sync();
   }
+  if (!failed && !wait_bounded(bar_o, (n_ktiles - 1) & 1)) failed = true;
+  failed = __syncthreads_or(failed);
+  tc05::fence_after_sync();
 
   if (!failed) {
-    // ---- out = O / l for the valid rows
-    const float inv = row_ok && lsum > 0.f ? 1.0f / lsum : 0.f;
-    const int tl = row / G, g = row - (row / G) * G;
-    __half *dst = p.out + (static_cast<long>(c_lo + t0 + tl) * p.num_q_heads + h * G + g) * kHeadDim;
-#pragma unroll 1
-    for (int c = 0; c < 4; ++c) {
-      uint32_t v[32];
-      tc05::tmem_ld32(tO + lane_base + 32 * c, v);
-      tc05::tmem_wait_ld();
-      if (row_ok) {
-        uint32_t hv[16];
+    // ---- out = O / l: l is the sum of the four column quarters' partial sums
+    red[cq * 128 + row] = lsum.x + lsum.y;
+    __syncthreads();
+    const float l = (red[row] + red[128 + row]) + (red[256 + row] + red[384 + row]);
+    const float inv = row_ok && l > 0.f ? 1.0f / l : 0.f;
+    uint32_t v[32];
+    tc05::tmem_ld32(tO + lane_base + 32 * cq, v);
+    tc05::tmem_wait_ld();
+    if (row_ok) {
+      const int tl = row / G, g = row - tl * G;
+      __half *dst = p.out + (static_cast<long>(c_lo + t0 + tl) * p.num_q_heads + h * G + g) * kHeadDim + 32 * cq;
+      uint32_t hv[16];
 #pragma unroll
-        for (int j = 0; j < 32; j += 2)
-          hv[j >> 1] = h2_as_u32(__floats2half2_rn(__uint_as_float(v[j]) * inv, __uint_as_float(v[j + 1]) * inv));
-        uint4 *o4 = reinterpret_cast<uint4 *>(dst + 32 * c);
+      for (int j = 0; j < 32; j += 2)
+        hv[j >> 1] = h2_as_u32(__floats2half2_rn(__uint_as_float(v[j]) * inv, __uint_as_float(v[j + 1]) * inv));
+      uint4 *o4 = reinterpret_cast<uint4 *>(dst);
 #pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) o4[q4] = make_uint4(hv[4 * q4], hv[4 * q4 + 1], hv[4 * q4 + 2], hv[4 * q4 + 3]);
-      }
+      for (int q4 = 0; q4 < 4; ++q4) o4[q4] = make_uint4(hv[4 * q4], hv[4 * q4 + 1], hv[4 * q4 + 2], hv[4 * q4 + 3]);
     }
   } else if (tid == 0) {
     flag_error(p.err, S4KV_EFLAG_TIMEOUT);
