@@ -262,7 +262,7 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(const PrefillPara
       for (int e = 0; e < 4; ++e) {
         const int w = widx + 64 * e;
         const int lane = dlane0 + 16 * (e & 1), t = 4 * (e >> 1) + dq;
-        const int dn = lane >> 2, di = lane & 3;
+        const int di = lane & 3;
         uint32_t a0, a1, a2, a3;
         unpack_codes(lds32_at(blk + kKCodeOff + 4 * w), a0, a1, a2, a3);
         const int c0 = 32 * di + 4 * t;
