@@ -336,6 +336,71 @@ def config_dict(spec, extra=None):
     return d
 
 
+def measured_tensor_peak():
+    """Dense fp16/bf16 tensor-core TFLOP/s measured on this machine (fp16 and bf16
+    MMAs run at the same nominal rate)."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured (bf16 cuBLAS burst; fp16 has the same nominal rate)"
+    except (OSError, KeyError, ValueError):
+        return 1590.0, "fallback"
+
+
+def prefill_flops(spec, lens, new):
+    """Algorithmic FLOPs of causal chunk attention: every q head of row j
+    (position L - n + j) does 2 * 128 multiply-adds per key for q.k and as
+    many for p.v over keys 0 .. L - n + j."""
+    f = 0
+    for L, n in zip(lens.tolist(), new.tolist()):
+        f += spec.num_q_heads * 4 * 128 * (n * (L - n) + n * (n + 1) // 2)
+    return f
+
+
+def measure_prefill(device, steps: int, workload: str = "llama3.1-8b-prefill"):
+    """Chunked-prefill attention (the cache's prefill side) on its own
+    workload: the chunk is appended once, then s4kv_prefill_attention is timed
+    with CUDA events on the launching stream."""
+    import torch
+    spec = W.SPECS[workload]
+    wl = DeviceWorkload(spec, device)
+    S = wl.S
+    cache = wl.caches[0]
+    S.s4kv_append(cache, wl.k_new[0], wl.v_new[0], wl.step_slots, wl.step_cu, wl.seq_lens, wl.bt, wl.max_new)
+    rows = int(wl.new.sum())
+    q = W.chunk_queries_torch(spec, 0, rows, device)
+    out = torch.empty_like(q)
+
+    def run():
+        S.s4kv_prefill_attention(cache, q, wl.step_cu, wl.seq_lens, wl.bt, out, wl.max_new)
+
+    for _ in range(3):
+        run()
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(steps):
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        run()
+        b.record()
+        times.append((a, b))
+    torch.cuda.synchronize()
+    ms = sum(x.elapsed_time(y) for x, y in times) / len(times)
+    flags = S.s4kv_get_error(cache)
+    if flags:
+        raise RuntimeError(f"prefill device error flags {flags}")
+    flops = prefill_flops(spec, wl.lens, wl.new)
+    peak, kind = measured_tensor_peak()
+    achieved = flops / (ms * 1e-3) / 1e12
+    # the kernel issues three 128x128x128 GEMMs per (query tile, key tile):
+    # Q K_hi^T, Q K_lo^T (keys carried to ~22 bits) and P V
+    return {"workload": spec.name, "model_shape": spec.description, "launches": steps,
+            "avg_launch_ms": ms, "tflops": achieved, "query_tokens": rows,
+            "roofline": {"bound": "tensor", "kernel": "prefill_kernel", "achieved": achieved, "peak": peak,
+                         "peak_kind": kind, "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
+                         "flops_per_launch": flops, "mma_flops_per_launch": 1.5 * flops}}
+
+
 def run_reference(args, spec):
     world, rank, _ = _dist()
     if rank != 0:
@@ -377,6 +442,8 @@ def main(argv=None):
     ap.add_argument("--batch", type=int, default=None,
                     help="override the workload's batch (smaller profiling cases)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-prefill", action="store_true",
+                    help="skip the chunked-prefill attention measurement")
     args = ap.parse_args(argv)
     spec = W.SPECS[args.workload]
     if args.batch is not None:
@@ -470,6 +537,9 @@ def main(argv=None):
     value = aggregate_gbs(world, bytes_per_step, step_ms)
     achieved = decode_bytes_per_launch / (dec_avg_ms * 1e-3) / 1e9
     tokens = int(wl.new.sum())
+    prefill = None
+    if world == 1 and not args.no_prefill:
+        prefill = measure_prefill(device, max(3, min(args.steps, 20)))
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(spec)
@@ -500,11 +570,13 @@ def main(argv=None):
                          "bytes_per_launch": decode_bytes_per_launch, "avg_launch_ms": dec_avg_ms},
             "e2e": {"value": aggregate_gbs(world, bytes_per_step, e2e_ms), "unit": "GB/s",
                     "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-            "gpu_launches": args.steps * wl.launches_per_step(),
+            "gpu_launches": args.steps * wl.launches_per_step(),  # inside the timed region
             "clocks": clocks.summary(),
         }
         if cpu is not None:
             line["cpu_baseline"] = cpu
+        if prefill is not None:
+            line["next_rows"] = {"prefill": prefill}
         print(json.dumps(line), flush=True)
     if world > 1:
         torch.distributed.destroy_process_group()
