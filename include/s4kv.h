@@ -254,6 +254,62 @@ S4KV_API int s4kv_prefill_attention(const s4kv_cache_t *cache, const void *q,
 S4KV_API int s4kv_dequant_page(const s4kv_cache_t *cache, int physical_page,
                       void *out_k, void *out_v, int out_fp32, void *stream);
 
+/* Dequantize a list of physical pages at once: pages is a device int32
+ * [n] list (n <= 65535); page i goes to out_k / out_v slot i, each
+ * [n][num_kv_heads][16][128] in the format of s4kv_dequant_page.  A page id
+ * outside the pool sets S4KV_EFLAG_PAGE_RANGE and its slot is left as is. */
+S4KV_API int s4kv_dequant_pages(const s4kv_cache_t *cache, const int32_t *pages, int n,
+                                void *out_k, void *out_v, int out_fp32, void *stream);
+
+/* ---- page movement: swap-out / swap-in and copy-on-write fork.  A paged
+ * cache allocates pages on demand, lets sequences share them through their
+ * page tables and copies a page only when it is written ("KV-Cache und
+ * PagedAttention: Warum Ihr LLM-Server langsamer wird", "Wie PagedAttention
+ * das loest").  A page RECORD is all kv heads' blocks of one physical page:
+ * num_kv_heads * 2816 contiguous bytes, the unit these calls move.  All page
+ * and row lists are device int32 arrays; an id out of range sets
+ * S4KV_EFLAG_PAGE_RANGE (rows: S4KV_EFLAG_SLOT) and that item is skipped.
+ * Every call is asynchronous on `stream`. */
+
+/* Bytes of one page record (num_kv_heads * 2816). */
+S4KV_API int s4kv_page_record_bytes(int num_kv_heads, size_t *bytes);
+
+/* dst (device, 16-B aligned, [n][num_kv_heads][2816]) slot i = page record
+ * pages[i]. */
+S4KV_API int s4kv_gather_pages(const s4kv_cache_t *cache, const int32_t *pages, int n,
+                               void *dst, void *stream);
+
+/* Page record pages[i] = src slot i (src: device, 16-B aligned).  The pages
+ * must be distinct. */
+S4KV_API int s4kv_scatter_pages(const s4kv_cache_t *cache, const int32_t *pages, int n,
+                                const void *src, void *stream);
+
+/* Page record dst_pages[i] = page record src_pages[i], inside the pool (the
+ * copy-on-write copy of a shared full page).  No dst page may appear among
+ * the src pages or twice among the dst pages. */
+S4KV_API int s4kv_copy_pages(const s4kv_cache_t *cache, const int32_t *src_pages,
+                             const int32_t *dst_pages, int n, void *stream);
+
+/* Residual rows (the fp16 keys and values of the partial last page, all kv
+ * heads) of batch row src_rows[i] copied to batch row dst_rows[i]: the fork
+ * of a sequence whose last page is shared and partial.  The full pages are
+ * shared by pointing the new row's page table at them; the next page the
+ * fork fills must be a page of its own.  No dst row may be a src row. */
+S4KV_API int s4kv_fork_residual(const s4kv_cache_t *cache, const int32_t *src_rows,
+                                const int32_t *dst_rows, int n, void *stream);
+
+/* Swap-out: s4kv_gather_pages into `staging` (device, n records), then one
+ * device-to-host copy of the n records into host_dst (page-locked host
+ * memory for an asynchronous copy). */
+S4KV_API int s4kv_swap_out(const s4kv_cache_t *cache, const int32_t *pages, int n,
+                           void *staging, void *host_dst, void *stream);
+
+/* Swap-in: one host-to-device copy of n records from host_src into
+ * `staging`, then s4kv_scatter_pages into `pages` (any free pages: the
+ * caller points the sequence's page table at them). */
+S4KV_API int s4kv_swap_in(const s4kv_cache_t *cache, const int32_t *pages, int n,
+                          void *staging, const void *host_src, void *stream);
+
 /* Synchronize `stream`, read the cache's err_flag into *flags and clear it
  * when `clear` != 0.  Returns S4KV_ERR_DEVICE_CHECK when bits were set. */
 S4KV_API int s4kv_get_error(const s4kv_cache_t *cache, uint32_t *flags, int clear,

@@ -47,6 +47,14 @@ _SIGS = {
     "s4kv_decode_attention_noalloc": ([_CP, _P, _I, _P, _P, _I, _I, ctypes.c_float, _P, _P], _I),
     "s4kv_prefill_attention": ([_CP, _P, _I, _I, _P, _P, _P, _I, _I, _I, ctypes.c_float, _P, _P], _I),
     "s4kv_dequant_page": ([_CP, _I, _P, _P, _I, _P], _I),
+    "s4kv_dequant_pages": ([_CP, _P, _I, _P, _P, _I, _P], _I),
+    "s4kv_page_record_bytes": ([_I, ctypes.POINTER(_SZ)], _I),
+    "s4kv_gather_pages": ([_CP, _P, _I, _P, _P], _I),
+    "s4kv_scatter_pages": ([_CP, _P, _I, _P, _P], _I),
+    "s4kv_copy_pages": ([_CP, _P, _P, _I, _P], _I),
+    "s4kv_fork_residual": ([_CP, _P, _P, _I, _P], _I),
+    "s4kv_swap_out": ([_CP, _P, _I, _P, _P, _P], _I),
+    "s4kv_swap_in": ([_CP, _P, _I, _P, _P, _P], _I),
     "s4kv_get_error": ([_CP, ctypes.POINTER(ctypes.c_uint32), _I, _P], _I),
 }
 EXPORTED = tuple(_SIGS)
@@ -225,6 +233,65 @@ def s4kv_dequant_page(cache: S4KVCache, physical_page: int, out_k, out_v, out_fp
     st = lib().s4kv_dequant_page(cache.ref, int(physical_page), _ptr(out_k), _ptr(out_v),
                                 1 if out_fp32 else 0, _stream(stream))
     _check(st, "s4kv_dequant_page")
+
+
+def s4kv_dequant_pages(cache: S4KVCache, pages, out_k, out_v, out_fp32: bool = True, stream=None):
+    import torch
+    st = lib().s4kv_dequant_pages(cache.ref, _ptr(pages, torch.int32, "pages"), pages.numel(), _ptr(out_k),
+                                 _ptr(out_v), 1 if out_fp32 else 0, _stream(stream))
+    _check(st, "s4kv_dequant_pages")
+
+
+def s4kv_page_record_bytes(num_kv_heads: int) -> int:
+    n = _SZ(0)
+    _check(lib().s4kv_page_record_bytes(num_kv_heads, ctypes.byref(n)), "s4kv_page_record_bytes")
+    return n.value
+
+
+def s4kv_gather_pages(cache: S4KVCache, pages, dst, stream=None):
+    import torch
+    st = lib().s4kv_gather_pages(cache.ref, _ptr(pages, torch.int32, "pages"), pages.numel(),
+                                _ptr(dst, torch.uint8, "dst"), _stream(stream))
+    _check(st, "s4kv_gather_pages")
+
+
+def s4kv_scatter_pages(cache: S4KVCache, pages, src, stream=None):
+    import torch
+    st = lib().s4kv_scatter_pages(cache.ref, _ptr(pages, torch.int32, "pages"), pages.numel(),
+                                 _ptr(src, torch.uint8, "src"), _stream(stream))
+    _check(st, "s4kv_scatter_pages")
+
+
+def s4kv_copy_pages(cache: S4KVCache, src_pages, dst_pages, stream=None):
+    import torch
+    st = lib().s4kv_copy_pages(cache.ref, _ptr(src_pages, torch.int32, "src_pages"),
+                              _ptr(dst_pages, torch.int32, "dst_pages"), src_pages.numel(), _stream(stream))
+    _check(st, "s4kv_copy_pages")
+
+
+def s4kv_fork_residual(cache: S4KVCache, src_rows, dst_rows, stream=None):
+    import torch
+    st = lib().s4kv_fork_residual(cache.ref, _ptr(src_rows, torch.int32, "src_rows"),
+                                 _ptr(dst_rows, torch.int32, "dst_rows"), src_rows.numel(), _stream(stream))
+    _check(st, "s4kv_fork_residual")
+
+
+def s4kv_swap_out(cache: S4KVCache, pages, staging, host_dst, stream=None):
+    """Gather the pages' records into `staging` (device) and copy them to
+    `host_dst` (pinned host uint8 tensor of the same size)."""
+    import torch
+    st = lib().s4kv_swap_out(cache.ref, _ptr(pages, torch.int32, "pages"), pages.numel(),
+                            _ptr(staging, torch.uint8, "staging"), ctypes.c_void_p(host_dst.data_ptr()),
+                            _stream(stream))
+    _check(st, "s4kv_swap_out")
+
+
+def s4kv_swap_in(cache: S4KVCache, pages, staging, host_src, stream=None):
+    import torch
+    st = lib().s4kv_swap_in(cache.ref, _ptr(pages, torch.int32, "pages"), pages.numel(),
+                           _ptr(staging, torch.uint8, "staging"), ctypes.c_void_p(host_src.data_ptr()),
+                           _stream(stream))
+    _check(st, "s4kv_swap_in")
 
 
 def s4kv_get_error(cache: S4KVCache, clear: bool = True, stream=None) -> int:

@@ -89,6 +89,25 @@ WsLayout ws_layout(int batch, int num_kv_heads, int num_workers) {
   return w;
 }
 
+int launch_records(const uint8_t *src, uint8_t *dst, const int32_t *src_idx, const int32_t *dst_idx,
+                   long long rec_bytes, int n, int src_limit, int dst_limit, uint32_t *err, uint32_t err_bit,
+                   void *stream) {
+  MoveParams p;
+  p.src_base = src;
+  p.dst_base = dst;
+  p.src_idx = src_idx;
+  p.dst_idx = dst_idx;
+  p.err = err;
+  p.rec_bytes = rec_bytes;
+  p.n = n;
+  p.src_limit = src_limit;
+  p.dst_limit = dst_limit;
+  p.err_bit = err_bit;
+  launch_move(p, static_cast<cudaStream_t>(stream));
+  if (cudaGetLastError() != cudaSuccess) return S4KV_ERR_CUDA;
+  return S4KV_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -278,12 +297,125 @@ int s4kv_dequant_page(const s4kv_cache_t *cache, int physical_page, void *out_k,
   p.pool = static_cast<const uint8_t *>(cache->pool);
   p.out_k = out_k;
   p.out_v = out_v;
+  p.pages = nullptr;
+  p.err = cache->err_flag;
   p.physical_page = physical_page;
+  p.n_pages = 1;
+  p.num_pages = cache->num_pages;
   p.num_kv_heads = cache->num_kv_heads;
   p.out_fp32 = out_fp32 ? 1 : 0;
   launch_dequant(p, static_cast<cudaStream_t>(stream));
   if (cudaGetLastError() != cudaSuccess) return S4KV_ERR_CUDA;
   return S4KV_OK;
+}
+
+int s4kv_dequant_pages(const s4kv_cache_t *cache, const int32_t *pages, int n, void *out_k, void *out_v,
+                       int out_fp32, void *stream) {
+  int rc = check_cache(cache);
+  if (rc != S4KV_OK) return rc;
+  if (n < 0 || n > 65535) return S4KV_ERR_INVALID_ARG;
+  if (n == 0) return S4KV_OK;
+  if (!pages || !out_k || !out_v || !aligned(pages, 4) || !aligned(out_k, 16) || !aligned(out_v, 16))
+    return S4KV_ERR_INVALID_ARG;
+  DequantParams p;
+  p.pool = static_cast<const uint8_t *>(cache->pool);
+  p.out_k = out_k;
+  p.out_v = out_v;
+  p.pages = pages;
+  p.err = cache->err_flag;
+  p.physical_page = 0;
+  p.n_pages = n;
+  p.num_pages = cache->num_pages;
+  p.num_kv_heads = cache->num_kv_heads;
+  p.out_fp32 = out_fp32 ? 1 : 0;
+  launch_dequant(p, static_cast<cudaStream_t>(stream));
+  if (cudaGetLastError() != cudaSuccess) return S4KV_ERR_CUDA;
+  return S4KV_OK;
+}
+
+int s4kv_page_record_bytes(int num_kv_heads, size_t *bytes) {
+  if (num_kv_heads <= 0 || bytes == nullptr) return S4KV_ERR_INVALID_ARG;
+  *bytes = static_cast<size_t>(num_kv_heads) * S4KV_BLOCK_BYTES;
+  return S4KV_OK;
+}
+
+int s4kv_gather_pages(const s4kv_cache_t *cache, const int32_t *pages, int n, void *dst, void *stream) {
+  int rc = check_cache(cache);
+  if (rc != S4KV_OK) return rc;
+  if (n < 0) return S4KV_ERR_INVALID_ARG;
+  if (n == 0) return S4KV_OK;
+  if (!pages || !dst || !aligned(pages, 4) || !aligned(dst, 16)) return S4KV_ERR_INVALID_ARG;
+  return launch_records(static_cast<const uint8_t *>(cache->pool), static_cast<uint8_t *>(dst), pages, nullptr,
+                        static_cast<long long>(cache->num_kv_heads) * S4KV_BLOCK_BYTES, n, cache->num_pages, n,
+                        cache->err_flag, S4KV_EFLAG_PAGE_RANGE, stream);
+}
+
+int s4kv_scatter_pages(const s4kv_cache_t *cache, const int32_t *pages, int n, const void *src, void *stream) {
+  int rc = check_cache(cache);
+  if (rc != S4KV_OK) return rc;
+  if (n < 0) return S4KV_ERR_INVALID_ARG;
+  if (n == 0) return S4KV_OK;
+  if (!pages || !src || !aligned(pages, 4) || !aligned(src, 16)) return S4KV_ERR_INVALID_ARG;
+  return launch_records(static_cast<const uint8_t *>(src), static_cast<uint8_t *>(cache->pool), nullptr, pages,
+                        static_cast<long long>(cache->num_kv_heads) * S4KV_BLOCK_BYTES, n, n, cache->num_pages,
+                        cache->err_flag, S4KV_EFLAG_PAGE_RANGE, stream);
+}
+
+int s4kv_copy_pages(const s4kv_cache_t *cache, const int32_t *src_pages, const int32_t *dst_pages, int n,
+                    void *stream) {
+  int rc = check_cache(cache);
+  if (rc != S4KV_OK) return rc;
+  if (n < 0) return S4KV_ERR_INVALID_ARG;
+  if (n == 0) return S4KV_OK;
+  if (!src_pages || !dst_pages || !aligned(src_pages, 4) || !aligned(dst_pages, 4)) return S4KV_ERR_INVALID_ARG;
+  return launch_records(static_cast<const uint8_t *>(cache->pool), static_cast<uint8_t *>(cache->pool), src_pages,
+                        dst_pages, static_cast<long long>(cache->num_kv_heads) * S4KV_BLOCK_BYTES, n,
+                        cache->num_pages, cache->num_pages, cache->err_flag, S4KV_EFLAG_PAGE_RANGE, stream);
+}
+
+int s4kv_fork_residual(const s4kv_cache_t *cache, const int32_t *src_rows, const int32_t *dst_rows, int n,
+                       void *stream) {
+  int rc = check_cache(cache);
+  if (rc != S4KV_OK) return rc;
+  if (n < 0) return S4KV_ERR_INVALID_ARG;
+  if (n == 0) return S4KV_OK;
+  if (!src_rows || !dst_rows || !aligned(src_rows, 4) || !aligned(dst_rows, 4)) return S4KV_ERR_INVALID_ARG;
+  const long long rec = static_cast<long long>(cache->num_kv_heads) * S4KV_PAGE_TOKENS * S4KV_HEAD_DIM * 2;
+  rc = launch_records(static_cast<const uint8_t *>(cache->res_k), static_cast<uint8_t *>(cache->res_k), src_rows,
+                      dst_rows, rec, n, cache->max_seqs, cache->max_seqs, cache->err_flag, S4KV_EFLAG_SLOT, stream);
+  if (rc != S4KV_OK) return rc;
+  return launch_records(static_cast<const uint8_t *>(cache->res_v), static_cast<uint8_t *>(cache->res_v), src_rows,
+                        dst_rows, rec, n, cache->max_seqs, cache->max_seqs, cache->err_flag, S4KV_EFLAG_SLOT, stream);
+}
+
+int s4kv_swap_out(const s4kv_cache_t *cache, const int32_t *pages, int n, void *staging, void *host_dst,
+                  void *stream) {
+  int rc = s4kv_gather_pages(cache, pages, n, staging, stream);
+  if (rc != S4KV_OK || n == 0) return rc;
+  if (host_dst == nullptr) return S4KV_ERR_INVALID_ARG;
+  const size_t bytes = static_cast<size_t>(n) * cache->num_kv_heads * S4KV_BLOCK_BYTES;
+  if (cudaMemcpyAsync(host_dst, staging, bytes, cudaMemcpyDeviceToHost, static_cast<cudaStream_t>(stream)) !=
+      cudaSuccess) {
+    cudaGetLastError();
+    return S4KV_ERR_CUDA;
+  }
+  return S4KV_OK;
+}
+
+int s4kv_swap_in(const s4kv_cache_t *cache, const int32_t *pages, int n, void *staging, const void *host_src,
+                 void *stream) {
+  int rc = check_cache(cache);
+  if (rc != S4KV_OK) return rc;
+  if (n < 0) return S4KV_ERR_INVALID_ARG;
+  if (n == 0) return S4KV_OK;
+  if (host_src == nullptr || staging == nullptr || !aligned(staging, 16)) return S4KV_ERR_INVALID_ARG;
+  const size_t bytes = static_cast<size_t>(n) * cache->num_kv_heads * S4KV_BLOCK_BYTES;
+  if (cudaMemcpyAsync(staging, host_src, bytes, cudaMemcpyHostToDevice, static_cast<cudaStream_t>(stream)) !=
+      cudaSuccess) {
+    cudaGetLastError();
+    return S4KV_ERR_CUDA;
+  }
+  return s4kv_scatter_pages(cache, pages, n, staging, stream);
 }
 
 int s4kv_get_error(const s4kv_cache_t *cache, uint32_t *flags, int clear, void *stream) {

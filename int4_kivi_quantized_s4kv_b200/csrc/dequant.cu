@@ -1,5 +1,6 @@
-// s4kv_dequant_page device side: one physical page, all kv heads, back to
-// natural [token][channel] order.  x = code * scale + zero in fp32 (the
+// s4kv_dequant_page / s4kv_dequant_pages device side: physical pages, all kv
+// heads, back to natural [token][channel] order (page i of a list goes to
+// output slot i).  x = code * scale + zero in fp32 (the
 // product of a 4-bit code and an fp16 scale is exact, so this is a single
 // rounding); the fp16 output is that fp32 value rounded to nearest even.
 #include "kernels.cuh"
@@ -14,7 +15,16 @@ __device__ __forceinline__ uint32_t code_at(const uint8_t *region, int word, int
 __global__ void __launch_bounds__(128) dequant_kernel(const DequantParams p) {
   const int h = blockIdx.x;
   const int c = threadIdx.x;  // channel
-  const uint8_t *blk = p.pool + (static_cast<long>(p.physical_page) * p.num_kv_heads + h) * kBlockBytes;
+  const int slot = blockIdx.y;
+  int page = p.physical_page;
+  if (p.pages != nullptr) {
+    page = __ldg(p.pages + slot);
+    if (static_cast<unsigned>(page) >= static_cast<unsigned>(p.num_pages)) {
+      if (c == 0) flag_error(p.err, S4KV_EFLAG_PAGE_RANGE);
+      return;
+    }
+  }
+  const uint8_t *blk = p.pool + (static_cast<long>(page) * p.num_kv_heads + h) * kBlockBytes;
   const float ks = __half2float(reinterpret_cast<const __half *>(blk + kKScaleOff)[c]);
   const int zslot = 16 * ((c & 31) >> 2) + 2 * (c >> 5) + (c & 1) + 8 * ((c & 3) >> 1);
   const float kz = __half2float(reinterpret_cast<const __half *>(blk + kKZeroOff)[zslot]);
@@ -35,7 +45,7 @@ __global__ void __launch_bounds__(128) dequant_kernel(const DequantParams p) {
     const float vz = __half2float(reinterpret_cast<const __half *>(blk + kVZeroOff)[g * kPage + t]);
     const float kx = __fadd_rn(__fmul_rn(kcode, ks), kz);
     const float vx = __fadd_rn(__fmul_rn(vcode, vs), vz);
-    const long o = (static_cast<long>(h) * kPage + t) * kHeadDim + c;
+    const long o = ((static_cast<long>(slot) * p.num_kv_heads + h) * kPage + t) * kHeadDim + c;
     if (p.out_fp32) {
       static_cast<float *>(p.out_k)[o] = kx;
       static_cast<float *>(p.out_v)[o] = vx;
@@ -47,7 +57,7 @@ __global__ void __launch_bounds__(128) dequant_kernel(const DequantParams p) {
 }
 
 void launch_dequant(const DequantParams &p, cudaStream_t stream) {
-  dequant_kernel<<<p.num_kv_heads, 128, 0, stream>>>(p);
+  dequant_kernel<<<dim3(p.num_kv_heads, p.n_pages), 128, 0, stream>>>(p);
 }
 
 }  // namespace s4kv

@@ -29,9 +29,30 @@ struct DequantParams {
   const uint8_t *pool;
   void *out_k;
   void *out_v;
+  const int32_t *pages;  // device page list, or nullptr: the one physical_page
+  uint32_t *err;
   int physical_page;
+  int n_pages;
+  int num_pages;
   int num_kv_heads;
   int out_fp32;
+};
+
+// Copy of whole records: item i copies rec_bytes from
+// src_base + (src_idx ? src_idx[i] : i) * rec_bytes to
+// dst_base + (dst_idx ? dst_idx[i] : i) * rec_bytes.  An index outside
+// [0, src_limit) / [0, dst_limit) sets err_bit and the item is skipped.
+struct MoveParams {
+  const uint8_t *src_base;
+  uint8_t *dst_base;
+  const int32_t *src_idx;
+  const int32_t *dst_idx;
+  uint32_t *err;
+  long long rec_bytes;  // a multiple of 16
+  int n;
+  int src_limit;
+  int dst_limit;
+  uint32_t err_bit;
 };
 
 struct DecodeParams {
@@ -77,6 +98,7 @@ struct PrefillParams {
 
 void launch_append(const AppendParams &p, int batch, int max_new, cudaStream_t stream);
 void launch_dequant(const DequantParams &p, cudaStream_t stream);
+void launch_move(const MoveParams &p, cudaStream_t stream);
 void launch_decode(const DecodeParams &p, int num_ctas, cudaStream_t stream);
 int decode_ctas_per_sm();
 int decode_warps_per_cta();

@@ -72,6 +72,14 @@ def lib():
         L.s4kv_ref_attention_fp16.argtypes = [P, P, P, i32, P, i32, i32, f64, P]
         L.s4kv_ref_prefill_attention.argtypes = [P, P, P, i32, i32, P, i32, P, P, P, i32, i32, f64, P]
         L.s4kv_ref_prefill_attention.restype = i32
+        L.s4kv_ref_gather_pages.argtypes = [P, i32, i32, P, i32, P]
+        L.s4kv_ref_gather_pages.restype = i32
+        L.s4kv_ref_scatter_pages.argtypes = [P, i32, i32, P, i32, P]
+        L.s4kv_ref_scatter_pages.restype = i32
+        L.s4kv_ref_copy_pages.argtypes = [P, i32, i32, P, P, i32]
+        L.s4kv_ref_copy_pages.restype = i32
+        L.s4kv_ref_fork_residual.argtypes = [P, P, i32, i32, P, P, i32]
+        L.s4kv_ref_fork_residual.restype = i32
         L.s4kv_ref_attention_fp16.restype = i32
         _lib = L
         del i64
@@ -221,6 +229,37 @@ class OracleCache:
         if rc != 0:
             raise ValueError(f"decode_attention rc={rc}")
         return out
+
+    def gather_pages(self, pages) -> np.ndarray:
+        """Page records of the listed physical pages: u8 [n][kv_heads][2816]."""
+        pg = np.ascontiguousarray(pages, dtype=np.int32)
+        out = np.zeros((len(pg), self.num_kv_heads, BLOCK_BYTES), np.uint8)
+        rc = lib().s4kv_ref_gather_pages(_p(self.pool), self.num_pages, self.num_kv_heads, _p(pg), len(pg), _p(out))
+        if rc != 0:
+            raise ValueError(f"gather_pages rc={rc}")
+        return out
+
+    def scatter_pages(self, pages, records) -> None:
+        pg = np.ascontiguousarray(pages, dtype=np.int32)
+        rec = np.ascontiguousarray(records, dtype=np.uint8)
+        rc = lib().s4kv_ref_scatter_pages(_p(self.pool), self.num_pages, self.num_kv_heads, _p(pg), len(pg), _p(rec))
+        if rc != 0:
+            raise ValueError(f"scatter_pages rc={rc}")
+
+    def copy_pages(self, src_pages, dst_pages) -> None:
+        s_ = np.ascontiguousarray(src_pages, dtype=np.int32)
+        d_ = np.ascontiguousarray(dst_pages, dtype=np.int32)
+        rc = lib().s4kv_ref_copy_pages(_p(self.pool), self.num_pages, self.num_kv_heads, _p(s_), _p(d_), len(s_))
+        if rc != 0:
+            raise ValueError(f"copy_pages rc={rc}")
+
+    def fork_residual(self, src_rows, dst_rows) -> None:
+        s_ = np.ascontiguousarray(src_rows, dtype=np.int32)
+        d_ = np.ascontiguousarray(dst_rows, dtype=np.int32)
+        rc = lib().s4kv_ref_fork_residual(_p(self.res_k), _p(self.res_v), self.max_seqs, self.num_kv_heads,
+                                         _p(s_), _p(d_), len(s_))
+        if rc != 0:
+            raise ValueError(f"fork_residual rc={rc}")
 
     def prefill_attention(self, q, cu_new, seq_lens, block_tables, sm_scale=None) -> np.ndarray:
         """Causal attention of the appended chunk's query rows (q: fp16

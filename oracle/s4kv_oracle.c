@@ -358,6 +358,62 @@ int s4kv_ref_dequant_page(const uint8_t *pool, int num_pages, int num_kv_heads,
     return REF_OK;
 }
 
+/* ------------------------------------------------ page movement ---- */
+/* Moving whole pages between the pool and other memory, as a paged cache
+ * does when it swaps sequences out and back in or forks one copy-on-write
+ * ("KV-Cache und PagedAttention: Warum Ihr LLM-Server langsamer wird", "Wie
+ * PagedAttention das loest": pages are allocated on demand, shared between
+ * sequences and copied only when written).  A page record is all kv heads'
+ * blocks of one physical page: num_kv_heads * 2816 contiguous bytes. */
+
+/* dst[i] = page record pages[i], i < n (dst: [n][num_kv_heads][2816]). */
+int s4kv_ref_gather_pages(const uint8_t *pool, int num_pages, int num_kv_heads,
+                          const int32_t *pages, int n, uint8_t *dst) {
+    long rec = (long)num_kv_heads * BLOCK_BYTES;
+    for (int i = 0; i < n; ++i)
+        if (pages[i] < 0 || pages[i] >= num_pages) return REF_BAD_SLOT;
+    for (int i = 0; i < n; ++i) memcpy(dst + i * rec, pool + pages[i] * rec, (size_t)rec);
+    return REF_OK;
+}
+
+/* page record pages[i] = src[i], i < n (pages must be distinct). */
+int s4kv_ref_scatter_pages(uint8_t *pool, int num_pages, int num_kv_heads,
+                           const int32_t *pages, int n, const uint8_t *src) {
+    long rec = (long)num_kv_heads * BLOCK_BYTES;
+    for (int i = 0; i < n; ++i)
+        if (pages[i] < 0 || pages[i] >= num_pages) return REF_BAD_SLOT;
+    for (int i = 0; i < n; ++i) memcpy(pool + pages[i] * rec, src + i * rec, (size_t)rec);
+    return REF_OK;
+}
+
+/* page record dst_pages[i] = page record src_pages[i] (a copy-on-write copy
+ * of a shared full page); no dst page may also be a src page. */
+int s4kv_ref_copy_pages(uint8_t *pool, int num_pages, int num_kv_heads,
+                        const int32_t *src_pages, const int32_t *dst_pages, int n) {
+    long rec = (long)num_kv_heads * BLOCK_BYTES;
+    for (int i = 0; i < n; ++i)
+        if (src_pages[i] < 0 || src_pages[i] >= num_pages || dst_pages[i] < 0 || dst_pages[i] >= num_pages)
+            return REF_BAD_SLOT;
+    for (int i = 0; i < n; ++i) memcpy(pool + dst_pages[i] * rec, pool + src_pages[i] * rec, (size_t)rec);
+    return REF_OK;
+}
+
+/* The partial last page lives in the residual of its batch row: a fork
+ * copies batch row src_rows[i]'s residual keys and values (all kv heads, all
+ * 16 rows) to batch row dst_rows[i]. */
+int s4kv_ref_fork_residual(uint16_t *res_k, uint16_t *res_v, int max_seqs, int num_kv_heads,
+                           const int32_t *src_rows, const int32_t *dst_rows, int n) {
+    long rec = (long)num_kv_heads * PAGE * HEAD_DIM;
+    for (int i = 0; i < n; ++i)
+        if (src_rows[i] < 0 || src_rows[i] >= max_seqs || dst_rows[i] < 0 || dst_rows[i] >= max_seqs)
+            return REF_BAD_SLOT;
+    for (int i = 0; i < n; ++i) {
+        memcpy(res_k + dst_rows[i] * rec, res_k + src_rows[i] * rec, 2 * (size_t)rec);
+        memcpy(res_v + dst_rows[i] * rec, res_v + src_rows[i] * rec, 2 * (size_t)rec);
+    }
+    return REF_OK;
+}
+
 /* Gather the K and V rows (fp32 [L][128]) of sequence b, kv head h: full
  * pages are dequantized page by page, the tail comes from the fp16
  * residual. */

@@ -546,3 +546,87 @@ def test_prefill_last_row_is_decode(oracle_mod):
     last = q[cu[1:] - 1]
     dec = c.decode_attention(last, np.array(after, np.int32), bt, sm_scale=0.07)
     assert np.array_equal(out[cu[1:] - 1], dec)
+
+
+# ------------------------------------------------------ page movement --
+
+def test_swap_out_and_in_elsewhere_preserves_attention(oracle_mod):
+    """Swap a sequence's pages out (gather), wipe them, swap them back into
+    other physical pages (scatter) and point its page table there: decode
+    attention must come out bit-identical, and the gathered records must be
+    the same bytes as before."""
+    rng = np.random.default_rng(41)
+    H, G = 2, 4
+    lens = [37, 70, 16]
+    k, v = _rand_kv(rng, 3, H, lens)
+    bt, NP = _tables(rng, lens, extra=8)
+    c = _build_cache(oracle_mod, k, v, lens, bt, NP, H, chunk=13)
+    q = rng.standard_normal((3, H * G, HD)).astype(np.float16)
+    before = c.decode_attention(q, np.array(lens, np.int32), bt)
+    full = [int(p) for p in bt[1, :lens[1] // PAGE]]
+    rec = c.gather_pages(full)
+    c.scatter_pages(full, np.zeros_like(rec))
+    used = set(int(p) for p in bt[bt >= 0].ravel())
+    free = [p for p in range(NP) if p not in used][:len(full)]
+    c.scatter_pages(free, rec)
+    bt2 = bt.copy()
+    bt2[1, :len(full)] = free
+    after = c.decode_attention(q, np.array(lens, np.int32), bt2)
+    assert np.array_equal(before, after)
+    assert np.array_equal(c.gather_pages(free), rec)
+    # the wiped pages really were read before: with the old table the output changes
+    assert not np.array_equal(c.decode_attention(q, np.array(lens, np.int32), bt)[1], before[1])
+
+
+def test_fork_shares_full_pages_and_copies_the_partial_page(oracle_mod):
+    """Fork sequence 0 into batch row 2: the full pages are shared through the
+    page table, the partial page is copied (fork_residual).  Both rows then
+    give the same attention; appending to the fork fills its own page and
+    leaves the original untouched, and the fork equals a cache built from its
+    whole token stream directly."""
+    rng = np.random.default_rng(42)
+    H, G = 2, 3
+    L0, extra = 37, 20
+    k, v = _rand_kv(rng, 1, H, [L0 + extra])
+    k2 = [k[0][:L0], k[0][:L0], k[0]]
+    v2 = [v[0][:L0], v[0][:L0], v[0]]
+    NP = 16
+    bt = np.full((3, 4), -1, np.int32)
+    bt[0, :3] = [5, 9, 2]
+    bt[1, :3] = [7, 1, 12]
+    c = oracle_mod.OracleCache(NP, H, 3)
+    _append_all(oracle_mod, c, k2, v2, [0, 0, 0], [L0, L0, 0], bt)
+    # fork 0 -> 2: share the two full pages, copy the partial page's residual
+    bt[2, :2] = bt[0, :2]
+    bt[2, 2:4] = [3, 14]
+    c.fork_residual([0], [2])
+    q = rng.standard_normal((3, H * G, HD)).astype(np.float16)
+    q[2] = q[0]
+    out = c.decode_attention(q, np.array([L0, L0, L0], np.int32), bt)
+    assert np.array_equal(out[2], out[0])
+    ref0 = out[0].copy()
+    # the fork diverges: 20 more tokens complete its page 2 and start page 3
+    _append_all(oracle_mod, c, k2, v2, [L0, L0, L0], [L0, L0, L0 + extra], bt)
+    out = c.decode_attention(q, np.array([L0, L0, L0 + extra], np.int32), bt)
+    assert np.array_equal(out[0], ref0)
+    direct = oracle_mod.OracleCache(NP, H, 1)
+    btd = bt[2:3].copy()
+    _append_all(oracle_mod, direct, [k[0]], [v[0]], [0], [L0 + extra], btd)
+    assert np.array_equal(direct.decode_attention(q[2:3], np.array([L0 + extra], np.int32), btd)[0], out[2])
+
+
+def test_copy_pages_then_remap_preserves_attention(oracle_mod):
+    rng = np.random.default_rng(43)
+    H = 1
+    lens = [64, 33]
+    k, v = _rand_kv(rng, 2, H, lens)
+    bt, NP = _tables(rng, lens, extra=6)
+    c = _build_cache(oracle_mod, k, v, lens, bt, NP, H)
+    q = rng.standard_normal((2, 4, HD)).astype(np.float16)
+    before = c.decode_attention(q, np.array(lens, np.int32), bt)
+    used = set(int(p) for p in bt[bt >= 0].ravel())
+    free = [p for p in range(NP) if p not in used][:4]
+    c.copy_pages(bt[0, :4], free)
+    bt2 = bt.copy()
+    bt2[0, :4] = free
+    assert np.array_equal(c.decode_attention(q, np.array(lens, np.int32), bt2), before)
