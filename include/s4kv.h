@@ -191,6 +191,23 @@ S4KV_API int s4kv_decode_attention(const s4kv_cache_t *cache, const void *q,
                           void *workspace, size_t workspace_bytes,
                           void *stream);
 
+/* One decode step in one launch: the append of one new token per sequence
+ * fused into s4kv_decode_attention (row (L-1) % 16 of the last page; a page
+ * completed by it is quantized inside the same kernel, before any read of it).
+ *  k_new, v_new  device fp16 [batch][num_kv_heads][128], 16-B aligned: the
+ *          token of sequence b at position seq_lens[b] - 1.  A sequence with
+ *          seq_lens[b] == 0 has no token and gets zeros.
+ *  seq_lens  lengths AFTER the append (each sequence grows by exactly one).
+ *  All other arguments, the output and the workspace: as
+ *  s4kv_decode_attention.  The cache afterwards is byte-identical to what
+ *  s4kv_append with the same tokens writes, and the output is that of
+ *  s4kv_decode_attention after it. */
+S4KV_API int s4kv_append_decode(const s4kv_cache_t *cache, const void *k_new, const void *v_new,
+                                const void *q, int num_q_heads, const int32_t *seq_lens,
+                                const int32_t *block_tables, int batch, int max_pages_per_seq,
+                                float sm_scale, void *out, void *workspace, size_t workspace_bytes,
+                                void *stream);
+
 /* Size of the fixed scratch array behind s4kv_decode_attention_noalloc. */
 #define S4KV_NOALLOC_SCRATCH_BYTES (24u * 1024u * 1024u)
 

@@ -45,6 +45,7 @@ _SIGS = {
     "s4kv_decode_workspace_size": ([_I, _I, ctypes.POINTER(_SZ)], _I),
     "s4kv_decode_attention": ([_CP, _P, _I, _P, _P, _I, _I, ctypes.c_float, _P, _P, _SZ, _P], _I),
     "s4kv_decode_attention_noalloc": ([_CP, _P, _I, _P, _P, _I, _I, ctypes.c_float, _P, _P], _I),
+    "s4kv_append_decode": ([_CP, _P, _P, _P, _I, _P, _P, _I, _I, ctypes.c_float, _P, _P, _SZ, _P], _I),
     "s4kv_prefill_attention": ([_CP, _P, _I, _I, _P, _P, _P, _I, _I, _I, ctypes.c_float, _P, _P], _I),
     "s4kv_dequant_page": ([_CP, _I, _P, _P, _I, _P], _I),
     "s4kv_dequant_pages": ([_CP, _P, _I, _P, _P, _I, _P], _I),
@@ -191,6 +192,23 @@ def s4kv_decode_attention(cache: S4KVCache, q, seq_lens, block_tables, out, work
                                     _ptr(workspace, torch.uint8, "workspace"), workspace.numel(),
                                     _stream(stream))
     _check(st, "s4kv_decode_attention")
+
+
+def s4kv_append_decode(cache: S4KVCache, k_new, v_new, q, seq_lens, block_tables, out, workspace,
+                       sm_scale: float | None = None, stream=None):
+    """One decode step in one launch: append each sequence's new token
+    (k_new, v_new fp16 [batch][kv_heads][128]) and attend over the result."""
+    import torch
+    batch, num_q_heads, _ = q.shape
+    if sm_scale is None:
+        sm_scale = HEAD_DIM ** -0.5
+    st = lib().s4kv_append_decode(cache.ref, _ptr(k_new, torch.float16, "k_new"), _ptr(v_new, torch.float16, "v_new"),
+                                 _ptr(q, torch.float16, "q"), num_q_heads,
+                                 _ptr(seq_lens, torch.int32, "seq_lens"),
+                                 _ptr(block_tables, torch.int32, "block_tables"), batch, block_tables.shape[1],
+                                 float(sm_scale), _ptr(out, torch.float16, "out"),
+                                 _ptr(workspace, torch.uint8, "workspace"), workspace.numel(), _stream(stream))
+    _check(st, "s4kv_append_decode")
 
 
 def s4kv_decode_attention_noalloc(cache: S4KVCache, q, seq_lens, block_tables, out,

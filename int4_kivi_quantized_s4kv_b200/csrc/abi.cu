@@ -108,6 +108,10 @@ int launch_records(const uint8_t *src, uint8_t *dst, const int32_t *src_idx, con
   return S4KV_OK;
 }
 
+int decode_call(const s4kv_cache_t *cache, const void *k_new, const void *v_new, const void *q, int num_q_heads,
+                const int32_t *seq_lens, const int32_t *block_tables, int batch, int max_pages_per_seq,
+                float sm_scale, void *out, void *workspace, size_t workspace_bytes, void *stream);
+
 }  // namespace
 
 extern "C" {
@@ -193,6 +197,26 @@ int s4kv_decode_attention(const s4kv_cache_t *cache, const void *q, int num_q_he
                           const int32_t *seq_lens, const int32_t *block_tables, int batch,
                           int max_pages_per_seq, float sm_scale, void *out, void *workspace,
                           size_t workspace_bytes, void *stream) {
+  return decode_call(cache, nullptr, nullptr, q, num_q_heads, seq_lens, block_tables, batch, max_pages_per_seq,
+                     sm_scale, out, workspace, workspace_bytes, stream);
+}
+
+int s4kv_append_decode(const s4kv_cache_t *cache, const void *k_new, const void *v_new, const void *q,
+                       int num_q_heads, const int32_t *seq_lens, const int32_t *block_tables, int batch,
+                       int max_pages_per_seq, float sm_scale, void *out, void *workspace, size_t workspace_bytes,
+                       void *stream) {
+  if (batch > 0 && (!k_new || !v_new || !aligned(k_new, 16) || !aligned(v_new, 16))) return S4KV_ERR_INVALID_ARG;
+  return decode_call(cache, k_new, v_new, q, num_q_heads, seq_lens, block_tables, batch, max_pages_per_seq,
+                     sm_scale, out, workspace, workspace_bytes, stream);
+}
+
+}  // extern "C"
+
+namespace {
+
+int decode_call(const s4kv_cache_t *cache, const void *k_new, const void *v_new, const void *q, int num_q_heads,
+                const int32_t *seq_lens, const int32_t *block_tables, int batch, int max_pages_per_seq,
+                float sm_scale, void *out, void *workspace, size_t workspace_bytes, void *stream) {
   int rc = check_cache(cache);
   if (rc != S4KV_OK) return rc;
   rc = s4kv_check_model(cache->head_dim, cache->page_tokens, num_q_heads, cache->num_kv_heads);
@@ -229,10 +253,17 @@ int s4kv_decode_attention(const s4kv_cache_t *cache, const void *q, int num_q_he
   p.num_pages = cache->num_pages;
   p.scale_log2 = static_cast<float>(static_cast<double>(sm_scale) * 1.4426950408889634);
   p.num_workers = d.num_workers;
-  launch_decode(p, d.num_ctas, static_cast<cudaStream_t>(stream));
+  FusedAppend f;
+  f.k_new = static_cast<const __half *>(k_new);
+  f.v_new = static_cast<const __half *>(v_new);
+  launch_decode(p, f, d.num_ctas, static_cast<cudaStream_t>(stream));
   if (cudaGetLastError() != cudaSuccess) return S4KV_ERR_CUDA;
   return S4KV_OK;
 }
+
+}  // namespace
+
+extern "C" {
 
 int s4kv_prefill_attention(const s4kv_cache_t *cache, const void *q, int num_q_heads, int n_tokens,
                            const int32_t *cu_new, const int32_t *seq_lens, const int32_t *block_tables,

@@ -16,26 +16,9 @@
 // after its own page has read the residual rows it needed, so one call can
 // complete a page and start the next one without a race.
 #include "kernels.cuh"
+#include "quant.cuh"
 
 namespace s4kv {
-
-// a < b in IEEE total order for non-NaN values (-0 below +0).
-__device__ __forceinline__ bool total_less(float a, float b) {
-  return a < b || (a == b && signbit(a) && !signbit(b));
-}
-
-// One quantization group in fp32: s = (max - min) / 15 and
-// code = s == 0 ? 0 : clamp(rint((x - min) / s), 0, 15), every operation
-// IEEE-rounded (no contraction, no fast math).
-__device__ __forceinline__ float group_scale(float mn, float mx) {
-  return __fdiv_rn(__fsub_rn(mx, mn), 15.0f);
-}
-__device__ __forceinline__ uint32_t group_code(float x, float mn, float s) {
-  if (s == 0.0f) return 0u;
-  float r = rintf(__fdiv_rn(__fsub_rn(x, mn), s));
-  r = fminf(fmaxf(r, 0.0f), 15.0f);
-  return static_cast<uint32_t>(r);
-}
 
 __global__ void __launch_bounds__(128) append_kernel(const AppendParams p) {
   const int slot = blockIdx.x;
@@ -101,60 +84,7 @@ __global__ void __launch_bounds__(128) append_kernel(const AppendParams p) {
 
     if (phys_ok) {
       uint8_t *blk = p.pool + (static_cast<long>(phys) * H + h) * kBlockBytes;
-      // keys: thread c quantizes channel c over the 16 tokens
-      {
-        const int c = tid;
-        float mn = __half2float(ks[0][c]), mx = mn;
-#pragma unroll
-        for (int t = 1; t < kPage; ++t) {
-          const float x = __half2float(ks[t][c]);
-          if (total_less(x, mn)) mn = x;
-          if (total_less(mx, x)) mx = x;
-        }
-        const float s = group_scale(mn, mx);
-#pragma unroll
-        for (int t = 0; t < kPage; ++t) kc[t][c] = static_cast<uint8_t>(group_code(__half2float(ks[t][c]), mn, s));
-        reinterpret_cast<__half *>(blk + kKScaleOff)[c] = __float2half_rn(s);
-        // zero points in the MMA k order: tile (c%32)/4, slot 2(c/32) + (c%2) + 8((c%4)/2)
-        const int zslot = 16 * ((c & 31) >> 2) + 2 * (c >> 5) + (c & 1) + 8 * ((c & 3) >> 1);
-        reinterpret_cast<__half *>(blk + kKZeroOff)[zslot] = __float2half_rn(mn);
-      }
-      // values: threads 0..63 each quantize one (token, 32-channel group)
-      if (tid < kPage * (kHeadDim / kVGroup)) {
-        const int t = tid >> 2, g = tid & 3;
-        float mn = __half2float(vs[t][g * kVGroup]), mx = mn;
-        for (int j = 1; j < kVGroup; ++j) {
-          const float x = __half2float(vs[t][g * kVGroup + j]);
-          if (total_less(x, mn)) mn = x;
-          if (total_less(mx, x)) mx = x;
-        }
-        const float s = group_scale(mn, mx);
-        for (int j = 0; j < kVGroup; ++j)
-          vc[t][g * kVGroup + j] = static_cast<uint8_t>(group_code(__half2float(vs[t][g * kVGroup + j]), mn, s));
-        reinterpret_cast<__half *>(blk + kVScaleOff)[g * kPage + t] = __float2half_rn(s);
-        reinterpret_cast<__half *>(blk + kVZeroOff)[g * kPage + t] = __float2half_rn(mn);
-      }
-      __syncthreads();
-      // pack: word w = 128*hh + 4*lane + q; nibble j is register j&3, half j>>2
-      // of that lane's m16n8k16 operand fragment (tile = 4*hh + q)
-      for (int w = tid; w < 256; w += 128) {
-        const int hh = w >> 7, lane = (w >> 2) & 31, q = w & 3;
-        const int n = lane >> 2, i = lane & 3, tile = 4 * hh + q;
-        uint32_t kw = 0, vw = 0;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          // keys: row = token, k axis = channel 32i + 4*tile + {0,1 | 2,3}
-          const int kt = 8 * (j & 1) + n;
-          const int kch = 32 * i + 4 * tile + 2 * ((j >> 1) & 1) + (j >> 2);
-          kw |= static_cast<uint32_t>(kc[kt][kch]) << (4 * j);
-          // values: row = channel of M-tile `tile`, k axis = token
-          const int vt = 2 * i + (j >> 2) + 8 * ((j >> 1) & 1);
-          const int vch = 32 * (tile >> 1) + 4 * n + 2 * (tile & 1) + (j & 1);
-          vw |= static_cast<uint32_t>(vc[vt][vch]) << (4 * j);
-        }
-        reinterpret_cast<uint32_t *>(blk + kKCodeOff)[w] = kw;
-        reinterpret_cast<uint32_t *>(blk + kVCodeOff)[w] = vw;
-      }
+      quantize_page_cta(ks, vs, kc, vc, blk, tid);
     }
     if (slot != 0) return;
     __syncthreads();  // residual rows read above before the tail overwrites them

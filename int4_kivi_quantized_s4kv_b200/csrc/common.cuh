@@ -23,6 +23,41 @@ __device__ __forceinline__ void flag_error(uint32_t *err, uint32_t bits) {
   if (err != nullptr) atomicOr(err, bits);
 }
 
+// ------------------------------------------------------------ quantizer --
+
+// a < b in IEEE total order for non-NaN values (-0 below +0).
+__device__ __forceinline__ bool total_less(float a, float b) {
+  return a < b || (a == b && signbit(a) && !signbit(b));
+}
+
+// One quantization group in fp32: s = (max - min) / 15 and
+// code = s == 0 ? 0 : clamp(rint((x - min) / s), 0, 15), every operation
+// IEEE-rounded (no contraction, no fast math).
+__device__ __forceinline__ float group_scale(float mn, float mx) {
+  return __fdiv_rn(__fsub_rn(mx, mn), 15.0f);
+}
+__device__ __forceinline__ uint32_t group_code(float x, float mn, float s) {
+  if (s == 0.0f) return 0u;
+  float r = rintf(__fdiv_rn(__fsub_rn(x, mn), s));
+  r = fminf(fmaxf(r, 0.0f), 15.0f);
+  return static_cast<uint32_t>(r);
+}
+
+// The same code with the division replaced by a product with inv_s =
+// RN(1 / s) wherever that cannot change it: with x_ = x - min and x_ / s <=
+// 16, the product is within 2^-19 of x_ / s and RN(x_ / s) within 2^-20, so
+// the two round to the same integer unless the product lies within 2^-10 of
+// a half-integer; only then is the division done.
+__device__ __forceinline__ uint32_t group_code_fast(float x, float mn, float s, float inv_s) {
+  if (s == 0.0f) return 0u;
+  const float d = __fsub_rn(x, mn);
+  const float q = __fmul_rn(d, inv_s);
+  float r = rintf(q);
+  if (fabsf(fabsf(__fsub_rn(q, r)) - 0.5f) < 0x1p-10f) r = rintf(__fdiv_rn(d, s));
+  r = fminf(fmaxf(r, 0.0f), 15.0f);
+  return static_cast<uint32_t>(r);
+}
+
 // ---------------------------------------------------------------- bit ops --
 
 // (a & b) | c in one LOP3.

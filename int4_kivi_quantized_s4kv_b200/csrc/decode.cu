@@ -43,6 +43,7 @@
 #include <cfloat>
 
 #include "kernels.cuh"
+#include "quant.cuh"
 
 namespace s4kv {
 
@@ -430,7 +431,57 @@ __device__ __forceinline__ void merge_pieces(const DecodeParams &p, long obase, 
   }
 }
 
-__global__ void __launch_bounds__(kThreads, S4KV_DECODE_MIN_CTAS) decode_kernel(const DecodeParams p) {
+// Fused append of one decode step for (sequence b, kv head h) whose length
+// after the append is L >= 1: the new token (row b of k_new / v_new) is
+// position L - 1, row (L - 1) % 16 of the sequence's last page.
+//  * If that row is not the page's last, one warp writes the token into the
+//    residual (lane l: channels 4l .. 4l + 3).
+//  * Otherwise the token completes the page, which is quantized from the
+//    residual rows 0..14 plus the token by the whole CTA (quantize_page_cta,
+//    the routine s4kv_append uses, so the bytes are the same).
+constexpr int kJobsPerWarp = 8;
+
+__device__ __forceinline__ void residual_row_write(const DecodeParams &p, const FusedAppend &f, int b, int h, int L,
+                                                   int lane) {
+  const int H = p.num_kv_heads;
+  const long rbase = (static_cast<long>(b) * H + h) * kPage * kHeadDim + 4 * lane;
+  const long nbase = (static_cast<long>(b) * H + h) * kHeadDim + 4 * lane;
+  const int r = (L - 1) % kPage;
+  // the cache is written only by the fused append (the parameters carry it
+  // read-only for the attention)
+  __half *res_k = const_cast<__half *>(p.res_k), *res_v = const_cast<__half *>(p.res_v);
+  *reinterpret_cast<uint2 *>(res_k + rbase + r * kHeadDim) = *reinterpret_cast<const uint2 *>(f.k_new + nbase);
+  *reinterpret_cast<uint2 *>(res_v + rbase + r * kHeadDim) = *reinterpret_cast<const uint2 *>(f.v_new + nbase);
+}
+
+// One completed page (job = sequence, kv head, physical page) quantized by
+// all threads of the CTA, with `scratch` (12 KB of shared memory) as staging.
+__device__ __forceinline__ void cta_quantize_job(const DecodeParams &p, const FusedAppend &f, int4 job, uint8_t *scratch,
+                                                 int tid) {
+  const int b = job.x, h = job.y, phys = job.w;
+  const int H = p.num_kv_heads;
+  auto ks = reinterpret_cast<__half (*)[kHeadDim]>(scratch);
+  auto vs = reinterpret_cast<__half (*)[kHeadDim]>(scratch + kPage * kHeadDim * 2);
+  auto kc = reinterpret_cast<uint8_t (*)[kHeadDim]>(scratch + 2 * kPage * kHeadDim * 2);
+  auto vc = reinterpret_cast<uint8_t (*)[kHeadDim]>(scratch + 2 * kPage * kHeadDim * 2 + kPage * kHeadDim);
+  const long res_base = (static_cast<long>(b) * H + h) * kPage * kHeadDim;
+  const long new_base = (static_cast<long>(b) * H + h) * kHeadDim;
+  for (int ch = tid; ch < kPage * (kHeadDim / 8); ch += kThreads) {
+    const int t = ch / (kHeadDim / 8), c8 = (ch % (kHeadDim / 8)) * 8;
+    const __half *sk = t < kPage - 1 ? p.res_k + res_base + t * kHeadDim + c8 : f.k_new + new_base + c8;
+    const __half *sv = t < kPage - 1 ? p.res_v + res_base + t * kHeadDim + c8 : f.v_new + new_base + c8;
+    *reinterpret_cast<uint4 *>(&ks[t][c8]) = *reinterpret_cast<const uint4 *>(sk);
+    *reinterpret_cast<uint4 *>(&vs[t][c8]) = *reinterpret_cast<const uint4 *>(sv);
+  }
+  __syncthreads();
+  quantize_page_cta(ks, vs, kc, vc, const_cast<uint8_t *>(p.pool) + (static_cast<long>(phys) * H + h) * kBlockBytes,
+                    tid);
+  __syncthreads();  // the scratch is reused by the next job
+}
+
+// kFused: the step's append is fused in (DecodeParams::k_new / v_new set).
+template <bool kFused>
+__global__ void __launch_bounds__(kThreads, S4KV_DECODE_MIN_CTAS) decode_kernel(const DecodeParams p, const FusedAppend f) {
   extern __shared__ __align__(128) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n = lane >> 2, i = lane & 3;
@@ -484,8 +535,11 @@ __global__ void __launch_bounds__(kThreads, S4KV_DECODE_MIN_CTAS) decode_kernel(
       }
     }
   }
-  if (worker >= W || T == 0) return;
-  const long long s = worker * T / W, e = (worker + 1) * T / W;
+  // with the fused append every warp of the CTA takes part in its barriers
+  if (kFused ? T == 0 : (worker >= W || T == 0)) return;
+  const bool active = worker < W;
+  const long long s = (kFused && !active) ? 0 : worker * T / W;
+  const long long e = (kFused && !active) ? 0 : (worker + 1) * T / W;
 
   // ---- locate the segment holding page s
   const unsigned hit = __ballot_sync(kFull, H * excl <= s && s < H * incl);
@@ -512,6 +566,50 @@ __global__ void __launch_bounds__(kThreads, S4KV_DECODE_MIN_CTAS) decode_kernel(
   cc.start = H * pre + static_cast<long long>(cc.h) * cc.np;
   const int range = static_cast<int>(e - s);
   const int p_first = static_cast<int>(s - cc.start);
+
+  // ---- fused append: the step's new token of every segment whose last page
+  // lies in this worker's range (each segment has exactly one such worker,
+  // the one that also reads that page) is written before any copy of it.  A
+  // token that completes its page makes a job for the whole CTA; jobs are
+  // collected up to kJobsPerWarp per warp and round, then quantized.
+  if (kFused) {
+    __shared__ int4 s_job[kWarpsPerCta][kJobsPerWarp];
+    __shared__ int s_njob[kWarpsPerCta];
+    Cursor ac = cc;
+    bool more = active;
+    while (true) {
+      int nj = 0;
+      while (more && nj < kJobsPerWarp) {
+        if (ac.b >= B || ac.start >= e) {
+          more = false;
+          break;
+        }
+        const long long last = ac.start + ac.np - 1;
+        if (last >= s && last < e && ac.len > 0) {
+          if (ac.len % kPage != 0) {
+            residual_row_write(p, f, ac.b, ac.h, ac.len, lane);
+          } else {
+            const int phys = __ldg(ac.bt + (ac.len - 1) / kPage);
+            if (static_cast<unsigned>(phys) >= static_cast<unsigned>(p.num_pages)) {
+              if (lane == 0) flag_error(p.err, S4KV_EFLAG_PAGE_RANGE);
+            } else {
+              if (lane == 0) s_job[warp][nj] = make_int4(ac.b, ac.h, ac.len, phys);
+              ++nj;
+            }
+          }
+        }
+        next_segment(ac, p);
+      }
+      if (lane == 0) s_njob[warp] = nj;
+      __syncthreads();
+      for (int w = 0; w < kWarpsPerCta; ++w)
+        for (int j = 0; j < s_njob[w]; ++j) cta_quantize_job(p, f, s_job[w][j], smem, threadIdx.x);
+      // the pool writes are read next by bulk copies (async proxy)
+      asm volatile("fence.proxy.async.global;" ::: "memory");
+      if (!__syncthreads_or(more)) break;
+    }
+    if (!active) return;
+  }
 
   // ---- producer: issue the next quantized page of [s, e) into the ring.
   // It walks the same pieces as the consumer.  The page ids of a piece are
@@ -808,19 +906,28 @@ __global__ void __launch_bounds__(kThreads, S4KV_DECODE_MIN_CTAS) decode_kernel(
 
 int decode_ctas_per_sm() {
   int n = 0;
-  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_kernel, kThreads, decode_smem_bytes());
+  int m = 0;
+  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_kernel<false>, kThreads, decode_smem_bytes());
+  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&m, decode_kernel<true>, kThreads, decode_smem_bytes());
+  n = n < m ? n : m;  // one launch shape (and workspace size) serves both
   return n;
 }
 
 int decode_warps_per_cta() { return kWarpsPerCta; }
 
 cudaError_t prepare_decode_kernel() {
-  return cudaFuncSetAttribute(decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  const cudaError_t e = cudaFuncSetAttribute(decode_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(decode_smem_bytes()));
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(decode_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                               static_cast<int>(decode_smem_bytes()));
 }
 
-void launch_decode(const DecodeParams &p, int num_ctas, cudaStream_t stream) {
-  decode_kernel<<<num_ctas, kThreads, decode_smem_bytes(), stream>>>(p);
+void launch_decode(const DecodeParams &p, const FusedAppend &f, int num_ctas, cudaStream_t stream) {
+  if (f.k_new != nullptr)
+    decode_kernel<true><<<num_ctas, kThreads, decode_smem_bytes(), stream>>>(p, f);
+  else
+    decode_kernel<false><<<num_ctas, kThreads, decode_smem_bytes(), stream>>>(p, f);
 }
 
 }  // namespace s4kv

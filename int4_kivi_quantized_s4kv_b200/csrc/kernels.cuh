@@ -77,6 +77,14 @@ struct DecodeParams {
   int num_workers;
 };
 
+// Fused append of a decode step: each sequence's new token (fp16
+// [batch][kv_heads][128]) is written into the cache before the attention
+// reads it.  Both nullptr for a plain decode.
+struct FusedAppend {
+  const __half *k_new;
+  const __half *v_new;
+};
+
 struct PrefillParams {
   const uint8_t *pool;
   const __half *res_k;
@@ -99,7 +107,7 @@ struct PrefillParams {
 void launch_append(const AppendParams &p, int batch, int max_new, cudaStream_t stream);
 void launch_dequant(const DequantParams &p, cudaStream_t stream);
 void launch_move(const MoveParams &p, cudaStream_t stream);
-void launch_decode(const DecodeParams &p, int num_ctas, cudaStream_t stream);
+void launch_decode(const DecodeParams &p, const FusedAppend &f, int num_ctas, cudaStream_t stream);
 int decode_ctas_per_sm();
 int decode_warps_per_cta();
 cudaError_t prepare_decode_kernel();
