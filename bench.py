@@ -401,6 +401,97 @@ def measure_prefill(device, steps: int, workload: str = "llama3.1-8b-prefill"):
                          "flops_per_launch": flops, "mma_flops_per_launch": 1.5 * flops}}
 
 
+def measure_page_moves(wl, device, reps: int = 10):
+    """Swap-side page movement on the decode workload's resident cache:
+    gathering page records into a staging buffer (HBM read + write), and a
+    whole swap-out / swap-in through pinned host memory (bound by the
+    host link)."""
+    import torch
+    S = wl.S
+    cache = wl.caches[0]
+    H = wl.spec.num_kv_heads
+    rec = S.s4kv_page_record_bytes(H)
+    nfull = (wl.lens // 16).astype(np.int64)
+    # gather: as many whole sequences as make > 2x L2 of records
+    rows, total = [], 0
+    for b in range(wl.spec.batch):
+        rows.append(wl.plan.block_tables[b, :nfull[b]])
+        total += int(nfull[b]) * rec
+        if total > 300e6:
+            break
+    pages = torch.from_numpy(np.ascontiguousarray(np.concatenate(rows).astype(np.int32))).to(device)
+    n = pages.numel()
+    staging = torch.empty((n, rec), dtype=torch.uint8, device=device)
+
+    def timed(fn, k):
+        fn()
+        torch.cuda.synchronize()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(k):
+            fn()
+        b.record()
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / k
+
+    g_ms = timed(lambda: S.s4kv_gather_pages(cache, pages, staging), reps)
+    # swap-out / swap-in of one sequence's pages through pinned host memory
+    sp = pages[: int(nfull[0])]
+    host = torch.empty((sp.numel(), rec), dtype=torch.uint8, pin_memory=True)
+    st = staging[: sp.numel()]
+    o_ms = timed(lambda: S.s4kv_swap_out(cache, sp, st, host), 3)
+    i_ms = timed(lambda: S.s4kv_swap_in(cache, sp, st, host), 3)   # writes the same bytes back
+    if S.s4kv_get_error(cache):
+        raise RuntimeError("page movement set device error flags")
+    peak, kind = measured_hbm_peak()
+    gbs = 2 * n * rec / (g_ms * 1e-3) / 1e9
+    swap_bytes = sp.numel() * rec
+    return {"gather": {"pages": n, "record_bytes": rec, "avg_launch_ms": g_ms,
+                       "roofline": {"bound": "hbm", "kernel": "move_kernel", "achieved": gbs, "peak": peak,
+                                    "peak_kind": kind, "unit": "GB/s", "frac": gbs / peak, "traffic": None,
+                                    "bytes_per_launch": 2 * n * rec}},
+            "swap_out": {"bytes": swap_bytes, "ms": o_ms, "GB_per_s": swap_bytes / (o_ms * 1e-3) / 1e9},
+            "swap_in": {"bytes": swap_bytes, "ms": i_ms, "GB_per_s": swap_bytes / (i_ms * 1e-3) / 1e9}}
+
+
+def measure_fused_step(wl, device, steps: int = 20):
+    """One decode step as two launches (s4kv_append, s4kv_decode_attention)
+    and as one (s4kv_append_decode) on the same resident workload; both
+    rewrite the same cache bytes each step."""
+    import torch
+    S = wl.S
+    spec = wl.spec
+    B, H = spec.batch, spec.num_kv_heads
+    kn = [k.view(B, H, 128) for k in wl.k_new]
+    vn = [v.view(B, H, 128) for v in wl.v_new]
+
+    def fused():
+        for layer in range(spec.layers):
+            S.s4kv_append_decode(wl.caches[layer], kn[layer], vn[layer], wl.q[layer], wl.seq_lens, wl.bt,
+                                 wl.out[layer], wl.ws)
+
+    def timed(fn):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(steps):
+            fn()
+        b.record()
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / steps
+
+    two = timed(wl.step)
+    one = timed(fused)
+    if any(S.s4kv_get_error(c) for c in wl.caches):
+        raise RuntimeError("fused step set device error flags")
+    return {"workload": spec.name, "layers": spec.layers, "two_launch_ms": two, "fused_ms": one,
+            "speedup": two / one, "launches_per_layer": {"two_launch": 2, "fused": 1}}
+
+
 def run_reference(args, spec):
     world, rank, _ = _dist()
     if rank != 0:
@@ -537,9 +628,14 @@ def main(argv=None):
     value = aggregate_gbs(world, bytes_per_step, step_ms)
     achieved = decode_bytes_per_launch / (dec_avg_ms * 1e-3) / 1e9
     tokens = int(wl.new.sum())
-    prefill = None
+    prefill = moves = fused = None
     if world == 1 and not args.no_prefill:
         prefill = measure_prefill(device, max(3, min(args.steps, 20)))
+        moves = measure_page_moves(wl, device)
+        fused = [measure_fused_step(wl, device)]
+        small = DeviceWorkload(W.SPECS["qwen2.5-7b"], device)
+        fused.append(measure_fused_step(small, device))
+        del small
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(spec)
@@ -576,7 +672,7 @@ def main(argv=None):
         if cpu is not None:
             line["cpu_baseline"] = cpu
         if prefill is not None:
-            line["next_rows"] = {"prefill": prefill}
+            line["next_rows"] = {"prefill": prefill, "page_moves": moves, "fused_step": fused}
         print(json.dumps(line), flush=True)
     if world > 1:
         torch.distributed.destroy_process_group()
