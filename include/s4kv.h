@@ -256,7 +256,7 @@ S4KV_API int s4kv_decode_attention_noalloc(const s4kv_cache_t *cache, const void
  * Runs on the tcgen05 tensor cores with the dequantized keys and values and
  * the softmax weights as fp16 MMA operands (fp32 accumulation), so results
  * agree with exact attention to about fp16 precision of those operands.
- * Allocates nothing; needs about 205 KB of shared memory per CTA. */
+ * Allocates nothing; needs about 171 KB of shared memory per CTA. */
 S4KV_API int s4kv_prefill_attention(const s4kv_cache_t *cache, const void *q,
                                     int num_q_heads, int n_tokens,
                                     const int32_t *cu_new, const int32_t *seq_lens,

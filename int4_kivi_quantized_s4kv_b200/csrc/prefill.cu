@@ -14,27 +14,29 @@
 // How (B200): this is a dense contraction, so it runs on the fifth-generation
 // tensor cores.  One CTA takes one (query tile, sequence, kv head); the tile's
 // 128 MMA rows are (token, head of the group) pairs, so a tile holds
-// floor(128 / G) tokens.  Keys are walked in tiles of 128 (8 pages):
-//  * the 8 page blocks of the next key tile are fetched by 1-D bulk copies
-//    (TMA engine, no multicast) into a second staging buffer while the
-//    current one is used;
-//  * all 128 threads dequantize the current tile into the 128-byte-swizzled
-//    fp16 operands.  A key is code * scale + zero in fp32 (exact product, one
-//    rounding, the value the oracle's dequantization gives) split into an
-//    fp16 hi part and the fp16 rounding of the remainder, so K_hi + K_lo
-//    carries it to about 22 bits: keys of outlier channels are large, and a
-//    single fp16 rounding of them moves the logits visibly.  A value is the
-//    fused fp16 multiply-add code * scale + zero (the correctly rounded fp16),
-//    stored transposed (V^T [channel][key]);
-//  * one thread issues S = Q K_hi^T + Q K_lo^T (16 tcgen05.mma, M = N = 128,
-//    K = 16 each) into tensor memory; the four warps read S back one row per thread, apply
-//    the causal mask and an online softmax in the exp2 domain whose reference
-//    moves only when a row maximum passes it by more than 8 (weights stay
-//    <= 256, fine for fp16), and write P (fp16) to shared memory;
-//  * one thread issues O += P V (8 tcgen05.mma) into a second tensor-memory
-//    accumulator; when a row's reference moves, that row of O is rescaled in
-//    tensor memory first.
-// Every wait is bounded; a timeout or a bad page id sets a bit in err_flag.
+// floor(128 / G) tokens.  Keys are walked in tiles of 64 (4 pages) by warps
+// with separate roles, handing buffers over through mbarriers so that the
+// dequantization, the tensor core and the softmax run at the same time:
+//  * a producer warp brings each key tile's page blocks into one of two
+//    staging buffers with 1-D bulk copies (TMA engine, no multicast);
+//  * 8 dequantization warps turn a staged tile into the 128-byte-swizzled
+//    fp16 operands of one of two operand buffers.  A key is code * scale +
+//    zero in fp32 (exact product, one rounding, the value the oracle's
+//    dequantization gives) split into an fp16 hi part and the fp16 rounding
+//    of the remainder, so K_hi + K_lo carries it to about 22 bits (keys of
+//    outlier channels are large, and a single fp16 rounding of them moves the
+//    logits visibly).  A value is the fused fp16 multiply-add code * scale +
+//    zero (the correctly rounded fp16), stored transposed (V^T);
+//  * one thread issues S(k) = Q K_hi^T + Q K_lo^T (M = 128, N = 64) into one
+//    of two tensor-memory buffers, then O += P(k-1) V(k-1) (N = 128, K = 64),
+//    so the tensor core computes the next logits during the softmax;
+//  * 4 softmax warps (one tensor-memory lane, i.e. one row, per thread) read
+//    S back, apply the causal mask and an online softmax in the exp2 domain
+//    whose reference moves only when a row maximum passes it by more than 8
+//    (weights stay <= 256, fine for fp16), rescale that row of O in tensor
+//    memory when it moves, and write P (fp16) to shared memory.
+// Every wait is bounded; a timeout sets a CTA-wide abort flag and an error
+// bit, and every role then leaves its loop.
 #include <cfloat>
 
 #include "kernels.cuh"
@@ -44,34 +46,53 @@ namespace s4kv {
 
 namespace {
 
-constexpr int kThreadsP = 512;
-constexpr int kKeyTile = 128;                    // keys per tile (MMA N of S)
-constexpr int kPagesPerTile = kKeyTile / kPage;  // 8
-constexpr uint32_t kOpBytes = 128 * 128 * 2;     // one fp16 [128][128] operand
+constexpr int kSoftmaxWarps = 4;   // warps 0..3: one row per thread
+constexpr int kDequantWarps = 8;   // warps 4..11
+constexpr int kMmaWarp = 12;
+constexpr int kProducerWarp = 13;
+constexpr int kThreadsP = 32 * 14;
+constexpr int kDqThreads = 32 * kDequantWarps;
+constexpr int kKeyTile = 64;                     // keys per tile (MMA N of S)
+constexpr int kPagesPerTile = kKeyTile / kPage;  // 4
+constexpr uint32_t kQBytes = 128 * 128 * 2;      // Q [128][128] fp16
+constexpr uint32_t kKBytes = 64 * 128 * 2;       // K [64][128] fp16
+constexpr uint32_t kVBytes = 128 * 64 * 2;       // V^T [128][64] fp16
+constexpr uint32_t kPBytes = 128 * 64 * 2;       // P [128][64] fp16
 constexpr uint32_t kStageBytes = kPagesPerTile * kBlockBytes;
 constexpr float kSlack = 8.0f;                   // log2 slack of the softmax reference
 constexpr long long kWaitLimit = 2000000000LL;   // about one second
-constexpr uint32_t kIdesc = tc05::idesc_f16_f32(128, 128);
+constexpr uint32_t kIdescS = tc05::idesc_f16_f32(128, 64);
+constexpr uint32_t kIdescO = tc05::idesc_f16_f32(128, 128);
 
-// smem: Q, K hi, K lo, V^T, P operands (1024-aligned), two staging buffers,
-// barriers
+// smem: operands (1024-aligned), two staging buffers, barriers
 constexpr uint32_t kOffQ = 0;
-constexpr uint32_t kOffK = kOpBytes;
-constexpr uint32_t kOffKlo = 2 * kOpBytes;
-constexpr uint32_t kOffV = 3 * kOpBytes;
-constexpr uint32_t kOffP = 4 * kOpBytes;
-constexpr uint32_t kOffStage = 5 * kOpBytes;
-constexpr uint32_t kOffBar = kOffStage + 2 * kStageBytes;  // 4 mbarriers + tmem slot
-constexpr uint32_t kOffRed = kOffBar + 64;                 // [4][128] fp32 row partials
-constexpr uint32_t kSmemBytes = kOffRed + 4 * 128 * 4 + 1024;  // + alignment slack
+constexpr uint32_t kOffKhi = kOffQ + kQBytes;         // [2]
+constexpr uint32_t kOffKlo = kOffKhi + 2 * kKBytes;   // [2]
+constexpr uint32_t kOffV = kOffKlo + 2 * kKBytes;     // [2]
+constexpr uint32_t kOffP = kOffV + 2 * kVBytes;
+constexpr uint32_t kOffStage = kOffP + kPBytes;       // [2]
+constexpr uint32_t kOffBar = kOffStage + 2 * kStageBytes;
+// barriers (8 bytes each): stage_full[2], stage_empty[2], kv_full[2],
+// kv_empty[2], s_full[2], s_empty[2], p_full, p_empty; then the tensor-memory
+// address and the abort flag
+constexpr uint32_t kNumBars = 14;
+constexpr uint32_t kOffSlot = kOffBar + 8 * kNumBars;
+constexpr uint32_t kOffAbort = kOffSlot + 4;
+constexpr uint32_t kSmemBytes = kOffAbort + 4 + 1024;  // + alignment slack
 
-__device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity) {
+// Bounded wait for a barrier phase; gives up after about a second or as soon
+// as another role has raised the CTA's abort flag.
+__device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, const volatile int *abort) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (clock64() - t0 > kWaitLimit) return false;
+    if (*abort || clock64() - t0 > kWaitLimit) return false;
   }
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 
 __device__ __forceinline__ void sts64(uint32_t addr, uint32_t a, uint32_t b) {
@@ -119,12 +140,23 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(const PrefillPara
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_addr(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
-  const uint32_t sQ = base + kOffQ, sK = base + kOffK, sKlo = base + kOffKlo, sV = base + kOffV, sP = base + kOffP;
+  const uint32_t sQ = base + kOffQ, sP = base + kOffP;
   const uint32_t stage0 = base + kOffStage;
-  const uint32_t bar_stage0 = base + kOffBar, bar_s = base + kOffBar + 16, bar_o = base + kOffBar + 24;
-  const uint32_t tslot = base + kOffBar + 32;
+  const uint32_t bars = base + kOffBar;
+  const uint32_t tslot = base + kOffSlot;
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem_raw + (base + kOffAbort - raw));
+  auto khi = [&](int s) { return base + kOffKhi + s * kKBytes; };
+  auto klo = [&](int s) { return base + kOffKlo + s * kKBytes; };
+  auto vop = [&](int s) { return base + kOffV + s * kVBytes; };
+  auto stage_full = [&](int s) { return bars + 8u * (0 + s); };
+  auto stage_empty = [&](int s) { return bars + 8u * (2 + s); };
+  auto kv_full = [&](int s) { return bars + 8u * (4 + s); };
+  auto kv_empty = [&](int s) { return bars + 8u * (6 + s); };
+  auto s_full = [&](int s) { return bars + 8u * (8 + s); };
+  auto s_empty = [&](int s) { return bars + 8u * (10 + s); };
+  const uint32_t p_full = bars + 8u * 12, p_empty = bars + 8u * 13;
 
-  const int tid = threadIdx.x, warp = tid >> 5;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int G = p.group, H = p.num_kv_heads;
   const int Tq = 128 / G;                                   // tokens per query tile
   const int b = blockIdx.y, h = blockIdx.z;
@@ -135,7 +167,7 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(const PrefillPara
   const int n = c_hi - c_lo;
   const int t0 = tile * Tq;
   if (n <= 0 || t0 >= n) return;
-  int L = __ldg(p.seq_lens + b);
+  const int L = __ldg(p.seq_lens + b);
   if (c_lo < 0 || c_hi > p.n_tokens || L < n || L > p.max_pages * kPage) {
     if (tid == 0 && t0 == 0 && h == 0) flag_error(p.err, S4KV_EFLAG_SEQ_LEN);
     return;
@@ -147,334 +179,361 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(const PrefillPara
   const int n_ktiles = (n_keys + kKeyTile - 1) / kKeyTile;
   const int nfull = L / kPage;
   const int np = (L + kPage - 1) / kPage;
-  const int32_t *bt = p.block_tables + static_cast<long>(b) * p.max_pages;
-  const uint8_t *head_pool = p.pool + static_cast<long>(h) * kBlockBytes;
-  const long long page_stride = static_cast<long long>(H) * kBlockBytes;
 
-  // ---- setup: tensor memory (S at columns 0..127, O at 128..255), barriers
+  // ---- setup: tensor memory (S buffers at columns 0 and 64, O at 128), barriers
   if (warp == 0) {
     tc05::tmem_alloc(tslot, 256);
     tc05::tmem_relinquish();
     tc05::fence_before_sync();
   }
   if (tid == 0) {
-    mbar_init(bar_stage0, 1);
-    mbar_init(bar_stage0 + 8, 1);
-    mbar_init(bar_s, 1);
-    mbar_init(bar_o, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(stage_full(s), 1);
+      mbar_init(stage_empty(s), kDqThreads);
+      mbar_init(kv_full(s), kDqThreads);
+      mbar_init(kv_empty(s), 1);
+      mbar_init(s_full(s), 1);
+      mbar_init(s_empty(s), 32 * kSoftmaxWarps);
+    }
+    mbar_init(p_full, 32 * kSoftmaxWarps);
+    mbar_init(p_empty, 1);
+    *abort_flag = 0;
     fence_barrier_init();
   }
-
-  // producer: the quantized pages of key tile kt into staging buffer kt & 1
-  int fetched = 0;  // tiles fetched so far (thread 0)
-  auto fetch = [&](int kt) {
-    ++fetched;
-    const int s = kt & 1;
-    const uint32_t bar = bar_stage0 + 8u * s, dst = stage0 + s * kStageBytes;
-    const int pg0 = kt * kPagesPerTile;
-    const int q = max(0, min(kPagesPerTile, nfull - pg0));
-    mbar_arrive_expect_tx(bar, static_cast<uint32_t>(q) * kBlockBytes);
-    for (int k = 0; k < q; ++k) {
-      int phys = __ldg(bt + pg0 + k);
-      if (static_cast<unsigned>(phys) >= static_cast<unsigned>(p.num_pages)) {
-        flag_error(p.err, S4KV_EFLAG_PAGE_RANGE);
-        phys = 0;
-      }
-      bulk_copy_g2s(dst + k * kBlockBytes, head_pool + phys * page_stride, kBlockBytes, bar);
-    }
-  };
-  __syncthreads();
-  if (tid == 0) fetch(0);
-
-  // ---- Q tile: row r = (token r / G, head r % G); rows >= rows are zero.
-  // Four threads per row, four 16-byte chunks each.
-  {
-    const int r = tid >> 2, cq = tid & 3;
+  // ---- Q tile: row r = (token r / G, head r % G); rows >= rows are zero
+  for (int ch = tid; ch < 128 * 16; ch += kThreadsP) {
+    const int r = ch >> 4, c = ch & 15;
     const int tl = r / G, g = r - tl * G;
-    const uint4 *src = reinterpret_cast<const uint4 *>(
-        p.q + (static_cast<long>(c_lo + t0 + tl) * p.num_q_heads + h * G + g) * kHeadDim);
-#pragma unroll
-    for (int c = 4 * cq; c < 4 * cq + 4; ++c) {
-      uint4 v = make_uint4(0, 0, 0, 0);
-      if (r < rows) v = __ldg(src + c);
-      sts128(sQ + tc05::sw128_offset(r, 8 * c, 128), v);
-    }
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (r < rows)
+      v = __ldg(reinterpret_cast<const uint4 *>(
+                    p.q + (static_cast<long>(c_lo + t0 + tl) * p.num_q_heads + h * G + g) * kHeadDim) + c);
+    sts128(sQ + tc05::sw128_offset(r, 8 * c, 128), v);
   }
-
+  fence_proxy_async();
+  __syncthreads();
   tc05::fence_after_sync();
   const uint32_t tmem = lds32_at(tslot);
-  const uint32_t tS = tmem, tO = tmem + 128;
-
-  // ---- dequant mapping: 64 threads per page of the key tile; thread word
-  // w = widx + 64 e (e = 0..3) of a code region, i.e. MMA lane (w % 128) / 4
-  // and tile 4 (w / 128) + w % 4
-  const int dpage = tid >> 6, widx = tid & 63;
-  const int dq = widx & 3, dlane0 = widx >> 2;
-  // swizzled store offsets of this thread's words (they do not change from
-  // tile to tile): keys row 16 dpage + dn (and + 8 rows = + 1024 bytes),
-  // channels 32 di + 4 t; values rows cb, cb + 1, keys 16 dpage + 2 di (+ 8)
-  uint32_t kofs[4], vofs[4][4];
-#pragma unroll
-  for (int e = 0; e < 4; ++e) {
-    const int lane = dlane0 + 16 * (e & 1), t = 4 * (e >> 1) + dq;
-    const int dn = lane >> 2, di = lane & 3;
-    kofs[e] = tc05::sw128_offset(dpage * 16 + dn, 32 * di + 4 * t, 128);
-    const int cb = 32 * (t >> 1) + 4 * dn + 2 * (t & 1);
-    const int key = dpage * 16 + 2 * di;
-    vofs[e][0] = tc05::sw128_offset(cb, key, 128);
-    vofs[e][1] = tc05::sw128_offset(cb + 1, key, 128);
-    vofs[e][2] = tc05::sw128_offset(cb, key + 8, 128);
-    vofs[e][3] = tc05::sw128_offset(cb + 1, key + 8, 128);
-  }
-
-  // ---- softmax mapping: warp w reads tensor-memory lanes 32 (w % 4) ..
-  // (row r = 32 (w % 4) + lane) and key columns 32 (w / 4) .. + 31
-  const int qd = warp & 3, cq = warp >> 2;
-  const int row = 32 * qd + (tid & 31);
-  const uint32_t lane_base = static_cast<uint32_t>(32 * qd) << 16;
-  const bool row_ok = row < rows;
-  const int pos_row = pos_first + (row_ok ? row / G : 0);
-  float ref = -INFINITY;
-  float2 lsum = make_float2(0.f, 0.f);  // this thread's columns only
-  const float sl2 = p.scale_log2;
-  float *red = reinterpret_cast<float *>(smem_raw + (base + kOffRed - raw));  // [4][128]
-
+  const uint32_t tO = tmem + 128;
+  auto tS = [&](int s) { return tmem + 64u * s; };
   bool failed = false;
-  int kt = 0;
-  for (; kt < n_ktiles; ++kt) {
-    const int s = kt & 1;
-    if (tid == 0 && kt + 1 < n_ktiles) fetch(kt + 1);
-    if (!wait_bounded(bar_stage0 + 8u * s, (kt >> 1) & 1)) failed = true;
-    if (__syncthreads_or(failed)) {
-      failed = true;
-      break;
+  auto fail = [&]() {
+    failed = true;
+    *abort_flag = 1;
+  };
+
+  if (warp == kProducerWarp) {
+    // ---------------------------------------------------------- producer
+    if (lane == 0) {
+      const int32_t *bt = p.block_tables + static_cast<long>(b) * p.max_pages;
+      const uint8_t *head_pool = p.pool + static_cast<long>(h) * kBlockBytes;
+      const long long page_stride = static_cast<long long>(H) * kBlockBytes;
+      int issued = 0;
+      for (int kt = 0; kt < n_ktiles && !failed; ++kt) {
+        const int s = kt & 1;
+        if (kt >= 2 && !wait_bounded(stage_empty(s), ((kt >> 1) - 1) & 1, abort_flag)) {
+          fail();
+          break;
+        }
+        ++issued;
+        const int pg0 = kt * kPagesPerTile;
+        const int q = max(0, min(kPagesPerTile, nfull - pg0));
+        mbar_arrive_expect_tx(stage_full(s), static_cast<uint32_t>(q) * kBlockBytes);
+        for (int k = 0; k < q; ++k) {
+          int phys = __ldg(bt + pg0 + k);
+          if (static_cast<unsigned>(phys) >= static_cast<unsigned>(p.num_pages)) {
+            flag_error(p.err, S4KV_EFLAG_PAGE_RANGE);
+            phys = 0;
+          }
+          bulk_copy_g2s(stage0 + s * kStageBytes + k * kBlockBytes, head_pool + phys * page_stride, kBlockBytes,
+                        stage_full(s));
+        }
+      }
+      // before the CTA exits, the copies in flight must have landed (bounded
+      // by time only, also after an abort)
+      const volatile int no_abort = 0;
+      for (int kt = max(0, issued - 2); kt < issued; ++kt) wait_bounded(stage_full(kt & 1), (kt >> 1) & 1, &no_abort);
     }
-    const uint32_t stg = stage0 + s * kStageBytes;
-    const int pg = kt * kPagesPerTile + dpage;
-    const uint32_t blk = stg + dpage * kBlockBytes;
-    const int rres = (pg == nfull && pg < np) ? L - nfull * kPage : 0;  // residual rows of a partial page
+  } else if (warp >= kSoftmaxWarps && warp < kSoftmaxWarps + kDequantWarps) {
+    // -------------------------------------------------------- dequantizer
+    const int t = tid - 32 * kSoftmaxWarps;  // 0 .. 255
+    const int dpage = t >> 6, widx = t & 63;
+    const int dq = widx & 3, dlane0 = widx >> 2;
+    // swizzled store offsets of this thread's words (the same for every
+    // tile): keys rows 16 dpage + dn (and + 8 rows = + 1024 bytes), channels
+    // 32 di + 4 tt; values rows cb, cb + 1, keys 16 dpage + 2 di (+ 8)
+    uint32_t kofs[4], vofs[4][4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int ln = dlane0 + 16 * (e & 1), tt = 4 * (e >> 1) + dq;
+      const int dn = ln >> 2, di = ln & 3;
+      kofs[e] = tc05::sw128_offset(dpage * 16 + dn, 32 * di + 4 * tt, 64);
+      const int cb = 32 * (tt >> 1) + 4 * dn + 2 * (tt & 1);
+      const int key = dpage * 16 + 2 * di;
+      vofs[e][0] = tc05::sw128_offset(cb, key, 128);
+      vofs[e][1] = tc05::sw128_offset(cb + 1, key, 128);
+      vofs[e][2] = tc05::sw128_offset(cb, key + 8, 128);
+      vofs[e][3] = tc05::sw128_offset(cb + 1, key + 8, 128);
+    }
     const long res_base = (static_cast<long>(b) * H + h) * kPage * kHeadDim;
-
-    // ---- keys of tile kt -> sK (hi) and sKlo; S(kt-1) finished before the
-    // softmax of kt-1, so both are free
-    if (pg < nfull) {
+    for (int kt = 0; kt < n_ktiles; ++kt) {
+      const int s = kt & 1;
+      if (!wait_bounded(stage_full(s), (kt >> 1) & 1, abort_flag)) {
+        fail();
+        break;
+      }
+      if (kt >= 2 && !wait_bounded(kv_empty(s), ((kt >> 1) - 1) & 1, abort_flag)) {
+        fail();
+        break;
+      }
+      const uint32_t sKh = khi(s), sKl = klo(s), sV = vop(s);
+      const int pg = kt * kPagesPerTile + dpage;
+      const uint32_t blk = stage0 + s * kStageBytes + dpage * kBlockBytes;
+      if (pg < nfull) {
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int w = widx + 64 * e;
-        const int lane = dlane0 + 16 * (e & 1), t = 4 * (e >> 1) + dq;
-        const int di = lane & 3;
-        uint32_t a0, a1, a2, a3;
-        unpack_codes(lds32_at(blk + kKCodeOff + 4 * w), a0, a1, a2, a3);
-        const int c0 = 32 * di + 4 * t;
-        const uint2 sc = lds64_at(blk + kKScaleOff + 2 * c0);
-        const uint32_t zslot = 16 * t + 2 * di;
-        const uint32_t z01 = lds32_at(blk + kKZeroOff + 2 * zslot);
-        const uint32_t z23 = lds32_at(blk + kKZeroOff + 2 * (zslot + 8));
-        const float2 s01 = __half22float2(u32_as_h2(sc.x)), s23 = __half22float2(u32_as_h2(sc.y));
-        const float2 zf01 = __half22float2(u32_as_h2(z01)), zf23 = __half22float2(u32_as_h2(z23));
-        uint32_t hi0, lo0, hi1, lo1, hi2, lo2, hi3, lo3;
-        split_key(a0, s01, zf01, hi0, lo0);
-        split_key(a1, s01, zf01, hi1, lo1);
-        split_key(a2, s23, zf23, hi2, lo2);
-        split_key(a3, s23, zf23, hi3, lo3);
-        const uint32_t o0 = kofs[e], o1 = kofs[e] + 1024;
-        sts64(sK + o0, hi0, hi2);
-        sts64(sK + o1, hi1, hi3);
-        sts64(sKlo + o0, lo0, lo2);
-        sts64(sKlo + o1, lo1, lo3);
+        for (int e = 0; e < 4; ++e) {
+          const int w = widx + 64 * e;
+          const int ln = dlane0 + 16 * (e & 1), tt = 4 * (e >> 1) + dq;
+          const int di = ln & 3;
+          // keys: tokens dn, dn + 8; channels c0 .. c0 + 3
+          {
+            uint32_t a0, a1, a2, a3;
+            unpack_codes(lds32_at(blk + kKCodeOff + 4 * w), a0, a1, a2, a3);
+            const int c0 = 32 * di + 4 * tt;
+            const uint2 sc = lds64_at(blk + kKScaleOff + 2 * c0);
+            const uint32_t zslot = 16 * tt + 2 * di;
+            const uint32_t z01 = lds32_at(blk + kKZeroOff + 2 * zslot);
+            const uint32_t z23 = lds32_at(blk + kKZeroOff + 2 * (zslot + 8));
+            const float2 s01 = __half22float2(u32_as_h2(sc.x)), s23 = __half22float2(u32_as_h2(sc.y));
+            const float2 zf01 = __half22float2(u32_as_h2(z01)), zf23 = __half22float2(u32_as_h2(z23));
+            uint32_t hi0, lo0, hi1, lo1, hi2, lo2, hi3, lo3;
+            split_key(a0, s01, zf01, hi0, lo0);
+            split_key(a1, s01, zf01, hi1, lo1);
+            split_key(a2, s23, zf23, hi2, lo2);
+            split_key(a3, s23, zf23, hi3, lo3);
+            sts64(sKh + kofs[e], hi0, hi2);
+            sts64(sKh + kofs[e] + 1024, hi1, hi3);
+            sts64(sKl + kofs[e], lo0, lo2);
+            sts64(sKl + kofs[e] + 1024, lo1, lo3);
+          }
+          // values: channels cb, cb + 1; tokens 2 di, 2 di + 1 (+ 8)
+          {
+            uint32_t a0, a1, a2, a3;
+            unpack_codes(lds32_at(blk + kVCodeOff + 4 * w), a0, a1, a2, a3);
+            const int g = tt >> 1;
+            const uint32_t sv_lo = lds32_at(blk + kVScaleOff + 2 * (16 * g + 2 * di));
+            const uint32_t sv_hi = lds32_at(blk + kVScaleOff + 2 * (16 * g + 2 * di + 8));
+            const uint32_t zv_lo = lds32_at(blk + kVZeroOff + 2 * (16 * g + 2 * di));
+            const uint32_t zv_hi = lds32_at(blk + kVZeroOff + 2 * (16 * g + 2 * di + 8));
+            sts32(sV + vofs[e][0], hfma2_u32(a0, sv_lo, zv_lo));
+            sts32(sV + vofs[e][1], hfma2_u32(a1, sv_lo, zv_lo));
+            sts32(sV + vofs[e][2], hfma2_u32(a2, sv_hi, zv_hi));
+            sts32(sV + vofs[e][3], hfma2_u32(a3, sv_hi, zv_hi));
+          }
+        }
+      } else {
+        // the partial last page (fp16 residual rows < L % 16) or no page:
+        // copy the valid rows, zero the rest, so masked keys hold finite values
+        const int rres = (pg == nfull && pg < np) ? L - nfull * kPage : 0;
+        const __half *rk = p.res_k + res_base;
+        const __half *rv = p.res_v + res_base;
+        for (int e = widx; e < kPage * kHeadDim / 2; e += 64) {
+          const int tk = e >> 6, c = 2 * (e & 63);
+          uint32_t kb = 0;
+          if (tk < rres) kb = *reinterpret_cast<const uint32_t *>(rk + tk * kHeadDim + c);
+          const uint32_t ko = tc05::sw128_offset(dpage * 16 + tk, c, 64);
+          sts32(sKh + ko, kb);
+          sts32(sKl + ko, 0u);
+        }
+        for (int e = widx; e < kPage * kHeadDim; e += 64) {
+          const int tk = e >> 7, c = e & 127;
+          uint16_t vb = 0;
+          if (tk < rres) vb = __half_as_ushort(rv[tk * kHeadDim + c]);
+          sts16(sV + tc05::sw128_offset(c, dpage * 16 + tk, 128), vb);
+        }
       }
-    } else {
-      // the partial last page (fp16 residual rows < L % 16) or no page: copy
-      // the valid rows, zero the rest, so masked keys hold finite values
-      const __half *rk = p.res_k + res_base;
-#pragma unroll 4
-      for (int e = widx; e < kPage * kHeadDim / 2; e += 64) {
-        const int tk = e >> 6, c = 2 * (e & 63);
-        uint32_t kb = 0;
-        if (tk < rres) kb = *reinterpret_cast<const uint32_t *>(rk + tk * kHeadDim + c);
-        const uint32_t ko = tc05::sw128_offset(dpage * 16 + tk, c, 128);
-        sts32(sK + ko, kb);
-        sts32(sKlo + ko, 0u);
-      }
+      fence_proxy_async();  // operand writes -> MMA reads; staging reads -> the next bulk copy
+      mbar_arrive(kv_full(s));
+      mbar_arrive(stage_empty(s));
     }
-    fence_proxy_async();
-    tc05::fence_before_sync();
-    __syncthreads();
-
-    // ---- S = Q K_hi^T + Q K_lo^T (overlaps the value dequantization below)
-    if (tid == 0) {
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      auto issue_pv = [&](int k) {  // O += P(k) V(k)
+        const int s = k & 1;
+        if (!wait_bounded(p_full, k & 1, abort_flag)) return false;
+        tc05::fence_after_sync();
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          tc05::mma_f16_ss(tO, tc05::smem_desc_sw128(sP + 32 * j), tc05::smem_desc_sw128(vop(s) + 32 * j), kIdescO,
+                           (k > 0 || j > 0) ? 1u : 0u);
+        tc05::mma_commit(p_empty);
+        tc05::mma_commit(kv_empty(s));
+        return true;
+      };
+      for (int kt = 0; kt < n_ktiles; ++kt) {
+        const int s = kt & 1;
+        if (!wait_bounded(kv_full(s), (kt >> 1) & 1, abort_flag) ||
+            (kt >= 2 && !wait_bounded(s_empty(s), ((kt >> 1) - 1) & 1, abort_flag))) {
+          fail();
+          break;
+        }
+        tc05::fence_after_sync();
+        // S(kt) = Q K_hi^T + Q K_lo^T
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const uint32_t qo = (j >> 2) * (kQBytes / 2) + (j & 3) * 32;
+          const uint32_t ko = (j >> 2) * (kKBytes / 2) + (j & 3) * 32;
+          tc05::mma_f16_ss(tS(s), tc05::smem_desc_sw128(sQ + qo), tc05::smem_desc_sw128(khi(s) + ko), kIdescS,
+                           j > 0 ? 1u : 0u);
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const uint32_t qo = (j >> 2) * (kQBytes / 2) + (j & 3) * 32;
+          const uint32_t ko = (j >> 2) * (kKBytes / 2) + (j & 3) * 32;
+          tc05::mma_f16_ss(tS(s), tc05::smem_desc_sw128(sQ + qo), tc05::smem_desc_sw128(klo(s) + ko), kIdescS, 1u);
+        }
+        tc05::mma_commit(s_full(s));
+        // O += P(kt-1) V(kt-1) while the softmax of kt runs
+        if (kt >= 1 && !issue_pv(kt - 1)) {
+          fail();
+          break;
+        }
+      }
+      if (!failed && !issue_pv(n_ktiles - 1)) fail();
+    }
+  } else {
+    // ---------------------------------------------------- softmax (rows)
+    const int row = tid;  // tensor-memory lane
+    const uint32_t lane_base = static_cast<uint32_t>(32 * warp) << 16;
+    const bool row_ok = row < rows;
+    const int pos_row = pos_first + (row_ok ? row / G : 0);
+    float ref = -INFINITY;
+    float2 lsum = make_float2(0.f, 0.f);
+    const float sl2 = p.scale_log2;
+    for (int kt = 0; kt < n_ktiles; ++kt) {
+      const int s = kt & 1;
+      if (!wait_bounded(s_full(s), (kt >> 1) & 1, abort_flag)) {
+        fail();
+        break;
+      }
       tc05::fence_after_sync();
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        const uint32_t off = (k >> 2) * (kOpBytes / 2) + (k & 3) * 32;
-        tc05::mma_f16_ss(tS, tc05::smem_desc_sw128(sQ + off), tc05::smem_desc_sw128(sK + off), kIdesc,
-                         k > 0 ? 1u : 0u);
+      uint32_t v[64];
+      {
+        uint32_t (&v0)[32] = *reinterpret_cast<uint32_t (*)[32]>(&v[0]);
+        uint32_t (&v1)[32] = *reinterpret_cast<uint32_t (*)[32]>(&v[32]);
+        tc05::tmem_ld32(tS(s) + lane_base, v0);
+        tc05::tmem_ld32(tS(s) + lane_base + 32, v1);
+        tc05::tmem_wait_ld();
       }
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        const uint32_t off = (k >> 2) * (kOpBytes / 2) + (k & 3) * 32;
-        tc05::mma_f16_ss(tS, tc05::smem_desc_sw128(sQ + off), tc05::smem_desc_sw128(sKlo + off), kIdesc, 1u);
-      }
-      tc05::mma_commit(bar_s);
-    }
-
-    // ---- values of tile kt -> sV (transposed), once O += P V of kt-1 is done
-    if (kt > 0 && !wait_bounded(bar_o, (kt - 1) & 1)) failed = true;
-    if (pg < nfull) {
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int w = widx + 64 * e;
-        const int lane = dlane0 + 16 * (e & 1), t = 4 * (e >> 1) + dq;
-        const int di = lane & 3;
-        uint32_t a0, a1, a2, a3;
-        unpack_codes(lds32_at(blk + kVCodeOff + 4 * w), a0, a1, a2, a3);
-        const int g = t >> 1;
-        const uint32_t sv_lo = lds32_at(blk + kVScaleOff + 2 * (16 * g + 2 * di));
-        const uint32_t sv_hi = lds32_at(blk + kVScaleOff + 2 * (16 * g + 2 * di + 8));
-        const uint32_t zv_lo = lds32_at(blk + kVZeroOff + 2 * (16 * g + 2 * di));
-        const uint32_t zv_hi = lds32_at(blk + kVZeroOff + 2 * (16 * g + 2 * di + 8));
-        sts32(sV + vofs[e][0], hfma2_u32(a0, sv_lo, zv_lo));
-        sts32(sV + vofs[e][1], hfma2_u32(a1, sv_lo, zv_lo));
-        sts32(sV + vofs[e][2], hfma2_u32(a2, sv_hi, zv_hi));
-        sts32(sV + vofs[e][3], hfma2_u32(a3, sv_hi, zv_hi));
-      }
-    } else {
-      const __half *rv = p.res_v + res_base;
-#pragma unroll 4
-      for (int e = widx; e < kPage * kHeadDim; e += 64) {
-        const int tk = e >> 7, c = e & 127;
-        uint16_t vb = 0;
-        if (tk < rres) vb = __half_as_ushort(rv[tk * kHeadDim + c]);
-        sts16(sV + tc05::sw128_offset(c, dpage * 16 + tk, 128), vb);
-      }
-    }
-    fence_proxy_async();
-    if (!wait_bounded(bar_s, kt & 1)) failed = true;
-    if (__syncthreads_or(failed)) {
-      failed = true;
-      break;
-    }
-    tc05::fence_after_sync();
-
-    // ---- online softmax: row `row`, key columns 32 cq .. 32 cq + 31.  A key
-    // tile wholly before the tile's first query position needs no mask
-    // (rows past the tile's last row hold q = 0, so finite logits, and are
-    // never written out).
-    {
-      const int key0 = kt * kKeyTile + 32 * cq;
-      const bool full = kt * kKeyTile + kKeyTile - 1 <= pos_first;
-      uint32_t v[32];
-      tc05::tmem_ld32(tS + lane_base + 32 * cq, v);
-      tc05::tmem_wait_ld();
+      tc05::fence_before_sync();
+      mbar_arrive(s_empty(s));
+      // a key tile wholly before the tile's first query position needs no
+      // mask (rows past the last row hold q = 0: finite logits, never written)
+      const int key0 = kt * kKeyTile;
+      const bool full = key0 + kKeyTile - 1 <= pos_first;
       float mx = -INFINITY;
       if (full) {
 #pragma unroll
-        for (int j = 0; j < 32; ++j) mx = fmaxf(mx, __uint_as_float(v[j]));
-        mx *= sl2;
+        for (int j = 0; j < 64; ++j) mx = fmaxf(mx, __uint_as_float(v[j]));
       } else {
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
+        for (int j = 0; j < 64; ++j) {
           const bool ok = row_ok && key0 + j <= pos_row;
           const float x = ok ? __uint_as_float(v[j]) : -INFINITY;
           v[j] = __float_as_uint(x);
           mx = fmaxf(mx, x);
         }
-        mx *= sl2;
       }
-      red[cq * 128 + row] = mx;
-      __syncthreads();
-      mx = fmaxf(fmaxf(red[row], red[128 + row]), fmaxf(red[256 + row], red[384 + row]));
+      mx *= sl2;
       // the reference moves only when the row maximum passes it by > 8
       const bool move = mx > ref + kSlack;
       const float new_ref = move ? mx : ref;
       const float alpha = move ? fast_exp2(ref - new_ref) : 1.0f;  // 0 when ref was -inf
-      if (__any_sync(0xFFFFFFFFu, move) && kt > 0) {
-        // this warp's rows, columns 32 cq .. of O (warp-wide tensor-memory access)
-        uint32_t o[32];
-        tc05::tmem_ld32(tO + lane_base + 32 * cq, o);
-        tc05::tmem_wait_ld();
-        const float2 a2 = make_float2(alpha, alpha);
-#pragma unroll
-        for (int j = 0; j < 32; j += 2) {
-          const float2 r = mul2(make_float2(__uint_as_float(o[j]), __uint_as_float(o[j + 1])), a2);
-          o[j] = __float_as_uint(r.x);
-          o[j + 1] = __float_as_uint(r.y);
+      // O and P are free once O += P(kt-1) V(kt-1) has completed
+      if (kt >= 1) {
+        if (!wait_bounded(p_empty, (kt - 1) & 1, abort_flag)) {
+          fail();
+          break;
         }
-        tc05::tmem_st32(tO + lane_base + 32 * cq, o);
-        tc05::tmem_wait_st();
+        tc05::fence_after_sync();
+        if (__any_sync(0xFFFFFFFFu, move)) {
+          const float2 a2 = make_float2(alpha, alpha);
+#pragma unroll 1
+          for (int c = 0; c < 4; ++c) {
+            uint32_t o[32];
+            tc05::tmem_ld32(tO + lane_base + 32 * c, o);
+            tc05::tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 32; j += 2) {
+              const float2 r = mul2(make_float2(__uint_as_float(o[j]), __uint_as_float(o[j + 1])), a2);
+              o[j] = __float_as_uint(r.x);
+              o[j + 1] = __float_as_uint(r.y);
+            }
+            tc05::tmem_st32(tO + lane_base + 32 * c, o);
+          }
+          tc05::tmem_wait_st();
+        }
       }
       lsum = mul2(lsum, make_float2(alpha, alpha));
       ref = new_ref;
-      // weights exp2(s * scale - ref); masked logits are -inf and give 0
-      // (ref is finite for every row with a valid key; a row without one has
-      // only masked logits, and its -inf reference is replaced by 0 so that
+      // weights exp2(s * scale - ref); masked logits are -inf and give 0 (a
+      // row without a valid key keeps a -inf reference, replaced by 0 so that
       // no inf - inf appears)
       const float nref = ref == -INFINITY ? 0.f : -ref;
       const float2 sc = make_float2(sl2, sl2), nr = make_float2(nref, nref);
-      uint32_t hp[16];
 #pragma unroll
-      for (int j = 0; j < 32; j += 2) {
-        const float2 x = fma2(make_float2(__uint_as_float(v[j]), __uint_as_float(v[j + 1])), sc, nr);
-        const __half2 ph = __floats2half2_rn(fast_exp2(x.x), fast_exp2(x.y));
-        // the row sum takes the fp16 weights the MMA multiplies with, so a
-        // dominant key's value comes through exactly
-        lsum = add2(lsum, __half22float2(ph));
-        hp[j >> 1] = h2_as_u32(ph);
+      for (int q8 = 0; q8 < 8; ++q8) {
+        uint32_t hp[4];
+#pragma unroll
+        for (int j = 0; j < 8; j += 2) {
+          const int k = 8 * q8 + j;
+          const float2 x = fma2(make_float2(__uint_as_float(v[k]), __uint_as_float(v[k + 1])), sc, nr);
+          const __half2 ph = __floats2half2_rn(fast_exp2(x.x), fast_exp2(x.y));
+          // the row sum takes the fp16 weights the MMA multiplies with
+          lsum = add2(lsum, __half22float2(ph));
+          hp[j >> 1] = h2_as_u32(ph);
+        }
+        sts128(sP + tc05::sw128_offset(row, 8 * q8, 128), make_uint4(hp[0], hp[1], hp[2], hp[3]));
       }
-#pragma unroll
-      for (int q4 = 0; q4 < 4; ++q4)
-        sts128(sP + tc05::sw128_offset(row, 32 * cq + 8 * q4, 128),
-               make_uint4(hp[4 * q4], hp[4 * q4 + 1], hp[4 * q4 + 2], hp[4 * q4 + 3]));
+      fence_proxy_async();
+      tc05::fence_before_sync();
+      mbar_arrive(p_full);
     }
-    fence_proxy_async();
-    tc05::fence_before_sync();
-    __syncthreads();
-
-    // ---- O += P V (overlaps the next tile's key dequantization)
-    if (tid == 0) {
+    // ---- out = O / l once the last O += P V has completed
+    if (!failed && !wait_bounded(p_empty, (n_ktiles - 1) & 1, abort_flag)) fail();
+    if (!failed) {
       tc05::fence_after_sync();
+      const float l = lsum.x + lsum.y;
+      const float inv = row_ok && l > 0.f ? 1.0f / l : 0.f;
+      const int tl = row / G, g = row - (row / G) * G;
+      __half *dst = p.out + (static_cast<long>(c_lo + t0 + tl) * p.num_q_heads + h * G + g) * kHeadDim;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        uint32_t o[32];
+        tc05::tmem_ld32(tO + lane_base + 32 * c, o);
+        tc05::tmem_wait_ld();
+        if (row_ok) {
+          uint32_t hv[16];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        const uint32_t off = (k >> 2) * (kOpBytes / 2) + (k & 3) * 32;
-        tc05::mma_f16_ss(tO, tc05::smem_desc_sw128(sP + off), tc05::smem_desc_sw128(sV + off), kIdesc,
-                         (kt > 0 || k > 0) ? 1u : 0u);
+          for (int j = 0; j < 32; j += 2)
+            hv[j >> 1] = h2_as_u32(__floats2half2_rn(__uint_as_float(o[j]) * inv, __uint_as_float(o[j + 1]) * inv));
+          uint4 *o4 = reinterpret_cast<uint4 *>(dst + 32 * c);
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4)
+            o4[q4] = make_uint4(hv[4 * q4], hv[4 * q4 + 1], hv[4 * q4 + 2], hv[4 * q4 + 3]);
+        }
       }
-      tc05::mma_commit(bar_o);
     }
   }
-  if (!failed && !wait_bounded(bar_o, (n_ktiles - 1) & 1)) failed = true;
-  failed = __syncthreads_or(failed);
-  tc05::fence_after_sync();
 
-  if (!failed) {
-    // ---- out = O / l: l is the sum of the four column quarters' partial sums
-    red[cq * 128 + row] = lsum.x + lsum.y;
-    __syncthreads();
-    const float l = (red[row] + red[128 + row]) + (red[256 + row] + red[384 + row]);
-    const float inv = row_ok && l > 0.f ? 1.0f / l : 0.f;
-    uint32_t v[32];
-    tc05::tmem_ld32(tO + lane_base + 32 * cq, v);
-    tc05::tmem_wait_ld();
-    if (row_ok) {
-      const int tl = row / G, g = row - tl * G;
-      __half *dst = p.out + (static_cast<long>(c_lo + t0 + tl) * p.num_q_heads + h * G + g) * kHeadDim + 32 * cq;
-      uint32_t hv[16];
-#pragma unroll
-      for (int j = 0; j < 32; j += 2)
-        hv[j >> 1] = h2_as_u32(__floats2half2_rn(__uint_as_float(v[j]) * inv, __uint_as_float(v[j + 1]) * inv));
-      uint4 *o4 = reinterpret_cast<uint4 *>(dst);
-#pragma unroll
-      for (int q4 = 0; q4 < 4; ++q4) o4[q4] = make_uint4(hv[4 * q4], hv[4 * q4 + 1], hv[4 * q4 + 2], hv[4 * q4 + 3]);
-    }
-  } else if (tid == 0) {
-    flag_error(p.err, S4KV_EFLAG_TIMEOUT);
-    // wait (bounded) for the bulk copies still in flight before the CTA exits
-    for (int f = kt; f < fetched; ++f) wait_bounded(bar_stage0 + 8u * (f & 1), (f >> 1) & 1);
-  }
-
+  if (failed) flag_error(p.err, S4KV_EFLAG_TIMEOUT);
   tc05::fence_before_sync();
   __syncthreads();
-  if (warp == 0) tc05::tmem_dealloc(tmem, 256);
+  if (warp == 0) {
+    tc05::fence_after_sync();
+    tc05::tmem_dealloc(tmem, 256);
+  }
 }
 
 size_t prefill_smem_bytes() { return kSmemBytes; }
