@@ -1,4 +1,4 @@
-"""CPU oracle for the int4 KIVI paged KV cache -- TEST INFRASTRUCTURE ONLY.
+"""CPU oracle for the int4 (and int8) KIVI paged KV cache -- TEST INFRASTRUCTURE ONLY.
 
 Thin ctypes/numpy wrapper around ``s4kv_oracle.c`` (plain C, single thread).
 Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
@@ -67,20 +67,33 @@ def lib():
         L.s4kv_ref_append.restype = i32
         L.s4kv_ref_dequant_page.argtypes = [P, i32, i32, i32, P, P]
         L.s4kv_ref_dequant_page.restype = i32
-        L.s4kv_ref_decode_attention.argtypes = [P, P, P, i32, i32, P, i32, P, P, i32, i32, f64, i32, P]
+        L.s4kv_ref_decode_attention.argtypes = [P, P, P, i32, i32, P, i32, P, P, i32, i32, f64, i32, P, i32]
         L.s4kv_ref_decode_attention.restype = i32
         L.s4kv_ref_attention_fp16.argtypes = [P, P, P, i32, P, i32, i32, f64, P]
-        L.s4kv_ref_prefill_attention.argtypes = [P, P, P, i32, i32, P, i32, P, P, P, i32, i32, f64, P]
+        L.s4kv_ref_prefill_attention.argtypes = [P, P, P, i32, i32, P, i32, P, P, P, i32, i32, f64, P, i32]
         L.s4kv_ref_prefill_attention.restype = i32
-        L.s4kv_ref_gather_pages.argtypes = [P, i32, i32, P, i32, P]
+        L.s4kv_ref_gather_pages.argtypes = [P, i32, i32, P, i32, P, i32]
         L.s4kv_ref_gather_pages.restype = i32
-        L.s4kv_ref_scatter_pages.argtypes = [P, i32, i32, P, i32, P]
+        L.s4kv_ref_scatter_pages.argtypes = [P, i32, i32, P, i32, P, i32]
         L.s4kv_ref_scatter_pages.restype = i32
-        L.s4kv_ref_copy_pages.argtypes = [P, i32, i32, P, P, i32]
+        L.s4kv_ref_copy_pages.argtypes = [P, i32, i32, P, P, i32, i32]
         L.s4kv_ref_copy_pages.restype = i32
         L.s4kv_ref_fork_residual.argtypes = [P, P, i32, i32, P, P, i32]
         L.s4kv_ref_fork_residual.restype = i32
         L.s4kv_ref_attention_fp16.restype = i32
+        L.s4kv_ref_quantize_group_bits.argtypes = [P, i32, i32, P, i32, i32, P, P]
+        L.s4kv_ref_quantize_group_bits.restype = f32
+        L.s4kv_ref_code_offset8.argtypes = [i32, i32, i32]
+        L.s4kv_ref_code_offset8.restype = ctypes.c_long
+        L.s4kv_ref_quantize_page_bits.argtypes = [P, P, P, i32]
+        L.s4kv_ref_unpack_codes_bits.argtypes = [P, P, P, i32]
+        L.s4kv_ref_dequant_block_bits.argtypes = [P, P, P, i32]
+        L.s4kv_ref_block_bytes_bits.argtypes = [i32]
+        L.s4kv_ref_block_bytes_bits.restype = ctypes.c_long
+        L.s4kv_ref_append_bits.argtypes = [P, P, P, i32, i32, i32, P, P, i32, P, P, P, P, i32, i32, i32]
+        L.s4kv_ref_append_bits.restype = i32
+        L.s4kv_ref_dequant_page_bits.argtypes = [P, i32, i32, i32, P, P, i32]
+        L.s4kv_ref_dequant_page_bits.restype = i32
         _lib = L
         del i64
     return _lib
@@ -142,33 +155,50 @@ def key_zero_slot(c: int) -> int:
     return int(lib().s4kv_ref_key_zero_slot(int(c)))
 
 
-def quantize_page(kp, vp) -> np.ndarray:
-    """fp16 K, V [16][128] of one page and kv head -> 2816-byte block."""
+def quantize_group_bits(x, bits: int) -> tuple[np.ndarray, int, int, float]:
+    """As quantize_group with (1 << bits) - 1 levels (bits = 4 or 8)."""
+    xb = _u16(np.asarray(x, dtype=np.float16) if not isinstance(x, np.ndarray) or x.dtype != np.uint16 else x)
+    n = xb.size
+    codes = np.zeros(n, np.uint8)
+    sh = np.zeros(1, np.uint16)
+    zh = np.zeros(1, np.uint16)
+    s = lib().s4kv_ref_quantize_group_bits(_p(xb), n, 1, _p(codes), 1, int(bits), _p(sh), _p(zh))
+    return codes, int(sh[0]), int(zh[0]), float(s)
+
+
+def code_offset8(is_value: bool, t: int, c: int) -> int:
+    """Byte offset of (token t, channel c) in an 8-bit code region."""
+    return int(lib().s4kv_ref_code_offset8(1 if is_value else 0, int(t), int(c)))
+
+
+def quantize_page(kp, vp, bits: int = 4) -> np.ndarray:
+    """fp16 K, V [16][128] of one page and kv head -> block (2816 bytes for
+    4-bit codes)."""
     kb = _u16(kp).reshape(PAGE, HEAD_DIM)
     vb = _u16(vp).reshape(PAGE, HEAD_DIM)
-    blk = np.zeros(BLOCK_BYTES, np.uint8)
-    lib().s4kv_ref_quantize_page(_p(np.ascontiguousarray(kb)), _p(np.ascontiguousarray(vb)), _p(blk))
+    blk = np.zeros(block_bytes(bits), np.uint8)
+    lib().s4kv_ref_quantize_page_bits(_p(np.ascontiguousarray(kb)), _p(np.ascontiguousarray(vb)), _p(blk), bits)
     return blk
 
 
-def unpack_codes(block: np.ndarray) -> tuple[np.ndarray, np.ndarray]:
+def unpack_codes(block: np.ndarray, bits: int = 4) -> tuple[np.ndarray, np.ndarray]:
     block = np.ascontiguousarray(block, dtype=np.uint8)
     kc = np.zeros((PAGE, HEAD_DIM), np.uint8)
     vc = np.zeros((PAGE, HEAD_DIM), np.uint8)
-    lib().s4kv_ref_unpack_codes(_p(block), _p(kc), _p(vc))
+    lib().s4kv_ref_unpack_codes_bits(_p(block), _p(kc), _p(vc), bits)
     return kc, vc
 
 
-def dequant_block(block: np.ndarray) -> tuple[np.ndarray, np.ndarray]:
+def dequant_block(block: np.ndarray, bits: int = 4) -> tuple[np.ndarray, np.ndarray]:
     block = np.ascontiguousarray(block, dtype=np.uint8)
     k = np.zeros((PAGE, HEAD_DIM), np.float32)
     v = np.zeros((PAGE, HEAD_DIM), np.float32)
-    lib().s4kv_ref_dequant_block(_p(block), _p(k), _p(v))
+    lib().s4kv_ref_dequant_block_bits(_p(block), _p(k), _p(v), bits)
     return k, v
 
 
-def block_bytes() -> int:
-    return int(lib().s4kv_ref_block_bytes())
+def block_bytes(bits: int = 4) -> int:
+    return int(lib().s4kv_ref_block_bytes_bits(int(bits)))
 
 
 def kv_payload_bytes(layers, kv_heads, head_dim, tokens, bytes_per_elem) -> float:
@@ -178,14 +208,17 @@ def kv_payload_bytes(layers, kv_heads, head_dim, tokens, bytes_per_elem) -> floa
 # ----------------------------------------------------------------- cache --
 
 class OracleCache:
-    """Host copy of the paged cache: pool u8 [NP][Hkv][2816], residual fp16
-    bits [max_seqs][Hkv][16][128] for K and V."""
+    """Host copy of the paged cache: pool u8 [NP][Hkv][block bytes] (2816 for
+    4-bit codes, 4864 for 8-bit), residual fp16 bits [max_seqs][Hkv][16][128]
+    for K and V."""
 
-    def __init__(self, num_pages: int, num_kv_heads: int, max_seqs: int):
+    def __init__(self, num_pages: int, num_kv_heads: int, max_seqs: int, bits: int = 4):
+        assert bits in (4, 8)
+        self.bits = bits
         self.num_pages = num_pages
         self.num_kv_heads = num_kv_heads
         self.max_seqs = max_seqs
-        self.pool = np.zeros((num_pages, num_kv_heads, BLOCK_BYTES), np.uint8)
+        self.pool = np.zeros((num_pages, num_kv_heads, block_bytes(bits)), np.uint8)
         self.res_k = np.zeros((max_seqs, num_kv_heads, PAGE, HEAD_DIM), np.uint16)
         self.res_v = np.zeros((max_seqs, num_kv_heads, PAGE, HEAD_DIM), np.uint16)
 
@@ -198,16 +231,16 @@ class OracleCache:
         bt = np.ascontiguousarray(block_tables, dtype=np.int32)
         batch, max_pages = bt.shape
         n_tokens = int(cu[-1]) if cu.size else 0
-        return int(lib().s4kv_ref_append(
+        return int(lib().s4kv_ref_append_bits(
             _p(self.pool), _p(self.res_k), _p(self.res_v), self.num_pages,
             self.num_kv_heads, self.max_seqs, _p(kb), _p(vb), n_tokens, _p(sm),
-            _p(cu), _p(sl), _p(bt), batch, max_pages))
+            _p(cu), _p(sl), _p(bt), batch, max_pages, self.bits))
 
     def dequant_page(self, physical_page: int) -> tuple[np.ndarray, np.ndarray]:
         ok = np.zeros((self.num_kv_heads, PAGE, HEAD_DIM), np.float32)
         ov = np.zeros((self.num_kv_heads, PAGE, HEAD_DIM), np.float32)
-        rc = lib().s4kv_ref_dequant_page(_p(self.pool), self.num_pages, self.num_kv_heads,
-                                         physical_page, _p(ok), _p(ov))
+        rc = lib().s4kv_ref_dequant_page_bits(_p(self.pool), self.num_pages, self.num_kv_heads,
+                                              physical_page, _p(ok), _p(ov), self.bits)
         if rc != 0:
             raise ValueError(f"dequant_page rc={rc}")
         return ok, ov
@@ -225,16 +258,17 @@ class OracleCache:
         rc = lib().s4kv_ref_decode_attention(
             _p(self.pool), _p(self.res_k), _p(self.res_v), self.num_pages,
             self.num_kv_heads, _p(qb), num_q_heads, _p(sl), _p(bt), batch,
-            bt.shape[1], float(sm_scale), 1 if use_double else 0, _p(out))
+            bt.shape[1], float(sm_scale), 1 if use_double else 0, _p(out), self.bits)
         if rc != 0:
             raise ValueError(f"decode_attention rc={rc}")
         return out
 
     def gather_pages(self, pages) -> np.ndarray:
-        """Page records of the listed physical pages: u8 [n][kv_heads][2816]."""
+        """Page records of the listed physical pages: u8 [n][kv_heads][block bytes]."""
         pg = np.ascontiguousarray(pages, dtype=np.int32)
-        out = np.zeros((len(pg), self.num_kv_heads, BLOCK_BYTES), np.uint8)
-        rc = lib().s4kv_ref_gather_pages(_p(self.pool), self.num_pages, self.num_kv_heads, _p(pg), len(pg), _p(out))
+        out = np.zeros((len(pg), self.num_kv_heads, block_bytes(self.bits)), np.uint8)
+        rc = lib().s4kv_ref_gather_pages(_p(self.pool), self.num_pages, self.num_kv_heads, _p(pg), len(pg), _p(out),
+                                        self.bits)
         if rc != 0:
             raise ValueError(f"gather_pages rc={rc}")
         return out
@@ -242,14 +276,16 @@ class OracleCache:
     def scatter_pages(self, pages, records) -> None:
         pg = np.ascontiguousarray(pages, dtype=np.int32)
         rec = np.ascontiguousarray(records, dtype=np.uint8)
-        rc = lib().s4kv_ref_scatter_pages(_p(self.pool), self.num_pages, self.num_kv_heads, _p(pg), len(pg), _p(rec))
+        rc = lib().s4kv_ref_scatter_pages(_p(self.pool), self.num_pages, self.num_kv_heads, _p(pg), len(pg), _p(rec),
+                                         self.bits)
         if rc != 0:
             raise ValueError(f"scatter_pages rc={rc}")
 
     def copy_pages(self, src_pages, dst_pages) -> None:
         s_ = np.ascontiguousarray(src_pages, dtype=np.int32)
         d_ = np.ascontiguousarray(dst_pages, dtype=np.int32)
-        rc = lib().s4kv_ref_copy_pages(_p(self.pool), self.num_pages, self.num_kv_heads, _p(s_), _p(d_), len(s_))
+        rc = lib().s4kv_ref_copy_pages(_p(self.pool), self.num_pages, self.num_kv_heads, _p(s_), _p(d_), len(s_),
+                                      self.bits)
         if rc != 0:
             raise ValueError(f"copy_pages rc={rc}")
 
@@ -277,7 +313,7 @@ class OracleCache:
         rc = lib().s4kv_ref_prefill_attention(
             _p(self.pool), _p(self.res_k), _p(self.res_v), self.num_pages,
             self.num_kv_heads, _p(qb), num_q_heads, _p(cu), _p(sl), _p(bt),
-            len(sl), bt.shape[1], float(sm_scale), _p(out))
+            len(sl), bt.shape[1], float(sm_scale), _p(out), self.bits)
         if rc != 0:
             raise ValueError(f"prefill_attention rc={rc}")
         return out

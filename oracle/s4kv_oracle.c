@@ -63,13 +63,18 @@
 #define HEAD_DIM 128
 #define PAGE 16
 #define VGROUP 32
-#define BLOCK_BYTES 2816
-#define KCODE_OFF 0
-#define VCODE_OFF 1024
-#define KSCALE_OFF 2048
-#define KZERO_OFF 2304
-#define VSCALE_OFF 2560
-#define VZERO_OFF 2688
+
+/* Block regions for `bits`-bit codes (4 or 8): K codes, V codes, then the
+ * fp16 metadata (K scale [128], K zero [128], V scale [4][16], V zero
+ * [4][16]); with 4-bit codes this is the 2816-byte block. */
+static long code_bytes(int bits) { return (long)PAGE * HEAD_DIM * bits / 8; }
+static long kcode_off(int bits) { (void)bits; return 0; }
+static long vcode_off(int bits) { return code_bytes(bits); }
+static long kscale_off(int bits) { return 2 * code_bytes(bits); }
+static long kzero_off(int bits) { return kscale_off(bits) + 2 * HEAD_DIM; }
+static long vscale_off(int bits) { return kzero_off(bits) + 2 * HEAD_DIM; }
+static long vzero_off(int bits) { return vscale_off(bits) + 2 * PAGE * (HEAD_DIM / VGROUP); }
+static long block_bytes_of(int bits) { return vzero_off(bits) + 2 * PAGE * (HEAD_DIM / VGROUP); }
 
 /* ---------------------------------------------------------------- fp16 -- */
 
@@ -125,13 +130,14 @@ static int total_less(float a, float b) {
     return 0;
 }
 
-/* Asymmetric int4 quantization of one group of n fp16 values (the KIVI
- * step of [S4KV] "Funktionsweise" 1).  x[k*stride] are the fp16 inputs;
- * codes[k*code_stride] receive the 4-bit codes.  Returns the fp32 scale so
- * that tests can check the rounding bound against it. */
-float s4kv_ref_quantize_group(const uint16_t *x, int n, int stride,
-                              uint8_t *codes, int code_stride,
-                              uint16_t *scale_h, uint16_t *zero_h) {
+/* Asymmetric quantization of one group of n fp16 values to `levels` + 1
+ * codes (the KIVI step of [S4KV] "Funktionsweise" 1: levels = 15 for int4,
+ * 255 for int8).  x[k*stride] are the fp16 inputs; codes[k*code_stride]
+ * receive the codes.  Returns the fp32 scale so that tests can check the
+ * rounding bound against it. */
+static float quantize_group_levels(const uint16_t *x, int n, int stride,
+                                   uint8_t *codes, int code_stride, int levels,
+                                   uint16_t *scale_h, uint16_t *zero_h) {
     float mn = s4kv_ref_half_to_float(x[0]);
     float mx = mn;
     for (int k = 1; k < n; ++k) {
@@ -140,7 +146,7 @@ float s4kv_ref_quantize_group(const uint16_t *x, int n, int stride,
         if (total_less(mx, xv)) mx = xv;
     }
     volatile float range = mx - mn; /* one fp32 rounding */
-    volatile float s = range / 15.0f; /* one fp32 rounding */
+    volatile float s = range / (float)levels; /* one fp32 rounding */
     for (int k = 0; k < n; ++k) {
         float xv = s4kv_ref_half_to_float(x[k * stride]);
         int code = 0;
@@ -149,7 +155,7 @@ float s4kv_ref_quantize_group(const uint16_t *x, int n, int stride,
             volatile float t = d / s;
             float r = nearbyintf(t); /* ties to even */
             if (r < 0.0f) r = 0.0f;
-            if (r > 15.0f) r = 15.0f;
+            if (r > (float)levels) r = (float)levels;
             code = (int)r;
         }
         codes[k * code_stride] = (uint8_t)code;
@@ -160,6 +166,19 @@ float s4kv_ref_quantize_group(const uint16_t *x, int n, int stride,
 }
 
 /* ------------------------------------------------------------- packing -- */
+
+float s4kv_ref_quantize_group(const uint16_t *x, int n, int stride,
+                              uint8_t *codes, int code_stride,
+                              uint16_t *scale_h, uint16_t *zero_h) {
+    return quantize_group_levels(x, n, stride, codes, code_stride, 15, scale_h, zero_h);
+}
+
+/* The same with (1 << bits) - 1 levels (bits = 4 or 8). */
+float s4kv_ref_quantize_group_bits(const uint16_t *x, int n, int stride,
+                                   uint8_t *codes, int code_stride, int bits,
+                                   uint16_t *scale_h, uint16_t *zero_h) {
+    return quantize_group_levels(x, n, stride, codes, code_stride, (1 << bits) - 1, scale_h, zero_h);
+}
 
 /* Position (in halves) of channel c's key zero point: the zero points are
  * stored in the order in which the MMA k axis visits the channels. */
@@ -185,6 +204,26 @@ void s4kv_ref_value_code_slot(int t, int c, int *word, int *nibble) {
     *word = 128 * (m / 4) + 4 * (4 * n + i) + (m % 4);
 }
 
+/* 8-bit codes keep the 4-bit layout's assignment of (token, channel) to MMA
+ * operand fragments -- tile 4*(word/128) + word%4, lane (word/4)%32, and
+ * within the lane's fragment register nibble%4, half nibble/4 -- with bytes
+ * for nibbles: a lane's 8 codes of a tile are 8 consecutive bytes, register
+ * r at bytes 2r (half 0) and 2r + 1 (half 1), and the 16 bytes of tiles
+ * 2m and 2m+1 of one lane sit together, lanes in order. */
+static long byte_offset8(int word, int nibble) {
+    int tile = 4 * (word / 128) + word % 4, lane = (word / 4) % 32;
+    return ((long)(tile / 2) * 32 + lane) * 16 + (tile % 2) * 8 + 2 * (nibble % 4) + nibble / 4;
+}
+
+/* Byte offset of the 8-bit code of (token t, channel c) inside the key
+ * (is_value = 0) or value (1) code region. */
+long s4kv_ref_code_offset8(int is_value, int t, int c) {
+    int w, nb;
+    if (is_value) s4kv_ref_value_code_slot(t, c, &w, &nb);
+    else s4kv_ref_key_code_slot(t, c, &w, &nb);
+    return byte_offset8(w, nb);
+}
+
 static void put_nibble(uint8_t *region, int word, int nibble, int code) {
     uint8_t *byte = region + 4 * word + nibble / 2; /* little-endian word */
     int sh = 4 * (nibble % 2);
@@ -196,6 +235,22 @@ static int get_nibble(const uint8_t *region, int word, int nibble) {
     return (*byte >> (4 * (nibble % 2))) & 0xf;
 }
 
+static void put_code(uint8_t *region, int is_value, int t, int c, int code, int bits) {
+    int w, nb;
+    if (is_value) s4kv_ref_value_code_slot(t, c, &w, &nb);
+    else s4kv_ref_key_code_slot(t, c, &w, &nb);
+    if (bits == 8) region[byte_offset8(w, nb)] = (uint8_t)code;
+    else put_nibble(region, w, nb, code);
+}
+
+static int get_code(const uint8_t *region, int is_value, int t, int c, int bits) {
+    int w, nb;
+    if (is_value) s4kv_ref_value_code_slot(t, c, &w, &nb);
+    else s4kv_ref_key_code_slot(t, c, &w, &nb);
+    if (bits == 8) return region[byte_offset8(w, nb)];
+    return get_nibble(region, w, nb);
+}
+
 static void put_half(uint8_t *p, uint16_t h) { memcpy(p, &h, 2); }
 static uint16_t get_half(const uint8_t *p) {
     uint16_t h;
@@ -203,74 +258,82 @@ static uint16_t get_half(const uint8_t *p) {
     return h;
 }
 
-/* Quantize one full page of one kv head.  kp, vp: fp16 [16][128] rows.
- * Writes the 2816-byte block. */
-void s4kv_ref_quantize_page(const uint16_t *kp, const uint16_t *vp,
-                            uint8_t *block) {
+/* Quantize one full page of one kv head with `bits`-bit codes.  kp, vp:
+ * fp16 [16][128] rows.  Writes the block_bytes_of(bits) block. */
+void s4kv_ref_quantize_page_bits(const uint16_t *kp, const uint16_t *vp,
+                                 uint8_t *block, int bits) {
     uint8_t kc[PAGE][HEAD_DIM], vc[PAGE][HEAD_DIM];
-    memset(block, 0, BLOCK_BYTES);
+    int levels = (1 << bits) - 1;
+    memset(block, 0, (size_t)block_bytes_of(bits));
     /* keys: one group per channel, over the page's 16 tokens */
     for (int c = 0; c < HEAD_DIM; ++c) {
         uint16_t sh, zh;
-        s4kv_ref_quantize_group(kp + c, PAGE, HEAD_DIM, &kc[0][c], HEAD_DIM,
-                                &sh, &zh);
-        put_half(block + KSCALE_OFF + 2 * c, sh);
-        put_half(block + KZERO_OFF + 2 * s4kv_ref_key_zero_slot(c), zh);
+        quantize_group_levels(kp + c, PAGE, HEAD_DIM, &kc[0][c], HEAD_DIM, levels, &sh, &zh);
+        put_half(block + kscale_off(bits) + 2 * c, sh);
+        put_half(block + kzero_off(bits) + 2 * s4kv_ref_key_zero_slot(c), zh);
     }
     /* values: one group per token and 32-channel slice */
     for (int t = 0; t < PAGE; ++t) {
         for (int g = 0; g < HEAD_DIM / VGROUP; ++g) {
             uint16_t sh, zh;
-            s4kv_ref_quantize_group(vp + t * HEAD_DIM + g * VGROUP, VGROUP, 1,
-                                    &vc[t][g * VGROUP], 1, &sh, &zh);
-            put_half(block + VSCALE_OFF + 2 * (g * PAGE + t), sh);
-            put_half(block + VZERO_OFF + 2 * (g * PAGE + t), zh);
+            quantize_group_levels(vp + t * HEAD_DIM + g * VGROUP, VGROUP, 1,
+                                  &vc[t][g * VGROUP], 1, levels, &sh, &zh);
+            put_half(block + vscale_off(bits) + 2 * (g * PAGE + t), sh);
+            put_half(block + vzero_off(bits) + 2 * (g * PAGE + t), zh);
         }
     }
     for (int t = 0; t < PAGE; ++t) {
         for (int c = 0; c < HEAD_DIM; ++c) {
-            int w, nb;
-            s4kv_ref_key_code_slot(t, c, &w, &nb);
-            put_nibble(block + KCODE_OFF, w, nb, kc[t][c]);
-            s4kv_ref_value_code_slot(t, c, &w, &nb);
-            put_nibble(block + VCODE_OFF, w, nb, vc[t][c]);
+            put_code(block + kcode_off(bits), 0, t, c, kc[t][c], bits);
+            put_code(block + vcode_off(bits), 1, t, c, vc[t][c], bits);
         }
     }
+}
+
+void s4kv_ref_quantize_page(const uint16_t *kp, const uint16_t *vp,
+                            uint8_t *block) {
+    s4kv_ref_quantize_page_bits(kp, vp, block, 4);
 }
 
 /* Read back the codes of one block in natural [token][channel] order. */
-void s4kv_ref_unpack_codes(const uint8_t *block, uint8_t *kcodes,
-                           uint8_t *vcodes) {
+void s4kv_ref_unpack_codes_bits(const uint8_t *block, uint8_t *kcodes,
+                                uint8_t *vcodes, int bits) {
     for (int t = 0; t < PAGE; ++t) {
         for (int c = 0; c < HEAD_DIM; ++c) {
-            int w, nb;
-            s4kv_ref_key_code_slot(t, c, &w, &nb);
-            kcodes[t * HEAD_DIM + c] = (uint8_t)get_nibble(block + KCODE_OFF, w, nb);
-            s4kv_ref_value_code_slot(t, c, &w, &nb);
-            vcodes[t * HEAD_DIM + c] = (uint8_t)get_nibble(block + VCODE_OFF, w, nb);
+            kcodes[t * HEAD_DIM + c] = (uint8_t)get_code(block + kcode_off(bits), 0, t, c, bits);
+            vcodes[t * HEAD_DIM + c] = (uint8_t)get_code(block + vcode_off(bits), 1, t, c, bits);
         }
     }
 }
 
+void s4kv_ref_unpack_codes(const uint8_t *block, uint8_t *kcodes,
+                           uint8_t *vcodes) {
+    s4kv_ref_unpack_codes_bits(block, kcodes, vcodes, 4);
+}
+
 /* Dequantize one block: x = code * scale + zero, in fp32 (the product of a
- * 4-bit code and an fp16 scale is exact in fp32, so this is one rounding).
- * kout, vout: fp32 [16][128]. */
-void s4kv_ref_dequant_block(const uint8_t *block, float *kout, float *vout) {
+ * 4- or 8-bit code and an fp16 scale is exact in fp32, so this is one
+ * rounding).  kout, vout: fp32 [16][128]. */
+void s4kv_ref_dequant_block_bits(const uint8_t *block, float *kout, float *vout, int bits) {
     uint8_t kc[PAGE * HEAD_DIM], vc[PAGE * HEAD_DIM];
-    s4kv_ref_unpack_codes(block, kc, vc);
+    s4kv_ref_unpack_codes_bits(block, kc, vc, bits);
     for (int t = 0; t < PAGE; ++t) {
         for (int c = 0; c < HEAD_DIM; ++c) {
-            float ks = s4kv_ref_half_to_float(get_half(block + KSCALE_OFF + 2 * c));
-            float kz = s4kv_ref_half_to_float(get_half(block + KZERO_OFF + 2 * s4kv_ref_key_zero_slot(c)));
+            float ks = s4kv_ref_half_to_float(get_half(block + kscale_off(bits) + 2 * c));
+            float kz = s4kv_ref_half_to_float(get_half(block + kzero_off(bits) + 2 * s4kv_ref_key_zero_slot(c)));
             int g = c / VGROUP;
-            float vs = s4kv_ref_half_to_float(get_half(block + VSCALE_OFF + 2 * (g * PAGE + t)));
-            float vz = s4kv_ref_half_to_float(get_half(block + VZERO_OFF + 2 * (g * PAGE + t)));
+            float vs = s4kv_ref_half_to_float(get_half(block + vscale_off(bits) + 2 * (g * PAGE + t)));
+            float vz = s4kv_ref_half_to_float(get_half(block + vzero_off(bits) + 2 * (g * PAGE + t)));
             volatile float kprod = (float)kc[t * HEAD_DIM + c] * ks;
             volatile float vprod = (float)vc[t * HEAD_DIM + c] * vs;
             kout[t * HEAD_DIM + c] = kprod + kz;
             vout[t * HEAD_DIM + c] = vprod + vz;
         }
     }
+}
+
+void s4kv_ref_dequant_block(const uint8_t *block, float *kout, float *vout) {
+    s4kv_ref_dequant_block_bits(block, kout, vout, 4);
 }
 
 /* --------------------------------------------------------------- cache -- */
@@ -283,6 +346,8 @@ void s4kv_ref_dequant_block(const uint8_t *block, float *kout, float *vout) {
 
 /* Bytes of one (page, kv head) block of this layout, derived from its
  * parts: 4-bit codes for K and V plus fp16 scale/zero metadata. */
+long s4kv_ref_block_bytes_bits(int bits) { return block_bytes_of(bits); }
+
 long s4kv_ref_block_bytes(void) {
     long codes = 2L * PAGE * HEAD_DIM / 2;                   /* K + V, 4 bits */
     long kmeta = 2L * HEAD_DIM * 2;                          /* scale + zero */
@@ -307,12 +372,12 @@ double s4kv_ref_kv_payload_bytes(long layers, long kv_heads, long head_dim,
  * cu_new[b]..cu_new[b+1] are sequence b's new tokens; seq_lens[b] is its
  * length after the append.  slot_mapping[tok] must equal
  * block_tables[b][pos/16] * 16 + pos % 16. */
-int s4kv_ref_append(uint8_t *pool, uint16_t *res_k, uint16_t *res_v,
-                    int num_pages, int num_kv_heads, int max_seqs,
-                    const uint16_t *k, const uint16_t *v, int n_tokens,
-                    const int64_t *slot_mapping, const int32_t *cu_new,
-                    const int32_t *seq_lens, const int32_t *block_tables,
-                    int batch, int max_pages_per_seq) {
+int s4kv_ref_append_bits(uint8_t *pool, uint16_t *res_k, uint16_t *res_v,
+                         int num_pages, int num_kv_heads, int max_seqs,
+                         const uint16_t *k, const uint16_t *v, int n_tokens,
+                         const int64_t *slot_mapping, const int32_t *cu_new,
+                         const int32_t *seq_lens, const int32_t *block_tables,
+                         int batch, int max_pages_per_seq, int bits) {
     if (batch < 0 || batch > max_seqs || n_tokens < 0) return REF_BAD_ARG;
     if (cu_new[0] != 0 || cu_new[batch] != n_tokens) return REF_BAD_ARG;
     const long row = HEAD_DIM;
@@ -336,8 +401,8 @@ int s4kv_ref_append(uint8_t *pool, uint16_t *res_k, uint16_t *res_v,
                 memcpy(rk + r * row, k + ((long)tok * num_kv_heads + h) * row, 2 * row);
                 memcpy(rv + r * row, v + ((long)tok * num_kv_heads + h) * row, 2 * row);
                 if (r == PAGE - 1) {
-                    uint8_t *blk = pool + ((long)page * num_kv_heads + h) * BLOCK_BYTES;
-                    s4kv_ref_quantize_page(rk, rv, blk);
+                    uint8_t *blk = pool + ((long)page * num_kv_heads + h) * block_bytes_of(bits);
+                    s4kv_ref_quantize_page_bits(rk, rv, blk, bits);
                 }
             }
         }
@@ -345,17 +410,32 @@ int s4kv_ref_append(uint8_t *pool, uint16_t *res_k, uint16_t *res_v,
     return REF_OK;
 }
 
+int s4kv_ref_append(uint8_t *pool, uint16_t *res_k, uint16_t *res_v,
+                    int num_pages, int num_kv_heads, int max_seqs,
+                    const uint16_t *k, const uint16_t *v, int n_tokens,
+                    const int64_t *slot_mapping, const int32_t *cu_new,
+                    const int32_t *seq_lens, const int32_t *block_tables,
+                    int batch, int max_pages_per_seq) {
+    return s4kv_ref_append_bits(pool, res_k, res_v, num_pages, num_kv_heads, max_seqs, k, v, n_tokens,
+                                slot_mapping, cu_new, seq_lens, block_tables, batch, max_pages_per_seq, 4);
+}
+
 /* Dequantize one physical page for all kv heads.  out_k, out_v: fp32
  * [kv_heads][16][128]. */
-int s4kv_ref_dequant_page(const uint8_t *pool, int num_pages, int num_kv_heads,
-                          int physical_page, float *out_k, float *out_v) {
+int s4kv_ref_dequant_page_bits(const uint8_t *pool, int num_pages, int num_kv_heads,
+                               int physical_page, float *out_k, float *out_v, int bits) {
     if (physical_page < 0 || physical_page >= num_pages) return REF_BAD_ARG;
     for (int h = 0; h < num_kv_heads; ++h) {
-        const uint8_t *blk = pool + ((long)physical_page * num_kv_heads + h) * BLOCK_BYTES;
-        s4kv_ref_dequant_block(blk, out_k + (long)h * PAGE * HEAD_DIM,
-                               out_v + (long)h * PAGE * HEAD_DIM);
+        const uint8_t *blk = pool + ((long)physical_page * num_kv_heads + h) * block_bytes_of(bits);
+        s4kv_ref_dequant_block_bits(blk, out_k + (long)h * PAGE * HEAD_DIM,
+                                    out_v + (long)h * PAGE * HEAD_DIM, bits);
     }
     return REF_OK;
+}
+
+int s4kv_ref_dequant_page(const uint8_t *pool, int num_pages, int num_kv_heads,
+                          int physical_page, float *out_k, float *out_v) {
+    return s4kv_ref_dequant_page_bits(pool, num_pages, num_kv_heads, physical_page, out_k, out_v, 4);
 }
 
 /* ------------------------------------------------ page movement ---- */
@@ -366,10 +446,11 @@ int s4kv_ref_dequant_page(const uint8_t *pool, int num_pages, int num_kv_heads,
  * sequences and copied only when written).  A page record is all kv heads'
  * blocks of one physical page: num_kv_heads * 2816 contiguous bytes. */
 
-/* dst[i] = page record pages[i], i < n (dst: [n][num_kv_heads][2816]). */
+/* dst[i] = page record pages[i], i < n (dst: [n][num_kv_heads][block bytes];
+ * the block bytes follow the code width `bits`). */
 int s4kv_ref_gather_pages(const uint8_t *pool, int num_pages, int num_kv_heads,
-                          const int32_t *pages, int n, uint8_t *dst) {
-    long rec = (long)num_kv_heads * BLOCK_BYTES;
+                          const int32_t *pages, int n, uint8_t *dst, int bits) {
+    long rec = (long)num_kv_heads * block_bytes_of(bits);
     for (int i = 0; i < n; ++i)
         if (pages[i] < 0 || pages[i] >= num_pages) return REF_BAD_SLOT;
     for (int i = 0; i < n; ++i) memcpy(dst + i * rec, pool + pages[i] * rec, (size_t)rec);
@@ -378,8 +459,8 @@ int s4kv_ref_gather_pages(const uint8_t *pool, int num_pages, int num_kv_heads,
 
 /* page record pages[i] = src[i], i < n (pages must be distinct). */
 int s4kv_ref_scatter_pages(uint8_t *pool, int num_pages, int num_kv_heads,
-                           const int32_t *pages, int n, const uint8_t *src) {
-    long rec = (long)num_kv_heads * BLOCK_BYTES;
+                           const int32_t *pages, int n, const uint8_t *src, int bits) {
+    long rec = (long)num_kv_heads * block_bytes_of(bits);
     for (int i = 0; i < n; ++i)
         if (pages[i] < 0 || pages[i] >= num_pages) return REF_BAD_SLOT;
     for (int i = 0; i < n; ++i) memcpy(pool + pages[i] * rec, src + i * rec, (size_t)rec);
@@ -389,8 +470,8 @@ int s4kv_ref_scatter_pages(uint8_t *pool, int num_pages, int num_kv_heads,
 /* page record dst_pages[i] = page record src_pages[i] (a copy-on-write copy
  * of a shared full page); no dst page may also be a src page. */
 int s4kv_ref_copy_pages(uint8_t *pool, int num_pages, int num_kv_heads,
-                        const int32_t *src_pages, const int32_t *dst_pages, int n) {
-    long rec = (long)num_kv_heads * BLOCK_BYTES;
+                        const int32_t *src_pages, const int32_t *dst_pages, int n, int bits) {
+    long rec = (long)num_kv_heads * block_bytes_of(bits);
     for (int i = 0; i < n; ++i)
         if (src_pages[i] < 0 || src_pages[i] >= num_pages || dst_pages[i] < 0 || dst_pages[i] >= num_pages)
             return REF_BAD_SLOT;
@@ -420,12 +501,12 @@ int s4kv_ref_fork_residual(uint16_t *res_k, uint16_t *res_v, int max_seqs, int n
 static void sequence_kv(const uint8_t *pool, const uint16_t *res_k,
                         const uint16_t *res_v, int num_kv_heads,
                         const int32_t *bt_row, int L, int b, int h,
-                        float *K, float *V) {
+                        float *K, float *V, int bits) {
     int full = L / PAGE;
     for (int p = 0; p < full; ++p) {
-        const uint8_t *blk = pool + ((long)bt_row[p] * num_kv_heads + h) * BLOCK_BYTES;
-        s4kv_ref_dequant_block(blk, K + (long)p * PAGE * HEAD_DIM,
-                               V + (long)p * PAGE * HEAD_DIM);
+        const uint8_t *blk = pool + ((long)bt_row[p] * num_kv_heads + h) * block_bytes_of(bits);
+        s4kv_ref_dequant_block_bits(blk, K + (long)p * PAGE * HEAD_DIM,
+                                    V + (long)p * PAGE * HEAD_DIM, bits);
     }
     for (int t = full * PAGE; t < L; ++t) {
         int r = t % PAGE;
@@ -451,7 +532,7 @@ int s4kv_ref_decode_attention(const uint8_t *pool, const uint16_t *res_k,
                               int num_q_heads, const int32_t *seq_lens,
                               const int32_t *block_tables, int batch,
                               int max_pages_per_seq, double sm_scale,
-                              int use_double, double *out) {
+                              int use_double, double *out, int bits) {
     if (num_kv_heads <= 0 || num_q_heads % num_kv_heads != 0) return REF_BAD_ARG;
     int G = num_q_heads / num_kv_heads;
     for (int b = 0; b < batch; ++b) {
@@ -467,7 +548,7 @@ int s4kv_ref_decode_attention(const uint8_t *pool, const uint16_t *res_k,
             float *V = (float *)malloc(sizeof(float) * rows * HEAD_DIM);
             double *logit = (double *)malloc(sizeof(double) * (size_t)(L > 0 ? L : 1));
             if (!K || !V || !logit) { free(K); free(V); free(logit); return REF_BAD_ARG; }
-            sequence_kv(pool, res_k, res_v, num_kv_heads, bt_row, L, b, h, K, V);
+            sequence_kv(pool, res_k, res_v, num_kv_heads, bt_row, L, b, h, K, V, bits);
             for (int g = 0; g < G; ++g) {
                 int qh = h * G + g;
                 const uint16_t *qv = q + ((long)b * num_q_heads + qh) * HEAD_DIM;
@@ -544,7 +625,7 @@ int s4kv_ref_prefill_attention(const uint8_t *pool, const uint16_t *res_k,
                                const int32_t *seq_lens,
                                const int32_t *block_tables, int batch,
                                int max_pages_per_seq, double sm_scale,
-                               double *out) {
+                               double *out, int bits) {
     if (num_kv_heads <= 0 || num_q_heads % num_kv_heads != 0) return REF_BAD_ARG;
     int G = num_q_heads / num_kv_heads;
     for (int b = 0; b < batch; ++b) {
@@ -561,7 +642,7 @@ int s4kv_ref_prefill_attention(const uint8_t *pool, const uint16_t *res_k,
         double *w = (double *)malloc(sizeof(double) * (size_t)L);
         if (!K || !V || !w) { free(K); free(V); free(w); return REF_BAD_ARG; }
         for (int h = 0; h < num_kv_heads; ++h) {
-            sequence_kv(pool, res_k, res_v, num_kv_heads, bt_row, L, b, h, K, V);
+            sequence_kv(pool, res_k, res_v, num_kv_heads, bt_row, L, b, h, K, V, bits);
             for (int j = 0; j < n; ++j) {
                 int pos = L - n + j;
                 long row = cu_new[b] + j;

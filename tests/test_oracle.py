@@ -21,6 +21,11 @@ Which pin covers which oracle function:
                                    quantizer represents exactly; single key; uniform
                                    weights; page permutation and shared-prefix
                                    invariance; GQA identical queries; fp32 vs fp64
+  int8 codes (quantize_group_bits, code_offset8, OracleCache(bits=8)) :
+                                   256-level closed forms and the rounding bound;
+                                   the byte layout against the int4 fragment map;
+                                   textbook attention on exact 256-level grids;
+                                   chunking invariance
   prefill_attention             : textbook causal softmax attention (numpy) on
                                    inputs the quantizer represents exactly, per
                                    query position; the chunk's last row equals
@@ -630,3 +635,134 @@ def test_copy_pages_then_remap_preserves_attention(oracle_mod):
     bt2 = bt.copy()
     bt2[0, :4] = free
     assert np.array_equal(c.decode_attention(q, np.array(lens, np.int32), bt2), before)
+
+
+# ------------------------------------------------------------- int8 codes --
+
+def test_int8_group_closed_forms(oracle_mod):
+    """255 levels: an exact 256-level grid gives its indices and step; the
+    all-equal group gives scale 0."""
+    x = np.arange(256, dtype=np.float16)
+    codes, sh, zh, s = oracle_mod.quantize_group_bits(x, 8)
+    assert list(codes) == list(range(256)) and s == 1.0 and sh == 0x3C00 and zh == 0
+    d, a = 2.0 ** -6, -2.0
+    k = np.random.default_rng(3).permutation(256)[:32]
+    k[0], k[1] = 0, 255
+    codes, sh, zh, s = oracle_mod.quantize_group_bits((a + k * d).astype(np.float16), 8)
+    assert list(codes) == list(k) and s == d and zh == f16bits(a)
+    codes, sh, zh, s = oracle_mod.quantize_group_bits(np.full(32, -1.25, np.float16), 8)
+    assert s == 0.0 and (codes == 0).all()
+
+
+def test_int8_group_rounding_bound(oracle_mod):
+    rng = np.random.default_rng(12)
+    for trial in range(80):
+        n = 16 if trial % 2 else 32
+        x = rng.standard_normal(n) * (1 if trial % 3 else 300)
+        x16 = x.astype(np.float16)
+        codes, sh, zh, s = oracle_mod.quantize_group_bits(x16, 8)
+        assert codes.max() <= 255
+        if s > 0:
+            assert _bound_ok(x16, codes, s, zh)
+            assert codes[np.argmin(x16)] == 0 and codes[np.argmax(x16)] == 255
+
+
+def test_int8_layout_is_the_int4_fragment_map_in_bytes(oracle_mod):
+    """8-bit codes sit where the 4-bit layout's MMA fragment assignment says,
+    with bytes for nibbles: a lane's 8 codes of one tile are consecutive
+    bytes (register r at bytes 2r, 2r + 1), tiles 2m and 2m+1 of a lane form
+    one 16-byte chunk, chunks in lane order.  Together with the fragment-table
+    pin of the 4-bit layout this ties the 8-bit layout to the PTX table; it
+    must also be a bijection onto the 2048-byte region."""
+    for is_value, slot in ((False, oracle_mod.key_code_slot), (True, oracle_mod.value_code_slot)):
+        seen = set()
+        for t in range(PAGE):
+            for c in range(HD):
+                off = oracle_mod.code_offset8(is_value, t, c)
+                chunk, within = divmod(off, 16)
+                m, lane = divmod(chunk, 32)
+                tile = 2 * m + within // 8
+                r, half = divmod(within % 8, 2)
+                word, nib = slot(t, c)
+                assert (tile, lane) == (4 * (word // 128) + word % 4, (word % 128) // 4)
+                assert (r, half) == (nib & 3, nib >> 2)
+                seen.add(off)
+        assert seen == set(range(2048))
+
+
+def test_int8_block_size(oracle_mod):
+    # 16 x 128 one-byte codes for K and V plus the same 768 bytes of fp16
+    # metadata as the int4 block
+    assert oracle_mod.block_bytes(8) == 2 * 2048 + 768 == 4864
+    assert oracle_mod.block_bytes(4) == 2816
+
+
+def _grid_page8(rng, per):
+    if per == "key":
+        d = 2.0 ** rng.integers(-8, -4, HD)
+        a = rng.integers(-8, 8, HD) * 0.25
+        codes = np.stack([rng.permutation(256)[:16] for _ in range(HD)], axis=1)
+        codes[0], codes[1] = 0, 255
+        return (a[None, :] + codes * d[None, :]).astype(np.float16)
+    d = 2.0 ** rng.integers(-8, -4, (PAGE, 4))
+    a = rng.integers(-8, 8, (PAGE, 4)) * 0.25
+    codes = np.stack([np.stack([rng.permutation(256)[:32] for _ in range(4)]) for _ in range(PAGE)])
+    codes[:, :, 0], codes[:, :, 1] = 0, 255
+    return (a[:, :, None] + codes * d[:, :, None]).reshape(PAGE, HD).astype(np.float16)
+
+
+def test_int8_decode_matches_textbook_on_exact_grids(oracle_mod):
+    """Pages whose key channels and value groups are exact 256-level grids
+    dequantize to themselves, so int8 decode attention equals numpy's."""
+    rng = np.random.default_rng(44)
+    H, G = 2, 4
+    lens = [40, 64, 9]
+    k, v = [], []
+    for L in lens:
+        npg = (L + PAGE - 1) // PAGE
+        kk = np.zeros((npg * PAGE, H, HD), np.float16)
+        vv = np.zeros((npg * PAGE, H, HD), np.float16)
+        for p in range(npg):
+            for h in range(H):
+                kk[p * PAGE:(p + 1) * PAGE, h] = _grid_page8(rng, "key")
+                vv[p * PAGE:(p + 1) * PAGE, h] = _grid_page8(rng, "value")
+        k.append(kk[:L])
+        v.append(vv[:L])
+    bt, NP = _tables(rng, lens)
+    c = oracle_mod.OracleCache(NP, H, len(lens), bits=8)
+    _append_all(oracle_mod, c, k, v, [0] * 3, lens, bt, 11)
+    q = rng.standard_normal((3, H * G, HD)).astype(np.float16)
+    out = c.decode_attention(q, np.array(lens, np.int32), bt)
+    for b, L in enumerate(lens):
+        for qh in range(H * G):
+            ref = _textbook_attention(q[b, qh], k[b][:, qh // G], v[b][:, qh // G], 1 / np.sqrt(HD))
+            assert np.allclose(out[b, qh], ref, rtol=1e-12, atol=1e-12)
+    # and int8 attention is closer to unquantized attention than int4 on random data
+    kr, vr = _rand_kv(rng, 2, 1, [96, 64])
+    btr, NPr = _tables(rng, [96, 64])
+    errs = []
+    for bits in (4, 8):
+        cc = oracle_mod.OracleCache(NPr, 1, 2, bits=bits)
+        _append_all(oracle_mod, cc, kr, vr, [0, 0], [96, 64], btr)
+        qq = rng.standard_normal((2, 4, HD)).astype(np.float16) if bits == 4 else qq
+        o = cc.decode_attention(qq, np.array([96, 64], np.int32), btr)
+        ref = np.stack([np.stack([_textbook_attention(qq[b, j], kr[b][:, 0], vr[b][:, 0], 1 / np.sqrt(HD))
+                                  for j in range(4)]) for b in range(2)])
+        errs.append(np.abs(o - ref).max())
+    assert errs[1] < errs[0] / 4
+
+
+def test_int8_append_chunking_invariance(oracle_mod):
+    rng = np.random.default_rng(45)
+    lens = [37, 50]
+    k, v = _rand_kv(rng, 2, 2, lens)
+    bt, NP = _tables(rng, lens)
+    pools = []
+    for chunk in (None, 1, 16, 23):
+        c = oracle_mod.OracleCache(NP, 2, 2, bits=8)
+        _append_all(oracle_mod, c, k, v, [0, 0], lens, bt, chunk)
+        pools.append((c.pool.copy(), c.res_k.copy()))
+    for p_, r_ in pools[1:]:
+        assert np.array_equal(p_, pools[0][0])
+        for b, L in enumerate(lens):
+            assert np.array_equal(r_[b, :, :L % 16], pools[0][1][b, :, :L % 16])
