@@ -136,8 +136,8 @@ class ClockSampler:
 
 # -------------------------------------------------------------- workload --
 
-def step_bytes(spec, plan, lens):
-    d = W.decode_bytes(spec, lens, plan)
+def step_bytes(spec, plan, lens, bits: int = 4):
+    d = W.decode_bytes(spec, lens, plan, block_bytes=4864 if bits == 8 else 2816)
     new = W.step_new_tokens(spec)
     kv_new = int(new.sum()) * spec.num_kv_heads * 128 * 2 * 2   # k and v read
     append = 2 * kv_new                                         # residual write (upper bound)
@@ -148,11 +148,11 @@ class DeviceWorkload:
     """All layers' caches of one workload on one GPU, filled through the C
     ABI, plus the step's inputs."""
 
-    def __init__(self, spec: W.Spec, device, prefill_tokens_per_call=1 << 18):
+    def __init__(self, spec: W.Spec, device, prefill_tokens_per_call=1 << 18, bits: int = 4):
         import torch
         import int4_kivi_quantized_s4kv_b200 as S
         self.S, self.torch = S, torch
-        self.spec, self.device = spec, device
+        self.spec, self.device, self.bits = spec, device, bits
         self.ctx = W.context_lens(spec)
         self.lens = W.final_lens(spec)
         self.new = W.step_new_tokens(spec)
@@ -167,7 +167,7 @@ class DeviceWorkload:
         self.max_new = int(self.new.max())
         self.caches, self.q, self.k_new, self.v_new = [], [], [], []
         for layer in range(spec.layers):
-            cache = S.S4KVCache(self.plan.num_pages, H, B, device=device)
+            cache = S.S4KVCache(self.plan.num_pages, H, B, device=device, bits=bits)
             ks = torch.from_numpy(W.key_channel_scale(spec, layer)).to(device)
             kn, vn = [], []
             b = 0
@@ -410,7 +410,7 @@ def measure_page_moves(wl, device, reps: int = 10):
     S = wl.S
     cache = wl.caches[0]
     H = wl.spec.num_kv_heads
-    rec = S.s4kv_page_record_bytes(H)
+    rec = S.s4kv_page_record_bytes(cache)
     nfull = (wl.lens // 16).astype(np.int64)
     # gather: as many whole sequences as make > 2x L2 of records
     rows, total = [], 0
@@ -490,6 +490,31 @@ def measure_fused_step(wl, device, steps: int = 20):
         raise RuntimeError("fused step set device error flags")
     return {"workload": spec.name, "layers": spec.layers, "two_launch_ms": two, "fused_ms": one,
             "speedup": two / one, "launches_per_layer": {"two_launch": 2, "fused": 1}}
+
+
+def measure_int8_decode(device, spec, steps: int = 20):
+    """The INT8 variant's decode step (append + decode, 4864-byte pages) on
+    the same workload as the headline, against the HBM roofline."""
+    import torch
+    wl = DeviceWorkload(spec, device, bits=8)
+    dbytes, _ = step_bytes(wl.spec, wl.plan, wl.lens, bits=8)
+    for _ in range(3):
+        wl.step()
+    torch.cuda.synchronize()
+    ev = ([], [])
+    for _ in range(steps):
+        wl.step(ev)
+    torch.cuda.synchronize()
+    ms = sum(a.elapsed_time(b) for a, b in zip(*ev)) / steps
+    if any(wl.S.s4kv_get_error(c) for c in wl.caches):
+        raise RuntimeError("int8 decode set device error flags")
+    peak, kind = measured_hbm_peak()
+    gbs = dbytes["algorithmic"] / (ms * 1e-3) / 1e9
+    return {"workload": spec.name, "bits": 8, "block_bytes": 4864, "avg_launch_ms": ms,
+            "tokens_per_s": int(wl.new.sum()) / (ms * 1e-3),
+            "roofline": {"bound": "hbm", "kernel": "decode_kernel<8>", "achieved": gbs, "peak": peak,
+                         "peak_kind": kind, "unit": "GB/s", "frac": gbs / peak, "traffic": None,
+                         "bytes_per_launch": dbytes["algorithmic"]}}
 
 
 def run_reference(args, spec):
@@ -654,7 +679,7 @@ def main(argv=None):
     value = aggregate_gbs(world, bytes_per_step, step_ms)
     achieved = decode_bytes_per_launch / (dec_avg_ms * 1e-3) / 1e9
     tokens = int(wl.new.sum())
-    prefill = moves = fused = None
+    prefill = moves = fused = int8 = None
     if world == 1 and not args.no_prefill:
         prefill = measure_prefill(device, max(3, min(args.steps, 20)))
         moves = measure_page_moves(wl, device)
@@ -662,6 +687,7 @@ def main(argv=None):
         small = DeviceWorkload(W.SPECS["qwen2.5-7b"], device)
         fused.append(measure_fused_step(small, device))
         del small
+        int8 = measure_int8_decode(device, spec)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(spec)
@@ -698,7 +724,7 @@ def main(argv=None):
         if cpu is not None:
             line["cpu_baseline"] = cpu
         if prefill is not None:
-            line["next_rows"] = {"prefill": prefill, "page_moves": moves, "fused_step": fused}
+            line["next_rows"] = {"prefill": prefill, "page_moves": moves, "fused_step": fused, "int8_decode": int8}
         print(json.dumps(line), flush=True)
     if world > 1:
         torch.distributed.destroy_process_group()

@@ -54,6 +54,15 @@
  *           and the key zero points follow the same k order, so one
  *           ldmatrix row is a lane quad's k columns; s4kv_dequant_page
  *           returns the natural [token][channel] order).
+ *           With 8-bit codes (s4kv_cache_t.bits == 8, the INT8 variant of the
+ *           same KIVI split: 255 levels, s = (mx - mn) / 255, codes clamped
+ *           to [0, 255]) the block is S4KV_BLOCK_BYTES_INT8 = 4864 bytes:
+ *             [   0,2048) key codes, [2048,4096) value codes, then the
+ *             same fp16 metadata at [4096,4864) in the order above.
+ *           A code keeps the 4-bit layout's place in the operand fragments,
+ *           with bytes for nibbles: the 8 codes of tile 4*h+q of lane l are
+ *           bytes ((32*m + l)*16 + 8*(tile%2) + 2*(j&3) + (j>>2)), m =
+ *           tile/2, j the 4-bit nibble index of that (token, channel).
  *  res_k,   fp16 [max_seqs][num_kv_heads][16][128] each.  Row r of batch
  *  res_v    row b holds token 16*floor(L/16) + r of that sequence for
  *           r < L mod 16 (L = its current length); other rows are
@@ -85,11 +94,12 @@
 extern "C" {
 #endif
 
-#define S4KV_VERSION 1
+#define S4KV_VERSION 2
 #define S4KV_HEAD_DIM 128
 #define S4KV_PAGE_TOKENS 16
 #define S4KV_VALUE_GROUP 32
-#define S4KV_BLOCK_BYTES 2816
+#define S4KV_BLOCK_BYTES 2816      /* 4-bit codes */
+#define S4KV_BLOCK_BYTES_INT8 4864 /* 8-bit codes */
 #define S4KV_MAX_GQA_GROUP 8
 
 /* status codes returned by every call */
@@ -118,6 +128,7 @@ typedef struct s4kv_cache {
     int32_t max_seqs;
     int32_t head_dim;    /* must be S4KV_HEAD_DIM */
     int32_t page_tokens; /* must be S4KV_PAGE_TOKENS */
+    int32_t bits;        /* code width: 4 (or 0, meaning 4) or 8 */
 } s4kv_cache_t;
 
 /* Library version (S4KV_VERSION). */
@@ -140,6 +151,11 @@ S4KV_API int s4kv_check_model(int head_dim, int page_tokens, int num_q_heads,
  * plus scale/zero metadata).  Host only; either output may be NULL. */
 S4KV_API int s4kv_cache_layout(int num_pages, int num_kv_heads, int max_seqs,
                       size_t *pool_bytes, size_t *residual_bytes);
+
+/* The same for a code width of `bits` (4 or 8; INT8 pages take
+ * S4KV_BLOCK_BYTES_INT8 bytes per kv head). */
+S4KV_API int s4kv_cache_layout_bits(int num_pages, int num_kv_heads, int max_seqs, int bits,
+                                    size_t *pool_bytes, size_t *residual_bytes);
 
 /* Append new tokens' K/V and quantize every page they complete.
  *  k, v          device fp16 [n_tokens][num_kv_heads][128], 16-B aligned,
@@ -256,7 +272,8 @@ S4KV_API int s4kv_decode_attention_noalloc(const s4kv_cache_t *cache, const void
  * Runs on the tcgen05 tensor cores with the dequantized keys and values and
  * the softmax weights as fp16 MMA operands (fp32 accumulation), so results
  * agree with exact attention to about fp16 precision of those operands.
- * Allocates nothing; needs about 171 KB of shared memory per CTA. */
+ * Allocates nothing; needs about 171 KB of shared memory per CTA.  4-bit
+ * codes only (an 8-bit cache is refused with S4KV_ERR_UNSUPPORTED). */
 S4KV_API int s4kv_prefill_attention(const s4kv_cache_t *cache, const void *q,
                                     int num_q_heads, int n_tokens,
                                     const int32_t *cu_new, const int32_t *seq_lens,
@@ -283,15 +300,16 @@ S4KV_API int s4kv_dequant_pages(const s4kv_cache_t *cache, const int32_t *pages,
  * page tables and copies a page only when it is written ("KV-Cache und
  * PagedAttention: Warum Ihr LLM-Server langsamer wird", "Wie PagedAttention
  * das loest").  A page RECORD is all kv heads' blocks of one physical page:
- * num_kv_heads * 2816 contiguous bytes, the unit these calls move.  All page
+ * num_kv_heads * block bytes (2816 with 4-bit codes, 4864 with 8-bit)
+ * contiguous bytes, the unit these calls move.  All page
  * and row lists are device int32 arrays; an id out of range sets
  * S4KV_EFLAG_PAGE_RANGE (rows: S4KV_EFLAG_SLOT) and that item is skipped.
  * Every call is asynchronous on `stream`. */
 
-/* Bytes of one page record (num_kv_heads * 2816). */
-S4KV_API int s4kv_page_record_bytes(int num_kv_heads, size_t *bytes);
+/* Bytes of one page record of this cache (num_kv_heads * block bytes). */
+S4KV_API int s4kv_page_record_bytes(const s4kv_cache_t *cache, size_t *bytes);
 
-/* dst (device, 16-B aligned, [n][num_kv_heads][2816]) slot i = page record
+/* dst (device, 16-B aligned, [n][page record]) slot i = page record
  * pages[i]. */
 S4KV_API int s4kv_gather_pages(const s4kv_cache_t *cache, const int32_t *pages, int n,
                                void *dst, void *stream);

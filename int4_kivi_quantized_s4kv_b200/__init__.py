@@ -18,6 +18,7 @@ HEAD_DIM = 128
 PAGE_TOKENS = 16
 VALUE_GROUP = 32
 BLOCK_BYTES = 2816
+BLOCK_BYTES_INT8 = 4864
 MAX_GQA_GROUP = 8
 NOALLOC_SCRATCH_BYTES = 24 * 1024 * 1024
 
@@ -31,7 +32,7 @@ class s4kv_cache_t(ctypes.Structure):
     _fields_ = [("pool", ctypes.c_void_p), ("res_k", ctypes.c_void_p), ("res_v", ctypes.c_void_p),
                 ("err_flag", ctypes.c_void_p), ("num_pages", ctypes.c_int32),
                 ("num_kv_heads", ctypes.c_int32), ("max_seqs", ctypes.c_int32),
-                ("head_dim", ctypes.c_int32), ("page_tokens", ctypes.c_int32)]
+                ("head_dim", ctypes.c_int32), ("page_tokens", ctypes.c_int32), ("bits", ctypes.c_int32)]
 
 
 _P, _I, _SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
@@ -41,6 +42,7 @@ _SIGS = {
     "s4kv_status_string": ([_I], ctypes.c_char_p),
     "s4kv_check_model": ([_I, _I, _I, _I], _I),
     "s4kv_cache_layout": ([_I, _I, _I, ctypes.POINTER(_SZ), ctypes.POINTER(_SZ)], _I),
+    "s4kv_cache_layout_bits": ([_I, _I, _I, _I, ctypes.POINTER(_SZ), ctypes.POINTER(_SZ)], _I),
     "s4kv_append": ([_CP, _P, _P, _I, _P, _P, _P, _P, _I, _I, _I, _P], _I),
     "s4kv_decode_workspace_size": ([_I, _I, ctypes.POINTER(_SZ)], _I),
     "s4kv_decode_attention": ([_CP, _P, _I, _P, _P, _I, _I, ctypes.c_float, _P, _P, _SZ, _P], _I),
@@ -49,7 +51,7 @@ _SIGS = {
     "s4kv_prefill_attention": ([_CP, _P, _I, _I, _P, _P, _P, _I, _I, _I, ctypes.c_float, _P, _P], _I),
     "s4kv_dequant_page": ([_CP, _I, _P, _P, _I, _P], _I),
     "s4kv_dequant_pages": ([_CP, _P, _I, _P, _P, _I, _P], _I),
-    "s4kv_page_record_bytes": ([_I, ctypes.POINTER(_SZ)], _I),
+    "s4kv_page_record_bytes": ([_CP, ctypes.POINTER(_SZ)], _I),
     "s4kv_gather_pages": ([_CP, _P, _I, _P, _P], _I),
     "s4kv_scatter_pages": ([_CP, _P, _I, _P, _P], _I),
     "s4kv_copy_pages": ([_CP, _P, _P, _I, _P], _I),
@@ -121,10 +123,10 @@ def s4kv_check_model(head_dim: int, page_tokens: int, num_q_heads: int, num_kv_h
     return lib().s4kv_check_model(head_dim, page_tokens, num_q_heads, num_kv_heads)
 
 
-def s4kv_cache_layout(num_pages: int, num_kv_heads: int, max_seqs: int) -> tuple[int, int]:
+def s4kv_cache_layout(num_pages: int, num_kv_heads: int, max_seqs: int, bits: int = 4) -> tuple[int, int]:
     pb, rb = _SZ(0), _SZ(0)
-    _check(lib().s4kv_cache_layout(num_pages, num_kv_heads, max_seqs, ctypes.byref(pb), ctypes.byref(rb)),
-           "s4kv_cache_layout")
+    _check(lib().s4kv_cache_layout_bits(num_pages, num_kv_heads, max_seqs, bits, ctypes.byref(pb),
+                                        ctypes.byref(rb)), "s4kv_cache_layout_bits")
     return pb.value, rb.value
 
 
@@ -140,18 +142,19 @@ class S4KVCache:
     """Caller-owned device memory of one layer's cache (torch tensors) and the
     plain C descriptor the library reads."""
 
-    def __init__(self, num_pages: int, num_kv_heads: int, max_seqs: int, device="cuda"):
+    def __init__(self, num_pages: int, num_kv_heads: int, max_seqs: int, device="cuda", bits: int = 4):
         import torch
-        pool_bytes, res_bytes = s4kv_cache_layout(num_pages, num_kv_heads, max_seqs)
-        self.num_pages, self.num_kv_heads, self.max_seqs = num_pages, num_kv_heads, max_seqs
-        self.pool = torch.zeros((num_pages, num_kv_heads, BLOCK_BYTES), dtype=torch.uint8, device=device)
+        pool_bytes, res_bytes = s4kv_cache_layout(num_pages, num_kv_heads, max_seqs, bits)
+        self.num_pages, self.num_kv_heads, self.max_seqs, self.bits = num_pages, num_kv_heads, max_seqs, bits
+        block = BLOCK_BYTES if bits == 4 else BLOCK_BYTES_INT8
+        self.pool = torch.zeros((num_pages, num_kv_heads, block), dtype=torch.uint8, device=device)
         self.res_k = torch.zeros((max_seqs, num_kv_heads, PAGE_TOKENS, HEAD_DIM), dtype=torch.float16, device=device)
         self.res_v = torch.zeros_like(self.res_k)
         self.err_flag = torch.zeros(1, dtype=torch.int32, device=device)
         assert self.pool.numel() == pool_bytes and self.res_k.numel() * 2 == res_bytes
         self.c = s4kv_cache_t(self.pool.data_ptr(), self.res_k.data_ptr(), self.res_v.data_ptr(),
                               self.err_flag.data_ptr(), num_pages, num_kv_heads, max_seqs,
-                              HEAD_DIM, PAGE_TOKENS)
+                              HEAD_DIM, PAGE_TOKENS, bits)
 
     @property
     def ref(self):
@@ -260,9 +263,9 @@ def s4kv_dequant_pages(cache: S4KVCache, pages, out_k, out_v, out_fp32: bool = T
     _check(st, "s4kv_dequant_pages")
 
 
-def s4kv_page_record_bytes(num_kv_heads: int) -> int:
+def s4kv_page_record_bytes(cache: S4KVCache) -> int:
     n = _SZ(0)
-    _check(lib().s4kv_page_record_bytes(num_kv_heads, ctypes.byref(n)), "s4kv_page_record_bytes")
+    _check(lib().s4kv_page_record_bytes(cache.ref, ctypes.byref(n)), "s4kv_page_record_bytes")
     return n.value
 
 

@@ -21,10 +21,16 @@ constexpr int kMaxDevices = 64;
 struct DeviceShape {
   bool ready = false;
   int num_sms = 0;
-  int ctas_per_sm = 0;
-  int num_ctas = 0;
-  int num_workers = 0;
+  int num_ctas[2] = {0, 0};     // decode grid for 4-bit / 8-bit pages
+  int num_workers[2] = {0, 0};  // worker warps of that grid
+  int max_workers = 0;          // sizes the (shared) decode workspace
 };
+
+int fmt_index(int bits) { return bits == 8 ? 1 : 0; }
+int cache_bits(const s4kv_cache_t *c) { return c->bits == 8 ? 8 : 4; }
+size_t record_bytes(const s4kv_cache_t *c) {
+  return static_cast<size_t>(c->num_kv_heads) * (cache_bits(c) == 8 ? S4KV_BLOCK_BYTES_INT8 : S4KV_BLOCK_BYTES);
+}
 
 std::mutex g_mu;
 DeviceShape g_shape[kMaxDevices];
@@ -49,12 +55,14 @@ int device_shape(DeviceShape *out) {
       cudaGetLastError();
       return S4KV_ERR_CUDA;
     }
-    const int per = decode_ctas_per_sm();
-    if (per <= 0 || sms <= 0) return S4KV_ERR_CUDA;
     d.num_sms = sms;
-    d.ctas_per_sm = per;
-    d.num_ctas = sms * per;
-    d.num_workers = d.num_ctas * decode_warps_per_cta();
+    for (int f = 0; f < 2; ++f) {
+      const int per = decode_ctas_per_sm(f ? 8 : 4);
+      if (per <= 0 || sms <= 0) return S4KV_ERR_CUDA;
+      d.num_ctas[f] = sms * per;
+      d.num_workers[f] = d.num_ctas[f] * decode_warps_per_cta();
+      d.max_workers = d.num_workers[f] > d.max_workers ? d.num_workers[f] : d.max_workers;
+    }
     d.ready = true;
   }
   *out = d;
@@ -70,6 +78,7 @@ int check_cache(const s4kv_cache_t *c) {
   if (c->num_pages <= 0 || c->num_kv_heads <= 0 || c->max_seqs <= 0) return S4KV_ERR_INVALID_ARG;
   if (!aligned(c->pool, 128) || !aligned(c->res_k, 16) || !aligned(c->res_v, 16)) return S4KV_ERR_INVALID_ARG;
   if (c->err_flag != nullptr && !aligned(c->err_flag, 4)) return S4KV_ERR_INVALID_ARG;
+  if (c->bits != 0 && c->bits != 4 && c->bits != 8) return S4KV_ERR_UNSUPPORTED;
   return S4KV_OK;
 }
 
@@ -148,6 +157,15 @@ int s4kv_cache_layout(int num_pages, int num_kv_heads, int max_seqs, size_t *poo
   return S4KV_OK;
 }
 
+int s4kv_cache_layout_bits(int num_pages, int num_kv_heads, int max_seqs, int bits, size_t *pool_bytes,
+                           size_t *residual_bytes) {
+  if (bits != 4 && bits != 8) return S4KV_ERR_UNSUPPORTED;
+  const int rc = s4kv_cache_layout(num_pages, num_kv_heads, max_seqs, pool_bytes, residual_bytes);
+  if (rc == S4KV_OK && pool_bytes && bits == 8)
+    *pool_bytes = static_cast<size_t>(num_pages) * num_kv_heads * S4KV_BLOCK_BYTES_INT8;
+  return rc;
+}
+
 int s4kv_append(const s4kv_cache_t *cache, const void *k, const void *v, int n_tokens,
                 const int64_t *slot_mapping, const int32_t *cu_new, const int32_t *seq_lens,
                 const int32_t *block_tables, int batch, int max_pages_per_seq, int max_new_per_seq,
@@ -179,6 +197,7 @@ int s4kv_append(const s4kv_cache_t *cache, const void *k, const void *v, int n_t
   p.max_pages = max_pages_per_seq;
   p.max_new = max_new_per_seq;
   p.n_tokens = n_tokens;
+  p.bits = cache_bits(cache);
   launch_append(p, batch, max_new_per_seq, static_cast<cudaStream_t>(stream));
   if (cudaGetLastError() != cudaSuccess) return S4KV_ERR_CUDA;
   return S4KV_OK;
@@ -189,7 +208,7 @@ int s4kv_decode_workspace_size(int batch, int num_kv_heads, size_t *bytes) {
   DeviceShape d;
   const int rc = device_shape(&d);
   if (rc != S4KV_OK) return rc;
-  *bytes = ws_layout(batch, num_kv_heads, d.num_workers).total;
+  *bytes = ws_layout(batch, num_kv_heads, d.max_workers).total;
   return S4KV_OK;
 }
 
@@ -230,7 +249,8 @@ int decode_call(const s4kv_cache_t *cache, const void *k_new, const void *v_new,
   DeviceShape d;
   rc = device_shape(&d);
   if (rc != S4KV_OK) return rc;
-  const WsLayout w = ws_layout(batch, cache->num_kv_heads, d.num_workers);
+  const WsLayout w = ws_layout(batch, cache->num_kv_heads, d.max_workers);
+  const int fi = fmt_index(cache_bits(cache));
   if (workspace == nullptr || workspace_bytes < w.total || !aligned(workspace, 16)) return S4KV_ERR_WORKSPACE;
   uint8_t *ws = static_cast<uint8_t *>(workspace);
   DecodeParams p;
@@ -252,11 +272,11 @@ int decode_call(const s4kv_cache_t *cache, const void *k_new, const void *v_new,
   p.max_pages = max_pages_per_seq;
   p.num_pages = cache->num_pages;
   p.scale_log2 = static_cast<float>(static_cast<double>(sm_scale) * 1.4426950408889634);
-  p.num_workers = d.num_workers;
+  p.num_workers = d.num_workers[fi];
   FusedAppend f;
   f.k_new = static_cast<const __half *>(k_new);
   f.v_new = static_cast<const __half *>(v_new);
-  launch_decode(p, f, d.num_ctas, static_cast<cudaStream_t>(stream));
+  launch_decode(p, f, cache_bits(cache), d.num_ctas[fi], static_cast<cudaStream_t>(stream));
   if (cudaGetLastError() != cudaSuccess) return S4KV_ERR_CUDA;
   return S4KV_OK;
 }
@@ -271,6 +291,7 @@ int s4kv_prefill_attention(const s4kv_cache_t *cache, const void *q, int num_q_h
                            void *stream) {
   int rc = check_cache(cache);
   if (rc != S4KV_OK) return rc;
+  if (cache_bits(cache) != 4) return S4KV_ERR_UNSUPPORTED;
   rc = s4kv_check_model(cache->head_dim, cache->page_tokens, num_q_heads, cache->num_kv_heads);
   if (rc != S4KV_OK) return rc;
   if (n_tokens < 0 || batch < 0 || batch > cache->max_seqs || max_pages_per_seq <= 0) return S4KV_ERR_INVALID_ARG;
@@ -335,6 +356,7 @@ int s4kv_dequant_page(const s4kv_cache_t *cache, int physical_page, void *out_k,
   p.num_pages = cache->num_pages;
   p.num_kv_heads = cache->num_kv_heads;
   p.out_fp32 = out_fp32 ? 1 : 0;
+  p.bits = cache_bits(cache);
   launch_dequant(p, static_cast<cudaStream_t>(stream));
   if (cudaGetLastError() != cudaSuccess) return S4KV_ERR_CUDA;
   return S4KV_OK;
@@ -359,14 +381,17 @@ int s4kv_dequant_pages(const s4kv_cache_t *cache, const int32_t *pages, int n, v
   p.num_pages = cache->num_pages;
   p.num_kv_heads = cache->num_kv_heads;
   p.out_fp32 = out_fp32 ? 1 : 0;
+  p.bits = cache_bits(cache);
   launch_dequant(p, static_cast<cudaStream_t>(stream));
   if (cudaGetLastError() != cudaSuccess) return S4KV_ERR_CUDA;
   return S4KV_OK;
 }
 
-int s4kv_page_record_bytes(int num_kv_heads, size_t *bytes) {
-  if (num_kv_heads <= 0 || bytes == nullptr) return S4KV_ERR_INVALID_ARG;
-  *bytes = static_cast<size_t>(num_kv_heads) * S4KV_BLOCK_BYTES;
+int s4kv_page_record_bytes(const s4kv_cache_t *cache, size_t *bytes) {
+  const int rc = check_cache(cache);
+  if (rc != S4KV_OK) return rc;
+  if (bytes == nullptr) return S4KV_ERR_INVALID_ARG;
+  *bytes = record_bytes(cache);
   return S4KV_OK;
 }
 
@@ -377,7 +402,7 @@ int s4kv_gather_pages(const s4kv_cache_t *cache, const int32_t *pages, int n, vo
   if (n == 0) return S4KV_OK;
   if (!pages || !dst || !aligned(pages, 4) || !aligned(dst, 16)) return S4KV_ERR_INVALID_ARG;
   return launch_records(static_cast<const uint8_t *>(cache->pool), static_cast<uint8_t *>(dst), pages, nullptr,
-                        static_cast<long long>(cache->num_kv_heads) * S4KV_BLOCK_BYTES, n, cache->num_pages, n,
+                        static_cast<long long>(record_bytes(cache)), n, cache->num_pages, n,
                         cache->err_flag, S4KV_EFLAG_PAGE_RANGE, stream);
 }
 
@@ -388,7 +413,7 @@ int s4kv_scatter_pages(const s4kv_cache_t *cache, const int32_t *pages, int n, c
   if (n == 0) return S4KV_OK;
   if (!pages || !src || !aligned(pages, 4) || !aligned(src, 16)) return S4KV_ERR_INVALID_ARG;
   return launch_records(static_cast<const uint8_t *>(src), static_cast<uint8_t *>(cache->pool), nullptr, pages,
-                        static_cast<long long>(cache->num_kv_heads) * S4KV_BLOCK_BYTES, n, n, cache->num_pages,
+                        static_cast<long long>(record_bytes(cache)), n, n, cache->num_pages,
                         cache->err_flag, S4KV_EFLAG_PAGE_RANGE, stream);
 }
 
@@ -400,7 +425,7 @@ int s4kv_copy_pages(const s4kv_cache_t *cache, const int32_t *src_pages, const i
   if (n == 0) return S4KV_OK;
   if (!src_pages || !dst_pages || !aligned(src_pages, 4) || !aligned(dst_pages, 4)) return S4KV_ERR_INVALID_ARG;
   return launch_records(static_cast<const uint8_t *>(cache->pool), static_cast<uint8_t *>(cache->pool), src_pages,
-                        dst_pages, static_cast<long long>(cache->num_kv_heads) * S4KV_BLOCK_BYTES, n,
+                        dst_pages, static_cast<long long>(record_bytes(cache)), n,
                         cache->num_pages, cache->num_pages, cache->err_flag, S4KV_EFLAG_PAGE_RANGE, stream);
 }
 
@@ -424,7 +449,7 @@ int s4kv_swap_out(const s4kv_cache_t *cache, const int32_t *pages, int n, void *
   int rc = s4kv_gather_pages(cache, pages, n, staging, stream);
   if (rc != S4KV_OK || n == 0) return rc;
   if (host_dst == nullptr) return S4KV_ERR_INVALID_ARG;
-  const size_t bytes = static_cast<size_t>(n) * cache->num_kv_heads * S4KV_BLOCK_BYTES;
+  const size_t bytes = static_cast<size_t>(n) * record_bytes(cache);
   if (cudaMemcpyAsync(host_dst, staging, bytes, cudaMemcpyDeviceToHost, static_cast<cudaStream_t>(stream)) !=
       cudaSuccess) {
     cudaGetLastError();
@@ -440,7 +465,7 @@ int s4kv_swap_in(const s4kv_cache_t *cache, const int32_t *pages, int n, void *s
   if (n < 0) return S4KV_ERR_INVALID_ARG;
   if (n == 0) return S4KV_OK;
   if (host_src == nullptr || staging == nullptr || !aligned(staging, 16)) return S4KV_ERR_INVALID_ARG;
-  const size_t bytes = static_cast<size_t>(n) * cache->num_kv_heads * S4KV_BLOCK_BYTES;
+  const size_t bytes = static_cast<size_t>(n) * record_bytes(cache);
   if (cudaMemcpyAsync(staging, host_src, bytes, cudaMemcpyHostToDevice, static_cast<cudaStream_t>(stream)) !=
       cudaSuccess) {
     cudaGetLastError();

@@ -83,8 +83,10 @@ __global__ void __launch_bounds__(128) append_kernel(const AppendParams p) {
     __syncthreads();
 
     if (phys_ok) {
-      uint8_t *blk = p.pool + (static_cast<long>(phys) * H + h) * kBlockBytes;
-      quantize_page_cta(ks, vs, kc, vc, blk, tid);
+      if (p.bits == 8)
+        quantize_page_cta<8>(ks, vs, kc, vc, p.pool + (static_cast<long>(phys) * H + h) * Fmt<8>::kBlock, tid);
+      else
+        quantize_page_cta<4>(ks, vs, kc, vc, p.pool + (static_cast<long>(phys) * H + h) * Fmt<4>::kBlock, tid);
     }
     if (slot != 0) return;
     __syncthreads();  // residual rows read above before the tail overwrites them

@@ -19,6 +19,30 @@ constexpr int kKZeroOff = 2304;
 constexpr int kVScaleOff = 2560;
 constexpr int kVZeroOff = 2688;
 
+// Block layout of one (page, kv head) with kBits-bit codes (4 or 8): K codes,
+// V codes, K scale fp16 [128], K zero fp16 [128] (MMA k order), V scale fp16
+// [4][16], V zero fp16 [4][16].  Fmt<4> is the 2816-byte int4 block above.
+// 8-bit codes keep the int4 assignment of (token, channel) to MMA operand
+// fragments with bytes for nibbles: a lane's 8 codes of one tile are 8
+// consecutive bytes (register r at bytes 2r, 2r + 1) and the 16 bytes of
+// tiles 2m, 2m + 1 of lane l sit at (32 m + l) * 16.
+template <int kBits>
+struct Fmt {
+  static constexpr int kCodeBytes = kPage * kHeadDim * kBits / 8;
+  static constexpr int kKCode = 0;
+  static constexpr int kVCode = kCodeBytes;
+  static constexpr int kKScale = 2 * kCodeBytes;
+  static constexpr int kKZero = kKScale + 2 * kHeadDim;
+  static constexpr int kVScale = kKZero + 2 * kHeadDim;
+  static constexpr int kVZero = kVScale + 2 * kPage * (kHeadDim / kVGroup);
+  static constexpr int kBlock = kVZero + 2 * kPage * (kHeadDim / kVGroup);
+  static constexpr int kLevels = (1 << kBits) - 1;
+};
+static_assert(Fmt<4>::kBlock == kBlockBytes && Fmt<4>::kVZero == kVZeroOff, "int4 block layout");
+static_assert(Fmt<8>::kBlock == S4KV_BLOCK_BYTES_INT8, "int8 block layout");
+
+__host__ __device__ constexpr int block_bytes_for(int bits) { return bits == 8 ? Fmt<8>::kBlock : Fmt<4>::kBlock; }
+
 __device__ __forceinline__ void flag_error(uint32_t *err, uint32_t bits) {
   if (err != nullptr) atomicOr(err, bits);
 }
@@ -33,8 +57,8 @@ __device__ __forceinline__ bool total_less(float a, float b) {
 // One quantization group in fp32: s = (max - min) / 15 and
 // code = s == 0 ? 0 : clamp(rint((x - min) / s), 0, 15), every operation
 // IEEE-rounded (no contraction, no fast math).
-__device__ __forceinline__ float group_scale(float mn, float mx) {
-  return __fdiv_rn(__fsub_rn(mx, mn), 15.0f);
+__device__ __forceinline__ float group_scale(float mn, float mx, int levels = 15) {
+  return __fdiv_rn(__fsub_rn(mx, mn), static_cast<float>(levels));
 }
 __device__ __forceinline__ uint32_t group_code(float x, float mn, float s) {
   if (s == 0.0f) return 0u;
@@ -45,16 +69,16 @@ __device__ __forceinline__ uint32_t group_code(float x, float mn, float s) {
 
 // The same code with the division replaced by a product with inv_s =
 // RN(1 / s) wherever that cannot change it: with x_ = x - min and x_ / s <=
-// 16, the product is within 2^-19 of x_ / s and RN(x_ / s) within 2^-20, so
+// 256, the product is within 2^-15 of x_ / s and RN(x_ / s) within 2^-16, so
 // the two round to the same integer unless the product lies within 2^-10 of
 // a half-integer; only then is the division done.
-__device__ __forceinline__ uint32_t group_code_fast(float x, float mn, float s, float inv_s) {
+__device__ __forceinline__ uint32_t group_code_fast(float x, float mn, float s, float inv_s, int levels = 15) {
   if (s == 0.0f) return 0u;
   const float d = __fsub_rn(x, mn);
   const float q = __fmul_rn(d, inv_s);
   float r = rintf(q);
   if (fabsf(fabsf(__fsub_rn(q, r)) - 0.5f) < 0x1p-10f) r = rintf(__fdiv_rn(d, s));
-  r = fminf(fmaxf(r, 0.0f), 15.0f);
+  r = fminf(fmaxf(r, 0.0f), static_cast<float>(levels));
   return static_cast<uint32_t>(r);
 }
 
@@ -89,6 +113,24 @@ __device__ __forceinline__ void unpack_codes(uint32_t w, uint32_t &a0, uint32_t 
   a1 = h2_as_u32(__hfma2(u32_as_h2(and_or(w, 0x00F000F0u, 0x64006400u)), k16th, kneg64));
   a2 = h2_as_u32(__hsub2(u32_as_h2(and_or(w8, 0x000F000Fu, 0x64006400u)), k1024));
   a3 = h2_as_u32(__hfma2(u32_as_h2(and_or(w8, 0x00F000F0u, 0x64006400u)), k16th, kneg64));
+}
+
+// One lane's 8-bit tile fragment (two words, registers 0-1 in w0 and 2-3 in
+// w1, the low half of a register in its lower byte) -> the four f16x2
+// registers: each byte pair is laid into the mantissa of 1024 (0x64 high
+// bytes, one byte permute) and the 1024 removed exactly in fp16.
+__device__ __forceinline__ void unpack_codes8(uint32_t w0, uint32_t w1, uint32_t &a0, uint32_t &a1,
+                                              uint32_t &a2, uint32_t &a3) {
+  const __half2 k1024 = u32_as_h2(0x64006400u);
+  uint32_t p0, p1, p2, p3;
+  asm("prmt.b32 %0, %1, %2, 0x7170;" : "=r"(p0) : "r"(w0), "r"(0x64646464u));
+  asm("prmt.b32 %0, %1, %2, 0x7372;" : "=r"(p1) : "r"(w0), "r"(0x64646464u));
+  asm("prmt.b32 %0, %1, %2, 0x7170;" : "=r"(p2) : "r"(w1), "r"(0x64646464u));
+  asm("prmt.b32 %0, %1, %2, 0x7372;" : "=r"(p3) : "r"(w1), "r"(0x64646464u));
+  a0 = h2_as_u32(__hsub2(u32_as_h2(p0), k1024));
+  a1 = h2_as_u32(__hsub2(u32_as_h2(p1), k1024));
+  a2 = h2_as_u32(__hsub2(u32_as_h2(p2), k1024));
+  a3 = h2_as_u32(__hsub2(u32_as_h2(p3), k1024));
 }
 
 // ------------------------------------------------------------- warp MMA --

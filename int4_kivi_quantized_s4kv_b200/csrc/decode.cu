@@ -58,7 +58,13 @@ namespace s4kv {
 #ifndef S4KV_DECODE_MIN_CTAS
 #define S4KV_DECODE_MIN_CTAS 3
 #endif
-constexpr int kStages = S4KV_DECODE_STAGES;
+#ifndef S4KV_DECODE_STAGES_INT8
+#define S4KV_DECODE_STAGES_INT8 5
+#endif
+// stages of a warp's ring for kBits-bit pages (the 4864-byte int8 blocks get
+// fewer, so that two CTAs still fit on an SM)
+template <int kBits>
+__host__ __device__ constexpr int stages_for() { return kBits == 8 ? S4KV_DECODE_STAGES_INT8 : S4KV_DECODE_STAGES; }
 constexpr int kWarpsPerCta = S4KV_DECODE_WARPS;
 constexpr int kThreads = 32 * kWarpsPerCta;
 constexpr long long kWaitLimitCycles = 2000000000LL;  // about one second
@@ -72,9 +78,12 @@ constexpr float kHeadroom = 4.0f;  // log2 headroom of the softmax reference
 #endif
 constexpr int kQBytesPerWarp = S4KV_Q_IN_SMEM ? 2048 : 0;
 
-size_t decode_smem_bytes() {
-  return static_cast<size_t>(kWarpsPerCta) * (kStages * (kBlockBytes + 8) + kQBytesPerWarp);
+template <int kBits>
+constexpr size_t smem_bytes_for() {
+  return static_cast<size_t>(kWarpsPerCta) * (stages_for<kBits>() * (Fmt<kBits>::kBlock + 8) + kQBytesPerWarp);
 }
+
+size_t decode_smem_bytes(int bits) { return bits == 8 ? smem_bytes_for<8>() : smem_bytes_for<4>(); }
 
 __device__ __forceinline__ int clamp_len(int L, int max_pages) {
   return min(max(L, 0), max_pages * kPage);
@@ -137,12 +146,13 @@ struct StageAddr {
   uint32_t code, kmeta, vscale, kzero, vzero;
 };
 
+template <int kBits>
 __device__ __forceinline__ StageAddr stage_addr_of(uint32_t stage_base, int lane) {
   const int i = lane & 3;
   const uint32_t half_k = (lane >> 4) ? 16u : 0u;
   return StageAddr{stage_base + 16u * lane, stage_base + 64u * i, stage_base + 4u * i,
-                   stage_base + kKZeroOff + half_k,
-                   stage_base + kVZeroOff + 32u * ((lane & 7) & 3) + half_k};
+                   stage_base + Fmt<kBits>::kKZero + half_k,
+                   stage_base + Fmt<kBits>::kVZero + 32u * ((lane & 7) & 3) + half_k};
 }
 
 // Logits of one quantized page: this lane's S^T[tokens n, n+8][heads 2i,
@@ -177,21 +187,44 @@ __device__ __forceinline__ void ldmatrix_kzero(uint32_t base, int kt, uint32_t &
   }
 }
 
+// Operand fragment of key / value tile kt of a quantized page (kt constant
+// after unrolling): one 4-bit code word, or two 8-bit words of the chunk
+// that holds tiles 2m, 2m + 1 of this lane.
+template <int kBits>
+__device__ __forceinline__ void tile_fragment(const uint32_t (&w)[8], int kt, uint32_t &a0, uint32_t &a1,
+                                              uint32_t &a2, uint32_t &a3) {
+  if (kBits == 8) unpack_codes8(w[2 * (kt & 1)], w[2 * (kt & 1) + 1], a0, a1, a2, a3);
+  else unpack_codes(w[kt], a0, a1, a2, a3);
+}
+
+template <int kBits>
 __device__ __forceinline__ void qk_page(const StageAddr &a, const QFrag &q, float (&S)[4]) {
+  using F = Fmt<kBits>;
   // three independent accumulators (hi part, lo part, zero-point term) keep
   // the dependent MMA chains 8 deep instead of 24
   float Sh[4] = {0.f, 0.f, 0.f, 0.f}, Sl[4] = {0.f, 0.f, 0.f, 0.f}, Sz[4] = {0.f, 0.f, 0.f, 0.f};
   // Sl and Sz both collect small terms (lo parts, zero points); even k-tiles
   // put their lo part in Sl and zero point in Sz, odd k-tiles the reverse,
   // so the two chains stay balanced and S = Sh + (Sl + Sz).
-  const uint4 kw0 = lds128<kKCodeOff>(a.code);
-  const uint4 kw1 = lds128<kKCodeOff + 512>(a.code);
-  const uint32_t kws[8] = {kw0.x, kw0.y, kw0.z, kw0.w, kw1.x, kw1.y, kw1.z, kw1.w};
+  // 4-bit: all 8 tiles' words in two 16-byte loads; 8-bit: tiles 2m, 2m+1
+  // per 16-byte load, inside the loop
+  uint32_t kws[8];
+  if (kBits == 4) {
+    const uint4 kw0 = lds128<F::kKCode>(a.code);
+    const uint4 kw1 = lds128<F::kKCode + 512>(a.code);
+    kws[0] = kw0.x; kws[1] = kw0.y; kws[2] = kw0.z; kws[3] = kw0.w;
+    kws[4] = kw1.x; kws[5] = kw1.y; kws[6] = kw1.z; kws[7] = kw1.w;
+  }
 #pragma unroll
   for (int m = 0; m < 4; ++m) {
+    if (kBits == 8) {
+      const uint4 cw = m == 0 ? lds128<F::kKCode>(a.code) : m == 1 ? lds128<F::kKCode + 512>(a.code)
+                     : m == 2 ? lds128<F::kKCode + 1024>(a.code) : lds128<F::kKCode + 1536>(a.code);
+      kws[0] = cw.x; kws[1] = cw.y; kws[2] = cw.z; kws[3] = cw.w;
+    }
     // key scales and query words for k-tiles 2m, 2m+1 (four channel pairs)
-    const uint4 sv = m == 0 ? lds128<kKScaleOff>(a.kmeta) : m == 1 ? lds128<kKScaleOff + 16>(a.kmeta)
-                   : m == 2 ? lds128<kKScaleOff + 32>(a.kmeta) : lds128<kKScaleOff + 48>(a.kmeta);
+    const uint4 sv = m == 0 ? lds128<F::kKScale>(a.kmeta) : m == 1 ? lds128<F::kKScale + 16>(a.kmeta)
+                   : m == 2 ? lds128<F::kKScale + 32>(a.kmeta) : lds128<F::kKScale + 48>(a.kmeta);
     const uint4 qv = q.pair(m);
     const uint32_t sk[4] = {sv.x, sv.y, sv.z, sv.w};
     const uint32_t qw[4] = {qv.x, qv.y, qv.z, qv.w};
@@ -199,7 +232,7 @@ __device__ __forceinline__ void qk_page(const StageAddr &a, const QFrag &q, floa
     for (int h = 0; h < 2; ++h) {
       const int kt = 2 * m + h;
       uint32_t a0, a1, a2, a3;
-      unpack_codes(kws[kt], a0, a1, a2, a3);
+      tile_fragment<kBits>(kws, kt, a0, a1, a2, a3);
       const __half2 qb0 = u32_as_h2(qw[2 * h]), qb1 = u32_as_h2(qw[2 * h + 1]);
       const __half2 s0 = u32_as_h2(sk[2 * h]), s1 = u32_as_h2(sk[2 * h + 1]);
       // q * sK split into fp16 hi + lo; the lo part is the exact remainder
@@ -284,11 +317,16 @@ __device__ __forceinline__ void softmax_page(const float (&S)[4], float scale_lo
 }
 
 // O += V^T P for one quantized page.
-template <int G4>
-__device__ __forceinline__ void pv_group(const StageAddr &a, const uint32_t (&P)[4], const uint32_t (&vws)[8],
+template <int kBits, int G4>
+__device__ __forceinline__ void pv_group(const StageAddr &a, const uint32_t (&P)[4], uint32_t (&vws)[8],
                                          Online &st) {
-  const __half2 sv0 = u32_as_h2(lds32<kVScaleOff + 32 * G4>(a.vscale));
-  const __half2 sv1 = u32_as_h2(lds32<kVScaleOff + 32 * G4 + 16>(a.vscale));
+  using F = Fmt<kBits>;
+  if (kBits == 8) {  // M-tiles 2 G4, 2 G4 + 1 of this lane: one 16-byte chunk
+    const uint4 cw = lds128<F::kVCode + 512 * G4>(a.code);
+    vws[0] = cw.x; vws[1] = cw.y; vws[2] = cw.z; vws[3] = cw.w;
+  }
+  const __half2 sv0 = u32_as_h2(lds32<F::kVScale + 32 * G4>(a.vscale));
+  const __half2 sv1 = u32_as_h2(lds32<F::kVScale + 32 * G4 + 16>(a.vscale));
   // (P * sV) in fp16 hi + lo: P-hi * sV exactly as two halves, plus P-lo * sV
   const __half2 bh0 = __hmul2(u32_as_h2(P[0]), sv0);
   const __half2 bh1 = __hmul2(u32_as_h2(P[1]), sv1);
@@ -298,20 +336,25 @@ __device__ __forceinline__ void pv_group(const StageAddr &a, const uint32_t (&P)
   for (int j = 0; j < 2; ++j) {
     const int mt = 2 * G4 + j;
     uint32_t a0, a1, a2, a3;
-    unpack_codes(vws[mt], a0, a1, a2, a3);
+    tile_fragment<kBits>(vws, mt, a0, a1, a2, a3);
     mma16816(st.O[mt], a0, a1, a2, a3, h2_as_u32(bh0), h2_as_u32(bh1));
     mma16816(st.O[mt], a0, a1, a2, a3, h2_as_u32(bl0), h2_as_u32(bl1));
   }
 }
 
+template <int kBits>
 __device__ __forceinline__ void pv_page(const StageAddr &a, const uint32_t (&P)[4], Online &st) {
-  const uint4 vw0 = lds128<kVCodeOff>(a.code);
-  const uint4 vw1 = lds128<kVCodeOff + 512>(a.code);
-  const uint32_t vws[8] = {vw0.x, vw0.y, vw0.z, vw0.w, vw1.x, vw1.y, vw1.z, vw1.w};
-  pv_group<0>(a, P, vws, st);
-  pv_group<1>(a, P, vws, st);
-  pv_group<2>(a, P, vws, st);
-  pv_group<3>(a, P, vws, st);
+  uint32_t vws[8];
+  if (kBits == 4) {
+    const uint4 vw0 = lds128<Fmt<4>::kVCode>(a.code);
+    const uint4 vw1 = lds128<Fmt<4>::kVCode + 512>(a.code);
+    vws[0] = vw0.x; vws[1] = vw0.y; vws[2] = vw0.z; vws[3] = vw0.w;
+    vws[4] = vw1.x; vws[5] = vw1.y; vws[6] = vw1.z; vws[7] = vw1.w;
+  }
+  pv_group<kBits, 0>(a, P, vws, st);
+  pv_group<kBits, 1>(a, P, vws, st);
+  pv_group<kBits, 2>(a, P, vws, st);
+  pv_group<kBits, 3>(a, P, vws, st);
   // value zero points: A row r carries group r % 4's zV (one ldmatrix), B = P
   uint32_t z0, z1, z2, z3;
   ldmatrix_x4<0>(a.vzero, z0, z1, z2, z3);
@@ -456,6 +499,7 @@ __device__ __forceinline__ void residual_row_write(const DecodeParams &p, const 
 
 // One completed page (job = sequence, kv head, physical page) quantized by
 // all threads of the CTA, with `scratch` (12 KB of shared memory) as staging.
+template <int kBits>
 __device__ __forceinline__ void cta_quantize_job(const DecodeParams &p, const FusedAppend &f, int4 job, uint8_t *scratch,
                                                  int tid) {
   const int b = job.x, h = job.y, phys = job.w;
@@ -474,14 +518,17 @@ __device__ __forceinline__ void cta_quantize_job(const DecodeParams &p, const Fu
     *reinterpret_cast<uint4 *>(&vs[t][c8]) = *reinterpret_cast<const uint4 *>(sv);
   }
   __syncthreads();
-  quantize_page_cta(ks, vs, kc, vc, const_cast<uint8_t *>(p.pool) + (static_cast<long>(phys) * H + h) * kBlockBytes,
+  quantize_page_cta<kBits>(ks, vs, kc, vc,
+                           const_cast<uint8_t *>(p.pool) + (static_cast<long>(phys) * H + h) * Fmt<kBits>::kBlock,
                     tid);
   __syncthreads();  // the scratch is reused by the next job
 }
 
 // kFused: the step's append is fused in (DecodeParams::k_new / v_new set).
-template <bool kFused>
+template <int kBits, bool kFused>
 __global__ void __launch_bounds__(kThreads, S4KV_DECODE_MIN_CTAS) decode_kernel(const DecodeParams p, const FusedAppend f) {
+  constexpr int kStages = stages_for<kBits>();
+  constexpr int kBlockBytes = Fmt<kBits>::kBlock;
   extern __shared__ __align__(128) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n = lane >> 2, i = lane & 3;
@@ -603,7 +650,7 @@ __global__ void __launch_bounds__(kThreads, S4KV_DECODE_MIN_CTAS) decode_kernel(
       if (lane == 0) s_njob[warp] = nj;
       __syncthreads();
       for (int w = 0; w < kWarpsPerCta; ++w)
-        for (int j = 0; j < s_njob[w]; ++j) cta_quantize_job(p, f, s_job[w][j], smem, threadIdx.x);
+        for (int j = 0; j < s_njob[w]; ++j) cta_quantize_job<kBits>(p, f, s_job[w][j], smem, threadIdx.x);
       // the pool writes are read next by bulk copies (async proxy)
       asm volatile("fence.proxy.async.global;" ::: "memory");
       if (!__syncthreads_or(more)) break;
@@ -687,7 +734,7 @@ __global__ void __launch_bounds__(kThreads, S4KV_DECODE_MIN_CTAS) decode_kernel(
     const bool ok = mbar_wait_bounded(q.bar, q.phase, kWaitLimitCycles);
     return !__any_sync(kFull, !ok);
   };
-  auto addr = [&](const Pos &q) { return stage_addr_of(ring0 + q.off, lane); };
+  auto addr = [&](const Pos &q) { return stage_addr_of<kBits>(ring0 + q.off, lane); };
   auto release = [&]() {      // the page at c0 has been read completely
     fence_proxy_async();
     __syncwarp();
@@ -756,22 +803,22 @@ __global__ void __launch_bounds__(kThreads, S4KV_DECODE_MIN_CTAS) decode_kernel(
       }
       {
         float S0[4];
-        qk_page(addr(c0), qf, S0);
+        qk_page<kBits>(addr(c0), qf, S0);
         if (nq > 1) {
           const Pos c1 = next_pos(c0);
           if (!wait_copy(c1)) {
             failed = true;
             break;
           }
-          qk_page(addr(c1), qf, Sa);
+          qk_page<kBits>(addr(c1), qf, Sa);
         }
         softmax_page(S0, p.scale_log2, st, Pa);
       }
       // one pipeline step: in (Pcur = P(j), Snext = S(j+1)), out (Pnext, Snext2)
       auto step = [&](const uint32_t (&Pcur)[4], const float (&Snext)[4], uint32_t (&Pnext)[4],
                       float (&Snext2)[4]) {
-        qk_page(addr(c2), qf, Snext2);
-        pv_page(addr(c0), Pcur, st);
+        qk_page<kBits>(addr(c2), qf, Snext2);
+        pv_page<kBits>(addr(c0), Pcur, st);
         softmax_page(Snext, p.scale_log2, st, Pnext);  // after PV(j): a rescale covers it
         release();
         c2 = next_pos(c2);
@@ -801,15 +848,15 @@ __global__ void __launch_bounds__(kThreads, S4KV_DECODE_MIN_CTAS) decode_kernel(
       // the last one or two pages
       uint32_t Pt[4];
       if (odd) {
-        pv_page(addr(c0), Pb, st);
+        pv_page<kBits>(addr(c0), Pb, st);
         if (nq > 1) softmax_page(Sb, p.scale_log2, st, Pt);
       } else {
-        pv_page(addr(c0), Pa, st);
+        pv_page<kBits>(addr(c0), Pa, st);
         if (nq > 1) softmax_page(Sa, p.scale_log2, st, Pt);
       }
       release();
       if (nq > 1) {
-        pv_page(addr(c0), Pt, st);
+        pv_page<kBits>(addr(c0), Pt, st);
         release();
       }
     }
@@ -904,30 +951,45 @@ __global__ void __launch_bounds__(kThreads, S4KV_DECODE_MIN_CTAS) decode_kernel(
   }
 }
 
-int decode_ctas_per_sm() {
-  int n = 0;
-  int m = 0;
-  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_kernel<false>, kThreads, decode_smem_bytes());
-  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&m, decode_kernel<true>, kThreads, decode_smem_bytes());
-  n = n < m ? n : m;  // one launch shape (and workspace size) serves both
-  return n;
+template <int kBits>
+int ctas_per_sm_for() {
+  int n = 0, m = 0;
+  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_kernel<kBits, false>, kThreads, smem_bytes_for<kBits>());
+  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&m, decode_kernel<kBits, true>, kThreads, smem_bytes_for<kBits>());
+  return n < m ? n : m;  // one launch shape serves the plain and the fused kernel
 }
+
+int decode_ctas_per_sm(int bits) { return bits == 8 ? ctas_per_sm_for<8>() : ctas_per_sm_for<4>(); }
 
 int decode_warps_per_cta() { return kWarpsPerCta; }
 
-cudaError_t prepare_decode_kernel() {
-  const cudaError_t e = cudaFuncSetAttribute(decode_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             static_cast<int>(decode_smem_bytes()));
+template <int kBits>
+cudaError_t prepare_for() {
+  const int bytes = static_cast<int>(smem_bytes_for<kBits>());
+  cudaError_t e = cudaFuncSetAttribute(decode_kernel<kBits, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
   if (e != cudaSuccess) return e;
-  return cudaFuncSetAttribute(decode_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              static_cast<int>(decode_smem_bytes()));
+  return cudaFuncSetAttribute(decode_kernel<kBits, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
 }
 
-void launch_decode(const DecodeParams &p, const FusedAppend &f, int num_ctas, cudaStream_t stream) {
-  if (f.k_new != nullptr)
-    decode_kernel<true><<<num_ctas, kThreads, decode_smem_bytes(), stream>>>(p, f);
-  else
-    decode_kernel<false><<<num_ctas, kThreads, decode_smem_bytes(), stream>>>(p, f);
+cudaError_t prepare_decode_kernel() {
+  const cudaError_t e = prepare_for<4>();
+  if (e != cudaSuccess) return e;
+  return prepare_for<8>();
+}
+
+void launch_decode(const DecodeParams &p, const FusedAppend &f, int bits, int num_ctas, cudaStream_t stream) {
+  const bool fused = f.k_new != nullptr;
+  if (bits == 8) {
+    if (fused)
+      decode_kernel<8, true><<<num_ctas, kThreads, smem_bytes_for<8>(), stream>>>(p, f);
+    else
+      decode_kernel<8, false><<<num_ctas, kThreads, smem_bytes_for<8>(), stream>>>(p, f);
+  } else {
+    if (fused)
+      decode_kernel<4, true><<<num_ctas, kThreads, smem_bytes_for<4>(), stream>>>(p, f);
+    else
+      decode_kernel<4, false><<<num_ctas, kThreads, smem_bytes_for<4>(), stream>>>(p, f);
+  }
 }
 
 }  // namespace s4kv

@@ -1,13 +1,21 @@
 // s4kv_dequant_page / s4kv_dequant_pages device side: physical pages, all kv
 // heads, back to natural [token][channel] order (page i of a list goes to
 // output slot i).  x = code * scale + zero in fp32 (the
-// product of a 4-bit code and an fp16 scale is exact, so this is a single
-// rounding); the fp16 output is that fp32 value rounded to nearest even.
+// product of a 4- or 8-bit code and an fp16 scale is exact, so this is a
+// single rounding); the fp16 output is that fp32 value rounded to nearest
+// even.
 #include "kernels.cuh"
 
 namespace s4kv {
 
-__device__ __forceinline__ uint32_t code_at(const uint8_t *region, int word, int nibble) {
+// The code at 4-bit position (word, nibble): that nibble, or with 8-bit
+// codes the byte holding the same fragment place (tile 4*(word/128) +
+// word%4, lane (word/4)%32, register nibble%4, half nibble/4).
+__device__ __forceinline__ uint32_t code_at(const uint8_t *region, int word, int nibble, int bits) {
+  if (bits == 8) {
+    const int tile = 4 * (word >> 7) + (word & 3), lane = (word >> 2) & 31;
+    return region[((tile >> 1) * 32 + lane) * 16 + (tile & 1) * 8 + 2 * (nibble & 3) + (nibble >> 2)];
+  }
   const uint32_t w = reinterpret_cast<const uint32_t *>(region)[word];
   return (w >> (4 * nibble)) & 0xFu;
 }
@@ -24,10 +32,14 @@ __global__ void __launch_bounds__(128) dequant_kernel(const DequantParams p) {
       return;
     }
   }
-  const uint8_t *blk = p.pool + (static_cast<long>(page) * p.num_kv_heads + h) * kBlockBytes;
-  const float ks = __half2float(reinterpret_cast<const __half *>(blk + kKScaleOff)[c]);
+  const bool b8 = p.bits == 8;
+  const int kcode_off = 0, vcode_off = b8 ? Fmt<8>::kVCode : Fmt<4>::kVCode;
+  const int kscale_off = b8 ? Fmt<8>::kKScale : Fmt<4>::kKScale, kzero_off = b8 ? Fmt<8>::kKZero : Fmt<4>::kKZero;
+  const int vscale_off = b8 ? Fmt<8>::kVScale : Fmt<4>::kVScale, vzero_off = b8 ? Fmt<8>::kVZero : Fmt<4>::kVZero;
+  const uint8_t *blk = p.pool + (static_cast<long>(page) * p.num_kv_heads + h) * block_bytes_for(p.bits);
+  const float ks = __half2float(reinterpret_cast<const __half *>(blk + kscale_off)[c]);
   const int zslot = 16 * ((c & 31) >> 2) + 2 * (c >> 5) + (c & 1) + 8 * ((c & 3) >> 1);
-  const float kz = __half2float(reinterpret_cast<const __half *>(blk + kKZeroOff)[zslot]);
+  const float kz = __half2float(reinterpret_cast<const __half *>(blk + kzero_off)[zslot]);
   const int g = c / kVGroup;
   // key fragment coordinates of channel c: lane quarter i, tile kt, pair e
   const int ki = c >> 5, kt = (c & 31) >> 2, ke = c & 3;
@@ -39,10 +51,10 @@ __global__ void __launch_bounds__(128) dequant_kernel(const DequantParams p) {
     const int vi = (t & 7) >> 1;
     const int vword = 128 * (vm >> 2) + 4 * (4 * vn + vi) + (vm & 3);
     const int vnib = (ve & 1) + 2 * (t >> 3) + 4 * (t & 1);
-    const float kcode = static_cast<float>(code_at(blk + kKCodeOff, kword, knib));
-    const float vcode = static_cast<float>(code_at(blk + kVCodeOff, vword, vnib));
-    const float vs = __half2float(reinterpret_cast<const __half *>(blk + kVScaleOff)[g * kPage + t]);
-    const float vz = __half2float(reinterpret_cast<const __half *>(blk + kVZeroOff)[g * kPage + t]);
+    const float kcode = static_cast<float>(code_at(blk + kcode_off, kword, knib, p.bits));
+    const float vcode = static_cast<float>(code_at(blk + vcode_off, vword, vnib, p.bits));
+    const float vs = __half2float(reinterpret_cast<const __half *>(blk + vscale_off)[g * kPage + t]);
+    const float vz = __half2float(reinterpret_cast<const __half *>(blk + vzero_off)[g * kPage + t]);
     const float kx = __fadd_rn(__fmul_rn(kcode, ks), kz);
     const float vx = __fadd_rn(__fmul_rn(vcode, vs), vz);
     const long o = ((static_cast<long>(slot) * p.num_kv_heads + h) * kPage + t) * kHeadDim + c;

@@ -23,6 +23,7 @@ struct AppendParams {
   int max_pages;
   int max_new;
   int n_tokens;
+  int bits;  // code width, 4 or 8
 };
 
 struct DequantParams {
@@ -36,6 +37,7 @@ struct DequantParams {
   int num_pages;
   int num_kv_heads;
   int out_fp32;
+  int bits;  // code width, 4 or 8
 };
 
 // Copy of whole records: item i copies rec_bytes from
@@ -107,11 +109,11 @@ struct PrefillParams {
 void launch_append(const AppendParams &p, int batch, int max_new, cudaStream_t stream);
 void launch_dequant(const DequantParams &p, cudaStream_t stream);
 void launch_move(const MoveParams &p, cudaStream_t stream);
-void launch_decode(const DecodeParams &p, const FusedAppend &f, int num_ctas, cudaStream_t stream);
-int decode_ctas_per_sm();
+void launch_decode(const DecodeParams &p, const FusedAppend &f, int bits, int num_ctas, cudaStream_t stream);
+int decode_ctas_per_sm(int bits);
 int decode_warps_per_cta();
 cudaError_t prepare_decode_kernel();
-size_t decode_smem_bytes();
+size_t decode_smem_bytes(int bits);
 void launch_prefill(const PrefillParams &p, int batch, int max_new, cudaStream_t stream);
 cudaError_t prepare_prefill_kernel();
 size_t prefill_smem_bytes();

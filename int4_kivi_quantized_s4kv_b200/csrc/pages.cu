@@ -1,5 +1,5 @@
 // Page movement: whole page records (all kv heads of one physical page,
-// num_kv_heads * 2816 contiguous bytes) gathered out of the pool, scattered
+// num_kv_heads * block bytes contiguous bytes) gathered out of the pool, scattered
 // back into it, copied inside it, and residual rows copied between batch
 // rows.  These are the operations a paged cache needs to swap sequences out
 // to host memory and back and to fork a sequence copy-on-write ("KV-Cache

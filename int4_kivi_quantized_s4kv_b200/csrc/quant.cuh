@@ -3,7 +3,9 @@
 //
 // KIVI split ("S4 KV -- int4 KV-Cache-Kompression fuer vLLM", "Funktionsweise"
 // step 1): keys asymmetric int4 per channel (one group = one channel over the
-// page's 16 tokens), values int4 per token (groups of 32 channels).
+// page's 16 tokens), values int4 per token (groups of 32 channels); the INT8
+// variant ("KV-Cache-Optimierung -- PagedAttention, quantisierter KV,
+// Speculative Cache", "Warum es zaehlt": INT8/INT4 KV) uses 255 levels.
 #pragma once
 
 #include "common.cuh"
@@ -15,9 +17,11 @@ namespace s4kv {
 // byte scratch in shared memory; blk: the 2816-byte block in global memory.
 // Called by all 128 threads of the CTA (tid = threadIdx.x, whole warps);
 // contains CTA barriers.
+template <int kBits>
 __device__ __forceinline__ void quantize_page_cta(const __half (*ks)[kHeadDim], const __half (*vs)[kHeadDim],
                                                   uint8_t (*kc)[kHeadDim], uint8_t (*vc)[kHeadDim], uint8_t *blk,
                                                   int tid) {
+  using F = Fmt<kBits>;
   // keys: thread c quantizes channel c over the 16 tokens
   {
     const int c = tid;
@@ -28,15 +32,15 @@ __device__ __forceinline__ void quantize_page_cta(const __half (*ks)[kHeadDim], 
       if (total_less(x, mn)) mn = x;
       if (total_less(mx, x)) mx = x;
     }
-    const float s = group_scale(mn, mx);
+    const float s = group_scale(mn, mx, F::kLevels);
     const float inv = __frcp_rn(s);
 #pragma unroll
     for (int t = 0; t < kPage; ++t)
-      kc[t][c] = static_cast<uint8_t>(group_code_fast(__half2float(ks[t][c]), mn, s, inv));
-    reinterpret_cast<__half *>(blk + kKScaleOff)[c] = __float2half_rn(s);
+      kc[t][c] = static_cast<uint8_t>(group_code_fast(__half2float(ks[t][c]), mn, s, inv, F::kLevels));
+    reinterpret_cast<__half *>(blk + F::kKScale)[c] = __float2half_rn(s);
     // zero points in the MMA k order: tile (c%32)/4, slot 2(c/32) + (c%2) + 8((c%4)/2)
     const int zslot = 16 * ((c & 31) >> 2) + 2 * (c >> 5) + (c & 1) + 8 * ((c & 3) >> 1);
-    reinterpret_cast<__half *>(blk + kKZeroOff)[zslot] = __float2half_rn(mn);
+    reinterpret_cast<__half *>(blk + F::kKZero)[zslot] = __float2half_rn(mn);
   }
   // values: one (token, 32-channel group) per thread pair; each thread takes
   // 16 channels and the pair combines its minima and maxima
@@ -52,36 +56,65 @@ __device__ __forceinline__ void quantize_page_cta(const __half (*ks)[kHeadDim], 
     const float omn = __shfl_xor_sync(0xFFFFFFFFu, mn, 1), omx = __shfl_xor_sync(0xFFFFFFFFu, mx, 1);
     if (total_less(omn, mn)) mn = omn;
     if (total_less(mx, omx)) mx = omx;
-    const float s = group_scale(mn, mx);
+    const float s = group_scale(mn, mx, F::kLevels);
     const float inv = __frcp_rn(s);
 #pragma unroll
     for (int j = 0; j < kVGroup / 2; ++j)
-      vc[t][c0 + j] = static_cast<uint8_t>(group_code_fast(__half2float(vs[t][c0 + j]), mn, s, inv));
+      vc[t][c0 + j] = static_cast<uint8_t>(group_code_fast(__half2float(vs[t][c0 + j]), mn, s, inv, F::kLevels));
     if ((tid & 1) == 0) {
-      reinterpret_cast<__half *>(blk + kVScaleOff)[g * kPage + t] = __float2half_rn(s);
-      reinterpret_cast<__half *>(blk + kVZeroOff)[g * kPage + t] = __float2half_rn(mn);
+      reinterpret_cast<__half *>(blk + F::kVScale)[g * kPage + t] = __float2half_rn(s);
+      reinterpret_cast<__half *>(blk + F::kVZero)[g * kPage + t] = __float2half_rn(mn);
     }
   }
   __syncthreads();
-  // pack: word w = 128*hh + 4*lane + q; nibble j is register j&3, half j>>2
-  // of that lane's m16n8k16 operand fragment (tile = 4*hh + q)
-  for (int w = tid; w < 256; w += 128) {
-    const int hh = w >> 7, lane = (w >> 2) & 31, q = w & 3;
-    const int n = lane >> 2, i = lane & 3, tile = 4 * hh + q;
-    uint32_t kw = 0, vw = 0;
+  // (token, channel) of nibble / byte j of tile `tile`, lane = 4n + i
+  auto key_tc = [](int tile, int n, int i, int j, int &t, int &c) {
+    t = 8 * (j & 1) + n;                                   // row = token
+    c = 32 * i + 4 * tile + 2 * ((j >> 1) & 1) + (j >> 2);  // k axis = channel
+  };
+  auto val_tc = [](int tile, int n, int i, int j, int &t, int &c) {
+    t = 2 * i + (j >> 2) + 8 * ((j >> 1) & 1);             // k axis = token
+    c = 32 * (tile >> 1) + 4 * n + 2 * (tile & 1) + (j & 1);  // row = channel
+  };
+  if (kBits == 4) {
+    // word w = 128*hh + 4*lane + q; nibble j is register j&3, half j>>2 of
+    // that lane's m16n8k16 operand fragment (tile = 4*hh + q)
+    for (int w = tid; w < 256; w += 128) {
+      const int hh = w >> 7, lane = (w >> 2) & 31, q = w & 3;
+      const int n = lane >> 2, i = lane & 3, tile = 4 * hh + q;
+      uint32_t kw = 0, vw = 0;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      // keys: row = token, k axis = channel 32i + 4*tile + {0,1 | 2,3}
-      const int kt = 8 * (j & 1) + n;
-      const int kch = 32 * i + 4 * tile + 2 * ((j >> 1) & 1) + (j >> 2);
-      kw |= static_cast<uint32_t>(kc[kt][kch]) << (4 * j);
-      // values: row = channel of M-tile `tile`, k axis = token
-      const int vt = 2 * i + (j >> 2) + 8 * ((j >> 1) & 1);
-      const int vch = 32 * (tile >> 1) + 4 * n + 2 * (tile & 1) + (j & 1);
-      vw |= static_cast<uint32_t>(vc[vt][vch]) << (4 * j);
+      for (int j = 0; j < 8; ++j) {
+        int t, c;
+        key_tc(tile, n, i, j, t, c);
+        kw |= static_cast<uint32_t>(kc[t][c]) << (4 * j);
+        val_tc(tile, n, i, j, t, c);
+        vw |= static_cast<uint32_t>(vc[t][c]) << (4 * j);
+      }
+      reinterpret_cast<uint32_t *>(blk + F::kKCode)[w] = kw;
+      reinterpret_cast<uint32_t *>(blk + F::kVCode)[w] = vw;
     }
-    reinterpret_cast<uint32_t *>(blk + kKCodeOff)[w] = kw;
-    reinterpret_cast<uint32_t *>(blk + kVCodeOff)[w] = vw;
+  } else {
+    // byte (32 m + lane) * 16 + 8 (tile % 2) + 2 r + half holds register r,
+    // half `half` (nibble index j = r + 4 half) of tile 2m + tile % 2
+    for (int w = tid; w < 512; w += 128) {
+      const int chunk = w >> 2, within = w & 3;
+      const int m = chunk >> 5, lane = chunk & 31;
+      const int tile = 2 * m + (within >> 1), r0 = 2 * (within & 1);
+      const int n = lane >> 2, i = lane & 3;
+      uint32_t kw = 0, vw = 0;
+#pragma unroll
+      for (int b = 0; b < 4; ++b) {
+        const int j = (r0 + (b >> 1)) + 4 * (b & 1);
+        int t, c;
+        key_tc(tile, n, i, j, t, c);
+        kw |= static_cast<uint32_t>(kc[t][c]) << (8 * b);
+        val_tc(tile, n, i, j, t, c);
+        vw |= static_cast<uint32_t>(vc[t][c]) << (8 * b);
+      }
+      reinterpret_cast<uint32_t *>(blk + F::kKCode)[w] = kw;
+      reinterpret_cast<uint32_t *>(blk + F::kVCode)[w] = vw;
+    }
   }
 }
 

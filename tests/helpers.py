@@ -56,7 +56,7 @@ class Pair:
     inputs (numpy backend)."""
 
     def __init__(self, spec: W.Spec, layer: int = 0, prefill_chunk=None, device="cuda",
-                 with_gpu=True):
+                 with_gpu=True, bits: int = 4):
         import oracle
         self.spec, self.layer = spec, layer
         self.ctx = W.context_lens(spec)
@@ -70,13 +70,14 @@ class Pair:
             self.k.append(kk)
             self.v.append(vv)
         self.q = W.queries_np(spec, layer)
-        self.oc = oracle.OracleCache(self.plan.num_pages, H, B)
+        self.bits = bits
+        self.oc = oracle.OracleCache(self.plan.num_pages, H, B, bits=bits)
         self.gpu = None
         self.device = device
         if with_gpu:
             import int4_kivi_quantized_s4kv_b200 as S
             self.S = S
-            self.gpu = S.S4KVCache(self.plan.num_pages, H, B, device=device)
+            self.gpu = S.S4KVCache(self.plan.num_pages, H, B, device=device, bits=bits)
             self.bt_dev = self._dev(self.plan.block_tables)
         self.append(np.zeros(B, np.int64), self.ctx, prefill_chunk)
         self.append(self.ctx, self.lens, None)

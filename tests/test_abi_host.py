@@ -69,6 +69,10 @@ def test_cache_layout_matches_block_size(S, oracle_mod):
     pool, res = S.s4kv_cache_layout(1000, 8, 256)
     assert pool == 1000 * 8 * oracle_mod.block_bytes()
     assert res == 256 * 8 * 16 * 128 * 2
+    pool8, res8 = S.s4kv_cache_layout(1000, 8, 256, bits=8)
+    assert pool8 == 1000 * 8 * oracle_mod.block_bytes(8) and res8 == res
+    with pytest.raises(S.S4KVError):
+        S.s4kv_cache_layout(10, 8, 1, bits=2)
     with pytest.raises(S.S4KVError):
         S.s4kv_cache_layout(0, 8, 1)
 
@@ -116,6 +120,14 @@ def test_invalid_calls_rejected_before_launch(S):
     assert L.s4kv_dequant_page(ctypes.byref(c), 10, P(fake), P(fake), 1, st) == S.ERR_INVALID_ARG
     assert L.s4kv_dequant_page(ctypes.byref(c), -1, P(fake), P(fake), 1, st) == S.ERR_INVALID_ARG
     assert L.s4kv_dequant_page(ctypes.byref(bad_dim), 0, P(fake), P(fake), 1, st) == S.ERR_UNSUPPORTED
+    # code width: 4 (or 0) and 8 only; prefill has no 8-bit path
+    bad_bits = S.s4kv_cache_t(fake, fake, fake, None, 10, 2, 4, 128, 16, 3)
+    assert L.s4kv_dequant_page(ctypes.byref(bad_bits), 0, P(fake), P(fake), 1, st) == S.ERR_UNSUPPORTED
+    c8 = S.s4kv_cache_t(fake, fake, fake, None, 10, 2, 4, 128, 16, 8)
+    assert pre(ctypes.byref(c8), P(fake), 8, 4, P(fake), P(fake), P(fake), 1, 1, 4, 0.088, P(fake), st) == S.ERR_UNSUPPORTED
+    n = ctypes.c_size_t(0)
+    assert L.s4kv_page_record_bytes(ctypes.byref(c8), ctypes.byref(n)) == S.OK and n.value == 2 * 4864
+    assert L.s4kv_page_record_bytes(ctypes.byref(c), ctypes.byref(n)) == S.OK and n.value == 2 * 2816
     # error read with no flag word needs no device
     flags = ctypes.c_uint32(7)
     assert L.s4kv_get_error(ctypes.byref(c), ctypes.byref(flags), 1, st) == S.OK and flags.value == 0

@@ -32,7 +32,7 @@ def test_gather_matches_oracle_and_dequant_pages():
     p = _pair()
     S = p.S
     pages = np.array(p.plan.block_tables[1, :int(p.lens[1]) // 16], np.int32)
-    rec = S.s4kv_page_record_bytes(p.spec.num_kv_heads)
+    rec = S.s4kv_page_record_bytes(p.gpu)
     dst = torch.empty((len(pages), rec), dtype=torch.uint8, device="cuda")
     S.s4kv_gather_pages(p.gpu, p._dev(pages), dst)
     torch.cuda.synchronize()
@@ -71,7 +71,7 @@ def test_swap_out_and_back_in_elsewhere():
     before = p.gpu_decode()
     nfull = int(p.lens[2]) // 16
     pages = np.array(p.plan.block_tables[2, :nfull], np.int32)
-    rec = S.s4kv_page_record_bytes(p.spec.num_kv_heads)
+    rec = S.s4kv_page_record_bytes(p.gpu)
     staging = torch.empty((nfull, rec), dtype=torch.uint8, device="cuda")
     host = torch.empty((nfull, rec), dtype=torch.uint8, pin_memory=True)
     S.s4kv_swap_out(p.gpu, p._dev(pages), staging, host)
@@ -158,7 +158,7 @@ def test_bad_page_ids_flag_instead_of_faulting():
     import torch
     p = _pair()
     S = p.S
-    rec = S.s4kv_page_record_bytes(p.spec.num_kv_heads)
+    rec = S.s4kv_page_record_bytes(p.gpu)
     pages = np.array([0, p.plan.num_pages + 3, -1, 1], np.int32)
     dst = torch.full((4, rec), 7, dtype=torch.uint8, device="cuda")
     S.s4kv_gather_pages(p.gpu, p._dev(pages), dst)
