@@ -85,6 +85,7 @@ def lib():
         L.s4kv_ref_quantize_group_bits.restype = f32
         L.s4kv_ref_code_offset8.argtypes = [i32, i32, i32]
         L.s4kv_ref_code_offset8.restype = ctypes.c_long
+        L.s4kv_ref_code_position2.argtypes = [i32, i32, i32, P, P]
         L.s4kv_ref_quantize_page_bits.argtypes = [P, P, P, i32]
         L.s4kv_ref_unpack_codes_bits.argtypes = [P, P, P, i32]
         L.s4kv_ref_dequant_block_bits.argtypes = [P, P, P, i32]
@@ -171,6 +172,14 @@ def code_offset8(is_value: bool, t: int, c: int) -> int:
     return int(lib().s4kv_ref_code_offset8(1 if is_value else 0, int(t), int(c)))
 
 
+def code_position2(is_value: bool, t: int, c: int) -> tuple[int, int]:
+    """(word, bit) of (token t, channel c) in a 2-bit code region."""
+    w = np.zeros(1, np.int64)
+    b = np.zeros(1, np.int32)
+    lib().s4kv_ref_code_position2(1 if is_value else 0, int(t), int(c), _p(w), _p(b))
+    return int(w[0]), int(b[0])
+
+
 def quantize_page(kp, vp, bits: int = 4) -> np.ndarray:
     """fp16 K, V [16][128] of one page and kv head -> block (2816 bytes for
     4-bit codes)."""
@@ -208,12 +217,12 @@ def kv_payload_bytes(layers, kv_heads, head_dim, tokens, bytes_per_elem) -> floa
 # ----------------------------------------------------------------- cache --
 
 class OracleCache:
-    """Host copy of the paged cache: pool u8 [NP][Hkv][block bytes] (2816 for
-    4-bit codes, 4864 for 8-bit), residual fp16 bits [max_seqs][Hkv][16][128]
-    for K and V."""
+    """Host copy of the paged cache: pool u8 [NP][Hkv][block bytes] (1792 for
+    2-bit codes, 2816 for 4-bit, 4864 for 8-bit), residual fp16 bits
+    [max_seqs][Hkv][16][128] for K and V."""
 
     def __init__(self, num_pages: int, num_kv_heads: int, max_seqs: int, bits: int = 4):
-        assert bits in (4, 8)
+        assert bits in (2, 4, 8)
         self.bits = bits
         self.num_pages = num_pages
         self.num_kv_heads = num_kv_heads

@@ -64,7 +64,7 @@
 #define PAGE 16
 #define VGROUP 32
 
-/* Block regions for `bits`-bit codes (4 or 8): K codes, V codes, then the
+/* Block regions for `bits`-bit codes (2, 4 or 8): K codes, V codes, then the
  * fp16 metadata (K scale [128], K zero [128], V scale [4][16], V zero
  * [4][16]); with 4-bit codes this is the 2816-byte block. */
 static long code_bytes(int bits) { return (long)PAGE * HEAD_DIM * bits / 8; }
@@ -215,6 +215,26 @@ static long byte_offset8(int word, int nibble) {
     return ((long)(tile / 2) * 32 + lane) * 16 + (tile % 2) * 8 + 2 * (nibble % 4) + nibble / 4;
 }
 
+/* 2-bit codes keep the same assignment with two bits per code: the 16 codes
+ * of tiles 2m and 2m+1 of one lane form one 32-bit word, word 4*lane + m of
+ * the region (a lane's four words sit together); half 0 of every register
+ * is in the low 16 bits and half 1 in the high 16 bits, register r of tile
+ * 2m+p at bits 2*(4*p + r) of its half. */
+static void bit_position2(int word, int nibble, long *word2, int *bit) {
+    int tile = 4 * (word / 128) + word % 4, lane = (word / 4) % 32;
+    *word2 = 4L * lane + tile / 2;
+    *bit = 16 * (nibble / 4) + 2 * (4 * (tile % 2) + nibble % 4);
+}
+
+/* Word index and bit of the 2-bit code of (token t, channel c) inside the
+ * key (is_value = 0) or value (1) code region. */
+void s4kv_ref_code_position2(int is_value, int t, int c, long *word, int *bit) {
+    int w, nb;
+    if (is_value) s4kv_ref_value_code_slot(t, c, &w, &nb);
+    else s4kv_ref_key_code_slot(t, c, &w, &nb);
+    bit_position2(w, nb, word, bit);
+}
+
 /* Byte offset of the 8-bit code of (token t, channel c) inside the key
  * (is_value = 0) or value (1) code region. */
 long s4kv_ref_code_offset8(int is_value, int t, int c) {
@@ -239,8 +259,19 @@ static void put_code(uint8_t *region, int is_value, int t, int c, int code, int 
     int w, nb;
     if (is_value) s4kv_ref_value_code_slot(t, c, &w, &nb);
     else s4kv_ref_key_code_slot(t, c, &w, &nb);
-    if (bits == 8) region[byte_offset8(w, nb)] = (uint8_t)code;
-    else put_nibble(region, w, nb, code);
+    if (bits == 8) {
+        region[byte_offset8(w, nb)] = (uint8_t)code;
+    } else if (bits == 2) {
+        long w2;
+        int bit;
+        bit_position2(w, nb, &w2, &bit);
+        uint32_t word;
+        memcpy(&word, region + 4 * w2, 4); /* little-endian words */
+        word = (word & ~(3u << bit)) | ((uint32_t)(code & 3) << bit);
+        memcpy(region + 4 * w2, &word, 4);
+    } else {
+        put_nibble(region, w, nb, code);
+    }
 }
 
 static int get_code(const uint8_t *region, int is_value, int t, int c, int bits) {
@@ -248,6 +279,14 @@ static int get_code(const uint8_t *region, int is_value, int t, int c, int bits)
     if (is_value) s4kv_ref_value_code_slot(t, c, &w, &nb);
     else s4kv_ref_key_code_slot(t, c, &w, &nb);
     if (bits == 8) return region[byte_offset8(w, nb)];
+    if (bits == 2) {
+        long w2;
+        int bit;
+        bit_position2(w, nb, &w2, &bit);
+        uint32_t word;
+        memcpy(&word, region + 4 * w2, 4);
+        return (int)((word >> bit) & 3u);
+    }
     return get_nibble(region, w, nb);
 }
 

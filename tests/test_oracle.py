@@ -21,6 +21,10 @@ Which pin covers which oracle function:
                                    quantizer represents exactly; single key; uniform
                                    weights; page permutation and shared-prefix
                                    invariance; GQA identical queries; fp32 vs fp64
+  int2 codes (code_position2, OracleCache(bits=2)) : 4-level closed forms,
+                                   the rounding bound, the bit-pair layout
+                                   against the int4 fragment map, exact-grid
+                                   attention, chunking invariance
   int8 codes (quantize_group_bits, code_offset8, OracleCache(bits=8)) :
                                    256-level closed forms and the rounding bound;
                                    the byte layout against the int4 fragment map;
@@ -766,3 +770,87 @@ def test_int8_append_chunking_invariance(oracle_mod):
         assert np.array_equal(p_, pools[0][0])
         for b, L in enumerate(lens):
             assert np.array_equal(r_[b, :, :L % 16], pools[0][1][b, :, :L % 16])
+
+
+# ------------------------------------------------------------- int2 codes --
+
+def test_int2_group_closed_forms_and_bound(oracle_mod):
+    """3 levels: a 4-level grid gives its indices and step; random groups
+    stay within half a step of their dequantized values."""
+    d, a = 0.5, -1.0
+    k = np.array([0, 3, 1, 2, 2, 1, 0, 3] * 4)
+    codes, sh, zh, s = oracle_mod.quantize_group_bits((a + k * d).astype(np.float16), 2)
+    assert list(codes) == list(k) and s == d and zh == f16bits(a)
+    rng = np.random.default_rng(13)
+    for trial in range(60):
+        x16 = (rng.standard_normal(16 if trial % 2 else 32) * 3).astype(np.float16)
+        codes, sh, zh, s = oracle_mod.quantize_group_bits(x16, 2)
+        assert codes.max() <= 3
+        if s > 0:
+            assert _bound_ok(x16, codes, s, zh)
+            assert codes[np.argmin(x16)] == 0 and codes[np.argmax(x16)] == 3
+
+
+def test_int2_layout_is_the_int4_fragment_map_in_bit_pairs(oracle_mod):
+    """2-bit codes keep the 4-bit fragment assignment: word 4*lane + m holds
+    tiles 2m, 2m+1 of that lane, half h of register r of tile 2m+p at bits
+    16h + 2(4p + r); every (word, bit pair) of the 512-byte region is used
+    exactly once."""
+    for is_value, slot in ((False, oracle_mod.key_code_slot), (True, oracle_mod.value_code_slot)):
+        seen = set()
+        for t in range(PAGE):
+            for c in range(HD):
+                w2, bit = oracle_mod.code_position2(is_value, t, c)
+                lane, m = divmod(w2, 4)
+                half, rest = divmod(bit, 16)
+                p, r = divmod(rest // 2, 4)
+                word, nib = slot(t, c)
+                assert (2 * m + p, lane) == (4 * (word // 128) + word % 4, (word % 128) // 4)
+                assert (r, half) == (nib & 3, nib >> 2) and bit % 2 == 0
+                seen.add((w2, bit))
+        assert seen == {(w, b) for w in range(128) for b in range(0, 32, 2)}
+    assert oracle_mod.block_bytes(2) == 2 * 512 + 768
+
+
+def _grid_page2(rng, per):
+    if per == "key":
+        d = 2.0 ** rng.integers(-4, 0, HD)
+        a = rng.integers(-8, 8, HD) * 0.25
+        codes = np.stack([rng.permutation(np.arange(16) % 4) for _ in range(HD)], axis=1)
+        return (a[None, :] + codes * d[None, :]).astype(np.float16)
+    d = 2.0 ** rng.integers(-4, 0, (PAGE, 4))
+    a = rng.integers(-8, 8, (PAGE, 4)) * 0.25
+    codes = np.stack([np.stack([rng.permutation(np.arange(32) % 4) for _ in range(4)]) for _ in range(PAGE)])
+    return (a[:, :, None] + codes * d[:, :, None]).reshape(PAGE, HD).astype(np.float16)
+
+
+def test_int2_decode_matches_textbook_on_exact_grids(oracle_mod):
+    rng = np.random.default_rng(46)
+    H, G = 1, 4
+    lens = [33, 48, 5]
+    k, v = [], []
+    for L in lens:
+        npg = (L + PAGE - 1) // PAGE
+        kk = np.zeros((npg * PAGE, H, HD), np.float16)
+        vv = np.zeros((npg * PAGE, H, HD), np.float16)
+        for p in range(npg):
+            kk[p * PAGE:(p + 1) * PAGE, 0] = _grid_page2(rng, "key")
+            vv[p * PAGE:(p + 1) * PAGE, 0] = _grid_page2(rng, "value")
+        k.append(kk[:L])
+        v.append(vv[:L])
+    bt, NP = _tables(rng, lens)
+    c = oracle_mod.OracleCache(NP, H, len(lens), bits=2)
+    _append_all(oracle_mod, c, k, v, [0] * 3, lens, bt, 7)
+    q = rng.standard_normal((3, H * G, HD)).astype(np.float16)
+    out = c.decode_attention(q, np.array(lens, np.int32), bt)
+    for b, L in enumerate(lens):
+        for qh in range(H * G):
+            ref = _textbook_attention(q[b, qh], k[b][:, 0], v[b][:, 0], 1 / np.sqrt(HD))
+            assert np.allclose(out[b, qh], ref, rtol=1e-12, atol=1e-12)
+    # chunking invariance of the 2-bit append
+    pools = []
+    for chunk in (None, 3, 16):
+        cc = oracle_mod.OracleCache(NP, H, len(lens), bits=2)
+        _append_all(oracle_mod, cc, k, v, [0] * 3, lens, bt, chunk)
+        pools.append(cc.pool.copy())
+    assert all(np.array_equal(p_, pools[0]) for p_ in pools[1:])
