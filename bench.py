@@ -137,7 +137,7 @@ class ClockSampler:
 # -------------------------------------------------------------- workload --
 
 def step_bytes(spec, plan, lens, bits: int = 4):
-    d = W.decode_bytes(spec, lens, plan, block_bytes=4864 if bits == 8 else 2816)
+    d = W.decode_bytes(spec, lens, plan, block_bytes={2: 1792, 4: 2816, 8: 4864}[bits])
     new = W.step_new_tokens(spec)
     kv_new = int(new.sum()) * spec.num_kv_heads * 128 * 2 * 2   # k and v read
     append = 2 * kv_new                                         # residual write (upper bound)
@@ -492,12 +492,15 @@ def measure_fused_step(wl, device, steps: int = 20):
             "speedup": two / one, "launches_per_layer": {"two_launch": 2, "fused": 1}}
 
 
-def measure_int8_decode(device, spec, steps: int = 20):
-    """The INT8 variant's decode step (append + decode, 4864-byte pages) on
-    the same workload as the headline, against the HBM roofline."""
+BLOCK_BYTES = {2: 1792, 4: 2816, 8: 4864}
+
+
+def measure_width_decode(device, spec, bits: int, steps: int = 20):
+    """The 8- or 2-bit variant's decode step (append + decode) on the same
+    workload as the headline, against the HBM roofline."""
     import torch
-    wl = DeviceWorkload(spec, device, bits=8)
-    dbytes, _ = step_bytes(wl.spec, wl.plan, wl.lens, bits=8)
+    wl = DeviceWorkload(spec, device, bits=bits)
+    dbytes, _ = step_bytes(wl.spec, wl.plan, wl.lens, bits=bits)
     for _ in range(3):
         wl.step()
     torch.cuda.synchronize()
@@ -507,12 +510,12 @@ def measure_int8_decode(device, spec, steps: int = 20):
     torch.cuda.synchronize()
     ms = sum(a.elapsed_time(b) for a, b in zip(*ev)) / steps
     if any(wl.S.s4kv_get_error(c) for c in wl.caches):
-        raise RuntimeError("int8 decode set device error flags")
+        raise RuntimeError(f"int{bits} decode set device error flags")
     peak, kind = measured_hbm_peak()
     gbs = dbytes["algorithmic"] / (ms * 1e-3) / 1e9
-    return {"workload": spec.name, "bits": 8, "block_bytes": 4864, "avg_launch_ms": ms,
+    return {"workload": spec.name, "bits": bits, "block_bytes": BLOCK_BYTES[bits], "avg_launch_ms": ms,
             "tokens_per_s": int(wl.new.sum()) / (ms * 1e-3),
-            "roofline": {"bound": "hbm", "kernel": "decode_kernel<8>", "achieved": gbs, "peak": peak,
+            "roofline": {"bound": "hbm", "kernel": f"decode_kernel<{bits}>", "achieved": gbs, "peak": peak,
                          "peak_kind": kind, "unit": "GB/s", "frac": gbs / peak, "traffic": None,
                          "bytes_per_launch": dbytes["algorithmic"]}}
 
@@ -679,7 +682,7 @@ def main(argv=None):
     value = aggregate_gbs(world, bytes_per_step, step_ms)
     achieved = decode_bytes_per_launch / (dec_avg_ms * 1e-3) / 1e9
     tokens = int(wl.new.sum())
-    prefill = moves = fused = int8 = None
+    prefill = moves = fused = int8 = int2 = None
     if world == 1 and not args.no_prefill:
         prefill = measure_prefill(device, max(3, min(args.steps, 20)))
         moves = measure_page_moves(wl, device)
@@ -687,7 +690,8 @@ def main(argv=None):
         small = DeviceWorkload(W.SPECS["qwen2.5-7b"], device)
         fused.append(measure_fused_step(small, device))
         del small
-        int8 = measure_int8_decode(device, spec)
+        int8 = measure_width_decode(device, spec, 8)
+        int2 = measure_width_decode(device, spec, 2)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(spec)
@@ -724,7 +728,8 @@ def main(argv=None):
         if cpu is not None:
             line["cpu_baseline"] = cpu
         if prefill is not None:
-            line["next_rows"] = {"prefill": prefill, "page_moves": moves, "fused_step": fused, "int8_decode": int8}
+            line["next_rows"] = {"prefill": prefill, "page_moves": moves, "fused_step": fused, "int8_decode": int8,
+                                 "int2_decode": int2}
         print(json.dumps(line), flush=True)
     if world > 1:
         torch.distributed.destroy_process_group()

@@ -63,6 +63,12 @@
  *           with bytes for nibbles: the 8 codes of tile 4*h+q of lane l are
  *           bytes ((32*m + l)*16 + 8*(tile%2) + 2*(j&3) + (j>>2)), m =
  *           tile/2, j the 4-bit nibble index of that (token, channel).
+ *           With 2-bit codes (bits == 2, 3 levels: s = (mx - mn) / 3, codes
+ *           clamped to [0, 3]) the block is S4KV_BLOCK_BYTES_INT2 = 1792
+ *           bytes: [0,512) key codes, [512,1024) value codes, metadata at
+ *           [1024,1792).  The 16 codes of tiles 2m, 2m+1 of lane l are the
+ *           32-bit word 4*l + m: code (register r = j&3, half j>>2) of tile
+ *           2m+p at bit 16*(j>>2) + 2*(4*p + r).
  *  res_k,   fp16 [max_seqs][num_kv_heads][16][128] each.  Row r of batch
  *  res_v    row b holds token 16*floor(L/16) + r of that sequence for
  *           r < L mod 16 (L = its current length); other rows are
@@ -100,6 +106,7 @@ extern "C" {
 #define S4KV_VALUE_GROUP 32
 #define S4KV_BLOCK_BYTES 2816      /* 4-bit codes */
 #define S4KV_BLOCK_BYTES_INT8 4864 /* 8-bit codes */
+#define S4KV_BLOCK_BYTES_INT2 1792 /* 2-bit codes */
 #define S4KV_MAX_GQA_GROUP 8
 
 /* status codes returned by every call */
@@ -128,7 +135,7 @@ typedef struct s4kv_cache {
     int32_t max_seqs;
     int32_t head_dim;    /* must be S4KV_HEAD_DIM */
     int32_t page_tokens; /* must be S4KV_PAGE_TOKENS */
-    int32_t bits;        /* code width: 4 (or 0, meaning 4) or 8 */
+    int32_t bits;        /* code width: 4 (or 0, meaning 4), 8 or 2 */
 } s4kv_cache_t;
 
 /* Library version (S4KV_VERSION). */
@@ -152,8 +159,9 @@ S4KV_API int s4kv_check_model(int head_dim, int page_tokens, int num_q_heads,
 S4KV_API int s4kv_cache_layout(int num_pages, int num_kv_heads, int max_seqs,
                       size_t *pool_bytes, size_t *residual_bytes);
 
-/* The same for a code width of `bits` (4 or 8; INT8 pages take
- * S4KV_BLOCK_BYTES_INT8 bytes per kv head). */
+/* The same for a code width of `bits` (2, 4 or 8; pages then take
+ * S4KV_BLOCK_BYTES_INT2 / S4KV_BLOCK_BYTES / S4KV_BLOCK_BYTES_INT8 bytes per
+ * kv head). */
 S4KV_API int s4kv_cache_layout_bits(int num_pages, int num_kv_heads, int max_seqs, int bits,
                                     size_t *pool_bytes, size_t *residual_bytes);
 
@@ -273,7 +281,7 @@ S4KV_API int s4kv_decode_attention_noalloc(const s4kv_cache_t *cache, const void
  * the softmax weights as fp16 MMA operands (fp32 accumulation), so results
  * agree with exact attention to about fp16 precision of those operands.
  * Allocates nothing; needs about 171 KB of shared memory per CTA.  4-bit
- * codes only (an 8-bit cache is refused with S4KV_ERR_UNSUPPORTED). */
+ * codes only (2- and 8-bit caches are refused with S4KV_ERR_UNSUPPORTED). */
 S4KV_API int s4kv_prefill_attention(const s4kv_cache_t *cache, const void *q,
                                     int num_q_heads, int n_tokens,
                                     const int32_t *cu_new, const int32_t *seq_lens,
@@ -300,7 +308,7 @@ S4KV_API int s4kv_dequant_pages(const s4kv_cache_t *cache, const int32_t *pages,
  * page tables and copies a page only when it is written ("KV-Cache und
  * PagedAttention: Warum Ihr LLM-Server langsamer wird", "Wie PagedAttention
  * das loest").  A page RECORD is all kv heads' blocks of one physical page:
- * num_kv_heads * block bytes (2816 with 4-bit codes, 4864 with 8-bit)
+ * num_kv_heads * block bytes (1792 / 2816 / 4864 with 2- / 4- / 8-bit codes)
  * contiguous bytes, the unit these calls move.  All page
  * and row lists are device int32 arrays; an id out of range sets
  * S4KV_EFLAG_PAGE_RANGE (rows: S4KV_EFLAG_SLOT) and that item is skipped.

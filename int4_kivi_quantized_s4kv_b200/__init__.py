@@ -19,6 +19,7 @@ PAGE_TOKENS = 16
 VALUE_GROUP = 32
 BLOCK_BYTES = 2816
 BLOCK_BYTES_INT8 = 4864
+BLOCK_BYTES_INT2 = 1792
 MAX_GQA_GROUP = 8
 NOALLOC_SCRATCH_BYTES = 24 * 1024 * 1024
 
@@ -146,7 +147,7 @@ class S4KVCache:
         import torch
         pool_bytes, res_bytes = s4kv_cache_layout(num_pages, num_kv_heads, max_seqs, bits)
         self.num_pages, self.num_kv_heads, self.max_seqs, self.bits = num_pages, num_kv_heads, max_seqs, bits
-        block = BLOCK_BYTES if bits == 4 else BLOCK_BYTES_INT8
+        block = {4: BLOCK_BYTES, 8: BLOCK_BYTES_INT8, 2: BLOCK_BYTES_INT2}[bits]
         self.pool = torch.zeros((num_pages, num_kv_heads, block), dtype=torch.uint8, device=device)
         self.res_k = torch.zeros((max_seqs, num_kv_heads, PAGE_TOKENS, HEAD_DIM), dtype=torch.float16, device=device)
         self.res_v = torch.zeros_like(self.res_k)

@@ -21,16 +21,18 @@ constexpr int kMaxDevices = 64;
 struct DeviceShape {
   bool ready = false;
   int num_sms = 0;
-  int num_ctas[2] = {0, 0};     // decode grid for 4-bit / 8-bit pages
-  int num_workers[2] = {0, 0};  // worker warps of that grid
+  int num_ctas[3] = {0, 0, 0};     // decode grid for 4-bit / 8-bit / 2-bit pages
+  int num_workers[3] = {0, 0, 0};  // worker warps of that grid
   int max_workers = 0;          // sizes the (shared) decode workspace
 };
 
-int fmt_index(int bits) { return bits == 8 ? 1 : 0; }
-int cache_bits(const s4kv_cache_t *c) { return c->bits == 8 ? 8 : 4; }
-size_t record_bytes(const s4kv_cache_t *c) {
-  return static_cast<size_t>(c->num_kv_heads) * (cache_bits(c) == 8 ? S4KV_BLOCK_BYTES_INT8 : S4KV_BLOCK_BYTES);
+int fmt_index(int bits) { return bits == 8 ? 1 : bits == 2 ? 2 : 0; }
+int fmt_bits(int index) { return index == 1 ? 8 : index == 2 ? 2 : 4; }
+int cache_bits(const s4kv_cache_t *c) { return c->bits == 8 || c->bits == 2 ? c->bits : 4; }
+size_t block_bytes(int bits) {
+  return bits == 8 ? S4KV_BLOCK_BYTES_INT8 : bits == 2 ? S4KV_BLOCK_BYTES_INT2 : S4KV_BLOCK_BYTES;
 }
+size_t record_bytes(const s4kv_cache_t *c) { return static_cast<size_t>(c->num_kv_heads) * block_bytes(cache_bits(c)); }
 
 std::mutex g_mu;
 DeviceShape g_shape[kMaxDevices];
@@ -56,8 +58,8 @@ int device_shape(DeviceShape *out) {
       return S4KV_ERR_CUDA;
     }
     d.num_sms = sms;
-    for (int f = 0; f < 2; ++f) {
-      const int per = decode_ctas_per_sm(f ? 8 : 4);
+    for (int f = 0; f < 3; ++f) {
+      const int per = decode_ctas_per_sm(fmt_bits(f));
       if (per <= 0 || sms <= 0) return S4KV_ERR_CUDA;
       d.num_ctas[f] = sms * per;
       d.num_workers[f] = d.num_ctas[f] * decode_warps_per_cta();
@@ -78,7 +80,7 @@ int check_cache(const s4kv_cache_t *c) {
   if (c->num_pages <= 0 || c->num_kv_heads <= 0 || c->max_seqs <= 0) return S4KV_ERR_INVALID_ARG;
   if (!aligned(c->pool, 128) || !aligned(c->res_k, 16) || !aligned(c->res_v, 16)) return S4KV_ERR_INVALID_ARG;
   if (c->err_flag != nullptr && !aligned(c->err_flag, 4)) return S4KV_ERR_INVALID_ARG;
-  if (c->bits != 0 && c->bits != 4 && c->bits != 8) return S4KV_ERR_UNSUPPORTED;
+  if (c->bits != 0 && c->bits != 2 && c->bits != 4 && c->bits != 8) return S4KV_ERR_UNSUPPORTED;
   return S4KV_OK;
 }
 
@@ -159,10 +161,9 @@ int s4kv_cache_layout(int num_pages, int num_kv_heads, int max_seqs, size_t *poo
 
 int s4kv_cache_layout_bits(int num_pages, int num_kv_heads, int max_seqs, int bits, size_t *pool_bytes,
                            size_t *residual_bytes) {
-  if (bits != 4 && bits != 8) return S4KV_ERR_UNSUPPORTED;
+  if (bits != 2 && bits != 4 && bits != 8) return S4KV_ERR_UNSUPPORTED;
   const int rc = s4kv_cache_layout(num_pages, num_kv_heads, max_seqs, pool_bytes, residual_bytes);
-  if (rc == S4KV_OK && pool_bytes && bits == 8)
-    *pool_bytes = static_cast<size_t>(num_pages) * num_kv_heads * S4KV_BLOCK_BYTES_INT8;
+  if (rc == S4KV_OK && pool_bytes) *pool_bytes = static_cast<size_t>(num_pages) * num_kv_heads * block_bytes(bits);
   return rc;
 }
 

@@ -85,6 +85,8 @@ __global__ void __launch_bounds__(128) append_kernel(const AppendParams p) {
     if (phys_ok) {
       if (p.bits == 8)
         quantize_page_cta<8>(ks, vs, kc, vc, p.pool + (static_cast<long>(phys) * H + h) * Fmt<8>::kBlock, tid);
+      else if (p.bits == 2)
+        quantize_page_cta<2>(ks, vs, kc, vc, p.pool + (static_cast<long>(phys) * H + h) * Fmt<2>::kBlock, tid);
       else
         quantize_page_cta<4>(ks, vs, kc, vc, p.pool + (static_cast<long>(phys) * H + h) * Fmt<4>::kBlock, tid);
     }

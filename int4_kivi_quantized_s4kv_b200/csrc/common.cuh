@@ -19,13 +19,16 @@ constexpr int kKZeroOff = 2304;
 constexpr int kVScaleOff = 2560;
 constexpr int kVZeroOff = 2688;
 
-// Block layout of one (page, kv head) with kBits-bit codes (4 or 8): K codes,
+// Block layout of one (page, kv head) with kBits-bit codes (2, 4 or 8): K codes,
 // V codes, K scale fp16 [128], K zero fp16 [128] (MMA k order), V scale fp16
 // [4][16], V zero fp16 [4][16].  Fmt<4> is the 2816-byte int4 block above.
 // 8-bit codes keep the int4 assignment of (token, channel) to MMA operand
 // fragments with bytes for nibbles: a lane's 8 codes of one tile are 8
 // consecutive bytes (register r at bytes 2r, 2r + 1) and the 16 bytes of
-// tiles 2m, 2m + 1 of lane l sit at (32 m + l) * 16.
+// tiles 2m, 2m + 1 of lane l sit at (32 m + l) * 16.  2-bit codes keep it
+// with bit pairs: the 16 codes of tiles 2m, 2m + 1 of lane l are word
+// 4 l + m, half 0 of every register in the low 16 bits and half 1 in the
+// high 16 bits, register r of tile 2m + p at bits 2 (4 p + r) of its half.
 template <int kBits>
 struct Fmt {
   static constexpr int kCodeBytes = kPage * kHeadDim * kBits / 8;
@@ -40,8 +43,11 @@ struct Fmt {
 };
 static_assert(Fmt<4>::kBlock == kBlockBytes && Fmt<4>::kVZero == kVZeroOff, "int4 block layout");
 static_assert(Fmt<8>::kBlock == S4KV_BLOCK_BYTES_INT8, "int8 block layout");
+static_assert(Fmt<2>::kBlock == S4KV_BLOCK_BYTES_INT2, "int2 block layout");
 
-__host__ __device__ constexpr int block_bytes_for(int bits) { return bits == 8 ? Fmt<8>::kBlock : Fmt<4>::kBlock; }
+__host__ __device__ constexpr int block_bytes_for(int bits) {
+  return bits == 8 ? Fmt<8>::kBlock : bits == 2 ? Fmt<2>::kBlock : Fmt<4>::kBlock;
+}
 
 __device__ __forceinline__ void flag_error(uint32_t *err, uint32_t bits) {
   if (err != nullptr) atomicOr(err, bits);
@@ -131,6 +137,32 @@ __device__ __forceinline__ void unpack_codes8(uint32_t w0, uint32_t w1, uint32_t
   a1 = h2_as_u32(__hsub2(u32_as_h2(p1), k1024));
   a2 = h2_as_u32(__hsub2(u32_as_h2(p2), k1024));
   a3 = h2_as_u32(__hsub2(u32_as_h2(p3), k1024));
+}
+
+// One register of a lane's 2-bit tile fragment: codes at bit 2k of both
+// halves of `w` (k = 4 * tile parity + register).  Below bit 10 a code c is
+// laid into the mantissa of 1024 as 1024 + c * 4^k (exact: at most 1792) and
+// scaled back exactly by one fp16 multiply-add; codes above are first moved
+// down by 10 bits.
+template <int k>
+__device__ __forceinline__ uint32_t unpack_code2(uint32_t w, uint32_t w10) {
+  constexpr int kk = k <= 4 ? k : k - 5;
+  const uint32_t src = k <= 4 ? w : w10;
+  const uint32_t x = and_or(src, 0x00030003u << (2 * kk), 0x64006400u);
+  if (kk == 0) return h2_as_u32(__hsub2(u32_as_h2(x), u32_as_h2(0x64006400u)));
+  // fp16 pairs of 4^-kk (1/4, 1/16, 1/64, 1/256) and -1024 * 4^-kk
+  constexpr uint32_t kScale = kk == 1 ? 0x34003400u : kk == 2 ? 0x2C002C00u : kk == 3 ? 0x24002400u : 0x1C001C00u;
+  constexpr uint32_t kBias = kk == 1 ? 0xDC00DC00u : kk == 2 ? 0xD400D400u : kk == 3 ? 0xCC00CC00u : 0xC400C400u;
+  return h2_as_u32(__hfma2(u32_as_h2(x), u32_as_h2(kScale), u32_as_h2(kBias)));
+}
+
+template <int kParity>
+__device__ __forceinline__ void unpack_codes2(uint32_t w, uint32_t &a0, uint32_t &a1, uint32_t &a2, uint32_t &a3) {
+  const uint32_t w10 = w >> 10;
+  a0 = unpack_code2<4 * kParity + 0>(w, w10);
+  a1 = unpack_code2<4 * kParity + 1>(w, w10);
+  a2 = unpack_code2<4 * kParity + 2>(w, w10);
+  a3 = unpack_code2<4 * kParity + 3>(w, w10);
 }
 
 // ------------------------------------------------------------- warp MMA --

@@ -83,7 +83,9 @@ constexpr size_t smem_bytes_for() {
   return static_cast<size_t>(kWarpsPerCta) * (stages_for<kBits>() * (Fmt<kBits>::kBlock + 8) + kQBytesPerWarp);
 }
 
-size_t decode_smem_bytes(int bits) { return bits == 8 ? smem_bytes_for<8>() : smem_bytes_for<4>(); }
+size_t decode_smem_bytes(int bits) {
+  return bits == 8 ? smem_bytes_for<8>() : bits == 2 ? smem_bytes_for<2>() : smem_bytes_for<4>();
+}
 
 __device__ __forceinline__ int clamp_len(int L, int max_pages) {
   return min(max(L, 0), max_pages * kPage);
@@ -194,7 +196,10 @@ template <int kBits>
 __device__ __forceinline__ void tile_fragment(const uint32_t (&w)[8], int kt, uint32_t &a0, uint32_t &a1,
                                               uint32_t &a2, uint32_t &a3) {
   if (kBits == 8) unpack_codes8(w[2 * (kt & 1)], w[2 * (kt & 1) + 1], a0, a1, a2, a3);
-  else unpack_codes(w[kt], a0, a1, a2, a3);
+  else if (kBits == 2) {
+    if (kt & 1) unpack_codes2<1>(w[kt >> 1], a0, a1, a2, a3);
+    else unpack_codes2<0>(w[kt >> 1], a0, a1, a2, a3);
+  } else unpack_codes(w[kt], a0, a1, a2, a3);
 }
 
 template <int kBits>
@@ -214,6 +219,9 @@ __device__ __forceinline__ void qk_page(const StageAddr &a, const QFrag &q, floa
     const uint4 kw1 = lds128<F::kKCode + 512>(a.code);
     kws[0] = kw0.x; kws[1] = kw0.y; kws[2] = kw0.z; kws[3] = kw0.w;
     kws[4] = kw1.x; kws[5] = kw1.y; kws[6] = kw1.z; kws[7] = kw1.w;
+  } else if (kBits == 2) {  // all 8 tiles' codes in one 16-byte load
+    const uint4 kw0 = lds128<F::kKCode>(a.code);
+    kws[0] = kw0.x; kws[1] = kw0.y; kws[2] = kw0.z; kws[3] = kw0.w;
   }
 #pragma unroll
   for (int m = 0; m < 4; ++m) {
@@ -350,6 +358,9 @@ __device__ __forceinline__ void pv_page(const StageAddr &a, const uint32_t (&P)[
     const uint4 vw1 = lds128<Fmt<4>::kVCode + 512>(a.code);
     vws[0] = vw0.x; vws[1] = vw0.y; vws[2] = vw0.z; vws[3] = vw0.w;
     vws[4] = vw1.x; vws[5] = vw1.y; vws[6] = vw1.z; vws[7] = vw1.w;
+  } else if (kBits == 2) {
+    const uint4 vw0 = lds128<Fmt<2>::kVCode>(a.code);
+    vws[0] = vw0.x; vws[1] = vw0.y; vws[2] = vw0.z; vws[3] = vw0.w;
   }
   pv_group<kBits, 0>(a, P, vws, st);
   pv_group<kBits, 1>(a, P, vws, st);
@@ -959,7 +970,9 @@ int ctas_per_sm_for() {
   return n < m ? n : m;  // one launch shape serves the plain and the fused kernel
 }
 
-int decode_ctas_per_sm(int bits) { return bits == 8 ? ctas_per_sm_for<8>() : ctas_per_sm_for<4>(); }
+int decode_ctas_per_sm(int bits) {
+  return bits == 8 ? ctas_per_sm_for<8>() : bits == 2 ? ctas_per_sm_for<2>() : ctas_per_sm_for<4>();
+}
 
 int decode_warps_per_cta() { return kWarpsPerCta; }
 
@@ -972,9 +985,11 @@ cudaError_t prepare_for() {
 }
 
 cudaError_t prepare_decode_kernel() {
-  const cudaError_t e = prepare_for<4>();
+  cudaError_t e = prepare_for<4>();
   if (e != cudaSuccess) return e;
-  return prepare_for<8>();
+  e = prepare_for<8>();
+  if (e != cudaSuccess) return e;
+  return prepare_for<2>();
 }
 
 void launch_decode(const DecodeParams &p, const FusedAppend &f, int bits, int num_ctas, cudaStream_t stream) {
@@ -984,6 +999,11 @@ void launch_decode(const DecodeParams &p, const FusedAppend &f, int bits, int nu
       decode_kernel<8, true><<<num_ctas, kThreads, smem_bytes_for<8>(), stream>>>(p, f);
     else
       decode_kernel<8, false><<<num_ctas, kThreads, smem_bytes_for<8>(), stream>>>(p, f);
+  } else if (bits == 2) {
+    if (fused)
+      decode_kernel<2, true><<<num_ctas, kThreads, smem_bytes_for<2>(), stream>>>(p, f);
+    else
+      decode_kernel<2, false><<<num_ctas, kThreads, smem_bytes_for<2>(), stream>>>(p, f);
   } else {
     if (fused)
       decode_kernel<4, true><<<num_ctas, kThreads, smem_bytes_for<4>(), stream>>>(p, f);

@@ -16,6 +16,11 @@ __device__ __forceinline__ uint32_t code_at(const uint8_t *region, int word, int
     const int tile = 4 * (word >> 7) + (word & 3), lane = (word >> 2) & 31;
     return region[((tile >> 1) * 32 + lane) * 16 + (tile & 1) * 8 + 2 * (nibble & 3) + (nibble >> 2)];
   }
+  if (bits == 2) {
+    const int tile = 4 * (word >> 7) + (word & 3), lane = (word >> 2) & 31;
+    const uint32_t w = reinterpret_cast<const uint32_t *>(region)[4 * lane + (tile >> 1)];
+    return (w >> (16 * (nibble >> 2) + 2 * (4 * (tile & 1) + (nibble & 3)))) & 3u;
+  }
   const uint32_t w = reinterpret_cast<const uint32_t *>(region)[word];
   return (w >> (4 * nibble)) & 0xFu;
 }
@@ -32,10 +37,11 @@ __global__ void __launch_bounds__(128) dequant_kernel(const DequantParams p) {
       return;
     }
   }
-  const bool b8 = p.bits == 8;
-  const int kcode_off = 0, vcode_off = b8 ? Fmt<8>::kVCode : Fmt<4>::kVCode;
-  const int kscale_off = b8 ? Fmt<8>::kKScale : Fmt<4>::kKScale, kzero_off = b8 ? Fmt<8>::kKZero : Fmt<4>::kKZero;
-  const int vscale_off = b8 ? Fmt<8>::kVScale : Fmt<4>::kVScale, vzero_off = b8 ? Fmt<8>::kVZero : Fmt<4>::kVZero;
+  // regions of the block: codes, then the same 768 bytes of fp16 metadata
+  const int code_bytes = kPage * kHeadDim * p.bits / 8;
+  const int kcode_off = 0, vcode_off = code_bytes;
+  const int kscale_off = 2 * code_bytes, kzero_off = kscale_off + 2 * kHeadDim;
+  const int vscale_off = kzero_off + 2 * kHeadDim, vzero_off = vscale_off + 2 * kPage * (kHeadDim / kVGroup);
   const uint8_t *blk = p.pool + (static_cast<long>(page) * p.num_kv_heads + h) * block_bytes_for(p.bits);
   const float ks = __half2float(reinterpret_cast<const __half *>(blk + kscale_off)[c]);
   const int zslot = 16 * ((c & 31) >> 2) + 2 * (c >> 5) + (c & 1) + 8 * ((c & 3) >> 1);

@@ -5,7 +5,8 @@
 // step 1): keys asymmetric int4 per channel (one group = one channel over the
 // page's 16 tokens), values int4 per token (groups of 32 channels); the INT8
 // variant ("KV-Cache-Optimierung -- PagedAttention, quantisierter KV,
-// Speculative Cache", "Warum es zaehlt": INT8/INT4 KV) uses 255 levels.
+// Speculative Cache", "Warum es zaehlt": INT8/INT4 KV) uses 255 levels and
+// the 2-bit one (KIVI's own width) 3.
 #pragma once
 
 #include "common.cuh"
@@ -90,6 +91,29 @@ __device__ __forceinline__ void quantize_page_cta(const __half (*ks)[kHeadDim], 
         kw |= static_cast<uint32_t>(kc[t][c]) << (4 * j);
         val_tc(tile, n, i, j, t, c);
         vw |= static_cast<uint32_t>(vc[t][c]) << (4 * j);
+      }
+      reinterpret_cast<uint32_t *>(blk + F::kKCode)[w] = kw;
+      reinterpret_cast<uint32_t *>(blk + F::kVCode)[w] = vw;
+    }
+  } else if (kBits == 2) {
+    // word 4 lane + m holds tiles 2m, 2m + 1 of the lane: register r, half
+    // `half` (nibble index j = r + 4 half) of tile 2m + p at bit
+    // 16 half + 2 (4 p + r)
+    for (int w = tid; w < 128; w += 128) {
+      const int lane = w >> 2, m = w & 3;
+      const int n = lane >> 2, i = lane & 3;
+      uint32_t kw = 0, vw = 0;
+#pragma unroll
+      for (int p = 0; p < 2; ++p) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int bit = 16 * (j >> 2) + 2 * (4 * p + (j & 3));
+          int t, c;
+          key_tc(2 * m + p, n, i, j, t, c);
+          kw |= static_cast<uint32_t>(kc[t][c]) << bit;
+          val_tc(2 * m + p, n, i, j, t, c);
+          vw |= static_cast<uint32_t>(vc[t][c]) << bit;
+        }
       }
       reinterpret_cast<uint32_t *>(blk + F::kKCode)[w] = kw;
       reinterpret_cast<uint32_t *>(blk + F::kVCode)[w] = vw;

@@ -71,8 +71,10 @@ def test_cache_layout_matches_block_size(S, oracle_mod):
     assert res == 256 * 8 * 16 * 128 * 2
     pool8, res8 = S.s4kv_cache_layout(1000, 8, 256, bits=8)
     assert pool8 == 1000 * 8 * oracle_mod.block_bytes(8) and res8 == res
+    pool2, _ = S.s4kv_cache_layout(1000, 8, 256, bits=2)
+    assert pool2 == 1000 * 8 * oracle_mod.block_bytes(2)
     with pytest.raises(S.S4KVError):
-        S.s4kv_cache_layout(10, 8, 1, bits=2)
+        S.s4kv_cache_layout(10, 8, 1, bits=3)
     with pytest.raises(S.S4KVError):
         S.s4kv_cache_layout(0, 8, 1)
 
@@ -120,7 +122,7 @@ def test_invalid_calls_rejected_before_launch(S):
     assert L.s4kv_dequant_page(ctypes.byref(c), 10, P(fake), P(fake), 1, st) == S.ERR_INVALID_ARG
     assert L.s4kv_dequant_page(ctypes.byref(c), -1, P(fake), P(fake), 1, st) == S.ERR_INVALID_ARG
     assert L.s4kv_dequant_page(ctypes.byref(bad_dim), 0, P(fake), P(fake), 1, st) == S.ERR_UNSUPPORTED
-    # code width: 4 (or 0) and 8 only; prefill has no 8-bit path
+    # code width: 4 (or 0), 8 and 2 only; prefill has no 8- or 2-bit path
     bad_bits = S.s4kv_cache_t(fake, fake, fake, None, 10, 2, 4, 128, 16, 3)
     assert L.s4kv_dequant_page(ctypes.byref(bad_bits), 0, P(fake), P(fake), 1, st) == S.ERR_UNSUPPORTED
     c8 = S.s4kv_cache_t(fake, fake, fake, None, 10, 2, 4, 128, 16, 8)

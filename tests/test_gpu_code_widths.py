@@ -1,7 +1,7 @@
-"""GPU parity of the INT8 variant (8-bit KIVI codes on the same layout
-machinery) against the oracle, through the C ABI: cache bytes and fp32
-dequantization bit-exact, decode attention (plain and fused with the step's
-append) within 2e-3 + 1e-3 |ref|."""
+"""GPU parity of the INT8 and 2-bit variants (8- and 2-bit KIVI codes on the
+same layout machinery) against the oracle, through the C ABI: cache bytes and
+fp32 dequantization bit-exact, decode attention (plain and fused with the
+step's append) within 2e-3 + 1e-3 |ref|."""
 import dataclasses
 
 import numpy as np
@@ -20,13 +20,17 @@ CASES = {
 }
 
 
+BLOCK = {8: 4864, 2: 1792}
+
+
+@pytest.mark.parametrize("bits", [8, 2])
 @pytest.mark.parametrize("name", list(CASES))
-def test_int8_cache_and_decode_match_oracle(name):
+def test_cache_and_decode_match_oracle(name, bits):
     import torch
     spec = W.SPECS[name] if not CASES[name] else W.scaled(W.SPECS[name], **CASES[name])
-    p = Pair(spec, prefill_chunk=33, bits=8)
+    p = Pair(spec, prefill_chunk=33, bits=bits)
     p.assert_cache_bit_exact()
-    err = assert_attention_close(p.gpu_decode(), p.oracle_decode(), f"int8 {name}")
+    err = assert_attention_close(p.gpu_decode(), p.oracle_decode(), f"int{bits} {name}")
     # fp32 dequantization of a few pages, bit-exact
     S = p.S
     pages = np.unique(p.plan.block_tables[p.plan.block_tables >= 0])[:5].astype(np.int32)
@@ -41,13 +45,14 @@ def test_int8_cache_and_decode_match_oracle(name):
             full = any(int(pg) in p.plan.block_tables[b, :int(p.lens[b]) // 16] for b in range(spec.batch))
             if full:
                 assert np.array_equal(ok[i].cpu().numpy(), rk) and np.array_equal(ov[i].cpu().numpy(), rv)
-    print(f"int8 {name}: max abs err {err:.3g}")
+    print(f"int{bits} {name}: max abs err {err:.3g}")
 
 
-def test_int8_fused_step_and_page_records():
-    """One fused decode step on an 8-bit cache (tokens that complete pages
-    included) writes the oracle's bytes; gathered page records have the
-    8-bit record size."""
+@pytest.mark.parametrize("bits", [8, 2])
+def test_fused_step_and_page_records(bits):
+    """One fused decode step on an 8- or 2-bit cache (tokens that complete
+    pages included) writes the oracle's bytes; gathered page records have
+    that width's record size."""
     import torch
     import oracle
     import int4_kivi_quantized_s4kv_b200 as S
@@ -63,8 +68,8 @@ def test_int8_fused_step_and_page_records():
         k.append(kk)
         v.append(vv)
     bt = plan.block_tables
-    oc = oracle.OracleCache(plan.num_pages, H, B, bits=8)
-    g = S.S4KVCache(plan.num_pages, H, B, bits=8)
+    oc = oracle.OracleCache(plan.num_pages, H, B, bits=bits)
+    g = S.S4KVCache(plan.num_pages, H, B, bits=bits)
     bt_dev = dev(bt)
     for kk, vv, sm, cu, sl, mx in append_batches(np.zeros(B, np.int64), ctx, k, v, bt, 16):
         assert oc.append(kk, vv, sm, cu, sl, bt) == 0
@@ -79,9 +84,9 @@ def test_int8_fused_step_and_page_records():
     torch.cuda.synchronize()
     assert S.s4kv_get_error(g) == 0
     assert np.array_equal(g.pool.cpu().numpy(), oc.pool)
-    assert_attention_close(out.float().cpu().numpy(), oc.decode_attention(q, lens, bt), "int8 fused")
+    assert_attention_close(out.float().cpu().numpy(), oc.decode_attention(q, lens, bt), f"int{bits} fused")
     rec = S.s4kv_page_record_bytes(g)
-    assert rec == H * 4864
+    assert rec == H * BLOCK[bits]
     pages = np.array(bt[2, :int(lens[2]) // 16], np.int32)
     dst = torch.empty((len(pages), rec), dtype=torch.uint8, device="cuda")
     S.s4kv_gather_pages(g, dev(pages), dst)
