@@ -61,16 +61,17 @@ def kernel_sources_sha() -> str:
     return h.hexdigest()
 
 
-def recorded_traffic(algorithmic_bytes: float):
+def recorded_traffic(algorithmic_bytes: float, bits: int = 4):
     """DRAM bytes (read + write) per decode launch from the committed ncu
-    capture, scaled from the captured case by algorithmic bytes; None when
-    the decode kernel's sources changed since the capture."""
+    capture of that code width, scaled from the captured case by algorithmic
+    bytes; None when the decode kernel's sources changed since the capture."""
     try:
         with open(os.path.join(ROOT, "profiles", "decode_traffic.json")) as f:
-            rec = json.load(f)
+            recs = json.load(f)
     except Exception:
         return None
-    if rec.get("kernel_sources_sha256") != kernel_sources_sha():
+    rec = recs.get("widths", {}).get(str(bits))
+    if rec is None or recs.get("kernel_sources_sha256") != kernel_sources_sha():
         return None
     return algorithmic_bytes * rec["dram_bytes"] / rec["algorithmic_bytes"]
 
@@ -235,7 +236,7 @@ class OracleSample:
     head) pairs of layer 0, prefilled untimed; one call of `run()` is the
     step (append of the new token(s) + decode) for the sampled sequences."""
 
-    def __init__(self, spec: W.Spec, n_seqs: int):
+    def __init__(self, spec: W.Spec, n_seqs: int, bits: int = 4):
         import oracle
         oracle.build()
         n_seqs = max(1, min(n_seqs, spec.batch))
@@ -251,7 +252,7 @@ class OracleSample:
             bt[j, :n] = np.arange(c, c + n)
             c += n
         self.bt = bt
-        self.cache = oracle.OracleCache(c + 1, spec.num_kv_heads, n_seqs)
+        self.cache = oracle.OracleCache(c + 1, spec.num_kv_heads, n_seqs, bits=bits)
         self.ctx = ctx[self.seqs]
         self.lens = lens[self.seqs]
         k, v = zip(*[W.kv_sequence_np(spec, 0, b, int(lens[b])) for b in self.seqs])
@@ -268,7 +269,8 @@ class OracleSample:
         self.q = W.queries_np(spec, 0)[self.seqs]
         sub = W.Spec(**{**spec.__dict__, "batch": n_seqs, "shared_prefix_tokens": 0,
                         "ctx_kind": "fixed", "ctx_fixed": tuple(int(x) for x in self.ctx)})
-        self.bytes = W.decode_bytes(sub, self.lens, W.PagePlan(bt, c + 1, 0, c))["algorithmic"]
+        self.bytes = W.decode_bytes(sub, self.lens, W.PagePlan(bt, c + 1, 0, c),
+                                    block_bytes={2: 1792, 4: 2816, 8: 4864}[bits])["algorithmic"]
         self.tokens = n_seqs
 
     def run(self):
@@ -277,13 +279,13 @@ class OracleSample:
         return self.cache.decode_attention(self.q, self.lens, self.bt)
 
 
-def cpu_baseline(spec, budget_s=12.0):
-    probe = OracleSample(spec, 1)
+def cpu_baseline(spec, budget_s=12.0, bits: int = 4):
+    probe = OracleSample(spec, 1, bits)
     t0 = time.perf_counter()
     probe.run()
     t1 = time.perf_counter() - t0
     n = int(max(1, min(spec.batch, budget_s / max(t1, 1e-3))))
-    samp = OracleSample(spec, n) if n > 1 else probe
+    samp = OracleSample(spec, n, bits) if n > 1 else probe
     t0 = time.perf_counter()
     samp.run()
     dt = time.perf_counter() - t0
@@ -561,6 +563,8 @@ def main(argv=None):
     ap.add_argument("--batch", type=int, default=None,
                     help="override the workload's batch (smaller profiling cases)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--bits", type=int, default=4, choices=[2, 4, 8],
+                    help="code width of the cache (4: the int4 KIVI path; 8 / 2: its variants)")
     ap.add_argument("--no-prefill", action="store_true",
                     help="skip the chunked-prefill attention measurement")
     args = ap.parse_args(argv)
@@ -589,8 +593,8 @@ def main(argv=None):
     if world > 1:
         torch.distributed.barrier()
 
-    wl = DeviceWorkload(replica_spec(spec, rank), device)
-    dbytes, abytes = step_bytes(wl.spec, wl.plan, wl.lens)
+    wl = DeviceWorkload(replica_spec(spec, rank), device, bits=args.bits)
+    dbytes, abytes = step_bytes(wl.spec, wl.plan, wl.lens, bits=args.bits)
     bytes_per_step = (dbytes["algorithmic"] + abytes) * spec.layers
     decode_bytes_per_launch = dbytes["algorithmic"]
 
@@ -694,16 +698,17 @@ def main(argv=None):
         int2 = measure_width_decode(device, spec, 2)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(spec)
+        cpu = cpu_baseline(spec, bits=args.bits)
     if world > 1:
         torch.distributed.barrier()
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "int4 codes, f16 MMA operands, f32 accumulate",
+            "vs_baseline": None, "dtype": f"int{args.bits} codes, f16 MMA operands, f32 accumulate",
             "data": "synthetic (seeded Gaussian K/V/q with outlier key channels; no dataset)",
             "config": config_dict(spec, {
+                "code_bits": args.bits,
                 "parallelism": f"replicas x{world}" if world > 1 else "1 GPU",
                 "context": {"min": int(wl.ctx.min()), "max": int(wl.ctx.max()), "mean": float(wl.ctx.mean())},
                 "new_tokens_per_seq": int(wl.new.max()),
@@ -716,9 +721,9 @@ def main(argv=None):
             "tokens_per_s": world * tokens / (step_ms * 1e-3),
             "sequences_per_s": world * spec.batch / (step_ms * 1e-3),
             "kv_tokens_per_s": world * spec.layers * int(wl.lens.sum()) / (step_ms * 1e-3),
-            "roofline": {"bound": "hbm", "kernel": "decode_kernel", "achieved": achieved, "peak": peak,
+            "roofline": {"bound": "hbm", "kernel": f"decode_kernel<{args.bits}>", "achieved": achieved, "peak": peak,
                          "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
-                         "traffic": recorded_traffic(decode_bytes_per_launch),
+                         "traffic": recorded_traffic(decode_bytes_per_launch, args.bits),
                          "bytes_per_launch": decode_bytes_per_launch, "avg_launch_ms": dec_avg_ms},
             "e2e": {"value": aggregate_gbs(world, bytes_per_step, e2e_ms), "unit": "GB/s",
                     "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
