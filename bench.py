@@ -371,9 +371,10 @@ def measure_prefill(device, steps: int, workload: str = "llama3.1-8b-prefill"):
     rows = int(wl.new.sum())
     q = W.chunk_queries_torch(spec, 0, rows, device)
     out = torch.empty_like(q)
+    ws = S.prefill_workspace(spec.num_kv_heads, spec.batch, wl.bt.shape[1], device)
 
     def run():
-        S.s4kv_prefill_attention(cache, q, wl.step_cu, wl.seq_lens, wl.bt, out, wl.max_new)
+        S.s4kv_prefill_attention(cache, q, wl.step_cu, wl.seq_lens, wl.bt, out, wl.max_new, workspace=ws)
 
     for _ in range(3):
         run()

@@ -100,7 +100,7 @@
 extern "C" {
 #endif
 
-#define S4KV_VERSION 2
+#define S4KV_VERSION 3
 #define S4KV_HEAD_DIM 128
 #define S4KV_PAGE_TOKENS 16
 #define S4KV_VALUE_GROUP 32
@@ -277,17 +277,34 @@ S4KV_API int s4kv_decode_attention_noalloc(const s4kv_cache_t *cache, const void
  *          sequence b (position L - n + j) gets softmax(sm_scale * q.K^T) V
  *          over the cache's tokens 0 .. L - n + j; rows of no sequence are
  *          left untouched.
- * Runs on the tcgen05 tensor cores with the dequantized keys and values and
- * the softmax weights as fp16 MMA operands (fp32 accumulation), so results
- * agree with exact attention to about fp16 precision of those operands.
- * Allocates nothing; needs about 171 KB of shared memory per CTA.  4-bit
- * codes only (2- and 8-bit caches are refused with S4KV_ERR_UNSUPPORTED). */
+ *  workspace, workspace_bytes  device scratch owned by the caller, 16-B
+ *          aligned, at least s4kv_prefill_workspace_size(num_kv_heads, batch,
+ *          max_pages_per_seq) bytes (else S4KV_ERR_WORKSPACE and nothing is
+ *          launched).  Its contents are overwritten and mean nothing after the
+ *          call; it must not be shared with work that runs concurrently.
+ * Two launches on `stream`: the first dequantizes every 64-key tile of each
+ * (sequence, kv head) once into the workspace as fp16 MMA operands (keys as
+ * an fp16 hi part plus the fp16 rounding of the remainder, about 22 bits;
+ * values correctly rounded to fp16); the second runs the attention on the
+ * tcgen05 tensor cores with those operands and the fp16 softmax weights
+ * (fp32 accumulation), so results agree with exact attention to about fp16
+ * precision of the values and the weights.  Allocates nothing; the attention
+ * launch needs about 215 KB of shared memory per CTA.  4-bit codes only (2-
+ * and 8-bit caches are refused with S4KV_ERR_UNSUPPORTED). */
 S4KV_API int s4kv_prefill_attention(const s4kv_cache_t *cache, const void *q,
                                     int num_q_heads, int n_tokens,
                                     const int32_t *cu_new, const int32_t *seq_lens,
                                     const int32_t *block_tables, int batch,
                                     int max_pages_per_seq, int max_new_per_seq,
-                                    float sm_scale, void *out, void *stream);
+                                    float sm_scale, void *out, void *workspace,
+                                    size_t workspace_bytes, void *stream);
+
+/* Bytes of workspace s4kv_prefill_attention needs: 48 KB per 64-key tile of
+ * max_pages_per_seq pages (rounded up to whole tiles), per sequence slot and
+ * kv head.  S4KV_ERR_INVALID_ARG for non-positive sizes or a total above
+ * 2^40 bytes. */
+S4KV_API int s4kv_prefill_workspace_size(int num_kv_heads, int batch, int max_pages_per_seq,
+                                         size_t *bytes);
 
 /* Dequantize one physical page for all kv heads into natural order:
  * out_k, out_v device [num_kv_heads][16][128], fp32 if out_fp32 != 0

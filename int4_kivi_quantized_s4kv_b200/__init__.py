@@ -49,7 +49,8 @@ _SIGS = {
     "s4kv_decode_attention": ([_CP, _P, _I, _P, _P, _I, _I, ctypes.c_float, _P, _P, _SZ, _P], _I),
     "s4kv_decode_attention_noalloc": ([_CP, _P, _I, _P, _P, _I, _I, ctypes.c_float, _P, _P], _I),
     "s4kv_append_decode": ([_CP, _P, _P, _P, _I, _P, _P, _I, _I, ctypes.c_float, _P, _P, _SZ, _P], _I),
-    "s4kv_prefill_attention": ([_CP, _P, _I, _I, _P, _P, _P, _I, _I, _I, ctypes.c_float, _P, _P], _I),
+    "s4kv_prefill_attention": ([_CP, _P, _I, _I, _P, _P, _P, _I, _I, _I, ctypes.c_float, _P, _P, _SZ, _P], _I),
+    "s4kv_prefill_workspace_size": ([_I, _I, _I, ctypes.POINTER(_SZ)], _I),
     "s4kv_dequant_page": ([_CP, _I, _P, _P, _I, _P], _I),
     "s4kv_dequant_pages": ([_CP, _P, _I, _P, _P, _I, _P], _I),
     "s4kv_page_record_bytes": ([_CP, ctypes.POINTER(_SZ)], _I),
@@ -232,21 +233,40 @@ def s4kv_decode_attention_noalloc(cache: S4KVCache, q, seq_lens, block_tables, o
     _check(st, "s4kv_decode_attention_noalloc")
 
 
+def prefill_workspace_bytes(num_kv_heads: int, batch: int, max_pages_per_seq: int) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().s4kv_prefill_workspace_size(num_kv_heads, batch, max_pages_per_seq, ctypes.byref(n)),
+           "s4kv_prefill_workspace_size")
+    return n.value
+
+
+def prefill_workspace(num_kv_heads: int, batch: int, max_pages_per_seq: int, device="cuda"):
+    """Device scratch for s4kv_prefill_attention (uint8)."""
+    import torch
+    return torch.empty(prefill_workspace_bytes(num_kv_heads, batch, max_pages_per_seq), dtype=torch.uint8,
+                       device=device)
+
+
 def s4kv_prefill_attention(cache: S4KVCache, q, cu_new, seq_lens, block_tables, out,
-                           max_new_per_seq: int, sm_scale: float | None = None, stream=None):
+                           max_new_per_seq: int, sm_scale: float | None = None, workspace=None, stream=None):
     """Causal attention of the appended chunk's query rows (q: fp16
     [n_tokens][num_q_heads][128], sequence b owning rows cu_new[b]..) over the
-    cache after s4kv_append wrote the chunk; fills out [n_tokens][num_q_heads][128]."""
+    cache after s4kv_append wrote the chunk; fills out [n_tokens][num_q_heads][128].
+    `workspace` (from prefill_workspace) is allocated per call when omitted."""
     import torch
     n_tokens, num_q_heads, _ = q.shape
     if sm_scale is None:
         sm_scale = HEAD_DIM ** -0.5
+    batch, max_pages = seq_lens.shape[0], block_tables.shape[1]
+    if workspace is None:
+        workspace = prefill_workspace(cache.num_kv_heads, max(batch, 1), max_pages, q.device)
     st = lib().s4kv_prefill_attention(cache.ref, _ptr(q, torch.float16, "q"), num_q_heads, n_tokens,
                                      _ptr(cu_new, torch.int32, "cu_new"),
                                      _ptr(seq_lens, torch.int32, "seq_lens"),
-                                     _ptr(block_tables, torch.int32, "block_tables"), seq_lens.shape[0],
-                                     block_tables.shape[1], int(max_new_per_seq), float(sm_scale),
-                                     _ptr(out, torch.float16, "out"), _stream(stream))
+                                     _ptr(block_tables, torch.int32, "block_tables"), batch,
+                                     max_pages, int(max_new_per_seq), float(sm_scale),
+                                     _ptr(out, torch.float16, "out"), _ptr(workspace, torch.uint8, "workspace"),
+                                     workspace.numel(), _stream(stream))
     _check(st, "s4kv_prefill_attention")
 
 

@@ -286,10 +286,19 @@ int decode_call(const s4kv_cache_t *cache, const void *k_new, const void *v_new,
 
 extern "C" {
 
+int s4kv_prefill_workspace_size(int num_kv_heads, int batch, int max_pages_per_seq, size_t *bytes) {
+  if (!bytes || num_kv_heads <= 0 || batch < 0 || max_pages_per_seq <= 0) return S4KV_ERR_INVALID_ARG;
+  const unsigned long long tiles = (static_cast<unsigned long long>(max_pages_per_seq) + 3) / 4;
+  const unsigned long long n = tiles * static_cast<unsigned long long>(batch) * num_kv_heads;
+  if (n > (1ull << 40) / prefill_tile_bytes()) return S4KV_ERR_INVALID_ARG;
+  *bytes = static_cast<size_t>(n * prefill_tile_bytes());
+  return S4KV_OK;
+}
+
 int s4kv_prefill_attention(const s4kv_cache_t *cache, const void *q, int num_q_heads, int n_tokens,
                            const int32_t *cu_new, const int32_t *seq_lens, const int32_t *block_tables,
                            int batch, int max_pages_per_seq, int max_new_per_seq, float sm_scale, void *out,
-                           void *stream) {
+                           void *workspace, size_t workspace_bytes, void *stream) {
   int rc = check_cache(cache);
   if (rc != S4KV_OK) return rc;
   if (cache_bits(cache) != 4) return S4KV_ERR_UNSUPPORTED;
@@ -303,6 +312,10 @@ int s4kv_prefill_attention(const s4kv_cache_t *cache, const void *q, int num_q_h
   if (!aligned(q, 16) || !aligned(out, 16) || !aligned(cu_new, 4) || !aligned(seq_lens, 4) ||
       !aligned(block_tables, 4))
     return S4KV_ERR_INVALID_ARG;
+  size_t need = 0;
+  rc = s4kv_prefill_workspace_size(cache->num_kv_heads, batch, max_pages_per_seq, &need);
+  if (rc != S4KV_OK) return rc;
+  if (!workspace || !aligned(workspace, 16) || workspace_bytes < need) return S4KV_ERR_WORKSPACE;
   const int group = num_q_heads / cache->num_kv_heads;
   const long long tiles = (static_cast<long long>(max_new_per_seq) + (128 / group) - 1) / (128 / group);
   if (tiles > 0x7FFFFFFF || batch > 65535 || cache->num_kv_heads > 65535) return S4KV_ERR_INVALID_ARG;
@@ -335,6 +348,8 @@ int s4kv_prefill_attention(const s4kv_cache_t *cache, const void *q, int num_q_h
   p.max_pages = max_pages_per_seq;
   p.num_pages = cache->num_pages;
   p.scale_log2 = static_cast<float>(static_cast<double>(sm_scale) * 1.4426950408889634);
+  p.ws = static_cast<uint8_t *>(workspace);
+  p.tiles_per_seq = (max_pages_per_seq + 3) / 4;
   launch_prefill(p, batch, max_new_per_seq, static_cast<cudaStream_t>(stream));
   if (cudaGetLastError() != cudaSuccess) return S4KV_ERR_CUDA;
   return S4KV_OK;

@@ -104,6 +104,8 @@ struct PrefillParams {
   int max_pages;
   int num_pages;
   float scale_log2;       // sm_scale * log2(e)
+  uint8_t *ws;            // operand tiles [batch][num_kv_heads][tiles_per_seq][48 KB]
+  int tiles_per_seq;      // ceil(max_pages / 4)
 };
 
 void launch_append(const AppendParams &p, int batch, int max_new, cudaStream_t stream);
@@ -117,5 +119,6 @@ size_t decode_smem_bytes(int bits);
 void launch_prefill(const PrefillParams &p, int batch, int max_new, cudaStream_t stream);
 cudaError_t prepare_prefill_kernel();
 size_t prefill_smem_bytes();
+size_t prefill_tile_bytes();
 
 }  // namespace s4kv

@@ -12,29 +12,36 @@
 // page from the fp16 residual.
 //
 // How (B200): this is a dense contraction, so it runs on the fifth-generation
-// tensor cores.  One CTA takes one (query tile, sequence, kv head); the tile's
-// 128 MMA rows are (token, head of the group) pairs, so a tile holds
-// floor(128 / G) tokens.  Keys are walked in tiles of 64 (4 pages) by warps
-// with separate roles, handing buffers over through mbarriers so that the
-// dequantization, the tensor core and the softmax run at the same time:
-//  * a producer warp brings each key tile's page blocks into one of two
-//    staging buffers with 1-D bulk copies (TMA engine, no multicast);
-//  * 8 dequantization warps turn a staged tile into the 128-byte-swizzled
-//    fp16 operands of one of two operand buffers.  A key is code * scale +
-//    zero in fp32 (exact product, one rounding, the value the oracle's
-//    dequantization gives) split into an fp16 hi part and the fp16 rounding
-//    of the remainder, so K_hi + K_lo carries it to about 22 bits (keys of
-//    outlier channels are large, and a single fp16 rounding of them moves the
-//    logits visibly).  A value is the fused fp16 multiply-add code * scale +
-//    zero (the correctly rounded fp16), stored transposed (V^T);
-//  * one thread issues S(k) = Q K_hi^T + Q K_lo^T (M = 128, N = 64) into one
-//    of two tensor-memory buffers, then O += P(k-1) V(k-1) (N = 128, K = 64),
-//    so the tensor core computes the next logits during the softmax;
-//  * 4 softmax warps (one tensor-memory lane, i.e. one row, per thread) read
-//    S back, apply the causal mask and an online softmax in the exp2 domain
-//    whose reference moves only when a row maximum passes it by more than 8
-//    (weights stay <= 256, fine for fp16), rescale that row of O in tensor
-//    memory when it moves, and write P (fp16) to shared memory.
+// tensor cores, in two launches.
+//  1. prefill_operands_kernel dequantizes every key tile (64 keys, 4 pages)
+//     of every (sequence, kv head) ONCE into a workspace tile of 48 KB that
+//     holds the MMA operands exactly as shared memory wants them (128-byte
+//     swizzled, K-major): K_hi, K_lo and V^T.  A key is code * scale + zero
+//     in fp32 (exact product, one rounding, the value the oracle's
+//     dequantization gives) split into an fp16 hi part and the fp16 rounding
+//     of the remainder, so K_hi + K_lo carries it to about 22 bits (keys of
+//     outlier channels are large, and a single fp16 rounding of them moves
+//     the logits visibly).  A value is the fused fp16 multiply-add
+//     code * scale + zero (the correctly rounded fp16), stored transposed.
+//     Every query tile of the sequence then reads these bytes (mostly from
+//     L2) instead of dequantizing the same pages again.
+//  2. prefill_kernel: one CTA takes one (query tile, sequence, kv head); the
+//     tile's 128 MMA rows are (token, head of the group) pairs, so a tile
+//     holds floor(128 / G) tokens.  Warps with separate roles hand buffers
+//     over through mbarriers:
+//      * a producer warp brings each key tile's 48 KB into one of three
+//        shared-memory stages with one 1-D bulk copy (TMA engine, no
+//        multicast);
+//      * one thread issues S(k) = Q K_hi^T + Q K_lo^T (M = 128, N = 64) into
+//        one of two tensor-memory buffers, then O += P(k-1) [V(k-1) | 1]
+//        (N = 144, K = 64): 16 rows of ones after V^T make the tensor core
+//        accumulate each row's sum of the fp16 weights next to O;
+//      * 4 softmax warps (one tensor-memory lane, i.e. one row, per thread)
+//        read S back, apply the causal mask and an online softmax in the exp2
+//        domain whose reference moves only when a row maximum passes it by
+//        more than 8 (weights stay <= 256, fine for fp16), rescale that row
+//        of O (and its sum) in tensor memory when it moves, and write P
+//        (fp16) into one of two shared-memory buffers.
 // Every wait is bounded; a timeout sets a CTA-wide abort flag and an error
 // bit, and every role then leaves its loop.
 #include <cfloat>
@@ -47,38 +54,45 @@ namespace s4kv {
 namespace {
 
 constexpr int kSoftmaxWarps = 4;   // warps 0..3: one row per thread
-constexpr int kDequantWarps = 8;   // warps 4..11
-constexpr int kMmaWarp = 12;
-constexpr int kProducerWarp = 13;
-constexpr int kThreadsP = 32 * 14;
-constexpr int kDqThreads = 32 * kDequantWarps;
+constexpr int kMmaWarp = 4;
+constexpr int kProducerWarp = 5;
+constexpr int kThreadsP = 32 * 6;
+constexpr int kOpThreads = 256;                  // operand kernel: 64 threads per page
 constexpr int kKeyTile = 64;                     // keys per tile (MMA N of S)
 constexpr int kPagesPerTile = kKeyTile / kPage;  // 4
+constexpr int kStages = 3;
 constexpr uint32_t kQBytes = 128 * 128 * 2;      // Q [128][128] fp16
 constexpr uint32_t kKBytes = 64 * 128 * 2;       // K [64][128] fp16
 constexpr uint32_t kVBytes = 128 * 64 * 2;       // V^T [128][64] fp16
+constexpr uint32_t kOnesBytes = 16 * 64 * 2;     // 16 rows of ones after V^T
 constexpr uint32_t kPBytes = 128 * 64 * 2;       // P [128][64] fp16
-constexpr uint32_t kStageBytes = kPagesPerTile * kBlockBytes;
+constexpr uint32_t kTileBytes = 2 * kKBytes + kVBytes;      // workspace tile: K_hi, K_lo, V^T
+constexpr uint32_t kStageBytes = kTileBytes + kOnesBytes;
+constexpr uint32_t kStagingBytes = kPagesPerTile * kBlockBytes;
+constexpr int kOutCols = 144;                    // O: 128 channels, then 16 copies of the row sum
 constexpr float kSlack = 8.0f;                   // log2 slack of the softmax reference
 constexpr long long kWaitLimit = 2000000000LL;   // about one second
 constexpr uint32_t kIdescS = tc05::idesc_f16_f32(128, 64);
-constexpr uint32_t kIdescO = tc05::idesc_f16_f32(128, 128);
+constexpr uint32_t kIdescO = tc05::idesc_f16_f32(128, kOutCols);
+constexpr uint32_t kTmemCols = 512;              // S[2] at 0 and 64, O at 128 .. 271
 
-// smem: operands (1024-aligned), two staging buffers, barriers
+// attention kernel smem: Q, three stages, two P buffers (1024-aligned), barriers
 constexpr uint32_t kOffQ = 0;
-constexpr uint32_t kOffKhi = kOffQ + kQBytes;         // [2]
-constexpr uint32_t kOffKlo = kOffKhi + 2 * kKBytes;   // [2]
-constexpr uint32_t kOffV = kOffKlo + 2 * kKBytes;     // [2]
-constexpr uint32_t kOffP = kOffV + 2 * kVBytes;
-constexpr uint32_t kOffStage = kOffP + kPBytes;       // [2]
-constexpr uint32_t kOffBar = kOffStage + 2 * kStageBytes;
-// barriers (8 bytes each): stage_full[2], stage_empty[2], kv_full[2],
-// kv_empty[2], s_full[2], s_empty[2], p_full, p_empty; then the tensor-memory
-// address and the abort flag
+constexpr uint32_t kOffStage = kOffQ + kQBytes;                  // [3]
+constexpr uint32_t kOffP = kOffStage + kStages * kStageBytes;    // [2]
+constexpr uint32_t kOffBar = kOffP + 2 * kPBytes;
+// barriers (8 bytes each): stage_full[3], stage_empty[3], s_full[2],
+// s_empty[2], p_full[2], p_empty[2]; then the tensor-memory address and the
+// abort flag
 constexpr uint32_t kNumBars = 14;
 constexpr uint32_t kOffSlot = kOffBar + 8 * kNumBars;
 constexpr uint32_t kOffAbort = kOffSlot + 4;
 constexpr uint32_t kSmemBytes = kOffAbort + 4 + 1024;  // + alignment slack
+static_assert(kSmemBytes <= 227 * 1024, "prefill shared memory");
+static_assert(kStageBytes % 1024 == 0 && kOffP % 1024 == 0, "1024-byte operand alignment");
+
+// operand kernel smem: the output tile, then the staged page blocks
+constexpr uint32_t kOpSmemBytes = kTileBytes + kStagingBytes + 1024;
 
 // Bounded wait for a barrier phase; gives up after about a second or as soon
 // as another role has raised the CTA's abort flag.
@@ -108,6 +122,11 @@ __device__ __forceinline__ void sts128(uint32_t addr, uint4 v) {
   asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
                : "memory");
 }
+__device__ __forceinline__ uint4 lds128_at(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  return v;
+}
 __device__ __forceinline__ uint32_t lds32_at(uint32_t addr) {
   uint32_t v;
   asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
@@ -134,27 +153,162 @@ __device__ __forceinline__ void split_key(uint32_t codes, float2 sc, float2 z, u
   lo = h2_as_u32(__floats2half2_rn(r.x, r.y));
 }
 
+// The rows of sequence b that the chunk holds, checked against the cache.
+// Returns false (and flags bad lengths once, from the attention kernel's
+// first CTA of the sequence) when there is nothing to do.
+struct SeqRows {
+  int c_lo, n, L;
+};
+__device__ __forceinline__ bool seq_rows(const PrefillParams &p, int b, bool flag, SeqRows &r) {
+  r.c_lo = __ldg(p.cu_new + b);
+  const int c_hi = __ldg(p.cu_new + b + 1);
+  r.n = c_hi - r.c_lo;
+  if (r.n <= 0) return false;
+  r.L = __ldg(p.seq_lens + b);
+  if (r.c_lo < 0 || c_hi > p.n_tokens || r.L < r.n || r.L > p.max_pages * kPage) {
+    if (flag) flag_error(p.err, S4KV_EFLAG_SEQ_LEN);
+    return false;
+  }
+  return true;
+}
+
 }  // namespace
 
+// ---------------------------------------------------------------------------
+// Launch 1: one CTA per (key tile, sequence, kv head) writes the tile's
+// operands [K_hi | K_lo | V^T] (16 KB each, 128-byte swizzled K-major) to the
+// workspace.  Keys at or past L (the rest of the partial last page, pages
+// after it) are written as zeros, so masked keys hold finite values.
+__global__ void __launch_bounds__(kOpThreads) prefill_operands_kernel(const PrefillParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_addr(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  const uint32_t sKh = base, sKl = base + kKBytes, sV = base + 2 * kKBytes;
+  const uint32_t stage = base + kTileBytes;
+  const int kt = blockIdx.x, b = blockIdx.y, h = blockIdx.z, H = p.num_kv_heads;
+  const int t = threadIdx.x;
+  SeqRows sr;
+  if (!seq_rows(p, b, false, sr)) return;
+  const int L = sr.L;
+  if (kt * kKeyTile >= L) return;
+  const int nfull = L / kPage;
+  const int np = (L + kPage - 1) / kPage;
+
+  // ---- the tile's full pages into shared memory, 16-byte loads
+  const int q = max(0, min(kPagesPerTile, nfull - kt * kPagesPerTile));
+  const int32_t *bt = p.block_tables + static_cast<long>(b) * p.max_pages + kt * kPagesPerTile;
+  constexpr int kChunks = kBlockBytes / 16;
+  for (int i = t; i < q * kChunks; i += kOpThreads) {
+    const int k = i / kChunks, c = i - k * kChunks;
+    int phys = __ldg(bt + k);
+    if (static_cast<unsigned>(phys) >= static_cast<unsigned>(p.num_pages)) {
+      if (c == 0) flag_error(p.err, S4KV_EFLAG_PAGE_RANGE);
+      phys = 0;
+    }
+    const uint4 *src = reinterpret_cast<const uint4 *>(
+        p.pool + (static_cast<long long>(phys) * H + h) * kBlockBytes);
+    sts128(stage + k * kBlockBytes + 16 * c, __ldg(src + c));
+  }
+  __syncthreads();
+
+  // ---- dequantize: 64 threads per page
+  const int dpage = t >> 6, widx = t & 63;
+  const int dq = widx & 3, dlane0 = widx >> 2;
+  const int pg = kt * kPagesPerTile + dpage;
+  if (pg < nfull) {
+    const uint32_t blk = stage + dpage * kBlockBytes;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int w = widx + 64 * e;
+      const int ln = dlane0 + 16 * (e & 1), tt = 4 * (e >> 1) + dq;
+      const int dn = ln >> 2, di = ln & 3;
+      // keys: tokens dn, dn + 8 of the page; channels c0 .. c0 + 3
+      {
+        uint32_t a0, a1, a2, a3;
+        unpack_codes(lds32_at(blk + kKCodeOff + 4 * w), a0, a1, a2, a3);
+        const int c0 = 32 * di + 4 * tt;
+        const uint2 sc = lds64_at(blk + kKScaleOff + 2 * c0);
+        const uint32_t zslot = 16 * tt + 2 * di;
+        const uint32_t z01 = lds32_at(blk + kKZeroOff + 2 * zslot);
+        const uint32_t z23 = lds32_at(blk + kKZeroOff + 2 * (zslot + 8));
+        const float2 s01 = __half22float2(u32_as_h2(sc.x)), s23 = __half22float2(u32_as_h2(sc.y));
+        const float2 zf01 = __half22float2(u32_as_h2(z01)), zf23 = __half22float2(u32_as_h2(z23));
+        uint32_t hi0, lo0, hi1, lo1, hi2, lo2, hi3, lo3;
+        split_key(a0, s01, zf01, hi0, lo0);
+        split_key(a1, s01, zf01, hi1, lo1);
+        split_key(a2, s23, zf23, hi2, lo2);
+        split_key(a3, s23, zf23, hi3, lo3);
+        const uint32_t ko = tc05::sw128_offset(dpage * 16 + dn, c0, 64);
+        sts64(sKh + ko, hi0, hi2);
+        sts64(sKh + ko + 1024, hi1, hi3);
+        sts64(sKl + ko, lo0, lo2);
+        sts64(sKl + ko + 1024, lo1, lo3);
+      }
+      // values: channels cb, cb + 1; tokens 2 di, 2 di + 1 (+ 8)
+      {
+        uint32_t a0, a1, a2, a3;
+        unpack_codes(lds32_at(blk + kVCodeOff + 4 * w), a0, a1, a2, a3);
+        const int g = tt >> 1;
+        const uint32_t sv_lo = lds32_at(blk + kVScaleOff + 2 * (16 * g + 2 * di));
+        const uint32_t sv_hi = lds32_at(blk + kVScaleOff + 2 * (16 * g + 2 * di + 8));
+        const uint32_t zv_lo = lds32_at(blk + kVZeroOff + 2 * (16 * g + 2 * di));
+        const uint32_t zv_hi = lds32_at(blk + kVZeroOff + 2 * (16 * g + 2 * di + 8));
+        const int cb = 32 * (tt >> 1) + 4 * dn + 2 * (tt & 1);
+        const int key = dpage * 16 + 2 * di;
+        sts32(sV + tc05::sw128_offset(cb, key, 128), hfma2_u32(a0, sv_lo, zv_lo));
+        sts32(sV + tc05::sw128_offset(cb + 1, key, 128), hfma2_u32(a1, sv_lo, zv_lo));
+        sts32(sV + tc05::sw128_offset(cb, key + 8, 128), hfma2_u32(a2, sv_hi, zv_hi));
+        sts32(sV + tc05::sw128_offset(cb + 1, key + 8, 128), hfma2_u32(a3, sv_hi, zv_hi));
+      }
+    }
+  } else {
+    // the partial last page (fp16 residual rows < L % 16) or no page: copy
+    // the valid rows, zero the rest
+    const int rres = (pg == nfull && pg < np) ? L - nfull * kPage : 0;
+    const long res_base = (static_cast<long>(b) * H + h) * kPage * kHeadDim;
+    const __half *rk = p.res_k + res_base;
+    const __half *rv = p.res_v + res_base;
+    for (int e = widx; e < kPage * kHeadDim / 2; e += 64) {
+      const int tk = e >> 6, c = 2 * (e & 63);
+      uint32_t kb = 0;
+      if (tk < rres) kb = *reinterpret_cast<const uint32_t *>(rk + tk * kHeadDim + c);
+      const uint32_t ko = tc05::sw128_offset(dpage * 16 + tk, c, 64);
+      sts32(sKh + ko, kb);
+      sts32(sKl + ko, 0u);
+    }
+    for (int e = widx; e < kPage * kHeadDim; e += 64) {
+      const int tk = e >> 7, c = e & 127;
+      uint16_t vb = 0;
+      if (tk < rres) vb = __half_as_ushort(rv[tk * kHeadDim + c]);
+      sts16(sV + tc05::sw128_offset(c, dpage * 16 + tk, 128), vb);
+    }
+  }
+  __syncthreads();
+
+  // ---- the tile to the workspace, coalesced 16-byte stores
+  uint4 *dst = reinterpret_cast<uint4 *>(
+      p.ws + ((static_cast<long long>(b) * H + h) * p.tiles_per_seq + kt) * kTileBytes);
+  for (int i = t; i < static_cast<int>(kTileBytes / 16); i += kOpThreads) dst[i] = lds128_at(base + 16 * i);
+}
+
+// ---------------------------------------------------------------------------
+// Launch 2: the attention itself, reading the operand tiles of launch 1.
 __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(const PrefillParams p) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_addr(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
-  const uint32_t sQ = base + kOffQ, sP = base + kOffP;
-  const uint32_t stage0 = base + kOffStage;
+  const uint32_t sQ = base + kOffQ;
   const uint32_t bars = base + kOffBar;
   const uint32_t tslot = base + kOffSlot;
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem_raw + (base + kOffAbort - raw));
-  auto khi = [&](int s) { return base + kOffKhi + s * kKBytes; };
-  auto klo = [&](int s) { return base + kOffKlo + s * kKBytes; };
-  auto vop = [&](int s) { return base + kOffV + s * kVBytes; };
+  auto stage = [&](int s) { return base + kOffStage + s * kStageBytes; };
+  auto pbuf = [&](int s) { return base + kOffP + s * kPBytes; };
   auto stage_full = [&](int s) { return bars + 8u * (0 + s); };
-  auto stage_empty = [&](int s) { return bars + 8u * (2 + s); };
-  auto kv_full = [&](int s) { return bars + 8u * (4 + s); };
-  auto kv_empty = [&](int s) { return bars + 8u * (6 + s); };
-  auto s_full = [&](int s) { return bars + 8u * (8 + s); };
-  auto s_empty = [&](int s) { return bars + 8u * (10 + s); };
-  const uint32_t p_full = bars + 8u * 12, p_empty = bars + 8u * 13;
+  auto stage_empty = [&](int s) { return bars + 8u * (3 + s); };
+  auto s_full = [&](int s) { return bars + 8u * (6 + s); };
+  auto s_empty = [&](int s) { return bars + 8u * (8 + s); };
+  auto p_full = [&](int s) { return bars + 8u * (10 + s); };
+  auto p_empty = [&](int s) { return bars + 8u * (12 + s); };
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int G = p.group, H = p.num_kv_heads;
@@ -163,44 +317,38 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(const PrefillPara
   const int tile = static_cast<int>(gridDim.x) - 1 - static_cast<int>(blockIdx.x);  // long tiles first
 
   // ---- this CTA's rows (uniform across the CTA; exits before any allocation)
-  const int c_lo = __ldg(p.cu_new + b), c_hi = __ldg(p.cu_new + b + 1);
-  const int n = c_hi - c_lo;
+  SeqRows sr;
+  if (!seq_rows(p, b, tile == 0 && h == 0 && tid == 0, sr)) return;
+  const int c_lo = sr.c_lo, n = sr.n, L = sr.L;
   const int t0 = tile * Tq;
-  if (n <= 0 || t0 >= n) return;
-  const int L = __ldg(p.seq_lens + b);
-  if (c_lo < 0 || c_hi > p.n_tokens || L < n || L > p.max_pages * kPage) {
-    if (tid == 0 && t0 == 0 && h == 0) flag_error(p.err, S4KV_EFLAG_SEQ_LEN);
-    return;
-  }
+  if (t0 >= n) return;
   const int tq = min(Tq, n - t0);
   const int rows = tq * G;
   const int pos_first = L - n + t0;
   const int n_keys = pos_first + tq;                         // keys 0 .. pos_last
   const int n_ktiles = (n_keys + kKeyTile - 1) / kKeyTile;
-  const int nfull = L / kPage;
-  const int np = (L + kPage - 1) / kPage;
 
-  // ---- setup: tensor memory (S buffers at columns 0 and 64, O at 128), barriers
+  // ---- setup: tensor memory, barriers, Q, the ones rows of every stage
   if (warp == 0) {
-    tc05::tmem_alloc(tslot, 256);
+    tc05::tmem_alloc(tslot, kTmemCols);
     tc05::tmem_relinquish();
     tc05::fence_before_sync();
   }
   if (tid == 0) {
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < kStages; ++s) {
       mbar_init(stage_full(s), 1);
-      mbar_init(stage_empty(s), kDqThreads);
-      mbar_init(kv_full(s), kDqThreads);
-      mbar_init(kv_empty(s), 1);
+      mbar_init(stage_empty(s), 1);
+    }
+    for (int s = 0; s < 2; ++s) {
       mbar_init(s_full(s), 1);
       mbar_init(s_empty(s), 32 * kSoftmaxWarps);
+      mbar_init(p_full(s), 32 * kSoftmaxWarps);
+      mbar_init(p_empty(s), 1);
     }
-    mbar_init(p_full, 32 * kSoftmaxWarps);
-    mbar_init(p_empty, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
-  // ---- Q tile: row r = (token r / G, head r % G); rows >= rows are zero
+  // Q tile: row r = (token r / G, head r % G); rows >= rows are zero
   for (int ch = tid; ch < 128 * 16; ch += kThreadsP) {
     const int r = ch >> 4, c = ch & 15;
     const int tl = r / G, g = r - tl * G;
@@ -209,6 +357,10 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(const PrefillPara
       v = __ldg(reinterpret_cast<const uint4 *>(
                     p.q + (static_cast<long>(c_lo + t0 + tl) * p.num_q_heads + h * G + g) * kHeadDim) + c);
     sts128(sQ + tc05::sw128_offset(r, 8 * c, 128), v);
+  }
+  for (int i = tid; i < kStages * static_cast<int>(kOnesBytes / 16); i += kThreadsP) {
+    const int s = i / (kOnesBytes / 16), c = i - s * (kOnesBytes / 16);
+    sts128(stage(s) + kTileBytes + 16 * c, make_uint4(0x3C003C00u, 0x3C003C00u, 0x3C003C00u, 0x3C003C00u));
   }
   fence_proxy_async();
   __syncthreads();
@@ -225,175 +377,64 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(const PrefillPara
   if (warp == kProducerWarp) {
     // ---------------------------------------------------------- producer
     if (lane == 0) {
-      const int32_t *bt = p.block_tables + static_cast<long>(b) * p.max_pages;
-      const uint8_t *head_pool = p.pool + static_cast<long>(h) * kBlockBytes;
-      const long long page_stride = static_cast<long long>(H) * kBlockBytes;
+      const uint8_t *tiles = p.ws + (static_cast<long long>(b) * H + h) * p.tiles_per_seq * kTileBytes;
       int issued = 0;
-      for (int kt = 0; kt < n_ktiles && !failed; ++kt) {
-        const int s = kt & 1;
-        if (kt >= 2 && !wait_bounded(stage_empty(s), ((kt >> 1) - 1) & 1, abort_flag)) {
+      for (int kt = 0; kt < n_ktiles; ++kt) {
+        const int s = kt % kStages, u = kt / kStages;
+        if (kt >= kStages && !wait_bounded(stage_empty(s), (u - 1) & 1, abort_flag)) {
           fail();
           break;
         }
         ++issued;
-        const int pg0 = kt * kPagesPerTile;
-        const int q = max(0, min(kPagesPerTile, nfull - pg0));
-        mbar_arrive_expect_tx(stage_full(s), static_cast<uint32_t>(q) * kBlockBytes);
-        for (int k = 0; k < q; ++k) {
-          int phys = __ldg(bt + pg0 + k);
-          if (static_cast<unsigned>(phys) >= static_cast<unsigned>(p.num_pages)) {
-            flag_error(p.err, S4KV_EFLAG_PAGE_RANGE);
-            phys = 0;
-          }
-          bulk_copy_g2s(stage0 + s * kStageBytes + k * kBlockBytes, head_pool + phys * page_stride, kBlockBytes,
-                        stage_full(s));
-        }
+        mbar_arrive_expect_tx(stage_full(s), kTileBytes);
+        bulk_copy_g2s(stage(s), tiles + static_cast<long long>(kt) * kTileBytes, kTileBytes, stage_full(s));
       }
       // before the CTA exits, the copies in flight must have landed (bounded
       // by time only, also after an abort)
       const volatile int no_abort = 0;
-      for (int kt = max(0, issued - 2); kt < issued; ++kt) wait_bounded(stage_full(kt & 1), (kt >> 1) & 1, &no_abort);
-    }
-  } else if (warp >= kSoftmaxWarps && warp < kSoftmaxWarps + kDequantWarps) {
-    // -------------------------------------------------------- dequantizer
-    const int t = tid - 32 * kSoftmaxWarps;  // 0 .. 255
-    const int dpage = t >> 6, widx = t & 63;
-    const int dq = widx & 3, dlane0 = widx >> 2;
-    // swizzled store offsets of this thread's words (the same for every
-    // tile): keys rows 16 dpage + dn (and + 8 rows = + 1024 bytes), channels
-    // 32 di + 4 tt; values rows cb, cb + 1, keys 16 dpage + 2 di (+ 8)
-    uint32_t kofs[4], vofs[4][4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int ln = dlane0 + 16 * (e & 1), tt = 4 * (e >> 1) + dq;
-      const int dn = ln >> 2, di = ln & 3;
-      kofs[e] = tc05::sw128_offset(dpage * 16 + dn, 32 * di + 4 * tt, 64);
-      const int cb = 32 * (tt >> 1) + 4 * dn + 2 * (tt & 1);
-      const int key = dpage * 16 + 2 * di;
-      vofs[e][0] = tc05::sw128_offset(cb, key, 128);
-      vofs[e][1] = tc05::sw128_offset(cb + 1, key, 128);
-      vofs[e][2] = tc05::sw128_offset(cb, key + 8, 128);
-      vofs[e][3] = tc05::sw128_offset(cb + 1, key + 8, 128);
-    }
-    const long res_base = (static_cast<long>(b) * H + h) * kPage * kHeadDim;
-    for (int kt = 0; kt < n_ktiles; ++kt) {
-      const int s = kt & 1;
-      if (!wait_bounded(stage_full(s), (kt >> 1) & 1, abort_flag)) {
-        fail();
-        break;
-      }
-      if (kt >= 2 && !wait_bounded(kv_empty(s), ((kt >> 1) - 1) & 1, abort_flag)) {
-        fail();
-        break;
-      }
-      const uint32_t sKh = khi(s), sKl = klo(s), sV = vop(s);
-      const int pg = kt * kPagesPerTile + dpage;
-      const uint32_t blk = stage0 + s * kStageBytes + dpage * kBlockBytes;
-      if (pg < nfull) {
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int w = widx + 64 * e;
-          const int ln = dlane0 + 16 * (e & 1), tt = 4 * (e >> 1) + dq;
-          const int di = ln & 3;
-          // keys: tokens dn, dn + 8; channels c0 .. c0 + 3
-          {
-            uint32_t a0, a1, a2, a3;
-            unpack_codes(lds32_at(blk + kKCodeOff + 4 * w), a0, a1, a2, a3);
-            const int c0 = 32 * di + 4 * tt;
-            const uint2 sc = lds64_at(blk + kKScaleOff + 2 * c0);
-            const uint32_t zslot = 16 * tt + 2 * di;
-            const uint32_t z01 = lds32_at(blk + kKZeroOff + 2 * zslot);
-            const uint32_t z23 = lds32_at(blk + kKZeroOff + 2 * (zslot + 8));
-            const float2 s01 = __half22float2(u32_as_h2(sc.x)), s23 = __half22float2(u32_as_h2(sc.y));
-            const float2 zf01 = __half22float2(u32_as_h2(z01)), zf23 = __half22float2(u32_as_h2(z23));
-            uint32_t hi0, lo0, hi1, lo1, hi2, lo2, hi3, lo3;
-            split_key(a0, s01, zf01, hi0, lo0);
-            split_key(a1, s01, zf01, hi1, lo1);
-            split_key(a2, s23, zf23, hi2, lo2);
-            split_key(a3, s23, zf23, hi3, lo3);
-            sts64(sKh + kofs[e], hi0, hi2);
-            sts64(sKh + kofs[e] + 1024, hi1, hi3);
-            sts64(sKl + kofs[e], lo0, lo2);
-            sts64(sKl + kofs[e] + 1024, lo1, lo3);
-          }
-          // values: channels cb, cb + 1; tokens 2 di, 2 di + 1 (+ 8)
-          {
-            uint32_t a0, a1, a2, a3;
-            unpack_codes(lds32_at(blk + kVCodeOff + 4 * w), a0, a1, a2, a3);
-            const int g = tt >> 1;
-            const uint32_t sv_lo = lds32_at(blk + kVScaleOff + 2 * (16 * g + 2 * di));
-            const uint32_t sv_hi = lds32_at(blk + kVScaleOff + 2 * (16 * g + 2 * di + 8));
-            const uint32_t zv_lo = lds32_at(blk + kVZeroOff + 2 * (16 * g + 2 * di));
-            const uint32_t zv_hi = lds32_at(blk + kVZeroOff + 2 * (16 * g + 2 * di + 8));
-            sts32(sV + vofs[e][0], hfma2_u32(a0, sv_lo, zv_lo));
-            sts32(sV + vofs[e][1], hfma2_u32(a1, sv_lo, zv_lo));
-            sts32(sV + vofs[e][2], hfma2_u32(a2, sv_hi, zv_hi));
-            sts32(sV + vofs[e][3], hfma2_u32(a3, sv_hi, zv_hi));
-          }
-        }
-      } else {
-        // the partial last page (fp16 residual rows < L % 16) or no page:
-        // copy the valid rows, zero the rest, so masked keys hold finite values
-        const int rres = (pg == nfull && pg < np) ? L - nfull * kPage : 0;
-        const __half *rk = p.res_k + res_base;
-        const __half *rv = p.res_v + res_base;
-        for (int e = widx; e < kPage * kHeadDim / 2; e += 64) {
-          const int tk = e >> 6, c = 2 * (e & 63);
-          uint32_t kb = 0;
-          if (tk < rres) kb = *reinterpret_cast<const uint32_t *>(rk + tk * kHeadDim + c);
-          const uint32_t ko = tc05::sw128_offset(dpage * 16 + tk, c, 64);
-          sts32(sKh + ko, kb);
-          sts32(sKl + ko, 0u);
-        }
-        for (int e = widx; e < kPage * kHeadDim; e += 64) {
-          const int tk = e >> 7, c = e & 127;
-          uint16_t vb = 0;
-          if (tk < rres) vb = __half_as_ushort(rv[tk * kHeadDim + c]);
-          sts16(sV + tc05::sw128_offset(c, dpage * 16 + tk, 128), vb);
-        }
-      }
-      fence_proxy_async();  // operand writes -> MMA reads; staging reads -> the next bulk copy
-      mbar_arrive(kv_full(s));
-      mbar_arrive(stage_empty(s));
+      for (int kt = max(0, issued - kStages); kt < issued; ++kt)
+        wait_bounded(stage_full(kt % kStages), (kt / kStages) & 1, &no_abort);
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      auto issue_pv = [&](int k) {  // O += P(k) V(k)
-        const int s = k & 1;
-        if (!wait_bounded(p_full, k & 1, abort_flag)) return false;
+      auto issue_pv = [&](int k) {  // O += P(k) [V(k) | 1]
+        const int ps = k & 1, vs = k % kStages;
+        if (!wait_bounded(p_full(ps), (k >> 1) & 1, abort_flag)) return false;
         tc05::fence_after_sync();
+        const uint32_t sv = stage(vs) + 2 * kKBytes;
 #pragma unroll
         for (int j = 0; j < 4; ++j)
-          tc05::mma_f16_ss(tO, tc05::smem_desc_sw128(sP + 32 * j), tc05::smem_desc_sw128(vop(s) + 32 * j), kIdescO,
+          tc05::mma_f16_ss(tO, tc05::smem_desc_sw128(pbuf(ps) + 32 * j), tc05::smem_desc_sw128(sv + 32 * j), kIdescO,
                            (k > 0 || j > 0) ? 1u : 0u);
-        tc05::mma_commit(p_empty);
-        tc05::mma_commit(kv_empty(s));
+        tc05::mma_commit(p_empty(ps));
+        tc05::mma_commit(stage_empty(vs));
         return true;
       };
       for (int kt = 0; kt < n_ktiles; ++kt) {
-        const int s = kt & 1;
-        if (!wait_bounded(kv_full(s), (kt >> 1) & 1, abort_flag) ||
-            (kt >= 2 && !wait_bounded(s_empty(s), ((kt >> 1) - 1) & 1, abort_flag))) {
+        const int s3 = kt % kStages, ss = kt & 1;
+        if (!wait_bounded(stage_full(s3), (kt / kStages) & 1, abort_flag) ||
+            (kt >= 2 && !wait_bounded(s_empty(ss), ((kt >> 1) - 1) & 1, abort_flag))) {
           fail();
           break;
         }
         tc05::fence_after_sync();
         // S(kt) = Q K_hi^T + Q K_lo^T
+        const uint32_t skh = stage(s3), skl = stage(s3) + kKBytes;
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           const uint32_t qo = (j >> 2) * (kQBytes / 2) + (j & 3) * 32;
           const uint32_t ko = (j >> 2) * (kKBytes / 2) + (j & 3) * 32;
-          tc05::mma_f16_ss(tS(s), tc05::smem_desc_sw128(sQ + qo), tc05::smem_desc_sw128(khi(s) + ko), kIdescS,
+          tc05::mma_f16_ss(tS(ss), tc05::smem_desc_sw128(sQ + qo), tc05::smem_desc_sw128(skh + ko), kIdescS,
                            j > 0 ? 1u : 0u);
         }
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           const uint32_t qo = (j >> 2) * (kQBytes / 2) + (j & 3) * 32;
           const uint32_t ko = (j >> 2) * (kKBytes / 2) + (j & 3) * 32;
-          tc05::mma_f16_ss(tS(s), tc05::smem_desc_sw128(sQ + qo), tc05::smem_desc_sw128(klo(s) + ko), kIdescS, 1u);
+          tc05::mma_f16_ss(tS(ss), tc05::smem_desc_sw128(sQ + qo), tc05::smem_desc_sw128(skl + ko), kIdescS, 1u);
         }
-        tc05::mma_commit(s_full(s));
+        tc05::mma_commit(s_full(ss));
         // O += P(kt-1) V(kt-1) while the softmax of kt runs
         if (kt >= 1 && !issue_pv(kt - 1)) {
           fail();
@@ -409,11 +450,15 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(const PrefillPara
     const bool row_ok = row < rows;
     const int pos_row = pos_first + (row_ok ? row / G : 0);
     float ref = -INFINITY;
-    float2 lsum = make_float2(0.f, 0.f);
     const float sl2 = p.scale_log2;
+    // the warp takes every decision together (its lanes run warp-wide
+    // tensor-memory loads and votes)
+    auto wait_warp = [&](uint32_t bar, uint32_t parity) {
+      return __all_sync(0xFFFFFFFFu, wait_bounded(bar, parity, abort_flag));
+    };
     for (int kt = 0; kt < n_ktiles; ++kt) {
-      const int s = kt & 1;
-      if (!wait_bounded(s_full(s), (kt >> 1) & 1, abort_flag)) {
+      const int ss = kt & 1;
+      if (!wait_warp(s_full(ss), (kt >> 1) & 1)) {
         fail();
         break;
       }
@@ -422,12 +467,12 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(const PrefillPara
       {
         uint32_t (&v0)[32] = *reinterpret_cast<uint32_t (*)[32]>(&v[0]);
         uint32_t (&v1)[32] = *reinterpret_cast<uint32_t (*)[32]>(&v[32]);
-        tc05::tmem_ld32(tS(s) + lane_base, v0);
-        tc05::tmem_ld32(tS(s) + lane_base + 32, v1);
+        tc05::tmem_ld32(tS(ss) + lane_base, v0);
+        tc05::tmem_ld32(tS(ss) + lane_base + 32, v1);
         tc05::tmem_wait_ld();
       }
       tc05::fence_before_sync();
-      mbar_arrive(s_empty(s));
+      mbar_arrive(s_empty(ss));
       // a key tile wholly before the tile's first query position needs no
       // mask (rows past the last row hold q = 0: finite logits, never written)
       const int key0 = kt * kKeyTile;
@@ -450,61 +495,71 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(const PrefillPara
       const bool move = mx > ref + kSlack;
       const float new_ref = move ? mx : ref;
       const float alpha = move ? fast_exp2(ref - new_ref) : 1.0f;  // 0 when ref was -inf
-      // O and P are free once O += P(kt-1) V(kt-1) has completed
-      if (kt >= 1) {
-        if (!wait_bounded(p_empty, (kt - 1) & 1, abort_flag)) {
+      // weights exp2(s * scale - ref) in registers; masked logits are -inf
+      // and give 0 (a row without a valid key keeps a -inf reference,
+      // replaced by 0 so that no inf - inf appears)
+      const float nref = new_ref == -INFINITY ? 0.f : -new_ref;
+      const float2 sc = make_float2(sl2, sl2), nr = make_float2(nref, nref);
+      uint32_t hp[32];
+#pragma unroll
+      for (int j = 0; j < 64; j += 2) {
+        const float2 x = fma2(make_float2(__uint_as_float(v[j]), __uint_as_float(v[j + 1])), sc, nr);
+        hp[j >> 1] = h2_as_u32(__floats2half2_rn(fast_exp2(x.x), fast_exp2(x.y)));
+      }
+      // a moved reference rescales O and its sum column once O += P(kt-1) V
+      // has completed (P(kt) is not yet handed over, so O is idle)
+      if (kt >= 1 && __any_sync(0xFFFFFFFFu, move)) {
+        if (!wait_warp(p_empty((kt - 1) & 1), ((kt - 1) >> 1) & 1)) {
           fail();
           break;
         }
         tc05::fence_after_sync();
-        if (__any_sync(0xFFFFFFFFu, move)) {
-          const float2 a2 = make_float2(alpha, alpha);
+        const float2 a2 = make_float2(alpha, alpha);
 #pragma unroll 1
-          for (int c = 0; c < 4; ++c) {
-            uint32_t o[32];
-            tc05::tmem_ld32(tO + lane_base + 32 * c, o);
-            tc05::tmem_wait_ld();
+        for (int c = 0; c < 4; ++c) {
+          uint32_t o[32];
+          tc05::tmem_ld32(tO + lane_base + 32 * c, o);
+          tc05::tmem_wait_ld();
 #pragma unroll
-            for (int j = 0; j < 32; j += 2) {
-              const float2 r = mul2(make_float2(__uint_as_float(o[j]), __uint_as_float(o[j + 1])), a2);
-              o[j] = __float_as_uint(r.x);
-              o[j + 1] = __float_as_uint(r.y);
-            }
-            tc05::tmem_st32(tO + lane_base + 32 * c, o);
+          for (int j = 0; j < 32; j += 2) {
+            const float2 r = mul2(make_float2(__uint_as_float(o[j]), __uint_as_float(o[j + 1])), a2);
+            o[j] = __float_as_uint(r.x);
+            o[j + 1] = __float_as_uint(r.y);
           }
-          tc05::tmem_wait_st();
+          tc05::tmem_st32(tO + lane_base + 32 * c, o);
         }
+        {
+          uint32_t o[16];
+          tc05::tmem_ld16(tO + lane_base + 128, o);
+          tc05::tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 16; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
+          tc05::tmem_st16(tO + lane_base + 128, o);
+        }
+        tc05::tmem_wait_st();
       }
-      lsum = mul2(lsum, make_float2(alpha, alpha));
       ref = new_ref;
-      // weights exp2(s * scale - ref); masked logits are -inf and give 0 (a
-      // row without a valid key keeps a -inf reference, replaced by 0 so that
-      // no inf - inf appears)
-      const float nref = ref == -INFINITY ? 0.f : -ref;
-      const float2 sc = make_float2(sl2, sl2), nr = make_float2(nref, nref);
-#pragma unroll
-      for (int q8 = 0; q8 < 8; ++q8) {
-        uint32_t hp[4];
-#pragma unroll
-        for (int j = 0; j < 8; j += 2) {
-          const int k = 8 * q8 + j;
-          const float2 x = fma2(make_float2(__uint_as_float(v[k]), __uint_as_float(v[k + 1])), sc, nr);
-          const __half2 ph = __floats2half2_rn(fast_exp2(x.x), fast_exp2(x.y));
-          // the row sum takes the fp16 weights the MMA multiplies with
-          lsum = add2(lsum, __half22float2(ph));
-          hp[j >> 1] = h2_as_u32(ph);
-        }
-        sts128(sP + tc05::sw128_offset(row, 8 * q8, 128), make_uint4(hp[0], hp[1], hp[2], hp[3]));
+      // P buffer ss is free once O += P(kt-2) V has completed
+      if (kt >= 2 && !wait_warp(p_empty(ss), ((kt >> 1) - 1) & 1)) {
+        fail();
+        break;
       }
+#pragma unroll
+      for (int q8 = 0; q8 < 8; ++q8)
+        sts128(pbuf(ss) + tc05::sw128_offset(row, 8 * q8, 128),
+               make_uint4(hp[4 * q8], hp[4 * q8 + 1], hp[4 * q8 + 2], hp[4 * q8 + 3]));
       fence_proxy_async();
       tc05::fence_before_sync();
-      mbar_arrive(p_full);
+      mbar_arrive(p_full(ss));
     }
     // ---- out = O / l once the last O += P V has completed
-    if (!failed && !wait_bounded(p_empty, (n_ktiles - 1) & 1, abort_flag)) fail();
+    if (!failed && !wait_warp(p_empty((n_ktiles - 1) & 1), ((n_ktiles - 1) >> 1) & 1)) fail();
     if (!failed) {
       tc05::fence_after_sync();
-      const float l = lsum.x + lsum.y;
+      uint32_t ls[16];
+      tc05::tmem_ld16(tO + lane_base + 128, ls);
+      tc05::tmem_wait_ld();
+      const float l = __uint_as_float(ls[0]);
       const float inv = row_ok && l > 0.f ? 1.0f / l : 0.f;
       const int tl = row / G, g = row - (row / G) * G;
       __half *dst = p.out + (static_cast<long>(c_lo + t0 + tl) * p.num_q_heads + h * G + g) * kHeadDim;
@@ -532,18 +587,24 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(const PrefillPara
   __syncthreads();
   if (warp == 0) {
     tc05::fence_after_sync();
-    tc05::tmem_dealloc(tmem, 256);
+    tc05::tmem_dealloc(tmem, kTmemCols);
   }
 }
 
 size_t prefill_smem_bytes() { return kSmemBytes; }
+size_t prefill_tile_bytes() { return kTileBytes; }
 
 cudaError_t prepare_prefill_kernel() {
-  return cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              static_cast<int>(kSmemBytes));
+  cudaError_t e = cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(kSmemBytes));
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(prefill_operands_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              static_cast<int>(kOpSmemBytes));
 }
 
 void launch_prefill(const PrefillParams &p, int batch, int max_new, cudaStream_t stream) {
+  const dim3 og(p.tiles_per_seq, batch, p.num_kv_heads);
+  prefill_operands_kernel<<<og, kOpThreads, kOpSmemBytes, stream>>>(p);
   const int Tq = 128 / p.group;
   const int tiles = (max_new + Tq - 1) / Tq;
   const dim3 grid(tiles, batch, p.num_kv_heads);

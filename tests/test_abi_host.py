@@ -106,9 +106,10 @@ def test_invalid_calls_rejected_before_launch(S):
     # prefill
     pre = L.s4kv_prefill_attention
     args = lambda **kw: dict(dict(cache=ctypes.byref(c), q=P(fake), hq=8, n=4, cu=P(fake), sl=P(fake), bt=P(fake),
-                                  batch=1, maxp=1, maxnew=4, scale=0.088, out=P(fake)), **kw)
+                                  batch=1, maxp=1, maxnew=4, scale=0.088, out=P(fake), ws=P(fake),
+                                  wsb=1 << 30), **kw)
     call = lambda a: pre(a["cache"], a["q"], a["hq"], a["n"], a["cu"], a["sl"], a["bt"], a["batch"], a["maxp"],
-                         a["maxnew"], a["scale"], a["out"], st)
+                         a["maxnew"], a["scale"], a["out"], a["ws"], a["wsb"], st)
     assert call(args(hq=18)) == S.ERR_UNSUPPORTED
     assert call(args(cache=ctypes.byref(bad_dim))) == S.ERR_UNSUPPORTED
     assert call(args(scale=float("nan"))) == S.ERR_INVALID_ARG
@@ -118,6 +119,18 @@ def test_invalid_calls_rejected_before_launch(S):
     assert call(args(maxnew=5)) == S.ERR_INVALID_ARG  # more than n_tokens
     assert call(args(batch=5)) == S.ERR_INVALID_ARG   # batch > max_seqs
     assert call(args(n=0)) == S.OK and call(args(batch=0)) == S.OK  # nothing to do
+    # workspace: 48 KB per 64-key tile per (sequence slot, kv head)
+    assert S.prefill_workspace_bytes(2, 1, 1) == 2 * 49152
+    assert S.prefill_workspace_bytes(8, 4, 512) == 4 * 8 * 128 * 49152
+    assert S.prefill_workspace_bytes(1, 1, 5) == 2 * 49152  # 5 pages round up to 2 tiles
+    n = ctypes.c_size_t(0)
+    assert L.s4kv_prefill_workspace_size(0, 1, 1, ctypes.byref(n)) == S.ERR_INVALID_ARG
+    assert L.s4kv_prefill_workspace_size(1, 1, 0, ctypes.byref(n)) == S.ERR_INVALID_ARG
+    assert L.s4kv_prefill_workspace_size(1, 1, 1, None) == S.ERR_INVALID_ARG
+    assert L.s4kv_prefill_workspace_size(65535, 65535, 1 << 30, ctypes.byref(n)) == S.ERR_INVALID_ARG
+    assert call(args(ws=None)) == S.ERR_WORKSPACE
+    assert call(args(ws=P(fake + 8))) == S.ERR_WORKSPACE  # not 16-B aligned
+    assert call(args(wsb=2 * 49152 - 1)) == S.ERR_WORKSPACE
     # dequant
     assert L.s4kv_dequant_page(ctypes.byref(c), 10, P(fake), P(fake), 1, st) == S.ERR_INVALID_ARG
     assert L.s4kv_dequant_page(ctypes.byref(c), -1, P(fake), P(fake), 1, st) == S.ERR_INVALID_ARG
@@ -126,7 +139,8 @@ def test_invalid_calls_rejected_before_launch(S):
     bad_bits = S.s4kv_cache_t(fake, fake, fake, None, 10, 2, 4, 128, 16, 3)
     assert L.s4kv_dequant_page(ctypes.byref(bad_bits), 0, P(fake), P(fake), 1, st) == S.ERR_UNSUPPORTED
     c8 = S.s4kv_cache_t(fake, fake, fake, None, 10, 2, 4, 128, 16, 8)
-    assert pre(ctypes.byref(c8), P(fake), 8, 4, P(fake), P(fake), P(fake), 1, 1, 4, 0.088, P(fake), st) == S.ERR_UNSUPPORTED
+    assert pre(ctypes.byref(c8), P(fake), 8, 4, P(fake), P(fake), P(fake), 1, 1, 4, 0.088, P(fake), P(fake), 1 << 30,
+               st) == S.ERR_UNSUPPORTED
     n = ctypes.c_size_t(0)
     assert L.s4kv_page_record_bytes(ctypes.byref(c8), ctypes.byref(n)) == S.OK and n.value == 2 * 4864
     assert L.s4kv_page_record_bytes(ctypes.byref(c), ctypes.byref(n)) == S.OK and n.value == 2 * 2816

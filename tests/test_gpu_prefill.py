@@ -60,12 +60,12 @@ class PrefillCase:
             self.S.s4kv_append(self.gpu, self.dev(k), self.dev(v), self.dev(sm), self.dev(cu), self.dev(sl),
                                self.bt_dev, mx)
 
-    def run(self, sm_scale=None):
+    def run(self, sm_scale=None, workspace=None):
         import torch
         qd = self.dev(self.q)
         out = torch.full_like(qd, float("nan"))
         self.S.s4kv_prefill_attention(self.gpu, qd, self.dev(self.cu), self.dev(self.after.astype(np.int32)),
-                                      self.bt_dev, out, int(max(self.n.max(), 1)), sm_scale)
+                                      self.bt_dev, out, int(max(self.n.max(), 1)), sm_scale, workspace=workspace)
         torch.cuda.synchronize()
         assert self.S.s4kv_get_error(self.gpu) == 0
         got = out.float().cpu().numpy()
@@ -114,3 +114,21 @@ def test_prefill_last_row_matches_decode():
     torch.cuda.synchronize()
     assert_attention_close(out.float().cpu().numpy(), ref[last], "decode of the last rows")
     assert_attention_close(got[last], ref[last], "prefill of the last rows")
+
+
+def test_prefill_ignores_stale_workspace_contents():
+    """Every operand byte the attention reads is written by the same call:
+    a workspace full of fp16 NaN patterns (0xFF bytes) gives the same output
+    as a fresh one, also for keys past L inside the last tile (zero-filled)."""
+    import torch
+    case = PrefillCase(80, 2, 4, before=[3, 70], after=[45, 200])
+    ws = case.S.prefill_workspace(2, 2, case.bt.shape[1])
+    ws.fill_(0xFF)
+    got, ref = case.run(workspace=ws)
+    assert not np.isnan(got[:int(case.cu[-1])]).any()
+    assert_attention_close(got, ref, "prefill, stale workspace")
+    # the workspace reused for a second case of smaller sequences
+    small = PrefillCase(81, 2, 4, before=[0, 17], after=[20, 33])
+    ws2 = ws[:case.S.prefill_workspace_bytes(2, 2, small.bt.shape[1])]
+    got2, ref2 = small.run(workspace=ws2)
+    assert_attention_close(got2, ref2, "prefill, reused workspace")
