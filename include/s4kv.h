@@ -282,14 +282,14 @@ S4KV_API int s4kv_decode_attention_noalloc(const s4kv_cache_t *cache, const void
  *          max_pages_per_seq) bytes (else S4KV_ERR_WORKSPACE and nothing is
  *          launched).  Its contents are overwritten and mean nothing after the
  *          call; it must not be shared with work that runs concurrently.
- * Two launches on `stream`: the first dequantizes every 64-key tile of each
+ * Two launches on `stream`: the first dequantizes every 128-key tile of each
  * (sequence, kv head) once into the workspace as fp16 MMA operands (keys as
  * an fp16 hi part plus the fp16 rounding of the remainder, about 22 bits;
  * values correctly rounded to fp16); the second runs the attention on the
  * tcgen05 tensor cores with those operands and the fp16 softmax weights
  * (fp32 accumulation), so results agree with exact attention to about fp16
  * precision of the values and the weights.  Allocates nothing; the attention
- * launch needs about 215 KB of shared memory per CTA.  4-bit codes only (2-
+ * launch needs about 225 KB of shared memory per CTA.  4-bit codes only (2-
  * and 8-bit caches are refused with S4KV_ERR_UNSUPPORTED). */
 S4KV_API int s4kv_prefill_attention(const s4kv_cache_t *cache, const void *q,
                                     int num_q_heads, int n_tokens,
@@ -299,9 +299,9 @@ S4KV_API int s4kv_prefill_attention(const s4kv_cache_t *cache, const void *q,
                                     float sm_scale, void *out, void *workspace,
                                     size_t workspace_bytes, void *stream);
 
-/* Bytes of workspace s4kv_prefill_attention needs: 48 KB per 64-key tile of
- * max_pages_per_seq pages (rounded up to whole tiles), per sequence slot and
- * kv head.  S4KV_ERR_INVALID_ARG for non-positive sizes or a total above
+/* Bytes of workspace s4kv_prefill_attention needs: 96 KB per 128-key tile
+ * of max_pages_per_seq pages (rounded up to whole tiles of 8 pages), per
+ * sequence slot and kv head.  S4KV_ERR_INVALID_ARG for non-positive sizes or a total above
  * 2^40 bytes. */
 S4KV_API int s4kv_prefill_workspace_size(int num_kv_heads, int batch, int max_pages_per_seq,
                                          size_t *bytes);

@@ -288,7 +288,7 @@ extern "C" {
 
 int s4kv_prefill_workspace_size(int num_kv_heads, int batch, int max_pages_per_seq, size_t *bytes) {
   if (!bytes || num_kv_heads <= 0 || batch < 0 || max_pages_per_seq <= 0) return S4KV_ERR_INVALID_ARG;
-  const unsigned long long tiles = (static_cast<unsigned long long>(max_pages_per_seq) + 3) / 4;
+  const unsigned long long tiles = static_cast<unsigned long long>(prefill_tiles_per_seq(max_pages_per_seq));
   const unsigned long long n = tiles * static_cast<unsigned long long>(batch) * num_kv_heads;
   if (n > (1ull << 40) / prefill_tile_bytes()) return S4KV_ERR_INVALID_ARG;
   *bytes = static_cast<size_t>(n * prefill_tile_bytes());
@@ -349,7 +349,7 @@ int s4kv_prefill_attention(const s4kv_cache_t *cache, const void *q, int num_q_h
   p.num_pages = cache->num_pages;
   p.scale_log2 = static_cast<float>(static_cast<double>(sm_scale) * 1.4426950408889634);
   p.ws = static_cast<uint8_t *>(workspace);
-  p.tiles_per_seq = (max_pages_per_seq + 3) / 4;
+  p.tiles_per_seq = prefill_tiles_per_seq(max_pages_per_seq);
   launch_prefill(p, batch, max_new_per_seq, static_cast<cudaStream_t>(stream));
   if (cudaGetLastError() != cudaSuccess) return S4KV_ERR_CUDA;
   return S4KV_OK;

@@ -104,8 +104,8 @@ struct PrefillParams {
   int max_pages;
   int num_pages;
   float scale_log2;       // sm_scale * log2(e)
-  uint8_t *ws;            // operand tiles [batch][num_kv_heads][tiles_per_seq][48 KB]
-  int tiles_per_seq;      // ceil(max_pages / 4)
+  uint8_t *ws;            // operand tiles [batch][num_kv_heads][tiles_per_seq][tile bytes]
+  int tiles_per_seq;      // key tiles of max_pages pages
 };
 
 void launch_append(const AppendParams &p, int batch, int max_new, cudaStream_t stream);
@@ -120,5 +120,6 @@ void launch_prefill(const PrefillParams &p, int batch, int max_new, cudaStream_t
 cudaError_t prepare_prefill_kernel();
 size_t prefill_smem_bytes();
 size_t prefill_tile_bytes();
+int prefill_tiles_per_seq(int max_pages);
 
 }  // namespace s4kv

@@ -13,10 +13,10 @@
 //
 // How (B200): this is a dense contraction, so it runs on the fifth-generation
 // tensor cores, in two launches.
-//  1. prefill_operands_kernel dequantizes every key tile (64 keys, 4 pages)
-//     of every (sequence, kv head) ONCE into a workspace tile of 48 KB that
+//  1. prefill_operands_kernel dequantizes every key tile (128 keys, 8 pages)
+//     of every (sequence, kv head) ONCE into a workspace tile of 96 KB that
 //     holds the MMA operands exactly as shared memory wants them (128-byte
-//     swizzled, K-major): K_hi, K_lo and V^T.  A key is code * scale + zero
+//     swizzled, K-major): [K_hi; K_lo] and V^T.  A key is code * scale + zero
 //     in fp32 (exact product, one rounding, the value the oracle's
 //     dequantization gives) split into an fp16 hi part and the fp16 rounding
 //     of the remainder, so K_hi + K_lo carries it to about 22 bits (keys of
@@ -29,19 +29,22 @@
 //     tile's 128 MMA rows are (token, head of the group) pairs, so a tile
 //     holds floor(128 / G) tokens.  Warps with separate roles hand buffers
 //     over through mbarriers:
-//      * a producer warp brings each key tile's 48 KB into one of three
-//        shared-memory stages with one 1-D bulk copy (TMA engine, no
-//        multicast);
-//      * one thread issues S(k) = Q K_hi^T + Q K_lo^T (M = 128, N = 64) into
-//        one of two tensor-memory buffers, then O += P(k-1) [V(k-1) | 1]
-//        (N = 144, K = 64): 16 rows of ones after V^T make the tensor core
-//        accumulate each row's sum of the fp16 weights next to O;
+//      * a producer warp brings each key tile's [K_hi; K_lo] (64 KB) and V^T
+//        (32 KB) into one of two K and one of two V buffers with 1-D bulk
+//        copies (TMA engine, no multicast); a K buffer is refilled as soon as
+//        the S MMAs that read it complete, a V buffer once the PV MMAs have;
+//      * one thread issues S(k) = Q [K_hi; K_lo]^T (M = 128, N = 256: the hi
+//        and lo rows of the 128 keys stacked, so one MMA instruction per
+//        16 channels covers both) into tensor memory, then
+//        O += P(k-1) V(k-1) (N = 128, K = 128) with P read from tensor
+//        memory.  Few, large MMA instructions keep the single issuing thread
+//        ahead of the tensor core;
 //      * 4 softmax warps (one tensor-memory lane, i.e. one row, per thread)
-//        read S back, apply the causal mask and an online softmax in the exp2
-//        domain whose reference moves only when a row maximum passes it by
-//        more than 8 (weights stay <= 256, fine for fp16), rescale that row
-//        of O (and its sum) in tensor memory when it moves, and write P
-//        (fp16) into one of two shared-memory buffers.
+//        read S_hi + S_lo back, apply the causal mask and an online softmax
+//        in the exp2 domain whose reference moves only when a row maximum
+//        passes it by more than 8 (weights stay <= 256, fine for fp16),
+//        rescale that row of O in tensor memory when it moves, and write P
+//        (fp16 pairs) into tensor memory.
 // Every wait is bounded; a timeout sets a CTA-wide abort flag and an error
 // bit, and every role then leaves its loop.
 #include <cfloat>
@@ -57,39 +60,40 @@ constexpr int kSoftmaxWarps = 4;   // warps 0..3: one row per thread
 constexpr int kMmaWarp = 4;
 constexpr int kProducerWarp = 5;
 constexpr int kThreadsP = 32 * 6;
-constexpr int kOpThreads = 256;                  // operand kernel: 64 threads per page
-constexpr int kKeyTile = 64;                     // keys per tile (MMA N of S)
-constexpr int kPagesPerTile = kKeyTile / kPage;  // 4
-constexpr int kStages = 3;
+constexpr int kKeyTile = 128;                    // keys per tile
+constexpr int kPagesPerTile = kKeyTile / kPage;  // 8
+constexpr int kOpThreads = 64 * kPagesPerTile;   // operand kernel: 64 threads per page
+constexpr int kStages = 2;                       // K and V buffers each
 constexpr uint32_t kQBytes = 128 * 128 * 2;      // Q [128][128] fp16
-constexpr uint32_t kKBytes = 64 * 128 * 2;       // K [64][128] fp16
-constexpr uint32_t kVBytes = 128 * 64 * 2;       // V^T [128][64] fp16
-constexpr uint32_t kOnesBytes = 16 * 64 * 2;     // 16 rows of ones after V^T
-constexpr uint32_t kPBytes = 128 * 64 * 2;       // P [128][64] fp16
-constexpr uint32_t kTileBytes = 2 * kKBytes + kVBytes;      // workspace tile: K_hi, K_lo, V^T
-constexpr uint32_t kStageBytes = kTileBytes + kOnesBytes;
+constexpr uint32_t kKBytes = 2 * kKeyTile * 128 * 2;   // [K_hi; K_lo] [256][128] fp16
+constexpr uint32_t kVBytes = 128 * kKeyTile * 2;       // V^T [128][128] fp16
+constexpr uint32_t kTileBytes = kKBytes + kVBytes;     // workspace tile
 constexpr uint32_t kStagingBytes = kPagesPerTile * kBlockBytes;
-constexpr int kOutCols = 144;                    // O: 128 channels, then 16 copies of the row sum
 constexpr float kSlack = 8.0f;                   // log2 slack of the softmax reference
 constexpr long long kWaitLimit = 2000000000LL;   // about one second
-constexpr uint32_t kIdescS = tc05::idesc_f16_f32(128, 64);
-constexpr uint32_t kIdescO = tc05::idesc_f16_f32(128, kOutCols);
-constexpr uint32_t kTmemCols = 512;              // S[2] at 0 and 64, O at 128 .. 271
+// S: M = 128, N = 256 (K_hi and K_lo rows stacked); PV: M = 128, N = 128
+constexpr uint32_t kIdescS = tc05::idesc_f16_f32(128, 2 * kKeyTile);
+constexpr uint32_t kIdescO = tc05::idesc_f16_f32(128, 128);
+// tensor memory (512 columns): S_hi at 0, S_lo at 128, O at 256, P (fp16
+// pairs, the PV A operand) at 384
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColS = 0, kColO = 256, kColP = 384;
 
-// attention kernel smem: Q, three stages, two P buffers (1024-aligned), barriers
+// attention kernel smem (1024-aligned operands): Q, two K and two V buffers,
+// barriers
 constexpr uint32_t kOffQ = 0;
-constexpr uint32_t kOffStage = kOffQ + kQBytes;                  // [3]
-constexpr uint32_t kOffP = kOffStage + kStages * kStageBytes;    // [2]
-constexpr uint32_t kOffBar = kOffP + 2 * kPBytes;
-// barriers (8 bytes each): stage_full[3], stage_empty[3], s_full[2],
-// s_empty[2], p_full[2], p_empty[2]; then the tensor-memory address and the
+constexpr uint32_t kOffK = kOffQ + kQBytes;                      // [2]
+constexpr uint32_t kOffV = kOffK + kStages * kKBytes;            // [2]
+constexpr uint32_t kOffBar = kOffV + kStages * kVBytes;
+// barriers (8 bytes each): k_full[2], k_empty[2], v_full[2], v_empty[2],
+// s_full, s_empty, p_full, p_empty; then the tensor-memory address and the
 // abort flag
-constexpr uint32_t kNumBars = 14;
+constexpr uint32_t kNumBars = 12;
 constexpr uint32_t kOffSlot = kOffBar + 8 * kNumBars;
 constexpr uint32_t kOffAbort = kOffSlot + 4;
 constexpr uint32_t kSmemBytes = kOffAbort + 4 + 1024;  // + alignment slack
 static_assert(kSmemBytes <= 227 * 1024, "prefill shared memory");
-static_assert(kStageBytes % 1024 == 0 && kOffP % 1024 == 0, "1024-byte operand alignment");
+static_assert(kKBytes % 1024 == 0 && kVBytes % 1024 == 0 && kOffBar % 1024 == 0, "1024-byte operand alignment");
 
 // operand kernel smem: the output tile, then the staged page blocks
 constexpr uint32_t kOpSmemBytes = kTileBytes + kStagingBytes + 1024;
@@ -102,6 +106,13 @@ __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, cons
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort || clock64() - t0 > kWaitLimit) return false;
+  }
+}
+
+// Bounded wait used while draining copies before the CTA exits (time only).
+__device__ __forceinline__ void wait_landed(uint32_t bar, uint32_t parity) {
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity) && clock64() - t0 <= kWaitLimit) {
   }
 }
 
@@ -176,14 +187,16 @@ __device__ __forceinline__ bool seq_rows(const PrefillParams &p, int b, bool fla
 
 // ---------------------------------------------------------------------------
 // Launch 1: one CTA per (key tile, sequence, kv head) writes the tile's
-// operands [K_hi | K_lo | V^T] (16 KB each, 128-byte swizzled K-major) to the
-// workspace.  Keys at or past L (the rest of the partial last page, pages
-// after it) are written as zeros, so masked keys hold finite values.
+// operands to the workspace: [K_hi; K_lo] as one [256][128] operand (rows
+// 0..127 the hi parts of keys 0..127, rows 128..255 their lo parts) and V^T
+// [128][128], both 128-byte swizzled K-major.  Keys at or past L (the rest of
+// the partial last page, pages after it) are written as zeros, so masked
+// keys hold finite values.
 __global__ void __launch_bounds__(kOpThreads) prefill_operands_kernel(const PrefillParams p) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_addr(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
-  const uint32_t sKh = base, sKl = base + kKBytes, sV = base + 2 * kKBytes;
+  const uint32_t sK = base, sV = base + kKBytes;
   const uint32_t stage = base + kTileBytes;
   const int kt = blockIdx.x, b = blockIdx.y, h = blockIdx.z, H = p.num_kv_heads;
   const int t = threadIdx.x;
@@ -238,11 +251,13 @@ __global__ void __launch_bounds__(kOpThreads) prefill_operands_kernel(const Pref
         split_key(a1, s01, zf01, hi1, lo1);
         split_key(a2, s23, zf23, hi2, lo2);
         split_key(a3, s23, zf23, hi3, lo3);
-        const uint32_t ko = tc05::sw128_offset(dpage * 16 + dn, c0, 64);
-        sts64(sKh + ko, hi0, hi2);
-        sts64(sKh + ko + 1024, hi1, hi3);
-        sts64(sKl + ko, lo0, lo2);
-        sts64(sKl + ko + 1024, lo1, lo3);
+        const int key = dpage * 16 + dn;
+        const uint32_t kh = tc05::sw128_offset(key, c0, 2 * kKeyTile);
+        const uint32_t kl = tc05::sw128_offset(kKeyTile + key, c0, 2 * kKeyTile);
+        sts64(sK + kh, hi0, hi2);
+        sts64(sK + kh + 1024, hi1, hi3);
+        sts64(sK + kl, lo0, lo2);
+        sts64(sK + kl + 1024, lo1, lo3);
       }
       // values: channels cb, cb + 1; tokens 2 di, 2 di + 1 (+ 8)
       {
@@ -272,9 +287,8 @@ __global__ void __launch_bounds__(kOpThreads) prefill_operands_kernel(const Pref
       const int tk = e >> 6, c = 2 * (e & 63);
       uint32_t kb = 0;
       if (tk < rres) kb = *reinterpret_cast<const uint32_t *>(rk + tk * kHeadDim + c);
-      const uint32_t ko = tc05::sw128_offset(dpage * 16 + tk, c, 64);
-      sts32(sKh + ko, kb);
-      sts32(sKl + ko, 0u);
+      sts32(sK + tc05::sw128_offset(dpage * 16 + tk, c, 2 * kKeyTile), kb);
+      sts32(sK + tc05::sw128_offset(kKeyTile + dpage * 16 + tk, c, 2 * kKeyTile), 0u);
     }
     for (int e = widx; e < kPage * kHeadDim; e += 64) {
       const int tk = e >> 7, c = e & 127;
@@ -301,14 +315,14 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(const PrefillPara
   const uint32_t bars = base + kOffBar;
   const uint32_t tslot = base + kOffSlot;
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem_raw + (base + kOffAbort - raw));
-  auto stage = [&](int s) { return base + kOffStage + s * kStageBytes; };
-  auto pbuf = [&](int s) { return base + kOffP + s * kPBytes; };
-  auto stage_full = [&](int s) { return bars + 8u * (0 + s); };
-  auto stage_empty = [&](int s) { return bars + 8u * (3 + s); };
-  auto s_full = [&](int s) { return bars + 8u * (6 + s); };
-  auto s_empty = [&](int s) { return bars + 8u * (8 + s); };
-  auto p_full = [&](int s) { return bars + 8u * (10 + s); };
-  auto p_empty = [&](int s) { return bars + 8u * (12 + s); };
+  auto kbuf = [&](int s) { return base + kOffK + s * kKBytes; };
+  auto vbuf = [&](int s) { return base + kOffV + s * kVBytes; };
+  auto k_full = [&](int s) { return bars + 8u * (0 + s); };
+  auto k_empty = [&](int s) { return bars + 8u * (2 + s); };
+  auto v_full = [&](int s) { return bars + 8u * (4 + s); };
+  auto v_empty = [&](int s) { return bars + 8u * (6 + s); };
+  const uint32_t s_full = bars + 8u * 8, s_empty = bars + 8u * 9;
+  const uint32_t p_full = bars + 8u * 10, p_empty = bars + 8u * 11;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int G = p.group, H = p.num_kv_heads;
@@ -328,7 +342,7 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(const PrefillPara
   const int n_keys = pos_first + tq;                         // keys 0 .. pos_last
   const int n_ktiles = (n_keys + kKeyTile - 1) / kKeyTile;
 
-  // ---- setup: tensor memory, barriers, Q, the ones rows of every stage
+  // ---- setup: tensor memory, barriers, Q
   if (warp == 0) {
     tc05::tmem_alloc(tslot, kTmemCols);
     tc05::tmem_relinquish();
@@ -336,15 +350,15 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(const PrefillPara
   }
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(stage_full(s), 1);
-      mbar_init(stage_empty(s), 1);
+      mbar_init(k_full(s), 1);
+      mbar_init(k_empty(s), 1);
+      mbar_init(v_full(s), 1);
+      mbar_init(v_empty(s), 1);
     }
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(s_full(s), 1);
-      mbar_init(s_empty(s), 32 * kSoftmaxWarps);
-      mbar_init(p_full(s), 32 * kSoftmaxWarps);
-      mbar_init(p_empty(s), 1);
-    }
+    mbar_init(s_full, 1);
+    mbar_init(s_empty, 32 * kSoftmaxWarps);
+    mbar_init(p_full, 32 * kSoftmaxWarps);
+    mbar_init(p_empty, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -358,16 +372,11 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(const PrefillPara
                     p.q + (static_cast<long>(c_lo + t0 + tl) * p.num_q_heads + h * G + g) * kHeadDim) + c);
     sts128(sQ + tc05::sw128_offset(r, 8 * c, 128), v);
   }
-  for (int i = tid; i < kStages * static_cast<int>(kOnesBytes / 16); i += kThreadsP) {
-    const int s = i / (kOnesBytes / 16), c = i - s * (kOnesBytes / 16);
-    sts128(stage(s) + kTileBytes + 16 * c, make_uint4(0x3C003C00u, 0x3C003C00u, 0x3C003C00u, 0x3C003C00u));
-  }
   fence_proxy_async();
   __syncthreads();
   tc05::fence_after_sync();
   const uint32_t tmem = lds32_at(tslot);
-  const uint32_t tO = tmem + 128;
-  auto tS = [&](int s) { return tmem + 64u * s; };
+  const uint32_t tS = tmem + kColS, tO = tmem + kColO, tP = tmem + kColP;
   bool failed = false;
   auto fail = [&]() {
     failed = true;
@@ -376,65 +385,72 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(const PrefillPara
 
   if (warp == kProducerWarp) {
     // ---------------------------------------------------------- producer
+    // K(kt) into K buffer kt % 2 once S(kt - 2) has read it; V(kt) into V
+    // buffer kt % 2 once O += P(kt - 2) V(kt - 2) has
     if (lane == 0) {
       const uint8_t *tiles = p.ws + (static_cast<long long>(b) * H + h) * p.tiles_per_seq * kTileBytes;
       int issued = 0;
       for (int kt = 0; kt < n_ktiles; ++kt) {
         const int s = kt % kStages, u = kt / kStages;
-        if (kt >= kStages && !wait_bounded(stage_empty(s), (u - 1) & 1, abort_flag)) {
+        const uint8_t *src = tiles + static_cast<long long>(kt) * kTileBytes;
+        if (kt >= kStages && !wait_bounded(k_empty(s), (u - 1) & 1, abort_flag)) {
           fail();
           break;
         }
-        ++issued;
-        mbar_arrive_expect_tx(stage_full(s), kTileBytes);
-        bulk_copy_g2s(stage(s), tiles + static_cast<long long>(kt) * kTileBytes, kTileBytes, stage_full(s));
+        mbar_arrive_expect_tx(k_full(s), kKBytes);
+        bulk_copy_g2s(kbuf(s), src, kKBytes, k_full(s));
+        issued = 2 * kt + 1;
+        if (kt >= kStages && !wait_bounded(v_empty(s), (u - 1) & 1, abort_flag)) {
+          fail();
+          break;
+        }
+        mbar_arrive_expect_tx(v_full(s), kVBytes);
+        bulk_copy_g2s(vbuf(s), src + kKBytes, kVBytes, v_full(s));
+        issued = 2 * kt + 2;
       }
       // before the CTA exits, the copies in flight must have landed (bounded
-      // by time only, also after an abort)
-      const volatile int no_abort = 0;
-      for (int kt = max(0, issued - kStages); kt < issued; ++kt)
-        wait_bounded(stage_full(kt % kStages), (kt / kStages) & 1, &no_abort);
+      // by time only, also after an abort): at most the last kStages of each
+      // kind can still be in flight
+      for (int c = max(0, issued - 2 * kStages); c < issued; ++c) {
+        const int kt = c >> 1, s = kt % kStages;
+        wait_landed((c & 1) ? v_full(s) : k_full(s), (kt / kStages) & 1);
+      }
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      auto issue_pv = [&](int k) {  // O += P(k) [V(k) | 1]
-        const int ps = k & 1, vs = k % kStages;
-        if (!wait_bounded(p_full(ps), (k >> 1) & 1, abort_flag)) return false;
+      auto issue_pv = [&](int k) {  // O += P(k) V(k), P read from tensor memory
+        const int vs = k % kStages;
+        if (!wait_bounded(v_full(vs), (k / kStages) & 1, abort_flag) || !wait_bounded(p_full, k & 1, abort_flag))
+          return false;
         tc05::fence_after_sync();
-        const uint32_t sv = stage(vs) + 2 * kKBytes;
 #pragma unroll
-        for (int j = 0; j < 4; ++j)
-          tc05::mma_f16_ss(tO, tc05::smem_desc_sw128(pbuf(ps) + 32 * j), tc05::smem_desc_sw128(sv + 32 * j), kIdescO,
-                           (k > 0 || j > 0) ? 1u : 0u);
-        tc05::mma_commit(p_empty(ps));
-        tc05::mma_commit(stage_empty(vs));
+        for (int j = 0; j < kKeyTile / 16; ++j)
+          tc05::mma_f16_ts(tO, tP + 8 * j, tc05::smem_desc_sw128(vbuf(vs) + (j >> 2) * (kVBytes / 2) + (j & 3) * 32),
+                           kIdescO, (k > 0 || j > 0) ? 1u : 0u);
+        tc05::mma_commit(p_empty);
+        tc05::mma_commit(v_empty(vs));
         return true;
       };
       for (int kt = 0; kt < n_ktiles; ++kt) {
-        const int s3 = kt % kStages, ss = kt & 1;
-        if (!wait_bounded(stage_full(s3), (kt / kStages) & 1, abort_flag) ||
-            (kt >= 2 && !wait_bounded(s_empty(ss), ((kt >> 1) - 1) & 1, abort_flag))) {
+        const int ks = kt % kStages;
+        // S(kt) = Q [K_hi; K_lo]^T once K(kt) has landed and the softmax has
+        // read S(kt - 1)
+        if (!wait_bounded(k_full(ks), (kt / kStages) & 1, abort_flag) ||
+            (kt >= 1 && !wait_bounded(s_empty, (kt - 1) & 1, abort_flag))) {
           fail();
           break;
         }
         tc05::fence_after_sync();
-        // S(kt) = Q K_hi^T + Q K_lo^T
-        const uint32_t skh = stage(s3), skl = stage(s3) + kKBytes;
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           const uint32_t qo = (j >> 2) * (kQBytes / 2) + (j & 3) * 32;
           const uint32_t ko = (j >> 2) * (kKBytes / 2) + (j & 3) * 32;
-          tc05::mma_f16_ss(tS(ss), tc05::smem_desc_sw128(sQ + qo), tc05::smem_desc_sw128(skh + ko), kIdescS,
+          tc05::mma_f16_ss(tS, tc05::smem_desc_sw128(sQ + qo), tc05::smem_desc_sw128(kbuf(ks) + ko), kIdescS,
                            j > 0 ? 1u : 0u);
         }
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const uint32_t qo = (j >> 2) * (kQBytes / 2) + (j & 3) * 32;
-          const uint32_t ko = (j >> 2) * (kKBytes / 2) + (j & 3) * 32;
-          tc05::mma_f16_ss(tS(ss), tc05::smem_desc_sw128(sQ + qo), tc05::smem_desc_sw128(skl + ko), kIdescS, 1u);
-        }
-        tc05::mma_commit(s_full(ss));
+        tc05::mma_commit(s_full);
+        tc05::mma_commit(k_empty(ks));
         // O += P(kt-1) V(kt-1) while the softmax of kt runs
         if (kt >= 1 && !issue_pv(kt - 1)) {
           fail();
@@ -450,6 +466,7 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(const PrefillPara
     const bool row_ok = row < rows;
     const int pos_row = pos_first + (row_ok ? row / G : 0);
     float ref = -INFINITY;
+    float2 lsum = make_float2(0.f, 0.f);
     const float sl2 = p.scale_log2;
     // the warp takes every decision together (its lanes run warp-wide
     // tensor-memory loads and votes)
@@ -457,109 +474,109 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(const PrefillPara
       return __all_sync(0xFFFFFFFFu, wait_bounded(bar, parity, abort_flag));
     };
     for (int kt = 0; kt < n_ktiles; ++kt) {
-      const int ss = kt & 1;
-      if (!wait_warp(s_full(ss), (kt >> 1) & 1)) {
+      if (!wait_warp(s_full, kt & 1)) {
         fail();
         break;
       }
       tc05::fence_after_sync();
-      uint32_t v[64];
-      {
-        uint32_t (&v0)[32] = *reinterpret_cast<uint32_t (*)[32]>(&v[0]);
-        uint32_t (&v1)[32] = *reinterpret_cast<uint32_t (*)[32]>(&v[32]);
-        tc05::tmem_ld32(tS(ss) + lane_base, v0);
-        tc05::tmem_ld32(tS(ss) + lane_base + 32, v1);
+      // S = S_hi + S_lo for the tile's 128 keys
+      float sv[kKeyTile];
+#pragma unroll
+      for (int c = 0; c < kKeyTile / 32; ++c) {
+        uint32_t hi[32], lo[32];
+        tc05::tmem_ld32(tS + lane_base + 32 * c, hi);
+        tc05::tmem_ld32(tS + lane_base + kKeyTile + 32 * c, lo);
         tc05::tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 32; j += 2) {
+          const float2 x = add2(make_float2(__uint_as_float(hi[j]), __uint_as_float(hi[j + 1])),
+                                make_float2(__uint_as_float(lo[j]), __uint_as_float(lo[j + 1])));
+          sv[32 * c + j] = x.x;
+          sv[32 * c + j + 1] = x.y;
+        }
       }
       tc05::fence_before_sync();
-      mbar_arrive(s_empty(ss));
+      mbar_arrive(s_empty);
       // a key tile wholly before the tile's first query position needs no
       // mask (rows past the last row hold q = 0: finite logits, never written)
       const int key0 = kt * kKeyTile;
       const bool full = key0 + kKeyTile - 1 <= pos_first;
-      float mx = -INFINITY;
+      float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
       if (full) {
 #pragma unroll
-        for (int j = 0; j < 64; ++j) mx = fmaxf(mx, __uint_as_float(v[j]));
+        for (int j = 0; j < kKeyTile; ++j) m4[j & 3] = fmaxf(m4[j & 3], sv[j]);
       } else {
 #pragma unroll
-        for (int j = 0; j < 64; ++j) {
+        for (int j = 0; j < kKeyTile; ++j) {
           const bool ok = row_ok && key0 + j <= pos_row;
-          const float x = ok ? __uint_as_float(v[j]) : -INFINITY;
-          v[j] = __float_as_uint(x);
-          mx = fmaxf(mx, x);
+          sv[j] = ok ? sv[j] : -INFINITY;
+          m4[j & 3] = fmaxf(m4[j & 3], sv[j]);
         }
       }
-      mx *= sl2;
+      const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * sl2;
       // the reference moves only when the row maximum passes it by > 8
       const bool move = mx > ref + kSlack;
       const float new_ref = move ? mx : ref;
       const float alpha = move ? fast_exp2(ref - new_ref) : 1.0f;  // 0 when ref was -inf
-      // weights exp2(s * scale - ref) in registers; masked logits are -inf
-      // and give 0 (a row without a valid key keeps a -inf reference,
-      // replaced by 0 so that no inf - inf appears)
+      // weights exp2(s * scale - ref); masked logits are -inf and give 0 (a
+      // row without a valid key keeps a -inf reference, replaced by 0 so that
+      // no inf - inf appears).  The row sum takes the fp16 weights the MMA
+      // multiplies with.
       const float nref = new_ref == -INFINITY ? 0.f : -new_ref;
       const float2 sc = make_float2(sl2, sl2), nr = make_float2(nref, nref);
-      uint32_t hp[32];
+      uint32_t hp[kKeyTile / 2];
+      float2 ts0 = make_float2(0.f, 0.f), ts1 = make_float2(0.f, 0.f);
 #pragma unroll
-      for (int j = 0; j < 64; j += 2) {
-        const float2 x = fma2(make_float2(__uint_as_float(v[j]), __uint_as_float(v[j + 1])), sc, nr);
-        hp[j >> 1] = h2_as_u32(__floats2half2_rn(fast_exp2(x.x), fast_exp2(x.y)));
+      for (int j = 0; j < kKeyTile; j += 2) {
+        const float2 x = fma2(make_float2(sv[j], sv[j + 1]), sc, nr);
+        const __half2 ph = __floats2half2_rn(fast_exp2(x.x), fast_exp2(x.y));
+        if (j & 2) ts1 = add2(ts1, __half22float2(ph));
+        else ts0 = add2(ts0, __half22float2(ph));
+        hp[j >> 1] = h2_as_u32(ph);
       }
-      // a moved reference rescales O and its sum column once O += P(kt-1) V
-      // has completed (P(kt) is not yet handed over, so O is idle)
-      if (kt >= 1 && __any_sync(0xFFFFFFFFu, move)) {
-        if (!wait_warp(p_empty((kt - 1) & 1), ((kt - 1) >> 1) & 1)) {
+      lsum = add2(mul2(lsum, make_float2(alpha, alpha)), add2(ts0, ts1));
+      // O and P are idle once O += P(kt-1) V has completed
+      if (kt >= 1) {
+        if (!wait_warp(p_empty, (kt - 1) & 1)) {
           fail();
           break;
         }
         tc05::fence_after_sync();
-        const float2 a2 = make_float2(alpha, alpha);
+        // a moved reference rescales O
+        if (__any_sync(0xFFFFFFFFu, move)) {
+          const float2 a2 = make_float2(alpha, alpha);
 #pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          uint32_t o[32];
-          tc05::tmem_ld32(tO + lane_base + 32 * c, o);
-          tc05::tmem_wait_ld();
+          for (int c = 0; c < 4; ++c) {
+            uint32_t o[32];
+            tc05::tmem_ld32(tO + lane_base + 32 * c, o);
+            tc05::tmem_wait_ld();
 #pragma unroll
-          for (int j = 0; j < 32; j += 2) {
-            const float2 r = mul2(make_float2(__uint_as_float(o[j]), __uint_as_float(o[j + 1])), a2);
-            o[j] = __float_as_uint(r.x);
-            o[j + 1] = __float_as_uint(r.y);
+            for (int j = 0; j < 32; j += 2) {
+              const float2 r = mul2(make_float2(__uint_as_float(o[j]), __uint_as_float(o[j + 1])), a2);
+              o[j] = __float_as_uint(r.x);
+              o[j + 1] = __float_as_uint(r.y);
+            }
+            tc05::tmem_st32(tO + lane_base + 32 * c, o);
           }
-          tc05::tmem_st32(tO + lane_base + 32 * c, o);
         }
-        {
-          uint32_t o[16];
-          tc05::tmem_ld16(tO + lane_base + 128, o);
-          tc05::tmem_wait_ld();
-#pragma unroll
-          for (int j = 0; j < 16; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
-          tc05::tmem_st16(tO + lane_base + 128, o);
-        }
-        tc05::tmem_wait_st();
       }
       ref = new_ref;
-      // P buffer ss is free once O += P(kt-2) V has completed
-      if (kt >= 2 && !wait_warp(p_empty(ss), ((kt >> 1) - 1) & 1)) {
-        fail();
-        break;
+      // P into tensor memory (fp16 pairs, the A operand of O += P V)
+      {
+        uint32_t (&h0)[32] = *reinterpret_cast<uint32_t (*)[32]>(&hp[0]);
+        uint32_t (&h1)[32] = *reinterpret_cast<uint32_t (*)[32]>(&hp[32]);
+        tc05::tmem_st32(tP + lane_base, h0);
+        tc05::tmem_st32(tP + lane_base + 32, h1);
       }
-#pragma unroll
-      for (int q8 = 0; q8 < 8; ++q8)
-        sts128(pbuf(ss) + tc05::sw128_offset(row, 8 * q8, 128),
-               make_uint4(hp[4 * q8], hp[4 * q8 + 1], hp[4 * q8 + 2], hp[4 * q8 + 3]));
-      fence_proxy_async();
+      tc05::tmem_wait_st();
       tc05::fence_before_sync();
-      mbar_arrive(p_full(ss));
+      mbar_arrive(p_full);
     }
     // ---- out = O / l once the last O += P V has completed
-    if (!failed && !wait_warp(p_empty((n_ktiles - 1) & 1), ((n_ktiles - 1) >> 1) & 1)) fail();
+    if (!failed && !wait_warp(p_empty, (n_ktiles - 1) & 1)) fail();
     if (!failed) {
       tc05::fence_after_sync();
-      uint32_t ls[16];
-      tc05::tmem_ld16(tO + lane_base + 128, ls);
-      tc05::tmem_wait_ld();
-      const float l = __uint_as_float(ls[0]);
+      const float l = lsum.x + lsum.y;
       const float inv = row_ok && l > 0.f ? 1.0f / l : 0.f;
       const int tl = row / G, g = row - (row / G) * G;
       __half *dst = p.out + (static_cast<long>(c_lo + t0 + tl) * p.num_q_heads + h * G + g) * kHeadDim;
@@ -593,6 +610,9 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(const PrefillPara
 
 size_t prefill_smem_bytes() { return kSmemBytes; }
 size_t prefill_tile_bytes() { return kTileBytes; }
+int prefill_tiles_per_seq(int max_pages) {
+  return static_cast<int>((static_cast<long long>(max_pages) + kPagesPerTile - 1) / kPagesPerTile);
+}
 
 cudaError_t prepare_prefill_kernel() {
   cudaError_t e = cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,

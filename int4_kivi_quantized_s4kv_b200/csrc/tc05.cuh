@@ -1,6 +1,6 @@
 // Thin wrappers over the sm_100a fifth-generation tensor-core instructions
 // (tcgen05.*) used by the prefill kernel: tensor-memory allocation, the
-// single-thread MMA with both operands in shared memory, its completion
+// single-thread MMA (A in shared or tensor memory, B in shared memory), its completion
 // signal on an mbarrier, and the warp-wide tensor-memory loads and stores.
 //
 // Shared-memory operands use the 128-byte-swizzled K-major canonical layout:
@@ -68,6 +68,18 @@ __device__ __forceinline__ void mma_f16_ss(uint32_t d_tmem, uint64_t a_desc, uin
       "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// D[tmem] (+)= A[tmem] . B[smem]^T, issued by one thread.  A (M = 128 rows,
+// K = 16) sits in tensor memory: row r in lane r, elements 2c and 2c + 1 of
+// the row packed in column c (the low half holds the lower k).
+__device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                           uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
 

@@ -119,10 +119,11 @@ def test_invalid_calls_rejected_before_launch(S):
     assert call(args(maxnew=5)) == S.ERR_INVALID_ARG  # more than n_tokens
     assert call(args(batch=5)) == S.ERR_INVALID_ARG   # batch > max_seqs
     assert call(args(n=0)) == S.OK and call(args(batch=0)) == S.OK  # nothing to do
-    # workspace: 48 KB per 64-key tile per (sequence slot, kv head)
-    assert S.prefill_workspace_bytes(2, 1, 1) == 2 * 49152
-    assert S.prefill_workspace_bytes(8, 4, 512) == 4 * 8 * 128 * 49152
-    assert S.prefill_workspace_bytes(1, 1, 5) == 2 * 49152  # 5 pages round up to 2 tiles
+    # workspace: 96 KB per 128-key tile (8 pages) per (sequence slot, kv head)
+    tile = 2 * 2 * 128 * 128 + 2 * 128 * 128  # [K_hi; K_lo] and V^T, fp16
+    assert S.prefill_workspace_bytes(2, 1, 1) == 2 * tile
+    assert S.prefill_workspace_bytes(8, 4, 512) == 4 * 8 * 64 * tile
+    assert S.prefill_workspace_bytes(1, 1, 9) == 2 * tile  # 9 pages round up to 2 tiles
     n = ctypes.c_size_t(0)
     assert L.s4kv_prefill_workspace_size(0, 1, 1, ctypes.byref(n)) == S.ERR_INVALID_ARG
     assert L.s4kv_prefill_workspace_size(1, 1, 0, ctypes.byref(n)) == S.ERR_INVALID_ARG
@@ -130,7 +131,7 @@ def test_invalid_calls_rejected_before_launch(S):
     assert L.s4kv_prefill_workspace_size(65535, 65535, 1 << 30, ctypes.byref(n)) == S.ERR_INVALID_ARG
     assert call(args(ws=None)) == S.ERR_WORKSPACE
     assert call(args(ws=P(fake + 8))) == S.ERR_WORKSPACE  # not 16-B aligned
-    assert call(args(wsb=2 * 49152 - 1)) == S.ERR_WORKSPACE
+    assert call(args(wsb=2 * tile - 1)) == S.ERR_WORKSPACE
     # dequant
     assert L.s4kv_dequant_page(ctypes.byref(c), 10, P(fake), P(fake), 1, st) == S.ERR_INVALID_ARG
     assert L.s4kv_dequant_page(ctypes.byref(c), -1, P(fake), P(fake), 1, st) == S.ERR_INVALID_ARG
