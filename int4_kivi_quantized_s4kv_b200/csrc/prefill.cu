@@ -16,7 +16,7 @@
 //  1. prefill_operands_kernel dequantizes every key tile (128 keys, 8 pages)
 //     of every (sequence, kv head) ONCE into a workspace tile of 96 KB that
 //     holds the MMA operands exactly as shared memory wants them (128-byte
-//     swizzled, K-major): [K_hi; K_lo] and V^T.  A key is code * scale + zero
+//     swizzled, K-major): K_hi, K_lo and V^T.  A key is code * scale + zero
 //     in fp32 (exact product, one rounding, the value the oracle's
 //     dequantization gives) split into an fp16 hi part and the fp16 rounding
 //     of the remainder, so K_hi + K_lo carries it to about 22 bits (keys of
@@ -29,18 +29,19 @@
 //     tile's 128 MMA rows are (token, head of the group) pairs, so a tile
 //     holds floor(128 / G) tokens.  Warps with separate roles hand buffers
 //     over through mbarriers:
-//      * a producer warp brings each key tile's [K_hi; K_lo] (64 KB) and V^T
+//      * a producer warp brings each key tile's K_hi, K_lo (64 KB) and V^T
 //        (32 KB) into one of two K and one of two V buffers with 1-D bulk
 //        copies (TMA engine, no multicast); a K buffer is refilled as soon as
 //        the S MMAs that read it complete, a V buffer once the PV MMAs have;
-//      * one thread issues S(k) = Q [K_hi; K_lo]^T (M = 128, N = 256: the hi
-//        and lo rows of the 128 keys stacked, so one MMA instruction per
-//        16 channels covers both) into tensor memory, then
+//      * one thread issues S(k) = Q K_hi^T + Q K_lo^T (M = 128, N = 128 keys,
+//        one accumulation over K = 256: the 128 channels against K_hi, then
+//        against K_lo) into one of two tensor-memory S buffers, then
 //        O += P(k-1) V(k-1) (N = 128, K = 128) with P read from tensor
 //        memory.  Few, large MMA instructions keep the single issuing thread
-//        ahead of the tensor core;
+//        ahead of the tensor core, and with two S buffers S(k+1) never waits
+//        for the softmax to have read S(k);
 //      * 4 softmax warps (one tensor-memory lane, i.e. one row, per thread)
-//        read S_hi + S_lo back, apply the causal mask and an online softmax
+//        read S back, apply the causal mask and an online softmax
 //        in the exp2 domain whose reference moves only when a row maximum
 //        passes it by more than 8 (weights stay <= 256, fine for fp16),
 //        rescale that row of O in tensor memory when it moves, and write P
@@ -65,16 +66,17 @@ constexpr int kPagesPerTile = kKeyTile / kPage;  // 8
 constexpr int kOpThreads = 64 * kPagesPerTile;   // operand kernel: 64 threads per page
 constexpr int kStages = 2;                       // K and V buffers each
 constexpr uint32_t kQBytes = 128 * 128 * 2;      // Q [128][128] fp16
-constexpr uint32_t kKBytes = 2 * kKeyTile * 128 * 2;   // [K_hi; K_lo] [256][128] fp16
+constexpr uint32_t kKBytes = 2 * kKeyTile * 128 * 2;   // K_hi, K_lo [128][128] fp16 each
 constexpr uint32_t kVBytes = 128 * kKeyTile * 2;       // V^T [128][128] fp16
 constexpr uint32_t kTileBytes = kKBytes + kVBytes;     // workspace tile
 constexpr uint32_t kStagingBytes = kPagesPerTile * kBlockBytes;
 constexpr float kSlack = 8.0f;                   // log2 slack of the softmax reference
 constexpr long long kWaitLimit = 2000000000LL;   // about one second
-// S: M = 128, N = 256 (K_hi and K_lo rows stacked); PV: M = 128, N = 128
-constexpr uint32_t kIdescS = tc05::idesc_f16_f32(128, 2 * kKeyTile);
+// S: M = 128, N = 128 keys, K = 256 (Q against K_hi, then Q against K_lo,
+// accumulated); PV: M = 128, N = 128
+constexpr uint32_t kIdescS = tc05::idesc_f16_f32(128, kKeyTile);
 constexpr uint32_t kIdescO = tc05::idesc_f16_f32(128, 128);
-// tensor memory (512 columns): S_hi at 0, S_lo at 128, O at 256, P (fp16
+// tensor memory (512 columns): two S buffers at 0 and 128, O at 256, P (fp16
 // pairs, the PV A operand) at 384
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0, kColO = 256, kColP = 384;
@@ -86,9 +88,9 @@ constexpr uint32_t kOffK = kOffQ + kQBytes;                      // [2]
 constexpr uint32_t kOffV = kOffK + kStages * kKBytes;            // [2]
 constexpr uint32_t kOffBar = kOffV + kStages * kVBytes;
 // barriers (8 bytes each): k_full[2], k_empty[2], v_full[2], v_empty[2],
-// s_full, s_empty, p_full, p_empty; then the tensor-memory address and the
-// abort flag
-constexpr uint32_t kNumBars = 12;
+// s_full[2], s_empty[2], p_full, p_empty; then the tensor-memory address and
+// the abort flag
+constexpr uint32_t kNumBars = 14;
 constexpr uint32_t kOffSlot = kOffBar + 8 * kNumBars;
 constexpr uint32_t kOffAbort = kOffSlot + 4;
 constexpr uint32_t kSmemBytes = kOffAbort + 4 + 1024;  // + alignment slack
@@ -149,6 +151,14 @@ __device__ __forceinline__ uint2 lds64_at(uint32_t addr) {
   return v;
 }
 
+// max of three floats in one instruction (sm_100); a NaN operand is ignored
+// as by fmaxf
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 __device__ __forceinline__ uint32_t hfma2_u32(uint32_t a, uint32_t b, uint32_t c) {
   return h2_as_u32(__hfma2(u32_as_h2(a), u32_as_h2(b), u32_as_h2(c)));
 }
@@ -187,9 +197,8 @@ __device__ __forceinline__ bool seq_rows(const PrefillParams &p, int b, bool fla
 
 // ---------------------------------------------------------------------------
 // Launch 1: one CTA per (key tile, sequence, kv head) writes the tile's
-// operands to the workspace: [K_hi; K_lo] as one [256][128] operand (rows
-// 0..127 the hi parts of keys 0..127, rows 128..255 their lo parts) and V^T
-// [128][128], both 128-byte swizzled K-major.  Keys at or past L (the rest of
+// operands to the workspace: K_hi, K_lo and V^T, each [128][128] fp16 and
+// 128-byte swizzled K-major.  Keys at or past L (the rest of
 // the partial last page, pages after it) are written as zeros, so masked
 // keys hold finite values.
 __global__ void __launch_bounds__(kOpThreads) prefill_operands_kernel(const PrefillParams p) {
@@ -251,13 +260,11 @@ __global__ void __launch_bounds__(kOpThreads) prefill_operands_kernel(const Pref
         split_key(a1, s01, zf01, hi1, lo1);
         split_key(a2, s23, zf23, hi2, lo2);
         split_key(a3, s23, zf23, hi3, lo3);
-        const int key = dpage * 16 + dn;
-        const uint32_t kh = tc05::sw128_offset(key, c0, 2 * kKeyTile);
-        const uint32_t kl = tc05::sw128_offset(kKeyTile + key, c0, 2 * kKeyTile);
-        sts64(sK + kh, hi0, hi2);
-        sts64(sK + kh + 1024, hi1, hi3);
-        sts64(sK + kl, lo0, lo2);
-        sts64(sK + kl + 1024, lo1, lo3);
+        const uint32_t ko = tc05::sw128_offset(dpage * 16 + dn, c0, kKeyTile);
+        sts64(sK + ko, hi0, hi2);
+        sts64(sK + ko + 1024, hi1, hi3);
+        sts64(sK + kKBytes / 2 + ko, lo0, lo2);
+        sts64(sK + kKBytes / 2 + ko + 1024, lo1, lo3);
       }
       // values: channels cb, cb + 1; tokens 2 di, 2 di + 1 (+ 8)
       {
@@ -287,8 +294,9 @@ __global__ void __launch_bounds__(kOpThreads) prefill_operands_kernel(const Pref
       const int tk = e >> 6, c = 2 * (e & 63);
       uint32_t kb = 0;
       if (tk < rres) kb = *reinterpret_cast<const uint32_t *>(rk + tk * kHeadDim + c);
-      sts32(sK + tc05::sw128_offset(dpage * 16 + tk, c, 2 * kKeyTile), kb);
-      sts32(sK + tc05::sw128_offset(kKeyTile + dpage * 16 + tk, c, 2 * kKeyTile), 0u);
+      const uint32_t ko = tc05::sw128_offset(dpage * 16 + tk, c, kKeyTile);
+      sts32(sK + ko, kb);
+      sts32(sK + kKBytes / 2 + ko, 0u);
     }
     for (int e = widx; e < kPage * kHeadDim; e += 64) {
       const int tk = e >> 7, c = e & 127;
@@ -321,8 +329,9 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(const PrefillPara
   auto k_empty = [&](int s) { return bars + 8u * (2 + s); };
   auto v_full = [&](int s) { return bars + 8u * (4 + s); };
   auto v_empty = [&](int s) { return bars + 8u * (6 + s); };
-  const uint32_t s_full = bars + 8u * 8, s_empty = bars + 8u * 9;
-  const uint32_t p_full = bars + 8u * 10, p_empty = bars + 8u * 11;
+  auto s_full = [&](int s) { return bars + 8u * (8 + s); };
+  auto s_empty = [&](int s) { return bars + 8u * (10 + s); };
+  const uint32_t p_full = bars + 8u * 12, p_empty = bars + 8u * 13;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int G = p.group, H = p.num_kv_heads;
@@ -355,8 +364,10 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(const PrefillPara
       mbar_init(v_full(s), 1);
       mbar_init(v_empty(s), 1);
     }
-    mbar_init(s_full, 1);
-    mbar_init(s_empty, 32 * kSoftmaxWarps);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(s_full(s), 1);
+      mbar_init(s_empty(s), 32 * kSoftmaxWarps);
+    }
     mbar_init(p_full, 32 * kSoftmaxWarps);
     mbar_init(p_empty, 1);
     *abort_flag = 0;
@@ -376,7 +387,8 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(const PrefillPara
   __syncthreads();
   tc05::fence_after_sync();
   const uint32_t tmem = lds32_at(tslot);
-  const uint32_t tS = tmem + kColS, tO = tmem + kColO, tP = tmem + kColP;
+  auto tS = [&](int s) { return tmem + kColS + 128u * s; };
+  const uint32_t tO = tmem + kColO, tP = tmem + kColP;
   bool failed = false;
   auto fail = [&]() {
     failed = true;
@@ -434,22 +446,23 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(const PrefillPara
       };
       for (int kt = 0; kt < n_ktiles; ++kt) {
         const int ks = kt % kStages;
-        // S(kt) = Q [K_hi; K_lo]^T once K(kt) has landed and the softmax has
-        // read S(kt - 1)
+        // S(kt) = Q K_hi^T + Q K_lo^T into S buffer kt % 2 once K(kt) has
+        // landed and the softmax has read S(kt - 2) from that buffer
+        const int sb = kt & 1;
         if (!wait_bounded(k_full(ks), (kt / kStages) & 1, abort_flag) ||
-            (kt >= 1 && !wait_bounded(s_empty, (kt - 1) & 1, abort_flag))) {
+            (kt >= 2 && !wait_bounded(s_empty(sb), ((kt >> 1) - 1) & 1, abort_flag))) {
           fail();
           break;
         }
         tc05::fence_after_sync();
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const uint32_t qo = (j >> 2) * (kQBytes / 2) + (j & 3) * 32;
-          const uint32_t ko = (j >> 2) * (kKBytes / 2) + (j & 3) * 32;
-          tc05::mma_f16_ss(tS, tc05::smem_desc_sw128(sQ + qo), tc05::smem_desc_sw128(kbuf(ks) + ko), kIdescS,
+        for (int j = 0; j < 16; ++j) {
+          const uint32_t qo = ((j >> 2) & 1) * (kQBytes / 2) + (j & 3) * 32;
+          const uint32_t ko = (j >> 3) * (kKBytes / 2) + ((j >> 2) & 1) * (kKBytes / 4) + (j & 3) * 32;
+          tc05::mma_f16_ss(tS(sb), tc05::smem_desc_sw128(sQ + qo), tc05::smem_desc_sw128(kbuf(ks) + ko), kIdescS,
                            j > 0 ? 1u : 0u);
         }
-        tc05::mma_commit(s_full);
+        tc05::mma_commit(s_full(sb));
         tc05::mma_commit(k_empty(ks));
         // O += P(kt-1) V(kt-1) while the softmax of kt runs
         if (kt >= 1 && !issue_pv(kt - 1)) {
@@ -474,45 +487,33 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(const PrefillPara
       return __all_sync(0xFFFFFFFFu, wait_bounded(bar, parity, abort_flag));
     };
     for (int kt = 0; kt < n_ktiles; ++kt) {
-      if (!wait_warp(s_full, kt & 1)) {
+      const int sb = kt & 1;
+      if (!wait_warp(s_full(sb), (kt >> 1) & 1)) {
         fail();
         break;
       }
       tc05::fence_after_sync();
-      // S = S_hi + S_lo for the tile's 128 keys
-      float sv[kKeyTile];
+      uint32_t sv[kKeyTile];
 #pragma unroll
       for (int c = 0; c < kKeyTile / 32; ++c) {
-        uint32_t hi[32], lo[32];
-        tc05::tmem_ld32(tS + lane_base + 32 * c, hi);
-        tc05::tmem_ld32(tS + lane_base + kKeyTile + 32 * c, lo);
-        tc05::tmem_wait_ld();
-#pragma unroll
-        for (int j = 0; j < 32; j += 2) {
-          const float2 x = add2(make_float2(__uint_as_float(hi[j]), __uint_as_float(hi[j + 1])),
-                                make_float2(__uint_as_float(lo[j]), __uint_as_float(lo[j + 1])));
-          sv[32 * c + j] = x.x;
-          sv[32 * c + j + 1] = x.y;
-        }
+        uint32_t (&w)[32] = *reinterpret_cast<uint32_t (*)[32]>(&sv[32 * c]);
+        tc05::tmem_ld32(tS(sb) + lane_base + 32 * c, w);
       }
+      tc05::tmem_wait_ld();
       tc05::fence_before_sync();
-      mbar_arrive(s_empty);
+      mbar_arrive(s_empty(sb));
       // a key tile wholly before the tile's first query position needs no
       // mask (rows past the last row hold q = 0: finite logits, never written)
       const int key0 = kt * kKeyTile;
       const bool full = key0 + kKeyTile - 1 <= pos_first;
       float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-      if (full) {
+      if (!full) {
 #pragma unroll
-        for (int j = 0; j < kKeyTile; ++j) m4[j & 3] = fmaxf(m4[j & 3], sv[j]);
-      } else {
-#pragma unroll
-        for (int j = 0; j < kKeyTile; ++j) {
-          const bool ok = row_ok && key0 + j <= pos_row;
-          sv[j] = ok ? sv[j] : -INFINITY;
-          m4[j & 3] = fmaxf(m4[j & 3], sv[j]);
-        }
+        for (int j = 0; j < kKeyTile; ++j) sv[j] = (row_ok && key0 + j <= pos_row) ? sv[j] : __float_as_uint(-INFINITY);
       }
+#pragma unroll
+      for (int j = 0; j < kKeyTile; j += 2)
+        m4[(j >> 1) & 3] = fmax3(m4[(j >> 1) & 3], __uint_as_float(sv[j]), __uint_as_float(sv[j + 1]));
       const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * sl2;
       // the reference moves only when the row maximum passes it by > 8
       const bool move = mx > ref + kSlack;
@@ -520,19 +521,20 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(const PrefillPara
       const float alpha = move ? fast_exp2(ref - new_ref) : 1.0f;  // 0 when ref was -inf
       // weights exp2(s * scale - ref); masked logits are -inf and give 0 (a
       // row without a valid key keeps a -inf reference, replaced by 0 so that
-      // no inf - inf appears).  The row sum takes the fp16 weights the MMA
-      // multiplies with.
+      // no inf - inf appears).  The row sum adds the fp32 weights; their fp16
+      // roundings, which the MMA multiplies with, differ from them by
+      // independent errors below 2^-11 relative that average out in the sum.
       const float nref = new_ref == -INFINITY ? 0.f : -new_ref;
       const float2 sc = make_float2(sl2, sl2), nr = make_float2(nref, nref);
       uint32_t hp[kKeyTile / 2];
       float2 ts0 = make_float2(0.f, 0.f), ts1 = make_float2(0.f, 0.f);
 #pragma unroll
       for (int j = 0; j < kKeyTile; j += 2) {
-        const float2 x = fma2(make_float2(sv[j], sv[j + 1]), sc, nr);
-        const __half2 ph = __floats2half2_rn(fast_exp2(x.x), fast_exp2(x.y));
-        if (j & 2) ts1 = add2(ts1, __half22float2(ph));
-        else ts0 = add2(ts0, __half22float2(ph));
-        hp[j >> 1] = h2_as_u32(ph);
+        const float2 x = fma2(make_float2(__uint_as_float(sv[j]), __uint_as_float(sv[j + 1])), sc, nr);
+        const float2 e = make_float2(fast_exp2(x.x), fast_exp2(x.y));
+        if (j & 2) ts1 = add2(ts1, e);
+        else ts0 = add2(ts0, e);
+        hp[j >> 1] = h2_as_u32(__floats2half2_rn(e.x, e.y));
       }
       lsum = add2(mul2(lsum, make_float2(alpha, alpha)), add2(ts0, ts1));
       // O and P are idle once O += P(kt-1) V has completed
