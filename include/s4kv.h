@@ -289,8 +289,8 @@ S4KV_API int s4kv_decode_attention_noalloc(const s4kv_cache_t *cache, const void
  * tcgen05 tensor cores with those operands and the fp16 softmax weights
  * (fp32 accumulation), so results agree with exact attention to about fp16
  * precision of the values and the weights.  Allocates nothing; the attention
- * launch needs about 225 KB of shared memory per CTA.  4-bit codes only (2-
- * and 8-bit caches are refused with S4KV_ERR_UNSUPPORTED). */
+ * launch needs about 225 KB of shared memory per CTA.  Any code width of
+ * the cache (4, 8 or 2 bits): only the first launch reads the codes. */
 S4KV_API int s4kv_prefill_attention(const s4kv_cache_t *cache, const void *q,
                                     int num_q_heads, int n_tokens,
                                     const int32_t *cu_new, const int32_t *seq_lens,

@@ -9,6 +9,7 @@
 #include <mutex>
 
 #include "kernels.cuh"
+#include "prefill.cuh"
 
 
 
@@ -301,7 +302,6 @@ int s4kv_prefill_attention(const s4kv_cache_t *cache, const void *q, int num_q_h
                            void *workspace, size_t workspace_bytes, void *stream) {
   int rc = check_cache(cache);
   if (rc != S4KV_OK) return rc;
-  if (cache_bits(cache) != 4) return S4KV_ERR_UNSUPPORTED;
   rc = s4kv_check_model(cache->head_dim, cache->page_tokens, num_q_heads, cache->num_kv_heads);
   if (rc != S4KV_OK) return rc;
   if (n_tokens < 0 || batch < 0 || batch > cache->max_seqs || max_pages_per_seq <= 0) return S4KV_ERR_INVALID_ARG;
@@ -350,6 +350,7 @@ int s4kv_prefill_attention(const s4kv_cache_t *cache, const void *q, int num_q_h
   p.scale_log2 = static_cast<float>(static_cast<double>(sm_scale) * 1.4426950408889634);
   p.ws = static_cast<uint8_t *>(workspace);
   p.tiles_per_seq = prefill_tiles_per_seq(max_pages_per_seq);
+  p.bits = cache_bits(cache);
   launch_prefill(p, batch, max_new_per_seq, static_cast<cudaStream_t>(stream));
   if (cudaGetLastError() != cudaSuccess) return S4KV_ERR_CUDA;
   return S4KV_OK;

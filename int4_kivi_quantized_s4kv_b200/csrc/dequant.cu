@@ -1,29 +1,13 @@
 // s4kv_dequant_page / s4kv_dequant_pages device side: physical pages, all kv
 // heads, back to natural [token][channel] order (page i of a list goes to
 // output slot i).  x = code * scale + zero in fp32 (the
-// product of a 4- or 8-bit code and an fp16 scale is exact, so this is a
-// single rounding); the fp16 output is that fp32 value rounded to nearest
+// product of a code of at most 8 bits and an fp16 scale is exact, so this is
+// a single rounding); the fp16 output is that fp32 value rounded to nearest
 // even.
+#include "code_map.cuh"
 #include "kernels.cuh"
 
 namespace s4kv {
-
-// The code at 4-bit position (word, nibble): that nibble, or with 8-bit
-// codes the byte holding the same fragment place (tile 4*(word/128) +
-// word%4, lane (word/4)%32, register nibble%4, half nibble/4).
-__device__ __forceinline__ uint32_t code_at(const uint8_t *region, int word, int nibble, int bits) {
-  if (bits == 8) {
-    const int tile = 4 * (word >> 7) + (word & 3), lane = (word >> 2) & 31;
-    return region[((tile >> 1) * 32 + lane) * 16 + (tile & 1) * 8 + 2 * (nibble & 3) + (nibble >> 2)];
-  }
-  if (bits == 2) {
-    const int tile = 4 * (word >> 7) + (word & 3), lane = (word >> 2) & 31;
-    const uint32_t w = reinterpret_cast<const uint32_t *>(region)[4 * lane + (tile >> 1)];
-    return (w >> (16 * (nibble >> 2) + 2 * (4 * (tile & 1) + (nibble & 3)))) & 3u;
-  }
-  const uint32_t w = reinterpret_cast<const uint32_t *>(region)[word];
-  return (w >> (4 * nibble)) & 0xFu;
-}
 
 __global__ void __launch_bounds__(128) dequant_kernel(const DequantParams p) {
   const int h = blockIdx.x;
@@ -44,19 +28,12 @@ __global__ void __launch_bounds__(128) dequant_kernel(const DequantParams p) {
   const int vscale_off = kzero_off + 2 * kHeadDim, vzero_off = vscale_off + 2 * kPage * (kHeadDim / kVGroup);
   const uint8_t *blk = p.pool + (static_cast<long>(page) * p.num_kv_heads + h) * block_bytes_for(p.bits);
   const float ks = __half2float(reinterpret_cast<const __half *>(blk + kscale_off)[c]);
-  const int zslot = 16 * ((c & 31) >> 2) + 2 * (c >> 5) + (c & 1) + 8 * ((c & 3) >> 1);
-  const float kz = __half2float(reinterpret_cast<const __half *>(blk + kzero_off)[zslot]);
+  const float kz = __half2float(reinterpret_cast<const __half *>(blk + kzero_off)[key_zero_slot(c)]);
   const int g = c / kVGroup;
-  // key fragment coordinates of channel c: lane quarter i, tile kt, pair e
-  const int ki = c >> 5, kt = (c & 31) >> 2, ke = c & 3;
-  // value fragment coordinates of channel c: M-tile m, row group n
-  const int vn = (c & 31) >> 2, ve = c & 3, vm = 2 * g + (ve >> 1);
   for (int t = 0; t < kPage; ++t) {
-    const int kword = 128 * (kt >> 2) + 4 * (4 * (t & 7) + ki) + (kt & 3);
-    const int knib = (t >> 3) + 2 * (ke >> 1) + 4 * (ke & 1);
-    const int vi = (t & 7) >> 1;
-    const int vword = 128 * (vm >> 2) + 4 * (4 * vn + vi) + (vm & 3);
-    const int vnib = (ve & 1) + 2 * (t >> 3) + 4 * (t & 1);
+    int kword, knib, vword, vnib;
+    key_position(t, c, kword, knib);
+    value_position(t, c, vword, vnib);
     const float kcode = static_cast<float>(code_at(blk + kcode_off, kword, knib, p.bits));
     const float vcode = static_cast<float>(code_at(blk + vcode_off, vword, vnib, p.bits));
     const float vs = __half2float(reinterpret_cast<const __half *>(blk + vscale_off)[g * kPage + t]);

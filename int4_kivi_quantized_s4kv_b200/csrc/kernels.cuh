@@ -87,27 +87,6 @@ struct FusedAppend {
   const __half *v_new;
 };
 
-struct PrefillParams {
-  const uint8_t *pool;
-  const __half *res_k;
-  const __half *res_v;
-  const __half *q;        // [n_tokens][num_q_heads][128]
-  __half *out;            // [n_tokens][num_q_heads][128]
-  const int32_t *cu_new;  // [batch + 1]
-  const int32_t *seq_lens;
-  const int32_t *block_tables;
-  uint32_t *err;
-  int n_tokens;
-  int num_q_heads;
-  int num_kv_heads;
-  int group;
-  int max_pages;
-  int num_pages;
-  float scale_log2;       // sm_scale * log2(e)
-  uint8_t *ws;            // operand tiles [batch][num_kv_heads][tiles_per_seq][tile bytes]
-  int tiles_per_seq;      // key tiles of max_pages pages
-};
-
 void launch_append(const AppendParams &p, int batch, int max_new, cudaStream_t stream);
 void launch_dequant(const DequantParams &p, cudaStream_t stream);
 void launch_move(const MoveParams &p, cudaStream_t stream);
@@ -116,10 +95,5 @@ int decode_ctas_per_sm(int bits);
 int decode_warps_per_cta();
 cudaError_t prepare_decode_kernel();
 size_t decode_smem_bytes(int bits);
-void launch_prefill(const PrefillParams &p, int batch, int max_new, cudaStream_t stream);
-cudaError_t prepare_prefill_kernel();
-size_t prefill_smem_bytes();
-size_t prefill_tile_bytes();
-int prefill_tiles_per_seq(int max_pages);
 
 }  // namespace s4kv

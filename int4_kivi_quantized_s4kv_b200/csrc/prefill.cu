@@ -50,7 +50,9 @@
 // bit, and every role then leaves its loop.
 #include <cfloat>
 
+#include "code_map.cuh"
 #include "kernels.cuh"
+#include "prefill.cuh"
 #include "tc05.cuh"
 
 namespace s4kv {
@@ -69,7 +71,6 @@ constexpr uint32_t kQBytes = 128 * 128 * 2;      // Q [128][128] fp16
 constexpr uint32_t kKBytes = 2 * kKeyTile * 128 * 2;   // K_hi, K_lo [128][128] fp16 each
 constexpr uint32_t kVBytes = 128 * kKeyTile * 2;       // V^T [128][128] fp16
 constexpr uint32_t kTileBytes = kKBytes + kVBytes;     // workspace tile
-constexpr uint32_t kStagingBytes = kPagesPerTile * kBlockBytes;
 constexpr float kSlack = 8.0f;                   // log2 slack of the softmax reference
 constexpr long long kWaitLimit = 2000000000LL;   // about one second
 // S: M = 128, N = 128 keys, K = 256 (Q against K_hi, then Q against K_lo,
@@ -98,7 +99,10 @@ static_assert(kSmemBytes <= 227 * 1024, "prefill shared memory");
 static_assert(kKBytes % 1024 == 0 && kVBytes % 1024 == 0 && kOffBar % 1024 == 0, "1024-byte operand alignment");
 
 // operand kernel smem: the output tile, then the staged page blocks
-constexpr uint32_t kOpSmemBytes = kTileBytes + kStagingBytes + 1024;
+template <int kBits>
+constexpr uint32_t op_smem_bytes() {
+  return kTileBytes + kPagesPerTile * Fmt<kBits>::kBlock + 1024;
+}
 
 // Bounded wait for a barrier phase; gives up after about a second or as soon
 // as another role has raised the CTA's abort flag.
@@ -201,7 +205,9 @@ __device__ __forceinline__ bool seq_rows(const PrefillParams &p, int b, bool fla
 // 128-byte swizzled K-major.  Keys at or past L (the rest of
 // the partial last page, pages after it) are written as zeros, so masked
 // keys hold finite values.
+template <int kBits>
 __global__ void __launch_bounds__(kOpThreads) prefill_operands_kernel(const PrefillParams p) {
+  using F = Fmt<kBits>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_addr(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -219,7 +225,7 @@ __global__ void __launch_bounds__(kOpThreads) prefill_operands_kernel(const Pref
   // ---- the tile's full pages into shared memory, 16-byte loads
   const int q = max(0, min(kPagesPerTile, nfull - kt * kPagesPerTile));
   const int32_t *bt = p.block_tables + static_cast<long>(b) * p.max_pages + kt * kPagesPerTile;
-  constexpr int kChunks = kBlockBytes / 16;
+  constexpr int kChunks = F::kBlock / 16;
   for (int i = t; i < q * kChunks; i += kOpThreads) {
     const int k = i / kChunks, c = i - k * kChunks;
     int phys = __ldg(bt + k);
@@ -228,8 +234,8 @@ __global__ void __launch_bounds__(kOpThreads) prefill_operands_kernel(const Pref
       phys = 0;
     }
     const uint4 *src = reinterpret_cast<const uint4 *>(
-        p.pool + (static_cast<long long>(phys) * H + h) * kBlockBytes);
-    sts128(stage + k * kBlockBytes + 16 * c, __ldg(src + c));
+        p.pool + (static_cast<long long>(phys) * H + h) * F::kBlock);
+    sts128(stage + k * F::kBlock + 16 * c, __ldg(src + c));
   }
   __syncthreads();
 
@@ -237,8 +243,41 @@ __global__ void __launch_bounds__(kOpThreads) prefill_operands_kernel(const Pref
   const int dpage = t >> 6, widx = t & 63;
   const int dq = widx & 3, dlane0 = widx >> 2;
   const int pg = kt * kPagesPerTile + dpage;
-  if (pg < nfull) {
-    const uint32_t blk = stage + dpage * kBlockBytes;
+  if (pg < nfull && kBits != 4) {
+    // 8- and 2-bit codes: element by element through the code map; two
+    // channels per thread, the page's 16 tokens
+    const uint8_t *blk = smem_raw + (stage + dpage * F::kBlock - raw);
+    const __half *kscale = reinterpret_cast<const __half *>(blk + F::kKScale);
+    const __half *kzero = reinterpret_cast<const __half *>(blk + F::kKZero);
+    const __half *vscale = reinterpret_cast<const __half *>(blk + F::kVScale);
+    const __half *vzero = reinterpret_cast<const __half *>(blk + F::kVZero);
+    const int c0 = 2 * widx;
+    const float ks0 = __half2float(kscale[c0]), ks1 = __half2float(kscale[c0 + 1]);
+    const float kz0 = __half2float(kzero[key_zero_slot(c0)]), kz1 = __half2float(kzero[key_zero_slot(c0 + 1)]);
+    const int g = c0 / kVGroup;
+    for (int t = 0; t < kPage; ++t) {
+      int w0, n0, w1, n1;
+      key_position(t, c0, w0, n0);
+      key_position(t, c0 + 1, w1, n1);
+      uint32_t hi, lo;
+      const uint32_t codes = h2_as_u32(__floats2half2_rn(static_cast<float>(code_at(blk + F::kKCode, w0, n0, kBits)),
+                                                         static_cast<float>(code_at(blk + F::kKCode, w1, n1, kBits))));
+      split_key(codes, make_float2(ks0, ks1), make_float2(kz0, kz1), hi, lo);
+      const int key = dpage * 16 + t;
+      const uint32_t ko = tc05::sw128_offset(key, c0, kKeyTile);
+      sts32(sK + ko, hi);
+      sts32(sK + kKBytes / 2 + ko, lo);
+      const __half vs = vscale[g * kPage + t], vz = vzero[g * kPage + t];
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        int vw, vn;
+        value_position(t, c0 + j, vw, vn);
+        const __half code = __float2half_rn(static_cast<float>(code_at(blk + F::kVCode, vw, vn, kBits)));
+        sts16(sV + tc05::sw128_offset(c0 + j, key, 128), __half_as_ushort(__hfma(code, vs, vz)));
+      }
+    }
+  } else if (pg < nfull) {
+    const uint32_t blk = stage + dpage * F::kBlock;
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       const int w = widx + 64 * e;
@@ -619,14 +658,26 @@ int prefill_tiles_per_seq(int max_pages) {
 cudaError_t prepare_prefill_kernel() {
   cudaError_t e = cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(kSmemBytes));
-  if (e != cudaSuccess) return e;
-  return cudaFuncSetAttribute(prefill_operands_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              static_cast<int>(kOpSmemBytes));
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(prefill_operands_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(op_smem_bytes<4>()));
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(prefill_operands_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(op_smem_bytes<8>()));
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(prefill_operands_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(op_smem_bytes<2>()));
+  return e;
 }
 
 void launch_prefill(const PrefillParams &p, int batch, int max_new, cudaStream_t stream) {
   const dim3 og(p.tiles_per_seq, batch, p.num_kv_heads);
-  prefill_operands_kernel<<<og, kOpThreads, kOpSmemBytes, stream>>>(p);
+  if (p.bits == 8)
+    prefill_operands_kernel<8><<<og, kOpThreads, op_smem_bytes<8>(), stream>>>(p);
+  else if (p.bits == 2)
+    prefill_operands_kernel<2><<<og, kOpThreads, op_smem_bytes<2>(), stream>>>(p);
+  else
+    prefill_operands_kernel<4><<<og, kOpThreads, op_smem_bytes<4>(), stream>>>(p);
   const int Tq = 128 / p.group;
   const int tiles = (max_new + Tq - 1) / Tq;
   const dim3 grid(tiles, batch, p.num_kv_heads);

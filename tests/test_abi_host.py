@@ -136,12 +136,16 @@ def test_invalid_calls_rejected_before_launch(S):
     assert L.s4kv_dequant_page(ctypes.byref(c), 10, P(fake), P(fake), 1, st) == S.ERR_INVALID_ARG
     assert L.s4kv_dequant_page(ctypes.byref(c), -1, P(fake), P(fake), 1, st) == S.ERR_INVALID_ARG
     assert L.s4kv_dequant_page(ctypes.byref(bad_dim), 0, P(fake), P(fake), 1, st) == S.ERR_UNSUPPORTED
-    # code width: 4 (or 0), 8 and 2 only; prefill has no 8- or 2-bit path
+    # code width: 4 (or 0), 8 and 2 only
     bad_bits = S.s4kv_cache_t(fake, fake, fake, None, 10, 2, 4, 128, 16, 3)
     assert L.s4kv_dequant_page(ctypes.byref(bad_bits), 0, P(fake), P(fake), 1, st) == S.ERR_UNSUPPORTED
     c8 = S.s4kv_cache_t(fake, fake, fake, None, 10, 2, 4, 128, 16, 8)
-    assert pre(ctypes.byref(c8), P(fake), 8, 4, P(fake), P(fake), P(fake), 1, 1, 4, 0.088, P(fake), P(fake), 1 << 30,
+    # prefill takes 8- and 2-bit caches too: its host checks still run first
+    # (these calls stop at them, before any launch)
+    assert pre(ctypes.byref(c8), P(fake), 18, 4, P(fake), P(fake), P(fake), 1, 1, 4, 0.088, P(fake), P(fake), 1 << 30,
                st) == S.ERR_UNSUPPORTED
+    assert pre(ctypes.byref(c8), P(fake), 8, 4, P(fake), P(fake), P(fake), 1, 1, 4, 0.088, P(fake), None, 1 << 30,
+               st) == S.ERR_WORKSPACE
     n = ctypes.c_size_t(0)
     assert L.s4kv_page_record_bytes(ctypes.byref(c8), ctypes.byref(n)) == S.OK and n.value == 2 * 4864
     assert L.s4kv_page_record_bytes(ctypes.byref(c), ctypes.byref(n)) == S.OK and n.value == 2 * 2816

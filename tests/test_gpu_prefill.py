@@ -18,7 +18,7 @@ pytestmark = pytest.mark.gpu
 
 
 class PrefillCase:
-    def __init__(self, seed, H, G, before, after, outliers=8, context_chunk=64):
+    def __init__(self, seed, H, G, before, after, outliers=8, context_chunk=64, bits=4):
         import torch
         import oracle
         import int4_kivi_quantized_s4kv_b200 as S
@@ -41,8 +41,8 @@ class PrefillCase:
         for b, m in enumerate(need):
             self.bt[b, :m] = perm[c:c + m]
             c += m
-        self.oc = oracle.OracleCache(NP, H, B)
-        self.gpu = S.S4KVCache(NP, H, B, device="cuda")
+        self.oc = oracle.OracleCache(NP, H, B, bits=bits)
+        self.gpu = S.S4KVCache(NP, H, B, device="cuda", bits=bits)
         self.dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
         self.bt_dev = self.dev(self.bt)
         self._append(np.zeros(B, np.int64), self.before, context_chunk)
@@ -132,3 +132,17 @@ def test_prefill_ignores_stale_workspace_contents():
     ws2 = ws[:case.S.prefill_workspace_bytes(2, 2, small.bt.shape[1])]
     got2, ref2 = small.run(workspace=ws2)
     assert_attention_close(got2, ref2, "prefill, reused workspace")
+
+
+@pytest.mark.parametrize("bits", [8, 2])
+def test_prefill_8_and_2_bit_caches(bits):
+    """The same attention over 8- and 2-bit pages: only the operand tiles'
+    dequantization differs (every code through the code map); the cache
+    bytes must match the oracle's and the output must be within the bound."""
+    case = PrefillCase(90 + bits, 2, 4, before=[0, 100, 300], after=[37, 290, 301], bits=bits)
+    assert np.array_equal(case.gpu.pool.cpu().numpy(), case.oc.pool)
+    got, ref = case.run()
+    assert_attention_close(got, ref, f"prefill int{bits}")
+    case8 = PrefillCase(95 + bits, 1, 8, before=[1000], after=[1200], bits=bits, context_chunk=256)
+    got, ref = case8.run(sm_scale=0.06)
+    assert_attention_close(got, ref, f"prefill int{bits} G=8")

@@ -493,7 +493,12 @@ def test_fp32_oracle_close_to_fp64(oracle_mod):
 
 # ------------------------------------------------------------ prefill --
 
-def _grid_streams(rng, lens, H):
+def _grid_streams(rng, lens, H, bits=4):
+    """Key/value streams whose every page is an exact grid of the code width
+    (the grid pages of each width are defined further down; looked up at
+    call time)."""
+    page = {4: lambda per: _grid_page(rng, per)[0], 8: lambda per: _grid_page8(rng, per),
+            2: lambda per: _grid_page2(rng, per)}[bits]
     k, v = [], []
     for L in lens:
         npg = (L + PAGE - 1) // PAGE
@@ -501,26 +506,28 @@ def _grid_streams(rng, lens, H):
         vv = np.zeros((npg * PAGE, H, HD), np.float16)
         for p in range(npg):
             for h in range(H):
-                kk[p * PAGE:(p + 1) * PAGE, h] = _grid_page(rng, "key")[0]
-                vv[p * PAGE:(p + 1) * PAGE, h] = _grid_page(rng, "value")[0]
+                kk[p * PAGE:(p + 1) * PAGE, h] = page("key")
+                vv[p * PAGE:(p + 1) * PAGE, h] = page("value")
         k.append(kk[:L])
         v.append(vv[:L])
     return k, v
 
 
-def test_prefill_matches_textbook_causal_attention_on_exact_grids(oracle_mod):
+@pytest.mark.parametrize("bits", [4, 8, 2])
+def test_prefill_matches_textbook_causal_attention_on_exact_grids(oracle_mod, bits):
     """A chunk of n new tokens appended to a context of L - n tokens: every
     query row at position pos must equal plain softmax attention (numpy,
     float64) over the original fp16 keys and values 0..pos.  On exact grids
-    the dequantized cache is the input itself, so this pins the causal
-    limit, the position of each chunk row, the GQA map and the page walk."""
-    rng = np.random.default_rng(31)
+    of the code width the dequantized cache is the input itself, so this
+    pins the causal limit, the position of each chunk row, the GQA map and
+    the page walk, for every width."""
+    rng = np.random.default_rng(31 + bits)
     H, G = 2, 3
     before = [21, 0, 32, 5]
     after = [40, 17, 50, 37]
-    k, v = _grid_streams(rng, after, H)
+    k, v = _grid_streams(rng, after, H, bits)
     bt, NP = _tables(rng, after)
-    c = oracle_mod.OracleCache(NP, H, len(after))
+    c = oracle_mod.OracleCache(NP, H, len(after), bits=bits)
     _append_all(oracle_mod, c, k, v, [0] * 4, before, bt)
     _append_all(oracle_mod, c, k, v, before, after, bt)
     n = np.array(after) - np.array(before)
