@@ -65,12 +65,14 @@ constexpr int kProducerWarp = 5;
 constexpr int kThreadsP = 32 * 6;
 constexpr int kKeyTile = 128;                    // keys per tile
 constexpr int kPagesPerTile = kKeyTile / kPage;  // 8
-constexpr int kOpThreads = 64 * kPagesPerTile;   // operand kernel: 64 threads per page
+constexpr int kOpPages = kPagesPerTile / 2;       // operand kernel: half a key tile per CTA
+constexpr int kOpThreads = 64 * kOpPages;        // 64 threads per page
 constexpr int kStages = 2;                       // K and V buffers each
 constexpr uint32_t kQBytes = 128 * 128 * 2;      // Q [128][128] fp16
 constexpr uint32_t kKBytes = 2 * kKeyTile * 128 * 2;   // K_hi, K_lo [128][128] fp16 each
 constexpr uint32_t kVBytes = 128 * kKeyTile * 2;       // V^T [128][128] fp16
 constexpr uint32_t kTileBytes = kKBytes + kVBytes;     // workspace tile
+constexpr uint32_t kHalfTileBytes = kTileBytes / 2;
 constexpr float kSlack = 8.0f;                   // log2 slack of the softmax reference
 constexpr long long kWaitLimit = 2000000000LL;   // about one second
 // S: M = 128, N = 128 keys, K = 256 (Q against K_hi, then Q against K_lo,
@@ -98,10 +100,10 @@ constexpr uint32_t kSmemBytes = kOffAbort + 4 + 1024;  // + alignment slack
 static_assert(kSmemBytes <= 227 * 1024, "prefill shared memory");
 static_assert(kKBytes % 1024 == 0 && kVBytes % 1024 == 0 && kOffBar % 1024 == 0, "1024-byte operand alignment");
 
-// operand kernel smem: the output tile, then the staged page blocks
+// operand kernel smem: the output half tile, then the staged page blocks
 template <int kBits>
 constexpr uint32_t op_smem_bytes() {
-  return kTileBytes + kPagesPerTile * Fmt<kBits>::kBlock + 1024;
+  return kHalfTileBytes + kOpPages * Fmt<kBits>::kBlock + 1024;
 }
 
 // Bounded wait for a barrier phase; gives up after about a second or as soon
@@ -200,31 +202,38 @@ __device__ __forceinline__ bool seq_rows(const PrefillParams &p, int b, bool fla
 }  // namespace
 
 // ---------------------------------------------------------------------------
-// Launch 1: one CTA per (key tile, sequence, kv head) writes the tile's
-// operands to the workspace: K_hi, K_lo and V^T, each [128][128] fp16 and
-// 128-byte swizzled K-major.  Keys at or past L (the rest of
-// the partial last page, pages after it) are written as zeros, so masked
-// keys hold finite values.
+// Launch 1: one CTA per (half key tile, sequence, kv head) writes that half
+// of the tile's operands to the workspace: K_hi, K_lo and V^T, each
+// [128][128] fp16 and 128-byte swizzled K-major.  Half hh holds keys
+// 64 hh .. 64 hh + 63: rows 64 hh .. of both column blocks of K_hi and K_lo
+// (8 KB each, the same bytes a 64-row operand has) and column block hh of V^T
+// (16 KB).  Keys at or past L (the rest of the partial last page, pages
+// after it) are written as zeros, so masked keys hold finite values.
 template <int kBits>
 __global__ void __launch_bounds__(kOpThreads) prefill_operands_kernel(const PrefillParams p) {
   using F = Fmt<kBits>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_addr(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
-  const uint32_t sK = base, sV = base + kKBytes;
-  const uint32_t stage = base + kTileBytes;
-  const int kt = blockIdx.x, b = blockIdx.y, h = blockIdx.z, H = p.num_kv_heads;
+  // half tile in smem: K_hi [64][128] (two 8 KB column blocks), K_lo the same,
+  // then V^T [128][64]
+  const uint32_t sK = base, sV = base + kKBytes / 2;
+  const uint32_t stage = base + kHalfTileBytes;
+  const int ht = blockIdx.x, b = blockIdx.y, h = blockIdx.z, H = p.num_kv_heads;
+  const int kt = ht >> 1, hh = ht & 1;
   const int t = threadIdx.x;
   SeqRows sr;
   if (!seq_rows(p, b, false, sr)) return;
   const int L = sr.L;
+  // a tile the attention reads is written whole: a half past L is zeros
   if (kt * kKeyTile >= L) return;
   const int nfull = L / kPage;
   const int np = (L + kPage - 1) / kPage;
+  const int pg0 = ht * kOpPages;  // first page of this half tile
 
-  // ---- the tile's full pages into shared memory, 16-byte loads
-  const int q = max(0, min(kPagesPerTile, nfull - kt * kPagesPerTile));
-  const int32_t *bt = p.block_tables + static_cast<long>(b) * p.max_pages + kt * kPagesPerTile;
+  // ---- the half tile's full pages into shared memory, 16-byte loads
+  const int q = max(0, min(kOpPages, nfull - pg0));
+  const int32_t *bt = p.block_tables + static_cast<long>(b) * p.max_pages + pg0;
   constexpr int kChunks = F::kBlock / 16;
   for (int i = t; i < q * kChunks; i += kOpThreads) {
     const int k = i / kChunks, c = i - k * kChunks;
@@ -242,7 +251,7 @@ __global__ void __launch_bounds__(kOpThreads) prefill_operands_kernel(const Pref
   // ---- dequantize: 64 threads per page
   const int dpage = t >> 6, widx = t & 63;
   const int dq = widx & 3, dlane0 = widx >> 2;
-  const int pg = kt * kPagesPerTile + dpage;
+  const int pg = pg0 + dpage;
   if (pg < nfull && kBits != 4) {
     // 8- and 2-bit codes: element by element through the code map; two
     // channels per thread, the page's 16 tokens
@@ -263,10 +272,10 @@ __global__ void __launch_bounds__(kOpThreads) prefill_operands_kernel(const Pref
       const uint32_t codes = h2_as_u32(__floats2half2_rn(static_cast<float>(code_at(blk + F::kKCode, w0, n0, kBits)),
                                                          static_cast<float>(code_at(blk + F::kKCode, w1, n1, kBits))));
       split_key(codes, make_float2(ks0, ks1), make_float2(kz0, kz1), hi, lo);
-      const int key = dpage * 16 + t;
-      const uint32_t ko = tc05::sw128_offset(key, c0, kKeyTile);
+      const int key = dpage * 16 + t;  // within the half tile
+      const uint32_t ko = tc05::sw128_offset(key, c0, kKeyTile / 2);
       sts32(sK + ko, hi);
-      sts32(sK + kKBytes / 2 + ko, lo);
+      sts32(sK + kKBytes / 4 + ko, lo);
       const __half vs = vscale[g * kPage + t], vz = vzero[g * kPage + t];
 #pragma unroll
       for (int j = 0; j < 2; ++j) {
@@ -299,11 +308,11 @@ __global__ void __launch_bounds__(kOpThreads) prefill_operands_kernel(const Pref
         split_key(a1, s01, zf01, hi1, lo1);
         split_key(a2, s23, zf23, hi2, lo2);
         split_key(a3, s23, zf23, hi3, lo3);
-        const uint32_t ko = tc05::sw128_offset(dpage * 16 + dn, c0, kKeyTile);
+        const uint32_t ko = tc05::sw128_offset(dpage * 16 + dn, c0, kKeyTile / 2);
         sts64(sK + ko, hi0, hi2);
         sts64(sK + ko + 1024, hi1, hi3);
-        sts64(sK + kKBytes / 2 + ko, lo0, lo2);
-        sts64(sK + kKBytes / 2 + ko + 1024, lo1, lo3);
+        sts64(sK + kKBytes / 4 + ko, lo0, lo2);
+        sts64(sK + kKBytes / 4 + ko + 1024, lo1, lo3);
       }
       // values: channels cb, cb + 1; tokens 2 di, 2 di + 1 (+ 8)
       {
@@ -333,9 +342,9 @@ __global__ void __launch_bounds__(kOpThreads) prefill_operands_kernel(const Pref
       const int tk = e >> 6, c = 2 * (e & 63);
       uint32_t kb = 0;
       if (tk < rres) kb = *reinterpret_cast<const uint32_t *>(rk + tk * kHeadDim + c);
-      const uint32_t ko = tc05::sw128_offset(dpage * 16 + tk, c, kKeyTile);
+      const uint32_t ko = tc05::sw128_offset(dpage * 16 + tk, c, kKeyTile / 2);
       sts32(sK + ko, kb);
-      sts32(sK + kKBytes / 2 + ko, 0u);
+      sts32(sK + kKBytes / 4 + ko, 0u);
     }
     for (int e = widx; e < kPage * kHeadDim; e += 64) {
       const int tk = e >> 7, c = e & 127;
@@ -346,10 +355,16 @@ __global__ void __launch_bounds__(kOpThreads) prefill_operands_kernel(const Pref
   }
   __syncthreads();
 
-  // ---- the tile to the workspace, coalesced 16-byte stores
-  uint4 *dst = reinterpret_cast<uint4 *>(
-      p.ws + ((static_cast<long long>(b) * H + h) * p.tiles_per_seq + kt) * kTileBytes);
-  for (int i = t; i < static_cast<int>(kTileBytes / 16); i += kOpThreads) dst[i] = lds128_at(base + 16 * i);
+  // ---- the half tile to its places in the workspace tile, coalesced 16-byte
+  // stores: smem 8 KB pieces 0..3 (K_hi, K_lo column blocks) go to
+  // 16 KB * piece + 8 KB * hh, the 16 KB of V^T to K bytes + 16 KB * hh
+  uint8_t *tile = p.ws + ((static_cast<long long>(b) * H + h) * p.tiles_per_seq + kt) * kTileBytes;
+  for (int i = t; i < static_cast<int>(kHalfTileBytes / 16); i += kOpThreads) {
+    const uint32_t off = 16u * i;
+    const uint32_t dst = off < kKBytes / 2 ? (off >> 13) * 16384u + 8192u * hh + (off & 8191u)
+                                           : kKBytes + 16384u * hh + (off - kKBytes / 2);
+    *reinterpret_cast<uint4 *>(tile + dst) = lds128_at(base + off);
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -671,7 +686,7 @@ cudaError_t prepare_prefill_kernel() {
 }
 
 void launch_prefill(const PrefillParams &p, int batch, int max_new, cudaStream_t stream) {
-  const dim3 og(p.tiles_per_seq, batch, p.num_kv_heads);
+  const dim3 og(2 * p.tiles_per_seq, batch, p.num_kv_heads);
   if (p.bits == 8)
     prefill_operands_kernel<8><<<og, kOpThreads, op_smem_bytes<8>(), stream>>>(p);
   else if (p.bits == 2)
