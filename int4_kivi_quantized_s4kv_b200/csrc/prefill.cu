@@ -1,6 +1,7 @@
 // s4kv_prefill_attention device side: causal attention of a chunk of new
-// query tokens over the int4 paged cache after the chunk was appended (the
-// prefill / chunked-append side of the cache that decode attention reads).
+// query tokens over the paged cache (4-bit codes, or the 8- and 2-bit
+// variants) after the chunk was appended (the prefill / chunked-append side
+// of the cache that decode attention reads).
 //
 // What it computes: sequence b owns query rows cu_new[b] .. cu_new[b+1]-1;
 // with n new tokens and L tokens after the append, row j sits at position
@@ -24,7 +25,10 @@
 //     the logits visibly).  A value is the fused fp16 multiply-add
 //     code * scale + zero (the correctly rounded fp16), stored transposed.
 //     Every query tile of the sequence then reads these bytes (mostly from
-//     L2) instead of dequantizing the same pages again.
+//     L2) instead of dequantizing the same pages again.  One CTA writes half
+//     a tile; int4 pages are read in their MMA-fragment order, 8- and 2-bit
+//     pages code by code through the code map.  Only this launch depends on
+//     the code width.
 //  2. prefill_kernel: one CTA takes one (query tile, sequence, kv head); the
 //     tile's 128 MMA rows are (token, head of the group) pairs, so a tile
 //     holds floor(128 / G) tokens.  Warps with separate roles hand buffers
