@@ -358,13 +358,13 @@ def prefill_flops(spec, lens, new):
     return f
 
 
-def measure_prefill(device, steps: int, workload: str = "llama3.1-8b-prefill"):
+def measure_prefill(device, steps: int, workload: str = "llama3.1-8b-prefill", bits: int = 4):
     """Chunked-prefill attention (the cache's prefill side) on its own
     workload: the chunk is appended once, then s4kv_prefill_attention is timed
     with CUDA events on the launching stream."""
     import torch
     spec = W.SPECS[workload]
-    wl = DeviceWorkload(spec, device)
+    wl = DeviceWorkload(spec, device, bits=bits)
     S = wl.S
     cache = wl.caches[0]
     S.s4kv_append(cache, wl.k_new[0], wl.v_new[0], wl.step_slots, wl.step_cu, wl.seq_lens, wl.bt, wl.max_new)
@@ -399,7 +399,8 @@ def measure_prefill(device, steps: int, workload: str = "llama3.1-8b-prefill"):
     # and the attention, whose MMAs per (query tile, key tile) are
     # Q [K_hi; K_lo]^T (keys carried to ~22 bits) and P V: 1.5x the
     # algorithmic FLOPs
-    return {"workload": spec.name, "model_shape": spec.description, "calls": steps, "launches": 2 * steps,
+    return {"workload": spec.name, "model_shape": spec.description, "code_bits": bits, "calls": steps,
+            "launches": 2 * steps,
             "avg_call_ms": ms, "tflops": achieved, "query_tokens": rows,
             "roofline": {"bound": "tensor", "kernel": "prefill_operands_kernel + prefill_kernel (one call)",
                          "achieved": achieved, "peak": peak, "peak_kind": kind, "unit": "TFLOP/s",
@@ -692,7 +693,7 @@ def main(argv=None):
     tokens = int(wl.new.sum())
     prefill = moves = fused = int8 = int2 = None
     if world == 1 and not args.no_prefill:
-        prefill = measure_prefill(device, max(3, min(args.steps, 20)))
+        prefill = [measure_prefill(device, max(3, min(args.steps, 20)), w, args.bits) for w in W.PREFILL_ORDER]
         moves = measure_page_moves(wl, device)
         fused = [measure_fused_step(wl, device)]
         small = DeviceWorkload(W.SPECS["qwen2.5-7b"], device)
