@@ -83,3 +83,59 @@ def test_full_size_sampled_parity(name):
     del wl
     gc.collect()
     torch.cuda.empty_cache()
+
+
+# chunked prefill: (sequence, rows) samples; the chunk's last rows see the
+# whole sequence, so the oracle recomputes them from a one-sequence cache
+PREFILL_SAMPLES = {
+    "llama3.1-8b-prefill": [0, 3],
+    "llama3-70b-prefill": [1],
+}
+
+
+@pytest.mark.parametrize("name", list(PREFILL_SAMPLES))
+def test_full_size_prefill_sampled_parity(name):
+    """The prefill workload at full shape in the launch configuration the
+    bench times (the whole chunk of every sequence in one call): sampled
+    sequences' pool pages bit-exact against the oracle's, and the last rows
+    of their chunks within 2e-3 + 1e-3 |ref|."""
+    import torch
+    import oracle
+    import bench
+    spec = W.SPECS[name]
+    dev = torch.device("cuda", 0)
+    wl = bench.DeviceWorkload(spec, dev)
+    S = wl.S
+    cache = wl.caches[0]
+    S.s4kv_append(cache, wl.k_new[0], wl.v_new[0], wl.step_slots, wl.step_cu, wl.seq_lens, wl.bt, wl.max_new)
+    rows = int(wl.new.sum())
+    q = W.chunk_queries_torch(spec, 0, rows, dev)
+    out = torch.full_like(q, float("nan"))
+    ws = S.prefill_workspace(spec.num_kv_heads, spec.batch, wl.bt.shape[1], dev)
+    S.s4kv_prefill_attention(cache, q, wl.step_cu, wl.seq_lens, wl.bt, out, wl.max_new, workspace=ws)
+    torch.cuda.synchronize()
+    assert S.s4kv_get_error(cache) == 0
+    assert bool(torch.isfinite(out.float()).all())
+    cu = wl.step_cu.cpu().numpy()
+    H = spec.num_kv_heads
+    for b in PREFILL_SAMPLES[name]:
+        L = int(wl.lens[b])
+        k, v = W.kv_sequence_torch(spec, 0, b, L, dev)
+        k, v = k.cpu().numpy(), v.cpu().numpy()
+        need = (L + PAGE - 1) // PAGE
+        bt = np.arange(need, dtype=np.int32)[None, :]
+        oc = oracle.OracleCache(need + 1, H, 1)
+        sm = W.slot_mapping(bt, [np.arange(L)])
+        assert oc.append(k, v, sm, np.array([0, L], np.int32), np.array([L], np.int32), bt) == 0
+        full = L // PAGE
+        gpu_pages = wl.plan.block_tables[b, :full]
+        pool = cache.pool[torch.from_numpy(gpu_pages.astype(np.int64)).to(dev)].cpu().numpy()
+        assert np.array_equal(pool, oc.pool[:full]), f"pool pages of seq {b}"
+        last = np.arange(int(cu[b + 1]) - 4, int(cu[b + 1]))
+        ref = oc.prefill_attention(q[torch.from_numpy(last).to(dev)].cpu().numpy(), np.array([0, 4], np.int32),
+                                   np.array([L], np.int32), bt)
+        got = out[torch.from_numpy(last).to(dev)].float().cpu().numpy()
+        assert_attention_close(got, ref, f"{spec.name} seq {b} last rows (L={L})")
+    del wl
+    gc.collect()
+    torch.cuda.empty_cache()
