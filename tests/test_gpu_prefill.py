@@ -146,3 +146,24 @@ def test_prefill_8_and_2_bit_caches(bits):
     case8 = PrefillCase(95 + bits, 1, 8, before=[1000], after=[1200], bits=bits, context_chunk=256)
     got, ref = case8.run(sm_scale=0.06)
     assert_attention_close(got, ref, f"prefill int{bits} G=8")
+
+
+def test_prefill_leaves_rows_of_no_sequence_untouched():
+    """q and out may hold more rows than cu_new[batch]: those rows belong to
+    no sequence and are neither read nor written."""
+    import torch
+    case = PrefillCase(85, 2, 4, before=[5, 60], after=[40, 61])
+    S = case.S
+    n = int(case.cu[-1])
+    extra = 7
+    q = np.concatenate([case.q, np.random.default_rng(1).standard_normal((extra, 8, HD)).astype(np.float16)])
+    qd = case.dev(q)
+    out = torch.full_like(qd, float("nan"))
+    S.s4kv_prefill_attention(case.gpu, qd, case.dev(case.cu), case.dev(case.after.astype(np.int32)), case.bt_dev,
+                             out, int(case.n.max()))
+    torch.cuda.synchronize()
+    assert S.s4kv_get_error(case.gpu) == 0
+    got = out.float().cpu().numpy()
+    assert np.isnan(got[n:]).all()
+    ref = case.oc.prefill_attention(case.q, case.cu, case.after.astype(np.int32), case.bt)
+    assert_attention_close(got[:n], ref, "prefill with trailing rows")
