@@ -102,6 +102,41 @@ def test_quantize_group_all_equal_and_signed_zero(oracle_mod):
     assert s == 0.0 and (codes == 0).all() and zh == 0x8000  # min in total order is -0
 
 
+def _half_to_even(t):
+    """Round to the nearest integer, ties to the even neighbour: the IEEE
+    default rounding that rint names, restated with Python's exact rationals
+    (independent of the C library the oracle calls)."""
+    t = Fraction(t)
+    f = t.numerator // t.denominator
+    rem = t - f
+    if rem > Fraction(1, 2) or (rem == Fraction(1, 2) and f % 2 == 1):
+        f += 1
+    return f
+
+
+@pytest.mark.parametrize("bits,n,lo,step", [(4, 16, 0.0, 1.0), (4, 32, -4.0, 0.5), (4, 16, 2.0, 0.25),
+                                            (8, 32, 0.0, 1.0), (8, 16, -8.0, 0.125), (2, 16, 0.0, 1.0),
+                                            (2, 32, -1.0, 0.5)])
+def test_quantize_group_ties_round_half_to_even(oracle_mod, bits, n, lo, step):
+    """Groups whose quotients (x - min) / s are exact half-integers (a grid of
+    spacing s/2 from min to min + levels*s, every point exact in fp16 and in
+    fp32): rint sends k + 1/2 to the even one of k and k + 1, so 0.5 -> 0,
+    1.5 -> 2, 2.5 -> 2, 3.5 -> 4.  Rounding ties away from zero (roundf), or
+    up (floor(t + 1/2)), gives odd codes here and fails."""
+    levels = (1 << bits) - 1
+    rng = np.random.default_rng(bits * 100 + n)
+    halves = (np.arange(levels) + 0.5)                     # every tie the grid has
+    t = np.concatenate([[0.0, float(levels)], rng.choice(halves, n - 2, replace=levels < n - 2)])
+    t = t[rng.permutation(n)]
+    x = (lo + t * step).astype(np.float16)
+    assert np.array_equal(x.astype(np.float64), lo + t * step)   # exact in fp16
+    codes, sh, zh, s = oracle_mod.quantize_group_bits(x, bits)
+    assert s == step and zh == f16bits(lo)
+    want = [_half_to_even(Fraction(v)) for v in t]
+    assert list(codes) == want
+    assert any(int(v * 2) % 4 == 1 for v in t) and any(int(v * 2) % 4 == 3 for v in t)  # both tie parities occur
+
+
 def _bound_ok(x16, codes, s32, zero_bits):
     mn = Fraction(float(np.uint16(zero_bits).view(np.float16)))
     S = Fraction(s32)
