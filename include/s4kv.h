@@ -165,7 +165,12 @@ S4KV_API int s4kv_cache_layout(int num_pages, int num_kv_heads, int max_seqs,
 S4KV_API int s4kv_cache_layout_bits(int num_pages, int num_kv_heads, int max_seqs, int bits,
                                     size_t *pool_bytes, size_t *residual_bytes);
 
-/* Append new tokens' K/V and quantize every page they complete.
+/* Append new tokens' K/V and quantize every page they complete: keys per
+ * channel and values per token, asymmetric ("S4 KV -- int4
+ * KV-Cache-Kompression fuer vLLM", "Funktionsweise" step 1), into 16-token
+ * pages reached through block_tables ("PagedAttention reduziert den
+ * KV-Cache-Speicherbedarf beim LLM-Serving erheblich", "Wichtigste
+ * Kernpunkte & Evidenz").
  *  k, v          device fp16 [n_tokens][num_kv_heads][128], 16-B aligned,
  *                sequence b's new tokens at rows cu_new[b]..cu_new[b+1]-1
  *                in position order.
@@ -191,10 +196,18 @@ S4KV_API int s4kv_append(const s4kv_cache_t *cache, const void *k, const void *v
 /* Bytes of device workspace s4kv_decode_attention needs on the CURRENT
  * device for this batch and kv head count.  The workspace must be
  * zero-filled once after allocation; every completed decode call leaves
- * its counters at zero again.  Needs a CUDA device (S4KV_ERR_CUDA if none). */
+ * its counters at zero again.  A workspace sized for a batch serves every
+ * smaller batch too (its per-sequence counters come last).  After a call
+ * that set S4KV_EFLAG_TIMEOUT some counters may be left nonzero: zero-fill
+ * the workspace again before reusing it.  Needs a CUDA device
+ * (S4KV_ERR_CUDA if none). */
 S4KV_API int s4kv_decode_workspace_size(int batch, int num_kv_heads, size_t *bytes);
 
-/* GQA paged decode attention over the quantized pages plus the residual.
+/* GQA paged decode attention over the quantized pages plus the residual
+ * (a group of query heads shares one kv head: "KV-Cache-Optimierung --
+ * PagedAttention, quantisierter KV, Speculative Cache", "Begriffe auf dieser
+ * Seite"; keys and values of full pages are the dequantized int4 codes of
+ * "S4 KV -- int4 KV-Cache-Kompression fuer vLLM", "Funktionsweise" step 1).
  *  q       device fp16 [batch][num_q_heads][128], 16-B aligned; query head
  *          j reads kv head j / (num_q_heads / num_kv_heads).
  *  seq_lens, block_tables as for s4kv_append (lengths including the tokens
@@ -306,7 +319,11 @@ S4KV_API int s4kv_prefill_attention(const s4kv_cache_t *cache, const void *q,
 S4KV_API int s4kv_prefill_workspace_size(int num_kv_heads, int batch, int max_pages_per_seq,
                                          size_t *bytes);
 
-/* Dequantize one physical page for all kv heads into natural order:
+/* Dequantize one physical page for all kv heads into natural order (the
+ * inverse of the KIVI step of "S4 KV -- int4 KV-Cache-Kompression fuer
+ * vLLM", "Funktionsweise" step 1, on one 16-token page of "PagedAttention
+ * reduziert den KV-Cache-Speicherbedarf beim LLM-Serving erheblich",
+ * "Wichtigste Kernpunkte & Evidenz"):
  * out_k, out_v device [num_kv_heads][16][128], fp32 if out_fp32 != 0
  * (x = code*scale + zero, exact product, one rounding) else fp16 (the fp32
  * value rounded to nearest even).  16-B aligned. */

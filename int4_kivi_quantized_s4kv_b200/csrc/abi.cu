@@ -85,8 +85,12 @@ int check_cache(const s4kv_cache_t *c) {
   return S4KV_OK;
 }
 
-// Workspace carve-up: [tickets: batch*kv_heads u32, padded to 256 B]
-// [m,l: 2*workers*8 float2] [partial O: 2*workers*8*128 float].
+// Workspace carve-up: [m,l: 2*workers*8 float2] [partial O:
+// 2*workers*8*128 float] [tickets: batch*kv_heads u32].  The two partial
+// regions depend only on the device's worker count, so they sit first and a
+// workspace sized for a large batch serves any smaller one: a call touches
+// a prefix of the ticket region, which it leaves at zero, and never reads
+// partial results as tickets.
 struct WsLayout {
   size_t tickets, ml, part, total;
 };
@@ -94,10 +98,10 @@ struct WsLayout {
 WsLayout ws_layout(int batch, int num_kv_heads, int num_workers) {
   auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
   WsLayout w;
-  w.tickets = 0;
-  w.ml = up(static_cast<size_t>(batch) * num_kv_heads * sizeof(uint32_t));
-  w.part = w.ml + up(static_cast<size_t>(2) * num_workers * 8 * 2 * sizeof(float));
-  w.total = w.part + static_cast<size_t>(2) * num_workers * 8 * S4KV_HEAD_DIM * sizeof(float);
+  w.ml = 0;
+  w.part = up(static_cast<size_t>(2) * num_workers * 8 * 2 * sizeof(float));
+  w.tickets = w.part + up(static_cast<size_t>(2) * num_workers * 8 * S4KV_HEAD_DIM * sizeof(float));
+  w.total = w.tickets + static_cast<size_t>(batch) * num_kv_heads * sizeof(uint32_t);
   return w;
 }
 
@@ -119,10 +123,6 @@ int launch_records(const uint8_t *src, uint8_t *dst, const int32_t *src_idx, con
   if (cudaGetLastError() != cudaSuccess) return S4KV_ERR_CUDA;
   return S4KV_OK;
 }
-
-int decode_call(const s4kv_cache_t *cache, const void *k_new, const void *v_new, const void *q, int num_q_heads,
-                const int32_t *seq_lens, const int32_t *block_tables, int batch, int max_pages_per_seq,
-                float sm_scale, void *out, void *workspace, size_t workspace_bytes, void *stream);
 
 }  // namespace
 
@@ -218,8 +218,8 @@ int s4kv_decode_attention(const s4kv_cache_t *cache, const void *q, int num_q_he
                           const int32_t *seq_lens, const int32_t *block_tables, int batch,
                           int max_pages_per_seq, float sm_scale, void *out, void *workspace,
                           size_t workspace_bytes, void *stream) {
-  return decode_call(cache, nullptr, nullptr, q, num_q_heads, seq_lens, block_tables, batch, max_pages_per_seq,
-                     sm_scale, out, workspace, workspace_bytes, stream);
+  return s4kv::decode_call(cache, nullptr, nullptr, q, num_q_heads, seq_lens, block_tables, batch,
+                           max_pages_per_seq, sm_scale, out, workspace, workspace_bytes, stream, false);
 }
 
 int s4kv_append_decode(const s4kv_cache_t *cache, const void *k_new, const void *v_new, const void *q,
@@ -227,17 +227,18 @@ int s4kv_append_decode(const s4kv_cache_t *cache, const void *k_new, const void 
                        int max_pages_per_seq, float sm_scale, void *out, void *workspace, size_t workspace_bytes,
                        void *stream) {
   if (batch > 0 && (!k_new || !v_new || !aligned(k_new, 16) || !aligned(v_new, 16))) return S4KV_ERR_INVALID_ARG;
-  return decode_call(cache, k_new, v_new, q, num_q_heads, seq_lens, block_tables, batch, max_pages_per_seq,
-                     sm_scale, out, workspace, workspace_bytes, stream);
+  return s4kv::decode_call(cache, k_new, v_new, q, num_q_heads, seq_lens, block_tables, batch,
+                           max_pages_per_seq, sm_scale, out, workspace, workspace_bytes, stream, false);
 }
 
 }  // extern "C"
 
-namespace {
+namespace s4kv {
 
 int decode_call(const s4kv_cache_t *cache, const void *k_new, const void *v_new, const void *q, int num_q_heads,
                 const int32_t *seq_lens, const int32_t *block_tables, int batch, int max_pages_per_seq,
-                float sm_scale, void *out, void *workspace, size_t workspace_bytes, void *stream) {
+                float sm_scale, void *out, void *workspace, size_t workspace_bytes, void *stream,
+                bool clear_tickets) {
   int rc = check_cache(cache);
   if (rc != S4KV_OK) return rc;
   rc = s4kv_check_model(cache->head_dim, cache->page_tokens, num_q_heads, cache->num_kv_heads);
@@ -255,6 +256,12 @@ int decode_call(const s4kv_cache_t *cache, const void *k_new, const void *v_new,
   const int fi = fmt_index(cache_bits(cache));
   if (workspace == nullptr || workspace_bytes < w.total || !aligned(workspace, 16)) return S4KV_ERR_WORKSPACE;
   uint8_t *ws = static_cast<uint8_t *>(workspace);
+  // every argument has been checked: only now may the tickets be cleared
+  if (clear_tickets && cudaMemsetAsync(ws + w.tickets, 0, w.total - w.tickets, static_cast<cudaStream_t>(stream)) !=
+                           cudaSuccess) {
+    cudaGetLastError();
+    return S4KV_ERR_CUDA;
+  }
   DecodeParams p;
   p.pool = static_cast<const uint8_t *>(cache->pool);
   p.res_k = static_cast<const __half *>(cache->res_k);
@@ -283,7 +290,7 @@ int decode_call(const s4kv_cache_t *cache, const void *k_new, const void *v_new,
   return S4KV_OK;
 }
 
-}  // namespace
+}  // namespace s4kv
 
 extern "C" {
 

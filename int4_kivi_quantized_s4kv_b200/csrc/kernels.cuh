@@ -96,4 +96,13 @@ int decode_warps_per_cta();
 cudaError_t prepare_decode_kernel();
 size_t decode_smem_bytes(int bits);
 
+// Host entry of every decode call (plain, fused append, no-alloc): checks all
+// arguments, then -- only when they pass and clear_tickets is set -- zeroes
+// the workspace's ticket words on `stream`, then launches.  Returns an
+// S4KV_* status; an invalid call touches nothing.
+int decode_call(const s4kv_cache_t *cache, const void *k_new, const void *v_new, const void *q, int num_q_heads,
+                const int32_t *seq_lens, const int32_t *block_tables, int batch, int max_pages_per_seq,
+                float sm_scale, void *out, void *workspace, size_t workspace_bytes, void *stream,
+                bool clear_tickets);
+
 }  // namespace s4kv

@@ -401,6 +401,9 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(const PrefillPara
   SeqRows sr;
   if (!seq_rows(p, b, tile == 0 && h == 0 && tid == 0, sr)) return;
   const int c_lo = sr.c_lo, n = sr.n, L = sr.L;
+  // more rows than max_new_per_seq sized the grid for: the rows past the
+  // last tile are not computed, which the caller learns from the flag
+  if (tile == 0 && h == 0 && tid == 0 && n > static_cast<int>(gridDim.x) * Tq) flag_error(p.err, S4KV_EFLAG_SEQ_LEN);
   const int t0 = tile * Tq;
   if (t0 >= n) return;
   const int tq = min(Tq, n - t0);

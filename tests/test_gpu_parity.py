@@ -188,3 +188,25 @@ def test_host_validation_launches_nothing():
     assert e.value.status == S.ERR_UNSUPPORTED
     torch.cuda.synchronize()
     assert S.s4kv_get_error(c) == 0
+
+
+def test_workspace_sized_for_a_large_batch_serves_smaller_ones():
+    """One zero-filled workspace sized for the largest batch, reused by calls
+    with fewer sequences and then more: every call must read zero tickets and
+    agree with the oracle (the partial results of a small call must never be
+    read as tickets by a larger one)."""
+    import torch
+    import int4_kivi_quantized_s4kv_b200 as S
+    spec = W.scaled(W.SPECS["llama3.1-8b"], batch=24, ctx_scale=1 / 16)   # 8 kv heads, 512+1 tokens
+    p = Pair(spec)
+    ref = p.oracle_decode()
+    ws = S.decode_workspace(spec.batch, spec.num_kv_heads)
+    q = p._dev(p.q)
+    lens = p._dev(p.lens)
+    for nb in (2, 24, 5, 24, 1):
+        out = torch.full_like(q[:nb], float("nan"))
+        S.s4kv_decode_attention(p.gpu, q[:nb].contiguous(), lens[:nb].contiguous(), p.bt_dev[:nb].contiguous(),
+                                out, ws)
+        torch.cuda.synchronize()
+        assert_attention_close(out.float().cpu().numpy(), ref[:nb], f"batch {nb} on a batch-24 workspace")
+    assert S.s4kv_get_error(p.gpu) == 0

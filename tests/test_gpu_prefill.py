@@ -167,3 +167,28 @@ def test_prefill_leaves_rows_of_no_sequence_untouched():
     assert np.isnan(got[n:]).all()
     ref = case.oc.prefill_attention(case.q, case.cu, case.after.astype(np.int32), case.bt)
     assert_attention_close(got[:n], ref, "prefill with trailing rows")
+
+
+def test_prefill_flags_a_chunk_longer_than_max_new_per_seq():
+    """A chunk longer than the host bound max_new_per_seq (which sizes the
+    grid) is reported through S4KV_EFLAG_SEQ_LEN; the rows the grid covers
+    are still computed, the others are left untouched."""
+    import torch
+    case = PrefillCase(86, 1, 4, before=[10, 0], after=[50, 300])   # chunks of 40 and 300 rows
+    S = case.S
+    qd = case.dev(case.q)
+    out = torch.full_like(qd, float("nan"))
+    bound = 40                                    # one 32-row query tile at G = 4 covers 32 rows
+    S.s4kv_prefill_attention(case.gpu, qd, case.dev(case.cu), case.dev(case.after.astype(np.int32)), case.bt_dev,
+                             out, bound)
+    torch.cuda.synchronize()
+    flags = S.s4kv_get_error(case.gpu)
+    assert flags & 4, flags                       # S4KV_EFLAG_SEQ_LEN
+    got = out.float().cpu().numpy()
+    ref = case.oc.prefill_attention(case.q, case.cu, case.after.astype(np.int32), case.bt)
+    tiles = -(-bound // 32)
+    covered = np.concatenate([np.arange(case.cu[b], case.cu[b] + min(int(case.n[b]), 32 * tiles))
+                              for b in range(2)])
+    assert_attention_close(got[covered], ref[covered], "prefill rows the grid covers")
+    rest = np.setdiff1d(np.arange(int(case.cu[-1])), covered)
+    assert rest.size > 0 and np.isnan(got[rest]).all()

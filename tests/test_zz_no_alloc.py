@@ -54,14 +54,32 @@ def test_noalloc_matches_workspace_entry_point_twice():
 
 
 def test_noalloc_rejects_batches_beyond_its_scratch():
+    """A batch whose decode workspace would not fit in the fixed scratch is
+    refused by a size query alone; no call is made with addresses that are
+    not real device memory."""
     import int4_kivi_quantized_s4kv_b200 as S
+    huge = 10_000_000
+    assert S.s4kv_decode_workspace_size(huge, 8) > S.NOALLOC_SCRATCH_BYTES
+    assert S.s4kv_decode_workspace_size(64, 8) <= S.NOALLOC_SCRATCH_BYTES
+
+
+def test_noalloc_checks_every_argument_before_touching_the_scratch():
+    """An unsupported code width is refused before the scratch is cleared or
+    anything is launched; the cache and the buffers are real, so nothing
+    could read outside them even if the refusal were missing."""
+    import torch
+    import int4_kivi_quantized_s4kv_b200 as S
+    spec = W.scaled(W.SPECS["llama3.2-3b-step"], batch=4, layers=1)
+    p = Pair(spec)
+    q = torch.from_numpy(p.q).cuda()
+    out = torch.full_like(q, float("nan"))
     L = S.lib()
     P = ctypes.c_void_p
-    fake = 0x100000   # never dereferenced: the call must be refused first
-    huge = 10_000_000
-    c = S.s4kv_cache_t(fake, fake, fake, None, 10, 8, huge, 128, 16)
-    need = S.s4kv_decode_workspace_size(huge, 8)
-    assert need > S.NOALLOC_SCRATCH_BYTES
-    rc = L.s4kv_decode_attention_noalloc(ctypes.byref(c), P(fake), 32, P(fake), P(fake), huge, 1,
-                                         0.088, P(fake), None)
-    assert rc == S.ERR_WORKSPACE
+    bad = S.s4kv_cache_t.from_buffer_copy(p.gpu.c)
+    bad.bits = 3
+    rc = L.s4kv_decode_attention_noalloc(ctypes.byref(bad), P(q.data_ptr()), q.shape[1],
+                                         P(torch.from_numpy(p.lens).cuda().data_ptr()), P(p.bt_dev.data_ptr()),
+                                         spec.batch, p.bt_dev.shape[1], 0.088, P(out.data_ptr()), None)
+    torch.cuda.synchronize()
+    assert rc == S.ERR_UNSUPPORTED
+    assert torch.isnan(out).all()
