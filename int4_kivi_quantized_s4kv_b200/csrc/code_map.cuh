@@ -7,21 +7,24 @@
 
 #include <cstdint>
 
+#include "common.cuh"
+
 namespace s4kv {
 
 // The code at 4-bit position (word, nibble): that nibble, or with 8-bit
 // codes the byte holding the same fragment place (tile 4*(word/128) +
-// word%4, lane (word/4)%32, register nibble%4, half nibble/4), or with 2-bit
-// codes the bit pair holding it.
+// word%4, lane (word/4)%32, register reg_of_nibble(nibble), half
+// half_of_nibble(nibble)), or with 2-bit codes the bit pair holding it.
 __device__ __forceinline__ uint32_t code_at(const uint8_t *region, int word, int nibble, int bits) {
+  const int r = reg_of_nibble(nibble), e = half_of_nibble(nibble);
   if (bits == 8) {
     const int tile = 4 * (word >> 7) + (word & 3), lane = (word >> 2) & 31;
-    return region[((tile >> 1) * 32 + lane) * 16 + (tile & 1) * 8 + 2 * (nibble & 3) + (nibble >> 2)];
+    return region[((tile >> 1) * 32 + lane) * 16 + (tile & 1) * 8 + 2 * r + e];
   }
   if (bits == 2) {
     const int tile = 4 * (word >> 7) + (word & 3), lane = (word >> 2) & 31;
     const uint32_t w = reinterpret_cast<const uint32_t *>(region)[4 * lane + (tile >> 1)];
-    return (w >> (16 * (nibble >> 2) + 2 * (4 * (tile & 1) + (nibble & 3)))) & 3u;
+    return (w >> (16 * e + 2 * (4 * (tile & 1) + r))) & 3u;
   }
   const uint32_t w = reinterpret_cast<const uint32_t *>(region)[word];
   return (w >> (4 * nibble)) & 0xFu;
@@ -32,12 +35,12 @@ __device__ __forceinline__ uint32_t code_at(const uint8_t *region, int word, int
 __device__ __forceinline__ void key_position(int t, int c, int &word, int &nibble) {
   const int ki = c >> 5, kt = (c & 31) >> 2, ke = c & 3;
   word = 128 * (kt >> 2) + 4 * (4 * (t & 7) + ki) + (kt & 3);
-  nibble = (t >> 3) + 2 * (ke >> 1) + 4 * (ke & 1);
+  nibble = nibble_of((t >> 3) + 2 * (ke >> 1), ke & 1);
 }
 __device__ __forceinline__ void value_position(int t, int c, int &word, int &nibble) {
   const int vn = (c & 31) >> 2, ve = c & 3, vm = 2 * (c >> 5) + (ve >> 1);
   word = 128 * (vm >> 2) + 4 * (4 * vn + ((t & 7) >> 1)) + (vm & 3);
-  nibble = (ve & 1) + 2 * (t >> 3) + 4 * (t & 1);
+  nibble = nibble_of((ve & 1) + 2 * (t >> 3), t & 1);
 }
 
 // Slot of channel c's key zero point (stored in MMA k order).

@@ -21,7 +21,8 @@ constexpr int kVZeroOff = 2688;
 
 // Block layout of one (page, kv head) with kBits-bit codes (2, 4 or 8): K codes,
 // V codes, K scale fp16 [128], K zero fp16 [128] (MMA k order), V scale fp16
-// [4][16], V zero fp16 [4][16].  Fmt<4> is the 2816-byte int4 block above.
+// [64] (lane-major, value_scale_slot), V zero fp16 [4][16].  Fmt<4> is the
+// 2816-byte int4 block above.
 // 8-bit codes keep the int4 assignment of (token, channel) to MMA operand
 // fragments with bytes for nibbles: a lane's 8 codes of one tile are 8
 // consecutive bytes (register r at bytes 2r, 2r + 1) and the 16 bytes of
@@ -104,21 +105,57 @@ __device__ __forceinline__ __half2 u32_as_h2(uint32_t u) {
   return *reinterpret_cast<__half2 *>(&u);
 }
 
-// Four 4-bit codes of a packed word -> the four f16x2 registers of one lane's
-// m16n8k16 operand fragment.  Nibble j goes to register j & 3, half j >> 2.
-// A nibble at bits 0-3 of a half becomes fp16 1024 + c (exponent fixed by the
-// 0x6400 pattern); at bits 4-7 it becomes 1024 + 16c.  The offset and the
-// factor 16 are removed exactly in fp16.
-__device__ __forceinline__ void unpack_codes(uint32_t w, uint32_t &a0, uint32_t &a1,
-                                             uint32_t &a2, uint32_t &a3) {
-  const uint32_t w8 = w >> 8;
-  const __half2 k1024 = u32_as_h2(0x64006400u);   // 1024
-  const __half2 k16th = u32_as_h2(0x2C002C00u);   // 1/16
-  const __half2 kneg64 = u32_as_h2(0xD400D400u);  // -64
-  a0 = h2_as_u32(__hsub2(u32_as_h2(and_or(w, 0x000F000Fu, 0x64006400u)), k1024));
-  a1 = h2_as_u32(__hfma2(u32_as_h2(and_or(w, 0x00F000F0u, 0x64006400u)), k16th, kneg64));
-  a2 = h2_as_u32(__hsub2(u32_as_h2(and_or(w8, 0x000F000Fu, 0x64006400u)), k1024));
-  a3 = h2_as_u32(__hfma2(u32_as_h2(and_or(w8, 0x00F000F0u, 0x64006400u)), k16th, kneg64));
+// Place of a code in a lane's m16n8k16 operand fragment (register r, half e)
+// <-> nibble of the lane's packed 32-bit word: the low nibbles of the word's
+// bytes 0-1 are register 0 and those of bytes 2-3 register 2, the high
+// nibbles of bytes 0-1 register 1 and of bytes 2-3 register 3, the lower
+// byte of each pair in the lower half.
+__host__ __device__ constexpr int nibble_of(int r, int e) { return (r & 1) + 2 * e + 4 * (r >> 1); }
+__host__ __device__ constexpr int reg_of_nibble(int j) { return (j & 1) + 2 * (j >> 2); }
+__host__ __device__ constexpr int half_of_nibble(int j) { return (j >> 1) & 1; }
+
+// Position (in halves) of the value scale of (token t, group g): lane quad
+// i = (t%8)/2 reads the token pairs 2i + 8e, 2i + 8e + 1 (e = t/8) of all four
+// groups as 32 consecutive bytes.
+__host__ __device__ constexpr int value_scale_slot(int t, int g) {
+  return 16 * ((t & 7) >> 1) + 8 * (t >> 3) + 2 * g + (t & 1);
+}
+
+// fp8 e4m3 pair -> f16x2, the lower byte into the lower half.  A 4-bit code c
+// in the low nibble of an e4m3 byte (sign and upper exponent bits zero) is
+// c * 2^-9 exactly: codes 0..7 are the subnormals m * 2^-9 and codes 8..15
+// the first normal binade 2^-6 (1 + m/8), whose step is the same 2^-9.
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint16_t x) {
+  uint32_t d;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(d) : "h"(x));
+  return d;
+}
+
+// Eight 4-bit codes of a packed word -> the four f16x2 registers of one
+// lane's m16n8k16 operand fragment, each value code * 2^-9 (exact): the low
+// and the high nibble of every byte masked into bytes of their own (one
+// shift, two LOP3), then one conversion per byte pair.
+__device__ __forceinline__ void unpack_codes_s9(uint32_t w, uint32_t &a0, uint32_t &a1, uint32_t &a2,
+                                                uint32_t &a3) {
+  const uint32_t lo = w & 0x0F0F0F0Fu, hi = (w >> 4) & 0x0F0F0F0Fu;
+  uint16_t l0, l1, h0, h1;
+  asm("mov.b32 {%0,%1}, %2;" : "=h"(l0), "=h"(l1) : "r"(lo));
+  asm("mov.b32 {%0,%1}, %2;" : "=h"(h0), "=h"(h1) : "r"(hi));
+  a0 = e4m3x2_to_f16x2(l0);
+  a1 = e4m3x2_to_f16x2(h0);
+  a2 = e4m3x2_to_f16x2(l1);
+  a3 = e4m3x2_to_f16x2(h1);
+}
+
+// The same registers holding the codes themselves (the exact factor 512
+// applied in fp16).
+__device__ __forceinline__ void unpack_codes(uint32_t w, uint32_t &a0, uint32_t &a1, uint32_t &a2, uint32_t &a3) {
+  unpack_codes_s9(w, a0, a1, a2, a3);
+  const __half2 k512 = u32_as_h2(0x60006000u);
+  a0 = h2_as_u32(__hmul2(u32_as_h2(a0), k512));
+  a1 = h2_as_u32(__hmul2(u32_as_h2(a1), k512));
+  a2 = h2_as_u32(__hmul2(u32_as_h2(a2), k512));
+  a3 = h2_as_u32(__hmul2(u32_as_h2(a3), k512));
 }
 
 // One lane's 8-bit tile fragment (two words, registers 0-1 in w0 and 2-3 in

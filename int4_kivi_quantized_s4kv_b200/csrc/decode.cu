@@ -17,29 +17,35 @@
 //    produces partial (m, l, O) results; the worker that finishes a
 //    segment's last piece (an atomic ticket per segment) merges them with a
 //    log-sum-exp and writes the output, then resets the ticket.
-//  * Staging.  Each warp owns a ring of shared-memory stages; lane 0 issues
-//    one 1-D bulk copy (TMA engine, no multicast) of a whole 2816-byte page
-//    block per stage, gathered through block_tables, completing on an
-//    mbarrier.  Waits are bounded and report a timeout through err_flag.
+//  * Staging.  Each warp owns a ring of shared-memory stages, one page block
+//    each, filled by 1-D bulk copies (TMA engine, no multicast) gathered
+//    through block_tables and completing on one mbarrier per stage.  The
+//    consumer takes pages two at a time: one vote waits for both stages, and
+//    lanes 0 and 1 refill both released stages with one copy instruction.
+//    Waits are bounded and report a timeout through err_flag.
 //  * Math.  Per page (16 tokens) and kv head, with tokens on the MMA's M, the
 //    G <= 8 query heads on N and channels on K:
-//      S = codes_K . (q * sK) + zK . q              (3 m16n8k16 per k-tile)
+//      S = codes_K . (q * sK) + zK . q
 //    and, with channels on M and tokens on K,
-//      O += codes_V^T . (P * sV) + [zV rows] . P    (per M-tile, plus 2 for z)
+//      O += codes_V^T . (P * sV) + [zV rows] . P
 //    The per-channel key scale and per-token value scale multiply the small
 //    operand, so the 4-bit codes (exact in fp16) feed the tensor cores
 //    directly; each scaled operand is split into fp16 hi + lo parts whose sum
 //    is exact (q and sK, P-hi and sV are fp16, their product fits in two
-//    halves), giving fp32-level accuracy.  The packed page layout makes each
-//    lane's 32-bit code word its own operand fragment (one 16-byte shared
-//    load per 4 tiles, 1 shift + 4 LOP3 + 4 fp16 ops to unpack 8 codes).
-//    The softmax is an online update in the exp2 domain whose reference
-//    only moves when a page's maximum passes it (with a headroom of 4, so
-//    every weight stays <= 1 and no fp16 operand can overflow); P is moved
-//    from the QK accumulator layout to the PV operand layout with movmatrix.
-//  * Pipelining.  Within a warp, the QK MMAs of page j+2, the softmax of page
-//    j+1 and the PV MMAs of page j are issued in one straight-line block, so
-//    the softmax's shuffle/exp latency overlaps tensor-core work.
+//    halves), giving fp32-level accuracy.  A lane's packed 32-bit code word is
+//    its own operand fragment: the low and high nibbles of its bytes are
+//    masked apart and each byte pair converted as an fp8 e4m3 pair, which
+//    yields code * 2^-9 exactly (1 shift, 2 LOP3 and 4 conversions per 8
+//    codes); the factor 512 is restored in fp32.  The key zero-point terms of
+//    a page pair come from one MMA per k-tile (rows 0-7 one page's zeros,
+//    rows 8-15 the other's).  The softmax is an online update in the exp2
+//    domain whose reference only moves when a maximum passes it (with a
+//    headroom of 4, so every weight stays <= 1 and no fp16 operand can
+//    overflow); P is moved from the QK accumulator layout to the PV operand
+//    layout with movmatrix.
+//  * Pipelining.  Within a warp, the QK MMAs of page pair k+1, the PV MMAs of
+//    pair k and the softmax of pair k+1 are issued in one straight-line
+//    block, so the softmax's latency overlaps tensor-core work.
 #include <cfloat>
 
 #include "kernels.cuh"
@@ -71,16 +77,9 @@ constexpr long long kWaitLimitCycles = 2000000000LL;  // about one second
 constexpr unsigned kFull = 0xFFFFFFFFu;
 constexpr float kHeadroom = 4.0f;  // log2 headroom of the softmax reference
 
-// Query fragments of the current piece can live in a per-warp shared slice
-// ([4 k-tile pairs][32 lanes][16 B]) instead of 16 registers per lane.
-#ifndef S4KV_Q_IN_SMEM
-#define S4KV_Q_IN_SMEM 0
-#endif
-constexpr int kQBytesPerWarp = S4KV_Q_IN_SMEM ? 2048 : 0;
-
 template <int kBits>
 constexpr size_t smem_bytes_for() {
-  return static_cast<size_t>(kWarpsPerCta) * (stages_for<kBits>() * (Fmt<kBits>::kBlock + 8) + kQBytesPerWarp);
+  return static_cast<size_t>(kWarpsPerCta) * stages_for<kBits>() * (Fmt<kBits>::kBlock + 8);
 }
 
 size_t decode_smem_bytes(int bits) {
@@ -137,44 +136,33 @@ struct Online {
   float Z[4];        // value zero-point term: sum_t zV[g][t] P[t][h]
 };
 
-// Per-lane shared addresses of one stage: the stage base plus this lane's
-// offset into the code words (16*lane), the key scale/zero rows (64*i), the
-// value scale pairs (4*i) and the value zero rows (32*(n%4) + 4*i).
-// The two zero-point operands are broadcast rows, fetched with ldmatrix:
-// kzero = this lane's row address in the key zero points (lanes 16..31 read
-// k columns 8..15), vzero = this lane's row address in the value zero points
-// (row r of the operand holds group r % 4).
-struct StageAddr {
-  uint32_t code, kmeta, vscale, kzero, vzero;
+// Per-lane byte offsets inside a stage: the lane's 16 bytes of code words
+// (16*lane), its key-scale run (64*i: channels 32i .. 32i+31), its value-scale
+// run (32*i: token pairs 2i, 2i+8 of the four groups), its row of the value
+// zero points for ldmatrix (row r of the operand holds group r % 4; lanes
+// 16..31 read tokens 8..15) and its row of the key zero points (lanes 16..31
+// read k columns 8..15).
+struct LaneOff {
+  uint32_t code, kmeta, vscale, vzero, kzero;
 };
 
 template <int kBits>
-__device__ __forceinline__ StageAddr stage_addr_of(uint32_t stage_base, int lane) {
-  const int i = lane & 3;
-  const uint32_t half_k = (lane >> 4) ? 16u : 0u;
-  return StageAddr{stage_base + 16u * lane, stage_base + 64u * i, stage_base + 4u * i,
-                   stage_base + Fmt<kBits>::kKZero + half_k,
-                   stage_base + Fmt<kBits>::kVZero + 32u * ((lane & 7) & 3) + half_k};
+__device__ __forceinline__ LaneOff lane_offsets(int lane) {
+  using F = Fmt<kBits>;
+  const uint32_t i = lane & 3, half_k = (lane >> 4) ? 16u : 0u;
+  return LaneOff{16u * lane, F::kKScale + 64u * i, F::kVScale + 32u * i, F::kVZero + 32u * (lane & 3) + half_k,
+                 F::kKZero + half_k};
 }
 
-// Logits of one quantized page: this lane's S^T[tokens n, n+8][heads 2i,
-// 2i+1] before scaling.
-// Query fragments of this lane: in registers, or in the warp's shared slice.
+// Query fragments of this lane (B operand of the QK MMAs: channels 32i ..
+// 32i + 31, head n).
 struct QFrag {
-#if S4KV_Q_IN_SMEM
-  uint32_t addr;  // this lane's 16 B in k-tile pair 0; pair m at + 512 m
-  __device__ __forceinline__ uint4 pair(int m) const { return m == 0 ? lds128<0>(addr) : m == 1 ? lds128<512>(addr) : m == 2 ? lds128<1024>(addr) : lds128<1536>(addr); }
-#else
   uint32_t w[16];
   __device__ __forceinline__ uint4 pair(int m) const { return make_uint4(w[4 * m], w[4 * m + 1], w[4 * m + 2], w[4 * m + 3]); }
-#endif
 };
 
 // Key zero-point operand of k-tile kt (kt is a constant after unrolling, so
-// the switch folds to one ldmatrix with an immediate offset).  Its rows are
-// all the same, so two of the four registers repeat the other two; they are
-// loaded as such, because an MMA's A operand must sit in four consecutive
-// registers and one register passed twice would cost copies.
+// the switch folds to one ldmatrix with an immediate offset).
 __device__ __forceinline__ void ldmatrix_kzero(uint32_t base, int kt, uint32_t &z0, uint32_t &z1, uint32_t &z2,
                                                uint32_t &z3) {
   switch (kt) {
@@ -190,8 +178,9 @@ __device__ __forceinline__ void ldmatrix_kzero(uint32_t base, int kt, uint32_t &
 }
 
 // Operand fragment of key / value tile kt of a quantized page (kt constant
-// after unrolling): one 4-bit code word, or two 8-bit words of the chunk
-// that holds tiles 2m, 2m + 1 of this lane.
+// after unrolling): one 4-bit code word (values code * 2^-9), or two 8-bit
+// words of the chunk that holds tiles 2m, 2m + 1 of this lane, or the 2-bit
+// word of tiles 2m, 2m + 1.
 template <int kBits>
 __device__ __forceinline__ void tile_fragment(const uint32_t (&w)[8], int kt, uint32_t &a0, uint32_t &a1,
                                               uint32_t &a2, uint32_t &a3) {
@@ -199,111 +188,149 @@ __device__ __forceinline__ void tile_fragment(const uint32_t (&w)[8], int kt, ui
   else if (kBits == 2) {
     if (kt & 1) unpack_codes2<1>(w[kt >> 1], a0, a1, a2, a3);
     else unpack_codes2<0>(w[kt >> 1], a0, a1, a2, a3);
-  } else unpack_codes(w[kt], a0, a1, a2, a3);
+  } else unpack_codes_s9(w[kt], a0, a1, a2, a3);
+}
+
+// What the code operand's values must be multiplied by to give the codes:
+// 4-bit codes enter the MMAs as code * 2^-9.
+template <int kBits>
+__host__ __device__ constexpr float code_unit_inv() { return kBits == 4 ? 512.0f : 1.0f; }
+
+// The key code words of a page for the whole QK (4- and 2-bit codes; 8-bit
+// codes are loaded per k-tile pair).
+template <int kBits>
+__device__ __forceinline__ void load_key_words(uint32_t code, uint32_t (&kw)[8]) {
+  using F = Fmt<kBits>;
+  if (kBits == 4) {
+    const uint4 w0 = lds128<F::kKCode>(code), w1 = lds128<F::kKCode + 512>(code);
+    kw[0] = w0.x; kw[1] = w0.y; kw[2] = w0.z; kw[3] = w0.w;
+    kw[4] = w1.x; kw[5] = w1.y; kw[6] = w1.z; kw[7] = w1.w;
+  } else if (kBits == 2) {
+    const uint4 w0 = lds128<F::kKCode>(code);
+    kw[0] = w0.x; kw[1] = w0.y; kw[2] = w0.z; kw[3] = w0.w;
+  }
 }
 
 template <int kBits>
-__device__ __forceinline__ void qk_page(const StageAddr &a, const QFrag &q, float (&S)[4]) {
+__device__ __forceinline__ void load_key_words8(uint32_t code, int m, uint32_t (&kw)[8]) {
   using F = Fmt<kBits>;
-  // three independent accumulators (hi part, lo part, zero-point term) keep
-  // the dependent MMA chains 8 deep instead of 24
-  float Sh[4] = {0.f, 0.f, 0.f, 0.f}, Sl[4] = {0.f, 0.f, 0.f, 0.f}, Sz[4] = {0.f, 0.f, 0.f, 0.f};
-  // Sl and Sz both collect small terms (lo parts, zero points); even k-tiles
-  // put their lo part in Sl and zero point in Sz, odd k-tiles the reverse,
-  // so the two chains stay balanced and S = Sh + (Sl + Sz).
-  // 4-bit: all 8 tiles' words in two 16-byte loads; 8-bit: tiles 2m, 2m+1
-  // per 16-byte load, inside the loop
-  uint32_t kws[8];
-  if (kBits == 4) {
-    const uint4 kw0 = lds128<F::kKCode>(a.code);
-    const uint4 kw1 = lds128<F::kKCode + 512>(a.code);
-    kws[0] = kw0.x; kws[1] = kw0.y; kws[2] = kw0.z; kws[3] = kw0.w;
-    kws[4] = kw1.x; kws[5] = kw1.y; kws[6] = kw1.z; kws[7] = kw1.w;
-  } else if (kBits == 2) {  // all 8 tiles' codes in one 16-byte load
-    const uint4 kw0 = lds128<F::kKCode>(a.code);
-    kws[0] = kw0.x; kws[1] = kw0.y; kws[2] = kw0.z; kws[3] = kw0.w;
+  if (kBits == 8) {
+    const uint4 cw = m == 0 ? lds128<F::kKCode>(code) : m == 1 ? lds128<F::kKCode + 512>(code)
+                   : m == 2 ? lds128<F::kKCode + 1024>(code) : lds128<F::kKCode + 1536>(code);
+    kw[0] = cw.x; kw[1] = cw.y; kw[2] = cw.z; kw[3] = cw.w;
   }
+}
+
+// One k-tile of one page's codes against q * sK (hi and lo parts into their
+// own accumulators).
+template <int kBits>
+__device__ __forceinline__ void qk_tile(const uint32_t (&kw)[8], int kt, uint32_t s0w, uint32_t s1w, uint32_t q0w,
+                                        uint32_t q1w, float (&Sh)[4], float (&Sl)[4]) {
+  uint32_t a0, a1, a2, a3;
+  tile_fragment<kBits>(kw, kt, a0, a1, a2, a3);
+  const __half2 qb0 = u32_as_h2(q0w), qb1 = u32_as_h2(q1w);
+  const __half2 s0 = u32_as_h2(s0w), s1 = u32_as_h2(s1w);
+  // q * sK split into fp16 hi + lo; the lo part is the exact remainder
+  const __half2 h0 = __hmul2(qb0, s0), h1 = __hmul2(qb1, s1);
+  const __half2 r0 = __hfma2(qb0, s0, __hneg2(h0));
+  const __half2 r1 = __hfma2(qb1, s1, __hneg2(h1));
+  mma16816(Sh, a0, a1, a2, a3, h2_as_u32(h0), h2_as_u32(h1));
+  mma16816(Sl, a0, a1, a2, a3, h2_as_u32(r0), h2_as_u32(r1));
+}
+
+// Logits of two quantized pages A and B (stage byte addresses sa, sb; B may
+// be A again): this lane's S^T[tokens n, n+8][heads 2i, 2i+1] of each page,
+// before sm_scale.  zrow: this lane's key-zero row address (page A's stage for
+// lanes 0-7 and 16-23, page B's for lanes 8-15 and 24-31), so that one MMA
+// per k-tile gives page A's zero-point terms in rows 0-7 and page B's in rows
+// 8-15.
+template <int kBits>
+__device__ __forceinline__ void qk_pair(uint32_t sa, uint32_t sb, uint32_t zrow, const LaneOff &lo, const QFrag &q,
+                                        float (&SA)[4], float (&SB)[4]) {
+  using F = Fmt<kBits>;
+  float ShA[4] = {0.f, 0.f, 0.f, 0.f}, SlA[4] = {0.f, 0.f, 0.f, 0.f};
+  float ShB[4] = {0.f, 0.f, 0.f, 0.f}, SlB[4] = {0.f, 0.f, 0.f, 0.f};
+  float Sz[4] = {0.f, 0.f, 0.f, 0.f};
+  const uint32_t ca = sa + lo.code, cb = sb + lo.code, ma = sa + lo.kmeta, mb = sb + lo.kmeta;
+  uint32_t kwa[8], kwb[8];
+  load_key_words<kBits>(ca, kwa);
+  load_key_words<kBits>(cb, kwb);
 #pragma unroll
   for (int m = 0; m < 4; ++m) {
-    if (kBits == 8) {
-      const uint4 cw = m == 0 ? lds128<F::kKCode>(a.code) : m == 1 ? lds128<F::kKCode + 512>(a.code)
-                     : m == 2 ? lds128<F::kKCode + 1024>(a.code) : lds128<F::kKCode + 1536>(a.code);
-      kws[0] = cw.x; kws[1] = cw.y; kws[2] = cw.z; kws[3] = cw.w;
-    }
+    load_key_words8<kBits>(ca, m, kwa);
+    load_key_words8<kBits>(cb, m, kwb);
     // key scales and query words for k-tiles 2m, 2m+1 (four channel pairs)
-    const uint4 sv = m == 0 ? lds128<F::kKScale>(a.kmeta) : m == 1 ? lds128<F::kKScale + 16>(a.kmeta)
-                   : m == 2 ? lds128<F::kKScale + 32>(a.kmeta) : lds128<F::kKScale + 48>(a.kmeta);
+    const uint4 sva = m == 0 ? lds128<0>(ma) : m == 1 ? lds128<16>(ma) : m == 2 ? lds128<32>(ma) : lds128<48>(ma);
+    const uint4 svb = m == 0 ? lds128<0>(mb) : m == 1 ? lds128<16>(mb) : m == 2 ? lds128<32>(mb) : lds128<48>(mb);
     const uint4 qv = q.pair(m);
-    const uint32_t sk[4] = {sv.x, sv.y, sv.z, sv.w};
+    const uint32_t ska[4] = {sva.x, sva.y, sva.z, sva.w}, skb[4] = {svb.x, svb.y, svb.z, svb.w};
     const uint32_t qw[4] = {qv.x, qv.y, qv.z, qv.w};
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       const int kt = 2 * m + h;
-      uint32_t a0, a1, a2, a3;
-      tile_fragment<kBits>(kws, kt, a0, a1, a2, a3);
-      const __half2 qb0 = u32_as_h2(qw[2 * h]), qb1 = u32_as_h2(qw[2 * h + 1]);
-      const __half2 s0 = u32_as_h2(sk[2 * h]), s1 = u32_as_h2(sk[2 * h + 1]);
-      // q * sK split into fp16 hi + lo; the lo part is the exact remainder
-      const __half2 h0 = __hmul2(qb0, s0), h1 = __hmul2(qb1, s1);
-      const __half2 r0 = __hfma2(qb0, s0, __hneg2(h0));
-      const __half2 r1 = __hfma2(qb1, s1, __hneg2(h1));
-      mma16816(Sh, a0, a1, a2, a3, h2_as_u32(h0), h2_as_u32(h1));
-      mma16816(h ? Sz : Sl, a0, a1, a2, a3, h2_as_u32(r0), h2_as_u32(r1));
-      // key zero point: every A row is zK, so each row gets sum_c zK q
+      qk_tile<kBits>(kwa, kt, ska[2 * h], ska[2 * h + 1], qw[2 * h], qw[2 * h + 1], ShA, SlA);
+      qk_tile<kBits>(kwb, kt, skb[2 * h], skb[2 * h + 1], qw[2 * h], qw[2 * h + 1], ShB, SlB);
+      // key zero points: A rows 0-7 are page A's zK, rows 8-15 page B's
       uint32_t z0, z1, z2, z3;
-      ldmatrix_kzero(a.kzero, 2 * m + h, z0, z1, z2, z3);
-      mma16816(h ? Sl : Sz, z0, z1, z2, z3, qw[2 * h], qw[2 * h + 1]);
+      ldmatrix_kzero(zrow, kt, z0, z1, z2, z3);
+      mma16816(Sz, z0, z1, z2, z3, qw[2 * h], qw[2 * h + 1]);
     }
   }
-  const float2 s01 = add2(add2(make_float2(Sh[0], Sh[1]), make_float2(Sl[0], Sl[1])), make_float2(Sz[0], Sz[1]));
-  const float2 s23 = add2(add2(make_float2(Sh[2], Sh[3]), make_float2(Sl[2], Sl[3])), make_float2(Sz[2], Sz[3]));
-  S[0] = s01.x;
-  S[1] = s01.y;
-  S[2] = s23.x;
-  S[3] = s23.y;
+  (void)F::kBlock;
+  const float cs = code_unit_inv<kBits>();
+  const float2 c2 = make_float2(cs, cs);
+  const float2 za = make_float2(Sz[0], Sz[1]), zb = make_float2(Sz[2], Sz[3]);
+  const float2 a01 = fma2(add2(make_float2(ShA[0], ShA[1]), make_float2(SlA[0], SlA[1])), c2, za);
+  const float2 a23 = fma2(add2(make_float2(ShA[2], ShA[3]), make_float2(SlA[2], SlA[3])), c2, za);
+  const float2 b01 = fma2(add2(make_float2(ShB[0], ShB[1]), make_float2(SlB[0], SlB[1])), c2, zb);
+  const float2 b23 = fma2(add2(make_float2(ShB[2], ShB[3]), make_float2(SlB[2], SlB[3])), c2, zb);
+  SA[0] = a01.x; SA[1] = a01.y; SA[2] = a23.x; SA[3] = a23.y;
+  SB[0] = b01.x; SB[1] = b01.y; SB[2] = b23.x; SB[3] = b23.y;
 }
 
-// Online softmax for one 16-token page.  S: this lane's logits (tokens n,
-// n+8; heads 2i, 2i+1).  Writes P^T fragments in the PV operand layout
-// (head n; tokens 2i, 2i+1 and 2i+8, 2i+9) as fp16 hi (P[0], P[1]) and lo
-// (P[2], P[3]) parts.  The reference moves (and the state is rescaled) only
-// when a page maximum passes it, for any lane of the warp.
-__device__ __forceinline__ void softmax_page(const float (&S)[4], float scale_log2, Online &st,
-                                             uint32_t (&P)[4]) {
+// Move the softmax reference when a logit of the page pair passes it (for any
+// lane of the warp): new reference = pair maximum + headroom, state rescaled.
+// m0, m1: this lane's maxima of heads 2i, 2i+1.
+__device__ __forceinline__ void softmax_reference(float m0, float m1, float scale_log2, Online &st) {
   // common case: no logit passes the reference (compared on the raw logits
   // against ref / scale, kept in thr), one vote and no shuffles
-  if (__any_sync(kFull, fmaxf(S[0], S[2]) > st.thr0 || fmaxf(S[1], S[3]) > st.thr1)) {
-    float pm0 = fmaxf(S[0], S[2]) * scale_log2, pm1 = fmaxf(S[1], S[3]) * scale_log2;
+  if (!__any_sync(kFull, m0 > st.thr0 || m1 > st.thr1)) return;
+  float pm0 = m0 * scale_log2, pm1 = m1 * scale_log2;
 #pragma unroll
-    for (int off = 4; off < 32; off <<= 1) {
-      pm0 = fmaxf(pm0, __shfl_xor_sync(kFull, pm0, off));
-      pm1 = fmaxf(pm1, __shfl_xor_sync(kFull, pm1, off));
-    }
-    const float r0 = -st.nref.x, r1 = -st.nref.y;
-    const float n0 = pm0 > r0 ? pm0 + kHeadroom : r0;
-    const float n1 = pm1 > r1 ? pm1 + kHeadroom : r1;
-    const float2 a = make_float2(fast_exp2(r0 - n0), fast_exp2(r1 - n1));
-    st.nref = make_float2(-n0, -n1);
-    // largest raw logit whose weight stays <= 1 (rounded down: never above)
-    st.thr0 = __fdiv_rd(n0, scale_log2);
-    st.thr1 = __fdiv_rd(n1, scale_log2);
-    st.l = mul2(st.l, a);
-#pragma unroll
-    for (int mt = 0; mt < 8; ++mt) {
-      const float2 o01 = mul2(make_float2(st.O[mt][0], st.O[mt][1]), a);
-      const float2 o23 = mul2(make_float2(st.O[mt][2], st.O[mt][3]), a);
-      st.O[mt][0] = o01.x;
-      st.O[mt][1] = o01.y;
-      st.O[mt][2] = o23.x;
-      st.O[mt][3] = o23.y;
-    }
-    const float2 z01 = mul2(make_float2(st.Z[0], st.Z[1]), a);
-    const float2 z23 = mul2(make_float2(st.Z[2], st.Z[3]), a);
-    st.Z[0] = z01.x;
-    st.Z[1] = z01.y;
-    st.Z[2] = z23.x;
-    st.Z[3] = z23.y;
+  for (int off = 4; off < 32; off <<= 1) {
+    pm0 = fmaxf(pm0, __shfl_xor_sync(kFull, pm0, off));
+    pm1 = fmaxf(pm1, __shfl_xor_sync(kFull, pm1, off));
   }
+  const float r0 = -st.nref.x, r1 = -st.nref.y;
+  const float n0 = pm0 > r0 ? pm0 + kHeadroom : r0;
+  const float n1 = pm1 > r1 ? pm1 + kHeadroom : r1;
+  const float2 a = make_float2(fast_exp2(r0 - n0), fast_exp2(r1 - n1));
+  st.nref = make_float2(-n0, -n1);
+  // largest raw logit whose weight stays <= 1 (rounded down: never above)
+  st.thr0 = __fdiv_rd(n0, scale_log2);
+  st.thr1 = __fdiv_rd(n1, scale_log2);
+  st.l = mul2(st.l, a);
+#pragma unroll
+  for (int mt = 0; mt < 8; ++mt) {
+    const float2 o01 = mul2(make_float2(st.O[mt][0], st.O[mt][1]), a);
+    const float2 o23 = mul2(make_float2(st.O[mt][2], st.O[mt][3]), a);
+    st.O[mt][0] = o01.x;
+    st.O[mt][1] = o01.y;
+    st.O[mt][2] = o23.x;
+    st.O[mt][3] = o23.y;
+  }
+  const float2 z01 = mul2(make_float2(st.Z[0], st.Z[1]), a);
+  const float2 z23 = mul2(make_float2(st.Z[2], st.Z[3]), a);
+  st.Z[0] = z01.x;
+  st.Z[1] = z01.y;
+  st.Z[2] = z23.x;
+  st.Z[3] = z23.y;
+}
+
+// Weights of one page against the current reference: P^T fragments in the PV
+// operand layout (head n; tokens 2i, 2i+1 and 2i+8, 2i+9) as fp16 hi (P[0],
+// P[1]) and lo (P[2], P[3]) parts; their fp32 sum goes into l.
+__device__ __forceinline__ void page_weights(const float (&S)[4], float scale_log2, Online &st, uint32_t (&P)[4]) {
   // exponents (S * scale - ref) for (heads 2i, 2i+1) of tokens n and n+8
   const float2 sc = make_float2(scale_log2, scale_log2);
   const float2 x01 = fma2(make_float2(S[0], S[1]), sc, st.nref);
@@ -324,17 +351,32 @@ __device__ __forceinline__ void softmax_page(const float (&S)[4], float scale_lo
   P[3] = movmatrix_trans(h2_as_u32(l23));
 }
 
-// O += V^T P for one quantized page.
+// Online softmax of a page pair.
+__device__ __forceinline__ void softmax_pair(const float (&SA)[4], const float (&SB)[4], float scale_log2, Online &st,
+                                             uint32_t (&PA)[4], uint32_t (&PB)[4]) {
+  const float m0 = fmaxf(fmaxf(SA[0], SA[2]), fmaxf(SB[0], SB[2]));
+  const float m1 = fmaxf(fmaxf(SA[1], SA[3]), fmaxf(SB[1], SB[3]));
+  softmax_reference(m0, m1, scale_log2, st);
+  page_weights(SA, scale_log2, st, PA);
+  page_weights(SB, scale_log2, st, PB);
+}
+
+// Online softmax of one page (the residual page).
+__device__ __forceinline__ void softmax_page(const float (&S)[4], float scale_log2, Online &st, uint32_t (&P)[4]) {
+  softmax_reference(fmaxf(S[0], S[2]), fmaxf(S[1], S[3]), scale_log2, st);
+  page_weights(S, scale_log2, st, P);
+}
+
+// O += V^T P for the two M-tiles of value group G4 of one quantized page.
 template <int kBits, int G4>
-__device__ __forceinline__ void pv_group(const StageAddr &a, const uint32_t (&P)[4], uint32_t (&vws)[8],
-                                         Online &st) {
+__device__ __forceinline__ void pv_group(uint32_t code, const uint32_t (&P)[4], uint32_t sv0w, uint32_t sv1w,
+                                         uint32_t (&vws)[8], Online &st) {
   using F = Fmt<kBits>;
   if (kBits == 8) {  // M-tiles 2 G4, 2 G4 + 1 of this lane: one 16-byte chunk
-    const uint4 cw = lds128<F::kVCode + 512 * G4>(a.code);
+    const uint4 cw = lds128<F::kVCode + 512 * G4>(code);
     vws[0] = cw.x; vws[1] = cw.y; vws[2] = cw.z; vws[3] = cw.w;
   }
-  const __half2 sv0 = u32_as_h2(lds32<F::kVScale + 32 * G4>(a.vscale));
-  const __half2 sv1 = u32_as_h2(lds32<F::kVScale + 32 * G4 + 16>(a.vscale));
+  const __half2 sv0 = u32_as_h2(sv0w), sv1 = u32_as_h2(sv1w);
   // (P * sV) in fp16 hi + lo: P-hi * sV exactly as two halves, plus P-lo * sV
   const __half2 bh0 = __hmul2(u32_as_h2(P[0]), sv0);
   const __half2 bh1 = __hmul2(u32_as_h2(P[1]), sv1);
@@ -350,25 +392,31 @@ __device__ __forceinline__ void pv_group(const StageAddr &a, const uint32_t (&P)
   }
 }
 
+// O += V^T P for one quantized page at stage address s (O in code units:
+// 2^-9 for 4-bit codes), Z += [zV rows] P.
 template <int kBits>
-__device__ __forceinline__ void pv_page(const StageAddr &a, const uint32_t (&P)[4], Online &st) {
+__device__ __forceinline__ void pv_page(uint32_t s, const LaneOff &lo, const uint32_t (&P)[4], Online &st) {
+  using F = Fmt<kBits>;
+  const uint32_t code = s + lo.code;
   uint32_t vws[8];
   if (kBits == 4) {
-    const uint4 vw0 = lds128<Fmt<4>::kVCode>(a.code);
-    const uint4 vw1 = lds128<Fmt<4>::kVCode + 512>(a.code);
+    const uint4 vw0 = lds128<F::kVCode>(code), vw1 = lds128<F::kVCode + 512>(code);
     vws[0] = vw0.x; vws[1] = vw0.y; vws[2] = vw0.z; vws[3] = vw0.w;
     vws[4] = vw1.x; vws[5] = vw1.y; vws[6] = vw1.z; vws[7] = vw1.w;
   } else if (kBits == 2) {
-    const uint4 vw0 = lds128<Fmt<2>::kVCode>(a.code);
+    const uint4 vw0 = lds128<F::kVCode>(code);
     vws[0] = vw0.x; vws[1] = vw0.y; vws[2] = vw0.z; vws[3] = vw0.w;
   }
-  pv_group<kBits, 0>(a, P, vws, st);
-  pv_group<kBits, 1>(a, P, vws, st);
-  pv_group<kBits, 2>(a, P, vws, st);
-  pv_group<kBits, 3>(a, P, vws, st);
+  // this lane's value scales: token pairs 2i (.x-.w: groups 0-3) and 2i + 8
+  const uint32_t vsa = s + lo.vscale;
+  const uint4 s0 = lds128<0>(vsa), s1 = lds128<16>(vsa);
+  pv_group<kBits, 0>(code, P, s0.x, s1.x, vws, st);
+  pv_group<kBits, 1>(code, P, s0.y, s1.y, vws, st);
+  pv_group<kBits, 2>(code, P, s0.z, s1.z, vws, st);
+  pv_group<kBits, 3>(code, P, s0.w, s1.w, vws, st);
   // value zero points: A row r carries group r % 4's zV (one ldmatrix), B = P
   uint32_t z0, z1, z2, z3;
-  ldmatrix_x4<0>(a.vzero, z0, z1, z2, z3);
+  ldmatrix_x4<0>(s + lo.vzero, z0, z1, z2, z3);
   mma16816(st.Z, z0, z1, z2, z3, P[0], P[1]);
   mma16816(st.Z, z0, z1, z2, z3, P[2], P[3]);
 }
@@ -545,10 +593,9 @@ __global__ void __launch_bounds__(kThreads, S4KV_DECODE_MIN_CTAS) decode_kernel(
   const int n = lane >> 2, i = lane & 3;
   const uint32_t ring0 = smem_addr(smem) + warp * kStages * kBlockBytes;
   const uint32_t bar0 = smem_addr(smem) + kWarpsPerCta * kStages * kBlockBytes + warp * kStages * 8;
-  const uint32_t qslice = smem_addr(smem) + kWarpsPerCta * kStages * (kBlockBytes + 8) + warp * kQBytesPerWarp;
-  (void)qslice;
   const long long worker = static_cast<long long>(blockIdx.x) * kWarpsPerCta + warp;
   const int B = p.batch, H = p.num_kv_heads, G = p.group;
+  const LaneOff lo = lane_offsets<kBits>(lane);
 
   if (lane == 0) {
 #pragma unroll
@@ -669,7 +716,7 @@ __global__ void __launch_bounds__(kThreads, S4KV_DECODE_MIN_CTAS) decode_kernel(
     if (!active) return;
   }
 
-  // ---- producer: issue the next quantized page of [s, e) into the ring.
+  // ---- producer: issue the next quantized pages of [s, e) into the ring.
   // It walks the same pieces as the consumer.  The page ids of a piece are
   // read 32 at a time into a window (lane l holds the l-th) with one
   // coalesced load, and taken with a shuffle, so no per-page global load
@@ -696,8 +743,7 @@ __global__ void __launch_bounds__(kThreads, S4KV_DECODE_MIN_CTAS) decode_kernel(
     p_window();
   };
   p_piece();
-  // fills the stage at byte offset `stage` (barrier `bar`): the ring is kept
-  // full, so that is always the stage the consumer released last
+  // issue one copy into `stage` (barrier `bar`)
   auto produce = [&](uint32_t stage, uint32_t bar) {
     while (p_q == 0) {
       if (p_left == 0) return;
@@ -722,7 +768,28 @@ __global__ void __launch_bounds__(kThreads, S4KV_DECODE_MIN_CTAS) decode_kernel(
     }
     ++issued;
   };
-  static_assert(kStages >= 4, "the pipeline holds three stages at once");
+  // issue copies into two stages: lanes 0 and 1 take one each when both
+  // pages are in the current window, otherwise one after the other
+  auto produce2 = [&](uint32_t st_a, uint32_t bar_a, uint32_t st_b, uint32_t bar_b) {
+    if (p_q >= 2 && p_widx <= 30) {
+      int phys = __shfl_sync(kFull, p_win, p_widx + (lane & 1));
+      p_widx += 2;
+      p_q -= 2;
+      const bool bad = static_cast<unsigned>(phys) >= static_cast<unsigned>(p.num_pages);
+      if (bad) phys = 0;
+      if (lane < 2) {
+        if (bad) flag_error(p.err, S4KV_EFLAG_PAGE_RANGE);
+        const uint32_t bar = lane ? bar_b : bar_a;
+        mbar_arrive_expect_tx(bar, kBlockBytes);
+        bulk_copy_g2s(ring0 + (lane ? st_b : st_a), p_head + phys * page_stride, kBlockBytes, bar);
+      }
+      issued += 2;
+    } else {
+      produce(st_a, bar_a);
+      produce(st_b, bar_b);
+    }
+  };
+  static_assert(kStages >= 5, "the pipeline holds four stages at once");
 #pragma unroll 1
   for (int k = 0; k < kStages; ++k) produce(static_cast<uint32_t>(k) * kBlockBytes, bar0 + 8u * k);
 
@@ -740,19 +807,30 @@ __global__ void __launch_bounds__(kThreads, S4KV_DECODE_MIN_CTAS) decode_kernel(
   int consumed = 0;
   bool failed = false;
   Pos c0{0u, bar0, 0u};
-  auto wait_copy = [&](const Pos &q) {
-    if (__all_sync(kFull, mbar_try_wait(q.bar, q.phase))) return true;
-    const bool ok = mbar_wait_bounded(q.bar, q.phase, kWaitLimitCycles);
+  // wait for the copies of stages a and (when `two`) b: lane 1 watches b
+  auto wait_pair = [&](const Pos &a, const Pos &b, bool two) {
+    const bool mine_b = two && (lane & 1);
+    const uint32_t bar = mine_b ? b.bar : a.bar, ph = mine_b ? b.phase : a.phase;
+    if (__all_sync(kFull, mbar_try_wait(bar, ph))) return true;
+    const bool ok = mbar_wait_bounded(bar, ph, kWaitLimitCycles);
     return !__any_sync(kFull, !ok);
   };
-  auto addr = [&](const Pos &q) { return stage_addr_of<kBits>(ring0 + q.off, lane); };
-  auto release = [&]() {      // the page at c0 has been read completely
+  // the key-zero row of this lane for the page pair (a, b)
+  auto zero_row = [&](const Pos &a, const Pos &b) { return ring0 + ((lane & 8) ? b.off : a.off) + lo.kzero; };
+  // the pages at c0 (and the next stage when `two`) have been read completely
+  auto release = [&](bool two) {
     fence_proxy_async();
     __syncwarp();
-    ++consumed;
-    const Pos done = c0;
-    c0 = next_pos(c0);
-    produce(done.off, done.bar);
+    const Pos a = c0, b = next_pos(c0);
+    if (two) {
+      consumed += 2;
+      c0 = next_pos(b);
+      produce2(a.off, a.bar, b.off, b.bar);
+    } else {
+      ++consumed;
+      c0 = b;
+      produce(a.off, a.bar);
+    }
   };
 
   int page = p_first, rem = range;
@@ -777,21 +855,10 @@ __global__ void __launch_bounds__(kThreads, S4KV_DECODE_MIN_CTAS) decode_kernel(
 #pragma unroll
         for (int k = 0; k < 4; ++k) qv[k] = __ldg(qp + k);
       }
-#if S4KV_Q_IN_SMEM
-      qf.addr = qslice + 16u * lane;
-      __syncwarp();  // the previous piece's reads of the slice are done
-#pragma unroll
-      for (int k = 0; k < 4; ++k)
-        asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(qf.addr + 512u * k), "r"(qv[k].x), "r"(qv[k].y),
-                     "r"(qv[k].z), "r"(qv[k].w)
-                     : "memory");
-      __syncwarp();
-#else
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
         qf.w[4 * k] = qv[k].x; qf.w[4 * k + 1] = qv[k].y; qf.w[4 * k + 2] = qv[k].z; qf.w[4 * k + 3] = qv[k].w;
       }
-#endif
     }
     Online st;
     st.nref = make_float2(INFINITY, INFINITY);
@@ -802,73 +869,61 @@ __global__ void __launch_bounds__(kThreads, S4KV_DECODE_MIN_CTAS) decode_kernel(
     st.Z[0] = st.Z[1] = st.Z[2] = st.Z[3] = 0.f;
 
     if (nq > 0) {
-      // software pipeline over the piece's quantized pages: each step issues
-      // QK(j+2), PV(j) and the softmax of page j+1 in one block; two steps
-      // per loop trip swap the roles of the P / S registers
-      uint32_t Pa[4], Pb[4];
-      float Sa[4], Sb[4];
-      Pos c2 = next_pos(next_pos(c0));
-      if (!wait_copy(c0)) {
-        failed = true;
-        break;
-      }
+      // software pipeline over the piece's quantized pages, two at a time:
+      // each step issues QK of pair k+1, PV of pair k and the softmax of pair
+      // k+1.  A pair whose second page is missing (odd count, last pair
+      // only) reads its first page twice and gives the copy zero weight.
+      uint32_t PA[4], PB[4];
       {
-        float S0[4];
-        qk_page<kBits>(addr(c0), qf, S0);
-        if (nq > 1) {
-          const Pos c1 = next_pos(c0);
-          if (!wait_copy(c1)) {
-            failed = true;
-            break;
-          }
-          qk_page<kBits>(addr(c1), qf, Sa);
+        const bool two = nq >= 2;
+        const Pos cb = next_pos(c0);
+        if (!wait_pair(c0, cb, two)) {
+          failed = true;
+          break;
         }
-        softmax_page(S0, p.scale_log2, st, Pa);
+        const Pos pb = two ? cb : c0;
+        float SA[4], SB[4];
+        qk_pair<kBits>(ring0 + c0.off, ring0 + pb.off, zero_row(c0, pb), lo, qf, SA, SB);
+        if (!two) SB[0] = SB[1] = SB[2] = SB[3] = -INFINITY;
+        softmax_pair(SA, SB, p.scale_log2, st, PA, PB);
       }
-      // one pipeline step: in (Pcur = P(j), Snext = S(j+1)), out (Pnext, Snext2)
-      auto step = [&](const uint32_t (&Pcur)[4], const float (&Snext)[4], uint32_t (&Pnext)[4],
-                      float (&Snext2)[4]) {
-        qk_page<kBits>(addr(c2), qf, Snext2);
-        pv_page<kBits>(addr(c0), Pcur, st);
-        softmax_page(Snext, p.scale_log2, st, Pnext);  // after PV(j): a rescale covers it
-        release();
-        c2 = next_pos(c2);
-      };
-      int j = 0;
-      bool odd = false;     // false: (Pa, Sa) hold (P(j), S(j+1)); true: (Pb, Sb)
+      int done = 0;  // pages before the current pair
 #pragma unroll 1
-      while (j + 2 < nq) {
-        if (!wait_copy(c2)) {
+      while (done + 2 < nq) {
+        const Pos cb = next_pos(c0), cn = next_pos(cb), cnb = next_pos(cn);
+        const bool two = done + 3 < nq;
+        if (!wait_pair(cn, cnb, two)) {
           failed = true;
           break;
         }
-        step(Pa, Sa, Pb, Sb);
-        ++j;
-        if (j + 2 >= nq) {
-          odd = true;
-          break;
-        }
-        if (!wait_copy(c2)) {
-          failed = true;
-          break;
-        }
-        step(Pb, Sb, Pa, Sa);
-        ++j;
+        const Pos pb = two ? cnb : cn;
+        float SA[4], SB[4];
+        qk_pair<kBits>(ring0 + cn.off, ring0 + pb.off, zero_row(cn, pb), lo, qf, SA, SB);
+        if (!two) SB[0] = SB[1] = SB[2] = SB[3] = -INFINITY;
+        pv_page<kBits>(ring0 + c0.off, lo, PA, st);
+        pv_page<kBits>(ring0 + cb.off, lo, PB, st);
+        softmax_pair(SA, SB, p.scale_log2, st, PA, PB);  // after PV of pair k: a rescale covers it
+        release(true);
+        done += 2;
       }
       if (failed) break;
-      // the last one or two pages
-      uint32_t Pt[4];
-      if (odd) {
-        pv_page<kBits>(addr(c0), Pb, st);
-        if (nq > 1) softmax_page(Sb, p.scale_log2, st, Pt);
-      } else {
-        pv_page<kBits>(addr(c0), Pa, st);
-        if (nq > 1) softmax_page(Sa, p.scale_log2, st, Pt);
-      }
-      release();
-      if (nq > 1) {
-        pv_page<kBits>(addr(c0), Pt, st);
-        release();
+      // the last pair
+      const bool two = done + 1 < nq;
+      pv_page<kBits>(ring0 + c0.off, lo, PA, st);
+      if (two) pv_page<kBits>(ring0 + next_pos(c0).off, lo, PB, st);
+      release(two);
+      // the code unit back to codes (4-bit codes entered as code * 2^-9)
+      if (code_unit_inv<kBits>() != 1.0f) {
+        const float2 cs = make_float2(code_unit_inv<kBits>(), code_unit_inv<kBits>());
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt) {
+          const float2 o01 = mul2(make_float2(st.O[mt][0], st.O[mt][1]), cs);
+          const float2 o23 = mul2(make_float2(st.O[mt][2], st.O[mt][3]), cs);
+          st.O[mt][0] = o01.x;
+          st.O[mt][1] = o01.y;
+          st.O[mt][2] = o23.x;
+          st.O[mt][3] = o23.y;
+        }
       }
     }
     if (p1 == cc.np && cc.np > cc.nfull) {

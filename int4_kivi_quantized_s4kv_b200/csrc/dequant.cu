@@ -36,7 +36,7 @@ __global__ void __launch_bounds__(128) dequant_kernel(const DequantParams p) {
     value_position(t, c, vword, vnib);
     const float kcode = static_cast<float>(code_at(blk + kcode_off, kword, knib, p.bits));
     const float vcode = static_cast<float>(code_at(blk + vcode_off, vword, vnib, p.bits));
-    const float vs = __half2float(reinterpret_cast<const __half *>(blk + vscale_off)[g * kPage + t]);
+    const float vs = __half2float(reinterpret_cast<const __half *>(blk + vscale_off)[value_scale_slot(t, g)]);
     const float vz = __half2float(reinterpret_cast<const __half *>(blk + vzero_off)[g * kPage + t]);
     const float kx = __fadd_rn(__fmul_rn(kcode, ks), kz);
     const float vx = __fadd_rn(__fmul_rn(vcode, vs), vz);

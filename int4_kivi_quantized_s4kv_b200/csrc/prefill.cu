@@ -280,7 +280,7 @@ __global__ void __launch_bounds__(kOpThreads) prefill_operands_kernel(const Pref
       const uint32_t ko = tc05::sw128_offset(key, c0, kKeyTile / 2);
       sts32(sK + ko, hi);
       sts32(sK + kKBytes / 4 + ko, lo);
-      const __half vs = vscale[g * kPage + t], vz = vzero[g * kPage + t];
+      const __half vs = vscale[value_scale_slot(t, g)], vz = vzero[g * kPage + t];
 #pragma unroll
       for (int j = 0; j < 2; ++j) {
         int vw, vn;
@@ -323,8 +323,8 @@ __global__ void __launch_bounds__(kOpThreads) prefill_operands_kernel(const Pref
         uint32_t a0, a1, a2, a3;
         unpack_codes(lds32_at(blk + kVCodeOff + 4 * w), a0, a1, a2, a3);
         const int g = tt >> 1;
-        const uint32_t sv_lo = lds32_at(blk + kVScaleOff + 2 * (16 * g + 2 * di));
-        const uint32_t sv_hi = lds32_at(blk + kVScaleOff + 2 * (16 * g + 2 * di + 8));
+        const uint32_t sv_lo = lds32_at(blk + kVScaleOff + 2 * value_scale_slot(2 * di, g));
+        const uint32_t sv_hi = lds32_at(blk + kVScaleOff + 2 * value_scale_slot(2 * di + 8, g));
         const uint32_t zv_lo = lds32_at(blk + kVZeroOff + 2 * (16 * g + 2 * di));
         const uint32_t zv_hi = lds32_at(blk + kVZeroOff + 2 * (16 * g + 2 * di + 8));
         const int cb = 32 * (tt >> 1) + 4 * dn + 2 * (tt & 1);

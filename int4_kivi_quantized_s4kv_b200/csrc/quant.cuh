@@ -63,42 +63,45 @@ __device__ __forceinline__ void quantize_page_cta(const __half (*ks)[kHeadDim], 
     for (int j = 0; j < kVGroup / 2; ++j)
       vc[t][c0 + j] = static_cast<uint8_t>(group_code_fast(__half2float(vs[t][c0 + j]), mn, s, inv, F::kLevels));
     if ((tid & 1) == 0) {
-      reinterpret_cast<__half *>(blk + F::kVScale)[g * kPage + t] = __float2half_rn(s);
+      reinterpret_cast<__half *>(blk + F::kVScale)[value_scale_slot(t, g)] = __float2half_rn(s);
       reinterpret_cast<__half *>(blk + F::kVZero)[g * kPage + t] = __float2half_rn(mn);
     }
   }
   __syncthreads();
-  // (token, channel) of nibble / byte j of tile `tile`, lane = 4n + i
-  auto key_tc = [](int tile, int n, int i, int j, int &t, int &c) {
-    t = 8 * (j & 1) + n;                                   // row = token
-    c = 32 * i + 4 * tile + 2 * ((j >> 1) & 1) + (j >> 2);  // k axis = channel
+  // (token, channel) at register r, half e of the operand fragment of tile
+  // `tile`, lane = 4n + i
+  auto key_tc = [](int tile, int n, int i, int r, int e, int &t, int &c) {
+    t = 8 * (r & 1) + n;                               // row = token
+    c = 32 * i + 4 * tile + 2 * (r >> 1) + e;          // k axis = channel
   };
-  auto val_tc = [](int tile, int n, int i, int j, int &t, int &c) {
-    t = 2 * i + (j >> 2) + 8 * ((j >> 1) & 1);             // k axis = token
-    c = 32 * (tile >> 1) + 4 * n + 2 * (tile & 1) + (j & 1);  // row = channel
+  auto val_tc = [](int tile, int n, int i, int r, int e, int &t, int &c) {
+    t = 2 * i + e + 8 * (r >> 1);                             // k axis = token
+    c = 32 * (tile >> 1) + 4 * n + 2 * (tile & 1) + (r & 1);  // row = channel
   };
   if (kBits == 4) {
-    // word w = 128*hh + 4*lane + q; nibble j is register j&3, half j>>2 of
-    // that lane's m16n8k16 operand fragment (tile = 4*hh + q)
+    // word w = 128*hh + 4*lane + q is lane's fragment of tile 4*hh + q;
+    // register r, half e at nibble nibble_of(r, e)
     for (int w = tid; w < 256; w += 128) {
       const int hh = w >> 7, lane = (w >> 2) & 31, q = w & 3;
       const int n = lane >> 2, i = lane & 3, tile = 4 * hh + q;
       uint32_t kw = 0, vw = 0;
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        int t, c;
-        key_tc(tile, n, i, j, t, c);
-        kw |= static_cast<uint32_t>(kc[t][c]) << (4 * j);
-        val_tc(tile, n, i, j, t, c);
-        vw |= static_cast<uint32_t>(vc[t][c]) << (4 * j);
+      for (int r = 0; r < 4; ++r) {
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          int t, c;
+          key_tc(tile, n, i, r, e, t, c);
+          kw |= static_cast<uint32_t>(kc[t][c]) << (4 * nibble_of(r, e));
+          val_tc(tile, n, i, r, e, t, c);
+          vw |= static_cast<uint32_t>(vc[t][c]) << (4 * nibble_of(r, e));
+        }
       }
       reinterpret_cast<uint32_t *>(blk + F::kKCode)[w] = kw;
       reinterpret_cast<uint32_t *>(blk + F::kVCode)[w] = vw;
     }
   } else if (kBits == 2) {
-    // word 4 lane + m holds tiles 2m, 2m + 1 of the lane: register r, half
-    // `half` (nibble index j = r + 4 half) of tile 2m + p at bit
-    // 16 half + 2 (4 p + r)
+    // word 4 lane + m holds tiles 2m, 2m + 1 of the lane: register r, half e
+    // of tile 2m + p at bit 16 e + 2 (4 p + r)
     for (int w = tid; w < 128; w += 128) {
       const int lane = w >> 2, m = w & 3;
       const int n = lane >> 2, i = lane & 3;
@@ -106,21 +109,24 @@ __device__ __forceinline__ void quantize_page_cta(const __half (*ks)[kHeadDim], 
 #pragma unroll
       for (int p = 0; p < 2; ++p) {
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const int bit = 16 * (j >> 2) + 2 * (4 * p + (j & 3));
-          int t, c;
-          key_tc(2 * m + p, n, i, j, t, c);
-          kw |= static_cast<uint32_t>(kc[t][c]) << bit;
-          val_tc(2 * m + p, n, i, j, t, c);
-          vw |= static_cast<uint32_t>(vc[t][c]) << bit;
+        for (int r = 0; r < 4; ++r) {
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int bit = 16 * e + 2 * (4 * p + r);
+            int t, c;
+            key_tc(2 * m + p, n, i, r, e, t, c);
+            kw |= static_cast<uint32_t>(kc[t][c]) << bit;
+            val_tc(2 * m + p, n, i, r, e, t, c);
+            vw |= static_cast<uint32_t>(vc[t][c]) << bit;
+          }
         }
       }
       reinterpret_cast<uint32_t *>(blk + F::kKCode)[w] = kw;
       reinterpret_cast<uint32_t *>(blk + F::kVCode)[w] = vw;
     }
   } else {
-    // byte (32 m + lane) * 16 + 8 (tile % 2) + 2 r + half holds register r,
-    // half `half` (nibble index j = r + 4 half) of tile 2m + tile % 2
+    // byte (32 m + lane) * 16 + 8 (tile % 2) + 2 r + e holds register r, half
+    // e of tile 2m + tile % 2
     for (int w = tid; w < 512; w += 128) {
       const int chunk = w >> 2, within = w & 3;
       const int m = chunk >> 5, lane = chunk & 31;
@@ -129,11 +135,11 @@ __device__ __forceinline__ void quantize_page_cta(const __half (*ks)[kHeadDim], 
       uint32_t kw = 0, vw = 0;
 #pragma unroll
       for (int b = 0; b < 4; ++b) {
-        const int j = (r0 + (b >> 1)) + 4 * (b & 1);
+        const int r = r0 + (b >> 1), e = b & 1;
         int t, c;
-        key_tc(tile, n, i, j, t, c);
+        key_tc(tile, n, i, r, e, t, c);
         kw |= static_cast<uint32_t>(kc[t][c]) << (8 * b);
-        val_tc(tile, n, i, j, t, c);
+        val_tc(tile, n, i, r, e, t, c);
         vw |= static_cast<uint32_t>(vc[t][c]) << (8 * b);
       }
       reinterpret_cast<uint32_t *>(blk + F::kKCode)[w] = kw;

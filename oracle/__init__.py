@@ -57,6 +57,8 @@ def lib():
         L.s4kv_ref_value_code_slot.argtypes = [i32, i32, P, P]
         L.s4kv_ref_key_zero_slot.argtypes = [i32]
         L.s4kv_ref_key_zero_slot.restype = i32
+        L.s4kv_ref_value_scale_slot.argtypes = [i32, i32]
+        L.s4kv_ref_value_scale_slot.restype = i32
         L.s4kv_ref_quantize_page.argtypes = [P, P, P]
         L.s4kv_ref_unpack_codes.argtypes = [P, P, P]
         L.s4kv_ref_dequant_block.argtypes = [P, P, P]
@@ -154,6 +156,12 @@ def value_code_slot(t: int, c: int) -> tuple[int, int]:
 def key_zero_slot(c: int) -> int:
     """Position (in halves, within the key-zero region) of channel c."""
     return int(lib().s4kv_ref_key_zero_slot(int(c)))
+
+
+def value_scale_slot(t: int, g: int) -> int:
+    """Position (in halves, within the value-scale region) of token t's scale
+    for channel group g."""
+    return int(lib().s4kv_ref_value_scale_slot(int(t), int(g)))
 
 
 def quantize_group_bits(x, bits: int) -> tuple[np.ndarray, int, int, float]:

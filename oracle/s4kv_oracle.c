@@ -39,14 +39,17 @@
  *   [2048,2304) key scale   : fp16 [128 channels]
  *   [2304,2560) key zero    : fp16 [8 k-tiles][16 k-slots], channel c at
  *                             k-tile (c%32)/4, slot 2*(c/32) + (c%2) + 8*((c%4)/2)
- *   [2560,2688) value scale : fp16 [4 groups][16 tokens]
+ *   [2560,2688) value scale : fp16, (token t, group g) at half
+ *                             16*((t%8)/2) + 8*(t/8) + 2*g + t%2
  *   [2688,2816) value zero  : fp16 [4 groups][16 tokens]
  * Code word w (0..255) splits as w = 128*h + 4*lane + q with lane = 4*n + i
- * (n 0..7, i 0..3, q 0..3).  Nibble j (bits 4j..4j+3) of the word holds
- *   keys  : token 8*(j&1) + n,
- *           channel 32*i + 4*(4*h + q) + 2*((j>>1)&1) + (j>>2);
- *   values: token 2*i + (j>>2) + 8*((j>>1)&1),
- *           channel 32*((4*h+q)>>1) + 4*n + 2*((4*h+q)&1) + (j&1).
+ * (n 0..7, i 0..3, q 0..3).  Nibble j (bits 4j..4j+3) of the word is
+ * register r = (j&1) + 2*(j>>2), half e = (j>>1)&1 of the lane's operand
+ * fragment and holds
+ *   keys  : token 8*(r&1) + n,
+ *           channel 32*i + 4*(4*h + q) + 2*(r>>1) + e;
+ *   values: token 2*i + e + 8*(r>>1),
+ *           channel 32*((4*h+q)>>1) + 4*n + 2*((4*h+q)&1) + (r&1).
  * Residual buffers hold fp16 [max_seqs][kv_heads][16][128] each for keys
  * and values: row r of sequence b is its token 16*floor(L/16) + r while
  * r < L mod 16; other rows are unspecified.
@@ -187,32 +190,56 @@ int s4kv_ref_key_zero_slot(int c) {
     return 16 * kt + 2 * i + (e % 2) + 8 * (e / 2);
 }
 
-/* (token, channel) -> (word, nibble) of the key code region. */
+/* A code's place in a lane's tensor-core operand fragment -- register r
+ * (0..3) and half e (0: low 16 bits) -- is held by nibble r%2 + 2e + 4(r/2)
+ * of the lane's 32-bit word: the even nibbles of the word's four bytes, then
+ * the odd ones, are registers 0 and 2 (byte pairs 0-1 and 2-3 of the even
+ * nibbles) and 1 and 3 (the same of the odd nibbles), the lower byte of a
+ * pair in the lower half. */
+static int nibble_of(int reg, int half) { return reg % 2 + 2 * half + 4 * (reg / 2); }
+static int reg_of(int nibble) { return nibble % 2 + 2 * (nibble / 4); }
+static int half_of(int nibble) { return (nibble / 2) % 2; }
+
+/* (token, channel) -> (word, nibble) of the key code region: tile kt =
+ * (c%32)/4 of lane 4n + i (n = t%8, i = c/32); rows are tokens (register
+ * bit 0: row n + 8), the k axis is the channel (register bit 1: k + 8, half:
+ * k + 1). */
 void s4kv_ref_key_code_slot(int t, int c, int *word, int *nibble) {
     int i = c / 32, kt = (c % 32) / 4, e = c % 4;
     int n = t % 8;
-    *nibble = (t / 8) + 2 * (e / 2) + 4 * (e % 2);
+    *nibble = nibble_of((t / 8) + 2 * (e / 2), e % 2);
     *word = 128 * (kt / 4) + 4 * (4 * n + i) + (kt % 4);
 }
 
-/* (token, channel) -> (word, nibble) of the value code region. */
+/* (token, channel) -> (word, nibble) of the value code region: M-tile m =
+ * 2(c/32) + (c%4)/2 of lane 4n + i (n = (c%32)/4, i = (t%8)/2); rows are
+ * channels (register bit 0: row + 8 = channel + 1), the k axis is the token
+ * (register bit 1: k + 8, half: k + 1). */
 void s4kv_ref_value_code_slot(int t, int c, int *word, int *nibble) {
     int grp = c / 32, n = (c % 32) / 4, e = c % 4;
     int m = 2 * grp + e / 2;
     int i = (t % 8) / 2;
-    *nibble = (e % 2) + 2 * (t / 8) + 4 * (t % 2);
+    *nibble = nibble_of((e % 2) + 2 * (t / 8), t % 2);
     *word = 128 * (m / 4) + 4 * (4 * n + i) + (m % 4);
+}
+
+/* Position (in halves) of the value scale of (token t, group g) in its
+ * region: lane quad i = (t%8)/2 owns 16 consecutive halves -- for k half
+ * e = t/8, the token pair 2i + 8e, 2i + 8e + 1 of groups 0..3 -- so that one
+ * lane reads all the scales it multiplies with two 16-byte loads. */
+int s4kv_ref_value_scale_slot(int t, int g) {
+    return 16 * ((t % 8) / 2) + 8 * (t / 8) + 2 * g + t % 2;
 }
 
 /* 8-bit codes keep the 4-bit layout's assignment of (token, channel) to MMA
  * operand fragments -- tile 4*(word/128) + word%4, lane (word/4)%32, and
- * within the lane's fragment register nibble%4, half nibble/4 -- with bytes
- * for nibbles: a lane's 8 codes of a tile are 8 consecutive bytes, register
- * r at bytes 2r (half 0) and 2r + 1 (half 1), and the 16 bytes of tiles
- * 2m and 2m+1 of one lane sit together, lanes in order. */
+ * within the lane's fragment register r and half e of the nibble -- with
+ * bytes for nibbles: a lane's 8 codes of a tile are 8 consecutive bytes,
+ * register r at bytes 2r (half 0) and 2r + 1 (half 1), and the 16 bytes of
+ * tiles 2m and 2m+1 of one lane sit together, lanes in order. */
 static long byte_offset8(int word, int nibble) {
     int tile = 4 * (word / 128) + word % 4, lane = (word / 4) % 32;
-    return ((long)(tile / 2) * 32 + lane) * 16 + (tile % 2) * 8 + 2 * (nibble % 4) + nibble / 4;
+    return ((long)(tile / 2) * 32 + lane) * 16 + (tile % 2) * 8 + 2 * reg_of(nibble) + half_of(nibble);
 }
 
 /* 2-bit codes keep the same assignment with two bits per code: the 16 codes
@@ -223,7 +250,7 @@ static long byte_offset8(int word, int nibble) {
 static void bit_position2(int word, int nibble, long *word2, int *bit) {
     int tile = 4 * (word / 128) + word % 4, lane = (word / 4) % 32;
     *word2 = 4L * lane + tile / 2;
-    *bit = 16 * (nibble / 4) + 2 * (4 * (tile % 2) + nibble % 4);
+    *bit = 16 * half_of(nibble) + 2 * (4 * (tile % 2) + reg_of(nibble));
 }
 
 /* Word index and bit of the 2-bit code of (token t, channel c) inside the
@@ -317,7 +344,7 @@ void s4kv_ref_quantize_page_bits(const uint16_t *kp, const uint16_t *vp,
             uint16_t sh, zh;
             quantize_group_levels(vp + t * HEAD_DIM + g * VGROUP, VGROUP, 1,
                                   &vc[t][g * VGROUP], 1, levels, &sh, &zh);
-            put_half(block + vscale_off(bits) + 2 * (g * PAGE + t), sh);
+            put_half(block + vscale_off(bits) + 2 * s4kv_ref_value_scale_slot(t, g), sh);
             put_half(block + vzero_off(bits) + 2 * (g * PAGE + t), zh);
         }
     }
@@ -361,7 +388,7 @@ void s4kv_ref_dequant_block_bits(const uint8_t *block, float *kout, float *vout,
             float ks = s4kv_ref_half_to_float(get_half(block + kscale_off(bits) + 2 * c));
             float kz = s4kv_ref_half_to_float(get_half(block + kzero_off(bits) + 2 * s4kv_ref_key_zero_slot(c)));
             int g = c / VGROUP;
-            float vs = s4kv_ref_half_to_float(get_half(block + vscale_off(bits) + 2 * (g * PAGE + t)));
+            float vs = s4kv_ref_half_to_float(get_half(block + vscale_off(bits) + 2 * s4kv_ref_value_scale_slot(t, g)));
             float vz = s4kv_ref_half_to_float(get_half(block + vzero_off(bits) + 2 * (g * PAGE + t)));
             volatile float kprod = (float)kc[t * HEAD_DIM + c] * ks;
             volatile float vprod = (float)vc[t * HEAD_DIM + c] * vs;

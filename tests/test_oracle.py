@@ -191,12 +191,15 @@ def _fragment_position(word, nibble):
     fragment table for mma.m16n8k16 (row-major A, f16): lane = 4*g + t holds
     a0 = (row g, cols 2t, 2t+1), a1 = (row g+8, same cols), a2 = (row g,
     cols 2t+8, 2t+9), a3 = (row g+8, cols 2t+8, 2t+9), the lower column in the
-    low half.  The library unpacks nibble j of a lane's word into register
-    j & 3, half j >> 2.  Returns (tile, lane, row, col)."""
+    low half.  The library unpacks a lane's word by keeping the low nibble of
+    every byte (bytes 0-1 -> register 0, bytes 2-3 -> register 2) and the high
+    nibble of every byte (-> registers 1 and 3), each byte pair converted to
+    an f16x2 with the lower byte in the low half: nibble j is register
+    (j & 1) + 2 (j >> 2), half (j >> 1) & 1.  Returns (tile, lane, row, col)."""
     tile = 4 * (word // 128) + word % 4
     lane = (word % 128) // 4
     g, t = lane // 4, lane % 4
-    r, e = nibble & 3, nibble >> 2
+    r, e = (nibble & 1) + 2 * (nibble >> 2), (nibble >> 1) & 1
     return tile, lane, g + 8 * (r & 1), 2 * t + e + 8 * (r >> 1)
 
 
@@ -216,6 +219,23 @@ def test_code_layout_is_the_mma_operand_order(oracle_mod):
             tile, lane, row, col = _fragment_position(*oracle_mod.value_code_slot(t, c))
             ch = 32 * (tile // 2) + 4 * (row % 8) + 2 * (tile % 2) + row // 8
             assert (col, ch) == (t, c)
+
+
+def test_value_scales_are_lane_major(oracle_mod):
+    """Value scales are stored so that the lane quad whose B-operand k rows
+    are tokens 2i, 2i+1 (and 2i+8, 2i+9) finds the scales of those tokens, for
+    all four channel groups, in one 32-byte run: quad i owns halves 16i ..
+    16i + 15, k half e (tokens + 8e) the 8 halves from 16i + 8e, group g the
+    token pair at 16i + 8e + 2g.  A bijection onto the 64 slots."""
+    seen = set()
+    for t in range(PAGE):
+        for g in range(4):
+            pos = oracle_mod.value_scale_slot(t, g)
+            i, e = (t % 8) // 2, t // 8
+            assert 16 * i + 8 * e <= pos < 16 * i + 8 * e + 8
+            assert pos == 16 * i + 8 * e + 2 * g + t % 2
+            seen.add(pos)
+    assert seen == set(range(64))
 
 
 def test_key_zero_order_is_the_mma_k_order(oracle_mod):
@@ -268,7 +288,8 @@ def test_page_axis_split_closed_form(oracle_mod):
     ks = blk[2048:2304].view(np.float16).astype(np.float64)
     kz_slots = blk[2304:2560].view(np.float16).astype(np.float64)
     kz = np.array([kz_slots[oracle_mod.key_zero_slot(c)] for c in range(HD)])
-    vs = blk[2560:2688].view(np.float16).astype(np.float64).reshape(4, 16)
+    vs_slots = blk[2560:2688].view(np.float16).astype(np.float64)
+    vs = np.array([[vs_slots[oracle_mod.value_scale_slot(t, g)] for t in range(PAGE)] for g in range(4)])
     vz = blk[2688:2816].view(np.float16).astype(np.float64).reshape(4, 16)
     assert np.array_equal(ks, kd) and np.array_equal(kz, ka)
     assert np.array_equal(vs, vd.T) and np.array_equal(vz, va.T)
@@ -731,7 +752,7 @@ def test_int8_layout_is_the_int4_fragment_map_in_bytes(oracle_mod):
                 r, half = divmod(within % 8, 2)
                 word, nib = slot(t, c)
                 assert (tile, lane) == (4 * (word // 128) + word % 4, (word % 128) // 4)
-                assert (r, half) == (nib & 3, nib >> 2)
+                assert (r, half) == ((nib & 1) + 2 * (nib >> 2), (nib >> 1) & 1)
                 seen.add(off)
         assert seen == set(range(2048))
 
@@ -848,7 +869,7 @@ def test_int2_layout_is_the_int4_fragment_map_in_bit_pairs(oracle_mod):
                 p, r = divmod(rest // 2, 4)
                 word, nib = slot(t, c)
                 assert (2 * m + p, lane) == (4 * (word // 128) + word % 4, (word % 128) // 4)
-                assert (r, half) == (nib & 3, nib >> 2) and bit % 2 == 0
+                assert (r, half) == ((nib & 1) + 2 * (nib >> 2), (nib >> 1) & 1) and bit % 2 == 0
                 seen.add((w2, bit))
         assert seen == {(w, b) for w in range(128) for b in range(0, 32, 2)}
     assert oracle_mod.block_bytes(2) == 2 * 512 + 768
