@@ -236,14 +236,14 @@ class OracleSample:
     head) pairs of layer 0, prefilled untimed; one call of `run()` is the
     step (append of the new token(s) + decode) for the sampled sequences."""
 
-    def __init__(self, spec: W.Spec, n_seqs: int, bits: int = 4):
+    def __init__(self, spec: W.Spec, n_seqs: int, bits: int = 4, first: int = 0):
         import oracle
         oracle.build()
-        n_seqs = max(1, min(n_seqs, spec.batch))
+        first = max(0, min(first, spec.batch - 1))
+        n_seqs = max(1, min(n_seqs, spec.batch - first))
         self.spec = spec
         ctx, lens = W.context_lens(spec), W.final_lens(spec)
-        plan = W.page_plan(spec)
-        self.seqs = list(range(n_seqs))
+        self.seqs = list(range(first, first + n_seqs))
         # compact page tables for the sample (shared pages become private)
         need = [(int(lens[b]) + 15) // 16 for b in self.seqs]
         bt = np.full((n_seqs, max(need)), -1, np.int32)
@@ -279,6 +279,50 @@ class OracleSample:
         return self.cache.decode_attention(self.q, self.lens, self.bt)
 
 
+def _oracle_slice(args):
+    """One process of the multi-core baseline: the unchanged oracle on a slice
+    of sequences (prefilled untimed), one timed step after all processes are
+    ready."""
+    spec, first, n, bits, barrier = args
+    samp = OracleSample(spec, n, bits, first=first)
+    barrier.wait()
+    t0 = time.perf_counter()
+    samp.run()
+    dt = time.perf_counter() - t0
+    return samp.bytes, samp.tokens, dt
+
+
+def cpu_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline_multicore(spec, n_single: int, bits: int = 4):
+    """The same oracle in one process per host core, each on its own slice of
+    sequences (n_single of them per process, the single-threaded sample's
+    size), started together: aggregate bytes over the slowest process's time.
+    Processes are spawned (not forked) so that no CUDA state is inherited."""
+    import multiprocessing as mp
+    cores = cpu_cores()
+    per = max(1, n_single)
+    nproc = max(1, min(cores, spec.batch // per))
+    ctx = mp.get_context("spawn")
+    with ctx.Manager() as mgr:
+        barrier = mgr.Barrier(nproc)
+        with ctx.Pool(nproc) as pool:
+            res = pool.map(_oracle_slice, [(spec, k * per, per, bits, barrier) for k in range(nproc)])
+    total_bytes = sum(r[0] for r in res)
+    total_tokens = sum(r[1] for r in res)
+    dt = max(r[2] for r in res)
+    return {"value": total_bytes / dt / 1e9, "unit": "GB/s", "cores": nproc, "host_cores": cores,
+            "kind": "oracle",
+            "sample": f"{nproc} processes x {per} sequences of layer 0 (all kv heads), one step "
+                      f"(append + decode) each, started together; {dt:.1f} s for the slowest",
+            "tokens_per_s": total_tokens / dt, "seconds": dt}
+
+
 def cpu_baseline(spec, budget_s=12.0, bits: int = 4):
     probe = OracleSample(spec, 1, bits)
     t0 = time.perf_counter()
@@ -289,10 +333,14 @@ def cpu_baseline(spec, budget_s=12.0, bits: int = 4):
     t0 = time.perf_counter()
     samp.run()
     dt = time.perf_counter() - t0
-    return {"value": samp.bytes / dt / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
-            "sample": f"{n} of {spec.batch} sequences of layer 0 (all kv heads), one step "
-                      f"(append + decode), {dt:.1f} s single-threaded",
-            "tokens_per_s": samp.tokens / dt, "seconds": dt}
+    single = {"value": samp.bytes / dt / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+              "sample": f"{n} of {spec.batch} sequences of layer 0 (all kv heads), one step "
+                        f"(append + decode), {dt:.1f} s single-threaded",
+              "tokens_per_s": samp.tokens / dt, "seconds": dt}
+    multi = cpu_baseline_multicore(spec, n, bits)
+    out = dict(multi)
+    out["single_core"] = single
+    return out
 
 
 # ------------------------------------------------------------------ main --
@@ -502,6 +550,54 @@ def measure_fused_step(wl, device, steps: int = 20):
 BLOCK_BYTES = {2: 1792, 4: 2816, 8: 4864}
 
 
+def measure_decode_config(device, name: str, steps: int = 20):
+    """Decode of one of the other large workloads (every layer): the average
+    s4kv_decode_attention launch against the HBM roofline on its unique bytes
+    (shared-prefix pages counted once), the logical bytes beside them, and the
+    whole step (append + decode of every layer) as two launches per layer and
+    as the fused one."""
+    import torch
+    spec = W.SPECS[name]
+    wl = DeviceWorkload(spec, device)
+    dbytes, abytes = step_bytes(wl.spec, wl.plan, wl.lens)
+    for _ in range(3):
+        wl.step()
+    torch.cuda.synchronize()
+    ev = ([], [])
+    for _ in range(steps):
+        wl.step(ev)
+    torch.cuda.synchronize()
+    dec_ms = sum(a.elapsed_time(b) for a, b in zip(*ev)) / len(ev[0])
+    fused = measure_fused_step(wl, device, steps=max(3, min(steps, 10) if spec.layers > 1 else steps))
+    if any(wl.S.s4kv_get_error(c) for c in wl.caches):
+        raise RuntimeError(f"{name} decode set device error flags")
+    peak, kind = measured_hbm_peak()
+    gbs = dbytes["algorithmic"] / (dec_ms * 1e-3) / 1e9
+    step_bytes_all = (dbytes["algorithmic"] + abytes) * spec.layers
+    tokens = int(wl.new.sum())
+    res = {"workload": name, "model_shape": spec.description, "layers": spec.layers, "batch": spec.batch,
+           "num_q_heads": spec.num_q_heads, "num_kv_heads": spec.num_kv_heads,
+           "context": {"min": int(wl.ctx.min()), "max": int(wl.ctx.max()), "mean": float(wl.ctx.mean())},
+           "shared_prefix_tokens": spec.shared_prefix_tokens,
+           "decode_launches": len(ev[0]), "avg_launch_ms": dec_ms,
+           "unique_bytes_per_launch": dbytes["algorithmic"], "logical_bytes_per_launch": dbytes["logical"],
+           "logical_GBs": dbytes["logical"] / (dec_ms * 1e-3) / 1e9,
+           "tokens_per_s": tokens / (dec_ms * 1e-3 * spec.layers),
+           "sequences_per_s": spec.batch / (dec_ms * 1e-3 * spec.layers),
+           "roofline": {"bound": "hbm", "kernel": "decode_kernel<4>", "achieved": gbs, "peak": peak,
+                        "peak_kind": kind, "unit": "GB/s", "frac": gbs / peak, "traffic": None,
+                        "bytes_per_launch": dbytes["algorithmic"]},
+           "step": {"two_launch_ms": fused["two_launch_ms"], "fused_ms": fused["fused_ms"],
+                    "two_launch_GBs": step_bytes_all / (fused["two_launch_ms"] * 1e-3) / 1e9,
+                    "fused_GBs": step_bytes_all / (fused["fused_ms"] * 1e-3) / 1e9,
+                    "tokens_per_s_two_launch": tokens / (fused["two_launch_ms"] * 1e-3),
+                    "tokens_per_s_fused": tokens / (fused["fused_ms"] * 1e-3),
+                    "launches_per_step": {"two_launch": 2 * spec.layers, "fused": spec.layers}}}
+    del wl
+    torch.cuda.empty_cache()
+    return res
+
+
 def measure_width_decode(device, spec, bits: int, steps: int = 20):
     """The 8- or 2-bit variant's decode step (append + decode) on the same
     workload as the headline, against the HBM roofline."""
@@ -691,7 +787,7 @@ def main(argv=None):
     value = aggregate_gbs(world, bytes_per_step, step_ms)
     achieved = decode_bytes_per_launch / (dec_avg_ms * 1e-3) / 1e9
     tokens = int(wl.new.sum())
-    prefill = moves = fused = int8 = int2 = None
+    prefill = moves = fused = int8 = int2 = configs = None
     if world == 1 and not args.no_prefill:
         prefill = [measure_prefill(device, max(3, min(args.steps, 20)), w, args.bits) for w in W.PREFILL_ORDER]
         moves = measure_page_moves(wl, device)
@@ -701,6 +797,8 @@ def main(argv=None):
         del small
         int8 = measure_width_decode(device, spec, 8)
         int2 = measure_width_decode(device, spec, 2)
+        configs = [measure_decode_config(device, name) for name in W.CONFIG_ORDER
+                   if name not in ("tiny", spec.name.split("-b")[0] if args.batch else spec.name)]
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(spec, bits=args.bits)
@@ -739,7 +837,7 @@ def main(argv=None):
             line["cpu_baseline"] = cpu
         if prefill is not None:
             line["next_rows"] = {"prefill": prefill, "page_moves": moves, "fused_step": fused, "int8_decode": int8,
-                                 "int2_decode": int2}
+                                 "int2_decode": int2, "decode_configs": configs}
         print(json.dumps(line), flush=True)
     if world > 1:
         torch.distributed.destroy_process_group()

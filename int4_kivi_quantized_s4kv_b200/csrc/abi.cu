@@ -63,7 +63,7 @@ int device_shape(DeviceShape *out) {
       const int per = decode_ctas_per_sm(fmt_bits(f));
       if (per <= 0 || sms <= 0) return S4KV_ERR_CUDA;
       d.num_ctas[f] = sms * per;
-      d.num_workers[f] = d.num_ctas[f] * decode_warps_per_cta();
+      d.num_workers[f] = d.num_ctas[f] * decode_warps_per_cta(fmt_bits(f));
       d.max_workers = d.num_workers[f] > d.max_workers ? d.num_workers[f] : d.max_workers;
     }
     d.ready = true;

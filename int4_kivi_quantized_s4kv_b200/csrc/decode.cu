@@ -43,8 +43,8 @@
 //    headroom of 4, so every weight stays <= 1 and no fp16 operand can
 //    overflow); P is moved from the QK accumulator layout to the PV operand
 //    layout with movmatrix.
-//  * Pipelining.  Within a warp, the QK MMAs of page pair k+1, the PV MMAs of
-//    pair k and the softmax of pair k+1 are issued in one straight-line
+//  * Pipelining.  Within a warp, the softmax of page pair k, the QK MMAs of
+//    pair k+1 and the PV MMAs of pair k are issued in one straight-line
 //    block, so the softmax's latency overlaps tensor-core work.
 #include <cfloat>
 
@@ -53,33 +53,42 @@
 
 namespace s4kv {
 
-// Build-time tuning constants (stages per warp ring, worker warps per CTA,
-// CTAs per SM the register budget is sized for).
+// Build-time tuning constants: stages per warp ring; worker warps per CTA
+// (4- and 2-bit pages: one CTA of 12 warps per SM, so that all warps of an SM
+// are equally old and the warp schedulers serve them alike; 4864-byte int8
+// blocks: two CTAs of 4 warps with 5 stages each); the fewest pages a worker
+// is given, so that small batches are not cut into many short pieces.
 #ifndef S4KV_DECODE_STAGES
 #define S4KV_DECODE_STAGES 6
 #endif
 #ifndef S4KV_DECODE_WARPS
-#define S4KV_DECODE_WARPS 4
-#endif
-#ifndef S4KV_DECODE_MIN_CTAS
-#define S4KV_DECODE_MIN_CTAS 3
+#define S4KV_DECODE_WARPS 12
 #endif
 #ifndef S4KV_DECODE_STAGES_INT8
 #define S4KV_DECODE_STAGES_INT8 5
 #endif
-// stages of a warp's ring for kBits-bit pages (the 4864-byte int8 blocks get
-// fewer, so that two CTAs still fit on an SM)
+#ifndef S4KV_DECODE_WARPS_INT8
+#define S4KV_DECODE_WARPS_INT8 4
+#endif
+#ifndef S4KV_DECODE_MIN_PAGES
+#define S4KV_DECODE_MIN_PAGES 16
+#endif
 template <int kBits>
 __host__ __device__ constexpr int stages_for() { return kBits == 8 ? S4KV_DECODE_STAGES_INT8 : S4KV_DECODE_STAGES; }
-constexpr int kWarpsPerCta = S4KV_DECODE_WARPS;
-constexpr int kThreads = 32 * kWarpsPerCta;
+template <int kBits>
+__host__ __device__ constexpr int warps_for() { return kBits == 8 ? S4KV_DECODE_WARPS_INT8 : S4KV_DECODE_WARPS; }
+template <int kBits>
+__host__ __device__ constexpr int threads_for() { return 32 * warps_for<kBits>(); }
+// registers: the whole file of an SM for 12 warps, half of it for 4
+template <int kBits>
+__host__ __device__ constexpr int min_ctas_for() { return 12 / warps_for<kBits>() > 1 ? 12 / warps_for<kBits>() : 1; }
 constexpr long long kWaitLimitCycles = 2000000000LL;  // about one second
 constexpr unsigned kFull = 0xFFFFFFFFu;
 constexpr float kHeadroom = 4.0f;  // log2 headroom of the softmax reference
 
 template <int kBits>
 constexpr size_t smem_bytes_for() {
-  return static_cast<size_t>(kWarpsPerCta) * stages_for<kBits>() * (Fmt<kBits>::kBlock + 8);
+  return static_cast<size_t>(warps_for<kBits>()) * stages_for<kBits>() * (Fmt<kBits>::kBlock + 8);
 }
 
 size_t decode_smem_bytes(int bits) {
@@ -558,7 +567,7 @@ __device__ __forceinline__ void residual_row_write(const DecodeParams &p, const 
 
 // One completed page (job = sequence, kv head, physical page) quantized by
 // all threads of the CTA, with `scratch` (12 KB of shared memory) as staging.
-template <int kBits>
+template <int kBits, int kThreads>
 __device__ __forceinline__ void cta_quantize_job(const DecodeParams &p, const FusedAppend &f, int4 job, uint8_t *scratch,
                                                  int tid) {
   const int b = job.x, h = job.y, phys = job.w;
@@ -585,15 +594,20 @@ __device__ __forceinline__ void cta_quantize_job(const DecodeParams &p, const Fu
 
 // kFused: the step's append is fused in (DecodeParams::k_new / v_new set).
 template <int kBits, bool kFused>
-__global__ void __launch_bounds__(kThreads, S4KV_DECODE_MIN_CTAS) decode_kernel(const DecodeParams p, const FusedAppend f) {
+__global__ void __launch_bounds__(threads_for<kBits>(), min_ctas_for<kBits>())
+    decode_kernel(const DecodeParams p, const FusedAppend f) {
   constexpr int kStages = stages_for<kBits>();
+  constexpr int kWarpsPerCta = warps_for<kBits>();
+  constexpr int kThreads = threads_for<kBits>();
   constexpr int kBlockBytes = Fmt<kBits>::kBlock;
   extern __shared__ __align__(128) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n = lane >> 2, i = lane & 3;
   const uint32_t ring0 = smem_addr(smem) + warp * kStages * kBlockBytes;
   const uint32_t bar0 = smem_addr(smem) + kWarpsPerCta * kStages * kBlockBytes + warp * kStages * 8;
-  const long long worker = static_cast<long long>(blockIdx.x) * kWarpsPerCta + warp;
+  // worker ids run over the CTAs first, so that a launch with fewer workers
+  // than warps spreads them over the SMs
+  const long long worker = static_cast<long long>(warp) * gridDim.x + blockIdx.x;
   const int B = p.batch, H = p.num_kv_heads, G = p.group;
   const LaneOff lo = lane_offsets<kBits>(lane);
 
@@ -602,7 +616,7 @@ __global__ void __launch_bounds__(kThreads, S4KV_DECODE_MIN_CTAS) decode_kernel(
     for (int st = 0; st < kStages; ++st) mbar_init(bar0 + 8 * st, 1);
     fence_barrier_init();
   }
-  __syncwarp();
+  __syncthreads();
 
   // ---- plan: pages per kv head of each lane's block of sequences, scanned
   const int per = (B + 31) >> 5;
@@ -624,7 +638,10 @@ __global__ void __launch_bounds__(kThreads, S4KV_DECODE_MIN_CTAS) decode_kernel(
   const long long excl = incl - lsum;
   const long long total = __shfl_sync(kFull, incl, 31);
   const long long T = total * H;
-  const long long W = max(1LL, min(static_cast<long long>(p.num_workers), T));
+  // workers: all resident warps, or fewer so that each gets at least
+  // S4KV_DECODE_MIN_PAGES pages
+  const long long W = max(1LL, min(static_cast<long long>(p.num_workers),
+                                   (T + S4KV_DECODE_MIN_PAGES - 1) / S4KV_DECODE_MIN_PAGES));
   if (worker == 0) {
     if (__any_sync(kFull, bad_len) && lane == 0) flag_error(p.err, S4KV_EFLAG_SEQ_LEN);
     // sequences with no tokens get zeros
@@ -640,11 +657,12 @@ __global__ void __launch_bounds__(kThreads, S4KV_DECODE_MIN_CTAS) decode_kernel(
       }
     }
   }
-  // with the fused append every warp of the CTA takes part in its barriers
-  if (kFused ? T == 0 : (worker >= W || T == 0)) return;
+  // every warp of the CTA, with work or not, takes part in its barriers (the
+  // fused append's and the final merge's)
+  if (T == 0) return;
   const bool active = worker < W;
-  const long long s = (kFused && !active) ? 0 : worker * T / W;
-  const long long e = (kFused && !active) ? 0 : (worker + 1) * T / W;
+  const long long s = active ? worker * T / W : 0;
+  const long long e = active ? (worker + 1) * T / W : 0;
 
   // ---- locate the segment holding page s
   const unsigned hit = __ballot_sync(kFull, H * excl <= s && s < H * incl);
@@ -708,14 +726,14 @@ __global__ void __launch_bounds__(kThreads, S4KV_DECODE_MIN_CTAS) decode_kernel(
       if (lane == 0) s_njob[warp] = nj;
       __syncthreads();
       for (int w = 0; w < kWarpsPerCta; ++w)
-        for (int j = 0; j < s_njob[w]; ++j) cta_quantize_job<kBits>(p, f, s_job[w][j], smem, threadIdx.x);
+        for (int j = 0; j < s_njob[w]; ++j) cta_quantize_job<kBits, kThreads>(p, f, s_job[w][j], smem, threadIdx.x);
       // the pool writes are read next by bulk copies (async proxy)
       asm volatile("fence.proxy.async.global;" ::: "memory");
       if (!__syncthreads_or(more)) break;
     }
-    if (!active) return;
   }
 
+  if (active) {
   // ---- producer: issue the next quantized pages of [s, e) into the ring.
   // It walks the same pieces as the consumer.  The page ids of a piece are
   // read 32 at a time into a window (lane l holds the l-th) with one
@@ -870,10 +888,12 @@ __global__ void __launch_bounds__(kThreads, S4KV_DECODE_MIN_CTAS) decode_kernel(
 
     if (nq > 0) {
       // software pipeline over the piece's quantized pages, two at a time:
-      // each step issues QK of pair k+1, PV of pair k and the softmax of pair
-      // k+1.  A pair whose second page is missing (odd count, last pair
-      // only) reads its first page twice and gives the copy zero weight.
-      uint32_t PA[4], PB[4];
+      // step k turns the logits of pair k into weights, issues the QK MMAs
+      // of pair k+1 (independent of that softmax, so they hide its latency)
+      // and then the PV MMAs of pair k.  A pair whose second page is missing
+      // (odd count, last pair only) reads its first page twice and gives the
+      // copy zero weight.
+      float SA[4], SB[4];
       {
         const bool two = nq >= 2;
         const Pos cb = next_pos(c0);
@@ -882,10 +902,8 @@ __global__ void __launch_bounds__(kThreads, S4KV_DECODE_MIN_CTAS) decode_kernel(
           break;
         }
         const Pos pb = two ? cb : c0;
-        float SA[4], SB[4];
         qk_pair<kBits>(ring0 + c0.off, ring0 + pb.off, zero_row(c0, pb), lo, qf, SA, SB);
         if (!two) SB[0] = SB[1] = SB[2] = SB[3] = -INFINITY;
-        softmax_pair(SA, SB, p.scale_log2, st, PA, PB);
       }
       int done = 0;  // pages before the current pair
 #pragma unroll 1
@@ -896,22 +914,26 @@ __global__ void __launch_bounds__(kThreads, S4KV_DECODE_MIN_CTAS) decode_kernel(
           failed = true;
           break;
         }
+        uint32_t PA[4], PB[4];
+        softmax_pair(SA, SB, p.scale_log2, st, PA, PB);
         const Pos pb = two ? cnb : cn;
-        float SA[4], SB[4];
         qk_pair<kBits>(ring0 + cn.off, ring0 + pb.off, zero_row(cn, pb), lo, qf, SA, SB);
         if (!two) SB[0] = SB[1] = SB[2] = SB[3] = -INFINITY;
         pv_page<kBits>(ring0 + c0.off, lo, PA, st);
         pv_page<kBits>(ring0 + cb.off, lo, PB, st);
-        softmax_pair(SA, SB, p.scale_log2, st, PA, PB);  // after PV of pair k: a rescale covers it
         release(true);
         done += 2;
       }
       if (failed) break;
       // the last pair
-      const bool two = done + 1 < nq;
-      pv_page<kBits>(ring0 + c0.off, lo, PA, st);
-      if (two) pv_page<kBits>(ring0 + next_pos(c0).off, lo, PB, st);
-      release(two);
+      {
+        const bool two = done + 1 < nq;
+        uint32_t PA[4], PB[4];
+        softmax_pair(SA, SB, p.scale_log2, st, PA, PB);
+        pv_page<kBits>(ring0 + c0.off, lo, PA, st);
+        if (two) pv_page<kBits>(ring0 + next_pos(c0).off, lo, PB, st);
+        release(two);
+      }
       // the code unit back to codes (4-bit codes entered as code * 2^-9)
       if (code_unit_inv<kBits>() != 1.0f) {
         const float2 cs = make_float2(code_unit_inv<kBits>(), code_unit_inv<kBits>());
@@ -1015,13 +1037,16 @@ __global__ void __launch_bounds__(kThreads, S4KV_DECODE_MIN_CTAS) decode_kernel(
       c0 = next_pos(c0);
     }
   }
+  }  // active
 }
 
 template <int kBits>
 int ctas_per_sm_for() {
   int n = 0, m = 0;
-  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_kernel<kBits, false>, kThreads, smem_bytes_for<kBits>());
-  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&m, decode_kernel<kBits, true>, kThreads, smem_bytes_for<kBits>());
+  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_kernel<kBits, false>, threads_for<kBits>(),
+                                                smem_bytes_for<kBits>());
+  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&m, decode_kernel<kBits, true>, threads_for<kBits>(),
+                                                smem_bytes_for<kBits>());
   return n < m ? n : m;  // one launch shape serves the plain and the fused kernel
 }
 
@@ -1029,7 +1054,9 @@ int decode_ctas_per_sm(int bits) {
   return bits == 8 ? ctas_per_sm_for<8>() : bits == 2 ? ctas_per_sm_for<2>() : ctas_per_sm_for<4>();
 }
 
-int decode_warps_per_cta() { return kWarpsPerCta; }
+int decode_warps_per_cta(int bits) {
+  return bits == 8 ? warps_for<8>() : bits == 2 ? warps_for<2>() : warps_for<4>();
+}
 
 template <int kBits>
 cudaError_t prepare_for() {
@@ -1051,19 +1078,19 @@ void launch_decode(const DecodeParams &p, const FusedAppend &f, int bits, int nu
   const bool fused = f.k_new != nullptr;
   if (bits == 8) {
     if (fused)
-      decode_kernel<8, true><<<num_ctas, kThreads, smem_bytes_for<8>(), stream>>>(p, f);
+      decode_kernel<8, true><<<num_ctas, threads_for<8>(), smem_bytes_for<8>(), stream>>>(p, f);
     else
-      decode_kernel<8, false><<<num_ctas, kThreads, smem_bytes_for<8>(), stream>>>(p, f);
+      decode_kernel<8, false><<<num_ctas, threads_for<8>(), smem_bytes_for<8>(), stream>>>(p, f);
   } else if (bits == 2) {
     if (fused)
-      decode_kernel<2, true><<<num_ctas, kThreads, smem_bytes_for<2>(), stream>>>(p, f);
+      decode_kernel<2, true><<<num_ctas, threads_for<2>(), smem_bytes_for<2>(), stream>>>(p, f);
     else
-      decode_kernel<2, false><<<num_ctas, kThreads, smem_bytes_for<2>(), stream>>>(p, f);
+      decode_kernel<2, false><<<num_ctas, threads_for<2>(), smem_bytes_for<2>(), stream>>>(p, f);
   } else {
     if (fused)
-      decode_kernel<4, true><<<num_ctas, kThreads, smem_bytes_for<4>(), stream>>>(p, f);
+      decode_kernel<4, true><<<num_ctas, threads_for<4>(), smem_bytes_for<4>(), stream>>>(p, f);
     else
-      decode_kernel<4, false><<<num_ctas, kThreads, smem_bytes_for<4>(), stream>>>(p, f);
+      decode_kernel<4, false><<<num_ctas, threads_for<4>(), smem_bytes_for<4>(), stream>>>(p, f);
   }
 }
 

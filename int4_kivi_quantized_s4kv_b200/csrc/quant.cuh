@@ -16,15 +16,16 @@ namespace s4kv {
 // Quantize one page of one kv head.  ks / vs: the page's fp16 keys and values
 // [16][128] in shared memory (complete before the call); kc / vc: [16][128]
 // byte scratch in shared memory; blk: the 2816-byte block in global memory.
-// Called by all 128 threads of the CTA (tid = threadIdx.x, whole warps);
-// contains CTA barriers.
+// Called by every thread of the CTA (tid = threadIdx.x, at least 128
+// threads, whole warps): threads 0..127 do the work, and all of them meet at
+// the CTA barrier inside.
 template <int kBits>
 __device__ __forceinline__ void quantize_page_cta(const __half (*ks)[kHeadDim], const __half (*vs)[kHeadDim],
                                                   uint8_t (*kc)[kHeadDim], uint8_t (*vc)[kHeadDim], uint8_t *blk,
                                                   int tid) {
   using F = Fmt<kBits>;
   // keys: thread c quantizes channel c over the 16 tokens
-  {
+  if (tid < 128) {
     const int c = tid;
     float mn = __half2float(ks[0][c]), mx = mn;
 #pragma unroll
@@ -45,7 +46,7 @@ __device__ __forceinline__ void quantize_page_cta(const __half (*ks)[kHeadDim], 
   }
   // values: one (token, 32-channel group) per thread pair; each thread takes
   // 16 channels and the pair combines its minima and maxima
-  {
+  if (tid < 128) {
     const int t = tid >> 3, g = (tid >> 1) & 3, c0 = g * kVGroup + (tid & 1) * (kVGroup / 2);
     float mn = __half2float(vs[t][c0]), mx = mn;
 #pragma unroll
@@ -68,6 +69,7 @@ __device__ __forceinline__ void quantize_page_cta(const __half (*ks)[kHeadDim], 
     }
   }
   __syncthreads();
+  if (tid >= 128) return;
   // (token, channel) at register r, half e of the operand fragment of tile
   // `tile`, lane = 4n + i
   auto key_tc = [](int tile, int n, int i, int r, int e, int &t, int &c) {

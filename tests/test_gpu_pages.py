@@ -133,7 +133,9 @@ def test_copy_on_write_fork():
     q = p.q.copy()
     q[4] = q[0]
     out = p.gpu_decode(q)
-    assert np.array_equal(out[4], out[0])
+    # same pages and query: the same attention (the two rows sit at different
+    # places of the split along the sequence, so the merges may round apart)
+    assert_attention_close(out[4], out[0], "fork before diverging")
     assert not out[3].any()
     ref0 = out[0].copy()
     # the fork diverges: its own continuation completes the partial page
@@ -147,7 +149,10 @@ def test_copy_on_write_fork():
     p.append(lens, after, None)
     p.lens = after
     out2 = p.gpu_decode(q)
-    assert np.array_equal(out2[0], ref0)
+    # the original is untouched (its pages are compared bit for bit below);
+    # its attention may round differently where the split along the
+    # sequence moved with the fork's new length
+    assert_attention_close(out2[0], ref0, "original after the fork diverged")
     assert_attention_close(out2, p.oracle_decode(q), "decode after fork")
     torch.cuda.synchronize()
     assert np.array_equal(p.gpu.pool.cpu().numpy(), p.oc.pool)
