@@ -74,6 +74,8 @@ def lib():
         L.s4kv_ref_attention_fp16.argtypes = [P, P, P, i32, P, i32, i32, f64, P]
         L.s4kv_ref_prefill_attention.argtypes = [P, P, P, i32, i32, P, i32, P, P, P, i32, i32, f64, P, i32]
         L.s4kv_ref_prefill_attention.restype = i32
+        L.s4kv_ref_attention_at.argtypes = [P, P, P, i32, i32, P, i32, i32, i32, P, i32, i32, f64, P, i32]
+        L.s4kv_ref_attention_at.restype = i32
         L.s4kv_ref_gather_pages.argtypes = [P, i32, i32, P, i32, P, i32]
         L.s4kv_ref_gather_pages.restype = i32
         L.s4kv_ref_scatter_pages.argtypes = [P, i32, i32, P, i32, P, i32]
@@ -333,6 +335,24 @@ class OracleCache:
             len(sl), bt.shape[1], float(sm_scale), _p(out), self.bits)
         if rc != 0:
             raise ValueError(f"prefill_attention rc={rc}")
+        return out
+
+    def attention_at(self, q_row, b: int, L: int, pos: int, bt_row, sm_scale=None) -> np.ndarray:
+        """One query row (fp16 [num_q_heads][128]) of batch row b at position
+        pos < L over the cache with L tokens (tokens 0..pos): the view that
+        row has inside a chunked prefill; fp64 [num_q_heads][128]."""
+        qb = np.ascontiguousarray(_u16(q_row))
+        num_q_heads, d = qb.shape
+        assert d == HEAD_DIM
+        bt = np.ascontiguousarray(bt_row, dtype=np.int32).ravel()
+        if sm_scale is None:
+            sm_scale = 1.0 / np.sqrt(HEAD_DIM)
+        out = np.zeros((num_q_heads, HEAD_DIM), np.float64)
+        rc = lib().s4kv_ref_attention_at(
+            _p(self.pool), _p(self.res_k), _p(self.res_v), self.num_pages, self.num_kv_heads, _p(qb),
+            num_q_heads, int(L), int(pos), _p(bt), bt.size, int(b), float(sm_scale), _p(out), self.bits)
+        if rc != 0:
+            raise ValueError(f"attention_at rc={rc}")
         return out
 
 

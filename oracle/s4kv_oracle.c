@@ -684,6 +684,30 @@ int s4kv_ref_decode_attention(const uint8_t *pool, const uint16_t *res_k,
  * sm_scale * q.k, a two-pass softmax and the weighted sum of values.
  * out: fp64 [n_tokens][num_q_heads][128]; rows of no sequence are left
  * untouched. */
+/* Softmax attention of one query head over tokens 0..pos of the dequantized
+ * K, V (fp64 logits, two-pass softmax); w: scratch of pos + 1 doubles. */
+static void attend_row(const float *K, const float *V, int pos, const uint16_t *qv, double sm_scale, double *w,
+                       double *o) {
+    double mx = -INFINITY;
+    for (int t = 0; t <= pos; ++t) {
+        double acc = 0.0;
+        for (int c = 0; c < HEAD_DIM; ++c)
+            acc += (double)s4kv_ref_half_to_float(qv[c]) * (double)K[(long)t * HEAD_DIM + c];
+        w[t] = sm_scale * acc;
+        if (w[t] > mx) mx = w[t];
+    }
+    double sum = 0.0;
+    for (int t = 0; t <= pos; ++t) {
+        w[t] = exp(w[t] - mx);
+        sum += w[t];
+    }
+    for (int c = 0; c < HEAD_DIM; ++c) {
+        double acc = 0.0;
+        for (int t = 0; t <= pos; ++t) acc += w[t] * (double)V[(long)t * HEAD_DIM + c];
+        o[c] = acc / sum;
+    }
+}
+
 int s4kv_ref_prefill_attention(const uint8_t *pool, const uint16_t *res_k,
                                const uint16_t *res_v, int num_pages,
                                int num_kv_heads, const uint16_t *q,
@@ -714,26 +738,8 @@ int s4kv_ref_prefill_attention(const uint8_t *pool, const uint16_t *res_k,
                 long row = cu_new[b] + j;
                 for (int g = 0; g < G; ++g) {
                     int qh = h * G + g;
-                    const uint16_t *qv = q + (row * num_q_heads + qh) * HEAD_DIM;
-                    double *o = out + (row * num_q_heads + qh) * HEAD_DIM;
-                    double mx = -INFINITY;
-                    for (int t = 0; t <= pos; ++t) {
-                        double acc = 0.0;
-                        for (int c = 0; c < HEAD_DIM; ++c)
-                            acc += (double)s4kv_ref_half_to_float(qv[c]) * (double)K[(long)t * HEAD_DIM + c];
-                        w[t] = sm_scale * acc;
-                        if (w[t] > mx) mx = w[t];
-                    }
-                    double sum = 0.0;
-                    for (int t = 0; t <= pos; ++t) {
-                        w[t] = exp(w[t] - mx);
-                        sum += w[t];
-                    }
-                    for (int c = 0; c < HEAD_DIM; ++c) {
-                        double acc = 0.0;
-                        for (int t = 0; t <= pos; ++t) acc += w[t] * (double)V[(long)t * HEAD_DIM + c];
-                        o[c] = acc / sum;
-                    }
+                    attend_row(K, V, pos, q + (row * num_q_heads + qh) * HEAD_DIM, sm_scale, w,
+                               out + (row * num_q_heads + qh) * HEAD_DIM);
                 }
             }
         }
@@ -741,6 +747,38 @@ int s4kv_ref_prefill_attention(const uint8_t *pool, const uint16_t *res_k,
         free(V);
         free(w);
     }
+    return REF_OK;
+}
+
+/* One query row (all q heads, [num_q_heads][128]) of sequence b at position
+ * pos < L, over the cache as it stands with L tokens: tokens 0..pos, full
+ * pages dequantized and the partial last page from the residual -- the view
+ * of row pos - (L - n) of a chunk of n rows in s4kv_ref_prefill_attention,
+ * without computing the chunk's other rows. */
+int s4kv_ref_attention_at(const uint8_t *pool, const uint16_t *res_k, const uint16_t *res_v, int num_pages,
+                          int num_kv_heads, const uint16_t *q, int num_q_heads, int L, int pos,
+                          const int32_t *bt_row, int max_pages_per_seq, int b, double sm_scale, double *out,
+                          int bits) {
+    if (num_kv_heads <= 0 || num_q_heads % num_kv_heads != 0) return REF_BAD_ARG;
+    if (L <= 0 || pos < 0 || pos >= L || (L + PAGE - 1) / PAGE > max_pages_per_seq) return REF_BAD_ARG;
+    for (int p = 0; p < L / PAGE; ++p)
+        if (bt_row[p] < 0 || bt_row[p] >= num_pages) return REF_BAD_SLOT;
+    int G = num_q_heads / num_kv_heads;
+    size_t rows = (size_t)((L + PAGE - 1) / PAGE + 1) * PAGE;
+    float *K = (float *)malloc(sizeof(float) * rows * HEAD_DIM);
+    float *V = (float *)malloc(sizeof(float) * rows * HEAD_DIM);
+    double *w = (double *)malloc(sizeof(double) * (size_t)L);
+    if (!K || !V || !w) { free(K); free(V); free(w); return REF_BAD_ARG; }
+    for (int h = 0; h < num_kv_heads; ++h) {
+        sequence_kv(pool, res_k, res_v, num_kv_heads, bt_row, L, b, h, K, V, bits);
+        for (int g = 0; g < G; ++g) {
+            int qh = h * G + g;
+            attend_row(K, V, pos, q + (long)qh * HEAD_DIM, sm_scale, w, out + (long)qh * HEAD_DIM);
+        }
+    }
+    free(K);
+    free(V);
+    free(w);
     return REF_OK;
 }
 

@@ -98,7 +98,7 @@ def test_full_size_prefill_sampled_parity(name):
     """The prefill workload at full shape in the launch configuration the
     bench times (the whole chunk of every sequence in one call): sampled
     sequences' pool pages bit-exact against the oracle's, and the last rows
-    of their chunks within 2e-3 + 1e-3 |ref|."""
+    of their chunks and sampled interior rows within 2e-3 + 1e-3 |ref|."""
     import torch
     import oracle
     import bench
@@ -136,6 +136,16 @@ def test_full_size_prefill_sampled_parity(name):
                                    np.array([L], np.int32), bt)
         got = out[torch.from_numpy(last).to(dev)].float().cpu().numpy()
         assert_attention_close(got, ref, f"{spec.name} seq {b} last rows (L={L})")
+        # interior rows of the chunk, where the causal limit cuts key tiles:
+        # the first row, both sides of a query-tile and a key-tile boundary,
+        # and one deep inside, each against the oracle's row at its position
+        n = int(cu[b + 1] - cu[b])
+        for j in (0, 127, 128, 1023):
+            row = int(cu[b]) + j
+            q_row = q[row].cpu().numpy()
+            ref_row = oc.attention_at(q_row, 0, L, L - n + j, bt[0])
+            got_row = out[row].float().cpu().numpy()
+            assert_attention_close(got_row, ref_row, f"{spec.name} seq {b} chunk row {j} (L={L})")
     del wl
     gc.collect()
     torch.cuda.empty_cache()

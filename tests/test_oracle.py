@@ -34,6 +34,8 @@ Which pin covers which oracle function:
                                    inputs the quantizer represents exactly, per
                                    query position; the chunk's last row equals
                                    decode attention
+  attention_at                  : the same textbook attention for one row at a
+                                   given position, and the chunk's row there
 """
 import os
 from fractions import Fraction
@@ -618,6 +620,35 @@ def test_prefill_last_row_is_decode(oracle_mod):
     last = q[cu[1:] - 1]
     dec = c.decode_attention(last, np.array(after, np.int32), bt, sm_scale=0.07)
     assert np.array_equal(out[cu[1:] - 1], dec)
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+def test_attention_at_matches_textbook_and_the_chunk_rows(oracle_mod, bits):
+    """One query row at position pos over the cache as it stands: plain
+    softmax attention (numpy, float64) over the fp16 keys and values 0..pos on
+    exact grids, and exactly the row a chunk whose row sits at pos gets.
+    Positions on both sides of page boundaries, inside the partial last
+    page, and 0."""
+    rng = np.random.default_rng(33 + bits)
+    H, G = 2, 3
+    after = [45, 33]
+    k, v = _grid_streams(rng, after, H, bits)
+    bt, NP = _tables(rng, after)
+    c = oracle_mod.OracleCache(NP, H, len(after), bits=bits)
+    _append_all(oracle_mod, c, k, v, [0, 0], after, bt)
+    n = np.array(after)
+    cu = np.concatenate([[0], np.cumsum(n)]).astype(np.int32)
+    q = rng.standard_normal((int(cu[-1]), H * G, HD)).astype(np.float16)
+    chunk = c.prefill_attention(q, cu, np.array(after, np.int32), bt)
+    scale = 1 / np.sqrt(HD)
+    for b, positions in ((0, [0, 15, 16, 31, 32, 40, 44]), (1, [0, 17, 31, 32])):
+        for pos in positions:
+            row = cu[b] + pos
+            got = c.attention_at(q[row], b, after[b], pos, bt[b])
+            assert np.array_equal(got, chunk[row]), (b, pos)
+            for qh in range(H * G):
+                ref = _textbook_attention(q[row, qh], k[b][:pos + 1, qh // G], v[b][:pos + 1, qh // G], scale)
+                assert np.allclose(got[qh], ref, rtol=1e-12, atol=1e-12), (b, pos, qh)
 
 
 # ------------------------------------------------------ page movement --
