@@ -788,17 +788,22 @@ def main(argv=None):
     achieved = decode_bytes_per_launch / (dec_avg_ms * 1e-3) / 1e9
     tokens = int(wl.new.sum())
     prefill = moves = fused = int8 = int2 = configs = None
+    extra_clocks = None
     if world == 1 and not args.no_prefill:
-        prefill = [measure_prefill(device, max(3, min(args.steps, 20)), w, args.bits) for w in W.PREFILL_ORDER]
-        moves = measure_page_moves(wl, device)
+        # the HBM-bound measurements first: the tensor-bound prefill runs at
+        # the power cap and leaves the clocks lower for a while afterwards
+        extra = ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ
+                             else int(os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local]))
+        extra.start()
         fused = [measure_fused_step(wl, device)]
-        small = DeviceWorkload(W.SPECS["qwen2.5-7b"], device)
-        fused.append(measure_fused_step(small, device))
-        del small
-        int8 = measure_width_decode(device, spec, 8)
-        int2 = measure_width_decode(device, spec, 2)
+        moves = measure_page_moves(wl, device)
         configs = [measure_decode_config(device, name) for name in W.CONFIG_ORDER
                    if name not in ("tiny", spec.name.split("-b")[0] if args.batch else spec.name)]
+        int8 = measure_width_decode(device, spec, 8)
+        int2 = measure_width_decode(device, spec, 2)
+        prefill = [measure_prefill(device, max(3, min(args.steps, 20)), w, args.bits) for w in W.PREFILL_ORDER]
+        extra.stop()
+        extra_clocks = extra.summary()
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(spec, bits=args.bits)
@@ -836,8 +841,9 @@ def main(argv=None):
         if cpu is not None:
             line["cpu_baseline"] = cpu
         if prefill is not None:
-            line["next_rows"] = {"prefill": prefill, "page_moves": moves, "fused_step": fused, "int8_decode": int8,
-                                 "int2_decode": int2, "decode_configs": configs}
+            line["next_rows"] = {"decode_configs": configs, "fused_step": fused, "int8_decode": int8,
+                                 "int2_decode": int2, "page_moves": moves, "prefill": prefill,
+                                 "clocks": extra_clocks}
         print(json.dumps(line), flush=True)
     if world > 1:
         torch.distributed.destroy_process_group()
