@@ -724,11 +724,14 @@ __global__ void __launch_bounds__(threads_for<kBits>(), min_ctas_for<kBits>())
         next_segment(ac, p);
       }
       if (lane == 0) s_njob[warp] = nj;
-      __syncthreads();
-      for (int w = 0; w < kWarpsPerCta; ++w)
-        for (int j = 0; j < s_njob[w]; ++j) cta_quantize_job<kBits, kThreads>(p, f, s_job[w][j], smem, threadIdx.x);
-      // the pool writes are read next by bulk copies (async proxy)
-      asm volatile("fence.proxy.async.global;" ::: "memory");
+      // one barrier tells whether any warp of the CTA found a completed page
+      // (most steps complete none): only then the CTA quantizes and fences
+      if (__syncthreads_or(nj > 0)) {
+        for (int w = 0; w < kWarpsPerCta; ++w)
+          for (int j = 0; j < s_njob[w]; ++j) cta_quantize_job<kBits, kThreads>(p, f, s_job[w][j], smem, threadIdx.x);
+        // the pool writes are read next by bulk copies (async proxy)
+        asm volatile("fence.proxy.async.global;" ::: "memory");
+      }
       if (!__syncthreads_or(more)) break;
     }
   }
