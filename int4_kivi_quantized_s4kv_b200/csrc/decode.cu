@@ -53,10 +53,10 @@
 
 namespace s4kv {
 
-// Build-time tuning constants: stages per warp ring; worker warps per CTA
-// (4- and 2-bit pages: one CTA of 12 warps per SM, so that all warps of an SM
-// are equally old and the warp schedulers serve them alike; 4864-byte int8
-// blocks: two CTAs of 4 warps with 5 stages each); the fewest pages a worker
+// Build-time tuning constants: stages per warp ring; worker warps per CTA,
+// one CTA per SM so that all warps of an SM are equally old and the warp
+// schedulers serve them alike (4- and 2-bit pages: 12 warps with 6 stages;
+// 4864-byte int8 blocks: 8 warps with 5 stages); the fewest pages a worker
 // is given, so that small batches are not cut into many short pieces.
 #ifndef S4KV_DECODE_STAGES
 #define S4KV_DECODE_STAGES 6
@@ -68,7 +68,7 @@ namespace s4kv {
 #define S4KV_DECODE_STAGES_INT8 5
 #endif
 #ifndef S4KV_DECODE_WARPS_INT8
-#define S4KV_DECODE_WARPS_INT8 4
+#define S4KV_DECODE_WARPS_INT8 8
 #endif
 #ifndef S4KV_DECODE_MIN_PAGES
 #define S4KV_DECODE_MIN_PAGES 16

@@ -119,6 +119,23 @@ def test_many_short_sequences_fewer_pages_than_workers():
     assert_attention_close(p.gpu_decode(), p.oracle_decode(), "short sequences")
 
 
+def test_large_batch_of_short_and_empty_sequences():
+    """600 sequences (more than 8 per lane of the plan's scan), lengths 0..70
+    with some empty: segments of a single page or only a residual, many
+    segments per worker, and the floor on pages per worker."""
+    rng = np.random.default_rng(5)
+    ctx = rng.integers(0, 70, 600)
+    ctx[rng.choice(600, 40, replace=False)] = 0
+    step = tuple(int(x) for x in np.where(ctx == 0, 0, 1))
+    spec = _spec("large-batch", batch=600, num_q_heads=16, num_kv_heads=2,
+                 ctx_fixed=tuple(int(x) for x in ctx), step_new=step)
+    p = Pair(spec)
+    p.assert_cache_bit_exact()
+    got = p.gpu_decode()
+    assert not got[p.lens == 0].any()
+    assert_attention_close(got[p.lens > 0], p.oracle_decode()[p.lens > 0], "600 short sequences")
+
+
 def test_sm_scale_parameter():
     spec = _spec("scale", batch=3, num_q_heads=8, num_kv_heads=2, ctx_fixed=(50, 70, 90))
     p = Pair(spec)
