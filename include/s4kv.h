@@ -228,9 +228,12 @@ S4KV_API int s4kv_decode_attention(const s4kv_cache_t *cache, const void *q,
                           void *workspace, size_t workspace_bytes,
                           void *stream);
 
-/* One decode step in one launch: the append of one new token per sequence
- * fused into s4kv_decode_attention (row (L-1) % 16 of the last page; a page
- * completed by it is quantized inside the same kernel, before any read of it).
+/* One decode step in one call: the append of one new token per sequence
+ * (row (L-1) % 16 of the last page; a page completed by it is quantized), then
+ * s4kv_decode_attention over the grown cache.  The append runs as its own
+ * grid and the decode grid is launched as its programmatic dependent: the
+ * decode grid's launch and split plan overlap the append, and it reads the
+ * cache only after the append grid has completed.
  *  k_new, v_new  device fp16 [batch][num_kv_heads][128], 16-B aligned: the
  *          token of sequence b at position seq_lens[b] - 1.  A sequence with
  *          seq_lens[b] == 0 has no token and gets zeros.

@@ -201,8 +201,9 @@ def s4kv_decode_attention(cache: S4KVCache, q, seq_lens, block_tables, out, work
 
 def s4kv_append_decode(cache: S4KVCache, k_new, v_new, q, seq_lens, block_tables, out, workspace,
                        sm_scale: float | None = None, stream=None):
-    """One decode step in one launch: append each sequence's new token
-    (k_new, v_new fp16 [batch][kv_heads][128]) and attend over the result."""
+    """One decode step in one call: append each sequence's new token
+    (k_new, v_new fp16 [batch][kv_heads][128]) and attend over the result
+    (an append grid, then the decode grid as its programmatic dependent)."""
     import torch
     batch, num_q_heads, _ = q.shape
     if sm_scale is None:

@@ -244,6 +244,8 @@ int decode_call(const s4kv_cache_t *cache, const void *k_new, const void *v_new,
   rc = s4kv_check_model(cache->head_dim, cache->page_tokens, num_q_heads, cache->num_kv_heads);
   if (rc != S4KV_OK) return rc;
   if (batch < 0 || batch > cache->max_seqs || max_pages_per_seq <= 0) return S4KV_ERR_INVALID_ARG;
+  // the step's append grid has one CTA per (sequence, kv head)
+  if (k_new && static_cast<long long>(batch) * cache->num_kv_heads > 0x7FFFFFFF) return S4KV_ERR_INVALID_ARG;
   if (!(std::isfinite(sm_scale)) || sm_scale <= 0.0f) return S4KV_ERR_INVALID_ARG;
   if (batch == 0) return S4KV_OK;
   if (!q || !seq_lens || !block_tables || !out) return S4KV_ERR_INVALID_ARG;
@@ -285,8 +287,10 @@ int decode_call(const s4kv_cache_t *cache, const void *k_new, const void *v_new,
   FusedAppend f;
   f.k_new = static_cast<const __half *>(k_new);
   f.v_new = static_cast<const __half *>(v_new);
-  launch_decode(p, f, cache_bits(cache), d.num_ctas[fi], static_cast<cudaStream_t>(stream));
-  if (cudaGetLastError() != cudaSuccess) return S4KV_ERR_CUDA;
+  if (launch_decode(p, f, cache_bits(cache), d.num_ctas[fi], static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+    cudaGetLastError();
+    return S4KV_ERR_CUDA;
+  }
   return S4KV_OK;
 }
 

@@ -542,15 +542,14 @@ __device__ __forceinline__ void merge_pieces(const DecodeParams &p, long obase, 
   }
 }
 
-// Fused append of one decode step for (sequence b, kv head h) whose length
-// after the append is L >= 1: the new token (row b of k_new / v_new) is
-// position L - 1, row (L - 1) % 16 of the sequence's last page.
+// Append of one decode step (s4kv_append_decode) for (sequence b, kv head h)
+// whose length after the append is L >= 1: the new token (row b of k_new /
+// v_new) is position L - 1, row (L - 1) % 16 of the sequence's last page.
 //  * If that row is not the page's last, one warp writes the token into the
 //    residual (lane l: channels 4l .. 4l + 3).
 //  * Otherwise the token completes the page, which is quantized from the
 //    residual rows 0..14 plus the token by the whole CTA (quantize_page_cta,
 //    the routine s4kv_append uses, so the bytes are the same).
-constexpr int kJobsPerWarp = 8;
 
 __device__ __forceinline__ void residual_row_write(const DecodeParams &p, const FusedAppend &f, int b, int h, int L,
                                                    int lane) {
@@ -558,7 +557,7 @@ __device__ __forceinline__ void residual_row_write(const DecodeParams &p, const 
   const long rbase = (static_cast<long>(b) * H + h) * kPage * kHeadDim + 4 * lane;
   const long nbase = (static_cast<long>(b) * H + h) * kHeadDim + 4 * lane;
   const int r = (L - 1) % kPage;
-  // the cache is written only by the fused append (the parameters carry it
+  // the cache is written only by the step's append (the parameters carry it
   // read-only for the attention)
   __half *res_k = const_cast<__half *>(p.res_k), *res_v = const_cast<__half *>(p.res_v);
   *reinterpret_cast<uint2 *>(res_k + rbase + r * kHeadDim) = *reinterpret_cast<const uint2 *>(f.k_new + nbase);
@@ -592,10 +591,41 @@ __device__ __forceinline__ void cta_quantize_job(const DecodeParams &p, const Fu
   __syncthreads();  // the scratch is reused by the next job
 }
 
-// kFused: the step's append is fused in (DecodeParams::k_new / v_new set).
-template <int kBits, bool kFused>
+// The step's append grid: one 128-thread CTA per (sequence, kv head), as in
+// s4kv_append, so that the pages completed in one step (all kv heads of a
+// sequence complete together) are quantized side by side.  Warp 0 writes a
+// row that completes nothing; the whole CTA quantizes a completed page.
+constexpr int kStepThreads = 128;
+constexpr int kQuantScratch = 2 * kPage * kHeadDim * 2 + 2 * kPage * kHeadDim;
+
+template <int kBits>
+__global__ void __launch_bounds__(kStepThreads) step_append_kernel(const DecodeParams p, const FusedAppend f) {
+  // the dependent decode grid may start now: it plans its split while this
+  // grid runs and waits for this grid's completion before it reads the cache
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  __shared__ __align__(16) uint8_t scratch[kQuantScratch];
+  const int H = p.num_kv_heads;
+  const int b = static_cast<int>(blockIdx.x / H), h = static_cast<int>(blockIdx.x % H);
+  const int L = __ldg(p.seq_lens + b);
+  // no token (L == 0), or a length the decode grid flags as out of range
+  if (L <= 0 || L > p.max_pages * kPage) return;
+  if (L % kPage != 0) {
+    if (threadIdx.x < 32) residual_row_write(p, f, b, h, L, threadIdx.x);
+    return;
+  }
+  const int phys = __ldg(p.block_tables + static_cast<long>(b) * p.max_pages + (L - 1) / kPage);
+  if (static_cast<unsigned>(phys) >= static_cast<unsigned>(p.num_pages)) {
+    if (threadIdx.x == 0) flag_error(p.err, S4KV_EFLAG_PAGE_RANGE);
+    return;
+  }
+  cta_quantize_job<kBits, kStepThreads>(p, f, make_int4(b, h, L, phys), scratch, threadIdx.x);
+  // the pool writes are read next by the decode grid's bulk copies (async proxy)
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+template <int kBits>
 __global__ void __launch_bounds__(threads_for<kBits>(), min_ctas_for<kBits>())
-    decode_kernel(const DecodeParams p, const FusedAppend f) {
+    decode_kernel(const DecodeParams p) {
   constexpr int kStages = stages_for<kBits>();
   constexpr int kWarpsPerCta = warps_for<kBits>();
   constexpr int kThreads = threads_for<kBits>();
@@ -657,8 +687,6 @@ __global__ void __launch_bounds__(threads_for<kBits>(), min_ctas_for<kBits>())
       }
     }
   }
-  // every warp of the CTA, with work or not, takes part in its barriers (the
-  // fused append's and the final merge's)
   if (T == 0) return;
   const bool active = worker < W;
   const long long s = active ? worker * T / W : 0;
@@ -690,51 +718,12 @@ __global__ void __launch_bounds__(threads_for<kBits>(), min_ctas_for<kBits>())
   const int range = static_cast<int>(e - s);
   const int p_first = static_cast<int>(s - cc.start);
 
-  // ---- fused append: the step's new token of every segment whose last page
-  // lies in this worker's range (each segment has exactly one such worker,
-  // the one that also reads that page) is written before any copy of it.  A
-  // token that completes its page makes a job for the whole CTA; jobs are
-  // collected up to kJobsPerWarp per warp and round, then quantized.
-  if (kFused) {
-    __shared__ int4 s_job[kWarpsPerCta][kJobsPerWarp];
-    __shared__ int s_njob[kWarpsPerCta];
-    Cursor ac = cc;
-    bool more = active;
-    while (true) {
-      int nj = 0;
-      while (more && nj < kJobsPerWarp) {
-        if (ac.b >= B || ac.start >= e) {
-          more = false;
-          break;
-        }
-        const long long last = ac.start + ac.np - 1;
-        if (last >= s && last < e && ac.len > 0) {
-          if (ac.len % kPage != 0) {
-            residual_row_write(p, f, ac.b, ac.h, ac.len, lane);
-          } else {
-            const int phys = __ldg(ac.bt + (ac.len - 1) / kPage);
-            if (static_cast<unsigned>(phys) >= static_cast<unsigned>(p.num_pages)) {
-              if (lane == 0) flag_error(p.err, S4KV_EFLAG_PAGE_RANGE);
-            } else {
-              if (lane == 0) s_job[warp][nj] = make_int4(ac.b, ac.h, ac.len, phys);
-              ++nj;
-            }
-          }
-        }
-        next_segment(ac, p);
-      }
-      if (lane == 0) s_njob[warp] = nj;
-      // one barrier tells whether any warp of the CTA found a completed page
-      // (most steps complete none): only then the CTA quantizes and fences
-      if (__syncthreads_or(nj > 0)) {
-        for (int w = 0; w < kWarpsPerCta; ++w)
-          for (int j = 0; j < s_njob[w]; ++j) cta_quantize_job<kBits, kThreads>(p, f, s_job[w][j], smem, threadIdx.x);
-        // the pool writes are read next by bulk copies (async proxy)
-        asm volatile("fence.proxy.async.global;" ::: "memory");
-      }
-      if (!__syncthreads_or(more)) break;
-    }
-  }
+  // s4kv_append_decode launches this grid as the programmatic dependent of
+  // its append grid: everything above (the plan, the zeroed outputs) reads
+  // nothing that grid writes, and here every thread waits for that grid's
+  // completion and its writes before the cache is read.  Launched plainly
+  // (no dependency), the wait returns at once.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 
   if (active) {
   // ---- producer: issue the next quantized pages of [s, e) into the ring.
@@ -1045,12 +1034,9 @@ __global__ void __launch_bounds__(threads_for<kBits>(), min_ctas_for<kBits>())
 
 template <int kBits>
 int ctas_per_sm_for() {
-  int n = 0, m = 0;
-  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_kernel<kBits, false>, threads_for<kBits>(),
-                                                smem_bytes_for<kBits>());
-  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&m, decode_kernel<kBits, true>, threads_for<kBits>(),
-                                                smem_bytes_for<kBits>());
-  return n < m ? n : m;  // one launch shape serves the plain and the fused kernel
+  int n = 0;
+  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_kernel<kBits>, threads_for<kBits>(), smem_bytes_for<kBits>());
+  return n;
 }
 
 int decode_ctas_per_sm(int bits) {
@@ -1063,10 +1049,8 @@ int decode_warps_per_cta(int bits) {
 
 template <int kBits>
 cudaError_t prepare_for() {
-  const int bytes = static_cast<int>(smem_bytes_for<kBits>());
-  cudaError_t e = cudaFuncSetAttribute(decode_kernel<kBits, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-  if (e != cudaSuccess) return e;
-  return cudaFuncSetAttribute(decode_kernel<kBits, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  return cudaFuncSetAttribute(decode_kernel<kBits>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              static_cast<int>(smem_bytes_for<kBits>()));
 }
 
 cudaError_t prepare_decode_kernel() {
@@ -1077,24 +1061,34 @@ cudaError_t prepare_decode_kernel() {
   return prepare_for<2>();
 }
 
-void launch_decode(const DecodeParams &p, const FusedAppend &f, int bits, int num_ctas, cudaStream_t stream) {
-  const bool fused = f.k_new != nullptr;
-  if (bits == 8) {
-    if (fused)
-      decode_kernel<8, true><<<num_ctas, threads_for<8>(), smem_bytes_for<8>(), stream>>>(p, f);
-    else
-      decode_kernel<8, false><<<num_ctas, threads_for<8>(), smem_bytes_for<8>(), stream>>>(p, f);
-  } else if (bits == 2) {
-    if (fused)
-      decode_kernel<2, true><<<num_ctas, threads_for<2>(), smem_bytes_for<2>(), stream>>>(p, f);
-    else
-      decode_kernel<2, false><<<num_ctas, threads_for<2>(), smem_bytes_for<2>(), stream>>>(p, f);
-  } else {
-    if (fused)
-      decode_kernel<4, true><<<num_ctas, threads_for<4>(), smem_bytes_for<4>(), stream>>>(p, f);
-    else
-      decode_kernel<4, false><<<num_ctas, threads_for<4>(), smem_bytes_for<4>(), stream>>>(p, f);
+template <int kBits>
+cudaError_t launch_for(const DecodeParams &p, const FusedAppend &f, int num_ctas, cudaStream_t stream) {
+  if (f.k_new == nullptr) {
+    decode_kernel<kBits><<<num_ctas, threads_for<kBits>(), smem_bytes_for<kBits>(), stream>>>(p);
+    return cudaGetLastError();
   }
+  // one decode step: the append grid, then the decode grid as its
+  // programmatic dependent (launched while the append runs; it waits for the
+  // append's completion before reading the cache)
+  step_append_kernel<kBits><<<static_cast<unsigned>(p.batch * p.num_kv_heads), kStepThreads, 0, stream>>>(p, f);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(num_ctas));
+  cfg.blockDim = dim3(threads_for<kBits>());
+  cfg.dynamicSmemBytes = smem_bytes_for<kBits>();
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, decode_kernel<kBits>, p);
+}
+
+cudaError_t launch_decode(const DecodeParams &p, const FusedAppend &f, int bits, int num_ctas, cudaStream_t stream) {
+  return bits == 8 ? launch_for<8>(p, f, num_ctas, stream)
+                   : bits == 2 ? launch_for<2>(p, f, num_ctas, stream) : launch_for<4>(p, f, num_ctas, stream);
 }
 
 }  // namespace s4kv

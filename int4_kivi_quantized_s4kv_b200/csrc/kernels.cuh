@@ -79,9 +79,9 @@ struct DecodeParams {
   int num_workers;
 };
 
-// Fused append of a decode step: each sequence's new token (fp16
-// [batch][kv_heads][128]) is written into the cache before the attention
-// reads it.  Both nullptr for a plain decode.
+// The append of a decode step (s4kv_append_decode): each sequence's new
+// token (fp16 [batch][kv_heads][128]) is written into the cache by an append
+// grid that the decode grid depends on.  Both nullptr for a plain decode.
 struct FusedAppend {
   const __half *k_new;
   const __half *v_new;
@@ -90,7 +90,7 @@ struct FusedAppend {
 void launch_append(const AppendParams &p, int batch, int max_new, cudaStream_t stream);
 void launch_dequant(const DequantParams &p, cudaStream_t stream);
 void launch_move(const MoveParams &p, cudaStream_t stream);
-void launch_decode(const DecodeParams &p, const FusedAppend &f, int bits, int num_ctas, cudaStream_t stream);
+cudaError_t launch_decode(const DecodeParams &p, const FusedAppend &f, int bits, int num_ctas, cudaStream_t stream);
 int decode_ctas_per_sm(int bits);
 int decode_warps_per_cta(int bits);
 cudaError_t prepare_decode_kernel();

@@ -1,5 +1,5 @@
 // Page quantization by one 128-thread CTA, shared by s4kv_append and the
-// fused append of s4kv_append_decode so that both write the same bytes.
+// step append grid of s4kv_append_decode so that both write the same bytes.
 //
 // KIVI split ("S4 KV -- int4 KV-Cache-Kompression fuer vLLM", "Funktionsweise"
 // step 1): keys asymmetric int4 per channel (one group = one channel over the

@@ -1,6 +1,7 @@
-"""GPU parity of s4kv_append_decode (one decode step in one launch: the
-append of one token per sequence fused into decode attention) against the
-oracle's append-then-decode, through the C ABI.  The cache after the step must
+"""GPU parity of s4kv_append_decode (one decode step in one call: the
+append of one token per sequence, then decode attention as a grid that
+depends on the append's) against the oracle's append-then-decode, through
+the C ABI.  The cache after the step must
 be byte-identical to the oracle's, the output within the decode tolerance,
 and the output bit-identical to the GPU's own two-launch path."""
 import dataclasses
@@ -69,6 +70,15 @@ def test_fused_step_completes_and_starts_pages():
     # 1 is a sequence's very first token; 17, 101, 201 land in the residual
     spec = dataclasses.replace(W.SPECS["llama3.2-3b-step"], name="fused-mix", layers=1, batch=7,
                                ctx_kind="fixed", ctx_fixed=(15, 31, 16, 100, 47, 200, 0), step_new=(1,))
+    _run(spec)
+
+
+def test_fused_step_every_segment_completes_a_page():
+    # every (sequence, kv head) completes a page: each append CTA quantizes
+    # the most pages it can hold, one after the other
+    ctx = tuple(16 * (1 + (b * 7) % 9) - 1 for b in range(40))
+    spec = dataclasses.replace(W.SPECS["llama3.2-3b-step"], name="fused-fills", layers=1, batch=len(ctx),
+                               ctx_kind="fixed", ctx_fixed=ctx, step_new=(1,))
     _run(spec)
 
 
