@@ -33,10 +33,13 @@
 //     tile's 128 MMA rows are (token, head of the group) pairs, so a tile
 //     holds floor(128 / G) tokens.  Warps with separate roles hand buffers
 //     over through mbarriers:
-//      * a producer warp brings each key tile's K_hi, K_lo (64 KB) and V^T
+//      * two producer warps bring each key tile's K_hi, K_lo (64 KB) and V^T
 //        (32 KB) into one of two K and one of two V buffers with 1-D bulk
 //        copies (TMA engine, no multicast); a K buffer is refilled as soon as
-//        the S MMAs that read it complete, a V buffer once the PV MMAs have;
+//        the S MMAs that read it complete, a V buffer once the PV MMAs have,
+//        each by its own warp so that neither copy queues behind the other's
+//        buffer (the tiles come from L2 at a few tens of bytes per cycle per
+//        SM, so K must be issued two tiles ahead);
 //      * one thread issues S(k) = Q K_hi^T + Q K_lo^T (M = 128, N = 128 keys,
 //        one accumulation over K = 256: the 128 channels against K_hi, then
 //        against K_lo) into one of two tensor-memory S buffers, then
@@ -65,8 +68,9 @@ namespace {
 
 constexpr int kSoftmaxWarps = 4;   // warps 0..3: one row per thread
 constexpr int kMmaWarp = 4;
-constexpr int kProducerWarp = 5;
-constexpr int kThreadsP = 32 * 6;
+constexpr int kKProducerWarp = 5;  // K tiles
+constexpr int kVProducerWarp = 6;  // V tiles
+constexpr int kThreadsP = 32 * 7;
 constexpr int kKeyTile = 128;                    // keys per tile
 constexpr int kPagesPerTile = kKeyTile / kPage;  // 8
 constexpr int kOpPages = kPagesPerTile / 2;       // operand kernel: half a key tile per CTA
@@ -78,6 +82,10 @@ constexpr uint32_t kVBytes = 128 * kKeyTile * 2;       // V^T [128][128] fp16
 constexpr uint32_t kTileBytes = kKBytes + kVBytes;     // workspace tile
 constexpr uint32_t kHalfTileBytes = kTileBytes / 2;
 constexpr float kSlack = 8.0f;                   // log2 slack of the softmax reference
+#ifndef S4KV_PREFILL_POLY_OF8
+#define S4KV_PREFILL_POLY_OF8 3
+#endif
+constexpr int kPolyOf8 = S4KV_PREFILL_POLY_OF8;  // eighths of the exponentials on the FMA pipe
 constexpr long long kWaitLimit = 2000000000LL;   // about one second
 // S: M = 128, N = 128 keys, K = 256 (Q against K_hi, then Q against K_lo,
 // accumulated); PV: M = 128, N = 128
@@ -126,6 +134,53 @@ __device__ __forceinline__ void wait_landed(uint32_t bar, uint32_t parity) {
   const long long t0 = clock64();
   while (!mbar_try_wait(bar, parity) && clock64() - t0 <= kWaitLimit) {
   }
+}
+
+
+// One elected lane of the (converged) warp issues the MMA / the commit.
+__device__ __forceinline__ void mma_ss_elect(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                             uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\telect.sync _|e, 0xffffffff;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void mma_ts_elect(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                             uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\telect.sync _|e, 0xffffffff;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void commit_elect(uint32_t bar) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(bar)
+      : "memory");
+}
+// 2^x for a pair, on the FMA/ALU pipes instead of the MUFU pipe.  Cody and
+// Waite's range reduction: x = j + f with j = rint(x) (adding 1.5 * 2^23
+// rounds x to an integer held in the sum's low mantissa bits) and
+// f in [-1/2, 1/2]; 2^f from a cubic; 2^j applied by adding j to the
+// exponent field (the sum's bits shifted left by 23 are j << 23, since the
+// constant's own bits vanish under the shift).  The cubic was fitted for this
+// kernel by iteratively reweighted least squares towards the smallest maximum
+// relative error over [-1/2, 1/2]: 7.5e-5 in fp32 Horner evaluation, well
+// below the 2^-11 of the fp16 rounding P goes through.  x is clamped at -125,
+// so that 2^j * p(f) stays a normal number (weights below 2^-125 are 0 to
+// fp16 and nothing to the fp32 row sum).
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+  const float2 xc = make_float2(fmaxf(x.x, -125.0f), fmaxf(x.y, -125.0f));
+  const float2 t = add2(xc, make_float2(kRound, kRound));
+  const float2 f = sub2(xc, sub2(t, make_float2(kRound, kRound)));
+  float2 q = fma2(f, make_float2(0.0551716685f, 0.0551716685f), make_float2(0.2426111400f, 0.2426111400f));
+  q = fma2(q, f, make_float2(0.6932609677f, 0.6932609677f));
+  q = fma2(q, f, make_float2(0.9999280572f, 0.9999280572f));
+  return make_float2(__uint_as_float(__float_as_uint(q.x) + (__float_as_uint(t.x) << 23)),
+                     __uint_as_float(__float_as_uint(q.y) + (__float_as_uint(t.y) << 23)));
 }
 
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
@@ -456,83 +511,88 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(const PrefillPara
     *abort_flag = 1;
   };
 
-  if (warp == kProducerWarp) {
-    // ---------------------------------------------------------- producer
-    // K(kt) into K buffer kt % 2 once S(kt - 2) has read it; V(kt) into V
+  if (warp == kKProducerWarp || warp == kVProducerWarp) {
+    // --------------------------------------------------------- producers
+    // one warp per operand, so that neither waits behind the other's buffer:
+    // K(kt) into K buffer kt % 2 once S(kt - 2) has read it, V(kt) into V
     // buffer kt % 2 once O += P(kt - 2) V(kt - 2) has
     if (lane == 0) {
-      const uint8_t *tiles = p.ws + (static_cast<long long>(b) * H + h) * p.tiles_per_seq * kTileBytes;
+      const bool is_k = warp == kKProducerWarp;
+      const uint32_t bytes = is_k ? kKBytes : kVBytes;
+      const uint8_t *tiles = p.ws + (static_cast<long long>(b) * H + h) * p.tiles_per_seq * kTileBytes + (is_k ? 0 : kKBytes);
+      auto full = [&](int s) { return is_k ? k_full(s) : v_full(s); };
       int issued = 0;
       for (int kt = 0; kt < n_ktiles; ++kt) {
         const int s = kt % kStages, u = kt / kStages;
-        const uint8_t *src = tiles + static_cast<long long>(kt) * kTileBytes;
-        if (kt >= kStages && !wait_bounded(k_empty(s), (u - 1) & 1, abort_flag)) {
+        if (kt >= kStages && !wait_bounded(is_k ? k_empty(s) : v_empty(s), (u - 1) & 1, abort_flag)) {
           fail();
           break;
         }
-        mbar_arrive_expect_tx(k_full(s), kKBytes);
-        bulk_copy_g2s(kbuf(s), src, kKBytes, k_full(s));
-        issued = 2 * kt + 1;
-        if (kt >= kStages && !wait_bounded(v_empty(s), (u - 1) & 1, abort_flag)) {
-          fail();
-          break;
-        }
-        mbar_arrive_expect_tx(v_full(s), kVBytes);
-        bulk_copy_g2s(vbuf(s), src + kKBytes, kVBytes, v_full(s));
-        issued = 2 * kt + 2;
+        mbar_arrive_expect_tx(full(s), bytes);
+        bulk_copy_g2s(is_k ? kbuf(s) : vbuf(s), tiles + static_cast<long long>(kt) * kTileBytes, bytes, full(s));
+        issued = kt + 1;
       }
       // before the CTA exits, the copies in flight must have landed (bounded
-      // by time only, also after an abort): at most the last kStages of each
-      // kind can still be in flight
-      for (int c = max(0, issued - 2 * kStages); c < issued; ++c) {
-        const int kt = c >> 1, s = kt % kStages;
-        wait_landed((c & 1) ? v_full(s) : k_full(s), (kt / kStages) & 1);
-      }
+      // by time only, also after an abort): at most the last kStages
+      for (int kt = max(0, issued - kStages); kt < issued; ++kt) wait_landed(full(kt % kStages), (kt / kStages) & 1);
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------- MMA issuer
-    if (lane == 0) {
-      auto issue_pv = [&](int k) {  // O += P(k) V(k), P read from tensor memory
-        const int vs = k % kStages;
-        if (!wait_bounded(v_full(vs), (k / kStages) & 1, abort_flag) || !wait_bounded(p_full, k & 1, abort_flag))
-          return false;
-        tc05::fence_after_sync();
+    // The whole warp runs the loop, so that descriptors and decisions stay
+    // warp-uniform; one elected lane issues each MMA and commit.
+    auto wait_w = [&](uint32_t bar, uint32_t parity) {
+      return __all_sync(0xFFFFFFFFu, wait_bounded(bar, parity, abort_flag));
+    };
+    const uint64_t dq = tc05::smem_desc_sw128(sQ);
+    const uint64_t dk0 = tc05::smem_desc_sw128(kbuf(0)), dk1 = tc05::smem_desc_sw128(kbuf(1));
+    const uint64_t dv0 = tc05::smem_desc_sw128(vbuf(0)), dv1 = tc05::smem_desc_sw128(vbuf(1));
+    auto issue_pv = [&](int k) {  // O += P(k) V(k), P read from tensor memory
+      const int vs = k % kStages;
+      const bool vf = mbar_try_wait(v_full(vs), (k / kStages) & 1);
+      const bool pf = mbar_try_wait(p_full, k & 1);
+      if (!__all_sync(0xFFFFFFFFu, vf && pf) && (!wait_w(v_full(vs), (k / kStages) & 1) || !wait_w(p_full, k & 1)))
+        return false;
+      tc05::fence_after_sync();
+      const uint64_t dv = vs ? dv1 : dv0;
 #pragma unroll
-        for (int j = 0; j < kKeyTile / 16; ++j)
-          tc05::mma_f16_ts(tO, tP + 8 * j, tc05::smem_desc_sw128(vbuf(vs) + (j >> 2) * (kVBytes / 2) + (j & 3) * 32),
-                           kIdescO, (k > 0 || j > 0) ? 1u : 0u);
-        tc05::mma_commit(p_empty);
-        tc05::mma_commit(v_empty(vs));
-        return true;
-      };
-      for (int kt = 0; kt < n_ktiles; ++kt) {
-        const int ks = kt % kStages;
-        // S(kt) = Q K_hi^T + Q K_lo^T into S buffer kt % 2 once K(kt) has
-        // landed and the softmax has read S(kt - 2) from that buffer
-        const int sb = kt & 1;
-        if (!wait_bounded(k_full(ks), (kt / kStages) & 1, abort_flag) ||
-            (kt >= 2 && !wait_bounded(s_empty(sb), ((kt >> 1) - 1) & 1, abort_flag))) {
-          fail();
-          break;
-        }
-        tc05::fence_after_sync();
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const uint32_t qo = ((j >> 2) & 1) * (kQBytes / 2) + (j & 3) * 32;
-          const uint32_t ko = (j >> 3) * (kKBytes / 2) + ((j >> 2) & 1) * (kKBytes / 4) + (j & 3) * 32;
-          tc05::mma_f16_ss(tS(sb), tc05::smem_desc_sw128(sQ + qo), tc05::smem_desc_sw128(kbuf(ks) + ko), kIdescS,
-                           j > 0 ? 1u : 0u);
-        }
-        tc05::mma_commit(s_full(sb));
-        tc05::mma_commit(k_empty(ks));
-        // O += P(kt-1) V(kt-1) while the softmax of kt runs
-        if (kt >= 1 && !issue_pv(kt - 1)) {
-          fail();
-          break;
-        }
+      for (int j = 0; j < kKeyTile / 16; ++j)
+        mma_ts_elect(tO, tP + 8 * j, dv + (((j >> 2) * (kVBytes / 2) + (j & 3) * 32) >> 4), kIdescO,
+                     (k > 0 || j > 0) ? 1u : 0u);
+      commit_elect(p_empty);
+      commit_elect(v_empty(vs));
+      return true;
+    };
+    for (int kt = 0; kt < n_ktiles; ++kt) {
+      const int ks = kt % kStages;
+      // S(kt) = Q K_hi^T + Q K_lo^T into S buffer kt % 2 once K(kt) has
+      // landed and the softmax has read S(kt - 2) from that buffer
+      const int sb = kt & 1;
+      // both barriers tested back to back (their latencies overlap); the
+      // bounded waits only when one of them is not complete yet
+      const bool kf = mbar_try_wait(k_full(ks), (kt / kStages) & 1);
+      const bool se = kt < 2 || mbar_try_wait(s_empty(sb), ((kt >> 1) - 1) & 1);
+      if (!__all_sync(0xFFFFFFFFu, kf && se) &&
+          (!wait_w(k_full(ks), (kt / kStages) & 1) || (kt >= 2 && !wait_w(s_empty(sb), ((kt >> 1) - 1) & 1)))) {
+        fail();
+        break;
       }
-      if (!failed && !issue_pv(n_ktiles - 1)) fail();
+      tc05::fence_after_sync();
+      const uint64_t dk = ks ? dk1 : dk0;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const uint32_t qo = ((j >> 2) & 1) * (kQBytes / 2) + (j & 3) * 32;
+        const uint32_t ko = (j >> 3) * (kKBytes / 2) + ((j >> 2) & 1) * (kKBytes / 4) + (j & 3) * 32;
+        mma_ss_elect(tS(sb), dq + (qo >> 4), dk + (ko >> 4), kIdescS, j > 0 ? 1u : 0u);
+      }
+      commit_elect(s_full(sb));
+      commit_elect(k_empty(ks));
+      // O += P(kt-1) V(kt-1) while the softmax of kt runs
+      if (kt >= 1 && !issue_pv(kt - 1)) {
+        fail();
+        break;
+      }
     }
+    if (!failed && !issue_pv(n_ktiles - 1)) fail();
   } else {
     // ---------------------------------------------------- softmax (rows)
     const int row = tid;  // tensor-memory lane
@@ -592,7 +652,10 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(const PrefillPara
 #pragma unroll
       for (int j = 0; j < kKeyTile; j += 2) {
         const float2 x = fma2(make_float2(__uint_as_float(sv[j]), __uint_as_float(sv[j + 1])), sc, nr);
-        const float2 e = make_float2(fast_exp2(x.x), fast_exp2(x.y));
+        // the exponentials are split between the MUFU pipe and the FMA pipe
+        // (both are otherwise the softmax's bound): pairs m % 8 < kPolyOf8
+        // of the tile's 64 take the polynomial
+        const float2 e = ((j >> 1) % 8 < kPolyOf8) ? exp2_poly2(x) : make_float2(fast_exp2(x.x), fast_exp2(x.y));
         if (j & 2) ts1 = add2(ts1, e);
         else ts0 = add2(ts0, e);
         hp[j >> 1] = h2_as_u32(__floats2half2_rn(e.x, e.y));
