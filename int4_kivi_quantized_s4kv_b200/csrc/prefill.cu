@@ -76,7 +76,6 @@ constexpr int kPagesPerTile = kKeyTile / kPage;  // 8
 constexpr int kOpPages = kPagesPerTile / 2;       // operand kernel: half a key tile per CTA
 constexpr int kOpThreads = 64 * kOpPages;        // 64 threads per page
 constexpr int kStages = 2;                       // K and V buffers each
-constexpr uint32_t kQBytes = 128 * 128 * 2;      // Q [128][128] fp16
 constexpr uint32_t kKBytes = 2 * kKeyTile * 128 * 2;   // K_hi, K_lo [128][128] fp16 each
 constexpr uint32_t kVBytes = 128 * kKeyTile * 2;       // V^T [128][128] fp16
 constexpr uint32_t kTileBytes = kKBytes + kVBytes;     // workspace tile
@@ -92,14 +91,15 @@ constexpr long long kWaitLimit = 2000000000LL;   // about one second
 constexpr uint32_t kIdescS = tc05::idesc_f16_f32(128, kKeyTile);
 constexpr uint32_t kIdescO = tc05::idesc_f16_f32(128, 128);
 // tensor memory (512 columns): two S buffers at 0 and 128, O at 256, P (fp16
-// pairs, the PV A operand) at 384
+// pairs, the PV A operand) at 384, Q (fp16 pairs, the S A operand) at 448.
+// With both A operands in tensor memory, each MMA reads only its B operand
+// from shared memory.
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS = 0, kColO = 256, kColP = 384;
+constexpr uint32_t kColS = 0, kColO = 256, kColP = 384, kColQ = 448;
 
-// attention kernel smem (1024-aligned operands): Q, two K and two V buffers,
+// attention kernel smem (1024-aligned operands): two K and two V buffers,
 // barriers
-constexpr uint32_t kOffQ = 0;
-constexpr uint32_t kOffK = kOffQ + kQBytes;                      // [2]
+constexpr uint32_t kOffK = 0;                                    // [2]
 constexpr uint32_t kOffV = kOffK + kStages * kKBytes;            // [2]
 constexpr uint32_t kOffBar = kOffV + kStages * kVBytes;
 // barriers (8 bytes each): k_full[2], k_empty[2], v_full[2], v_empty[2],
@@ -138,14 +138,6 @@ __device__ __forceinline__ void wait_landed(uint32_t bar, uint32_t parity) {
 
 
 // One elected lane of the (converged) warp issues the MMA / the commit.
-__device__ __forceinline__ void mma_ss_elect(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                             uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p, e;\n\telect.sync _|e, 0xffffffff;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
 __device__ __forceinline__ void mma_ts_elect(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
                                              uint32_t accumulate) {
   asm volatile(
@@ -432,7 +424,6 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(const PrefillPara
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_addr(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
-  const uint32_t sQ = base + kOffQ;
   const uint32_t bars = base + kOffBar;
   const uint32_t tslot = base + kOffSlot;
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem_raw + (base + kOffAbort - raw));
@@ -489,22 +480,36 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(const PrefillPara
     *abort_flag = 0;
     fence_barrier_init();
   }
-  // Q tile: row r = (token r / G, head r % G); rows >= rows are zero
-  for (int ch = tid; ch < 128 * 16; ch += kThreadsP) {
-    const int r = ch >> 4, c = ch & 15;
-    const int tl = r / G, g = r - tl * G;
-    uint4 v = make_uint4(0, 0, 0, 0);
-    if (r < rows)
-      v = __ldg(reinterpret_cast<const uint4 *>(
-                    p.q + (static_cast<long>(c_lo + t0 + tl) * p.num_q_heads + h * G + g) * kHeadDim) + c);
-    sts128(sQ + tc05::sw128_offset(r, 8 * c, 128), v);
-  }
-  fence_proxy_async();
   __syncthreads();
   tc05::fence_after_sync();
   const uint32_t tmem = lds32_at(tslot);
   auto tS = [&](int s) { return tmem + kColS + 128u * s; };
-  const uint32_t tO = tmem + kColO, tP = tmem + kColP;
+  const uint32_t tO = tmem + kColO, tP = tmem + kColP, tQ = tmem + kColQ;
+  // Q tile into tensor memory: row r = (token r / G, head r % G), one row
+  // per softmax thread (its lane), channels 2c and 2c + 1 in column c; rows
+  // >= rows are zero
+  if (warp < kSoftmaxWarps) {
+    const int r = tid, tl = r / G, g = r - (r / G) * G;
+    const uint4 *src = reinterpret_cast<const uint4 *>(
+        p.q + (static_cast<long>(c_lo + t0 + tl) * p.num_q_heads + h * G + g) * kHeadDim);
+#pragma unroll
+    for (int hc = 0; hc < 2; ++hc) {
+      uint32_t v[32];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const uint4 x = r < rows ? __ldg(src + 8 * hc + c) : make_uint4(0, 0, 0, 0);
+        v[4 * c] = x.x;
+        v[4 * c + 1] = x.y;
+        v[4 * c + 2] = x.z;
+        v[4 * c + 3] = x.w;
+      }
+      tc05::tmem_st32(tQ + (static_cast<uint32_t>(32 * warp) << 16) + 32 * hc, v);
+    }
+    tc05::tmem_wait_st();
+    tc05::fence_before_sync();
+  }
+  __syncthreads();
+  tc05::fence_after_sync();
   bool failed = false;
   auto fail = [&]() {
     failed = true;
@@ -543,7 +548,6 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(const PrefillPara
     auto wait_w = [&](uint32_t bar, uint32_t parity) {
       return __all_sync(0xFFFFFFFFu, wait_bounded(bar, parity, abort_flag));
     };
-    const uint64_t dq = tc05::smem_desc_sw128(sQ);
     const uint64_t dk0 = tc05::smem_desc_sw128(kbuf(0)), dk1 = tc05::smem_desc_sw128(kbuf(1));
     const uint64_t dv0 = tc05::smem_desc_sw128(vbuf(0)), dv1 = tc05::smem_desc_sw128(vbuf(1));
     auto issue_pv = [&](int k) {  // O += P(k) V(k), P read from tensor memory
@@ -580,9 +584,10 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(const PrefillPara
       const uint64_t dk = ks ? dk1 : dk0;
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
-        const uint32_t qo = ((j >> 2) & 1) * (kQBytes / 2) + (j & 3) * 32;
+        // Q channels 16 (j % 8) .. + 15 (tensor-memory columns 8 (j % 8) ..)
+        // against the same channels of K_hi (j < 8), then of K_lo
         const uint32_t ko = (j >> 3) * (kKBytes / 2) + ((j >> 2) & 1) * (kKBytes / 4) + (j & 3) * 32;
-        mma_ss_elect(tS(sb), dq + (qo >> 4), dk + (ko >> 4), kIdescS, j > 0 ? 1u : 0u);
+        mma_ts_elect(tS(sb), tQ + 8 * (j & 7), dk + (ko >> 4), kIdescS, j > 0 ? 1u : 0u);
       }
       commit_elect(s_full(sb));
       commit_elect(k_empty(ks));
