@@ -38,21 +38,23 @@
 //        copies (TMA engine, no multicast); a K buffer is refilled as soon as
 //        the S MMAs that read it complete, a V buffer once the PV MMAs have,
 //        each by its own warp so that neither copy queues behind the other's
-//        buffer (the tiles come from L2 at a few tens of bytes per cycle per
-//        SM, so K must be issued two tiles ahead);
-//      * one thread issues S(k) = Q K_hi^T + Q K_lo^T (M = 128, N = 128 keys,
+//        buffer;
+//      * one warp issues S(k) = Q K_hi^T + Q K_lo^T (M = 128, N = 128 keys,
 //        one accumulation over K = 256: the 128 channels against K_hi, then
-//        against K_lo) into one of two tensor-memory S buffers, then
-//        O += P(k-1) V(k-1) (N = 128, K = 128) with P read from tensor
-//        memory.  Few, large MMA instructions keep the single issuing thread
-//        ahead of the tensor core, and with two S buffers S(k+1) never waits
-//        for the softmax to have read S(k);
+//        against K_lo; Q read from tensor memory) into one of two
+//        tensor-memory S buffers, another issues O += P(k) V(k) (N = 128,
+//        K = 128) with P read from tensor memory, so that S(k+1) never
+//        queues behind a PV that waits for its softmax; with two S buffers
+//        S(k+1) never waits for the softmax to have read S(k);
 //      * 4 softmax warps (one tensor-memory lane, i.e. one row, per thread)
 //        read S back, apply the causal mask and an online softmax
 //        in the exp2 domain whose reference moves only when a row maximum
 //        passes it by more than 8 (weights stay <= 256, fine for fp16),
 //        rescale that row of O in tensor memory when it moves, and write P
-//        (fp16 pairs) into tensor memory.
+//        (fp16 pairs) into tensor memory; three exponentials in eight are
+//        computed on the FMA pipe (exp2_poly2), the rest on the MUFU pipe.
+//     The Q tile sits in tensor memory too, so every MMA reads only its B
+//     operand (K or V) from shared memory.
 // Every wait is bounded; a timeout sets a CTA-wide abort flag and an error
 // bit, and every role then leaves its loop.
 #include <cfloat>
@@ -67,19 +69,23 @@ namespace s4kv {
 namespace {
 
 constexpr int kSoftmaxWarps = 4;   // warps 0..3: one row per thread
-constexpr int kMmaWarp = 4;
+constexpr int kMmaWarp = 4;        // S MMAs
 constexpr int kKProducerWarp = 5;  // K tiles
 constexpr int kVProducerWarp = 6;  // V tiles
-constexpr int kThreadsP = 32 * 7;
+constexpr int kPvWarp = 7;         // PV MMAs
+constexpr int kThreadsP = 32 * 8;
 constexpr int kKeyTile = 128;                    // keys per tile
 constexpr int kPagesPerTile = kKeyTile / kPage;  // 8
 constexpr int kOpPages = kPagesPerTile / 2;       // operand kernel: half a key tile per CTA
 constexpr int kOpThreads = 64 * kOpPages;        // 64 threads per page
 constexpr int kStages = 2;                       // K and V buffers each
-constexpr uint32_t kKBytes = 2 * kKeyTile * 128 * 2;   // K_hi, K_lo [128][128] fp16 each
+constexpr uint32_t kKHiBytes = kKeyTile * 128 * 2;     // K_hi [128][128] fp16
+constexpr uint32_t kKLoBytes = kKeyTile * 128;         // K_lo [128][128] e5m2
+constexpr uint32_t kKBytes = kKHiBytes + kKLoBytes;    // one K buffer
 constexpr uint32_t kVBytes = 128 * kKeyTile * 2;       // V^T [128][128] fp16
 constexpr uint32_t kTileBytes = kKBytes + kVBytes;     // workspace tile
 constexpr uint32_t kHalfTileBytes = kTileBytes / 2;
+constexpr uint32_t kQ8Bytes = 128 * 128;               // Q [128][128] e5m2
 constexpr float kSlack = 8.0f;                   // log2 slack of the softmax reference
 #ifndef S4KV_PREFILL_POLY_OF8
 #define S4KV_PREFILL_POLY_OF8 3
@@ -90,6 +96,7 @@ constexpr long long kWaitLimit = 2000000000LL;   // about one second
 // accumulated); PV: M = 128, N = 128
 constexpr uint32_t kIdescS = tc05::idesc_f16_f32(128, kKeyTile);
 constexpr uint32_t kIdescO = tc05::idesc_f16_f32(128, 128);
+constexpr uint32_t kIdescS8 = tc05::idesc_e5m2_f32(128, kKeyTile);  // Q8 . K_lo^T
 // tensor memory (512 columns): two S buffers at 0 and 128, O at 256, P (fp16
 // pairs, the PV A operand) at 384, Q (fp16 pairs, the S A operand) at 448.
 // With both A operands in tensor memory, each MMA reads only its B operand
@@ -101,7 +108,8 @@ constexpr uint32_t kColS = 0, kColO = 256, kColP = 384, kColQ = 448;
 // barriers
 constexpr uint32_t kOffK = 0;                                    // [2]
 constexpr uint32_t kOffV = kOffK + kStages * kKBytes;            // [2]
-constexpr uint32_t kOffBar = kOffV + kStages * kVBytes;
+constexpr uint32_t kOffQ8 = kOffV + kStages * kVBytes;
+constexpr uint32_t kOffBar = kOffQ8 + kQ8Bytes;
 // barriers (8 bytes each): k_full[2], k_empty[2], v_full[2], v_empty[2],
 // s_full[2], s_empty[2], p_full, p_empty; then the tensor-memory address and
 // the abort flag
@@ -110,7 +118,9 @@ constexpr uint32_t kOffSlot = kOffBar + 8 * kNumBars;
 constexpr uint32_t kOffAbort = kOffSlot + 4;
 constexpr uint32_t kSmemBytes = kOffAbort + 4 + 1024;  // + alignment slack
 static_assert(kSmemBytes <= 227 * 1024, "prefill shared memory");
-static_assert(kKBytes % 1024 == 0 && kVBytes % 1024 == 0 && kOffBar % 1024 == 0, "1024-byte operand alignment");
+static_assert(kKHiBytes % 1024 == 0 && kKBytes % 1024 == 0 && kVBytes % 1024 == 0 && kOffQ8 % 1024 == 0 &&
+                  kOffBar % 1024 == 0,
+              "1024-byte operand alignment");
 
 // operand kernel smem: the output half tile, then the staged page blocks
 template <int kBits>
@@ -144,6 +154,14 @@ __device__ __forceinline__ void mma_ts_elect(uint32_t d_tmem, uint32_t a_tmem, u
       "{\n\t.reg .pred p, e;\n\telect.sync _|e, 0xffffffff;\n\tsetp.ne.b32 p, %4, 0;\n\t"
       "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void mma_ss_e5m2_elect(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                                  uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\telect.sync _|e, 0xffffffff;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
 __device__ __forceinline__ void commit_elect(uint32_t bar) {
@@ -220,15 +238,37 @@ __device__ __forceinline__ uint32_t hfma2_u32(uint32_t a, uint32_t b, uint32_t c
   return h2_as_u32(__hfma2(u32_as_h2(a), u32_as_h2(b), u32_as_h2(c)));
 }
 
+// Two fp32 values rounded to e5m2 (round to nearest even, saturating), the
+// first in the low byte.
+__device__ __forceinline__ uint16_t e5m2x2(float first, float second) {
+  uint16_t d;
+  asm("cvt.rn.satfinite.e5m2x2.f32 %0, %1, %2;" : "=h"(d) : "f"(second), "f"(first));
+  return d;
+}
+// Two fp16 values (a pair in one word, the lower element in the low half)
+// rounded to e5m2, the lower element in the low byte.
+__device__ __forceinline__ uint16_t e5m2x2_of_f16x2(uint32_t x) {
+  uint16_t d;
+  asm("cvt.rn.satfinite.e5m2x2.f16x2 %0, %1;" : "=h"(d) : "r"(x));
+  return d;
+}
+
 // Two keys (fp16 codes in `codes`) dequantized in fp32 (code * scale + zero:
-// the product is exact, so one rounding) and split into fp16 hi and lo parts.
-__device__ __forceinline__ void split_key(uint32_t codes, float2 sc, float2 z, uint32_t &hi, uint32_t &lo) {
+// the product is exact, so one rounding) and split into an fp16 hi part and
+// the e5m2 rounding of the remainder (lo, the lower key in the low byte).
+__device__ __forceinline__ void split_key(uint32_t codes, float2 sc, float2 z, uint32_t &hi, uint16_t &lo) {
   const float2 c = __half22float2(u32_as_h2(codes));
   const float2 k = fma2(c, sc, z);
   const __half2 h = __floats2half2_rn(k.x, k.y);
   const float2 r = sub2(k, __half22float2(h));
   hi = h2_as_u32(h);
-  lo = h2_as_u32(__floats2half2_rn(r.x, r.y));
+  lo = e5m2x2(r.x, r.y);
+}
+
+// Byte offset of element (r, k) of a [rows][128] 8-bit K-major operand in the
+// 128-byte-swizzled layout (one 128-byte row per r).
+__device__ __forceinline__ uint32_t sw128_offset_b8(int r, int k) {
+  return static_cast<uint32_t>((r >> 3) * 1024 + (r & 7) * 128 + ((((k >> 4) ^ (r & 7))) << 4) + (k & 15));
 }
 
 // The rows of sequence b that the chunk holds, checked against the cache.
@@ -266,9 +306,9 @@ __global__ void __launch_bounds__(kOpThreads) prefill_operands_kernel(const Pref
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_addr(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
-  // half tile in smem: K_hi [64][128] (two 8 KB column blocks), K_lo the same,
-  // then V^T [128][64]
-  const uint32_t sK = base, sV = base + kKBytes / 2;
+  // half tile in smem: K_hi [64][128] (two 8 KB column blocks), K_lo
+  // [64][128] e5m2 (8 KB), then V^T [128][64]
+  const uint32_t sK = base, sKlo = base + kKHiBytes / 2, sV = base + kKBytes / 2;
   const uint32_t stage = base + kHalfTileBytes;
   const int ht = blockIdx.x, b = blockIdx.y, h = blockIdx.z, H = p.num_kv_heads;
   const int kt = ht >> 1, hh = ht & 1;
@@ -319,14 +359,14 @@ __global__ void __launch_bounds__(kOpThreads) prefill_operands_kernel(const Pref
       int w0, n0, w1, n1;
       key_position(t, c0, w0, n0);
       key_position(t, c0 + 1, w1, n1);
-      uint32_t hi, lo;
+      uint32_t hi;
+      uint16_t lo;
       const uint32_t codes = h2_as_u32(__floats2half2_rn(static_cast<float>(code_at(blk + F::kKCode, w0, n0, kBits)),
                                                          static_cast<float>(code_at(blk + F::kKCode, w1, n1, kBits))));
       split_key(codes, make_float2(ks0, ks1), make_float2(kz0, kz1), hi, lo);
       const int key = dpage * 16 + t;  // within the half tile
-      const uint32_t ko = tc05::sw128_offset(key, c0, kKeyTile / 2);
-      sts32(sK + ko, hi);
-      sts32(sK + kKBytes / 4 + ko, lo);
+      sts32(sK + tc05::sw128_offset(key, c0, kKeyTile / 2), hi);
+      sts16(sKlo + sw128_offset_b8(key, c0), lo);
       const __half vs = vscale[value_scale_slot(t, g)], vz = vzero[g * kPage + t];
 #pragma unroll
       for (int j = 0; j < 2; ++j) {
@@ -354,7 +394,8 @@ __global__ void __launch_bounds__(kOpThreads) prefill_operands_kernel(const Pref
         const uint32_t z23 = lds32_at(blk + kKZeroOff + 2 * (zslot + 8));
         const float2 s01 = __half22float2(u32_as_h2(sc.x)), s23 = __half22float2(u32_as_h2(sc.y));
         const float2 zf01 = __half22float2(u32_as_h2(z01)), zf23 = __half22float2(u32_as_h2(z23));
-        uint32_t hi0, lo0, hi1, lo1, hi2, lo2, hi3, lo3;
+        uint32_t hi0, hi1, hi2, hi3;
+        uint16_t lo0, lo1, lo2, lo3;
         split_key(a0, s01, zf01, hi0, lo0);
         split_key(a1, s01, zf01, hi1, lo1);
         split_key(a2, s23, zf23, hi2, lo2);
@@ -362,8 +403,10 @@ __global__ void __launch_bounds__(kOpThreads) prefill_operands_kernel(const Pref
         const uint32_t ko = tc05::sw128_offset(dpage * 16 + dn, c0, kKeyTile / 2);
         sts64(sK + ko, hi0, hi2);
         sts64(sK + ko + 1024, hi1, hi3);
-        sts64(sK + kKBytes / 4 + ko, lo0, lo2);
-        sts64(sK + kKBytes / 4 + ko + 1024, lo1, lo3);
+        // tokens dn and dn + 8 are 8 rows (1024 bytes) apart in both layouts
+        const uint32_t ko8 = sw128_offset_b8(dpage * 16 + dn, c0);
+        sts32(sKlo + ko8, static_cast<uint32_t>(lo0) | (static_cast<uint32_t>(lo2) << 16));
+        sts32(sKlo + ko8 + 1024, static_cast<uint32_t>(lo1) | (static_cast<uint32_t>(lo3) << 16));
       }
       // values: channels cb, cb + 1; tokens 2 di, 2 di + 1 (+ 8)
       {
@@ -393,9 +436,9 @@ __global__ void __launch_bounds__(kOpThreads) prefill_operands_kernel(const Pref
       const int tk = e >> 6, c = 2 * (e & 63);
       uint32_t kb = 0;
       if (tk < rres) kb = *reinterpret_cast<const uint32_t *>(rk + tk * kHeadDim + c);
-      const uint32_t ko = tc05::sw128_offset(dpage * 16 + tk, c, kKeyTile / 2);
-      sts32(sK + ko, kb);
-      sts32(sK + kKBytes / 4 + ko, 0u);
+      // residual keys are fp16 already: K_lo is zero
+      sts32(sK + tc05::sw128_offset(dpage * 16 + tk, c, kKeyTile / 2), kb);
+      sts16(sKlo + sw128_offset_b8(dpage * 16 + tk, c), 0);
     }
     for (int e = widx; e < kPage * kHeadDim; e += 64) {
       const int tk = e >> 7, c = e & 127;
@@ -407,13 +450,15 @@ __global__ void __launch_bounds__(kOpThreads) prefill_operands_kernel(const Pref
   __syncthreads();
 
   // ---- the half tile to its places in the workspace tile, coalesced 16-byte
-  // stores: smem 8 KB pieces 0..3 (K_hi, K_lo column blocks) go to
-  // 16 KB * piece + 8 KB * hh, the 16 KB of V^T to K bytes + 16 KB * hh
+  // stores: smem 8 KB pieces 0, 1 (K_hi column blocks) go to
+  // 16 KB * piece + 8 KB * hh, the 8 KB of K_lo to K_hi bytes + 8 KB * hh,
+  // the 16 KB of V^T to K bytes + 16 KB * hh
   uint8_t *tile = p.ws + ((static_cast<long long>(b) * H + h) * p.tiles_per_seq + kt) * kTileBytes;
   for (int i = t; i < static_cast<int>(kHalfTileBytes / 16); i += kOpThreads) {
     const uint32_t off = 16u * i;
-    const uint32_t dst = off < kKBytes / 2 ? (off >> 13) * 16384u + 8192u * hh + (off & 8191u)
-                                           : kKBytes + 16384u * hh + (off - kKBytes / 2);
+    const uint32_t dst = off < kKHiBytes / 2 ? (off >> 13) * 16384u + 8192u * hh + (off & 8191u)
+                         : off < kKBytes / 2 ? kKHiBytes + 8192u * hh + (off - kKHiBytes / 2)
+                                             : kKBytes + 16384u * hh + (off - kKBytes / 2);
     *reinterpret_cast<uint4 *>(tile + dst) = lds128_at(base + off);
   }
 }
@@ -504,9 +549,21 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(const PrefillPara
         v[4 * c + 3] = x.w;
       }
       tc05::tmem_st32(tQ + (static_cast<uint32_t>(32 * warp) << 16) + 32 * hc, v);
+      // the same channels in e5m2 into the Q8 tile (shared memory, the A
+      // operand of Q8 . K_lo^T): 16-byte chunks 4 hc .. 4 hc + 3 of row r
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t w[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          w[i] = static_cast<uint32_t>(e5m2x2_of_f16x2(v[8 * cc + 2 * i])) |
+                 (static_cast<uint32_t>(e5m2x2_of_f16x2(v[8 * cc + 2 * i + 1])) << 16);
+        sts128(base + kOffQ8 + sw128_offset_b8(r, 16 * (4 * hc + cc)), make_uint4(w[0], w[1], w[2], w[3]));
+      }
     }
     tc05::tmem_wait_st();
     tc05::fence_before_sync();
+    fence_proxy_async();  // the Q8 tile is read by the MMAs (async proxy)
   }
   __syncthreads();
   tc05::fence_after_sync();
@@ -541,63 +598,72 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(const PrefillPara
       // by time only, also after an abort): at most the last kStages
       for (int kt = max(0, issued - kStages); kt < issued; ++kt) wait_landed(full(kt % kStages), (kt / kStages) & 1);
     }
-  } else if (warp == kMmaWarp) {
-    // ------------------------------------------------------- MMA issuer
-    // The whole warp runs the loop, so that descriptors and decisions stay
-    // warp-uniform; one elected lane issues each MMA and commit.
+  } else if (warp == kMmaWarp || warp == kPvWarp) {
+    // -------------------------------------------------------- MMA issuers
+    // Two warps issue: S(kt) goes out as soon as K(kt) has landed and the
+    // softmax has read S(kt - 2) from its buffer, without waiting behind
+    // O += P V of an earlier tile, whose issue waits for that tile's softmax.
+    // Each warp runs its loop on all lanes (descriptors and decisions stay
+    // warp-uniform); one elected lane issues each MMA and commit, and a
+    // commit tracks the MMAs of its own thread only.
     auto wait_w = [&](uint32_t bar, uint32_t parity) {
       return __all_sync(0xFFFFFFFFu, wait_bounded(bar, parity, abort_flag));
     };
-    const uint64_t dk0 = tc05::smem_desc_sw128(kbuf(0)), dk1 = tc05::smem_desc_sw128(kbuf(1));
-    const uint64_t dv0 = tc05::smem_desc_sw128(vbuf(0)), dv1 = tc05::smem_desc_sw128(vbuf(1));
-    auto issue_pv = [&](int k) {  // O += P(k) V(k), P read from tensor memory
-      const int vs = k % kStages;
-      const bool vf = mbar_try_wait(v_full(vs), (k / kStages) & 1);
-      const bool pf = mbar_try_wait(p_full, k & 1);
-      if (!__all_sync(0xFFFFFFFFu, vf && pf) && (!wait_w(v_full(vs), (k / kStages) & 1) || !wait_w(p_full, k & 1)))
-        return false;
-      tc05::fence_after_sync();
-      const uint64_t dv = vs ? dv1 : dv0;
+    if (warp == kPvWarp) {
+      const uint64_t dv0 = tc05::smem_desc_sw128(vbuf(0)), dv1 = tc05::smem_desc_sw128(vbuf(1));
+      for (int k = 0; k < n_ktiles; ++k) {
+        // O += P(k) V(k), P read from tensor memory, once V(k) has landed and
+        // the softmax has written P(k)
+        const int vs = k % kStages;
+        const bool vf = mbar_try_wait(v_full(vs), (k / kStages) & 1);
+        const bool pf = mbar_try_wait(p_full, k & 1);
+        if (!__all_sync(0xFFFFFFFFu, vf && pf) &&
+            (!wait_w(v_full(vs), (k / kStages) & 1) || !wait_w(p_full, k & 1))) {
+          fail();
+          break;
+        }
+        tc05::fence_after_sync();
+        const uint64_t dv = vs ? dv1 : dv0;
 #pragma unroll
-      for (int j = 0; j < kKeyTile / 16; ++j)
-        mma_ts_elect(tO, tP + 8 * j, dv + (((j >> 2) * (kVBytes / 2) + (j & 3) * 32) >> 4), kIdescO,
-                     (k > 0 || j > 0) ? 1u : 0u);
-      commit_elect(p_empty);
-      commit_elect(v_empty(vs));
-      return true;
-    };
-    for (int kt = 0; kt < n_ktiles; ++kt) {
-      const int ks = kt % kStages;
-      // S(kt) = Q K_hi^T + Q K_lo^T into S buffer kt % 2 once K(kt) has
-      // landed and the softmax has read S(kt - 2) from that buffer
-      const int sb = kt & 1;
-      // both barriers tested back to back (their latencies overlap); the
-      // bounded waits only when one of them is not complete yet
-      const bool kf = mbar_try_wait(k_full(ks), (kt / kStages) & 1);
-      const bool se = kt < 2 || mbar_try_wait(s_empty(sb), ((kt >> 1) - 1) & 1);
-      if (!__all_sync(0xFFFFFFFFu, kf && se) &&
-          (!wait_w(k_full(ks), (kt / kStages) & 1) || (kt >= 2 && !wait_w(s_empty(sb), ((kt >> 1) - 1) & 1)))) {
-        fail();
-        break;
+        for (int j = 0; j < kKeyTile / 16; ++j)
+          mma_ts_elect(tO, tP + 8 * j, dv + (((j >> 2) * (kVBytes / 2) + (j & 3) * 32) >> 4), kIdescO,
+                       (k > 0 || j > 0) ? 1u : 0u);
+        commit_elect(p_empty);
+        commit_elect(v_empty(vs));
       }
-      tc05::fence_after_sync();
-      const uint64_t dk = ks ? dk1 : dk0;
+    } else {
+      const uint64_t dk0 = tc05::smem_desc_sw128(kbuf(0)), dk1 = tc05::smem_desc_sw128(kbuf(1));
+      const uint64_t dq8 = tc05::smem_desc_sw128(base + kOffQ8);
+      for (int kt = 0; kt < n_ktiles; ++kt) {
+        const int ks = kt % kStages;
+        // S(kt) = Q K_hi^T + Q K_lo^T into S buffer kt % 2 once K(kt) has
+        // landed and the softmax has read S(kt - 2) from that buffer
+        const int sb = kt & 1;
+        // both barriers tested back to back (their latencies overlap); the
+        // bounded waits only when one of them is not complete yet
+        const bool kf = mbar_try_wait(k_full(ks), (kt / kStages) & 1);
+        const bool se = kt < 2 || mbar_try_wait(s_empty(sb), ((kt >> 1) - 1) & 1);
+        if (!__all_sync(0xFFFFFFFFu, kf && se) &&
+            (!wait_w(k_full(ks), (kt / kStages) & 1) || (kt >= 2 && !wait_w(s_empty(sb), ((kt >> 1) - 1) & 1)))) {
+          fail();
+          break;
+        }
+        tc05::fence_after_sync();
+        const uint64_t dk = ks ? dk1 : dk0;
+        // Q channels 16 j .. + 15 (tensor-memory columns 8 j ..) against the
+        // same channels of K_hi (fp16, K = 16 per MMA) ...
 #pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        // Q channels 16 (j % 8) .. + 15 (tensor-memory columns 8 (j % 8) ..)
-        // against the same channels of K_hi (j < 8), then of K_lo
-        const uint32_t ko = (j >> 3) * (kKBytes / 2) + ((j >> 2) & 1) * (kKBytes / 4) + (j & 3) * 32;
-        mma_ts_elect(tS(sb), tQ + 8 * (j & 7), dk + (ko >> 4), kIdescS, j > 0 ? 1u : 0u);
-      }
-      commit_elect(s_full(sb));
-      commit_elect(k_empty(ks));
-      // O += P(kt-1) V(kt-1) while the softmax of kt runs
-      if (kt >= 1 && !issue_pv(kt - 1)) {
-        fail();
-        break;
+        for (int j = 0; j < 8; ++j)
+          mma_ts_elect(tS(sb), tQ + 8 * j, dk + ((((j >> 2) * (kKHiBytes / 2)) + (j & 3) * 32) >> 4), kIdescS,
+                       j > 0 ? 1u : 0u);
+        // ... then Q8 channels 32 j .. + 31 against K_lo (e5m2, K = 32)
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          mma_ss_e5m2_elect(tS(sb), dq8 + ((32 * j) >> 4), dk + ((kKHiBytes + 32 * j) >> 4), kIdescS8, 1u);
+        commit_elect(s_full(sb));
+        commit_elect(k_empty(ks));
       }
     }
-    if (!failed && !issue_pv(n_ktiles - 1)) fail();
   } else {
     // ---------------------------------------------------- softmax (rows)
     const int row = tid;  // tensor-memory lane
@@ -612,9 +678,14 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(const PrefillPara
     auto wait_warp = [&](uint32_t bar, uint32_t parity) {
       return __all_sync(0xFFFFFFFFu, wait_bounded(bar, parity, abort_flag));
     };
+    // barrier tests whose answer is needed only later are made while a
+    // tensor-memory load or store is in flight (an S(kt + 1) test after P(kt)
+    // goes out, a P-buffer test after S(kt) is requested), so that a
+    // complete barrier costs no wait of its own
+    bool s_ready = false;
     for (int kt = 0; kt < n_ktiles; ++kt) {
       const int sb = kt & 1;
-      if (!wait_warp(s_full(sb), (kt >> 1) & 1)) {
+      if (!__all_sync(0xFFFFFFFFu, s_ready) && !wait_warp(s_full(sb), (kt >> 1) & 1)) {
         fail();
         break;
       }
@@ -625,6 +696,7 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(const PrefillPara
         uint32_t (&w)[32] = *reinterpret_cast<uint32_t (*)[32]>(&sv[32 * c]);
         tc05::tmem_ld32(tS(sb) + lane_base + 32 * c, w);
       }
+      const bool p_ready = kt == 0 || mbar_try_wait(p_empty, (kt - 1) & 1);
       tc05::tmem_wait_ld();
       tc05::fence_before_sync();
       mbar_arrive(s_empty(sb));
@@ -668,7 +740,7 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(const PrefillPara
       lsum = add2(mul2(lsum, make_float2(alpha, alpha)), add2(ts0, ts1));
       // O and P are idle once O += P(kt-1) V has completed
       if (kt >= 1) {
-        if (!wait_warp(p_empty, (kt - 1) & 1)) {
+        if (!__all_sync(0xFFFFFFFFu, p_ready) && !wait_warp(p_empty, (kt - 1) & 1)) {
           fail();
           break;
         }
@@ -699,6 +771,7 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(const PrefillPara
         tc05::tmem_st32(tP + lane_base, h0);
         tc05::tmem_st32(tP + lane_base + 32, h1);
       }
+      s_ready = kt + 1 < n_ktiles && mbar_try_wait(s_full(sb ^ 1), ((kt + 1) >> 1) & 1);
       tc05::tmem_wait_st();
       tc05::fence_before_sync();
       mbar_arrive(p_full);

@@ -40,6 +40,13 @@ __host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N) {
   return (1u << 4) | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
 }
 
+// Instruction descriptor of a kind::f8f6f4 MMA with e5m2 A and B (the same
+// type on both sides), fp32 accumulator, both operands K-major, shape M x N.
+__host__ __device__ constexpr uint32_t idesc_e5m2_f32(int M, int N) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
+         (static_cast<uint32_t>(M >> 4) << 24);
+}
+
 // Tensor-memory allocation (one whole warp executes these).  The allocated
 // base address is written to shared memory at `slot`.
 __device__ __forceinline__ void tmem_alloc(uint32_t slot, uint32_t ncols) {
