@@ -299,13 +299,13 @@ S4KV_API int s4kv_decode_attention_noalloc(const s4kv_cache_t *cache, const void
  *          launched).  Its contents are overwritten and mean nothing after the
  *          call; it must not be shared with work that runs concurrently.
  * Two launches on `stream`: the first dequantizes every 128-key tile of each
- * (sequence, kv head) once into the workspace as fp16 MMA operands (keys as
- * an fp16 hi part plus the fp16 rounding of the remainder, about 22 bits;
- * values correctly rounded to fp16); the second runs the attention on the
- * tcgen05 tensor cores with those operands and the fp16 softmax weights
- * (fp32 accumulation), so results agree with exact attention to about fp16
- * precision of the values and the weights.  Allocates nothing; the attention
- * launch needs about 225 KB of shared memory per CTA.  Any code width of
+ * (sequence, kv head) once into the workspace as MMA operands (keys as an
+ * fp16 hi part plus the e5m2 rounding of the remainder, which carries them
+ * to about 2^-14 relative; values correctly rounded to fp16); the second runs
+ * the attention on the tcgen05 tensor cores with those operands and the fp16
+ * softmax weights (fp32 accumulation), so results agree with exact attention
+ * to about fp16 precision of the values and the weights.  Allocates nothing;
+ * the attention launch needs about 178 KB of shared memory per CTA.  Any code width of
  * the cache (4, 8 or 2 bits): only the first launch reads the codes. */
 S4KV_API int s4kv_prefill_attention(const s4kv_cache_t *cache, const void *q,
                                     int num_q_heads, int n_tokens,
@@ -315,7 +315,7 @@ S4KV_API int s4kv_prefill_attention(const s4kv_cache_t *cache, const void *q,
                                     float sm_scale, void *out, void *workspace,
                                     size_t workspace_bytes, void *stream);
 
-/* Bytes of workspace s4kv_prefill_attention needs: 96 KB per 128-key tile
+/* Bytes of workspace s4kv_prefill_attention needs: 80 KB per 128-key tile
  * of max_pages_per_seq pages (rounded up to whole tiles of 8 pages), per
  * sequence slot and kv head.  S4KV_ERR_INVALID_ARG for non-positive sizes or a total above
  * 2^40 bytes. */

@@ -15,14 +15,15 @@
 // How (B200): this is a dense contraction, so it runs on the fifth-generation
 // tensor cores, in two launches.
 //  1. prefill_operands_kernel dequantizes every key tile (128 keys, 8 pages)
-//     of every (sequence, kv head) ONCE into a workspace tile of 96 KB that
+//     of every (sequence, kv head) ONCE into a workspace tile of 80 KB that
 //     holds the MMA operands exactly as shared memory wants them (128-byte
 //     swizzled, K-major): K_hi, K_lo and V^T.  A key is code * scale + zero
 //     in fp32 (exact product, one rounding, the value the oracle's
-//     dequantization gives) split into an fp16 hi part and the fp16 rounding
-//     of the remainder, so K_hi + K_lo carries it to about 22 bits (keys of
-//     outlier channels are large, and a single fp16 rounding of them moves
-//     the logits visibly).  A value is the fused fp16 multiply-add
+//     dequantization gives) split into an fp16 hi part and the e5m2 rounding
+//     of the remainder (at most 2^-12 of the key, so its 2^-3 relative error
+//     leaves the key carried to about 2^-14 relative; keys of outlier
+//     channels are large, and a single fp16 rounding of them moves the logits
+//     visibly).  A value is the fused fp16 multiply-add
 //     code * scale + zero (the correctly rounded fp16), stored transposed.
 //     Every query tile of the sequence then reads these bytes (mostly from
 //     L2) instead of dequantizing the same pages again.  One CTA writes half
@@ -33,16 +34,17 @@
 //     tile's 128 MMA rows are (token, head of the group) pairs, so a tile
 //     holds floor(128 / G) tokens.  Warps with separate roles hand buffers
 //     over through mbarriers:
-//      * two producer warps bring each key tile's K_hi, K_lo (64 KB) and V^T
+//      * two producer warps bring each key tile's K_hi, K_lo (48 KB) and V^T
 //        (32 KB) into one of two K and one of two V buffers with 1-D bulk
 //        copies (TMA engine, no multicast); a K buffer is refilled as soon as
 //        the S MMAs that read it complete, a V buffer once the PV MMAs have,
 //        each by its own warp so that neither copy queues behind the other's
 //        buffer;
-//      * one warp issues S(k) = Q K_hi^T + Q K_lo^T (M = 128, N = 128 keys,
-//        one accumulation over K = 256: the 128 channels against K_hi, then
-//        against K_lo; Q read from tensor memory) into one of two
-//        tensor-memory S buffers, another issues O += P(k) V(k) (N = 128,
+//      * one warp issues S(k) = Q K_hi^T + Q8 K_lo^T (M = 128, N = 128 keys,
+//        one accumulation: the 128 channels of Q, read from tensor memory,
+//        against K_hi with fp16 MMAs, then those of Q8, an e5m2 copy of Q in
+//        shared memory, against K_lo with e5m2 MMAs at twice the rate) into
+//        one of two tensor-memory S buffers, another issues O += P(k) V(k) (N = 128,
 //        K = 128) with P read from tensor memory, so that S(k+1) never
 //        queues behind a PV that waits for its softmax; with two S buffers
 //        S(k+1) never waits for the softmax to have read S(k);
@@ -92,8 +94,8 @@ constexpr float kSlack = 8.0f;                   // log2 slack of the softmax re
 #endif
 constexpr int kPolyOf8 = S4KV_PREFILL_POLY_OF8;  // eighths of the exponentials on the FMA pipe
 constexpr long long kWaitLimit = 2000000000LL;   // about one second
-// S: M = 128, N = 128 keys, K = 256 (Q against K_hi, then Q against K_lo,
-// accumulated); PV: M = 128, N = 128
+// S: M = 128, N = 128 keys (Q against K_hi, fp16 K = 16 per MMA, then Q8
+// against K_lo, e5m2 K = 32 per MMA, accumulated); PV: M = 128, N = 128
 constexpr uint32_t kIdescS = tc05::idesc_f16_f32(128, kKeyTile);
 constexpr uint32_t kIdescO = tc05::idesc_f16_f32(128, 128);
 constexpr uint32_t kIdescS8 = tc05::idesc_e5m2_f32(128, kKeyTile);  // Q8 . K_lo^T
@@ -294,11 +296,11 @@ __device__ __forceinline__ bool seq_rows(const PrefillParams &p, int b, bool fla
 
 // ---------------------------------------------------------------------------
 // Launch 1: one CTA per (half key tile, sequence, kv head) writes that half
-// of the tile's operands to the workspace: K_hi, K_lo and V^T, each
-// [128][128] fp16 and 128-byte swizzled K-major.  Half hh holds keys
-// 64 hh .. 64 hh + 63: rows 64 hh .. of both column blocks of K_hi and K_lo
-// (8 KB each, the same bytes a 64-row operand has) and column block hh of V^T
-// (16 KB).  Keys at or past L (the rest of the partial last page, pages
+// of the tile's operands to the workspace: K_hi and V^T [128][128] fp16,
+// K_lo [128][128] e5m2, each 128-byte swizzled K-major.  Half hh holds keys
+// 64 hh .. 64 hh + 63: rows 64 hh .. of both column blocks of K_hi (8 KB
+// each, the same bytes a 64-row operand has), rows 64 hh .. of K_lo (8 KB)
+// and column block hh of V^T (16 KB).  Keys at or past L (the rest of the partial last page, pages
 // after it) are written as zeros, so masked keys hold finite values.
 template <int kBits>
 __global__ void __launch_bounds__(kOpThreads) prefill_operands_kernel(const PrefillParams p) {

@@ -119,8 +119,8 @@ def test_invalid_calls_rejected_before_launch(S):
     assert call(args(maxnew=5)) == S.ERR_INVALID_ARG  # more than n_tokens
     assert call(args(batch=5)) == S.ERR_INVALID_ARG   # batch > max_seqs
     assert call(args(n=0)) == S.OK and call(args(batch=0)) == S.OK  # nothing to do
-    # workspace: 96 KB per 128-key tile (8 pages) per (sequence slot, kv head)
-    tile = 2 * 2 * 128 * 128 + 2 * 128 * 128  # [K_hi; K_lo] and V^T, fp16
+    # workspace: 80 KB per 128-key tile (8 pages) per (sequence slot, kv head)
+    tile = 2 * 128 * 128 + 128 * 128 + 2 * 128 * 128  # K_hi fp16, K_lo e5m2, V^T fp16
     assert S.prefill_workspace_bytes(2, 1, 1) == 2 * tile
     assert S.prefill_workspace_bytes(8, 4, 512) == 4 * 8 * 64 * tile
     assert S.prefill_workspace_bytes(1, 1, 9) == 2 * tile  # 9 pages round up to 2 tiles
