@@ -445,7 +445,8 @@ def measure_prefill(device, steps: int, workload: str = "llama3.1-8b-prefill", b
     achieved = flops / (ms * 1e-3) / 1e12
     # a call is two launches: the operand tiles (each page dequantized once)
     # and the attention, whose MMAs per (query tile, key tile) are
-    # Q [K_hi; K_lo]^T (keys carried to ~22 bits) and P V: 1.5x the
+    # Q K_hi^T + Q8 K_lo^T (keys carried to about 2^-14 relative; the K_lo
+    # part on the e5m2 MMA at twice the fp16 rate) and P V: 1.5x the
     # algorithmic FLOPs
     return {"workload": spec.name, "model_shape": spec.description, "code_bits": bits, "calls": steps,
             "launches": 2 * steps,
