@@ -1,26 +1,21 @@
 // Host side of the s4kv C ABI: argument validation, workspace sizing and
 // kernel launches.  Every host-visible argument is checked before anything
-// is launched; the library allocates no memory and keeps no per-cache state
-// (only a per-device record of the decode kernel's launch shape).
+// is launched; the library allocates no memory and keeps no state: launch
+// shapes are worked out and kernel attributes set at every call.
 #include <cuda_runtime.h>
 
 #include <cmath>
 #include <cstdint>
-#include <mutex>
 
 #include "kernels.cuh"
 #include "prefill.cuh"
-
-
 
 using namespace s4kv;
 
 namespace {
 
-constexpr int kMaxDevices = 64;
 
 struct DeviceShape {
-  bool ready = false;
   int num_sms = 0;
   int num_ctas[3] = {0, 0, 0};     // decode grid for 4-bit / 8-bit / 2-bit pages
   int num_workers[3] = {0, 0, 0};  // worker warps of that grid
@@ -35,38 +30,21 @@ size_t block_bytes(int bits) {
 }
 size_t record_bytes(const s4kv_cache_t *c) { return static_cast<size_t>(c->num_kv_heads) * block_bytes(cache_bits(c)); }
 
-std::mutex g_mu;
-DeviceShape g_shape[kMaxDevices];
-
-// Decode launch shape of the current device: one persistent CTA per
-// resident slot on every SM.
+// Decode launch shape of the current device, worked out at every call (the
+// library keeps no state): one persistent CTA per SM.
 int device_shape(DeviceShape *out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0) {
     cudaGetLastError();
     return S4KV_ERR_CUDA;
   }
-  std::lock_guard<std::mutex> lock(g_mu);
-  DeviceShape &d = g_shape[dev];
-  if (!d.ready) {
-    int sms = 0;
-    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
-      cudaGetLastError();
-      return S4KV_ERR_CUDA;
-    }
-    if (prepare_decode_kernel() != cudaSuccess) {
-      cudaGetLastError();
-      return S4KV_ERR_CUDA;
-    }
-    d.num_sms = sms;
-    for (int f = 0; f < 3; ++f) {
-      const int per = decode_ctas_per_sm(fmt_bits(f));
-      if (per <= 0 || sms <= 0) return S4KV_ERR_CUDA;
-      d.num_ctas[f] = sms * per;
-      d.num_workers[f] = d.num_ctas[f] * decode_warps_per_cta(fmt_bits(f));
-      d.max_workers = d.num_workers[f] > d.max_workers ? d.num_workers[f] : d.max_workers;
-    }
-    d.ready = true;
+  DeviceShape d;
+  d.num_sms = sms;
+  for (int f = 0; f < 3; ++f) {
+    d.num_ctas[f] = sms;
+    d.num_workers[f] = sms * decode_warps_per_cta(fmt_bits(f));
+    d.max_workers = d.num_workers[f] > d.max_workers ? d.num_workers[f] : d.max_workers;
   }
   *out = d;
   return S4KV_OK;
@@ -330,18 +308,6 @@ int s4kv_prefill_attention(const s4kv_cache_t *cache, const void *q, int num_q_h
   const int group = num_q_heads / cache->num_kv_heads;
   const long long tiles = (static_cast<long long>(max_new_per_seq) + (128 / group) - 1) / (128 / group);
   if (tiles > 0x7FFFFFFF || batch > 65535 || cache->num_kv_heads > 65535) return S4KV_ERR_INVALID_ARG;
-  static std::once_flag prepared[kMaxDevices];
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
-    cudaGetLastError();
-    return S4KV_ERR_CUDA;
-  }
-  cudaError_t perr = cudaSuccess;
-  std::call_once(prepared[dev], [&]() { perr = prepare_prefill_kernel(); });
-  if (perr != cudaSuccess) {
-    cudaGetLastError();
-    return S4KV_ERR_CUDA;
-  }
   PrefillParams p;
   p.pool = static_cast<const uint8_t *>(cache->pool);
   p.res_k = static_cast<const __half *>(cache->res_k);
@@ -362,8 +328,10 @@ int s4kv_prefill_attention(const s4kv_cache_t *cache, const void *q, int num_q_h
   p.ws = static_cast<uint8_t *>(workspace);
   p.tiles_per_seq = prefill_tiles_per_seq(max_pages_per_seq);
   p.bits = cache_bits(cache);
-  launch_prefill(p, batch, max_new_per_seq, static_cast<cudaStream_t>(stream));
-  if (cudaGetLastError() != cudaSuccess) return S4KV_ERR_CUDA;
+  if (launch_prefill(p, batch, max_new_per_seq, static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+    cudaGetLastError();
+    return S4KV_ERR_CUDA;
+  }
   return S4KV_OK;
 }
 

@@ -1032,16 +1032,11 @@ __global__ void __launch_bounds__(threads_for<kBits>(), min_ctas_for<kBits>())
   }  // active
 }
 
-template <int kBits>
-int ctas_per_sm_for() {
-  int n = 0;
-  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_kernel<kBits>, threads_for<kBits>(), smem_bytes_for<kBits>());
-  return n;
-}
-
-int decode_ctas_per_sm(int bits) {
-  return bits == 8 ? ctas_per_sm_for<8>() : bits == 2 ? ctas_per_sm_for<2>() : ctas_per_sm_for<4>();
-}
+// One CTA per SM by design for every code width: its ring takes more than
+// half of an SM's shared memory, so no second CTA fits.
+static_assert(2 * smem_bytes_for<4>() > 228 * 1024 && 2 * smem_bytes_for<8>() > 228 * 1024 &&
+                  2 * smem_bytes_for<2>() > 228 * 1024,
+              "one decode CTA per SM");
 
 int decode_warps_per_cta(int bits) {
   return bits == 8 ? warps_for<8>() : bits == 2 ? warps_for<2>() : warps_for<4>();
@@ -1053,16 +1048,12 @@ cudaError_t prepare_for() {
                               static_cast<int>(smem_bytes_for<kBits>()));
 }
 
-cudaError_t prepare_decode_kernel() {
-  cudaError_t e = prepare_for<4>();
-  if (e != cudaSuccess) return e;
-  e = prepare_for<8>();
-  if (e != cudaSuccess) return e;
-  return prepare_for<2>();
-}
-
 template <int kBits>
 cudaError_t launch_for(const DecodeParams &p, const FusedAppend &f, int num_ctas, cudaStream_t stream) {
+  // the kernel's shared-memory allowance, set at every launch (the library
+  // keeps no record of what it configured)
+  cudaError_t pe = prepare_for<kBits>();
+  if (pe != cudaSuccess) return pe;
   if (f.k_new == nullptr) {
     decode_kernel<kBits><<<num_ctas, threads_for<kBits>(), smem_bytes_for<kBits>(), stream>>>(p);
     return cudaGetLastError();

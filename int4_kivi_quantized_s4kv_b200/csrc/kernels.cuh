@@ -91,9 +91,7 @@ void launch_append(const AppendParams &p, int batch, int max_new, cudaStream_t s
 void launch_dequant(const DequantParams &p, cudaStream_t stream);
 void launch_move(const MoveParams &p, cudaStream_t stream);
 cudaError_t launch_decode(const DecodeParams &p, const FusedAppend &f, int bits, int num_ctas, cudaStream_t stream);
-int decode_ctas_per_sm(int bits);
 int decode_warps_per_cta(int bits);
-cudaError_t prepare_decode_kernel();
 size_t decode_smem_bytes(int bits);
 
 // Host entry of every decode call (plain, fused append, no-alloc): checks all

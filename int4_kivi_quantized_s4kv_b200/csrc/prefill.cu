@@ -820,33 +820,29 @@ int prefill_tiles_per_seq(int max_pages) {
   return static_cast<int>((static_cast<long long>(max_pages) + kPagesPerTile - 1) / kPagesPerTile);
 }
 
-cudaError_t prepare_prefill_kernel() {
-  cudaError_t e = cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(kSmemBytes));
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(prefill_operands_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(op_smem_bytes<4>()));
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(prefill_operands_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(op_smem_bytes<8>()));
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(prefill_operands_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(op_smem_bytes<2>()));
-  return e;
+// Both launches of a call; their shared-memory allowances are set at every
+// call (the library keeps no record of what it configured).
+template <int kBits>
+cudaError_t launch_operands(const PrefillParams &p, dim3 grid, cudaStream_t stream) {
+  const cudaError_t e = cudaFuncSetAttribute(prefill_operands_kernel<kBits>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(op_smem_bytes<kBits>()));
+  if (e != cudaSuccess) return e;
+  prefill_operands_kernel<kBits><<<grid, kOpThreads, op_smem_bytes<kBits>(), stream>>>(p);
+  return cudaGetLastError();
 }
 
-void launch_prefill(const PrefillParams &p, int batch, int max_new, cudaStream_t stream) {
+cudaError_t launch_prefill(const PrefillParams &p, int batch, int max_new, cudaStream_t stream) {
   const dim3 og(2 * p.tiles_per_seq, batch, p.num_kv_heads);
-  if (p.bits == 8)
-    prefill_operands_kernel<8><<<og, kOpThreads, op_smem_bytes<8>(), stream>>>(p);
-  else if (p.bits == 2)
-    prefill_operands_kernel<2><<<og, kOpThreads, op_smem_bytes<2>(), stream>>>(p);
-  else
-    prefill_operands_kernel<4><<<og, kOpThreads, op_smem_bytes<4>(), stream>>>(p);
+  cudaError_t e = p.bits == 8 ? launch_operands<8>(p, og, stream)
+                  : p.bits == 2 ? launch_operands<2>(p, og, stream) : launch_operands<4>(p, og, stream);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kSmemBytes));
+  if (e != cudaSuccess) return e;
   const int Tq = 128 / p.group;
   const int tiles = (max_new + Tq - 1) / Tq;
   const dim3 grid(tiles, batch, p.num_kv_heads);
   prefill_kernel<<<grid, kThreadsP, kSmemBytes, stream>>>(p);
+  return cudaGetLastError();
 }
 
 }  // namespace s4kv

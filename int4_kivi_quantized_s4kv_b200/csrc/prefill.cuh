@@ -30,8 +30,7 @@ struct PrefillParams {
   int bits;               // code width, 2, 4 or 8
 };
 
-void launch_prefill(const PrefillParams &p, int batch, int max_new, cudaStream_t stream);
-cudaError_t prepare_prefill_kernel();
+cudaError_t launch_prefill(const PrefillParams &p, int batch, int max_new, cudaStream_t stream);
 size_t prefill_smem_bytes();
 size_t prefill_tile_bytes();
 int prefill_tiles_per_seq(int max_pages);
