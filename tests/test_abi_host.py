@@ -103,6 +103,16 @@ def test_invalid_calls_rejected_before_launch(S):
     assert dec(ctypes.byref(c), P(fake), 8, P(fake), P(fake), 1, 1, -1.0, P(fake), P(fake), 1 << 30, st) == S.ERR_INVALID_ARG
     assert dec(ctypes.byref(c), None, 8, P(fake), P(fake), 1, 1, 0.088, P(fake), P(fake), 1 << 30, st) == S.ERR_INVALID_ARG
     assert dec(ctypes.byref(c), P(fake), 8, P(fake), P(fake), 0, 1, 0.088, P(fake), P(fake), 1 << 30, st) == S.OK
+    # the one-call decode step: missing or unaligned new tokens, and an append grid (one CTA per
+    # sequence and kv head) beyond the launch limit, are refused before anything runs
+    step = L.s4kv_append_decode
+    assert step(ctypes.byref(c), None, P(fake), P(fake), 8, P(fake), P(fake), 1, 1, 0.088, P(fake), P(fake),
+                1 << 30, st) == S.ERR_INVALID_ARG
+    assert step(ctypes.byref(c), P(fake), P(fake + 8), P(fake), 8, P(fake), P(fake), 1, 1, 0.088, P(fake), P(fake),
+                1 << 30, st) == S.ERR_INVALID_ARG
+    wide = S.s4kv_cache_t(fake, fake, fake, None, 10, 65536, 40000, 128, 16)
+    assert step(ctypes.byref(wide), P(fake), P(fake), P(fake), 65536, P(fake), P(fake), 40000, 1, 0.088, P(fake),
+                P(fake), 1 << 30, st) == S.ERR_INVALID_ARG
     # prefill
     pre = L.s4kv_prefill_attention
     args = lambda **kw: dict(dict(cache=ctypes.byref(c), q=P(fake), hq=8, n=4, cu=P(fake), sl=P(fake), bt=P(fake),
