@@ -166,6 +166,7 @@ class DeviceWorkload:
         self.step_slots = dev(W.slot_mapping(self.plan.block_tables, pos))
         self.step_cu = dev(np.concatenate([[0], np.cumsum(self.new)]).astype(np.int32))
         self.max_new = int(self.new.max())
+        self.one_token = bool((self.new == 1).all())
         self.caches, self.q, self.k_new, self.v_new = [], [], [], []
         for layer in range(spec.layers):
             cache = S.S4KVCache(self.plan.num_pages, H, B, device=device, bits=bits)
@@ -211,8 +212,19 @@ class DeviceWorkload:
             if flags:
                 raise RuntimeError(f"device flags {flags} after prefill")
 
-    def step(self, dec_events=None):
+    def step(self, dec_events=None, one_call=False):
+        """One decode step of every layer.  With `one_call` (and one new token
+        per sequence) each layer is one s4kv_append_decode call; otherwise
+        s4kv_append then s4kv_decode_attention, with `dec_events` (if given)
+        recorded around the decode launch."""
         S = self.S
+        if one_call and self.one_token and dec_events is None:
+            B, H = self.spec.batch, self.spec.num_kv_heads
+            for layer in range(self.spec.layers):
+                S.s4kv_append_decode(self.caches[layer], self.k_new[layer].view(B, H, 128),
+                                     self.v_new[layer].view(B, H, 128), self.q[layer], self.seq_lens, self.bt,
+                                     self.out[layer], self.ws)
+            return
         for layer in range(self.spec.layers):
             S.s4kv_append(self.caches[layer], self.k_new[layer], self.v_new[layer], self.step_slots,
                           self.step_cu, self.seq_lens, self.bt, self.max_new)
@@ -702,28 +714,37 @@ def main(argv=None):
     bytes_per_step = (dbytes["algorithmic"] + abytes) * spec.layers
     decode_bytes_per_launch = dbytes["algorithmic"]
 
+    # the step: one s4kv_append_decode call per layer (the append grid and
+    # the decode grid as its programmatic dependent) when every sequence gets
+    # one new token, else s4kv_append then s4kv_decode_attention
     for _ in range(args.warmup):
-        wl.step()
+        wl.step(one_call=True)
     torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
     clocks = ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ
                           else int(os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local]))
     clocks.start()
-    ev = ([], [])
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
     t_start.record()
     for _ in range(args.steps):
-        wl.step(ev)
+        wl.step(one_call=True)
     t_end.record()
     torch.cuda.synchronize()
     clocks.stop()
     step_ms = t_start.elapsed_time(t_end) / args.steps
+    step_ms = reduce_max(step_ms, world, device)
+    # the decode kernel on its own for the roofline: the same steps as two
+    # calls, with events around each decode launch (a dependent grid of the
+    # one-call step cannot be bracketed by events of its own)
+    ev = ([], [])
+    for _ in range(args.steps):
+        wl.step(ev)
+    torch.cuda.synchronize()
     dec_ms = [a.elapsed_time(b) for a, b in zip(*ev)]
     dec_avg_ms = sum(dec_ms) / len(dec_ms)
-    step_ms = reduce_max(step_ms, world, device)
 
     # end to end through the public API: every step copies its inputs (q and
     # the new tokens' K/V) in from pinned host memory and its output back.
@@ -761,7 +782,7 @@ def main(argv=None):
                 h2d_copy(i + 1)
             comp.wait_event(loaded[i % 2])
             wl.q, wl.k_new, wl.v_new, wl.out = sets[i % 2]
-            wl.step()
+            wl.step(one_call=True)
             done[i % 2].record(comp)
             with torch.cuda.stream(copy):
                 copy.wait_event(done[i % 2])
@@ -823,6 +844,8 @@ def main(argv=None):
                 "parallelism": f"replicas x{world}" if world > 1 else "1 GPU",
                 "context": {"min": int(wl.ctx.min()), "max": int(wl.ctx.max()), "mean": float(wl.ctx.mean())},
                 "new_tokens_per_seq": int(wl.new.max()),
+                "step_calls": ("s4kv_append_decode per layer" if wl.one_token
+                               else "s4kv_append + s4kv_decode_attention per layer"),
                 "shared_prefix_tokens": spec.shared_prefix_tokens,
                 "decode_bytes_per_layer": dbytes, "append_bytes_per_layer": abytes,
                 "l2": f"inputs larger than L2: {bytes_per_step / 1e9:.2f} GB read per step vs 126 MB L2"
