@@ -148,30 +148,6 @@ __device__ __forceinline__ void wait_landed(uint32_t bar, uint32_t parity) {
   }
 }
 
-
-// One elected lane of the (converged) warp issues the MMA / the commit.
-__device__ __forceinline__ void mma_ts_elect(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
-                                             uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p, e;\n\telect.sync _|e, 0xffffffff;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-__device__ __forceinline__ void mma_ss_e5m2_elect(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                                  uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p, e;\n\telect.sync _|e, 0xffffffff;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-      "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-__device__ __forceinline__ void commit_elect(uint32_t bar) {
-  asm volatile(
-      "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
-      "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(bar)
-      : "memory");
-}
 // 2^x for a pair, on the FMA/ALU pipes instead of the MUFU pipe.  Cody and
 // Waite's range reduction: x = j + f with j = rint(x) (adding 1.5 * 2^23
 // rounds x to an integer held in the sum's low mantissa bits) and
@@ -628,10 +604,10 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(const PrefillPara
         const uint64_t dv = vs ? dv1 : dv0;
 #pragma unroll
         for (int j = 0; j < kKeyTile / 16; ++j)
-          mma_ts_elect(tO, tP + 8 * j, dv + (((j >> 2) * (kVBytes / 2) + (j & 3) * 32) >> 4), kIdescO,
+          tc05::mma_f16_ts(tO, tP + 8 * j, dv + (((j >> 2) * (kVBytes / 2) + (j & 3) * 32) >> 4), kIdescO,
                        (k > 0 || j > 0) ? 1u : 0u);
-        commit_elect(p_empty);
-        commit_elect(v_empty(vs));
+        tc05::mma_commit(p_empty);
+        tc05::mma_commit(v_empty(vs));
       }
     } else {
       const uint64_t dk0 = tc05::smem_desc_sw128(kbuf(0)), dk1 = tc05::smem_desc_sw128(kbuf(1));
@@ -656,14 +632,14 @@ __global__ void __launch_bounds__(kThreadsP, 1) prefill_kernel(const PrefillPara
         // same channels of K_hi (fp16, K = 16 per MMA) ...
 #pragma unroll
         for (int j = 0; j < 8; ++j)
-          mma_ts_elect(tS(sb), tQ + 8 * j, dk + ((((j >> 2) * (kKHiBytes / 2)) + (j & 3) * 32) >> 4), kIdescS,
+          tc05::mma_f16_ts(tS(sb), tQ + 8 * j, dk + ((((j >> 2) * (kKHiBytes / 2)) + (j & 3) * 32) >> 4), kIdescS,
                        j > 0 ? 1u : 0u);
         // ... then Q8 channels 32 j .. + 31 against K_lo (e5m2, K = 32)
 #pragma unroll
         for (int j = 0; j < 4; ++j)
-          mma_ss_e5m2_elect(tS(sb), dq8 + ((32 * j) >> 4), dk + ((kKHiBytes + 32 * j) >> 4), kIdescS8, 1u);
-        commit_elect(s_full(sb));
-        commit_elect(k_empty(ks));
+          tc05::mma_e5m2_ss(tS(sb), dq8 + ((32 * j) >> 4), dk + ((kKHiBytes + 32 * j) >> 4), kIdescS8, 1u);
+        tc05::mma_commit(s_full(sb));
+        tc05::mma_commit(k_empty(ks));
       }
     }
   } else {
